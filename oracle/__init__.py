@@ -1,0 +1,150 @@
+"""CPU oracle for piecewise sparse attention (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it, and it imports nothing
+from the product.
+
+Thin ctypes wrapper over ``pisa_oracle.cpp`` (fp64 math, canonical fp32
+selection).  All arrays are numpy, C-contiguous, layout [BH, L, d].
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        f64p = ctypes.c_void_p
+        li = ctypes.c_long
+        L.oracle_block_stats.argtypes = [f32p, f32p, li, li, li, li, f64p, f64p, f64p, f64p, ctypes.c_int]
+        L.oracle_select.argtypes = [f32p, f32p, li, li, li, li, li, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_int]
+        L.oracle_pisa_attention.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
+        L.oracle_pisa_bruteforce.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
+                                             ctypes.c_int, f64p, ctypes.c_int]
+        L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
+        for fn in ("oracle_block_stats", "oracle_select", "oracle_pisa_attention",
+                   "oracle_pisa_bruteforce", "oracle_dense_attention"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(x):
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle: {what} rejected the shape/arguments")
+
+
+def block_stats(k, v, B, order=2, nthreads=None):
+    """fp64 (kbar [BH,nblk,d], vsum [BH,nblk,d], H [BH,nblk,d,d] or None, C or None).
+
+    H[bh, j, a, b] = sum_n v[n, a] * (k[n, b] - kbar[b]);  C = (1/B) sum_n dev dev^T.
+    """
+    k, v = _f32(k), _f32(v)
+    BH, L, d = k.shape
+    nblk = L // B
+    kbar = np.zeros((BH, nblk, d))
+    vsum = np.zeros((BH, nblk, d))
+    H = np.zeros((BH, nblk, d, d)) if order >= 1 else None
+    C = np.zeros((BH, nblk, d, d)) if order == 2 else None
+    rc = lib().oracle_block_stats(k, v, BH, L, d, B, _ptr(kbar), _ptr(vsum), _ptr(H), _ptr(C),
+                                  nthreads or default_threads())
+    _check(rc, "block_stats")
+    return kbar, vsum, H, C
+
+
+def select(q, k, B, K, nthreads=None, want_scores=False):
+    """Canonical fp32 selection: (idx [BH,nblk,K] int32 ascending, mask [BH,nblk,words] uint32,
+    scores [BH,nblk,nblk] float32 or None)."""
+    q, k = _f32(q), _f32(k)
+    BH, L, d = q.shape
+    nblk = L // B
+    words = (nblk + 31) // 32
+    idx = np.zeros((BH, nblk, K), np.int32)
+    mask = np.zeros((BH, nblk, words), np.uint32)
+    scores = np.zeros((BH, nblk, nblk), np.float32) if want_scores else None
+    rc = lib().oracle_select(q, k, BH, L, d, B, K, _ptr(idx), _ptr(mask), _ptr(scores),
+                             nthreads or default_threads())
+    _check(rc, "select")
+    return idx, mask, scores
+
+
+def pisa_attention(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, want_lse=False):
+    """Statistics-form output.  With tiles=None returns [BH, L, d] fp64; otherwise
+    ``tiles`` is a sequence of (bh, i) query tiles and the result is [ntiles, B, d].
+    With want_lse the log-denominator log(D_t) is returned too (same leading shape)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BH, L, d = q.shape
+    nblk = L // B
+    full = tiles is None
+    if full:
+        tl = np.array([(bh, i) for bh in range(BH) for i in range(nblk)], dtype=np.int64)
+    else:
+        tl = np.ascontiguousarray(np.asarray(tiles, dtype=np.int64).reshape(-1, 2))
+    out = np.zeros((tl.shape[0], B, d))
+    lse = np.zeros((tl.shape[0], B)) if want_lse else None
+    rc = lib().oracle_pisa_attention(q, k, v, BH, L, d, B, K, int(order), int(bool(gate)),
+                                     _ptr(tl), tl.shape[0], _ptr(out), _ptr(lse),
+                                     nthreads or default_threads())
+    _check(rc, "pisa_attention")
+    if full:
+        out = out.reshape(BH, L, d)
+        lse = lse.reshape(BH, L) if want_lse else None
+    return (out, lse) if want_lse else out
+
+
+def pisa_bruteforce(q, k, v, B, K, order=1, gate=True, nthreads=None):
+    """Token-wise first-order form without block statistics, [BH, L, d] fp64."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BH, L, d = q.shape
+    out = np.zeros((BH, L, d))
+    rc = lib().oracle_pisa_bruteforce(q, k, v, BH, L, d, B, K, int(order), int(bool(gate)),
+                                      _ptr(out), nthreads or default_threads())
+    _check(rc, "pisa_bruteforce")
+    return out
+
+
+def dense_attention(q, k, v, nthreads=None):
+    """softmax(q k^T) v in fp64, [BH, L, d]."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BH, L, d = q.shape
+    out = np.zeros((BH, L, d))
+    rc = lib().oracle_dense_attention(q, k, v, BH, L, d, _ptr(out), nthreads or default_threads())
+    _check(rc, "dense_attention")
+    return out
+
+
+def rel_l2(a, b) -> float:
+    """||a - b||_F / ||b||_F."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
+
+
+LN = math.log

@@ -1,0 +1,455 @@
+// Plain CPU oracle for piecewise sparse attention (PISA / PWT).
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+// call this file: only the test-suite, the package smoke check and the CPU
+// baseline leg of the benchmark use it.  It shares no code with the CUDA
+// library (no headers, helpers or tables) and is deliberately slow: fp64
+// arithmetic, one query at a time, loops written in the order the pages state
+// the method.  Every floating-point result here is fp64 except the block
+// selection, which follows a canonical fp32 procedure (below) so that the GPU
+// can reproduce it bit for bit.
+//
+// Sources (the web pages this method is described on):
+//   [blog1] "Sparse Linear Attention" (haoyizhu.site), notation paragraph and
+//           sections "Sparse Attention", "Sparse Linear Attention",
+//           "Going Further: Adding the Second-Order Term (PWT)".
+//   [blog2] "Sparse Linear Attention: When Sparsity Meets Linear Attention (2)",
+//           section "Picking Up Where We Left Off" (defines w_{t,j} and H_j).
+//   [pisa]  "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion
+//           Transformers": section 3.1 Eq. 1, section 3.2 "Formulation"
+//           (o_t = N_t / D_t and D_t), Figure 3 caption (prepare phase),
+//           Appendix C "Notation" (k-bar_j, alpha_{t,j}, delta_{t,j,n}).
+//
+// Readings taken where the pages are silent (each is also listed in the
+// design notes):
+//   * N_t is not printed in any surviving equation; [blog1] "Sparse Linear
+//     Attention" names its three parts (exact, zeroth order, first-order
+//     correction with H_j), which gives
+//       N_t = sum_{S} sum_n e^{x} v_n + sum_{U} e^{s-bar + w} (vsum_j + H_j q_t).
+//   * Selection is per query tile of B rows and scores the tile-mean query
+//     against each key centroid ([pisa] Figure 3 caption and section 3.2);
+//     ties go to the lower block index.  Eq. 7's softmax is monotone and is
+//     dropped; the 1/sqrt(d) is already inside q.
+//   * C_j carries 1/B (the second-order expansion of the block mean of
+//     e^{y} gives (1/2B) sum_n y_n^2 = 1/2 q^T C_j q).
+//   * The PWT gate: w is set to 0 (not clamped) when w > ln B.
+//
+// Build: g++ -O2 -std=c++17 -fPIC -shared -pthread -ffp-contract=off
+// (contraction off so that the fp32 selection rounds every product and sum).
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Canonical fp32 reduction: pairwise tree over a power-of-two count.
+// For h = n/2, n/4, ..., 1: a[i] = a[i] + a[i+h] for i < h.  Result a[0].
+// Every add is one IEEE fp32 round-to-nearest operation.
+// ---------------------------------------------------------------------------
+float tree_sum_f32(float* a, long n) {
+    for (long h = n / 2; h >= 1; h /= 2) {
+        for (long i = 0; i < h; ++i) {
+            volatile float s = a[i] + a[i + h];  // volatile: no reassociation
+            a[i] = s;
+        }
+    }
+    return a[0];
+}
+
+bool is_pow2(long x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Per (bh): fp64 block statistics of the keys and values.
+//   kbar_j = (1/B) sum_n k_{j,n}                         ([blog1] notation)
+//   vsum_j = sum_n v_{j,n}                               ([pisa] Figure 3)
+//   H_j[a][b] = sum_n v_{j,n}[a] (k_{j,n}[b] - kbar_j[b]) ([blog1] "Sparse Linear Attention")
+//   C_j[a][b] = (1/B) sum_n (k-kbar)[a] (k-kbar)[b]      ([blog1] PWT section)
+void block_stats_one(const float* k, const float* v, long L, long d, long B,
+                     double* kbar, double* vsum, double* H, double* C) {
+    const long nblk = L / B;
+    std::vector<double> dev(B * d);
+    for (long j = 0; j < nblk; ++j) {
+        const float* kj = k + j * B * d;
+        const float* vj = v + j * B * d;
+        double* kb = kbar + j * d;
+        for (long c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (long n = 0; n < B; ++n) s += (double)kj[n * d + c];
+            kb[c] = s / (double)B;
+        }
+        if (vsum) {
+            double* vs = vsum + j * d;
+            for (long c = 0; c < d; ++c) {
+                double s = 0.0;
+                for (long n = 0; n < B; ++n) s += (double)vj[n * d + c];
+                vs[c] = s;
+            }
+        }
+        for (long n = 0; n < B; ++n)
+            for (long c = 0; c < d; ++c) dev[n * d + c] = (double)kj[n * d + c] - kb[c];
+        if (H) {
+            double* Hj = H + j * d * d;
+            for (long a = 0; a < d; ++a)
+                for (long b = 0; b < d; ++b) {
+                    double s = 0.0;
+                    for (long n = 0; n < B; ++n) s += (double)vj[n * d + a] * dev[n * d + b];
+                    Hj[a * d + b] = s;
+                }
+        }
+        if (C) {
+            double* Cj = C + j * d * d;
+            for (long a = 0; a < d; ++a)
+                for (long b = 0; b < d; ++b) {
+                    double s = 0.0;
+                    for (long n = 0; n < B; ++n) s += dev[n * d + a] * dev[n * d + b];
+                    Cj[a * d + b] = s / (double)B;
+                }
+        }
+    }
+}
+
+// Canonical fp32 block selection for one (bh).  For each query tile i:
+//   qbar_i[c] = tree_sum_f32(q[iB..iB+B)[c]) * (1/B)      (fp32)
+//   kbar_j[c] = tree_sum_f32(k[jB..jB+B)[c]) * (1/B)      (fp32)
+//   s_ij      = tree_sum_f32(qbar_i[c] * kbar_j[c] over c) (products rounded)
+//   S_i = the K blocks first in the order (s descending, j ascending).
+void select_one(const float* q, const float* k, long L, long d, long B, long K,
+                int32_t* idx, uint32_t* mask, float* scores) {
+    const long nblk = L / B;
+    const long words = (nblk + 31) / 32;
+    const float inv_b = 1.0f / (float)B;
+    std::vector<float> qbar(nblk * d), kbar(nblk * d), col(B), prod(d), s(nblk);
+    for (long j = 0; j < nblk; ++j)
+        for (long c = 0; c < d; ++c) {
+            for (long n = 0; n < B; ++n) col[n] = k[(j * B + n) * d + c];
+            volatile float m = tree_sum_f32(col.data(), B) * inv_b;
+            kbar[j * d + c] = m;
+        }
+    for (long i = 0; i < nblk; ++i)
+        for (long c = 0; c < d; ++c) {
+            for (long n = 0; n < B; ++n) col[n] = q[(i * B + n) * d + c];
+            volatile float m = tree_sum_f32(col.data(), B) * inv_b;
+            qbar[i * d + c] = m;
+        }
+    std::vector<long> order(nblk);
+    for (long i = 0; i < nblk; ++i) {
+        for (long j = 0; j < nblk; ++j) {
+            for (long c = 0; c < d; ++c) {
+                volatile float p = qbar[i * d + c] * kbar[j * d + c];
+                prod[c] = p;
+            }
+            s[j] = tree_sum_f32(prod.data(), d);
+            if (scores) scores[i * nblk + j] = s[j];
+        }
+        for (long j = 0; j < nblk; ++j) order[j] = j;
+        std::stable_sort(order.begin(), order.end(), [&](long a, long b) {
+            if (s[a] > s[b]) return true;
+            if (s[a] < s[b]) return false;
+            return a < b;
+        });
+        uint32_t* mrow = mask ? mask + i * words : nullptr;
+        if (mrow) std::memset(mrow, 0, sizeof(uint32_t) * words);
+        std::vector<long> chosen(order.begin(), order.begin() + K);
+        std::sort(chosen.begin(), chosen.end());
+        for (long r = 0; r < K; ++r) {
+            if (idx) idx[i * K + r] = (int32_t)chosen[r];
+            if (mrow) mrow[chosen[r] / 32] |= (1u << (chosen[r] % 32));
+        }
+    }
+}
+
+// One query row of the statistics form ([pisa] section 3.2 "Formulation",
+// [blog1] "Sparse Linear Attention" and PWT section):
+//   x_{j,n} = q.k_{j,n}                      j in S (exact)
+//   l_j     = q.kbar_j + w_j                  j in U (virtual token logit)
+//   w_j     = order 2 ? 1/2 q^T C_j q : 0; with the gate, w_j = 0 when w_j > ln B
+//   D = sum_S sum_n e^{x} + sum_U B e^{l}
+//   N = sum_S sum_n e^{x} v_n + sum_U e^{l} (vsum_j + [order>=1] H_j q)
+//   o = N / D                   (evaluated with the common shift m = max logit)
+void row_stats_form(const float* qrow, const float* k, const float* v, long d, long B,
+                    long nblk, const uint8_t* sel, int order, int gate,
+                    const double* kbar, const double* vsum, const double* H, const double* C,
+                    double* out, double* lse, std::vector<double>& xs,
+                    std::vector<double>& ls, std::vector<double>& num) {
+    std::vector<double> q(d);
+    for (long c = 0; c < d; ++c) q[c] = (double)qrow[c];
+    const double ln_b = std::log((double)B);
+    double m = -INFINITY;
+    for (long j = 0; j < nblk; ++j) {
+        if (sel[j]) {
+            for (long n = 0; n < B; ++n) {
+                const float* kr = k + (j * B + n) * d;
+                double x = 0.0;
+                for (long c = 0; c < d; ++c) x += q[c] * (double)kr[c];
+                xs[j * B + n] = x;
+                m = std::max(m, x);
+            }
+        } else {
+            double sb = 0.0;
+            for (long c = 0; c < d; ++c) sb += q[c] * kbar[j * d + c];
+            double w = 0.0;
+            if (order == 2) {
+                const double* Cj = C + j * d * d;
+                for (long a = 0; a < d; ++a) {
+                    double t = 0.0;
+                    for (long b = 0; b < d; ++b) t += Cj[a * d + b] * q[b];
+                    w += q[a] * t;
+                }
+                w *= 0.5;
+                if (gate && w > ln_b) w = 0.0;
+            }
+            ls[j] = sb + w;
+            m = std::max(m, ls[j]);
+        }
+    }
+    double D = 0.0;
+    std::fill(num.begin(), num.end(), 0.0);
+    for (long j = 0; j < nblk; ++j) {
+        if (sel[j]) {
+            for (long n = 0; n < B; ++n) {
+                const double e = std::exp(xs[j * B + n] - m);
+                const float* vr = v + (j * B + n) * d;
+                D += e;
+                for (long c = 0; c < d; ++c) num[c] += e * (double)vr[c];
+            }
+        } else {
+            const double a = std::exp(ls[j] - m);
+            D += (double)B * a;
+            const double* vs = vsum + j * d;
+            for (long c = 0; c < d; ++c) num[c] += a * vs[c];
+            if (order >= 1) {
+                const double* Hj = H + j * d * d;
+                for (long r = 0; r < d; ++r) {
+                    double t = 0.0;
+                    for (long c = 0; c < d; ++c) t += Hj[r * d + c] * q[c];
+                    num[r] += a * t;
+                }
+            }
+        }
+    }
+    for (long c = 0; c < d; ++c) out[c] = num[c] / D;
+    if (lse) *lse = m + std::log(D);  // log of the unshifted denominator D_t
+}
+
+// The same row without any block statistic: every unselected token keeps the
+// first-order weight e^{l_j}(1 + delta_n), delta_n = q.(k_n - kbar_j)
+// ([pisa] Appendix C notation; [blog1] "Sparse Linear Attention").  Summing
+// these per token must give the statistics form because sum_n delta_n = 0.
+void row_brute(const float* qrow, const float* k, const float* v, long d, long B, long nblk,
+               const uint8_t* sel, int order, int gate, double* out) {
+    std::vector<double> q(d), kb(d), num(d, 0.0);
+    for (long c = 0; c < d; ++c) q[c] = (double)qrow[c];
+    const double ln_b = std::log((double)B);
+    // logits per token for S, per block for U; find the shift
+    std::vector<double> xs(nblk * B), ls(nblk), sb(nblk);
+    double m = -INFINITY;
+    for (long j = 0; j < nblk; ++j) {
+        for (long n = 0; n < B; ++n) {
+            const float* kr = k + (j * B + n) * d;
+            double x = 0.0;
+            for (long c = 0; c < d; ++c) x += q[c] * (double)kr[c];
+            xs[j * B + n] = x;
+        }
+        if (sel[j]) {
+            for (long n = 0; n < B; ++n) m = std::max(m, xs[j * B + n]);
+        } else {
+            for (long c = 0; c < d; ++c) {
+                double s = 0.0;
+                for (long n = 0; n < B; ++n) s += (double)k[(j * B + n) * d + c];
+                kb[c] = s / (double)B;
+            }
+            double s = 0.0;
+            for (long c = 0; c < d; ++c) s += q[c] * kb[c];
+            sb[j] = s;
+            double w = 0.0;
+            if (order == 2) {
+                // w = (1/2B) sum_n delta_n^2 : the mean of the squared deviation
+                for (long n = 0; n < B; ++n) {
+                    double dl = 0.0;
+                    for (long c = 0; c < d; ++c) dl += q[c] * ((double)k[(j * B + n) * d + c] - kb[c]);
+                    w += dl * dl;
+                }
+                w /= 2.0 * (double)B;
+                if (gate && w > ln_b) w = 0.0;
+            }
+            ls[j] = s + w;
+            m = std::max(m, ls[j]);
+        }
+    }
+    double D = 0.0;
+    for (long j = 0; j < nblk; ++j) {
+        for (long n = 0; n < B; ++n) {
+            double wt;
+            if (sel[j]) {
+                wt = std::exp(xs[j * B + n] - m);
+            } else {
+                const double dl = (order >= 1) ? xs[j * B + n] - sb[j] : 0.0;
+                wt = std::exp(ls[j] - m) * (1.0 + dl);
+            }
+            D += wt;
+            const float* vr = v + (j * B + n) * d;
+            for (long c = 0; c < d; ++c) num[c] += wt * (double)vr[c];
+        }
+    }
+    for (long c = 0; c < d; ++c) out[c] = num[c] / D;
+}
+
+template <class F>
+void parallel_for(long n, int nthreads, F&& fn) {
+    if (nthreads <= 1 || n <= 1) {
+        for (long i = 0; i < n; ++i) fn(i);
+        return;
+    }
+    std::atomic<long> next(0);
+    std::vector<std::thread> pool;
+    const int nt = (int)std::min<long>(nthreads, n);
+    for (int t = 0; t < nt; ++t)
+        pool.emplace_back([&]() {
+            for (;;) {
+                long i = next.fetch_add(1);
+                if (i >= n) break;
+                fn(i);
+            }
+        });
+    for (auto& th : pool) th.join();
+}
+
+}  // namespace
+
+extern "C" {
+
+// Returns 0 on success, -1 on a shape the oracle does not define.
+int oracle_block_stats(const float* k, const float* v, long BH, long L, long d, long B,
+                       double* kbar, double* vsum, double* H, double* C, int nthreads) {
+    if (B <= 0 || L % B) return -1;
+    const long nblk = L / B;
+    parallel_for(BH, nthreads, [&](long bh) {
+        block_stats_one(k + bh * L * d, v + bh * L * d, L, d, B, kbar + bh * nblk * d,
+                        vsum ? vsum + bh * nblk * d : nullptr,
+                        H ? H + bh * nblk * d * d : nullptr,
+                        C ? C + bh * nblk * d * d : nullptr);
+    });
+    return 0;
+}
+
+int oracle_select(const float* q, const float* k, long BH, long L, long d, long B, long K,
+                  int32_t* idx, uint32_t* mask, float* scores, int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B) return -1;
+    const long nblk = L / B;
+    if (K < 0 || K > nblk) return -1;
+    const long words = (nblk + 31) / 32;
+    parallel_for(BH, nthreads, [&](long bh) {
+        select_one(q + bh * L * d, k + bh * L * d, L, d, B, K,
+                   idx ? idx + bh * nblk * K : nullptr, mask ? mask + bh * nblk * words : nullptr,
+                   scores ? scores + bh * nblk * nblk : nullptr);
+    });
+    return 0;
+}
+
+// Statistics-form output for a list of query tiles.  tiles[2*r] = bh,
+// tiles[2*r+1] = tile index i; out receives [ntiles, B, d] fp64 rows and, when
+// lse is not null, lse receives [ntiles, B] values log(D_t) (unshifted).
+// The selection (canonical fp32) is recomputed here from q and k.
+int oracle_pisa_attention(const float* q, const float* k, const float* v, long BH, long L,
+                          long d, long B, long K, int order, int gate, const int64_t* tiles,
+                          long ntiles, double* out, double* lse, int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
+    const long nblk = L / B;
+    if (K < 0 || K > nblk) return -1;
+    // statistics and selection for every bh that appears in the tile list
+    std::vector<char> need(BH, 0);
+    for (long r = 0; r < ntiles; ++r) {
+        if (tiles[2 * r] < 0 || tiles[2 * r] >= BH || tiles[2 * r + 1] < 0 || tiles[2 * r + 1] >= nblk)
+            return -1;
+        need[tiles[2 * r]] = 1;
+    }
+    std::vector<long> bhs;
+    for (long bh = 0; bh < BH; ++bh)
+        if (need[bh]) bhs.push_back(bh);
+    const long words = (nblk + 31) / 32;
+    std::vector<std::vector<double>> kbar(BH), vsum(BH), H(BH), C(BH);
+    std::vector<std::vector<uint32_t>> mask(BH);
+    parallel_for((long)bhs.size(), nthreads, [&](long r) {
+        const long bh = bhs[r];
+        kbar[bh].assign(nblk * d, 0.0);
+        vsum[bh].assign(nblk * d, 0.0);
+        H[bh].assign(order >= 1 ? nblk * d * d : 0, 0.0);
+        C[bh].assign(order == 2 ? nblk * d * d : 0, 0.0);
+        block_stats_one(k + bh * L * d, v + bh * L * d, L, d, B, kbar[bh].data(), vsum[bh].data(),
+                        order >= 1 ? H[bh].data() : nullptr, order == 2 ? C[bh].data() : nullptr);
+        mask[bh].assign(nblk * words, 0u);
+        select_one(q + bh * L * d, k + bh * L * d, L, d, B, K, nullptr, mask[bh].data(), nullptr);
+    });
+    parallel_for(ntiles, nthreads, [&](long r) {
+        const long bh = tiles[2 * r], i = tiles[2 * r + 1];
+        std::vector<uint8_t> sel(nblk);
+        for (long j = 0; j < nblk; ++j) sel[j] = (mask[bh][i * words + j / 32] >> (j % 32)) & 1u;
+        std::vector<double> xs(nblk * B), ls(nblk), num(d);
+        for (long m = 0; m < B; ++m) {
+            const long t = i * B + m;
+            row_stats_form(q + (bh * L + t) * d, k + bh * L * d, v + bh * L * d, d, B, nblk,
+                           sel.data(), order, gate, kbar[bh].data(), vsum[bh].data(),
+                           H[bh].data(), C[bh].data(), out + (r * B + m) * d,
+                           lse ? lse + r * B + m : nullptr, xs, ls, num);
+        }
+    });
+    return 0;
+}
+
+// Token-wise form (no block statistics), same selection; full output [BH, L, d].
+int oracle_pisa_bruteforce(const float* q, const float* k, const float* v, long BH, long L,
+                           long d, long B, long K, int order, int gate, double* out,
+                           int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
+    const long nblk = L / B;
+    if (K < 0 || K > nblk) return -1;
+    const long words = (nblk + 31) / 32;
+    parallel_for(BH, nthreads, [&](long bh) {
+        std::vector<uint32_t> mask(nblk * words);
+        select_one(q + bh * L * d, k + bh * L * d, L, d, B, K, nullptr, mask.data(), nullptr);
+        std::vector<uint8_t> sel(nblk);
+        for (long i = 0; i < nblk; ++i) {
+            for (long j = 0; j < nblk; ++j) sel[j] = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+            for (long m = 0; m < B; ++m) {
+                const long t = i * B + m;
+                row_brute(q + (bh * L + t) * d, k + bh * L * d, v + bh * L * d, d, B, nblk,
+                          sel.data(), order, gate, out + (bh * L + t) * d);
+            }
+        }
+    });
+    return 0;
+}
+
+// Dense softmax attention o_t = sum_i softmax(q_t.k_i) v_i ([pisa] Eq. 1), fp64.
+int oracle_dense_attention(const float* q, const float* k, const float* v, long BH, long L,
+                           long d, double* out, int nthreads) {
+    parallel_for(BH * L, nthreads, [&](long r) {
+        const long bh = r / L;
+        const float* qr = q + r * d;
+        const float* kh = k + bh * L * d;
+        const float* vh = v + bh * L * d;
+        std::vector<double> x(L), num(d, 0.0);
+        double m = -INFINITY;
+        for (long i = 0; i < L; ++i) {
+            double s = 0.0;
+            for (long c = 0; c < d; ++c) s += (double)qr[c] * (double)kh[i * d + c];
+            x[i] = s;
+            m = std::max(m, s);
+        }
+        double D = 0.0;
+        for (long i = 0; i < L; ++i) {
+            const double e = std::exp(x[i] - m);
+            D += e;
+            for (long c = 0; c < d; ++c) num[c] += e * (double)vh[i * d + c];
+        }
+        for (long c = 0; c < d; ++c) out[r * d + c] = num[c] / D;
+    });
+    return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,329 @@
+"""Pins for the CPU oracle: checks against facts the pages and the mathematics fix.
+
+None of these tests compares the oracle with itself.  Each pin reaches the
+expected value through a different route: a library routine (torch fp64
+softmax), a closed form, a special case that reduces to exact attention, an
+invariant, the error bound of the PISA paper's Appendix C, brute force per
+token, or a hand-built fixture.  A plausible mistake in the oracle (a dropped
+term, a wrong sign, a transposed statistic, a wrong normalisation, a wrong tie
+rule, a clamp instead of the gate) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pisa_synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def torch_dense(q, k, v):
+    """softmax(q k^T) v in fp64 through torch (PISA paper section 3.1, Eq. 1)."""
+    qt, kt, vt = (torch.from_numpy(np.asarray(x, np.float64)) for x in (q, k, v))
+    return torch.softmax(qt @ kt.transpose(-1, -2), dim=-1).matmul(vt).numpy()
+
+
+def torch_lse(q, k):
+    qt, kt = (torch.from_numpy(np.asarray(x, np.float64)) for x in (q, k))
+    return torch.logsumexp(qt @ kt.transpose(-1, -2), dim=-1).numpy()
+
+
+def small(seed, BH=2, L=256, d=16, scale=1.0):
+    return pisa_synth.random_qkv(seed, BH, L, d, scale=scale)
+
+
+# ----------------------------------------------------------------------------
+# exact special cases
+# ----------------------------------------------------------------------------
+
+def test_dense_oracle_matches_torch():
+    q, k, v = small(1, L=128, d=8, scale=3.0)
+    np.testing.assert_allclose(oracle.dense_attention(q, k, v), torch_dense(q, k, v), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_all_blocks_selected_equals_dense(order):
+    # With U empty the method is exact softmax attention (PISA section 3.2, D_t with U = {}).
+    q, k, v = small(2, L=256, d=16, scale=2.0)
+    B = 16
+    o = oracle.pisa_attention(q, k, v, B, 256 // B, order=order)
+    np.testing.assert_allclose(o, torch_dense(q, k, v), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("K", [0, 3, 17])
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_block_size_one_is_exact(K, order):
+    # B = 1: every centroid is its key, every deviation is zero.
+    q, k, v = small(3, L=32, d=8, scale=2.0)
+    o = oracle.pisa_attention(q, k, v, 1, K, order=order)
+    np.testing.assert_allclose(o, torch_dense(q, k, v), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_identical_keys_per_block_is_exact(order):
+    # K = 0 with equal keys inside each block: the Taylor expansion is exact.
+    q, k, v = small(4, L=128, d=8, scale=2.0)
+    B = 16
+    k = np.repeat(k[:, ::B, :], B, axis=1).copy()
+    o = oracle.pisa_attention(q, k, v, B, 0, order=order)
+    np.testing.assert_allclose(o, torch_dense(q, k, v), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+@pytest.mark.parametrize("K", [0, 2, 8])
+def test_zero_queries_give_mean_value(order, K):
+    # q = 0: every logit is 0 and every weight (exact or virtual token) is uniform.
+    _, k, v = small(5, L=128, d=8)
+    q = np.zeros_like(k)
+    o = oracle.pisa_attention(q, k, v, 16, K, order=order)
+    np.testing.assert_allclose(o, np.broadcast_to(v.astype(np.float64).mean(axis=1, keepdims=True), o.shape), atol=1e-13)
+
+
+def test_constant_values_per_block_remove_first_order():
+    # H_j = sum_n v_n (k_n - kbar_j)^T vanishes when v is constant in the block.
+    q, k, v = small(6, L=128, d=8, scale=2.0)
+    B = 16
+    v = np.repeat(v[:, ::B, :], B, axis=1).copy()
+    o1 = oracle.pisa_attention(q, k, v, B, 2, order=1)
+    o0 = oracle.pisa_attention(q, k, v, B, 2, order=0)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# brute force per token (no block statistics)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+@pytest.mark.parametrize("gate", [True, False])
+@pytest.mark.parametrize("B,d,K", [(16, 16, 3), (32, 8, 1), (8, 32, 10), (64, 16, 0)])
+def test_statistics_form_equals_token_form(order, gate, B, d, K):
+    q, k, v = small(7 + B + d, L=256, d=d, scale=2.0)
+    o = oracle.pisa_attention(q, k, v, B, K, order=order, gate=gate)
+    ob = oracle.pisa_bruteforce(q, k, v, B, K, order=order, gate=gate)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# block statistics: invariants and closed forms
+# ----------------------------------------------------------------------------
+
+def test_statistics_invariants():
+    q, k, v = small(8, BH=1, L=128, d=16, scale=1.0)
+    B = 8  # B < d, so rank(H_j) <= B - 1 < d is visible
+    kbar, vsum, H, C = oracle.block_stats(k, v, B, order=2)
+    kb = k[0].reshape(-1, B, 16).astype(np.float64)
+    vb = v[0].reshape(-1, B, 16).astype(np.float64)
+    np.testing.assert_allclose(kbar[0], kb.mean(axis=1), atol=1e-14)
+    np.testing.assert_allclose(vsum[0], vb.sum(axis=1), atol=1e-13)
+    for j in range(kb.shape[0]):
+        dev = kb[j] - kb[j].mean(axis=0)
+        # H_j q = sum_n v_n (q . (k_n - kbar_j)): pins the orientation (rows = value channel)
+        qq = q[0, j].astype(np.float64)
+        np.testing.assert_allclose(H[0, j] @ qq, (vb[j] * (dev @ qq)[:, None]).sum(axis=0), atol=1e-12)
+        # the deviations sum to zero, so H_j annihilates nothing in general but H_j has rank <= B - 1
+        sv = np.linalg.svd(H[0, j], compute_uv=False)
+        assert sv[B - 1] < 1e-10 * sv[0]
+        # trace C_j = (1/B) sum_n |k_n - kbar|^2 = (1/2B^2) sum_{n,n'} |k_n - k_n'|^2
+        pair = ((kb[j][:, None, :] - kb[j][None, :, :]) ** 2).sum()
+        assert abs(np.trace(C[0, j]) - pair / (2 * B * B)) < 1e-12
+        # C_j is symmetric positive semi-definite
+        np.testing.assert_allclose(C[0, j], C[0, j].T, atol=0)
+        assert np.linalg.eigvalsh(C[0, j]).min() > -1e-12
+
+
+def test_statistics_vanish_for_identical_keys_and_constant_values():
+    _, k, v = small(9, BH=1, L=64, d=8)
+    B = 16
+    k = np.repeat(k[:, ::B, :], B, axis=1).copy()
+    _, _, H, C = oracle.block_stats(k, v, B, order=2)
+    assert np.abs(H).max() == 0.0 and np.abs(C).max() == 0.0
+    _, k2, _ = small(10, BH=1, L=64, d=8)
+    v2 = np.repeat(v[:, ::B, :], B, axis=1).copy()
+    _, _, H2, _ = oracle.block_stats(k2, v2, B, order=1)
+    assert np.abs(H2).max() < 1e-13
+
+
+def test_second_order_two_point_block_closed_form():
+    # Keys kbar + a (B/2 tokens) and kbar - a (B/2 tokens): C_j = a a^T, so
+    # w = 1/2 (q.a)^2 exactly, and the single virtual token has mass B e^{q.kbar + w}
+    # ("Sparse Linear Attention" blog, PWT section).  The true mass is
+    # B e^{q.kbar} cosh(q.a), which e^{w} approaches more closely than 1 does.
+    rng = np.random.default_rng(11)
+    B, d = 16, 8
+    kbar = rng.integers(-2, 3, d).astype(np.float32) / 4
+    a = rng.integers(-2, 3, d).astype(np.float32) / 8
+    k = np.concatenate([np.tile(kbar + a, (B // 2, 1)), np.tile(kbar - a, (B // 2, 1))])[None]
+    q = (rng.integers(-3, 4, (1, B, d)).astype(np.float32) / 8)
+    v = rng.standard_normal((1, B, d)).astype(np.float32)
+    _, lse2 = oracle.pisa_attention(q, k, v, B, 0, order=2, gate=False, want_lse=True)
+    _, lse1 = oracle.pisa_attention(q, k, v, B, 0, order=1, want_lse=True)
+    qa = q[0].astype(np.float64) @ a.astype(np.float64)
+    qk = q[0].astype(np.float64) @ kbar.astype(np.float64)
+    np.testing.assert_allclose(lse1[0], math.log(B) + qk, atol=1e-12)
+    np.testing.assert_allclose(lse2[0], math.log(B) + qk + 0.5 * qa ** 2, atol=1e-12)
+    true = np.log(B * np.exp(qk) * np.cosh(qa))
+    assert np.all(np.abs(lse2[0] - true) <= np.abs(lse1[0] - true) + 1e-15)
+
+
+def test_second_order_gate_zeroes_not_clamps():
+    # Huge within-block spread: every w exceeds ln B, so the gated order-2 result
+    # must equal order 1 exactly (a clamp at ln B would not).
+    q, k, v = small(12, L=128, d=8, scale=1.0)
+    B = 16
+    k = k * np.float32(40.0)
+    o1 = oracle.pisa_attention(q, k, v, B, 2, order=1)
+    o2 = oracle.pisa_attention(q, k, v, B, 2, order=2, gate=True)
+    o2n = oracle.pisa_attention(q, k, v, B, 2, order=2, gate=False)
+    assert np.array_equal(o1, o2)
+    assert not np.allclose(o1, o2n)
+
+
+# ----------------------------------------------------------------------------
+# denominators and the error bound (PISA paper, Appendix C)
+# ----------------------------------------------------------------------------
+
+def test_jensen_denominator_and_nonnegative_w():
+    # B alpha_{t,j} <= sum_n exp(q k_{j,n}) (Appendix C), so the approximate
+    # denominator never exceeds the dense one; w >= 0 so order 2 adds mass.
+    q, k, v = small(13, L=256, d=16, scale=2.0)
+    B = 16
+    dense = torch_lse(q, k)
+    _, l1 = oracle.pisa_attention(q, k, v, B, 4, order=1, want_lse=True)
+    _, l0 = oracle.pisa_attention(q, k, v, B, 4, order=0, want_lse=True)
+    _, l2 = oracle.pisa_attention(q, k, v, B, 4, order=2, gate=False, want_lse=True)
+    assert np.all(l1 <= dense + 1e-12)
+    np.testing.assert_array_equal(l0, l1)  # the first-order mass is exactly zero
+    assert np.all(l2 >= l1 - 1e-12)
+
+
+def _bound_terms(q, k, v, B, K):
+    """Per row: C_v e^{eta} S_2 / D-hat for the per-block first-order form."""
+    q64, k64, v64 = (np.asarray(x, np.float64) for x in (q, k, v))
+    BH, L, d = q.shape
+    nblk = L // B
+    _, mask, _ = oracle.select(q, k, B, K)
+    bound = np.zeros((BH, L))
+    for bh in range(BH):
+        cv = np.linalg.norm(v64[bh], axis=1).max()
+        kb = k64[bh].reshape(nblk, B, d)
+        kbar = kb.mean(axis=1)
+        for i in range(nblk):
+            sel = np.array([(mask[bh, i, j // 32] >> (j % 32)) & 1 for j in range(nblk)], bool)
+            qt = q64[bh, i * B:(i + 1) * B]                       # [B, d]
+            x = np.einsum("td,jnd->tjn", qt, kb)                   # logits
+            sbar = qt @ kbar.T                                     # [B, nblk]
+            delta = x - sbar[:, :, None]
+            alpha = np.exp(sbar)
+            dhat = (np.exp(x) * sel[None, :, None]).sum(axis=(1, 2)) + (B * alpha * ~sel[None, :]).sum(axis=1)
+            s2 = (alpha[:, ~sel] * (delta[:, ~sel, :] ** 2).sum(axis=2)).sum(axis=1)
+            eta = np.abs(delta[:, ~sel, :]).max(axis=(1, 2)) if (~sel).any() else np.zeros(B)
+            bound[bh, i * B:(i + 1) * B] = cv * np.exp(eta) * s2 / dhat
+    return bound
+
+
+def test_taylor_error_bound_appendix_c():
+    # ||o-hat - o*|| <= C_v e^{eta} S_2 / D-hat for block-wise H_j (Appendix C);
+    # the zeroth-order variant, which drops H_j q, must break it somewhere at
+    # small eta (its error is first order in eta).
+    B, K = 16, 4
+    for scale in (1.0, 0.25, 0.02):
+        q, k, v = small(14, BH=2, L=256, d=16, scale=scale)
+        bound = _bound_terms(q, k, v, B, K)
+        dense = torch_dense(q, k, v)
+        err1 = np.linalg.norm(oracle.pisa_attention(q, k, v, B, K, order=1) - dense, axis=-1)
+        assert np.all(err1 <= bound * (1 + 1e-9) + 1e-15)
+        if scale == 0.02:
+            err0 = np.linalg.norm(oracle.pisa_attention(q, k, v, B, K, order=0) - dense, axis=-1)
+            assert np.any(err0 > bound)
+
+
+# ----------------------------------------------------------------------------
+# canonical fp32 selection
+# ----------------------------------------------------------------------------
+
+def np_tree_sum(a, axis):
+    """The canonical pairwise tree in numpy float32 (a[i] += a[i + h], h = n/2 .. 1)."""
+    a = np.moveaxis(np.asarray(a, np.float32), axis, 0).copy()
+    n = a.shape[0]
+    while n > 1:
+        h = n // 2
+        a[:h] = a[:h] + a[h:n]
+        n = h
+    return a[0]
+
+
+def np_select(q, k, B, K):
+    BH, L, d = q.shape
+    nblk = L // B
+    inv = np.float32(1.0 / B)
+    idx = np.zeros((BH, nblk, K), np.int32)
+    scores = np.zeros((BH, nblk, nblk), np.float32)
+    for bh in range(BH):
+        qbar = np_tree_sum(q[bh].reshape(nblk, B, d), 1) * inv
+        kbar = np_tree_sum(k[bh].reshape(nblk, B, d), 1) * inv
+        prod = qbar[:, None, :] * kbar[None, :, :]
+        s = np_tree_sum(prod, 2)
+        scores[bh] = s
+        for i in range(nblk):
+            order = np.lexsort((np.arange(nblk), -s[i].astype(np.float64)))
+            idx[bh, i] = np.sort(order[:K])
+    return idx, scores
+
+
+@pytest.mark.parametrize("B,d,K,dtype", [(16, 16, 5, "f32"), (64, 64, 4, "f32"), (32, 128, 7, "bf16"),
+                                         (8, 8, 0, "f32"), (8, 8, 32, "f32")])
+def test_selection_matches_numpy_restatement_bitwise(B, d, K, dtype):
+    L = 256
+    q, k, _ = pisa_synth.random_qkv(15 + B, 2, L, d, scale=4.0, dtype=dtype)
+    idx, mask, scores = oracle.select(q, k, B, K, want_scores=True)
+    idx_np, scores_np = np_select(q, k, B, K)
+    assert np.array_equal(scores.view(np.uint32), scores_np.view(np.uint32))
+    assert np.array_equal(idx, idx_np)
+    nblk = L // B
+    for bh in range(2):
+        for i in range(nblk):
+            bits = [j for j in range(nblk) if (mask[bh, i, j // 32] >> (j % 32)) & 1]
+            assert bits == list(idx[bh, i])
+
+
+def test_selection_tie_rule_golden():
+    with open(os.path.join(GOLDEN, "tie_break.json")) as f:
+        g = json.load(f)
+    q = np.asarray(g["q"], np.float32)[None]
+    k = np.asarray(g["k"], np.float32)[None]
+    _, _, scores = oracle.select(q, k, g["B"], 1, want_scores=True)
+    np.testing.assert_array_equal(scores[0], np.asarray(g["scores_by_hand"], np.float32))
+    for K, want in g["expected_idx"].items():
+        idx, _, _ = oracle.select(q, k, g["B"], int(K))
+        np.testing.assert_array_equal(idx[0], np.asarray(want, np.int32))
+
+
+def test_selection_agrees_with_fp64_ranking_away_from_ties():
+    q, k, _ = pisa_synth.random_qkv(16, 2, 512, 32, scale=4.0)
+    B, K = 16, 6
+    idx, _, _ = oracle.select(q, k, B, K)
+    q64, k64 = q.astype(np.float64), k.astype(np.float64)
+    nblk = 512 // B
+    for bh in range(2):
+        s = q64[bh].reshape(nblk, B, -1).mean(1) @ k64[bh].reshape(nblk, B, -1).mean(1).T
+        for i in range(nblk):
+            srt = np.sort(s[i])[::-1]
+            gap = srt[K - 1] - srt[K]
+            if gap > 1e-4 * max(1.0, abs(srt[K])):
+                want = np.sort(np.argsort(-s[i], kind="stable")[:K])
+                assert np.array_equal(idx[bh, i], want)
+
+
+def test_oracle_rejects_undefined_shapes():
+    q, k, v = small(17, L=96, d=8)
+    with pytest.raises(ValueError):
+        oracle.select(q, k, 12, 2)        # B not a power of two
+    with pytest.raises(ValueError):
+        oracle.pisa_attention(q, k, v, 64, 1)  # L % B != 0
+    with pytest.raises(ValueError):
+        oracle.pisa_attention(q, k, v, 16, 7)  # K > nblk
