@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of piecewise sparse attention on B200.
+
+One step = one forward pass of the whole hot path on one batch of synthetic
+input: block centroids -> top-K block selection -> fused attention (exact
+blocks, Taylor-compensated unselected blocks, normalisation), i.e. exactly the
+kernels ``pisa_attention`` runs, called stage by stage through the C ABI so
+that each kernel is bracketed by CUDA events on the launching stream.
+
+Default workload: Wan2.1-shaped attention, 1 x 40 heads, L = 32768, d = 128,
+bf16, B = 64, K = 77, order 1 (inputs 1 GiB > L2, so no flush is needed
+between steps).  Metric: full-attention-equivalent TFLOP/s, 4 L^2 d H / t,
+whole job (sum over ranks; weak scaling: every rank runs the full workload on
+its own inputs).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU: launched by torch.distributed.run, one rank per GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call & full-attn-equiv TFLOP/s at Wan-shape L=32K; % of roofline"
+UNIT = "TFLOP/s (full-attention-equivalent, 4*L^2*d*heads per call)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="c3")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--heads", type=int, default=None, help="override head count (profiling small cases)")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_taylor_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(workload: str):
+    """DRAM bytes per launch of the attention kernel from a committed ncu
+    summary, only if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"attn_tc_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [x for x in sm if x > 0.5 * (mx or 1)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's value (timings are reported as the max over ranks)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def rank_workload(w, rank: int):
+    """Weak scaling: rank r runs the same workload on its own seeded inputs
+    (rank 0 keeps the canonical seed)."""
+    return w.with_(seed=w.seed + 1000 * rank) if rank else w
+
+
+def cpu_baseline(w, q, k, v, budget_s=20.0):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload:
+    the block statistics of head 0 plus a few query tiles of head 0,
+    extrapolated to the whole call (all heads, all tiles)."""
+    import oracle
+
+    nthreads = oracle.default_threads()
+    qh, kh, vh = q[:1], k[:1], v[:1]
+    t0 = time.perf_counter()
+    oracle.block_stats(kh, vh, w.B, order=w.order, nthreads=nthreads)
+    t_stats = time.perf_counter() - t0
+    ntiles = max(1, min(w.nblk, nthreads))
+    tiles = [(0, int(i)) for i in np.linspace(0, w.nblk - 1, ntiles).round()]
+    t0 = time.perf_counter()
+    oracle.pisa_attention(qh, kh, vh, w.B, w.K, w.order, tiles=tiles, nthreads=nthreads)
+    t_call = time.perf_counter() - t0
+    # oracle.pisa_attention also recomputes the head's statistics and selection
+    t_tiles = max(t_call - t_stats, 1e-9)
+    per_tile = t_tiles / len(tiles)
+    # the oracle computes the statistics of different heads on different threads
+    t_full = w.BH * (t_stats / min(nthreads, w.BH) + per_tile * w.nblk)
+    flops = 4.0 * w.L * w.L * w.d * w.BH
+    return {
+        "value": flops / t_full / 1e12,
+        "unit": UNIT,
+        "cores": nthreads,
+        "kind": "oracle",
+        "sample": (f"head 0 of {w.BH}: block statistics ({t_stats:.2f} s) + {len(tiles)} of {w.nblk} query tiles "
+                   f"({t_tiles:.2f} s, includes re-running that head's statistics and selection); extrapolated to "
+                   f"{w.BH} heads x {w.nblk} tiles = {t_full:.0f} s per call"),
+        "seconds_measured": t_stats + t_call,
+    }
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, on the same workload/metric."""
+    import pisa_synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = pisa_synth.workloads()[args.workload]
+    q, k, v = pisa_synth.generate(w.with_(heads=1))
+    times = []
+    base = None
+    for _ in range(args.warmup + args.steps):
+        r = cpu_baseline(w, q, k, v)
+        times.append(r)
+        base = r
+    vals = [r["value"] for r in times[args.warmup:]] or [base["value"]]
+    val = statistics.median(vals)
+    ms = 4.0 * w.L * w.L * w.d * w.BH / (val * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: Wan2.1-shaped, {w.BH} heads, L={w.L}, d={w.d}, B={w.B}, K={w.K}, "
+                               f"order={w.order}", "l2": "n/a (CPU)"},
+        "cpu_baseline": {"kind": base["kind"], "cores": base["cores"], "sample": base["sample"], "value": val,
+                         "unit": UNIT},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+
+    import block_sparse_taylor_b200 as pisa
+    import pisa_synth
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    w = pisa_synth.workloads()[args.workload]
+    if args.heads:
+        w = w.with_(heads=args.heads)
+    # weak scaling: every rank draws its own inputs of the full workload
+    wr = rank_workload(w, rank)
+    q_h, k_h, v_h = pisa_synth.generate(wr)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.from_numpy(q_h).to(tdt).cuda()
+    k = torch.from_numpy(k_h).to(tdt).cuda()
+    v = torch.from_numpy(v_h).to(tdt).cuda()
+    BH, L, d, B, K, order = w.BH, w.L, w.d, w.B, w.K, w.order
+    nblk = L // B
+    path = pisa.pisa_resolve_path(1, BH, L, d, B, K, order, tdt)
+    out = torch.empty_like(q)
+    kbar = torch.empty((BH, nblk, d), dtype=torch.float32, device="cuda")
+    words = (nblk + 31) // 32
+    idx = torch.empty((BH, nblk, K), dtype=torch.int32, device="cuda")
+    mask = torch.empty((BH, nblk, words), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    stats_full = None
+    if path == "stats":
+        stats_full = pisa.pisa_stats(k, v, B, order)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if path == "stats":
+            st = pisa.pisa_stats(k, v, B, order, buf=stats_full.buf)
+        else:
+            st = pisa.pisa_centroids(k, B, kbar=kbar)
+        if ev is not None:
+            ev[1].record(stream)
+        lib = pisa.lib()
+        pisa._check(lib.pisa_select(q.data_ptr(), pisa.ctypes.byref(st.raw), K, idx.data_ptr() if K else None,
+                                    mask.data_ptr(), stream.cuda_stream))
+        if ev is not None:
+            ev[2].record(stream)
+        pisa.pisa_fused_attention(q, k, v, B, mask, order, path=path, stats=st if path == "stats" else None,
+                                  out=out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    pisa.pisa_poll_device_status()
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    k_prep = [e[0].elapsed_time(e[1]) for e in evs]
+    k_sel = [e[1].elapsed_time(e[2]) for e in evs]
+    k_attn = [e[2].elapsed_time(e[3]) for e in evs]
+    attn_ms = statistics.mean(k_attn)
+
+    dense_flops = 4.0 * L * L * d * BH
+    value = dense_flops * world / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    if path == "recompute_tc":
+        exec_flops = 4.0 * L * L * d * BH  # QK^T and PV over every key block
+        achieved = exec_flops / (attn_ms * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic_record(w.name) if not args.heads else None,
+                "kernel": f"attn_tc_kernel<{d},{B}>",
+                "algorithmic_flops_per_launch": exec_flops,
+                "peak_source": f"{peak_kind} bf16 dense (burst; the kernel is timed alone inside the step)"}
+    else:
+        # statistics path: CUDA-core kernel; report against the HBM roofline of its reads
+        nbytes = 3 * BH * L * d * q.element_size()
+        achieved = nbytes / (attn_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "kernel": f"attn_stats_kernel<{d},{B}>", "peak_source": peak_kind}
+    # HBM figures of the small kernels (centroids read K once; select reads Q once + writes the mask)
+    prep_bytes = BH * L * d * q.element_size() + BH * nblk * d * 4
+    sel_bytes = BH * L * d * q.element_size() + BH * nblk * (words + K) * 4
+    hbm = float(peaks["hbm_gbs"])
+    per_kernel = {
+        "centroids_ms": statistics.mean(k_prep), "select_ms": statistics.mean(k_sel), "attn_ms": attn_ms,
+        "centroids_gbs": prep_bytes / (statistics.mean(k_prep) * 1e-3) / 1e9,
+        "select_gbs": sel_bytes / (statistics.mean(k_sel) * 1e-3) / 1e9,
+    }
+    per_kernel["centroids_frac_hbm"] = per_kernel["centroids_gbs"] / hbm
+    per_kernel["select_frac_hbm"] = per_kernel["select_gbs"] / hbm
+
+    # end to end through the public call with host buffers: pinned H2D, pisa_attention, D2H
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(pisa.pisa_workspace_bytes(1, BH, L, d, B, K, order, tdt), dtype=torch.uint8,
+                         device="cuda")
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            pisa.pisa_attention(dq, dk, dv, B, K, order, out=out, workspace=ws)
+            ho.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world)
+        e2e = {"value": dense_flops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+               "d2h_bytes_per_step": out.numel() * out.element_size()}
+        pisa.pisa_poll_device_status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, q_h, k_h, v_h)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": f"{w.name}: Wan2.1-shaped DiT attention, batch 1 x {BH} heads, L={L} "
+                                   f"(8x64x64 video grid), d={d}, B={B}, K={K}, order={order}",
+                       "path": path, "global_batch": world, "seq_len": L,
+                       "parallelism": f"replicas x{world} (heads independent, no collective)",
+                       "l2": "inputs exceed L2 (3 x {:.0f} MiB per rank), no flush".format(
+                           q.numel() * q.element_size() / 2 ** 20)},
+            "roofline": roof,
+            "per_kernel": per_kernel,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "tflops_executed_attn": roof["achieved"] if roof["unit"] == "TFLOP/s" else None,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

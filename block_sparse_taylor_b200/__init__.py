@@ -1,0 +1,261 @@
+"""Python binding of the B200 piecewise sparse attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libpisa_b200.so`` (C ABI in ``include/pisa.h``).  PyTorch is used
+for device memory and streams.  There is no fallback: if the compiled library
+is missing, importing a function raises ``PisaLibraryMissing``; build it with
+``python -m block_sparse_taylor_b200.build``.
+
+The functions carry the names of the C entry points:
+
+* ``pisa_stats(k, v, B, order)``: block statistics (centroids, value sums,
+  H_j, C_j), the prepare phase of the PISA paper (section 3.4, Figure 3).
+* ``pisa_select(q, stats, K)``: per query tile, the top-K key blocks by the
+  tile-mean query's centroid score, reproducible bit for bit.
+* ``pisa_attention(q, k, v, B, K, order)``: the full forward pass of piecewise
+  sparse attention (PISA paper section 3.2; "Sparse Linear Attention" blog,
+  PWT section for order 2).
+
+Tensors are [batch*heads, L, d] (or [batch, heads, L, d]) contiguous CUDA
+tensors of dtype float32 or bfloat16; q must already be multiplied by
+1/sqrt(d).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libpisa_b200.so")
+
+PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
+PISA_F32, PISA_BF16 = 0, 1
+PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2}
+PATH_NAMES = {v: k for k, v in PATHS.items()}
+
+
+class PisaLibraryMissing(ImportError):
+    pass
+
+
+class PisaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"pisa status {status}: {msg}")
+        self.status = status
+
+
+class _StatsT(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("heads", ctypes.c_int), ("L", ctypes.c_int), ("d", ctypes.c_int),
+                ("B", ctypes.c_int), ("nblk", ctypes.c_int), ("order", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("kbar", ctypes.c_void_p), ("vsum", ctypes.c_void_p), ("hstat", ctypes.c_void_p),
+                ("cov", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library (raises PisaLibraryMissing if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise PisaLibraryMissing(f"{LIB_PATH} not found: run `python -m block_sparse_taylor_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i, sz, vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+        L.pisa_version.restype = ctypes.c_char_p
+        L.pisa_last_error.restype = ctypes.c_char_p
+        L.pisa_stats_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.pisa_stats_bytes.restype = sz
+        L.pisa_stats_bind.argtypes = [ctypes.POINTER(_StatsT), vp, sz, i, i, i, i, i, i, i]
+        L.pisa_stats.argtypes = [vp, vp, ctypes.POINTER(_StatsT), vp]
+        L.pisa_select.argtypes = [vp, ctypes.POINTER(_StatsT), i, vp, vp, vp]
+        L.pisa_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        L.pisa_workspace_bytes.restype = sz
+        L.pisa_workspace_bytes_ex.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.pisa_workspace_bytes_ex.restype = sz
+        L.pisa_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp, sz, vp]
+        L.pisa_attention_ex.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp, sz, vp]
+        L.pisa_resolve_path.argtypes = [i, i, i, i, i, i, i, i]
+        L.pisa_poll_device_status.argtypes = [vp]
+        L.pisa_centroids.argtypes = [vp, i, i, i, i, i, i, vp, vp]
+        L.pisa_fused_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, ctypes.POINTER(_StatsT),
+                                           vp, vp]
+        for fn in ("pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
+                   "pisa_poll_device_status", "pisa_resolve_path"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != PISA_OK:
+        raise PisaError(status, lib().pisa_last_error().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return PISA_BF16
+    if t == torch.float32:
+        return PISA_F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _shape(x: torch.Tensor):
+    if x.dim() == 4:
+        return x.shape[0], x.shape[1], x.shape[2], x.shape[3]
+    if x.dim() == 3:
+        return 1, x.shape[0], x.shape[1], x.shape[2]
+    raise ValueError("expected [batch, heads, L, d] or [batch*heads, L, d]")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def version() -> str:
+    return lib().pisa_version().decode()
+
+
+class Stats(NamedTuple):
+    kbar: torch.Tensor            # [BH, nblk, d] fp32
+    vsum: torch.Tensor            # [BH, nblk, d] fp32
+    hstat: Optional[torch.Tensor]  # [BH, nblk, d, d] (rows = value channel)
+    cov: Optional[torch.Tensor]    # [BH, nblk, d, d]
+    raw: _StatsT
+    buf: torch.Tensor
+
+
+def pisa_stats_bytes(batch, heads, L, d, B, order, dtype: torch.dtype) -> int:
+    return int(lib().pisa_stats_bytes(batch, heads, L, d, B, order, _dtype_code(dtype)))
+
+
+def pisa_stats(k: torch.Tensor, v: torch.Tensor, B: int, order: int = 2, buf: Optional[torch.Tensor] = None,
+               stream=None) -> Stats:
+    """Block statistics of k, v (prepare phase).  Returns views into ``buf``."""
+    _need_cuda(k, v)
+    batch, heads, L, d = _shape(k)
+    code = _dtype_code(k.dtype)
+    nbytes = pisa_stats_bytes(batch, heads, L, d, B, order, k.dtype)
+    if nbytes == 0:
+        raise PisaError(PISA_ERR_INVALID_ARG, "invalid dimensions for pisa_stats")
+    if buf is None:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=k.device)
+    st = _StatsT()
+    _check(lib().pisa_stats_bind(ctypes.byref(st), buf.data_ptr(), buf.numel(), batch, heads, L, d, B, order, code))
+    _check(lib().pisa_stats(k.data_ptr(), v.data_ptr(), ctypes.byref(st), _stream(stream)))
+    return _stats_views(st, buf, k.dtype)
+
+
+def _stats_views(st: _StatsT, buf: torch.Tensor, dtype: torch.dtype) -> Stats:
+    BH = st.batch * st.heads
+    base = buf.data_ptr()
+
+    def view(ptr, shape, dt):
+        if not ptr:
+            return None
+        n = 1
+        for s in shape:
+            n *= s
+        off = ptr - base
+        es = torch.empty((), dtype=dt).element_size()
+        return buf[off:off + n * es].view(dt).view(*shape)
+
+    kbar = view(st.kbar, (BH, st.nblk, st.d), torch.float32)
+    vsum = view(st.vsum, (BH, st.nblk, st.d), torch.float32)
+    hstat = view(st.hstat, (BH, st.nblk, st.d, st.d), dtype)
+    cov = view(st.cov, (BH, st.nblk, st.d, st.d), dtype)
+    return Stats(kbar, vsum, hstat, cov, st, buf)
+
+
+def pisa_centroids(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, stream=None) -> Stats:
+    """Canonical fp32 centroids only (what the selection needs); returns a Stats
+    whose other arrays are None."""
+    _need_cuda(k)
+    batch, heads, L, d = _shape(k)
+    if kbar is None:
+        kbar = torch.empty((batch * heads, L // B, d), dtype=torch.float32, device=k.device)
+    _check(lib().pisa_centroids(k.data_ptr(), batch, heads, L, d, _dtype_code(k.dtype), B, kbar.data_ptr(),
+                                _stream(stream)))
+    st = _StatsT(batch, heads, L, d, B, L // B, 0, _dtype_code(k.dtype), kbar.data_ptr(), None, None, None)
+    return Stats(kbar, None, None, None, st, kbar)
+
+
+def pisa_fused_attention(q, k, v, B: int, mask: torch.Tensor, order: int = 1, gate: bool = True,
+                         path: str = "auto", stats: Optional[Stats] = None, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """The fused attention kernel alone, given the selection mask of pisa_select."""
+    _need_cuda(q, k, v, mask)
+    batch, heads, L, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    st = ctypes.byref(stats.raw) if stats is not None else None
+    _check(lib().pisa_fused_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d,
+                                      _dtype_code(q.dtype), B, order, int(bool(gate)), PATHS[path],
+                                      mask.data_ptr(), st, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def pisa_select(q: torch.Tensor, stats: Stats, K: int, stream=None):
+    """(idx [BH, nblk, K] int32 ascending, mask [BH, nblk, ceil(nblk/32)] int32 bit words)."""
+    _need_cuda(q)
+    st = stats.raw
+    BH = st.batch * st.heads
+    words = (st.nblk + 31) // 32
+    idx = torch.empty((BH, st.nblk, max(K, 0)), dtype=torch.int32, device=q.device)
+    mask = torch.empty((BH, st.nblk, words), dtype=torch.int32, device=q.device)
+    _check(lib().pisa_select(q.data_ptr(), ctypes.byref(st), K, idx.data_ptr() if K > 0 else None,
+                             mask.data_ptr(), _stream(stream)))
+    return idx, mask
+
+
+def pisa_workspace_bytes(batch, heads, L, d, B, K, order, dtype: torch.dtype, path: str = "auto") -> int:
+    return int(lib().pisa_workspace_bytes_ex(batch, heads, L, d, B, K, order, _dtype_code(dtype), PATHS[path]))
+
+
+def pisa_resolve_path(batch, heads, L, d, B, K, order, dtype: torch.dtype) -> str:
+    p = lib().pisa_resolve_path(batch, heads, L, d, B, K, order, _dtype_code(dtype))
+    if p < 0:
+        raise PisaError(PISA_ERR_INVALID_ARG, "no path for these arguments")
+    return PATH_NAMES[p]
+
+
+def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
+                   gate: bool = True, path: str = "auto", out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Piecewise sparse attention forward; returns ``out`` (same shape and dtype as q)."""
+    _need_cuda(q, k, v)
+    if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share shape and dtype")
+    batch, heads, L, d = _shape(q)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    _need_cuda(out)
+    nbytes = pisa_workspace_bytes(batch, heads, L, d, B, K, order, q.dtype, path)
+    if nbytes == 0:
+        raise PisaError(PISA_ERR_INVALID_ARG if path == "auto" else PISA_ERR_UNSUPPORTED,
+                        f"no workspace size for these arguments (path={path})")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().pisa_attention_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d, code, B, K,
+                                   order, int(bool(gate)), PATHS[path], out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel(), _stream(stream)))
+    return out
+
+
+def pisa_poll_device_status(stream=None):
+    """Synchronise and raise PisaError if a device-side bounded wait gave up."""
+    _check(lib().pisa_poll_device_status(_stream(stream)))

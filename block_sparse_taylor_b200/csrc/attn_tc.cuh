@@ -1,0 +1,450 @@
+// Piecewise sparse attention on tcgen05 tensor cores (token form).
+//
+// What it computes (PISA paper, section 3.2 "Formulation"; "Sparse Linear
+// Attention" blog, sections "Sparse Linear Attention" and "Going Further:
+// Adding the Second-Order Term (PWT)"): for query row t of tile i and key block
+// j, with x_n = q_t.k_{j,n} and s-bar = q_t.kbar_j = mean_n x_n,
+//   j in S_i :  weights e^{x_n}                                (exact)
+//   j in U_i :  weights e^{l}(1 + x_n - s-bar),  l = s-bar + w  (order >= 1)
+//               weights e^{l}                                  (order 0)
+//               denominator mass B e^{l}
+//   w = 1/2 q^T C_j q = (1/2B) sum_n (x_n - s-bar)^2 for order 2 (0 above ln B
+//   when gated), 0 otherwise.
+// Summing e^{l}(1 + x_n - s-bar) v_n over the block gives exactly the paper's
+// e^{l}(vsum_j + H_j q_t): the first-order numerator of the unselected block is
+// evaluated through the block's tokens instead of the d x d statistic H_j.
+// When d = 2B the two associations cost the same per (query, block), and this
+// one needs no H_j stream and yields w from the same logits.  Both branches
+// share one running max and one denominator (one online softmax).
+//
+// Structure (one CTA = 256 query rows of one (batch, head) = two 128-row M
+// tiles; all key tiles of 128 keys are visited in order):
+//   warp 0      TMA producer: Q once, then K and V tiles through NS stages
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2-5   softmax group 0 (M tile 0), warps 6-9 softmax group 1
+// TMEM (512 columns): S0 | S1 | O0 | O1.  The softmax writes P (bf16) over the
+// first half of its S columns and the PV MMA reads it from TMEM as operand A.
+// MMA order per key tile jt: PV0(jt), S0(jt+1), PV1(jt), S1(jt+1), so each
+// softmax group works while the tensor core runs the other group's products.
+// The running max is raised only when it grows by more than 2^8 (the output is
+// rescaled then), so most tiles need no correction of O.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace pisa {
+
+constexpr int kTcThreads = 320;
+constexpr long long kWaitLimitCycles = 2000000000ll;  // ~1 s at B200 clocks
+
+template <int D>
+struct TcCfg {
+    static constexpr int NK = 128;                 // keys per tile
+    static constexpr int MQ = 128;                 // rows per M tile
+    static constexpr int NS = (D == 128) ? 2 : 4;  // K/V stages
+    static constexpr int BOX = 64;                 // bf16 columns per 128-byte swizzle box
+    static constexpr int NBOX = D / BOX;
+    static constexpr uint32_t BOX_BYTES = 128 * 128;     // 128 rows x 128 bytes
+    static constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t K_OFF = Q_OFF + 2 * TILE_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + NS * TILE_BYTES;
+    static constexpr uint32_t BAR_OFF = V_OFF + NS * TILE_BYTES;
+    static constexpr uint32_t NBAR = 1 + 4 * NS + 2 + 2 + 2 + 1;
+    static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
+    static constexpr uint32_t O_COL0 = 256;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ mask, bf16* __restrict__ out,
+                   int L, int nblk, int words, int order, int gate, float ln_b, unsigned* status) {
+    using C = TcCfg<D>;
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, N = 128 keys
+    constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);     // O += P V, N = d, V MN-major
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = tc::smem_addr(smem);
+    uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);
+    uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
+    auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+    const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS;
+    const int B_SFULL = 1 + 4 * C::NS, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_DONE = B_OFULL + 2;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int bh = blockIdx.y;
+    const int q0 = blockIdx.x * 256;
+    const int NT = L / C::NK;
+    bool aborted = false;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar(B_QFULL), 1);
+        for (int s = 0; s < C::NS; ++s) {
+            tc::mbar_init(bar(B_KFULL + s), 1);
+            tc::mbar_init(bar(B_KEMPTY + s), 1);
+            tc::mbar_init(bar(B_VFULL + s), 1);
+            tc::mbar_init(bar(B_VEMPTY + s), 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            tc::mbar_init(bar(B_SFULL + h), 1);
+            tc::mbar_init(bar(B_PFULL + h), 128);
+            tc::mbar_init(bar(B_OFULL + h), 1);
+        }
+        tc::mbar_init(bar(B_DONE), 1);
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch(&tm_q);
+            tc::tma_prefetch(&tm_k);
+            tc::tma_prefetch(&tm_v);
+            const int row0 = bh * L + q0;
+            tc::mbar_expect_tx(bar(B_QFULL), 2 * C::TILE_BYTES);
+            for (int h = 0; h < 2; ++h)
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::Q_OFF + h * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q, bar(B_QFULL),
+                                    b * C::BOX, row0 + h * C::MQ);
+            int lastK = -1, lastV = -1;
+            for (int jt = 0; jt < NT; ++jt) {
+                const int st = jt % C::NS, u = jt / C::NS;
+                if (u > 0 && !tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::K_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_k,
+                                    bar(B_KFULL + st), b * C::BOX, bh * L + jt * C::NK);
+                lastK = jt;
+                if (u > 0 && !tc::mbar_wait(bar(B_VEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::V_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_v,
+                                    bar(B_VFULL + st), b * C::BOX, bh * L + jt * C::NK);
+                lastV = jt;
+            }
+            if (aborted) {
+                // let every copy already issued land before the CTA exits
+                bool a2 = false;
+                tc::mbar_wait(bar(B_QFULL), 0, a2, status, kWaitLimitCycles);
+                for (int jt = (lastK - C::NS + 1 > 0 ? lastK - C::NS + 1 : 0); jt <= lastK; ++jt) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_KFULL + jt % C::NS), (jt / C::NS) & 1, a2, status, kWaitLimitCycles);
+                }
+                for (int jt = (lastV - C::NS + 1 > 0 ? lastV - C::NS + 1 : 0); jt <= lastV; ++jt) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_VFULL + jt % C::NS), (jt / C::NS) & 1, a2, status, kWaitLimitCycles);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            auto issue_s = [&](int h, int st) {
+                const uint32_t qa = sbase + C::Q_OFF + h * C::TILE_BYTES;
+                const uint32_t ka = sbase + C::K_OFF + st * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
+                    tc::mma_ss(tmem + (uint32_t)(h * 128), tc::sdesc_sw128(qa + off, 16, 1024),
+                               tc::sdesc_sw128(ka + off, 16, 1024), IDESC_S, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int h, int st, bool first) {
+                const uint32_t va = sbase + C::V_OFF + st * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::NK / 16; ++kk) {
+                    tc::mma_ts(tmem + C::O_COL0 + h * D, tmem + (uint32_t)(h * 128) + kk * 8,
+                               tc::sdesc_sw128(va + kk * 16 * 128, C::BOX_BYTES, 1024), IDESC_O,
+                               (first && kk == 0) ? 0u : 1u);
+                }
+            };
+            bool ok = tc::mbar_wait(bar(B_QFULL), 0, aborted, status, kWaitLimitCycles);
+            ok = ok && tc::mbar_wait(bar(B_KFULL + 0), 0, aborted, status, kWaitLimitCycles);
+            if (ok) {
+                issue_s(0, 0);
+                tc::mma_commit(bar(B_SFULL + 0));
+                issue_s(1, 0);
+                tc::mma_commit(bar(B_SFULL + 1));
+                tc::mma_commit(bar(B_KEMPTY + 0));
+            }
+            for (int jt = 0; ok && jt < NT; ++jt) {
+                const int st = jt % C::NS, u = jt / C::NS;
+                const int st1 = (jt + 1) % C::NS, u1 = (jt + 1) / C::NS;
+                const bool more = jt + 1 < NT;
+                if (!tc::mbar_wait(bar(B_VFULL + st), u & 1, aborted, status, kWaitLimitCycles)) break;
+                if (!tc::mbar_wait(bar(B_PFULL + 0), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(0, st, jt == 0);
+                if (!more) tc::mma_commit(bar(B_OFULL + 0));
+                if (more) {
+                    if (!tc::mbar_wait(bar(B_KFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
+                    issue_s(0, st1);
+                    tc::mma_commit(bar(B_SFULL + 0));
+                }
+                if (!tc::mbar_wait(bar(B_PFULL + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(1, st, jt == 0);
+                if (!more) tc::mma_commit(bar(B_OFULL + 1));
+                tc::mma_commit(bar(B_VEMPTY + st));
+                if (more) {
+                    issue_s(1, st1);
+                    tc::mma_commit(bar(B_SFULL + 1));
+                    tc::mma_commit(bar(B_KEMPTY + st1));
+                }
+            }
+            // every MMA issued by this thread has completed before TMEM is freed
+            tc::mma_commit(bar(B_DONE));
+            bool a2 = false;
+            tc::mbar_wait(bar(B_DONE), 0, a2, status, kWaitLimitCycles);
+        }
+    } else {
+        // ------------------------------------------------------------- softmax
+        const int h = (warp - 2) / 4;             // M tile of this group
+        const int quarter = warp % 4;             // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;        // row inside the M tile = TMEM lane
+        const int qrow = q0 + h * C::MQ + r;      // query row inside the head
+        const bool valid = qrow < L;
+        int qt = (qrow < L ? qrow : L - 1) / BS;  // query tile (selection row)
+        const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t s_addr = lane_base + (uint32_t)(h * 128);
+        const uint32_t o_addr = lane_base + C::O_COL0 + h * D;
+        constexpr int BPT = C::NK / BS;           // blocks per key tile
+        constexpr int CPB = BS / 32;              // 32-column chunks per block
+        const float inv_bs = 1.0f / (float)BS;
+        float m_run = -INFINITY;                  // running max (log2 units)
+        float dsum = 0.f;                         // denominator (scaled by 2^-m_run)
+
+        for (int jt = 0; jt < NT; ++jt) {
+            if (!tc::mbar_wait_warp(bar(B_SFULL + h), jt & 1, aborted, status, kWaitLimitCycles)) break;
+            tc::fence_after_sync();
+            bool sel[BPT];
+            float cand[BPT], sbar[BPT], l2[BPT];
+#pragma unroll
+            for (int b = 0; b < BPT; ++b) {
+                const int j = jt * BPT + b;
+                sel[b] = (__ldg(mrow + (j >> 5)) >> (j & 31)) & 1u;
+            }
+            // pass 1: per-block statistics of the logits
+#pragma unroll
+            for (int b = 0; b < BPT; ++b) {
+                float mx = -INFINITY, sm = 0.f, sq = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPB; ++c) {
+                    uint32_t raw[32];
+                    tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float x = __uint_as_float(raw[e]);
+                        mx = fmaxf(mx, x);
+                        sm += x;
+                        sq = fmaf(x, x, sq);
+                    }
+                }
+                if (sel[b]) {
+                    cand[b] = mx * LOG2E;
+                    sbar[b] = 0.f;
+                    l2[b] = 0.f;
+                } else {
+                    const float sb = sm * inv_bs;
+                    float w = 0.f;
+                    if (order == 2) {
+                        w = 0.5f * fmaf(-sb, sb, sq * inv_bs);
+                        if (gate && w > ln_b) w = 0.f;
+                    }
+                    sbar[b] = sb;
+                    l2[b] = (sb + w) * LOG2E;
+                    cand[b] = l2[b];
+                }
+            }
+            float mc = cand[0];
+#pragma unroll
+            for (int b = 1; b < BPT; ++b) mc = fmaxf(mc, cand[b]);
+            // raise the running max only when it grows by more than 2^8; the
+            // decision is per row, the O correction is done by the whole warp
+            const bool raise = mc > m_run + 8.0f;
+            const float scale = raise ? tc::ex2(m_run - mc) : 1.0f;
+            if (raise) {
+                dsum *= scale;
+                m_run = mc;
+            }
+            if (__any_sync(0xffffffffu, raise) && jt > 0) {
+                // the previous PV of this tile is complete (covered by S_FULL)
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t raw[32];
+                    tc::tmem_ld32(o_addr + c * 32, raw);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
+                    tc::tmem_st32(o_addr + c * 32, raw);
+                }
+            }
+            // pass 2: weights, written as bf16 over the S columns
+#pragma unroll
+            for (int b = 0; b < BPT; ++b) {
+                if (sel[b]) {
+#pragma unroll
+                    for (int c = 0; c < CPB; ++c) {
+                        uint32_t raw[32], pk[16];
+                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = tc::ex2(fmaf(__uint_as_float(raw[2 * e]), LOG2E, -m_run));
+                            const float p1 = tc::ex2(fmaf(__uint_as_float(raw[2 * e + 1]), LOG2E, -m_run));
+                            dsum += p0 + p1;
+                            pk[e] = tc::pack_bf16x2(p0, p1);
+                        }
+                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                    }
+                } else {
+                    const float alpha = tc::ex2(l2[b] - m_run);
+                    dsum = fmaf((float)BS, alpha, dsum);
+                    if (order >= 1) {
+                        const float c0 = alpha * (1.0f - sbar[b]);
+#pragma unroll
+                        for (int c = 0; c < CPB; ++c) {
+                            uint32_t raw[32], pk[16];
+                            tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                pk[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(raw[2 * e]), c0),
+                                                        fmaf(alpha, __uint_as_float(raw[2 * e + 1]), c0));
+                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                        }
+                    } else {
+                        uint32_t pk[16];
+                        const uint32_t a2 = tc::pack_bf16x2(alpha, alpha);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = a2;
+#pragma unroll
+                        for (int c = 0; c < CPB; ++c) tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                    }
+                }
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_PFULL + h));
+        }
+        // epilogue: o = N / D
+        if (tc::mbar_wait_warp(bar(B_OFULL + h), 0, aborted, status, kWaitLimitCycles)) {
+            tc::fence_after_sync();
+            const float inv = 1.0f / dsum;
+            bf16* orow = out + ((size_t)bh * L + (valid ? qrow : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t raw[32];
+                tc::tmem_ld32(o_addr + c * 32, raw);
+                tc::tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = tc::pack_bf16x2(__uint_as_float(raw[2 * e]) * inv, __uint_as_float(raw[2 * e + 1]) * inv);
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+inline bool attn_tc_supported(int d, int B) { return (d == 64 || d == 128) && (B == 64 || B == 128); }
+
+// Host: build the tensor maps and launch.  Requires L % 128 == 0 (checked).
+inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, const uint32_t* mask, void* out, long BH,
+                               int L, int d, int B, int nblk, int words, int order, int gate, unsigned* status,
+                               cudaStream_t s, std::string* err) {
+    if (L % 128) {
+        *err = "tensor-core path needs L % 128 == 0";
+        return PISA_ERR_UNSUPPORTED;
+    }
+    if (BH * (long)L > 0x7fffffffL) {
+        *err = "tensor-core path needs batch*heads*L < 2^31";
+        return PISA_ERR_UNSUPPORTED;
+    }
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess || !fn) {
+            *err = "cuTensorMapEncodeTiled not available";
+            return PISA_ERR_CUDA;
+        }
+        encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    }
+    CUtensorMap maps[3];
+    const void* ptrs[3] = {q, k, v};
+    for (int t = 0; t < 3; ++t) {
+        cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)(BH * L)};
+        cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
+        cuuint32_t box[2] = {64, 128};
+        cuuint32_t estride[2] = {1, 1};
+        CUresult cr = encode(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[t]), gdim, gstride,
+                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS) {
+            *err = "cuTensorMapEncodeTiled failed (" + std::to_string((int)cr) + ")";
+            return PISA_ERR_CUDA;
+        }
+    }
+    const float ln_b = logf((float)B);
+    dim3 grid((unsigned)((L + 255) / 256), (unsigned)BH);
+    cudaError_t e = cudaSuccess;
+#define PISA_TC_LAUNCH(DD, BB)                                                                                 \
+    if (d == DD && B == BB) {                                                                                  \
+        auto kern = attn_tc_kernel<DD, BB>;                                                                    \
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcCfg<DD>::SMEM);     \
+        if (e == cudaSuccess) {                                                                                \
+            kern<<<grid, kTcThreads, TcCfg<DD>::SMEM, s>>>(maps[0], maps[1], maps[2], mask, (bf16*)out, L, nblk, \
+                                                           words, order, gate, ln_b, status);                 \
+            e = cudaGetLastError();                                                                            \
+        }                                                                                                      \
+    } else
+    PISA_TC_LAUNCH(64, 64)
+    PISA_TC_LAUNCH(64, 128)
+    PISA_TC_LAUNCH(128, 64)
+    PISA_TC_LAUNCH(128, 128) {
+        *err = "no tensor-core kernel for this d/B";
+        return PISA_ERR_UNSUPPORTED;
+    }
+#undef PISA_TC_LAUNCH
+    if (e != cudaSuccess) {
+        *err = std::string("attn_tc_kernel launch: ") + cudaGetErrorString(e);
+        return PISA_ERR_CUDA;
+    }
+    return PISA_OK;
+}
+
+}  // namespace pisa

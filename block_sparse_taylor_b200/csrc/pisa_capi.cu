@@ -1,0 +1,460 @@
+// C ABI of the piecewise sparse attention library (declared in include/pisa.h).
+//
+// Host side only: argument validation, workspace layout, kernel selection and
+// launches.  Every launch is asynchronous on the caller's stream; nothing here
+// allocates device memory or synchronises, except pisa_poll_device_status.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/pisa.h"
+#include "common.cuh"
+#include "stats.cuh"
+#include "select.cuh"
+#include "attn_stats.cuh"
+#include "attn_tc.cuh"
+
+using pisa::bf16;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// One status word per device (module-scope device variable).
+__device__ unsigned int g_device_status;
+
+pisa_status fail(pisa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+pisa_status fail(pisa_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+pisa_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(PISA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+unsigned int* device_status_ptr() {
+    static unsigned int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        cache[dev] = (unsigned int*)p;
+    }
+    return cache[dev];
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+size_t esize(pisa_dtype t) { return t == PISA_BF16 ? 2 : 4; }
+
+struct Dims {
+    long BH, L, d, B, nblk, words;
+};
+
+// Shape validation common to every entry point.
+pisa_status check_dims(int batch, int heads, int L, int d, int B, int order, pisa_dtype dtype, Dims* out) {
+    if (batch <= 0 || heads <= 0 || L <= 0 || d <= 0 || B <= 0)
+        return fail(PISA_ERR_INVALID_ARG, "batch, heads, L, d and B must be positive");
+    if (dtype != PISA_F32 && dtype != PISA_BF16) return fail(PISA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (order < 0 || order > 2) return fail(PISA_ERR_INVALID_ARG, "order must be 0, 1 or 2 (got %d)", order);
+    if (L % B) return fail(PISA_ERR_INVALID_ARG, "L (%d) must be a multiple of B (%d)", L, B);
+    if (d != 64 && d != 128) return fail(PISA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+    if (B != 64 && B != 128) return fail(PISA_ERR_UNSUPPORTED, "B must be 64 or 128 (got %d)", B);
+    const long nblk = L / B;
+    if (nblk > 4096) return fail(PISA_ERR_UNSUPPORTED, "L/B must be <= 4096 (got %ld)", nblk);
+    out->BH = (long)batch * heads;
+    out->L = L;
+    out->d = d;
+    out->B = B;
+    out->nblk = nblk;
+    out->words = (nblk + 31) / 32;
+    return PISA_OK;
+}
+
+struct StatsLayout {
+    size_t kbar, vsum, hstat, cov, total;
+};
+
+StatsLayout stats_layout(const Dims& g, int order, pisa_dtype dtype) {
+    StatsLayout s{};
+    size_t o = 0;
+    s.kbar = o;
+    o += align_up(sizeof(float) * g.BH * g.nblk * g.d);
+    s.vsum = o;
+    o += align_up(sizeof(float) * g.BH * g.nblk * g.d);
+    s.hstat = o;
+    if (order >= 1) o += align_up(esize(dtype) * g.BH * g.nblk * g.d * g.d);
+    s.cov = o;
+    if (order == 2) o += align_up(esize(dtype) * g.BH * g.nblk * g.d * g.d);
+    s.total = o;
+    return s;
+}
+
+int next_pow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers (template dispatch over dtype, d, B)
+// ---------------------------------------------------------------------------
+
+template <typename F>
+pisa_status dispatch(pisa_dtype dtype, int d, int B, F&& f) {
+#define PISA_CASE(T, DD, BB) \
+    if (d == DD && B == BB) return f(T(), std::integral_constant<int, DD>(), std::integral_constant<int, BB>());
+    if (dtype == PISA_BF16) {
+        PISA_CASE(bf16, 64, 64)
+        PISA_CASE(bf16, 64, 128)
+        PISA_CASE(bf16, 128, 64)
+        PISA_CASE(bf16, 128, 128)
+    } else {
+        PISA_CASE(float, 64, 64)
+        PISA_CASE(float, 64, 128)
+        PISA_CASE(float, 128, 64)
+        PISA_CASE(float, 128, 128)
+    }
+#undef PISA_CASE
+    return fail(PISA_ERR_UNSUPPORTED, "no kernel for d=%d B=%d", d, B);
+}
+
+template <typename K>
+pisa_status set_smem(K kernel, size_t bytes) {
+    static int max_optin = -1;
+    if (max_optin < 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            max_optin = 0;
+    }
+    if ((long)bytes > max_optin)
+        return fail(PISA_ERR_UNSUPPORTED, "kernel needs %zu bytes of shared memory (device allows %d)", bytes,
+                    max_optin);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    return PISA_OK;
+}
+
+pisa_status launch_check(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return PISA_OK;
+}
+
+pisa_status run_centroids(const void* k, float* kbar, const Dims& g, pisa_dtype dtype, cudaStream_t s) {
+    return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        pisa::centroid_kernel<T, D, BS><<<grid, D, 0, s>>>((const T*)k, kbar, (int)g.L, (int)g.nblk);
+        return launch_check("centroid_kernel");
+    });
+}
+
+pisa_status run_stats(const void* k, const void* v, const pisa_stats_t* st, const Dims& g, cudaStream_t s) {
+    return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const size_t smem = sizeof(float) * ((size_t)2 * BS * (D + 1) + D);
+        auto kern = pisa::stats_simt_kernel<T, D, BS>;
+        pisa_status r = set_smem(kern, smem);
+        if (r != PISA_OK) return r;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        kern<<<grid, 256, smem, s>>>((const T*)k, (const T*)v, st->kbar, st->vsum, (T*)st->hstat, (T*)st->cov,
+                                     (int)g.L, (int)g.nblk, st->order);
+        return launch_check("stats_simt_kernel");
+    });
+}
+
+pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dtype dtype, int K, int32_t* idx,
+                       uint32_t* mask, cudaStream_t s) {
+    return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const int P = next_pow2((int)g.nblk < 2 ? 2 : (int)g.nblk);
+        const size_t smem = sizeof(unsigned long long) * P + sizeof(float) * D + sizeof(uint32_t) * 2 * g.words;
+        auto kern = pisa::select_kernel<T, D, BS>;
+        pisa_status r = set_smem(kern, smem);
+        if (r != PISA_OK) return r;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        kern<<<grid, 256, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K, (int)g.words, P, idx, mask);
+        return launch_check("select_kernel");
+    });
+}
+
+pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pisa_stats_t* st,
+                           const uint32_t* mask, void* out, const Dims& g, int order, int gate,
+                           cudaStream_t s) {
+    return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const size_t smem = pisa::AttnStatsSmem<T, D, BS>::bytes;
+        auto kern = pisa::attn_stats_kernel<T, D, BS>;
+        pisa_status r = set_smem(kern, smem);
+        if (r != PISA_OK) return r;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        kern<<<grid, 256, smem, s>>>((const T*)q, (const T*)k, (const T*)v, st->kbar, st->vsum,
+                                     (const T*)st->hstat, (const T*)st->cov, mask, (T*)out, (int)g.L,
+                                     (int)g.nblk, (int)g.words, order, gate, logf((float)g.B));
+        return launch_check("attn_stats_kernel");
+    });
+}
+
+// ---------------------------------------------------------------------------
+// workspace layout of pisa_attention
+// ---------------------------------------------------------------------------
+struct WsLayout {
+    size_t stats, mask, idx, total;
+    StatsLayout sl;
+};
+
+WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path path) {
+    WsLayout w{};
+    // The recompute path needs only the centroids (for the selection).
+    const int stats_order = (path == PISA_PATH_RECOMPUTE_TC) ? 0 : order;
+    w.sl = stats_layout(g, stats_order, dtype);
+    size_t o = 0;
+    w.stats = o;
+    o += w.sl.total;
+    w.mask = o;
+    o += align_up(sizeof(uint32_t) * g.BH * g.nblk * g.words);
+    w.idx = o;
+    o += align_up(sizeof(int32_t) * g.BH * g.nblk * (K > 0 ? K : 1));
+    w.total = o;
+    return w;
+}
+
+bool tc_path_available(const Dims& g, pisa_dtype dtype) {
+    return dtype == PISA_BF16 && pisa::attn_tc_supported((int)g.d, (int)g.B) && g.L % 128 == 0 &&
+           g.BH * g.L <= 0x7fffffffL;
+}
+
+// The tensor-core token-form path whenever it can run the shape, else the
+// statistics path on CUDA cores.
+pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
+    (void)K;
+    (void)order;
+    return tc_path_available(g, dtype) ? PISA_PATH_RECOMPUTE_TC : PISA_PATH_STATS;
+}
+
+pisa_status check_stats(const pisa_stats_t* st, Dims* g) {
+    if (!st) return fail(PISA_ERR_INVALID_ARG, "null pisa_stats_t");
+    pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, st->order, st->dtype, g);
+    if (r != PISA_OK) return r;
+    if (st->nblk != g->nblk) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t.nblk inconsistent with L/B");
+    if (!st->kbar || !st->vsum) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null kbar or vsum");
+    if (st->order >= 1 && !st->hstat) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null hstat for order >= 1");
+    if (st->order == 2 && !st->cov) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null cov for order 2");
+    return PISA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pisa_version(void) { return "pisa-b200 0.1"; }
+
+const char* pisa_last_error(void) { return g_last_error.c_str(); }
+
+size_t pisa_stats_bytes(int batch, int heads, int L, int d, int B, int order, pisa_dtype dtype) {
+    Dims g;
+    if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return 0;
+    return stats_layout(g, order, dtype).total;
+}
+
+pisa_status pisa_stats_bind(pisa_stats_t* st, void* buf, size_t bytes, int batch, int heads, int L, int d, int B,
+                            int order, pisa_dtype dtype) {
+    if (!st || !buf) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_bind: null st or buf");
+    if ((uintptr_t)buf % kAlign) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_bind: buf must be 256-byte aligned");
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    StatsLayout s = stats_layout(g, order, dtype);
+    if (bytes < s.total)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_stats_bind: buffer of %zu bytes, need %zu", bytes, s.total);
+    char* b = (char*)buf;
+    st->batch = batch;
+    st->heads = heads;
+    st->L = L;
+    st->d = d;
+    st->B = B;
+    st->nblk = (int)g.nblk;
+    st->order = order;
+    st->dtype = dtype;
+    st->kbar = (float*)(b + s.kbar);
+    st->vsum = (float*)(b + s.vsum);
+    st->hstat = order >= 1 ? (void*)(b + s.hstat) : nullptr;
+    st->cov = order == 2 ? (void*)(b + s.cov) : nullptr;
+    return PISA_OK;
+}
+
+pisa_status pisa_stats(const void* k, const void* v, const pisa_stats_t* st, void* stream) {
+    Dims g;
+    pisa_status r = check_stats(st, &g);
+    if (r != PISA_OK) return r;
+    if (!k || !v) return fail(PISA_ERR_INVALID_ARG, "pisa_stats: null k or v");
+    return run_stats(k, v, st, g, (cudaStream_t)stream);
+}
+
+pisa_status pisa_select(const void* q, const pisa_stats_t* st, int K, int32_t* idx, uint32_t* mask, void* stream) {
+    Dims g;
+    if (!st) return fail(PISA_ERR_INVALID_ARG, "null pisa_stats_t");
+    pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, 0, st->dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!st->kbar) return fail(PISA_ERR_INVALID_ARG, "pisa_select: null kbar");
+    if (!q) return fail(PISA_ERR_INVALID_ARG, "pisa_select: null q");
+    if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
+    if (!idx && !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_select: idx and mask both null");
+    return run_select(q, st->kbar, g, st->dtype, K, K > 0 ? idx : nullptr, mask, (cudaStream_t)stream);
+}
+
+int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order, pisa_dtype dtype) {
+    Dims g;
+    if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return -1;
+    if (K < 0 || K > g.nblk) return -1;
+    return (int)resolve(g, K, order, dtype);
+}
+
+size_t pisa_workspace_bytes_ex(int batch, int heads, int L, int d, int B, int K, int order, pisa_dtype dtype,
+                               pisa_path path) {
+    Dims g;
+    if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return 0;
+    if (K < 0 || K > g.nblk) return 0;
+    if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
+    if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype)) return 0;
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC) return 0;
+    return ws_layout(g, K, order, dtype, path).total;
+}
+
+size_t pisa_workspace_bytes(int batch, int heads, int L, int d, int B, int K, int order, pisa_dtype dtype) {
+    return pisa_workspace_bytes_ex(batch, heads, L, d, B, K, order, dtype, PISA_PATH_AUTO);
+}
+
+pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                              pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
+    if (!q || !k || !v || !out) return fail(PISA_ERR_INVALID_ARG, "pisa_attention: null q, k, v or out");
+    if (!workspace) return fail(PISA_ERR_INVALID_ARG, "pisa_attention: null workspace");
+    if ((uintptr_t)workspace % kAlign)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention: workspace must be 256-byte aligned");
+    if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
+    if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype))
+        return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC)
+        return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
+    const WsLayout w = ws_layout(g, K, order, dtype, path);
+    if (ws_bytes < w.total)
+        return fail(PISA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, w.total);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    pisa_stats_t st{};
+    st.batch = batch;
+    st.heads = heads;
+    st.L = L;
+    st.d = d;
+    st.B = B;
+    st.nblk = (int)g.nblk;
+    st.dtype = dtype;
+    st.order = (path == PISA_PATH_RECOMPUTE_TC) ? 0 : order;
+    st.kbar = (float*)(ws + w.stats + w.sl.kbar);
+    st.vsum = (float*)(ws + w.stats + w.sl.vsum);
+    st.hstat = st.order >= 1 ? (void*)(ws + w.stats + w.sl.hstat) : nullptr;
+    st.cov = st.order == 2 ? (void*)(ws + w.stats + w.sl.cov) : nullptr;
+    uint32_t* mask = (uint32_t*)(ws + w.mask);
+    int32_t* idx = (int32_t*)(ws + w.idx);
+
+    if (path == PISA_PATH_RECOMPUTE_TC) {
+        r = run_centroids(k, st.kbar, g, dtype, s);
+        if (r != PISA_OK) return r;
+    } else {
+        r = run_stats(k, v, &st, g, s);
+        if (r != PISA_OK) return r;
+    }
+    r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s);
+    if (r != PISA_OK) return r;
+    if (path == PISA_PATH_RECOMPUTE_TC) {
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
+                                 (int)g.words, order, gate_w, status, s, &g_last_error);
+    }
+    return run_attn_stats(q, k, v, &st, mask, out, g, order, gate_w, s);
+}
+
+pisa_status pisa_attention(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                           pisa_dtype dtype, int B, int K, int order, void* out, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    return pisa_attention_ex(q, k, v, batch, heads, L, d, dtype, B, K, order, 1, PISA_PATH_AUTO, out, workspace,
+                             ws_bytes, stream);
+}
+
+pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pisa_dtype dtype, int B, float* kbar,
+                           void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, 0, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!k || !kbar) return fail(PISA_ERR_INVALID_ARG, "pisa_centroids: null k or kbar");
+    return run_centroids(k, kbar, g, dtype, (cudaStream_t)stream);
+}
+
+pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                                 pisa_dtype dtype, int B, int order, int gate_w, pisa_path path,
+                                 const uint32_t* mask, const pisa_stats_t* st, void* out, void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!q || !k || !v || !out || !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: null pointer");
+    if (path == PISA_PATH_AUTO) path = resolve(g, 0, order, dtype);
+    if (path == PISA_PATH_RECOMPUTE_TC) {
+        if (!tc_path_available(g, dtype))
+            return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
+                                 (int)g.words, order, gate_w, status, (cudaStream_t)stream, &g_last_error);
+    }
+    if (path != PISA_PATH_STATS) return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
+    Dims gs;
+    r = check_stats(st, &gs);
+    if (r != PISA_OK) return r;
+    if (gs.BH != g.BH || gs.L != g.L || gs.d != g.d || gs.B != g.B || st->dtype != dtype)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: statistics of another shape");
+    if (st->order < order) return fail(PISA_ERR_INVALID_ARG, "statistics of order %d for attention of order %d",
+                                       st->order, order);
+    return run_attn_stats(q, k, v, st, mask, out, g, order, gate_w, (cudaStream_t)stream);
+}
+
+pisa_status pisa_poll_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int* p = device_status_ptr();
+    if (!p) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    const unsigned int zero = 0;
+    e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status reset)");
+    if (v & pisa::kStatusTimeout)
+        return fail(PISA_ERR_DEVICE_TIMEOUT, "a device-side wait gave up (status 0x%x)", v);
+    if (v) return fail(PISA_ERR_CUDA, "device status 0x%x", v);
+    return PISA_OK;
+}
+
+}  // extern "C"

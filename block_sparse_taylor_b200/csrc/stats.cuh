@@ -1,0 +1,111 @@
+// Prepare phase: per key block j of B tokens, the centroid kbar_j, the value
+// sum vsum_j, the first-order cross statistic H_j and the key covariance C_j.
+//
+// PISA paper, section 3.4 and Figure 3 (centroids and value sums computed in
+// one pass before the fused kernel); "Sparse Linear Attention" blog, section
+// "Sparse Linear Attention" (H_j = sum_n v_n (k_n - kbar_j)^T) and section
+// "Going Further: Adding the Second-Order Term (PWT)" (C_j, the within-block
+// key covariance with the 1/B normalisation).
+#pragma once
+
+#include "common.cuh"
+
+namespace pisa {
+
+// Centroid of every key block in the canonical fp32 order: thread c owns
+// column c, holds the B values in registers and reduces them with the
+// pairwise tree; the mean is the tree sum times 1/B (exact for B = 2^k).
+// grid (nblk, BH), block D threads.
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(D) centroid_kernel(const T* __restrict__ k, float* __restrict__ kbar,
+                                                     int L, int nblk) {
+    const int j = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+    const T* src = k + ((size_t)bh * L + (size_t)j * BS) * D + c;
+    float a[BS];
+#pragma unroll
+    for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
+    const float s = tree_sum<BS>(a);
+    kbar[((size_t)bh * nblk + j) * D + c] = __fmul_rn(s, 1.0f / (float)BS);
+}
+
+// Full statistics on CUDA cores.  One CTA per (block, bh), 256 threads.
+// The keys are centred in shared memory with the canonical centroid, then
+// H_j[a][b] = sum_n v[n][a] dev[n][b] and C_j[a][b] = (1/B) sum_n dev[n][a] dev[n][b]
+// are accumulated in fp32; each thread owns a (D/16) x (D/16) tile of outputs
+// with rows a = a0 + 16*i and columns b = b0 + 16*i' (conflict-free reads).
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(256) stats_simt_kernel(const T* __restrict__ k, const T* __restrict__ v,
+                                                         float* __restrict__ kbar, float* __restrict__ vsum,
+                                                         T* __restrict__ hstat, T* __restrict__ cov, int L,
+                                                         int nblk, int order) {
+    constexpr int S = D + 1;  // padded fp32 row stride
+    constexpr int R = D / 16;
+    extern __shared__ __align__(16) float sm_stats[];
+    float* ks = sm_stats;       // [BS][S] keys, then deviations
+    float* vs = ks + BS * S;    // [BS][S]
+    float* kb = vs + BS * S;    // [D]
+    const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const size_t base = ((size_t)bh * L + (size_t)j * BS) * D;
+    for (int e = tid; e < BS * D; e += 256) {
+        const int n = e / D, c = e % D;
+        ks[n * S + c] = to_f(k[base + e]);
+        vs[n * S + c] = to_f(v[base + e]);
+    }
+    __syncthreads();
+    const size_t so = ((size_t)bh * nblk + j) * D;
+    if (tid < D) {
+        float a[BS];
+#pragma unroll
+        for (int n = 0; n < BS; ++n) a[n] = ks[n * S + tid];
+        const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+        kb[tid] = m;
+        kbar[so + tid] = m;
+        float s = 0.f;
+        for (int n = 0; n < BS; ++n) s += vs[n * S + tid];
+        vsum[so + tid] = s;
+    }
+    __syncthreads();
+    if (order == 0) return;
+    for (int e = tid; e < BS * D; e += 256) {
+        const int n = e / D, c = e % D;
+        ks[n * S + c] -= kb[c];
+    }
+    __syncthreads();
+    const int a0 = tid / 16, b0 = tid % 16;
+    float h[R][R], cv[R][R];
+#pragma unroll
+    for (int x = 0; x < R; ++x)
+#pragma unroll
+        for (int y = 0; y < R; ++y) h[x][y] = cv[x][y] = 0.f;
+    const bool want_c = (order == 2);
+    for (int n = 0; n < BS; ++n) {
+        float va[R], da[R], db[R];
+#pragma unroll
+        for (int x = 0; x < R; ++x) {
+            va[x] = vs[n * S + a0 + 16 * x];
+            da[x] = ks[n * S + a0 + 16 * x];
+            db[x] = ks[n * S + b0 + 16 * x];
+        }
+#pragma unroll
+        for (int x = 0; x < R; ++x)
+#pragma unroll
+            for (int y = 0; y < R; ++y) h[x][y] = fmaf(va[x], db[y], h[x][y]);
+        if (want_c) {
+#pragma unroll
+            for (int x = 0; x < R; ++x)
+#pragma unroll
+                for (int y = 0; y < R; ++y) cv[x][y] = fmaf(da[x], db[y], cv[x][y]);
+        }
+    }
+    const size_t ho = ((size_t)bh * nblk + j) * D * D;
+#pragma unroll
+    for (int x = 0; x < R; ++x)
+#pragma unroll
+        for (int y = 0; y < R; ++y) {
+            const int a = a0 + 16 * x, b = b0 + 16 * y;
+            hstat[ho + a * D + b] = from_f<T>(h[x][y]);
+            if (want_c) cov[ho + a * D + b] = from_f<T>(cv[x][y] * (1.0f / (float)BS));
+        }
+}
+
+}  // namespace pisa

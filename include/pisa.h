@@ -1,0 +1,188 @@
+/*
+ * pisa.h -- C ABI of the B200 (sm_100a) piecewise sparse attention library.
+ *
+ * The operation (PISA / PWT piecewise sparse attention):
+ *   Keys and values of each (batch, head) are cut in order into blocks of B
+ *   tokens.  Query tile i (rows iB .. iB+B-1) keeps the K key blocks whose
+ *   centroid scores highest against the tile's mean query (S_i) and gets exact
+ *   softmax attention on them; every other block j (U_i) is replaced by its
+ *   Taylor expansion around the key centroid kbar_j.  Both parts share one
+ *   softmax max and one denominator:
+ *     D_t = sum_{j in S_i} sum_n e^{q_t.k_{j,n}} + sum_{j in U_i} B e^{l_tj}
+ *     N_t = sum_{j in S_i} sum_n e^{q_t.k_{j,n}} v_{j,n}
+ *         + sum_{j in U_i} e^{l_tj} (vsum_j + [order>=1] H_j q_t)
+ *     o_t = N_t / D_t,   l_tj = q_t.kbar_j + w_tj,
+ *     w_tj = [order==2] 1/2 q_t^T C_j q_t  (set to 0 when it exceeds ln B and
+ *            the gate is on).
+ *   Definitions: PISA paper ("PISA: Piecewise Sparse Attention Is Wiser for
+ *   Efficient Diffusion Transformers"), section 3.2 "Formulation" (o_t, D_t),
+ *   Figure 3 caption and section 3.4 (prepare phase, phases 1-2), Appendix C
+ *   "Notation" (kbar_j, alpha_tj, delta_tjn); "Sparse Linear Attention" blog,
+ *   sections "Sparse Linear Attention" (virtual token, H_j) and "Going Further:
+ *   Adding the Second-Order Term (PWT)" (w_tj, C_j, the ln B gate).
+ *   The softmax scale is folded into q: callers pass q already multiplied by
+ *   1/sqrt(d) (PISA paper section 3.1, Eq. 1; blog notation paragraph).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major [batch*heads, L, d] ("BHLD" with batch and heads
+ *     folded), contiguous, element type given by pisa_dtype.
+ *   - Every pointer argument is device memory owned by the caller unless a
+ *     comment says otherwise.  The library allocates no memory (except the
+ *     variant documented at its declaration) and keeps no state other than one
+ *     device status word per device.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it; no call
+ *     synchronises the host, except pisa_poll_device_status.
+ *   - Supported on the GPU path: d in {64, 128}, B in {64, 128}, L % B == 0,
+ *     0 <= K <= L/B, order in {0, 1, 2}, L/B <= 4096.  Other shapes return
+ *     PISA_ERR_UNSUPPORTED (valid but not implemented) or
+ *     PISA_ERR_INVALID_ARG (meaningless).
+ *   - Non-finite inputs give undefined (but memory-safe) results.
+ *   - On a non-OK status, pisa_last_error() returns a message for the calling
+ *     thread.  Argument errors are detected before anything is enqueued.
+ */
+#ifndef PISA_H_
+#define PISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PISA_OK = 0,
+    PISA_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, workspace too small */
+    PISA_ERR_UNSUPPORTED = 2,    /* valid but not implemented on this path */
+    PISA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+    PISA_ERR_DEVICE_TIMEOUT = 4  /* a bounded device-side wait gave up */
+} pisa_status;
+
+typedef enum { PISA_F32 = 0, PISA_BF16 = 1 } pisa_dtype;
+
+/* Which formulation pisa_attention_ex evaluates the unselected blocks with.
+ *   PISA_PATH_AUTO          : PISA_PATH_RECOMPUTE_TC when it can run the
+ *                             shape, else PISA_PATH_STATS.
+ *   PISA_PATH_STATS         : statistics form: uses kbar_j, vsum_j, H_j, C_j
+ *                             from pisa_stats (CUDA cores, fp32 accumulation).
+ *   PISA_PATH_RECOMPUTE_TC  : token form on tcgen05 tensor cores: the
+ *                             unselected block's first-order numerator
+ *                             e^{l}(vsum_j + H_j q) is evaluated as
+ *                             sum_n e^{l}(1 + q.(k_n - kbar_j)) v_n, which is
+ *                             the same quantity; w is taken from the same
+ *                             logits.  bf16 only, L % 128 == 0. */
+typedef enum {
+    PISA_PATH_AUTO = 0,
+    PISA_PATH_STATS = 1,
+    PISA_PATH_RECOMPUTE_TC = 2
+} pisa_path;
+
+/* Block statistics of one call (all device pointers, caller-owned).
+ *   kbar  [BH, nblk, d] fp32 : centroid, canonical fp32 mean (see pisa_select)
+ *   vsum  [BH, nblk, d] fp32 : sum_n v_{j,n}
+ *   hstat [BH, nblk, d, d]   : H_j[a][b] = sum_n v_{j,n}[a] (k_{j,n}[b] - kbar_j[b])
+ *                              (row = value channel), element type = dtype
+ *   cov   [BH, nblk, d, d]   : C_j = (1/B) sum_n (k-kbar)(k-kbar)^T, element
+ *                              type = dtype; NULL unless order == 2.
+ * hstat is NULL when order == 0.  Fill with pisa_stats_bind. */
+typedef struct {
+    int batch, heads, L, d, B, nblk, order;
+    pisa_dtype dtype;
+    float* kbar;
+    float* vsum;
+    void* hstat;
+    void* cov;
+} pisa_stats_t;
+
+/* Bytes of device memory pisa_stats_bind needs for these dimensions
+ * (each array 256-byte aligned).  Returns 0 for invalid dimensions. */
+size_t pisa_stats_bytes(int batch, int heads, int L, int d, int B, int order, pisa_dtype dtype);
+
+/* Lay out a pisa_stats_t inside caller memory `buf` of `bytes` bytes
+ * (buf 256-byte aligned).  No device work.  Errors: INVALID_ARG for a null
+ * st/buf, a too-small buffer or invalid dimensions. */
+pisa_status pisa_stats_bind(pisa_stats_t* st, void* buf, size_t bytes, int batch, int heads,
+                            int L, int d, int B, int order, pisa_dtype dtype);
+
+/* Prepare phase (PISA paper section 3.4, Figure 3): one pass over k and v
+ * ([BH, L, d], element type st->dtype) writing every array of *st. */
+pisa_status pisa_stats(const void* k, const void* v, const pisa_stats_t* st, void* stream);
+
+/* Block selection (PISA paper section 3.2 and Figure 3; MoBA-style scoring,
+ * "Sparse Linear Attention" blog section "Sparse Attention").
+ * For each query tile i of q ([BH, L, d], type st->dtype), in fp32 with a fixed
+ * reduction order so that the result is reproducible bit for bit:
+ *   tsum(a[0..n)) : for h = n/2, ..., 1: a[i] = a[i] + a[i+h] (i < h); a[0]
+ *   qbar_i[c] = tsum(q rows of the tile, column c) * (1/B)
+ *   s_ij      = tsum over c of (qbar_i[c] * st->kbar[j][c])   (rounded products)
+ *   S_i       = the K blocks first under (s descending, j ascending).
+ * Outputs: idx [BH, nblk, K] int32, each row ascending (may be NULL);
+ *          mask [BH, nblk, ceil(nblk/32)] uint32, bit j%32 of word j/32 set iff
+ *          j in S_i (may be NULL).  Only st->kbar is read (pisa_stats or
+ *          pisa_centroids output); the other arrays of *st may be NULL. */
+pisa_status pisa_select(const void* q, const pisa_stats_t* st, int K, int32_t* idx,
+                        uint32_t* mask, void* stream);
+
+/* Centroids only: kbar [BH, nblk, d] fp32 of k ([BH, L, d], `dtype`), in the
+ * canonical fp32 order of pisa_select (pairwise tree over the B rows, times
+ * 1/B).  This is the part of the prepare phase the token-form path needs. */
+pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pisa_dtype dtype, int B,
+                           float* kbar, void* stream);
+
+/* The fused attention kernel alone, given a selection mask from pisa_select
+ * (phases 1-2 of the PISA paper's section 3.4 plus the normalisation).
+ *   path PISA_PATH_STATS needs `st` (pisa_stats output with st->order >= order);
+ *   path PISA_PATH_RECOMPUTE_TC ignores `st` (may be NULL); AUTO picks as
+ *   pisa_attention does.
+ * mask: [BH, nblk, ceil(nblk/32)] uint32 as written by pisa_select. */
+pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, int batch, int heads, int L,
+                                 int d, pisa_dtype dtype, int B, int order, int gate_w, pisa_path path,
+                                 const uint32_t* mask, const pisa_stats_t* st, void* out, void* stream);
+
+/* Device workspace pisa_attention needs (bytes) for the AUTO path. */
+size_t pisa_workspace_bytes(int batch, int heads, int L, int d, int B, int K, int order,
+                            pisa_dtype dtype);
+
+/* Workspace for an explicit path; 0 if the path cannot run this shape. */
+size_t pisa_workspace_bytes_ex(int batch, int heads, int L, int d, int B, int K, int order,
+                               pisa_dtype dtype, pisa_path path);
+
+/* Full forward pass: statistics, selection and the fused attention, enqueued
+ * on `stream`.  q, k, v: [BH, L, d] of `dtype`; q pre-scaled by 1/sqrt(d).
+ * out: [BH, L, d] of `dtype` (bf16 output is rounded to nearest even from fp32).
+ * workspace: caller device memory of ws_bytes >= pisa_workspace_bytes(...),
+ * 256-byte aligned; its contents on return are the statistics and the
+ * selection of this call.  Gate on for order 2. */
+pisa_status pisa_attention(const void* q, const void* k, const void* v, int batch, int heads,
+                           int L, int d, pisa_dtype dtype, int B, int K, int order, void* out,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* As pisa_attention with the PWT gate switchable (gate_w = 0: w is never
+ * zeroed) and an explicit path. */
+pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads,
+                              int L, int d, pisa_dtype dtype, int B, int K, int order, int gate_w,
+                              pisa_path path, void* out, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* The path AUTO resolves to for these arguments (or -1 if none can run). */
+int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order,
+                      pisa_dtype dtype);
+
+/* Message for the last non-OK status returned on this host thread. */
+const char* pisa_last_error(void);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device.  Returns PISA_ERR_DEVICE_TIMEOUT if a bounded device-side
+ * wait of an earlier kernel gave up (that kernel's output is then invalid),
+ * PISA_ERR_CUDA on a CUDA error, PISA_OK otherwise. */
+pisa_status pisa_poll_device_status(void* stream);
+
+/* Library version string. */
+const char* pisa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H_ */

@@ -36,8 +36,9 @@ def lib():
                                             ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_bruteforce.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                              ctypes.c_int, f64p, ctypes.c_int]
+        L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
-        for fn in ("oracle_block_stats", "oracle_select", "oracle_pisa_attention",
+        for fn in ("oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
                    "oracle_pisa_bruteforce", "oracle_dense_attention"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -77,6 +78,16 @@ def block_stats(k, v, B, order=2, nthreads=None):
                                   nthreads or default_threads())
     _check(rc, "block_stats")
     return kbar, vsum, H, C
+
+
+def centroids_f32(k, B, nthreads=None):
+    """Canonical fp32 key centroids [BH, nblk, d] (tree sum times 1/B), as used by the selection."""
+    k = _f32(k)
+    BH, L, d = k.shape
+    out = np.zeros((BH, L // B, d), np.float32)
+    rc = lib().oracle_centroids_f32(k, BH, L, d, B, _ptr(out), nthreads or default_threads())
+    _check(rc, "centroids_f32")
+    return out
 
 
 def select(q, k, B, K, nthreads=None, want_scores=False):

@@ -337,6 +337,23 @@ int oracle_block_stats(const float* k, const float* v, long BH, long L, long d, 
     return 0;
 }
 
+// Canonical fp32 centroids (the means the selection uses): [BH, nblk, d].
+int oracle_centroids_f32(const float* k, long BH, long L, long d, long B, float* kbar, int nthreads) {
+    if (!is_pow2(B) || L % B) return -1;
+    const long nblk = L / B;
+    parallel_for(BH, nthreads, [&](long bh) {
+        std::vector<float> col(B);
+        const float inv_b = 1.0f / (float)B;
+        for (long j = 0; j < nblk; ++j)
+            for (long c = 0; c < d; ++c) {
+                for (long n = 0; n < B; ++n) col[n] = k[(bh * L + j * B + n) * d + c];
+                volatile float m = tree_sum_f32(col.data(), B) * inv_b;
+                kbar[(bh * nblk + j) * d + c] = m;
+            }
+    });
+    return 0;
+}
+
 int oracle_select(const float* q, const float* k, long BH, long L, long d, long B, long K,
                   int32_t* idx, uint32_t* mask, float* scores, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B) return -1;

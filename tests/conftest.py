@@ -8,6 +8,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    # Build (or refresh) the CPU oracle and the CUDA library in-tree.
+    from oracle import build as ob
+    from block_sparse_taylor_b200 import build as lb
+
+    ob.build()
+    lb.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")

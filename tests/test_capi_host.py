@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+declared in include/pisa.h, and rejects bad arguments before touching a GPU.
+
+These run without a GPU: validation happens before any CUDA call, so the
+pointers passed here are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_taylor_b200 as pisa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(pisa_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pisa_stats", "pisa_select", "pisa_attention", "pisa_workspace_bytes", "pisa_last_error",
+                     "pisa_poll_device_status", "pisa_stats_bind", "pisa_stats_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(pisa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_string():
+    assert pisa.version().startswith("pisa-b200")
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+
+
+def call_ex(L=1024, d=64, B=64, K=4, order=1, dtype=pisa.PISA_BF16, path=0, ws_bytes=1 << 30, batch=1, heads=1,
+            q=FAKE, ws=FAKE):
+    return pisa.lib().pisa_attention_ex(q, FAKE, FAKE, batch, heads, L, d, dtype, B, K, order, 1, path, FAKE, ws,
+                                        ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=1000), pisa.PISA_ERR_INVALID_ARG),          # L % B
+    (dict(K=17), pisa.PISA_ERR_INVALID_ARG),            # K > nblk
+    (dict(K=-1), pisa.PISA_ERR_INVALID_ARG),
+    (dict(order=3), pisa.PISA_ERR_INVALID_ARG),
+    (dict(dtype=7), pisa.PISA_ERR_INVALID_ARG),
+    (dict(batch=0), pisa.PISA_ERR_INVALID_ARG),
+    (dict(d=96), pisa.PISA_ERR_UNSUPPORTED),
+    (dict(B=32, L=1024), pisa.PISA_ERR_UNSUPPORTED),
+    (dict(q=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(ws=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), pisa.PISA_ERR_INVALID_ARG),
+    (dict(ws=ctypes.c_void_p(0x1008)), pisa.PISA_ERR_INVALID_ARG),  # misaligned workspace
+    (dict(path=9), pisa.PISA_ERR_INVALID_ARG),
+    (dict(path=2, dtype=pisa.PISA_F32), pisa.PISA_ERR_UNSUPPORTED),  # tensor cores need bf16
+    (dict(L=1024 * 8192, B=64), pisa.PISA_ERR_UNSUPPORTED),          # nblk > 4096
+])
+def test_bad_arguments_are_rejected_before_launch(kw, status):
+    assert call_ex(**kw) == status
+    assert len(pisa.lib().pisa_last_error()) > 0
+
+
+def test_workspace_sizes_and_paths():
+    bf, f32 = pisa.PISA_BF16, pisa.PISA_F32
+    lib = pisa.lib()
+    # fp32 can only take the statistics path
+    assert lib.pisa_resolve_path(1, 1, 1024, 64, 64, 4, 1, f32) == pisa.PATHS["stats"]
+    assert lib.pisa_resolve_path(1, 40, 32768, 128, 64, 77, 1, bf) == pisa.PATHS["recompute_tc"]
+    assert lib.pisa_resolve_path(1, 1, 1000, 64, 64, 4, 1, bf) == -1
+    ws_stats = lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 2, bf, 1)
+    ws_tc = lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 2, bf, 2)
+    # the statistics path holds H_j and C_j (2 x 12 x 128 x 64 x 64 bf16), the recompute path does not
+    assert ws_stats - ws_tc >= 2 * 12 * 128 * 64 * 64 * 2
+    assert lib.pisa_workspace_bytes_ex(1, 1, 1024, 64, 64, 4, 1, f32, 2) == 0
+    assert lib.pisa_workspace_bytes(1, 1, 1024, 64, 64, 4, 1, f32) == lib.pisa_workspace_bytes_ex(
+        1, 1, 1024, 64, 64, 4, 1, f32, 1)
+
+
+def test_stats_bind_layout():
+    st = pisa._StatsT()
+    lib = pisa.lib()
+    n = lib.pisa_stats_bytes(2, 3, 1024, 64, 64, 2, pisa.PISA_BF16)
+    assert n >= 2 * 6 * 16 * 64 * 4 + 2 * 6 * 16 * 64 * 64 * 2
+    base = 0x10000
+    assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n, 2, 3, 1024, 64, 64, 2, pisa.PISA_BF16) == 0
+    assert st.nblk == 16 and st.kbar == base and st.cov is not None and st.hstat is not None
+    assert (st.vsum - base) % 256 == 0 and (st.hstat - base) % 256 == 0 and (st.cov - base) % 256 == 0
+    assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n - 1, 2, 3, 1024, 64, 64, 2,
+                               pisa.PISA_BF16) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n, 2, 3, 1024, 64, 64, 1, pisa.PISA_BF16) == 0
+    assert st.cov is None

@@ -1,0 +1,243 @@
+"""GPU parity: every kernel of the library against the CPU oracle.
+
+* statistics: centroids bit-exact (canonical fp32), sums and d x d statistics
+  within the storage precision;
+* selection: index lists and masks bit-exact, on small shapes, planted ties and
+  every full-size workload;
+* attention: relative L2 error (||gpu - oracle||_F / ||oracle||_F) at most 1e-4
+  on the fp32 path and 2e-2 on the bf16 path, on small shapes end to end and on
+  sampled query tiles (first, last and seeded random ones) of the full-size
+  workloads, through both formulations.
+"""
+import functools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_taylor_b200 as pisa
+import oracle
+import pisa_synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+TDT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def dev(x, dt):
+    return torch.from_numpy(np.ascontiguousarray(x)).to("cuda").to(TDT[dt])
+
+
+@functools.lru_cache(maxsize=3)
+def workload(name):
+    w = pisa_synth.workloads()[name]
+    return w, pisa_synth.generate(w)
+
+
+def sample_tiles(BH, nblk, per_head, seed, heads=None):
+    rng = np.random.default_rng(seed)
+    hs = range(BH) if heads is None else heads
+    out = []
+    for bh in hs:
+        pick = {0, nblk - 1}
+        while len(pick) < min(per_head, nblk):
+            pick.add(int(rng.integers(0, nblk)))
+        out += [(bh, i) for i in sorted(pick)]
+    return out
+
+
+def rows_of(o, tiles, B):
+    return np.stack([o[bh, i * B:(i + 1) * B] for bh, i in tiles])
+
+
+def rel_l2(a, b):
+    return oracle.rel_l2(a, b)
+
+
+# ---------------------------------------------------------------------------
+# statistics
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("order", [1, 2])
+def test_stats_parity(dt, d, B, order):
+    q, k, v = pisa_synth.random_qkv(100 + d + B, 2, 1024, d, dtype=dt)
+    st = pisa.pisa_stats(dev(k, dt), dev(v, dt), B, order)
+    torch.cuda.synchronize()
+    kbar_ref = oracle.centroids_f32(k, B)
+    assert np.array_equal(st.kbar.cpu().numpy().view(np.uint32), kbar_ref.view(np.uint32))
+    _, vsum, H, C = oracle.block_stats(k, v, B, order=2)
+    assert rel_l2(st.vsum.cpu().numpy(), vsum) < 1e-6
+    tol = 1e-5 if dt == "f32" else 8e-3
+    assert rel_l2(st.hstat.float().cpu().numpy(), H) < tol
+    if order == 2:
+        assert rel_l2(st.cov.float().cpu().numpy(), C) < tol
+    else:
+        assert st.cov is None
+
+
+# ---------------------------------------------------------------------------
+# selection
+# ---------------------------------------------------------------------------
+
+def gpu_select(q, k, B, K, dt):
+    st = pisa.pisa_stats(dev(k, dt), dev(k, dt), B, 0)
+    idx, mask = pisa.pisa_select(dev(q, dt), st, K)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), mask.cpu().numpy().view(np.uint32)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d,B,L", [(64, 64, 2048), (128, 64, 4096), (128, 128, 4096), (64, 128, 1024)])
+@pytest.mark.parametrize("Kfrac", [0.0, 0.1, 0.5, 1.0])
+def test_select_parity(dt, d, B, L, Kfrac):
+    nblk = L // B
+    K = int(round(Kfrac * nblk))
+    q, k, _ = pisa_synth.random_qkv(200 + d + L, 3, L, d, scale=4.0, dtype=dt)
+    idx, mask = gpu_select(q, k, B, K, dt)
+    ridx, rmask, _ = oracle.select(q, k, B, K)
+    assert np.array_equal(mask, rmask)
+    assert np.array_equal(idx, ridx)
+
+
+def test_select_planted_ties():
+    # Key blocks whose centroids are exact multiples of unit vectors and query
+    # tiles whose means are exact, so that many scores tie exactly; the lower
+    # block index must win.
+    d, B, L = 64, 64, 64 * 16
+    nblk = L // B
+    rng = np.random.default_rng(5)
+    k = np.zeros((1, L, d), np.float32)
+    q = np.zeros((1, L, d), np.float32)
+    for j in range(nblk):
+        k[0, j * B:(j + 1) * B, j % 3] = float(1 + (j % 2))
+        q[0, j * B:(j + 1) * B, rng.integers(0, 3)] = 1.0
+    for K in (1, 3, 5, 8):
+        idx, mask = gpu_select(q, k, B, K, "f32")
+        ridx, rmask, _ = oracle.select(q, k, B, K)
+        assert np.array_equal(idx, ridx) and np.array_equal(mask, rmask)
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5_L16896_s90"])
+def test_select_full_size(name):
+    w, (q, k, v) = workload(name)
+    idx, mask = gpu_select(q, k, w.B, w.K, w.dtype)
+    ridx, rmask, _ = oracle.select(q, k, w.B, w.K)
+    assert np.array_equal(mask, rmask)
+    assert np.array_equal(idx, ridx)
+
+
+# ---------------------------------------------------------------------------
+# attention, small shapes, whole output
+# ---------------------------------------------------------------------------
+
+def run_attn(q, k, v, B, K, order, dt, path="auto", gate=True):
+    out = pisa.pisa_attention(dev(q, dt), dev(k, dt), dev(v, dt), B, K, order, gate=gate, path=path)
+    pisa.pisa_poll_device_status()
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("path", ["stats", "recompute_tc"])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_attention_small_bf16(path, d, B, order):
+    L = 1024
+    q, k, v = pisa_synth.random_qkv(300 + d + B + order, 2, L, d, scale=2.0, dtype="bf16")
+    K = (L // B) // 4
+    got = run_attn(q, k, v, B, K, order, "bf16", path)
+    ref = oracle.pisa_attention(q, k, v, B, K, order)
+    err = rel_l2(got, ref)
+    assert err <= TOL["bf16"], err
+    assert err <= 5e-3, err  # the expected bf16 rounding level; a formulation slip is far above it
+
+
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128)])
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_attention_small_f32(d, B, order):
+    L = 1024
+    q, k, v = pisa_synth.random_qkv(400 + d + B + order, 2, L, d, scale=2.0, dtype="f32")
+    K = (L // B) // 4
+    got = run_attn(q, k, v, B, K, order, "f32")
+    ref = oracle.pisa_attention(q, k, v, B, K, order)
+    assert rel_l2(got, ref) <= TOL["f32"]
+
+
+def test_attention_c1_fp32():
+    w, (q, k, v) = workload("c1")
+    got = run_attn(q, k, v, w.B, w.K, w.order, w.dtype)
+    ref = oracle.pisa_attention(q, k, v, w.B, w.K, w.order)
+    assert rel_l2(got, ref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("path", ["stats", "recompute_tc"])
+@pytest.mark.parametrize("case", ["K0", "Kall", "ragged", "batched", "sharp", "gate"])
+def test_attention_edge_cases(path, case):
+    d, B, L, BH, K, order, scale = 128, 64, 1024, 2, 4, 1, 2.0
+    batch = 1
+    if case == "K0":
+        K = 0
+    elif case == "Kall":
+        K = L // B
+    elif case == "ragged":
+        L = 1152  # 4.5 CTAs of 256 rows: the last CTA has one live 128-row tile
+    elif case == "batched":
+        batch, BH = 2, 6
+    elif case == "sharp":
+        scale = 8.0  # large logits: exercises the running-max correction
+    q, k, v = pisa_synth.random_qkv(500 + len(case), BH, L, d, scale=scale, dtype="bf16")
+    if case == "gate":
+        order = 2
+        k[:, :, 7] *= 30.0  # an outlier channel: w exceeds ln B on many blocks
+        k = pisa_synth.round_bf16(k)
+    qt, kt, vt = (dev(x, "bf16") for x in (q, k, v))
+    if batch > 1:
+        qt, kt, vt = (x.view(batch, BH // batch, L, d) for x in (qt, kt, vt))
+    got = pisa.pisa_attention(qt, kt, vt, B, K, order, path=path).float().cpu().numpy().reshape(BH, L, d)
+    pisa.pisa_poll_device_status()
+    ref = oracle.pisa_attention(q, k, v, B, K, order)
+    assert rel_l2(got, ref) <= TOL["bf16"]
+    if case == "Kall":
+        assert rel_l2(got, oracle.dense_attention(q, k, v)) <= TOL["bf16"]
+
+
+def test_gate_changes_the_result_when_w_is_large():
+    d, B, L = 64, 64, 1024
+    q, k, v = pisa_synth.random_qkv(600, 1, L, d, scale=2.0, dtype="bf16")
+    k[:, :, 3] *= 30.0
+    k = pisa_synth.round_bf16(k)
+    for path in ("stats", "recompute_tc"):
+        on = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=True)
+        off = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=False)
+        assert rel_l2(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True)) <= TOL["bf16"]
+        assert rel_l2(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False)) <= TOL["bf16"]
+        assert rel_l2(on, off) > 1e-2
+
+
+# ---------------------------------------------------------------------------
+# attention, full-size workloads, sampled tiles
+# ---------------------------------------------------------------------------
+
+FULL = [("c2", "recompute_tc", 1, 6), ("c2o2", "recompute_tc", 1, 6), ("c2", "stats", 1, 6),
+        ("c2o2", "stats", 1, 6), ("c3", "recompute_tc", 2, None), ("c4", "recompute_tc", 1, 8),
+        ("c5_L4608_s50", "recompute_tc", 2, None), ("c5_L4608_s95", "recompute_tc", 2, None),
+        ("c5_L16896_s75", "recompute_tc", 2, 8), ("c5_L16896_s90", "recompute_tc", 2, 8)]
+
+
+@pytest.mark.parametrize("name,path,per_head,nheads", FULL)
+def test_attention_full_size_sampled(name, path, per_head, nheads):
+    w, (q, k, v) = workload(name)
+    got = run_attn(q, k, v, w.B, w.K, w.order, w.dtype, path)
+    heads = None if nheads is None else list(np.random.default_rng(7).choice(w.BH, nheads, replace=False))
+    tiles = sample_tiles(w.BH, w.nblk, per_head, seed=11, heads=heads)
+    ref = oracle.pisa_attention(q, k, v, w.B, w.K, w.order, tiles=tiles)
+    err = rel_l2(rows_of(got, tiles, w.B), ref)
+    assert err <= TOL[w.dtype], (name, err)
+
+
+def test_device_status_is_clean():
+    q, k, v = pisa_synth.random_qkv(700, 1, 1024, 128, dtype="bf16")
+    run_attn(q, k, v, 64, 4, 1, "bf16", "recompute_tc")
+    pisa.pisa_poll_device_status()

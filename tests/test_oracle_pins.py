@@ -327,3 +327,11 @@ def test_oracle_rejects_undefined_shapes():
         oracle.pisa_attention(q, k, v, 64, 1)  # L % B != 0
     with pytest.raises(ValueError):
         oracle.pisa_attention(q, k, v, 16, 7)  # K > nblk
+
+
+def test_canonical_centroids_match_numpy_restatement():
+    _, k, _ = pisa_synth.random_qkv(18, 2, 512, 64, dtype="bf16")
+    for B in (16, 64, 128):
+        c = oracle.centroids_f32(k, B)
+        ref = np_tree_sum(k.reshape(2, 512 // B, B, 64), 2) * np.float32(1.0 / B)
+        assert np.array_equal(c.view(np.uint32), ref.view(np.uint32))
