@@ -222,9 +222,13 @@ struct WsLayout {
 
 WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path path) {
     WsLayout w{};
-    // The recompute path needs only the centroids (for the selection).
-    const int stats_order = (path == PISA_PATH_RECOMPUTE_TC) ? 0 : order;
-    w.sl = stats_layout(g, stats_order, dtype);
+    if (path == PISA_PATH_RECOMPUTE_TC) {
+        // The token-form path needs only the centroids (for the selection).
+        w.sl = StatsLayout{};
+        w.sl.total = align_up(sizeof(float) * g.BH * g.nblk * g.d);
+    } else {
+        w.sl = stats_layout(g, order, dtype);
+    }
     size_t o = 0;
     w.stats = o;
     o += w.sl.total;
@@ -373,7 +377,7 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     st.dtype = dtype;
     st.order = (path == PISA_PATH_RECOMPUTE_TC) ? 0 : order;
     st.kbar = (float*)(ws + w.stats + w.sl.kbar);
-    st.vsum = (float*)(ws + w.stats + w.sl.vsum);
+    st.vsum = (path == PISA_PATH_RECOMPUTE_TC) ? nullptr : (float*)(ws + w.stats + w.sl.vsum);
     st.hstat = st.order >= 1 ? (void*)(ws + w.stats + w.sl.hstat) : nullptr;
     st.cov = st.order == 2 ? (void*)(ws + w.stats + w.sl.cov) : nullptr;
     uint32_t* mask = (uint32_t*)(ws + w.mask);
