@@ -83,7 +83,9 @@ def lib():
         L.pisa_centroids.argtypes = [vp, i, i, i, i, i, i, vp, vp]
         L.pisa_fused_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, ctypes.POINTER(_StatsT),
                                            vp, vp]
-        for fn in ("pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
+        L.pisa_attention_noalloc.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp]
+        L.pisa_noalloc_scratch_bytes.restype = sz
+        for fn in ("pisa_attention_noalloc", "pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
                    "pisa_poll_device_status", "pisa_resolve_path"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -253,6 +255,21 @@ def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K:
     _check(lib().pisa_attention_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d, code, B, K,
                                    order, int(bool(gate)), PATHS[path], out.data_ptr(), workspace.data_ptr(),
                                    workspace.numel(), _stream(stream)))
+    return out
+
+
+def pisa_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
+                           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pisa_attention without a workspace argument, for callers that may not
+    allocate device memory: the library's built-in scratch array is used (see
+    include/pisa.h).  ``out`` must be given by such callers (it is created
+    here only for convenience when omitted)."""
+    _need_cuda(q, k, v)
+    batch, heads, L, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().pisa_attention_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d,
+                                        _dtype_code(q.dtype), B, K, order, out.data_ptr(), _stream(stream)))
     return out
 
 

@@ -462,3 +462,72 @@ pisa_status pisa_poll_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of pisa_attention.
+//
+// pisa_attention asks its caller for device workspace (centroids, selection
+// and, on the statistics path, H_j and C_j).  Some callers cannot provide it
+// because they may not allocate device memory at all: a plugin inside a host
+// application that owns the whole device memory pool and forbids cudaMalloc,
+// or a latency-critical loop where cudaMalloc/cudaFree are not allowed
+// (cudaFree synchronises the whole device).  For them this entry point takes
+// its workspace from a fixed array compiled into the library instead.
+//
+// The array lives in device memory of every GPU that loads this library, for
+// as long as the process runs.  Its name is only a host-side stand-in, so its
+// device address is looked up once per device (cudaGetSymbolAddress with that
+// device current) and cached.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = (size_t)32 << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Set-up of the current device: resolve the scratch array's device address.
+pisa_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "pisa_attention_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(PISA_ERR_UNSUPPORTED, "pisa_attention_noalloc: device id %d >= 64", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "pisa_attention_noalloc: cudaGetSymbolAddress");
+        if (!p) return fail(PISA_ERR_CUDA, "pisa_attention_noalloc: null scratch address");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return PISA_OK;
+}
+
+}  // namespace
+
+extern "C" pisa_status pisa_attention_noalloc(const void* q, const void* k, const void* v, int batch, int heads,
+                                              int L, int d, pisa_dtype dtype, int B, int K, int order, void* out,
+                                              void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
+    const size_t need = pisa_workspace_bytes(batch, heads, L, d, B, K, order, dtype);
+    if (need == 0) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_noalloc: no path for these arguments");
+    if (need > kNoallocScratchBytes)
+        return fail(PISA_ERR_INVALID_ARG,
+                    "pisa_attention_noalloc: this call needs %zu bytes of scratch but the library's built-in "
+                    "scratch holds %zu bytes; use pisa_attention with a caller-provided workspace",
+                    need, kNoallocScratchBytes);
+    void* scratch = nullptr;
+    r = noalloc_scratch(&scratch);
+    if (r != PISA_OK) return r;
+    return pisa_attention_ex(q, k, v, batch, heads, L, d, dtype, B, K, order, 1, PISA_PATH_AUTO, out, scratch,
+                             kNoallocScratchBytes, stream);
+}
+
+extern "C" size_t pisa_noalloc_scratch_bytes(void) { return kNoallocScratchBytes; }

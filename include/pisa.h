@@ -165,6 +165,30 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
                               pisa_path path, void* out, void* workspace, size_t ws_bytes,
                               void* stream);
 
+/* Allocation-free pisa_attention (the paper has no counterpart: this is an
+ * interface for callers that may not allocate device memory, such as a plugin
+ * whose host application owns the whole device memory pool, or a loop where
+ * cudaMalloc/cudaFree, which can synchronise the device, are not allowed).
+ * Same arguments and result as pisa_attention (AUTO path, gate on), minus the
+ * workspace: the scratch comes from one array of pisa_noalloc_scratch_bytes()
+ * (32 MiB) compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  The caller still passes q, k, v and out.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - A call whose workspace (pisa_workspace_bytes) exceeds the scratch size is
+ *     rejected with PISA_ERR_INVALID_ARG before any work is enqueued.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Every kernel overwrites the parts it reads, so nothing has to
+ *     start at zero, but calls that overlap on the GPU (different streams, no
+ *     ordering between them) race on the scratch and give wrong results. */
+pisa_status pisa_attention_noalloc(const void* q, const void* k, const void* v, int batch, int heads, int L,
+                                   int d, pisa_dtype dtype, int B, int K, int order, void* out, void* stream);
+
+/* Size in bytes of the scratch array pisa_attention_noalloc uses. */
+size_t pisa_noalloc_scratch_bytes(void);
+
 /* The path AUTO resolves to for these arguments (or -1 if none can run). */
 int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order,
                       pisa_dtype dtype);
