@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="c3")
@@ -94,7 +94,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -349,6 +349,31 @@ def main():
     per_kernel["centroids_frac_hbm"] = per_kernel["centroids_gbs"] / hbm
     per_kernel["select_frac_hbm"] = per_kernel["select_gbs"] / hbm
 
+    # The statistics kernel (block statistics k-bar, v-sum, H_j and, for order 2,
+    # C_j) is not on the token-form path; it is timed here on its own against
+    # the HBM roofline of its compulsory traffic.
+    stats_rec = None
+    if path != "stats":
+        sorder = max(order, 1)
+        sbuf = torch.empty(pisa.pisa_stats_bytes(1, BH, L, d, B, sorder, tdt), dtype=torch.uint8, device="cuda")
+        for _ in range(2):
+            pisa.pisa_stats(k, v, B, sorder, buf=sbuf)
+        sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        sa.record(stream)
+        for _ in range(reps):
+            pisa.pisa_stats(k, v, B, sorder, buf=sbuf)
+        sb.record(stream)
+        torch.cuda.synchronize()
+        s_ms = sa.elapsed_time(sb) / reps
+        es = q.element_size()
+        s_bytes = 2 * BH * L * d * es + 2 * BH * nblk * d * 4 + BH * nblk * d * d * es * (2 if sorder == 2 else 1)
+        kname = "stats_tc_kernel" if tdt == torch.bfloat16 else "stats_simt_kernel"
+        stats_rec = {"kernel": f"{kname}<{d},{B},{sorder}>", "order": sorder, "ms": s_ms,
+                     "algorithmic_bytes": s_bytes, "gbs": s_bytes / (s_ms * 1e-3) / 1e9,
+                     "frac_hbm": s_bytes / (s_ms * 1e-3) / 1e9 / hbm}
+        del sbuf
+
     # end to end through the public call with host buffers: pinned H2D, pisa_attention, D2H
     e2e = None
     if not args.no_e2e:
@@ -401,6 +426,7 @@ def main():
                            q.numel() * q.element_size() / 2 ** 20)},
             "roofline": roof,
             "per_kernel": per_kernel,
+            "stats_kernel": stats_rec,
             "cpu_baseline": cpu,
             "clocks": clk,
             "e2e": e2e,

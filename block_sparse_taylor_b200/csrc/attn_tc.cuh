@@ -61,11 +61,11 @@ struct TcCfg {
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
-template <int D, int BS>
+template <int D, int BS, int ORDER>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ mask, bf16* __restrict__ out,
-                   int L, int nblk, int words, int order, int gate, float ln_b, unsigned* status) {
+                   int L, int nblk, int words, int gate, float ln_b, unsigned* status) {
     using C = TcCfg<D>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, N = 128 keys
@@ -158,23 +158,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
+            // descriptors of the operand bases; a K-step adds its byte offset >> 4
+            // to the start-address field (addresses stay below 2^18)
+            const uint64_t qdesc0 = tc::sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+            const uint64_t kdesc0 = tc::sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+            const uint64_t vdesc0 = tc::sdesc_sw128(sbase + C::V_OFF, C::BOX_BYTES, 1024);
+            constexpr uint64_t kTileStep = C::TILE_BYTES >> 4;  // one tile further in shared memory
             auto issue_s = [&](int h, int st) {
-                const uint32_t qa = sbase + C::Q_OFF + h * C::TILE_BYTES;
-                const uint32_t ka = sbase + C::K_OFF + st * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::BOX_BYTES + (kk % 4) * 32;
-                    tc::mma_ss(tmem + (uint32_t)(h * 128), tc::sdesc_sw128(qa + off, 16, 1024),
-                               tc::sdesc_sw128(ka + off, 16, 1024), IDESC_S, kk > 0);
+                    const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+                    tc::mma_ss(tmem + (uint32_t)(h * 128), qdesc0 + h * kTileStep + off, kdesc0 + st * kTileStep + off,
+                               IDESC_S, kk > 0);
                 }
             };
             auto issue_pv = [&](int h, int st, bool first) {
-                const uint32_t va = sbase + C::V_OFF + st * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < C::NK / 16; ++kk) {
                     tc::mma_ts(tmem + C::O_COL0 + h * D, tmem + (uint32_t)(h * 128) + kk * 8,
-                               tc::sdesc_sw128(va + kk * 16 * 128, C::BOX_BYTES, 1024), IDESC_O,
-                               (first && kk == 0) ? 0u : 1u);
+                               vdesc0 + st * kTileStep + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O, (first && kk == 0) ? 0u : 1u);
                 }
             };
             bool ok = tc::mbar_wait(bar(B_QFULL), 0, aborted, status, kWaitLimitCycles);
@@ -233,42 +235,64 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float inv_bs = 1.0f / (float)BS;
         float m_run = -INFINITY;                  // running max (log2 units)
         float dsum = 0.f;                         // denominator (scaled by 2^-m_run)
+        int mword_idx = -1;                       // cached selection-mask word
+        uint32_t mword = 0u;
 
         for (int jt = 0; jt < NT; ++jt) {
             if (!tc::mbar_wait_warp(bar(B_SFULL + h), jt & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
             bool sel[BPT];
             float cand[BPT], sbar[BPT], l2[BPT];
-#pragma unroll
-            for (int b = 0; b < BPT; ++b) {
-                const int j = jt * BPT + b;
-                sel[b] = (__ldg(mrow + (j >> 5)) >> (j & 31)) & 1u;
+            if (((jt * BPT) >> 5) != mword_idx) {
+                mword_idx = (jt * BPT) >> 5;
+                mword = __ldg(mrow + mword_idx);
             }
-            // pass 1: per-block statistics of the logits
 #pragma unroll
             for (int b = 0; b < BPT; ++b) {
-                float mx = -INFINITY, sm = 0.f, sq = 0.f;
+                const int j = jt * BPT + b;  // the BPT blocks of a tile share one mask word
+                sel[b] = (mword >> (j & 31)) & 1u;
+            }
+            // pass 1: per-block statistics of the logits (exact: max; Taylor:
+            // sum, and the sum of squares for order 2), four partial
+            // accumulators each so that the reductions are not one long chain
 #pragma unroll
-                for (int c = 0; c < CPB; ++c) {
-                    uint32_t raw[32];
-                    tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = __uint_as_float(raw[e]);
-                        mx = fmaxf(mx, x);
-                        sm += x;
-                        sq = fmaf(x, x, sq);
-                    }
-                }
+            for (int b = 0; b < BPT; ++b) {
                 if (sel[b]) {
-                    cand[b] = mx * LOG2E;
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < CPB; c += 2) {
+                        uint32_t r0[32], r1[32];
+                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
+                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(r0[e]));
+                            m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(r1[e]));
+                        }
+                    }
+                    cand[b] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
                     sbar[b] = 0.f;
                     l2[b] = 0.f;
                 } else {
-                    const float sb = sm * inv_bs;
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f}, q4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int c = 0; c < CPB; c += 2) {
+                        uint32_t r0[32], r1[32];
+                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
+                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float x0 = __uint_as_float(r0[e]), x1 = __uint_as_float(r1[e]);
+                            s4[e & 3] += x0 + x1;
+                            if (ORDER == 2) q4[e & 3] = fmaf(x0, x0, fmaf(x1, x1, q4[e & 3]));
+                        }
+                    }
+                    const float sb = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs;
                     float w = 0.f;
-                    if (order == 2) {
+                    if (ORDER == 2) {
+                        const float sq = (q4[0] + q4[1]) + (q4[2] + q4[3]);
                         w = 0.5f * fmaf(-sb, sb, sq * inv_bs);
                         if (gate && w > ln_b) w = 0.f;
                     }
@@ -304,35 +328,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int b = 0; b < BPT; ++b) {
                 if (sel[b]) {
+                    float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < CPB; ++c) {
-                        uint32_t raw[32], pk[16];
-                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
+                    for (int c = 0; c < CPB; c += 2) {
+                        uint32_t r0[32], r1[32], p0[16], p1[16];
+                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
+                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float p0 = tc::ex2(fmaf(__uint_as_float(raw[2 * e]), LOG2E, -m_run));
-                            const float p1 = tc::ex2(fmaf(__uint_as_float(raw[2 * e + 1]), LOG2E, -m_run));
-                            dsum += p0 + p1;
-                            pk[e] = tc::pack_bf16x2(p0, p1);
+                            const float a0 = tc::ex2(fmaf(__uint_as_float(r0[2 * e]), LOG2E, -m_run));
+                            const float a1 = tc::ex2(fmaf(__uint_as_float(r0[2 * e + 1]), LOG2E, -m_run));
+                            const float b0 = tc::ex2(fmaf(__uint_as_float(r1[2 * e]), LOG2E, -m_run));
+                            const float b1 = tc::ex2_fma(fmaf(__uint_as_float(r1[2 * e + 1]), LOG2E, -m_run));
+                            d4[e & 3] += (a0 + a1) + (b0 + b1);
+                            p0[e] = tc::pack_bf16x2(a0, a1);
+                            p1[e] = tc::pack_bf16x2(b0, b1);
                         }
-                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, p0);
+                        tc::tmem_st16(s_addr + (b * CPB + c + 1) * 16, p1);
                     }
+                    dsum += (d4[0] + d4[1]) + (d4[2] + d4[3]);
                 } else {
                     const float alpha = tc::ex2(l2[b] - m_run);
                     dsum = fmaf((float)BS, alpha, dsum);
-                    if (order >= 1) {
+                    if (ORDER >= 1) {
                         const float c0 = alpha * (1.0f - sbar[b]);
 #pragma unroll
-                        for (int c = 0; c < CPB; ++c) {
-                            uint32_t raw[32], pk[16];
-                            tc::tmem_ld32(s_addr + (b * CPB + c) * 32, raw);
+                        for (int c = 0; c < CPB; c += 2) {
+                            uint32_t r0[32], r1[32], p0[16], p1[16];
+                            tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
+                            tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
                             tc::tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                pk[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(raw[2 * e]), c0),
-                                                        fmaf(alpha, __uint_as_float(raw[2 * e + 1]), c0));
-                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                            for (int e = 0; e < 16; ++e) {
+                                p0[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(r0[2 * e]), c0),
+                                                        fmaf(alpha, __uint_as_float(r0[2 * e + 1]), c0));
+                                p1[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(r1[2 * e]), c0),
+                                                        fmaf(alpha, __uint_as_float(r1[2 * e + 1]), c0));
+                            }
+                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, p0);
+                            tc::tmem_st16(s_addr + (b * CPB + c + 1) * 16, p1);
                         }
                     } else {
                         uint32_t pk[16];
@@ -422,21 +458,29 @@ inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, cons
     const float ln_b = logf((float)B);
     dim3 grid((unsigned)((L + 255) / 256), (unsigned)BH);
     cudaError_t e = cudaSuccess;
-#define PISA_TC_LAUNCH(DD, BB)                                                                                 \
-    if (d == DD && B == BB) {                                                                                  \
-        auto kern = attn_tc_kernel<DD, BB>;                                                                    \
+#define PISA_TC_LAUNCH(DD, BB, OO)                                                                             \
+    if (d == DD && B == BB && order == OO) {                                                                   \
+        auto kern = attn_tc_kernel<DD, BB, OO>;                                                                \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcCfg<DD>::SMEM);     \
         if (e == cudaSuccess) {                                                                                \
             kern<<<grid, kTcThreads, TcCfg<DD>::SMEM, s>>>(maps[0], maps[1], maps[2], mask, (bf16*)out, L, nblk, \
-                                                           words, order, gate, ln_b, status);                 \
+                                                           words, gate, ln_b, status);                         \
             e = cudaGetLastError();                                                                            \
         }                                                                                                      \
     } else
-    PISA_TC_LAUNCH(64, 64)
-    PISA_TC_LAUNCH(64, 128)
-    PISA_TC_LAUNCH(128, 64)
-    PISA_TC_LAUNCH(128, 128) {
-        *err = "no tensor-core kernel for this d/B";
+    PISA_TC_LAUNCH(64, 64, 0)
+    PISA_TC_LAUNCH(64, 64, 1)
+    PISA_TC_LAUNCH(64, 64, 2)
+    PISA_TC_LAUNCH(64, 128, 0)
+    PISA_TC_LAUNCH(64, 128, 1)
+    PISA_TC_LAUNCH(64, 128, 2)
+    PISA_TC_LAUNCH(128, 64, 0)
+    PISA_TC_LAUNCH(128, 64, 1)
+    PISA_TC_LAUNCH(128, 64, 2)
+    PISA_TC_LAUNCH(128, 128, 0)
+    PISA_TC_LAUNCH(128, 128, 1)
+    PISA_TC_LAUNCH(128, 128, 2) {
+        *err = "no tensor-core kernel for this d/B/order";
         return PISA_ERR_UNSUPPORTED;
     }
 #undef PISA_TC_LAUNCH

@@ -17,6 +17,7 @@
 #include "select.cuh"
 #include "attn_stats.cuh"
 #include "attn_tc.cuh"
+#include "stats_tc.cuh"
 
 using pisa::bf16;
 
@@ -157,13 +158,24 @@ pisa_status run_centroids(const void* k, float* kbar, const Dims& g, pisa_dtype 
     return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const size_t smem = sizeof(T) * BS * D;
+        auto kern = pisa::centroid_kernel<T, D, BS>;
+        pisa_status r = set_smem(kern, smem);
+        if (r != PISA_OK) return r;
         dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
-        pisa::centroid_kernel<T, D, BS><<<grid, D, 0, s>>>((const T*)k, kbar, (int)g.L, (int)g.nblk);
+        kern<<<grid, 128, smem, s>>>((const T*)k, kbar, (int)g.L, (int)g.nblk);
         return launch_check("centroid_kernel");
     });
 }
 
 pisa_status run_stats(const void* k, const void* v, const pisa_stats_t* st, const Dims& g, cudaStream_t s) {
+    if (st->dtype == PISA_BF16 && st->order >= 1) {
+        // bf16: the Gram products H_j and C_j on the tensor cores
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        return pisa::run_stats_tc(k, v, st->kbar, st->vsum, st->hstat, st->cov, g.BH, (int)g.L, (int)g.d, (int)g.B,
+                                  (int)g.nblk, st->order, status, s, &g_last_error);
+    }
     return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
@@ -183,13 +195,14 @@ pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dty
     return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
-        const int P = next_pow2((int)g.nblk < 2 ? 2 : (int)g.nblk);
-        const size_t smem = sizeof(unsigned long long) * P + sizeof(float) * D + sizeof(uint32_t) * 2 * g.words;
+        const int QT = pisa::select_tiles_per_cta<D>((int)g.nblk);
+        const size_t smem = pisa::select_smem_bytes<D>(QT, (int)g.nblk);
         auto kern = pisa::select_kernel<T, D, BS>;
         pisa_status r = set_smem(kern, smem);
         if (r != PISA_OK) return r;
-        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
-        kern<<<grid, 256, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K, (int)g.words, P, idx, mask);
+        dim3 grid((unsigned)((g.nblk + QT - 1) / QT), (unsigned)g.BH);
+        kern<<<grid, pisa::SelectCfg<D>::THREADS, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K,
+                                                              (int)g.words, QT, idx, mask);
         return launch_check("select_kernel");
     });
 }

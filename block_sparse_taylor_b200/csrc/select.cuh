@@ -8,7 +8,9 @@
 //
 // Every fp32 operation follows the canonical order of the C ABI comment:
 // tile means by the pairwise tree over the B rows, scores by the pairwise
-// tree over the d products, each product and sum rounded on its own.
+// tree over the d products, each product and sum rounded on its own.  The
+// score tree runs on packed fp32x2 operations (two independent IEEE
+// round-to-nearest operations each), which leaves every rounding unchanged.
 #pragma once
 
 #include "common.cuh"
@@ -23,99 +25,161 @@ __device__ __forceinline__ uint32_t ordered_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// One CTA per (query tile, bh); 256 threads.  P = power of two >= nblk.
-template <typename T, int D, int BS>
-__global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
-                                                     int L, int nblk, int K, int words, int P,
-                                                     int32_t* __restrict__ idx, uint32_t* __restrict__ mask) {
-    extern __shared__ __align__(16) unsigned long long sm_sel[];
-    unsigned long long* keys = sm_sel;                      // [P]
-    float* qbar = (float*)(keys + P);                       // [D]
-    uint32_t* mw = (uint32_t*)(qbar + D);                   // [words]
-    uint32_t* off = mw + words;                             // [words]
-    const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const int warp = tid / 32, lane = tid % 32;
+__device__ __forceinline__ unsigned long long f2_pack(float2 v) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long r) {
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 
-    // 1. canonical tile mean, thread c owns column c
-    if (tid < D) {
-        const T* src = q + ((size_t)bh * L + (size_t)i * BS) * D + tid;
+// Canonical score: p_c = q_c * k_c rounded, then the pairwise tree
+// a[i] = a[i] + a[i + h], h = D/2 .. 1.  Lanes of packed pairs hold
+// (a[2m], a[2m+1]); every level with h >= 2 pairs up element-wise.
+template <int D>
+__device__ __forceinline__ float canonical_dot(const unsigned long long (&q2)[D / 2], const float* __restrict__ k) {
+    unsigned long long a[D / 4];
+    const float4* k4 = reinterpret_cast<const float4*>(k);
+#pragma unroll
+    for (int m = 0; m < D / 4; m += 2) {
+        // products of columns 2m .. 2m+3 and of D/2 + 2m .. D/2 + 2m + 3
+        const float4 lo = k4[m / 2], hi = k4[(D / 2 + 2 * m) / 4];
+        const unsigned long long plo0 = f2_mul(q2[m], f2_pack(make_float2(lo.x, lo.y)));
+        const unsigned long long plo1 = f2_mul(q2[m + 1], f2_pack(make_float2(lo.z, lo.w)));
+        const unsigned long long phi0 = f2_mul(q2[D / 4 + m], f2_pack(make_float2(hi.x, hi.y)));
+        const unsigned long long phi1 = f2_mul(q2[D / 4 + m + 1], f2_pack(make_float2(hi.z, hi.w)));
+        a[m] = f2_add(plo0, phi0);
+        a[m + 1] = f2_add(plo1, phi1);
+    }
+#pragma unroll
+    for (int h = D / 8; h >= 1; h >>= 1) {
+#pragma unroll
+        for (int m = 0; m < h; ++m) a[m] = f2_add(a[m], a[m + h]);
+    }
+    const float2 last = f2_unpack(a[0]);
+    return __fadd_rn(last.x, last.y);
+}
+
+template <int D>
+struct SelectCfg {
+    static constexpr int THREADS = 256;
+    static constexpr int JC = 64;  // centroids staged per chunk
+};
+
+// Query tiles per CTA (one per lane of a warp, at most 32) so that the score
+// table fits next to the staged tile means and centroids.
+template <int D>
+inline int select_tiles_per_cta(int nblk) {
+    const long budget = 200 * 1024 - (long)sizeof(float) * (32 * D + SelectCfg<D>::JC * D);
+    long qt = budget / ((long)sizeof(float) * (nblk + 1));
+    return (int)(qt > 32 ? 32 : (qt < 1 ? 1 : qt));
+}
+
+template <int D>
+inline size_t select_smem_bytes(int QT, int nblk) {
+    return sizeof(float) * ((size_t)QT * D + (size_t)SelectCfg<D>::JC * D + (size_t)QT * (nblk + 1));
+}
+
+// One CTA per (group of QT query tiles, bh), 8 warps.
+//   1. canonical tile means (thread per (tile, column));
+//   2. scores: lane t of every warp holds tile t's mean in registers, the
+//      centroids are staged JC at a time and read as broadcasts; warp w takes
+//      the blocks jj = w, w+8, ... of each chunk;
+//   3. top-K per tile (warp per tile): binary search for the K-th largest
+//      ordered score, then ties broken by ascending block index with ballots;
+//      the ballots are the mask words and give the ascending index list.
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+                                                        int L, int nblk, int K, int words, int QT,
+                                                        int32_t* __restrict__ idx, uint32_t* __restrict__ mask) {
+    using C = SelectCfg<D>;
+    extern __shared__ __align__(16) float sm_sel[];
+    float* qbar = sm_sel;                 // [QT][D]
+    float* kst = qbar + QT * D;           // [JC][D]
+    float* sc = kst + C::JC * D;          // [QT][nblk + 1]
+    const int SS = nblk + 1;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, bh = blockIdx.y;
+    const int i0 = blockIdx.x * QT;
+    const int nq = min(QT, nblk - i0);
+
+    // 1. tile means
+    for (int e = tid; e < nq * D; e += C::THREADS) {
+        const int t = e / D, c = e % D;
+        const T* src = q + ((size_t)bh * L + (size_t)(i0 + t) * BS) * D + c;
         float a[BS];
 #pragma unroll
         for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
-        qbar[tid] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-    }
-    for (int e = tid; e < words; e += 256) mw[e] = 0u;
-    __syncthreads();
-
-    // 2. scores, one warp per block j; lane holds columns lane + 32*w
-    constexpr int W = D / 32;
-    float qv[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) qv[w] = qbar[lane + 32 * w];
-    const float* kb = kbar + (size_t)bh * nblk * D;
-    for (int j = warp; j < P; j += 8) {
-        if (j >= nblk) {
-            if (lane == 0) keys[j] = 0ull;
-            continue;
-        }
-        float p[W];
-#pragma unroll
-        for (int w = 0; w < W; ++w) p[w] = __fmul_rn(qv[w], kb[(size_t)j * D + lane + 32 * w]);
-        // tree levels h = D/2 .. 32 inside the lane, h = 16 .. 1 across lanes
-#pragma unroll
-        for (int h = W / 2; h >= 1; h >>= 1) {
-#pragma unroll
-            for (int w = 0; w < h; ++w) p[w] = __fadd_rn(p[w], p[w + h]);
-        }
-        float s = p[0];
-#pragma unroll
-        for (int h = 16; h >= 1; h >>= 1) s = __fadd_rn(s, __shfl_down_sync(0xffffffffu, s, h));
-        if (lane == 0) keys[j] = ((unsigned long long)ordered_key(s) << 32) | (0xffffffffu - (uint32_t)j);
+        qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
     }
     __syncthreads();
 
-    // 3. bitonic sort, descending
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = tid; t < P / 2; t += 256) {
-                const int lo = 2 * stride * (t / stride) + (t % stride);
-                const int hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const unsigned long long a = keys[lo], b = keys[hi];
-                if ((a < b) == desc) {
-                    keys[lo] = b;
-                    keys[hi] = a;
-                }
+    // 2. scores
+    const bool live = lane < nq;
+    unsigned long long q2[D / 2];
+    {
+        const float2* qs = reinterpret_cast<const float2*>(qbar + (live ? lane : 0) * D);
+#pragma unroll
+        for (int m = 0; m < D / 2; ++m) q2[m] = f2_pack(qs[m]);
+    }
+    const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nblk * D);
+    for (int j0 = 0; j0 < nblk; j0 += C::JC) {
+        const int nj = min(C::JC, nblk - j0);
+        float4* kst4 = reinterpret_cast<float4*>(kst);
+        for (int e = tid; e < nj * D / 4; e += C::THREADS) kst4[e] = kb4[(size_t)j0 * D / 4 + e];
+        __syncthreads();
+        for (int jj = warp; jj < nj; jj += 8) {
+            const float s = canonical_dot<D>(q2, kst + jj * D);
+            if (live) sc[lane * SS + j0 + jj] = s;
+        }
+        __syncthreads();
+    }
+
+    // 3. top-K, one warp per tile
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int t = warp; t < nq; t += 8) {
+        const float* st = sc + t * SS;
+        const size_t row = (size_t)bh * nblk + i0 + t;
+        uint32_t T = 0u;  // K-th largest ordered score (unused when K is 0 or nblk)
+        int need = 0;     // how many of the ties at T to take, lowest index first
+        if (K > 0 && K < nblk) {
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t cand = T | (1u << bit);
+                int cnt = 0;
+                for (int j = lane; j < nblk; j += 32) cnt += ordered_key(st[j]) >= cand;
+                cnt = __reduce_add_sync(0xffffffffu, cnt);
+                if (cnt >= K) T = cand;
             }
-            __syncthreads();
+            int gt = 0;
+            for (int j = lane; j < nblk; j += 32) gt += ordered_key(st[j]) > T;
+            need = K - __reduce_add_sync(0xffffffffu, gt);
         }
-    }
-
-    // 4. mask of the first K, then the ascending index list
-    for (int t = tid; t < K; t += 256) {
-        const uint32_t j = 0xffffffffu - (uint32_t)(keys[t] & 0xffffffffull);
-        atomicOr(&mw[j >> 5], 1u << (j & 31));
-    }
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t acc = 0;
+        int off = 0, eq_seen = 0;
         for (int w = 0; w < words; ++w) {
-            off[w] = acc;
-            acc += __popc(mw[w]);
-        }
-    }
-    __syncthreads();
-    const size_t row = (size_t)bh * nblk + i;
-    for (int w = tid; w < words; w += 256) {
-        const uint32_t bits = mw[w];
-        if (mask) mask[row * words + w] = bits;
-        if (idx) {
-            uint32_t b = bits, o = off[w];
-            while (b) {
-                const int t = __ffs(b) - 1;
-                idx[row * K + o++] = w * 32 + t;
-                b &= b - 1;
-            }
+            // every lane takes part in every ballot; lanes past nblk vote "no"
+            const int j = w * 32 + lane;
+            const bool in = j < nblk;
+            const uint32_t o = in ? ordered_key(st[j]) : 0u;
+            const unsigned eq = __ballot_sync(0xffffffffu, in && o == T);
+            const int rank = eq_seen + __popc(eq & lt_mask);
+            eq_seen += __popc(eq);
+            const bool sel = in && (K == nblk || (K > 0 && (o > T || (o == T && rank < need))));
+            const unsigned bits = __ballot_sync(0xffffffffu, sel);
+            if (mask && lane == 0) mask[row * words + w] = bits;
+            if (idx && sel) idx[row * K + off + __popc(bits & lt_mask)] = j;
+            off += __popc(bits);
         }
     }
 }

@@ -12,20 +12,29 @@
 
 namespace pisa {
 
-// Centroid of every key block in the canonical fp32 order: thread c owns
-// column c, holds the B values in registers and reduces them with the
-// pairwise tree; the mean is the tree sum times 1/B (exact for B = 2^k).
-// grid (nblk, BH), block D threads.
+// Centroid of every key block in the canonical fp32 order.  One CTA per
+// (block, bh): the B x D tile is staged in shared memory with 16-byte loads,
+// then the thread of column c reduces its B values with the pairwise tree; the
+// mean is the tree sum times 1/B (exact for B = 2^k).  grid (nblk, BH), 128
+// threads, BS * D * sizeof(T) bytes of dynamic shared memory.
 template <typename T, int D, int BS>
-__global__ void __launch_bounds__(D) centroid_kernel(const T* __restrict__ k, float* __restrict__ kbar,
-                                                     int L, int nblk) {
-    const int j = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-    const T* src = k + ((size_t)bh * L + (size_t)j * BS) * D + c;
-    float a[BS];
+__global__ void __launch_bounds__(128) centroid_kernel(const T* __restrict__ k, float* __restrict__ kbar,
+                                                       int L, int nblk) {
+    extern __shared__ __align__(16) uint8_t sm_cent[];
+    T* tile = reinterpret_cast<T*>(sm_cent);
+    const int j = blockIdx.x, bh = blockIdx.y;
+    const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * L + (size_t)j * BS) * D);
+    uint4* dst = reinterpret_cast<uint4*>(tile);
+    constexpr int NV = BS * D * (int)sizeof(T) / 16;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < NV; e += 128) dst[e] = __ldg(src + e);
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += 128) {
+        float a[BS];
 #pragma unroll
-    for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
-    const float s = tree_sum<BS>(a);
-    kbar[((size_t)bh * nblk + j) * D + c] = __fmul_rn(s, 1.0f / (float)BS);
+        for (int n = 0; n < BS; ++n) a[n] = to_f(tile[n * D + c]);
+        kbar[((size_t)bh * nblk + j) * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+    }
 }
 
 // Full statistics on CUDA cores.  One CTA per (block, bh), 256 threads.

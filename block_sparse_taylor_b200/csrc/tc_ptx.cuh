@@ -185,6 +185,19 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for x in [-125, 64]: x = n + f with n = round(x)
+// (the 1.5 * 2^23 addition rounds to nearest and leaves n in the low mantissa
+// bits), 2^f for f in [-1/2, 1/2] by a cubic fitted to minimise the relative
+// error (max 7.5e-5, well below bf16's 2^-9), then n added to the exponent.
+// Used for part of the exponentials so that the MUFU and FMA pipes share them.
+__device__ __forceinline__ float ex2_fma(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    const float p = fmaf(fmaf(fmaf(0.05517139f, f, 0.24261111f), f, 0.69326103f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);

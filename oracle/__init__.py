@@ -34,11 +34,13 @@ def lib():
                                     ctypes.c_void_p, ctypes.c_int]
         L.oracle_pisa_attention.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
+        L.oracle_pisa_hybrid.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_bruteforce.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                              ctypes.c_int, f64p, ctypes.c_int]
         L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
-        for fn in ("oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
+        for fn in ("oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
                    "oracle_pisa_bruteforce", "oracle_dense_attention"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -104,6 +106,33 @@ def select(q, k, B, K, nthreads=None, want_scores=False):
                              nthreads or default_threads())
     _check(rc, "select")
     return idx, mask, scores
+
+
+def _attention(fn, q, k, v, B, K, order, gate, tiles, nthreads, want_lse):
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    BH, L, d = q.shape
+    nblk = L // B
+    full = tiles is None
+    if full:
+        tl = np.array([(bh, i) for bh in range(BH) for i in range(nblk)], dtype=np.int64)
+    else:
+        tl = np.ascontiguousarray(np.asarray(tiles, dtype=np.int64).reshape(-1, 2))
+    out = np.zeros((tl.shape[0], B, d))
+    lse = np.zeros((tl.shape[0], B)) if want_lse else None
+    rc = fn(q, k, v, BH, L, d, B, K, int(order), int(bool(gate)), _ptr(tl), tl.shape[0], _ptr(out), _ptr(lse),
+            nthreads or default_threads())
+    _check(rc, "attention")
+    if full:
+        out = out.reshape(BH, L, d)
+        lse = lse.reshape(BH, L) if want_lse else None
+    return (out, lse) if want_lse else out
+
+
+def pisa_hybrid(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, want_lse=False):
+    """PISA hybrid output: as pisa_attention but the first-order term uses the
+    global H-bar = (B/L) sum_j H_j of each (batch, head) for every unselected
+    block (same return convention as pisa_attention)."""
+    return _attention(lib().oracle_pisa_hybrid, q, k, v, B, K, order, gate, tiles, nthreads, want_lse)
 
 
 def pisa_attention(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, want_lse=False):

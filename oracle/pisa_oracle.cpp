@@ -171,10 +171,13 @@ void select_one(const float* q, const float* k, long L, long d, long B, long K,
 //   D = sum_S sum_n e^{x} + sum_U B e^{l}
 //   N = sum_S sum_n e^{x} v_n + sum_U e^{l} (vsum_j + [order>=1] H_j q)
 //   o = N / D                   (evaluated with the common shift m = max logit)
+// With Hbar given, H_j is replaced by the global statistic H-bar (the PISA
+// hybrid: first-order term (sum_U e^{l}) H-bar q; [blog1] "Sparse Linear
+// Attention", [pisa] section 3.3 and Appendix C, R_t = sum_U alpha (H_j - H-bar)).
 void row_stats_form(const float* qrow, const float* k, const float* v, long d, long B,
                     long nblk, const uint8_t* sel, int order, int gate,
                     const double* kbar, const double* vsum, const double* H, const double* C,
-                    double* out, double* lse, std::vector<double>& xs,
+                    const double* Hbar, double* out, double* lse, std::vector<double>& xs,
                     std::vector<double>& ls, std::vector<double>& num) {
     std::vector<double> q(d);
     for (long c = 0; c < d; ++c) q[c] = (double)qrow[c];
@@ -223,7 +226,8 @@ void row_stats_form(const float* qrow, const float* k, const float* v, long d, l
             const double* vs = vsum + j * d;
             for (long c = 0; c < d; ++c) num[c] += a * vs[c];
             if (order >= 1) {
-                const double* Hj = H + j * d * d;
+                // per-block H_j, or the global H-bar of the PISA hybrid
+                const double* Hj = Hbar ? Hbar : H + j * d * d;
                 for (long r = 0; r < d; ++r) {
                     double t = 0.0;
                     for (long c = 0; c < d; ++c) t += Hj[r * d + c] * q[c];
@@ -372,9 +376,10 @@ int oracle_select(const float* q, const float* k, long BH, long L, long d, long 
 // tiles[2*r+1] = tile index i; out receives [ntiles, B, d] fp64 rows and, when
 // lse is not null, lse receives [ntiles, B] values log(D_t) (unshifted).
 // The selection (canonical fp32) is recomputed here from q and k.
-int oracle_pisa_attention(const float* q, const float* k, const float* v, long BH, long L,
-                          long d, long B, long K, int order, int gate, const int64_t* tiles,
-                          long ntiles, double* out, double* lse, int nthreads) {
+static int pisa_attention_impl(const float* q, const float* k, const float* v, long BH, long L,
+                               long d, long B, long K, int order, int gate, int global_h,
+                               const int64_t* tiles, long ntiles, double* out, double* lse,
+                               int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     const long nblk = L / B;
     if (K < 0 || K > nblk) return -1;
@@ -389,7 +394,7 @@ int oracle_pisa_attention(const float* q, const float* k, const float* v, long B
     for (long bh = 0; bh < BH; ++bh)
         if (need[bh]) bhs.push_back(bh);
     const long words = (nblk + 31) / 32;
-    std::vector<std::vector<double>> kbar(BH), vsum(BH), H(BH), C(BH);
+    std::vector<std::vector<double>> kbar(BH), vsum(BH), H(BH), C(BH), Hbar(BH);
     std::vector<std::vector<uint32_t>> mask(BH);
     parallel_for((long)bhs.size(), nthreads, [&](long r) {
         const long bh = bhs[r];
@@ -401,6 +406,13 @@ int oracle_pisa_attention(const float* q, const float* k, const float* v, long B
                         order >= 1 ? H[bh].data() : nullptr, order == 2 ? C[bh].data() : nullptr);
         mask[bh].assign(nblk * words, 0u);
         select_one(q + bh * L * d, k + bh * L * d, L, d, B, K, nullptr, mask[bh].data(), nullptr);
+        if (global_h && order >= 1) {
+            // H-bar = (B / L) sum over all blocks of H_j  ([blog1] "Sparse Linear Attention")
+            Hbar[bh].assign(d * d, 0.0);
+            for (long j = 0; j < nblk; ++j)
+                for (long e = 0; e < d * d; ++e) Hbar[bh][e] += H[bh][j * d * d + e];
+            for (long e = 0; e < d * d; ++e) Hbar[bh][e] *= (double)B / (double)L;
+        }
     });
     parallel_for(ntiles, nthreads, [&](long r) {
         const long bh = tiles[2 * r], i = tiles[2 * r + 1];
@@ -411,11 +423,28 @@ int oracle_pisa_attention(const float* q, const float* k, const float* v, long B
             const long t = i * B + m;
             row_stats_form(q + (bh * L + t) * d, k + bh * L * d, v + bh * L * d, d, B, nblk,
                            sel.data(), order, gate, kbar[bh].data(), vsum[bh].data(),
-                           H[bh].data(), C[bh].data(), out + (r * B + m) * d,
+                           H[bh].data(), C[bh].data(),
+                           (global_h && order >= 1) ? Hbar[bh].data() : nullptr, out + (r * B + m) * d,
                            lse ? lse + r * B + m : nullptr, xs, ls, num);
         }
     });
     return 0;
+}
+
+int oracle_pisa_attention(const float* q, const float* k, const float* v, long BH, long L,
+                          long d, long B, long K, int order, int gate, const int64_t* tiles,
+                          long ntiles, double* out, double* lse, int nthreads) {
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 0, tiles, ntiles, out, lse,
+                               nthreads);
+}
+
+// The PISA hybrid: as oracle_pisa_attention with every H_j replaced by the
+// global H-bar = (B/L) sum_j H_j of the (batch, head).
+int oracle_pisa_hybrid(const float* q, const float* k, const float* v, long BH, long L, long d,
+                       long B, long K, int order, int gate, const int64_t* tiles, long ntiles,
+                       double* out, double* lse, int nthreads) {
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 1, tiles, ntiles, out, lse,
+                               nthreads);
 }
 
 // Token-wise form (no block statistics), same selection; full output [BH, L, d].

@@ -91,7 +91,8 @@ def gpu_select(q, k, B, K, dt):
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-@pytest.mark.parametrize("d,B,L", [(64, 64, 2048), (128, 64, 4096), (128, 128, 4096), (64, 128, 1024)])
+@pytest.mark.parametrize("d,B,L", [(64, 64, 2048), (128, 64, 4096), (128, 128, 4096), (64, 128, 1024),
+                                   (128, 64, 2560), (64, 64, 4608), (128, 128, 1152)])
 @pytest.mark.parametrize("Kfrac", [0.0, 0.1, 0.5, 1.0])
 def test_select_parity(dt, d, B, L, Kfrac):
     nblk = L // B
@@ -121,7 +122,7 @@ def test_select_planted_ties():
         assert np.array_equal(idx, ridx) and np.array_equal(mask, rmask)
 
 
-@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5_L16896_s90"])
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5_L4608_s75", "c5_L16896_s90"])
 def test_select_full_size(name):
     w, (q, k, v) = workload(name)
     idx, mask = gpu_select(q, k, w.B, w.K, w.dtype)

@@ -335,3 +335,59 @@ def test_canonical_centroids_match_numpy_restatement():
         c = oracle.centroids_f32(k, B)
         ref = np_tree_sum(k.reshape(2, 512 // B, B, 64), 2) * np.float32(1.0 / B)
         assert np.array_equal(c.view(np.uint32), ref.view(np.uint32))
+
+
+# ----------------------------------------------------------------------------
+# the PISA hybrid (global H-bar), "Sparse Linear Attention" blog and PISA
+# paper section 3.3 / Appendix C
+# ----------------------------------------------------------------------------
+
+def test_hybrid_equals_per_block_when_every_block_has_the_same_statistic():
+    # Shifting a block's keys by a constant leaves its deviations unchanged, so
+    # blocks built as (base keys + shift_j, base values) all share one H_j;
+    # then H-bar = H_j and the hybrid is the per-block first-order form.
+    rng = np.random.default_rng(19)
+    B, d, nblk = 16, 8, 16
+    # dyadic values: every shifted key is exact in fp32, so the deviations agree bit for bit
+    kb = (rng.integers(-16, 17, (B, d)) / 8.0).astype(np.float32)
+    vb = rng.standard_normal((B, d)).astype(np.float32)
+    shifts = (rng.integers(-4, 5, (nblk, 1, d)) / 4.0).astype(np.float32)
+    k = (kb[None] + shifts).reshape(1, nblk * B, d).astype(np.float32)
+    v = np.tile(vb, (nblk, 1))[None].astype(np.float32)
+    q = (rng.standard_normal((1, nblk * B, d)) * 0.5).astype(np.float32)
+    np.testing.assert_allclose(oracle.pisa_hybrid(q, k, v, B, 3, 1), oracle.pisa_attention(q, k, v, B, 3, 1),
+                               rtol=0, atol=1e-12)
+
+
+def test_hybrid_numerator_differs_by_the_appendix_c_residual():
+    # N_hybrid - N_per-block = sum_U alpha_tj (H-bar - H_j) q_t  (= -q R_t in
+    # Appendix C) while the denominators agree, so
+    # (o_hybrid - o_per-block) * D-hat = sum_U alpha_tj (H-bar - H_j) q_t.
+    q, k, v = small(20, BH=1, L=256, d=16, scale=1.0)
+    B, K = 16, 3
+    oh, lh = oracle.pisa_hybrid(q, k, v, B, K, 1, want_lse=True)
+    op, lp = oracle.pisa_attention(q, k, v, B, K, 1, want_lse=True)
+    np.testing.assert_allclose(lh, lp, rtol=0, atol=1e-12)
+    q64, k64, v64 = (np.asarray(x[0], np.float64) for x in (q, k, v))
+    nblk = 256 // B
+    kb = k64.reshape(nblk, B, 16)
+    vb = v64.reshape(nblk, B, 16)
+    H = np.einsum("jna,jnb->jab", vb, kb - kb.mean(axis=1, keepdims=True))
+    Hbar = H.mean(axis=0)
+    _, mask, _ = oracle.select(q, k, B, K)
+    for i in range(nblk):
+        sel = np.array([(mask[0, i, j // 32] >> (j % 32)) & 1 for j in range(nblk)], bool)
+        for m in range(B):
+            t = i * B + m
+            alpha = np.exp(q64[t] @ kb.mean(axis=1).T)                 # unshifted e^{q.kbar_j}
+            resid = sum(alpha[j] * ((Hbar - H[j]) @ q64[t]) for j in range(nblk) if not sel[j])
+            np.testing.assert_allclose((oh[0, t] - op[0, t]) * np.exp(lh[0, t]), resid, rtol=1e-9, atol=1e-9)
+
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_hybrid_special_cases(order):
+    q, k, v = small(21, L=256, d=16, scale=2.0)
+    B = 16
+    np.testing.assert_allclose(oracle.pisa_hybrid(q, k, v, B, 16, order), torch_dense(q, k, v), rtol=0, atol=1e-12)
+    if order == 0:
+        np.testing.assert_array_equal(oracle.pisa_hybrid(q, k, v, B, 4, 0), oracle.pisa_attention(q, k, v, B, 4, 0))
