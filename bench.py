@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--heads", type=int, default=None, help="override head count (profiling small cases)")
+    p.add_argument("--no-hybrid", action="store_true", help="skip the PISA-hybrid (global H-bar) record")
     return p.parse_args()
 
 
@@ -374,6 +375,30 @@ def main():
                      "frac_hbm": s_bytes / (s_ms * 1e-3) / 1e9 / hbm}
         del sbuf
 
+    # The PISA hybrid (global H-bar, the paper's own speed path) on the same
+    # inputs: a separate record, timed as whole calls of pisa_attention.
+    hybrid_rec = None
+    if not args.no_hybrid and tdt == torch.bfloat16 and order <= 1:
+        hws = torch.empty(pisa.pisa_workspace_bytes(1, BH, L, d, B, K, order, tdt, "hybrid_tc"), dtype=torch.uint8,
+                          device="cuda")
+        hout = torch.empty_like(q)
+        for _ in range(3):
+            pisa.pisa_attention(q, k, v, B, K, order, path="hybrid_tc", out=hout, workspace=hws)
+        ha, hb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(5, args.steps)
+        ha.record(stream)
+        for _ in range(reps):
+            pisa.pisa_attention(q, k, v, B, K, order, path="hybrid_tc", out=hout, workspace=hws)
+        hb.record(stream)
+        torch.cuda.synchronize()
+        pisa.pisa_poll_device_status()
+        h_ms = ha.elapsed_time(hb) / reps
+        hybrid_rec = {"method": "PISA hybrid: exact selected blocks, zeroth-order virtual tokens, global H-bar "
+                                "first-order term (not the per-block H_j formulation of the main line)",
+                      "ms_per_call": h_ms, "full_attn_equiv_tflops": dense_flops / (h_ms * 1e-3) / 1e12,
+                      "speedup_vs_per_block_path": ms_step / h_ms, "launches_per_call": 5}
+        del hws, hout
+
     # end to end through the public call with host buffers: pinned H2D, pisa_attention, D2H
     e2e = None
     if not args.no_e2e:
@@ -427,6 +452,7 @@ def main():
             "roofline": roof,
             "per_kernel": per_kernel,
             "stats_kernel": stats_rec,
+            "hybrid": hybrid_rec,
             "cpu_baseline": cpu,
             "clocks": clk,
             "e2e": e2e,

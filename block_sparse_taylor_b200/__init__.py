@@ -33,7 +33,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libpisa_b200.so")
 
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
 PISA_F32, PISA_BF16 = 0, 1
-PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2}
+PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2, "hybrid_tc": 3}
 PATH_NAMES = {v: k for k, v in PATHS.items()}
 
 

@@ -18,6 +18,8 @@
 #include "attn_stats.cuh"
 #include "attn_tc.cuh"
 #include "stats_tc.cuh"
+#include "hybrid_prep.cuh"
+#include "attn_hybrid.cuh"
 
 using pisa::bf16;
 
@@ -100,12 +102,6 @@ StatsLayout stats_layout(const Dims& g, int order, pisa_dtype dtype) {
     if (order == 2) o += align_up(esize(dtype) * g.BH * g.nblk * g.d * g.d);
     s.total = o;
     return s;
-}
-
-int next_pow2(int x) {
-    int p = 1;
-    while (p < x) p <<= 1;
-    return p;
 }
 
 // ---------------------------------------------------------------------------
@@ -231,12 +227,13 @@ pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pi
 struct WsLayout {
     size_t stats, mask, idx, total;
     StatsLayout sl;
+    size_t kbar_bf, vsum_bf, hbar_acc, hbar_bf;  // hybrid path only
 };
 
 WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path path) {
     WsLayout w{};
-    if (path == PISA_PATH_RECOMPUTE_TC) {
-        // The token-form path needs only the centroids (for the selection).
+    if (path == PISA_PATH_RECOMPUTE_TC || path == PISA_PATH_HYBRID_TC) {
+        // The token-form and hybrid paths need only the fp32 centroids (for the selection).
         w.sl = StatsLayout{};
         w.sl.total = align_up(sizeof(float) * g.BH * g.nblk * g.d);
     } else {
@@ -249,8 +246,23 @@ WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path 
     o += align_up(sizeof(uint32_t) * g.BH * g.nblk * g.words);
     w.idx = o;
     o += align_up(sizeof(int32_t) * g.BH * g.nblk * (K > 0 ? K : 1));
+    if (path == PISA_PATH_HYBRID_TC) {
+        w.kbar_bf = o;
+        o += align_up(2 * g.BH * g.nblk * g.d);
+        w.vsum_bf = o;
+        o += align_up(2 * g.BH * g.nblk * g.d);
+        w.hbar_acc = o;
+        o += align_up(4 * g.BH * g.d * g.d);
+        w.hbar_bf = o;
+        o += align_up(2 * g.BH * g.d * g.d);
+    }
     w.total = o;
     return w;
+}
+
+bool hybrid_path_available(const Dims& g, pisa_dtype dtype, int order) {
+    return dtype == PISA_BF16 && pisa::attn_tc_supported((int)g.d, (int)g.B) && g.L % 128 == 0 && order <= 1 &&
+           g.BH * g.L <= 0x7fffffffL;
 }
 
 bool tc_path_available(const Dims& g, pisa_dtype dtype) {
@@ -351,7 +363,8 @@ size_t pisa_workspace_bytes_ex(int batch, int heads, int L, int d, int B, int K,
     if (K < 0 || K > g.nblk) return 0;
     if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
     if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype)) return 0;
-    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC) return 0;
+    if (path == PISA_PATH_HYBRID_TC && !hybrid_path_available(g, dtype, order)) return 0;
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC) return 0;
     return ws_layout(g, K, order, dtype, path).total;
 }
 
@@ -373,7 +386,9 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
     if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype))
         return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
-    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC)
+    if (path == PISA_PATH_HYBRID_TC && !hybrid_path_available(g, dtype, order))
+        return fail(PISA_ERR_UNSUPPORTED, "hybrid path needs bf16, d and B in {64, 128}, L %% 128 == 0, order <= 1");
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC)
         return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
     const WsLayout w = ws_layout(g, K, order, dtype, path);
     if (ws_bytes < w.total)
@@ -388,14 +403,31 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     st.B = B;
     st.nblk = (int)g.nblk;
     st.dtype = dtype;
-    st.order = (path == PISA_PATH_RECOMPUTE_TC) ? 0 : order;
+    st.order = (path == PISA_PATH_RECOMPUTE_TC || path == PISA_PATH_HYBRID_TC) ? 0 : order;
     st.kbar = (float*)(ws + w.stats + w.sl.kbar);
-    st.vsum = (path == PISA_PATH_RECOMPUTE_TC) ? nullptr : (float*)(ws + w.stats + w.sl.vsum);
+    st.vsum = (path == PISA_PATH_STATS) ? (float*)(ws + w.stats + w.sl.vsum) : nullptr;
     st.hstat = st.order >= 1 ? (void*)(ws + w.stats + w.sl.hstat) : nullptr;
     st.cov = st.order == 2 ? (void*)(ws + w.stats + w.sl.cov) : nullptr;
     uint32_t* mask = (uint32_t*)(ws + w.mask);
     int32_t* idx = (int32_t*)(ws + w.idx);
 
+    if (path == PISA_PATH_HYBRID_TC) {
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        bf16* kbar_bf = (bf16*)(ws + w.kbar_bf);
+        bf16* vsum_bf = (bf16*)(ws + w.vsum_bf);
+        float* hacc = (float*)(ws + w.hbar_acc);
+        bf16* hbf = (bf16*)(ws + w.hbar_bf);
+        cudaError_t e = cudaMemsetAsync(hacc, 0, sizeof(float) * g.BH * g.d * g.d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(H-bar)");
+        r = pisa::run_hybrid_prep(k, v, st.kbar, kbar_bf, vsum_bf, hacc, hbf, g.BH, (int)g.L, (int)g.d, (int)g.B,
+                                  (int)g.nblk, status, s, &g_last_error);
+        if (r != PISA_OK) return r;
+        r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s);
+        if (r != PISA_OK) return r;
+        return pisa::run_attn_hybrid(q, k, v, kbar_bf, vsum_bf, hbf, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B,
+                                     (int)g.nblk, (int)g.words, order, status, s, &g_last_error);
+    }
     if (path == PISA_PATH_RECOMPUTE_TC) {
         r = run_centroids(k, st.kbar, g, dtype, s);
         if (r != PISA_OK) return r;

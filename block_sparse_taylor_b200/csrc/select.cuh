@@ -115,14 +115,29 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
     const int i0 = blockIdx.x * QT;
     const int nq = min(QT, nblk - i0);
 
-    // 1. tile means
-    for (int e = tid; e < nq * D; e += C::THREADS) {
-        const int t = e / D, c = e % D;
+    // 1. tile means; bf16 tiles of 64 rows are read as bf16x2 pairs (two
+    // columns per thread) so that more bytes are in flight per thread
+    constexpr int VEC = (sizeof(T) == 2 && BS <= 64) ? 2 : 1;
+    constexpr int CPT = D / VEC;  // threads per tile
+    for (int e = tid; e < nq * CPT; e += C::THREADS) {
+        const int t = e / CPT, c = (e % CPT) * VEC;
         const T* src = q + ((size_t)bh * L + (size_t)(i0 + t) * BS) * D + c;
-        float a[BS];
+        if constexpr (VEC == 2) {
+            float a0[BS], a1[BS];
 #pragma unroll
-        for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
-        qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+            for (int n = 0; n < BS; ++n) {
+                const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(src + (size_t)n * D);
+                a0[n] = __low2float(p);
+                a1[n] = __high2float(p);
+            }
+            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a0), 1.0f / (float)BS);
+            qbar[t * D + c + 1] = __fmul_rn(tree_sum<BS>(a1), 1.0f / (float)BS);
+        } else {
+            float a[BS];
+#pragma unroll
+            for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
+            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+        }
     }
     __syncthreads();
 
@@ -152,18 +167,18 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
     for (int t = warp; t < nq; t += 8) {
         const float* st = sc + t * SS;
         const size_t row = (size_t)bh * nblk + i0 + t;
-        uint32_t T = 0u;  // K-th largest ordered score (unused when K is 0 or nblk)
+        uint32_t thr = 0u;  // K-th largest ordered score (unused when K is 0 or nblk)
         int need = 0;     // how many of the ties at T to take, lowest index first
         if (K > 0 && K < nblk) {
             for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t cand = T | (1u << bit);
+                const uint32_t cand = thr | (1u << bit);
                 int cnt = 0;
                 for (int j = lane; j < nblk; j += 32) cnt += ordered_key(st[j]) >= cand;
                 cnt = __reduce_add_sync(0xffffffffu, cnt);
-                if (cnt >= K) T = cand;
+                if (cnt >= K) thr = cand;
             }
             int gt = 0;
-            for (int j = lane; j < nblk; j += 32) gt += ordered_key(st[j]) > T;
+            for (int j = lane; j < nblk; j += 32) gt += ordered_key(st[j]) > thr;
             need = K - __reduce_add_sync(0xffffffffu, gt);
         }
         int off = 0, eq_seen = 0;
@@ -172,10 +187,10 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
             const int j = w * 32 + lane;
             const bool in = j < nblk;
             const uint32_t o = in ? ordered_key(st[j]) : 0u;
-            const unsigned eq = __ballot_sync(0xffffffffu, in && o == T);
+            const unsigned eq = __ballot_sync(0xffffffffu, in && o == thr);
             const int rank = eq_seen + __popc(eq & lt_mask);
             eq_seen += __popc(eq);
-            const bool sel = in && (K == nblk || (K > 0 && (o > T || (o == T && rank < need))));
+            const bool sel = in && (K == nblk || (K > 0 && (o > thr || (o == thr && rank < need))));
             const unsigned bits = __ballot_sync(0xffffffffu, sel);
             if (mask && lane == 0) mask[row * words + w] = bits;
             if (idx && sel) idx[row * K + off + __popc(bits & lt_mask)] = j;

@@ -75,8 +75,16 @@ typedef enum { PISA_F32 = 0, PISA_BF16 = 1 } pisa_dtype;
 typedef enum {
     PISA_PATH_AUTO = 0,
     PISA_PATH_STATS = 1,
-    PISA_PATH_RECOMPUTE_TC = 2
+    PISA_PATH_RECOMPUTE_TC = 2,
+    PISA_PATH_HYBRID_TC = 3
 } pisa_path;
+/* PISA_PATH_HYBRID_TC is another method, requested explicitly (AUTO never
+ * picks it): the PISA paper's hybrid, where every H_j of the first-order term
+ * is replaced by the global statistic H-bar = (B/L) sum_j H_j of the (batch,
+ * head), so the numerator's first-order part is (sum_{j in U_i} e^{l_tj})
+ * H-bar q_t (PISA paper section 3.3 and Figure 3, phase 3; H-bar as in the
+ * "Sparse Linear Attention" blog).  Unselected blocks cost one virtual token
+ * each instead of their tokens.  bf16, order 0 or 1, L % 128 == 0. */
 
 /* Block statistics of one call (all device pointers, caller-owned).
  *   kbar  [BH, nblk, d] fp32 : centroid, canonical fp32 mean (see pisa_select)

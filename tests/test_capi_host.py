@@ -67,6 +67,7 @@ def call_ex(L=1024, d=64, B=64, K=4, order=1, dtype=pisa.PISA_BF16, path=0, ws_b
     (dict(ws=ctypes.c_void_p(0x1008)), pisa.PISA_ERR_INVALID_ARG),  # misaligned workspace
     (dict(path=9), pisa.PISA_ERR_INVALID_ARG),
     (dict(path=2, dtype=pisa.PISA_F32), pisa.PISA_ERR_UNSUPPORTED),  # tensor cores need bf16
+    (dict(path=3, order=2), pisa.PISA_ERR_UNSUPPORTED),              # the hybrid has orders 0 and 1
     (dict(L=1024 * 8192, B=64), pisa.PISA_ERR_UNSUPPORTED),          # nblk > 4096
 ])
 def test_bad_arguments_are_rejected_before_launch(kw, status):

@@ -242,3 +242,48 @@ def test_device_status_is_clean():
     q, k, v = pisa_synth.random_qkv(700, 1, 1024, 128, dtype="bf16")
     run_attn(q, k, v, 64, 4, 1, "bf16", "recompute_tc")
     pisa.pisa_poll_device_status()
+
+
+# ---------------------------------------------------------------------------
+# the PISA hybrid path (global H-bar): GPU vs the oracle's hybrid form
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("Kfrac", [0.0, 0.25, 1.0])
+def test_hybrid_small(d, B, order, Kfrac):
+    L = 2048
+    nblk = L // B
+    K = int(round(Kfrac * nblk))
+    q, k, v = pisa_synth.random_qkv(800 + d + B + order, 2, L, d, scale=2.0, dtype="bf16")
+    got = run_attn(q, k, v, B, K, order, "bf16", "hybrid_tc")
+    ref = oracle.pisa_hybrid(q, k, v, B, K, order)
+    err = rel_l2(got, ref)
+    assert err <= TOL["bf16"], err
+    assert err <= 5e-3, err
+
+
+@pytest.mark.parametrize("case", ["ragged", "clustered", "sharp"])
+def test_hybrid_edge_cases(case):
+    d, B, L, K = 128, 64, 1152, 4
+    scale = 8.0 if case == "sharp" else 2.0
+    if case == "clustered":
+        w = pisa_synth.workloads()["c2"].with_(heads=2, L=2048, n_centres=32, d=128)
+        q, k, v = pisa_synth.generate(w)
+        L, K = 2048, 4
+    else:
+        q, k, v = pisa_synth.random_qkv(850 + len(case), 2, L, d, scale=scale, dtype="bf16")
+    got = run_attn(q, k, v, B, K, 1, "bf16", "hybrid_tc")
+    ref = oracle.pisa_hybrid(q, k, v, B, K, 1)
+    assert rel_l2(got, ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name,per_head,nheads", [("c3", 2, 8), ("c5_L16896_s90", 2, 8), ("c4", 1, 4)])
+def test_hybrid_full_size_sampled(name, per_head, nheads):
+    w, (q, k, v) = workload(name)
+    got = run_attn(q, k, v, w.B, w.K, 1, w.dtype, "hybrid_tc")
+    heads = list(np.random.default_rng(9).choice(w.BH, nheads, replace=False))
+    tiles = sample_tiles(w.BH, w.nblk, per_head, seed=13, heads=heads)
+    ref = oracle.pisa_hybrid(q, k, v, w.B, w.K, 1, tiles=tiles)
+    err = rel_l2(rows_of(got, tiles, w.B), ref)
+    assert err <= TOL[w.dtype], (name, err)
