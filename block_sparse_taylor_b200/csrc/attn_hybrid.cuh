@@ -308,90 +308,98 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int jt = 0; jt < NT; ++jt) {
             if (!tc::mbar_wait_warp(bar(B_SFULL + h), jt & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
-            if (jt < nut) {
-                // ---- union tile: BPT blocks
-                int blk[BPT];
-                bool sel[BPT], live[BPT];
-                float cand[BPT], l2[BPT];
+            // the whole 128-column S tile in registers: one TMEM round trip
+            uint32_t sv[C::NK];
+#pragma unroll
+            for (int c = 0; c < C::NK / 32; ++c)
+                tc::tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c));
+            tc::tmem_wait_ld();
+            // per-column weight rule of this tile: 0 = off, 1 = exact e^{x}, 2 = virtual weight
+            float mc = -INFINITY;
+            bool sel[BPT], live[BPT];
+            float l2[BPT];
+            uint32_t okw[4] = {0u, 0u, 0u, 0u};
+            const bool is_union = jt < nut;
+            if (is_union) {
 #pragma unroll
                 for (int b = 0; b < BPT; ++b) {
                     const int li = jt * BPT + b;
                     live[b] = li < nu;
-                    blk[b] = blist[live[b] ? li : 0];
-                    sel[b] = live[b] && ((myw[blk[b] >> 5] >> (blk[b] & 31)) & 1u);
-                }
-#pragma unroll
-                for (int b = 0; b < BPT; ++b) {
-                    cand[b] = -INFINITY;
+                    const int blk = blist[live[b] ? li : 0];
+                    sel[b] = live[b] && ((myw[blk >> 5] >> (blk & 31)) & 1u);
                     l2[b] = 0.f;
                     if (!live[b]) continue;
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < CPB; c += 2) {
-                        uint32_t r0[32], r1[32];
-                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float x0 = __uint_as_float(r0[e]), x1 = __uint_as_float(r1[e]);
-                            if (sel[b]) {
-                                m4[e & 3] = fmaxf(m4[e & 3], fmaxf(x0, x1));
-                            } else {
-                                s4[e & 3] += x0 + x1;
-                            }
-                        }
-                    }
+                    const uint32_t* x = sv + b * BS;
                     if (sel[b]) {
-                        cand[b] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
+                        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                        for (int e = 0; e < BS; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(x[e]));
+                        mc = fmaxf(mc, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E);
                     } else {
+                        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int e = 0; e < BS; ++e) s4[e & 3] += __uint_as_float(x[e]);
                         l2[b] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs * LOG2E;
-                        cand[b] = l2[b];
+                        mc = fmaxf(mc, l2[b]);
                     }
                 }
-                float mc = cand[0];
+            } else {
+                // virtual tile: 128 centroids; a column counts unless its block is
+                // in the union or past nblk
+                const int vj0 = (jt - nut) * 128;
 #pragma unroll
-                for (int b = 1; b < BPT; ++b) mc = fmaxf(mc, cand[b]);
-                const bool raise = mc > m_run + 8.0f;
-                const float scale = raise ? tc::ex2(m_run - mc) : 1.0f;
-                if (raise) {
-                    dsum *= scale;
-                    amass *= scale;
-                    m_run = mc;
+                for (int w = 0; w < 4; ++w) {
+                    const int j = vj0 + 32 * w;
+                    uint32_t inb = 0u;
+                    if (j < nblk) inb = (nblk - j >= 32) ? 0xffffffffu : ((1u << (nblk - j)) - 1u);
+                    okw[w] = inb & ~((j >> 5) < words ? uwords[j >> 5] : 0u);
                 }
-                if (__any_sync(0xffffffffu, raise) && jt > 0) {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t raw[32];
-                        tc::tmem_ld32(o_addr + c * 32, raw);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
-                        tc::tmem_st32(o_addr + c * 32, raw);
-                    }
+                for (int e = 0; e < C::NK; ++e) {
+                    const float x = ((okw[e >> 5] >> (e & 31)) & 1u) ? __uint_as_float(sv[e]) : -INFINITY;
+                    m4[e & 3] = fmaxf(m4[e & 3], x);
                 }
+                mc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
+            }
+            const bool raise = mc > m_run + 8.0f;
+            const float scale = raise ? tc::ex2(m_run - mc) : 1.0f;
+            if (raise) {
+                dsum *= scale;
+                amass *= scale;
+                m_run = mc;
+            }
+            if (__any_sync(0xffffffffu, raise) && jt > 0) {
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t raw[16];
+                    tc::tmem_ld16(o_addr + c * 16, raw);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
+                    tc::tmem_st16(o_addr + c * 16, raw);
+                }
+            }
+            if (is_union) {
 #pragma unroll
                 for (int b = 0; b < BPT; ++b) {
+                    const uint32_t* x = sv + b * BS;
                     if (live[b] && sel[b]) {
                         float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int c = 0; c < CPB; c += 2) {
-                            uint32_t r0[32], r1[32], p0[16], p1[16];
-                            tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                            tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                            tc::tmem_wait_ld();
+                        for (int c = 0; c < CPB; ++c) {
+                            uint32_t pk[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                const float a0 = tc::ex2(fmaf(__uint_as_float(r0[2 * e]), LOG2E, -m_run));
-                                const float a1 = tc::ex2(fmaf(__uint_as_float(r0[2 * e + 1]), LOG2E, -m_run));
-                                const float b0 = tc::ex2(fmaf(__uint_as_float(r1[2 * e]), LOG2E, -m_run));
-                                const float b1 = tc::ex2_fma(fmaf(__uint_as_float(r1[2 * e + 1]), LOG2E, -m_run));
-                                d4[e & 3] += (a0 + a1) + (b0 + b1);
-                                p0[e] = tc::pack_bf16x2(a0, a1);
-                                p1[e] = tc::pack_bf16x2(b0, b1);
+                                const float xa = __uint_as_float(x[32 * c + 2 * e]);
+                                const float xb = __uint_as_float(x[32 * c + 2 * e + 1]);
+                                const float a0 = tc::ex2(fmaf(xa, LOG2E, -m_run));
+                                const float a1 = (e & 1) ? tc::ex2_fma(fmaf(xb, LOG2E, -m_run))
+                                                         : tc::ex2(fmaf(xb, LOG2E, -m_run));
+                                d4[e & 3] += a0 + a1;
+                                pk[e] = tc::pack_bf16x2(a0, a1);
                             }
-                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, p0);
-                            tc::tmem_st16(s_addr + (b * CPB + c + 1) * 16, p1);
+                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
                         }
                         dsum += (d4[0] + d4[1]) + (d4[2] + d4[3]);
                     } else {
@@ -408,73 +416,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
             } else {
-                // ---- virtual tile: 128 centroids; a column counts unless its block
-                // is in the union or past nblk
-                const int vj0 = (jt - nut) * 128;
-                uint32_t okw[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int j = vj0 + 32 * w;
-                    uint32_t inb = 0u;
-                    if (j < nblk) inb = (nblk - j >= 32) ? 0xffffffffu : ((1u << (nblk - j)) - 1u);
-                    okw[w] = inb & ~((j >> 5) < words ? uwords[j >> 5] : 0u);
-                }
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < 4; c += 2) {
-                    uint32_t r0[32], r1[32];
-                    tc::tmem_ld32(s_addr + c * 32, r0);
-                    tc::tmem_ld32(s_addr + (c + 1) * 32, r1);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x0 = ((okw[c] >> e) & 1u) ? __uint_as_float(r0[e]) : -INFINITY;
-                        const float x1 = ((okw[c + 1] >> e) & 1u) ? __uint_as_float(r1[e]) : -INFINITY;
-                        m4[e & 3] = fmaxf(m4[e & 3], fmaxf(x0, x1));
-                    }
-                }
-                const float mc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
-                const bool raise = mc > m_run + 8.0f;
-                const float scale = raise ? tc::ex2(m_run - mc) : 1.0f;
-                if (raise) {
-                    dsum *= scale;
-                    amass *= scale;
-                    m_run = mc;
-                }
-                if (__any_sync(0xffffffffu, raise) && jt > 0) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t raw[32];
-                        tc::tmem_ld32(o_addr + c * 32, raw);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
-                        tc::tmem_st32(o_addr + c * 32, raw);
-                    }
-                }
                 float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 4; c += 2) {
-                    uint32_t r0[32], r1[32], p0[16], p1[16];
-                    tc::tmem_ld32(s_addr + c * 32, r0);
-                    tc::tmem_ld32(s_addr + (c + 1) * 32, r1);
-                    tc::tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float a0 = ((okw[c] >> (2 * e)) & 1u)
-                                             ? tc::ex2(fmaf(__uint_as_float(r0[2 * e]), LOG2E, -m_run)) : 0.f;
+                        const int e0 = 32 * c + 2 * e;
+                        const float a0 = ((okw[c] >> (2 * e)) & 1u) ? tc::ex2(fmaf(__uint_as_float(sv[e0]), LOG2E, -m_run))
+                                                                    : 0.f;
                         const float a1 = ((okw[c] >> (2 * e + 1)) & 1u)
-                                             ? tc::ex2(fmaf(__uint_as_float(r0[2 * e + 1]), LOG2E, -m_run)) : 0.f;
-                        const float b0 = ((okw[c + 1] >> (2 * e)) & 1u)
-                                             ? tc::ex2(fmaf(__uint_as_float(r1[2 * e]), LOG2E, -m_run)) : 0.f;
-                        const float b1 = ((okw[c + 1] >> (2 * e + 1)) & 1u)
-                                             ? tc::ex2(fmaf(__uint_as_float(r1[2 * e + 1]), LOG2E, -m_run)) : 0.f;
-                        a4[e & 3] += (a0 + a1) + (b0 + b1);
-                        p0[e] = tc::pack_bf16x2(a0, a1);
-                        p1[e] = tc::pack_bf16x2(b0, b1);
+                                             ? tc::ex2(fmaf(__uint_as_float(sv[e0 + 1]), LOG2E, -m_run))
+                                             : 0.f;
+                        a4[e & 3] += a0 + a1;
+                        pk[e] = tc::pack_bf16x2(a0, a1);
                     }
-                    tc::tmem_st16(s_addr + c * 16, p0);
-                    tc::tmem_st16(s_addr + (c + 1) * 16, p1);
+                    tc::tmem_st16(s_addr + c * 16, pk);
                 }
                 const float asum = (a4[0] + a4[1]) + (a4[2] + a4[3]);
                 dsum = fmaf((float)BS, asum, dsum);

@@ -252,42 +252,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int j = jt * BPT + b;  // the BPT blocks of a tile share one mask word
                 sel[b] = (mword >> (j & 31)) & 1u;
             }
+            // the whole 128-column S tile in registers: one TMEM round trip per
+            // tile, and pass 2 reuses the values
+            uint32_t sv[C::NK];
+#pragma unroll
+            for (int c = 0; c < C::NK / 32; ++c)
+                tc::tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c));
+            tc::tmem_wait_ld();
             // pass 1: per-block statistics of the logits (exact: max; Taylor:
             // sum, and the sum of squares for order 2), four partial
             // accumulators each so that the reductions are not one long chain
 #pragma unroll
             for (int b = 0; b < BPT; ++b) {
+                const uint32_t* x = sv + b * BS;
                 if (sel[b]) {
                     float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < CPB; c += 2) {
-                        uint32_t r0[32], r1[32];
-                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(r0[e]));
-                            m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(r1[e]));
-                        }
-                    }
+                    for (int e = 0; e < BS; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(x[e]));
                     cand[b] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
                     sbar[b] = 0.f;
                     l2[b] = 0.f;
                 } else {
                     float s4[4] = {0.f, 0.f, 0.f, 0.f}, q4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < CPB; c += 2) {
-                        uint32_t r0[32], r1[32];
-                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float x0 = __uint_as_float(r0[e]), x1 = __uint_as_float(r1[e]);
-                            s4[e & 3] += x0 + x1;
-                            if (ORDER == 2) q4[e & 3] = fmaf(x0, x0, fmaf(x1, x1, q4[e & 3]));
-                        }
+                    for (int e = 0; e < BS; ++e) {
+                        const float xe = __uint_as_float(x[e]);
+                        s4[e & 3] += xe;
+                        if (ORDER == 2) q4[e & 3] = fmaf(xe, xe, q4[e & 3]);
                     }
                     const float sb = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs;
                     float w = 0.f;
@@ -314,39 +305,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (__any_sync(0xffffffffu, raise) && jt > 0) {
                 // the previous PV of this tile is complete (covered by S_FULL)
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t raw[32];
-                    tc::tmem_ld32(o_addr + c * 32, raw);
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t raw[16];
+                    tc::tmem_ld16(o_addr + c * 16, raw);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
-                    tc::tmem_st32(o_addr + c * 32, raw);
+                    for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * scale);
+                    tc::tmem_st16(o_addr + c * 16, raw);
                 }
             }
-            // pass 2: weights, written as bf16 over the S columns
+            // pass 2: weights, written as bf16 over the S columns (32 columns
+            // -> 16 packed words per store)
 #pragma unroll
             for (int b = 0; b < BPT; ++b) {
+                const uint32_t* x = sv + b * BS;
                 if (sel[b]) {
                     float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < CPB; c += 2) {
-                        uint32_t r0[32], r1[32], p0[16], p1[16];
-                        tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                        tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                        tc::tmem_wait_ld();
+                    for (int c = 0; c < CPB; ++c) {
+                        uint32_t pk[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float a0 = tc::ex2(fmaf(__uint_as_float(r0[2 * e]), LOG2E, -m_run));
-                            const float a1 = tc::ex2(fmaf(__uint_as_float(r0[2 * e + 1]), LOG2E, -m_run));
-                            const float b0 = tc::ex2(fmaf(__uint_as_float(r1[2 * e]), LOG2E, -m_run));
-                            const float b1 = tc::ex2_fma(fmaf(__uint_as_float(r1[2 * e + 1]), LOG2E, -m_run));
-                            d4[e & 3] += (a0 + a1) + (b0 + b1);
-                            p0[e] = tc::pack_bf16x2(a0, a1);
-                            p1[e] = tc::pack_bf16x2(b0, b1);
+                            const float xa = __uint_as_float(x[32 * c + 2 * e]);
+                            const float xb = __uint_as_float(x[32 * c + 2 * e + 1]);
+                            const float a0 = tc::ex2(fmaf(xa, LOG2E, -m_run));
+                            // every fourth exponential on the FMA pipe
+                            const float a1 = (e & 1) ? tc::ex2_fma(fmaf(xb, LOG2E, -m_run))
+                                                     : tc::ex2(fmaf(xb, LOG2E, -m_run));
+                            d4[e & 3] += a0 + a1;
+                            pk[e] = tc::pack_bf16x2(a0, a1);
                         }
-                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, p0);
-                        tc::tmem_st16(s_addr + (b * CPB + c + 1) * 16, p1);
+                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
                     }
                     dsum += (d4[0] + d4[1]) + (d4[2] + d4[3]);
                 } else {
@@ -355,20 +345,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (ORDER >= 1) {
                         const float c0 = alpha * (1.0f - sbar[b]);
 #pragma unroll
-                        for (int c = 0; c < CPB; c += 2) {
-                            uint32_t r0[32], r1[32], p0[16], p1[16];
-                            tc::tmem_ld32(s_addr + (b * CPB + c) * 32, r0);
-                            tc::tmem_ld32(s_addr + (b * CPB + c + 1) * 32, r1);
-                            tc::tmem_wait_ld();
+                        for (int c = 0; c < CPB; ++c) {
+                            uint32_t pk[16];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                p0[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(r0[2 * e]), c0),
-                                                        fmaf(alpha, __uint_as_float(r0[2 * e + 1]), c0));
-                                p1[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(r1[2 * e]), c0),
-                                                        fmaf(alpha, __uint_as_float(r1[2 * e + 1]), c0));
-                            }
-                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, p0);
-                            tc::tmem_st16(s_addr + (b * CPB + c + 1) * 16, p1);
+                            for (int e = 0; e < 16; ++e)
+                                pk[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(x[32 * c + 2 * e]), c0),
+                                                        fmaf(alpha, __uint_as_float(x[32 * c + 2 * e + 1]), c0));
+                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
                         }
                     } else {
                         uint32_t pk[16];

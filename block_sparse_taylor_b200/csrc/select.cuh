@@ -162,24 +162,47 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
         __syncthreads();
     }
 
-    // 3. top-K, one warp per tile
+    // 3. top-K, one warp per tile.  For nblk <= 1024 every lane keeps its
+    // blocks' ordered keys (j = lane + 32 i) in registers during the search.
     const unsigned lt_mask = (1u << lane) - 1u;
+    const int nk = (nblk + 31) / 32;
     for (int t = warp; t < nq; t += 8) {
         const float* st = sc + t * SS;
         const size_t row = (size_t)bh * nblk + i0 + t;
         uint32_t thr = 0u;  // K-th largest ordered score (unused when K is 0 or nblk)
-        int need = 0;     // how many of the ties at T to take, lowest index first
+        int need = 0;       // how many of the ties at thr to take, lowest index first
         if (K > 0 && K < nblk) {
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t cand = thr | (1u << bit);
-                int cnt = 0;
-                for (int j = lane; j < nblk; j += 32) cnt += ordered_key(st[j]) >= cand;
-                cnt = __reduce_add_sync(0xffffffffu, cnt);
-                if (cnt >= K) thr = cand;
+            if (nk <= 32) {
+                uint32_t kv[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int j = lane + 32 * i;
+                    kv[i] = (i < nk && j < nblk) ? ordered_key(st[j]) : 0u;  // 0 sorts below every score
+                }
+                for (int bit = 31; bit >= 0; --bit) {
+                    const uint32_t cand = thr | (1u << bit);
+                    int cnt = 0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) cnt += (i < nk) & (kv[i] >= cand);
+                    cnt = __reduce_add_sync(0xffffffffu, cnt);
+                    if (cnt >= K) thr = cand;
+                }
+                int gt = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) gt += (i < nk) & (kv[i] > thr);
+                need = K - __reduce_add_sync(0xffffffffu, gt);
+            } else {
+                for (int bit = 31; bit >= 0; --bit) {
+                    const uint32_t cand = thr | (1u << bit);
+                    int cnt = 0;
+                    for (int j = lane; j < nblk; j += 32) cnt += ordered_key(st[j]) >= cand;
+                    cnt = __reduce_add_sync(0xffffffffu, cnt);
+                    if (cnt >= K) thr = cand;
+                }
+                int gt = 0;
+                for (int j = lane; j < nblk; j += 32) gt += ordered_key(st[j]) > thr;
+                need = K - __reduce_add_sync(0xffffffffu, gt);
             }
-            int gt = 0;
-            for (int j = lane; j < nblk; j += 32) gt += ordered_key(st[j]) > thr;
-            need = K - __reduce_add_sync(0xffffffffu, gt);
         }
         int off = 0, eq_seen = 0;
         for (int w = 0; w < words; ++w) {

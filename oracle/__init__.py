@@ -36,11 +36,14 @@ def lib():
                                             ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_hybrid.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
+        L.oracle_pisa_attention_ex.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, li,
+                                               f64p, f64p, ctypes.c_int]
         L.oracle_pisa_bruteforce.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                              ctypes.c_int, f64p, ctypes.c_int]
         L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
-        for fn in ("oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
+        for fn in ("oracle_pisa_attention_ex", "oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
                    "oracle_pisa_bruteforce", "oracle_dense_attention"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -133,6 +136,18 @@ def pisa_hybrid(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, wa
     global H-bar = (B/L) sum_j H_j of each (batch, head) for every unselected
     block (same return convention as pisa_attention)."""
     return _attention(lib().oracle_pisa_hybrid, q, k, v, B, K, order, gate, tiles, nthreads, want_lse)
+
+
+def pisa_attention_ex(q, k, v, B, K, order=1, gate=True, hybrid=False, w_pooled=False, tiles=None, nthreads=None,
+                      want_lse=False):
+    """General form: ``hybrid`` uses the global H-bar (PISA hybrid), ``w_pooled``
+    PWT's diagonal + pooled second-order correction (order 2)."""
+    fn = lib().oracle_pisa_attention_ex
+
+    def call(q_, k_, v_, BH, L, d, B_, K_, o_, g_, tl, n, out, lse, nt):
+        return fn(q_, k_, v_, BH, L, d, B_, K_, o_, g_, int(bool(hybrid)), int(bool(w_pooled)), tl, n, out, lse, nt)
+
+    return _attention(call, q, k, v, B, K, order, gate, tiles, nthreads, want_lse)
 
 
 def pisa_attention(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, want_lse=False):

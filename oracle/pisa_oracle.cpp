@@ -177,8 +177,8 @@ void select_one(const float* q, const float* k, long L, long d, long B, long K,
 void row_stats_form(const float* qrow, const float* k, const float* v, long d, long B,
                     long nblk, const uint8_t* sel, int order, int gate,
                     const double* kbar, const double* vsum, const double* H, const double* C,
-                    const double* Hbar, double* out, double* lse, std::vector<double>& xs,
-                    std::vector<double>& ls, std::vector<double>& num) {
+                    const double* Hbar, const double* wpool, double* out, double* lse,
+                    std::vector<double>& xs, std::vector<double>& ls, std::vector<double>& num) {
     std::vector<double> q(d);
     for (long c = 0; c < d; ++c) q[c] = (double)qrow[c];
     const double ln_b = std::log((double)B);
@@ -196,7 +196,9 @@ void row_stats_form(const float* qrow, const float* k, const float* v, long d, l
             double sb = 0.0;
             for (long c = 0; c < d; ++c) sb += q[c] * kbar[j * d + c];
             double w = 0.0;
-            if (order == 2) {
+            if (order == 2 && wpool) {
+                w = wpool[j];  // the tile's pooled diagonal estimate (gate already applied)
+            } else if (order == 2) {
                 const double* Cj = C + j * d * d;
                 for (long a = 0; a < d; ++a) {
                     double t = 0.0;
@@ -378,8 +380,8 @@ int oracle_select(const float* q, const float* k, long BH, long L, long d, long 
 // The selection (canonical fp32) is recomputed here from q and k.
 static int pisa_attention_impl(const float* q, const float* k, const float* v, long BH, long L,
                                long d, long B, long K, int order, int gate, int global_h,
-                               const int64_t* tiles, long ntiles, double* out, double* lse,
-                               int nthreads) {
+                               int w_pooled, const int64_t* tiles, long ntiles, double* out,
+                               double* lse, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     const long nblk = L / B;
     if (K < 0 || K > nblk) return -1;
@@ -419,12 +421,34 @@ static int pisa_attention_impl(const float* q, const float* k, const float* v, l
         std::vector<uint8_t> sel(nblk);
         for (long j = 0; j < nblk; ++j) sel[j] = (mask[bh][i * words + j / 32] >> (j % 32)) & 1u;
         std::vector<double> xs(nblk * B), ls(nblk), num(d);
+        // PWT's cheap w ([blog1] PWT section): the diagonal of C_j (the within-block
+        // variance of each channel) weighted by the tile mean of q^2 (square first,
+        // then average), one value per (tile, block), gated at ln B.
+        std::vector<double> wpool;
+        if (order == 2 && w_pooled) {
+            std::vector<double> q2(d, 0.0);
+            for (long m = 0; m < B; ++m)
+                for (long c = 0; c < d; ++c) {
+                    const double x = (double)q[(bh * L + i * B + m) * d + c];
+                    q2[c] += x * x;
+                }
+            for (long c = 0; c < d; ++c) q2[c] /= (double)B;
+            wpool.assign(nblk, 0.0);
+            const double ln_b = std::log((double)B);
+            for (long j = 0; j < nblk; ++j) {
+                double w = 0.0;
+                for (long c = 0; c < d; ++c) w += q2[c] * C[bh][j * d * d + c * d + c];
+                w *= 0.5;
+                wpool[j] = (gate && w > ln_b) ? 0.0 : w;
+            }
+        }
         for (long m = 0; m < B; ++m) {
             const long t = i * B + m;
             row_stats_form(q + (bh * L + t) * d, k + bh * L * d, v + bh * L * d, d, B, nblk,
                            sel.data(), order, gate, kbar[bh].data(), vsum[bh].data(),
                            H[bh].data(), C[bh].data(),
-                           (global_h && order >= 1) ? Hbar[bh].data() : nullptr, out + (r * B + m) * d,
+                           (global_h && order >= 1) ? Hbar[bh].data() : nullptr,
+                           wpool.empty() ? nullptr : wpool.data(), out + (r * B + m) * d,
                            lse ? lse + r * B + m : nullptr, xs, ls, num);
         }
     });
@@ -434,8 +458,18 @@ static int pisa_attention_impl(const float* q, const float* k, const float* v, l
 int oracle_pisa_attention(const float* q, const float* k, const float* v, long BH, long L,
                           long d, long B, long K, int order, int gate, const int64_t* tiles,
                           long ntiles, double* out, double* lse, int nthreads) {
-    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 0, tiles, ntiles, out, lse,
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 0, 0, tiles, ntiles, out, lse,
                                nthreads);
+}
+
+// General form: global_h selects the PISA hybrid's H-bar, w_pooled PWT's
+// diagonal + pooled second-order correction (order 2).
+int oracle_pisa_attention_ex(const float* q, const float* k, const float* v, long BH, long L,
+                             long d, long B, long K, int order, int gate, int global_h, int w_pooled,
+                             const int64_t* tiles, long ntiles, double* out, double* lse,
+                             int nthreads) {
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, global_h, w_pooled, tiles,
+                               ntiles, out, lse, nthreads);
 }
 
 // The PISA hybrid: as oracle_pisa_attention with every H_j replaced by the
@@ -443,7 +477,7 @@ int oracle_pisa_attention(const float* q, const float* k, const float* v, long B
 int oracle_pisa_hybrid(const float* q, const float* k, const float* v, long BH, long L, long d,
                        long B, long K, int order, int gate, const int64_t* tiles, long ntiles,
                        double* out, double* lse, int nthreads) {
-    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 1, tiles, ntiles, out, lse,
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 1, 0, tiles, ntiles, out, lse,
                                nthreads);
 }
 

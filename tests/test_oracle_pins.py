@@ -391,3 +391,56 @@ def test_hybrid_special_cases(order):
     np.testing.assert_allclose(oracle.pisa_hybrid(q, k, v, B, 16, order), torch_dense(q, k, v), rtol=0, atol=1e-12)
     if order == 0:
         np.testing.assert_array_equal(oracle.pisa_hybrid(q, k, v, B, 4, 0), oracle.pisa_attention(q, k, v, B, 4, 0))
+
+
+# ----------------------------------------------------------------------------
+# PWT's diagonal + pooled second-order correction ("Sparse Linear Attention"
+# blog, PWT section): w_ij = 1/2 sum_c mean_{t in tile i}(q_tc^2) sigma^2_jc
+# ----------------------------------------------------------------------------
+
+def test_pooled_w_equals_exact_w_for_constant_tile_queries_and_diagonal_covariance():
+    # Keys that vary in one channel only make C_j diagonal; queries that are the
+    # same on every row of a tile make mean(q^2) = q^2.  Then the pooled
+    # diagonal estimate equals the exact 1/2 q^T C_j q.
+    rng = np.random.default_rng(22)
+    B, d, nblk = 16, 8, 8
+    L = B * nblk
+    k = np.repeat(rng.standard_normal((1, nblk, 1, d)), B, axis=2).astype(np.float32)
+    k[..., 0] += (rng.integers(-4, 5, (1, nblk, B)) / 4.0).astype(np.float32)
+    k = k.reshape(1, L, d)
+    q = np.repeat((rng.standard_normal((1, nblk, 1, d)) * 0.4).astype(np.float32), B, axis=2).reshape(1, L, d)
+    v = rng.standard_normal((1, L, d)).astype(np.float32)
+    for gate in (True, False):
+        e = oracle.pisa_attention_ex(q, k, v, B, 2, 2, gate=gate)
+        p = oracle.pisa_attention_ex(q, k, v, B, 2, 2, gate=gate, w_pooled=True)
+        np.testing.assert_allclose(p, e, rtol=0, atol=1e-12)
+
+
+def test_pooled_w_closed_form_and_square_before_mean():
+    # One block (K = 0): log D_t = log B + q_t . kbar + w with one w for the tile,
+    # w = 1/2 sum_c mean_t(q_tc^2) var_c(k).  Rows +a and -a have mean q = 0, so a
+    # "square of the mean" pooling would give w = 0; the blog's pooling does not.
+    rng = np.random.default_rng(23)
+    B, d = 16, 8
+    k = (rng.integers(-8, 9, (1, B, d)) / 8.0).astype(np.float32)
+    a = (rng.integers(-4, 5, d) / 16.0).astype(np.float32)
+    q = np.concatenate([np.tile(a, (B // 2, 1)), np.tile(-a, (B // 2, 1))])[None].astype(np.float32)
+    v = rng.standard_normal((1, B, d)).astype(np.float32)
+    _, lse = oracle.pisa_attention_ex(q, k, v, B, 0, 2, gate=False, w_pooled=True, want_lse=True)
+    k64 = k[0].astype(np.float64)
+    var = ((k64 - k64.mean(axis=0)) ** 2).mean(axis=0)
+    q64 = q[0].astype(np.float64)
+    w = 0.5 * ((q64 ** 2).mean(axis=0) * var).sum()
+    assert w > 0
+    np.testing.assert_allclose(lse[0], np.log(B) + q64 @ k64.mean(axis=0) + w, rtol=0, atol=1e-12)
+
+
+def test_pooled_w_gate_and_other_orders():
+    q, k, v = small(24, L=128, d=8, scale=1.0)
+    B = 16
+    k40 = k * np.float32(40.0)  # every pooled w exceeds ln B: the gate gives order 1 back
+    np.testing.assert_array_equal(oracle.pisa_attention_ex(q, k40, v, B, 2, 2, w_pooled=True),
+                                  oracle.pisa_attention(q, k40, v, B, 2, 1))
+    # the pooled flag changes nothing below order 2
+    np.testing.assert_array_equal(oracle.pisa_attention_ex(q, k, v, B, 2, 1, w_pooled=True),
+                                  oracle.pisa_attention(q, k, v, B, 2, 1))
