@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libpisa_b200.so")
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
 PISA_F32, PISA_BF16 = 0, 1
 PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2, "hybrid_tc": 3}
+FLAG_GATE_W, FLAG_POOLED_W = 1, 2
 PATH_NAMES = {v: k for k, v in PATHS.items()}
 
 
@@ -236,8 +237,10 @@ def pisa_resolve_path(batch, heads, L, d, B, K, order, dtype: torch.dtype) -> st
 
 def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
                    gate: bool = True, path: str = "auto", out: Optional[torch.Tensor] = None,
-                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Piecewise sparse attention forward; returns ``out`` (same shape and dtype as q)."""
+                   workspace: Optional[torch.Tensor] = None, stream=None, w_mode: str = "exact") -> torch.Tensor:
+    """Piecewise sparse attention forward; returns ``out`` (same shape and dtype as q).
+    ``w_mode`` ("exact" or "pooled") picks the order-2 correction: the exact
+    1/2 q^T C_j q, or PWT's diagonal + pooled [query tile x block] estimate."""
     _need_cuda(q, k, v)
     if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k, v must share shape and dtype")
@@ -253,7 +256,8 @@ def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K:
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     _check(lib().pisa_attention_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d, code, B, K,
-                                   order, int(bool(gate)), PATHS[path], out.data_ptr(), workspace.data_ptr(),
+                                   order, (FLAG_GATE_W if gate else 0) | (FLAG_POOLED_W if w_mode == "pooled" else 0),
+                                   PATHS[path], out.data_ptr(), workspace.data_ptr(),
                                    workspace.numel(), _stream(stream)))
     return out
 

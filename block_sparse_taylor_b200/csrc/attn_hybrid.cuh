@@ -66,7 +66,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
                        const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_hb,
                        const uint32_t* __restrict__ mask, bf16* __restrict__ out, int L, int nblk, int words,
-                       unsigned* status) {
+                       const float* __restrict__ wmat, unsigned* status) {
+    // ORDER: 0 zeroth, 1 first (H-bar), 3 first + the pooled diagonal second-order
+    // term of wmat ([BH, nblk, nblk], row = query tile, gated) on every virtual token
     using C = HybCfg<D, BS>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool valid = qrow < L;
         const int tq = (h * C::MQ + r) / BS;  // query tile of this row inside the CTA (0 .. NQT-1)
         const uint32_t* myw = qwords + tq * 128;
+        const float* wrow = (ORDER == 3) ? wmat + ((size_t)bh * nblk + min(qt0 + tq, nblk - 1)) * nblk : nullptr;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t s_addr = lane_base + (uint32_t)(h * 128);
         const uint32_t o_addr = lane_base + C::O_COL0 + h * D;
@@ -339,7 +342,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int e = 0; e < BS; ++e) s4[e & 3] += __uint_as_float(x[e]);
-                        l2[b] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs * LOG2E;
+                        float wv = 0.f;
+                        if (ORDER == 3) wv = __ldg(wrow + blk);
+                        l2[b] = (((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs + wv) * LOG2E;
                         mc = fmaxf(mc, l2[b]);
                     }
                 }
@@ -353,6 +358,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     uint32_t inb = 0u;
                     if (j < nblk) inb = (nblk - j >= 32) ? 0xffffffffu : ((1u << (nblk - j)) - 1u);
                     okw[w] = inb & ~((j >> 5) < words ? uwords[j >> 5] : 0u);
+                }
+                if (ORDER == 3) {
+                    // the virtual token's logit carries the tile's pooled w (in place)
+#pragma unroll
+                    for (int e = 0; e < C::NK; ++e)
+                        if ((okw[e >> 5] >> (e & 31)) & 1u)
+                            sv[e] = __float_as_uint(__uint_as_float(sv[e]) + __ldg(wrow + vj0 + e));
                 }
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -482,10 +494,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // Host: tensor maps and launch of the hybrid kernel.  kbar_bf, vsum_bf: [BH, nblk, d] bf16;
 // hbar_bf: [BH, d, d] bf16 (row = value channel).  Requires L % 128 == 0 (checked by the caller).
+// order 3 = first order + the pooled w matrix `wmat` (the hybrid's second order).
 inline pisa_status run_attn_hybrid(const void* q, const void* k, const void* v, const void* kbar_bf,
                                    const void* vsum_bf, const void* hbar_bf, const uint32_t* mask, void* out,
-                                   long BH, int L, int d, int B, int nblk, int words, int order, unsigned* status,
-                                   cudaStream_t s, std::string* err) {
+                                   long BH, int L, int d, int B, int nblk, int words, int order, const float* wmat,
+                                   unsigned* status, cudaStream_t s, std::string* err) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
@@ -520,19 +533,23 @@ inline pisa_status run_attn_hybrid(const void* q, const void* k, const void* v, 
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HybCfg<DD, BB>::SMEM); \
         if (e == cudaSuccess) {                                                                                 \
             kern<<<grid, kTcThreads, HybCfg<DD, BB>::SMEM, s>>>(mq, mk, mv, mkb, mvs, mhb, mask, (bf16*)out, L,   \
-                                                                nblk, words, status);                           \
+                                                                nblk, words, wmat, status);                     \
             e = cudaGetLastError();                                                                             \
         }                                                                                                       \
     } else
     PISA_HYB_LAUNCH(64, 64, 0)
     PISA_HYB_LAUNCH(64, 64, 1)
+    PISA_HYB_LAUNCH(64, 64, 3)
     PISA_HYB_LAUNCH(64, 128, 0)
     PISA_HYB_LAUNCH(64, 128, 1)
+    PISA_HYB_LAUNCH(64, 128, 3)
     PISA_HYB_LAUNCH(128, 64, 0)
     PISA_HYB_LAUNCH(128, 64, 1)
+    PISA_HYB_LAUNCH(128, 64, 3)
     PISA_HYB_LAUNCH(128, 128, 0)
-    PISA_HYB_LAUNCH(128, 128, 1) {
-        *err = "no hybrid kernel for this d/B/order (orders 0 and 1)";
+    PISA_HYB_LAUNCH(128, 128, 1)
+    PISA_HYB_LAUNCH(128, 128, 3) {
+        *err = "no hybrid kernel for this d/B/order";
         return PISA_ERR_UNSUPPORTED;
     }
 #undef PISA_HYB_LAUNCH

@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const float* __restrict__ kbar, const float* __restrict__ vsum, const T* __restrict__ hstat,
     const T* __restrict__ cov, const uint32_t* __restrict__ mask, T* __restrict__ out, int L, int nblk,
-    int words, int order, int gate, float ln_b) {
+    int words, int order, int gate, float ln_b, const float* __restrict__ wmat) {
+    // wmat (order 2, optional): PWT's pooled diagonal w per (query tile, block), gated
     using SM = AttnStatsSmem<T, D, BS>;
     constexpr int QS = SM::QS, XS = SM::XS, W = D / 32;
     extern __shared__ __align__(16) float sm_attn[];
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
                 const T* hj = hstat + so * D;
                 for (int e = tid; e < D * D; e += 256) st0[(e / D) * XS + e % D] = hj[e];
             }
-            if (order == 2) {
+            if (order == 2 && !wmat) {
                 const T* cj = cov + so * D;
                 for (int e = tid; e < D * D; e += 256) st1[(e / D) * XS + e % D] = cj[e];
             }
@@ -137,7 +138,9 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
                 for (int w = 0; w < W; ++w) s = fmaf(qr[lane + 32 * w], aux[lane + 32 * w], s);
                 s = warp_sum(s);
                 float wq = 0.f;
-                if (order == 2) {
+                if (order == 2 && wmat) {
+                    wq = wmat[((size_t)bh * nblk + i) * nblk + j];
+                } else if (order == 2) {
                     float part = 0.f;
 #pragma unroll
                     for (int w = 0; w < W; ++w) {

@@ -65,7 +65,10 @@ template <int D, int BS, int ORDER>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ mask, bf16* __restrict__ out,
-                   int L, int nblk, int words, int gate, float ln_b, unsigned* status) {
+                   int L, int nblk, int words, int gate, float ln_b, const float* __restrict__ wmat,
+                   unsigned* status) {
+    // ORDER: 0 zeroth, 1 first, 2 first + exact w from the logits, 3 first + the
+    // pooled diagonal w of wmat ([BH, nblk, nblk], row = query tile, already gated)
     using C = TcCfg<D>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, N = 128 keys
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool valid = qrow < L;
         int qt = (qrow < L ? qrow : L - 1) / BS;  // query tile (selection row)
         const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
+        const float* wrow = (ORDER == 3) ? wmat + ((size_t)bh * nblk + qt) * nblk : nullptr;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t s_addr = lane_base + (uint32_t)(h * 128);
         const uint32_t o_addr = lane_base + C::O_COL0 + h * D;
@@ -286,6 +290,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const float sq = (q4[0] + q4[1]) + (q4[2] + q4[3]);
                         w = 0.5f * fmaf(-sb, sb, sq * inv_bs);
                         if (gate && w > ln_b) w = 0.f;
+                    } else if (ORDER == 3) {
+                        w = __ldg(wrow + jt * BPT + b);
                     }
                     sbar[b] = sb;
                     l2[b] = (sb + w) * LOG2E;
@@ -402,9 +408,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 inline bool attn_tc_supported(int d, int B) { return (d == 64 || d == 128) && (B == 64 || B == 128); }
 
 // Host: build the tensor maps and launch.  Requires L % 128 == 0 (checked).
+// order 3 = order 2 with the pooled w matrix `wmat` ([BH, nblk, nblk] fp32, gated).
 inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, const uint32_t* mask, void* out, long BH,
-                               int L, int d, int B, int nblk, int words, int order, int gate, unsigned* status,
-                               cudaStream_t s, std::string* err) {
+                               int L, int d, int B, int nblk, int words, int order, int gate, const float* wmat,
+                               unsigned* status, cudaStream_t s, std::string* err) {
     if (L % 128) {
         *err = "tensor-core path needs L % 128 == 0";
         return PISA_ERR_UNSUPPORTED;
@@ -447,22 +454,26 @@ inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, cons
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcCfg<DD>::SMEM);     \
         if (e == cudaSuccess) {                                                                                \
             kern<<<grid, kTcThreads, TcCfg<DD>::SMEM, s>>>(maps[0], maps[1], maps[2], mask, (bf16*)out, L, nblk, \
-                                                           words, gate, ln_b, status);                         \
+                                                           words, gate, ln_b, wmat, status);                   \
             e = cudaGetLastError();                                                                            \
         }                                                                                                      \
     } else
     PISA_TC_LAUNCH(64, 64, 0)
     PISA_TC_LAUNCH(64, 64, 1)
     PISA_TC_LAUNCH(64, 64, 2)
+    PISA_TC_LAUNCH(64, 64, 3)
     PISA_TC_LAUNCH(64, 128, 0)
     PISA_TC_LAUNCH(64, 128, 1)
     PISA_TC_LAUNCH(64, 128, 2)
+    PISA_TC_LAUNCH(64, 128, 3)
     PISA_TC_LAUNCH(128, 64, 0)
     PISA_TC_LAUNCH(128, 64, 1)
     PISA_TC_LAUNCH(128, 64, 2)
+    PISA_TC_LAUNCH(128, 64, 3)
     PISA_TC_LAUNCH(128, 128, 0)
     PISA_TC_LAUNCH(128, 128, 1)
-    PISA_TC_LAUNCH(128, 128, 2) {
+    PISA_TC_LAUNCH(128, 128, 2)
+    PISA_TC_LAUNCH(128, 128, 3) {
         *err = "no tensor-core kernel for this d/B/order";
         return PISA_ERR_UNSUPPORTED;
     }

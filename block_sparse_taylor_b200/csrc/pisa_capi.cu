@@ -205,7 +205,7 @@ pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dty
 
 pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pisa_stats_t* st,
                            const uint32_t* mask, void* out, const Dims& g, int order, int gate,
-                           cudaStream_t s) {
+                           cudaStream_t s, const float* wmat = nullptr) {
     return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
@@ -216,8 +216,30 @@ pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pi
         dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
         kern<<<grid, 256, smem, s>>>((const T*)q, (const T*)k, (const T*)v, st->kbar, st->vsum,
                                      (const T*)st->hstat, (const T*)st->cov, mask, (T*)out, (int)g.L,
-                                     (int)g.nblk, (int)g.words, order, gate, logf((float)g.B));
+                                     (int)g.nblk, (int)g.words, order, gate, logf((float)g.B), wmat);
         return launch_check("attn_stats_kernel");
+    });
+}
+
+// PWT's cheap second-order term: per-block channel variances of k, tile means
+// of q^2, then the gated [query tile x block] matrix w.
+pisa_status run_wpool(const void* q, const void* k, const Dims& g, pisa_dtype dtype, int gate, float* var, float* q2,
+                      float* wmat, cudaStream_t s) {
+    return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const size_t smem = sizeof(T) * BS * D;
+        auto kv = pisa::colstat_kernel<T, D, BS, 1>;
+        auto kq = pisa::colstat_kernel<T, D, BS, 2>;
+        pisa_status r = set_smem(kv, smem);
+        if (r != PISA_OK) return r;
+        r = set_smem(kq, smem);
+        if (r != PISA_OK) return r;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        kv<<<grid, 128, smem, s>>>((const T*)k, var, (int)g.L, (int)g.nblk);
+        kq<<<grid, 128, smem, s>>>((const T*)q, q2, (int)g.L, (int)g.nblk);
+        pisa::wpool_kernel<D><<<grid, 256, 0, s>>>(q2, var, wmat, (int)g.nblk, gate, logf((float)g.B));
+        return launch_check("pooled-w kernels");
     });
 }
 
@@ -228,6 +250,7 @@ struct WsLayout {
     size_t stats, mask, idx, total;
     StatsLayout sl;
     size_t kbar_bf, vsum_bf, hbar_acc, hbar_bf;  // hybrid path only
+    size_t var, q2, wmat;                        // order 2: PWT's pooled w (used with the pooled flag)
 };
 
 WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path path) {
@@ -256,12 +279,21 @@ WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path 
         w.hbar_bf = o;
         o += align_up(2 * g.BH * g.d * g.d);
     }
+    if (order == 2) {
+        w.var = o;
+        o += align_up(4 * g.BH * g.nblk * g.d);
+        w.q2 = o;
+        o += align_up(4 * g.BH * g.nblk * g.d);
+        w.wmat = o;
+        o += align_up(4 * g.BH * g.nblk * g.nblk);
+    }
     w.total = o;
     return w;
 }
 
+// The hybrid supports orders 0 and 1, and order 2 in PWT's pooled form only.
 bool hybrid_path_available(const Dims& g, pisa_dtype dtype, int order) {
-    return dtype == PISA_BF16 && pisa::attn_tc_supported((int)g.d, (int)g.B) && g.L % 128 == 0 && order <= 1 &&
+    return dtype == PISA_BF16 && pisa::attn_tc_supported((int)g.d, (int)g.B) && g.L % 128 == 0 && order <= 2 &&
            g.BH * g.L <= 0x7fffffffL;
 }
 
@@ -387,7 +419,11 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype))
         return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
     if (path == PISA_PATH_HYBRID_TC && !hybrid_path_available(g, dtype, order))
-        return fail(PISA_ERR_UNSUPPORTED, "hybrid path needs bf16, d and B in {64, 128}, L %% 128 == 0, order <= 1");
+        return fail(PISA_ERR_UNSUPPORTED, "hybrid path needs bf16, d and B in {64, 128}, L %% 128 == 0");
+    const int gate = gate_w & PISA_FLAG_GATE_W;
+    const bool pooled = (gate_w & PISA_FLAG_POOLED_W) != 0;
+    if (path == PISA_PATH_HYBRID_TC && order == 2 && !pooled)
+        return fail(PISA_ERR_UNSUPPORTED, "the hybrid's second order needs the pooled w (PISA_FLAG_POOLED_W)");
     if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC)
         return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
     const WsLayout w = ws_layout(g, K, order, dtype, path);
@@ -411,6 +447,13 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     uint32_t* mask = (uint32_t*)(ws + w.mask);
     int32_t* idx = (int32_t*)(ws + w.idx);
 
+    float* wmat = nullptr;
+    if (order == 2 && pooled) {
+        wmat = (float*)(ws + w.wmat);
+        r = run_wpool(q, k, g, dtype, gate, (float*)(ws + w.var), (float*)(ws + w.q2), wmat, s);
+        if (r != PISA_OK) return r;
+    }
+    const int korder = (order == 2 && pooled) ? 3 : order;  // kernel order code (3 = pooled w)
     if (path == PISA_PATH_HYBRID_TC) {
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
@@ -426,7 +469,7 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s);
         if (r != PISA_OK) return r;
         return pisa::run_attn_hybrid(q, k, v, kbar_bf, vsum_bf, hbf, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B,
-                                     (int)g.nblk, (int)g.words, order, status, s, &g_last_error);
+                                     (int)g.nblk, (int)g.words, korder, wmat, status, s, &g_last_error);
     }
     if (path == PISA_PATH_RECOMPUTE_TC) {
         r = run_centroids(k, st.kbar, g, dtype, s);
@@ -441,9 +484,9 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
         return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
-                                 (int)g.words, order, gate_w, status, s, &g_last_error);
+                                 (int)g.words, korder, gate, wmat, status, s, &g_last_error);
     }
-    return run_attn_stats(q, k, v, &st, mask, out, g, order, gate_w, s);
+    return run_attn_stats(q, k, v, &st, mask, out, g, order, gate, s, wmat);
 }
 
 pisa_status pisa_attention(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
@@ -475,8 +518,11 @@ pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, in
             return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        if (gate_w & PISA_FLAG_POOLED_W)
+            return fail(PISA_ERR_UNSUPPORTED, "pisa_fused_attention: the pooled w needs pisa_attention_ex");
         return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
-                                 (int)g.words, order, gate_w, status, (cudaStream_t)stream, &g_last_error);
+                                 (int)g.words, order, gate_w & PISA_FLAG_GATE_W, nullptr, status,
+                                 (cudaStream_t)stream, &g_last_error);
     }
     if (path != PISA_PATH_STATS) return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
     Dims gs;
@@ -486,7 +532,9 @@ pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, in
         return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: statistics of another shape");
     if (st->order < order) return fail(PISA_ERR_INVALID_ARG, "statistics of order %d for attention of order %d",
                                        st->order, order);
-    return run_attn_stats(q, k, v, st, mask, out, g, order, gate_w, (cudaStream_t)stream);
+    if (gate_w & PISA_FLAG_POOLED_W)
+        return fail(PISA_ERR_UNSUPPORTED, "pisa_fused_attention: the pooled w needs pisa_attention_ex");
+    return run_attn_stats(q, k, v, st, mask, out, g, order, gate_w & PISA_FLAG_GATE_W, (cudaStream_t)stream);
 }
 
 pisa_status pisa_poll_device_status(void* stream) {

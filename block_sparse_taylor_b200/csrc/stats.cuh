@@ -118,3 +118,71 @@ __global__ void __launch_bounds__(256) stats_simt_kernel(const T* __restrict__ k
 }
 
 }  // namespace pisa
+
+namespace pisa {
+
+// Column statistics of every B-row tile for PWT's cheap second-order term
+// ("Sparse Linear Attention" blog, PWT section): MODE 1 = within-block variance
+// of each channel of the keys, (1/B) sum_n (k_nc - mean_c)^2 (the diagonal of
+// C_j, two passes in fp32); MODE 2 = mean of the squared queries of a tile,
+// (1/B) sum_t q_tc^2 (square first, then average).  Same staging as the
+// centroid kernel; grid (nblk, BH), 128 threads.
+template <typename T, int D, int BS, int MODE>
+__global__ void __launch_bounds__(128) colstat_kernel(const T* __restrict__ x, float* __restrict__ out, int L,
+                                                      int nblk) {
+    extern __shared__ __align__(16) uint8_t sm_col[];
+    T* tile = reinterpret_cast<T*>(sm_col);
+    const int j = blockIdx.x, bh = blockIdx.y;
+    const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)bh * L + (size_t)j * BS) * D);
+    uint4* dst = reinterpret_cast<uint4*>(tile);
+    constexpr int NV = BS * D * (int)sizeof(T) / 16;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < NV; e += 128) dst[e] = __ldg(src + e);
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += 128) {
+        float r;
+        if (MODE == 1) {
+            float m = 0.f;
+            for (int n = 0; n < BS; ++n) m += to_f(tile[n * D + c]);
+            m *= 1.0f / (float)BS;
+            float v = 0.f;
+            for (int n = 0; n < BS; ++n) {
+                const float dv = to_f(tile[n * D + c]) - m;
+                v = fmaf(dv, dv, v);
+            }
+            r = v * (1.0f / (float)BS);
+        } else {
+            float s = 0.f;
+            for (int n = 0; n < BS; ++n) {
+                const float xv = to_f(tile[n * D + c]);
+                s = fmaf(xv, xv, s);
+            }
+            r = s * (1.0f / (float)BS);
+        }
+        out[((size_t)bh * nblk + j) * D + c] = r;
+    }
+}
+
+// The [query tile x key block] matrix of PWT's cheap second-order term:
+// w_ij = 1/2 sum_c q2_ic var_jc, set to 0 when it exceeds ln B and the gate is
+// on.  grid (nblk, BH) over query tiles i, 256 threads: one warp per block j,
+// lanes over channels.
+template <int D>
+__global__ void __launch_bounds__(256) wpool_kernel(const float* __restrict__ q2, const float* __restrict__ var,
+                                                    float* __restrict__ w, int nblk, int gate, float ln_b) {
+    __shared__ float qs[D];
+    const int i = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    for (int c = threadIdx.x; c < D; c += 256) qs[c] = q2[((size_t)bh * nblk + i) * D + c];
+    __syncthreads();
+    const float* vb = var + (size_t)bh * nblk * D;
+    float* wrow = w + ((size_t)bh * nblk + i) * nblk;
+    for (int j = warp; j < nblk; j += 8) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = lane; c < D; c += 32) s = fmaf(qs[c], vb[(size_t)j * D + c], s);
+        s = 0.5f * warp_sum(s);
+        if (lane == 0) wrow[j] = (gate && s > ln_b) ? 0.f : s;
+    }
+}
+
+}  // namespace pisa

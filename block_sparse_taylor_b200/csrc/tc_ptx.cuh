@@ -40,6 +40,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0u;
 }
 
+// try_wait with a suspend-time hint (ns): the waiting thread is parked until the
+// phase completes or the hint expires, so that it does not take issue slots
+// from the warps doing work on its SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0u;
+}
+
 // Bounded wait: gives up after `limit` clock cycles, records the timeout in the
 // device status word and sets `aborted`; every later wait of an aborted thread
 // returns false at once so that the CTA drains and exits.
@@ -49,7 +64,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool& a
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity)) return true;
         if (clock64() - t0 > limit) {
             atomicOr(status, kStatusTimeout);
             aborted = true;

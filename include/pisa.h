@@ -84,7 +84,8 @@ typedef enum {
  * head), so the numerator's first-order part is (sum_{j in U_i} e^{l_tj})
  * H-bar q_t (PISA paper section 3.3 and Figure 3, phase 3; H-bar as in the
  * "Sparse Linear Attention" blog).  Unselected blocks cost one virtual token
- * each instead of their tokens.  bf16, order 0 or 1, L % 128 == 0. */
+ * each instead of their tokens.  bf16, L % 128 == 0; order 2 only with the
+ * pooled w (PISA_FLAG_POOLED_W). */
 
 /* Block statistics of one call (all device pointers, caller-owned).
  *   kbar  [BH, nblk, d] fp32 : centroid, canonical fp32 mean (see pisa_select)
@@ -166,8 +167,17 @@ pisa_status pisa_attention(const void* q, const void* k, const void* v, int batc
                            int L, int d, pisa_dtype dtype, int B, int K, int order, void* out,
                            void* workspace, size_t ws_bytes, void* stream);
 
-/* As pisa_attention with the PWT gate switchable (gate_w = 0: w is never
- * zeroed) and an explicit path. */
+/* Bits of the gate_w argument of pisa_attention_ex and pisa_fused_attention. */
+#define PISA_FLAG_GATE_W 1   /* zero w when it exceeds ln B (pisa_attention sets it) */
+#define PISA_FLAG_POOLED_W 2 /* order 2: PWT's cheap form of w ("Sparse Linear Attention"
+                              * blog, PWT section): w_ij = 1/2 sum_c mean_{t in tile i}(q_tc^2)
+                              * var_c(keys of block j), one value per (query tile, block),
+                              * instead of the exact per-query 1/2 q^T C_j q.  Required
+                              * for order 2 on the hybrid path; pisa_attention_ex only. */
+
+/* As pisa_attention with the PWT options as flags (gate_w: PISA_FLAG_GATE_W,
+ * PISA_FLAG_POOLED_W; 0 = exact w, never zeroed) and an explicit path.  The
+ * workspace of an order-2 call also holds the pooled-w arrays. */
 pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads,
                               int L, int d, pisa_dtype dtype, int B, int K, int order, int gate_w,
                               pisa_path path, void* out, void* workspace, size_t ws_bytes,

@@ -287,3 +287,49 @@ def test_hybrid_full_size_sampled(name, per_head, nheads):
     ref = oracle.pisa_hybrid(q, k, v, w.B, w.K, 1, tiles=tiles)
     err = rel_l2(rows_of(got, tiles, w.B), ref)
     assert err <= TOL[w.dtype], (name, err)
+
+
+# ---------------------------------------------------------------------------
+# PWT's diagonal + pooled w (order 2, PISA_FLAG_POOLED_W)
+# ---------------------------------------------------------------------------
+
+def run_attn_w(q, k, v, B, K, order, dt, path, w_mode, gate=True):
+    out = pisa.pisa_attention(dev(q, dt), dev(k, dt), dev(v, dt), B, K, order, gate=gate, path=path, w_mode=w_mode)
+    pisa.pisa_poll_device_status()
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("path", ["recompute_tc", "stats", "hybrid_tc"])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (128, 128)])
+@pytest.mark.parametrize("gate", [True, False])
+def test_pooled_w_small(path, d, B, gate):
+    L = 2048
+    K = (L // B) // 4
+    q, k, v = pisa_synth.random_qkv(900 + d + B, 2, L, d, scale=2.0, dtype="bf16")
+    got = run_attn_w(q, k, v, B, K, 2, "bf16", path, "pooled", gate)
+    ref = oracle.pisa_attention_ex(q, k, v, B, K, 2, gate=gate, hybrid=(path == "hybrid_tc"), w_pooled=True)
+    err = rel_l2(got, ref)
+    assert err <= TOL["bf16"], err
+    assert err <= 5e-3, err
+
+
+def test_pooled_w_fp32_statistics_path():
+    q, k, v = pisa_synth.random_qkv(950, 2, 1024, 64, scale=2.0, dtype="f32")
+    got = run_attn_w(q, k, v, 64, 4, 2, "f32", "stats", "pooled")
+    ref = oracle.pisa_attention_ex(q, k, v, 64, 4, 2, w_pooled=True)
+    assert rel_l2(got, ref) <= TOL["f32"]
+
+
+def test_hybrid_order2_needs_pooled_w():
+    q, k, v = pisa_synth.random_qkv(951, 1, 1024, 64, dtype="bf16")
+    with pytest.raises(pisa.PisaError):
+        run_attn_w(q, k, v, 64, 4, 2, "bf16", "hybrid_tc", "exact")
+
+
+@pytest.mark.parametrize("path", ["recompute_tc", "hybrid_tc"])
+def test_pooled_w_full_size_c2(path):
+    w, (q, k, v) = workload("c2o2")
+    got = run_attn_w(q, k, v, w.B, w.K, 2, w.dtype, path, "pooled")
+    tiles = sample_tiles(w.BH, w.nblk, 4, seed=17, heads=[0, 5, 11])
+    ref = oracle.pisa_attention_ex(q, k, v, w.B, w.K, 2, hybrid=(path == "hybrid_tc"), w_pooled=True, tiles=tiles)
+    assert rel_l2(rows_of(got, tiles, w.B), ref) <= TOL[w.dtype]
