@@ -399,23 +399,23 @@ def main():
                       "speedup_vs_per_block_path": ms_step / h_ms, "launches_per_call": 5}
         del hws, hout
 
-    # end to end through the public call with host buffers: pinned H2D, pisa_attention, D2H
+    # end to end through the public host-buffer call: pisa_attention_host on
+    # pinned host q, k, v, out (per chunk of heads: H2D copies, the attention,
+    # D2H copy; two streams so that the copies overlap the kernels)
     e2e = None
     if not args.no_e2e:
         hq = q.cpu().pin_memory()
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
         ho = torch.empty_like(hq).pin_memory()
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        ws = torch.empty(pisa.pisa_workspace_bytes(1, BH, L, d, B, K, order, tdt), dtype=torch.uint8,
-                         device="cuda")
+        plan = pisa.HostPlan(hq, B, K, order, chunk_heads=max(1, BH // 8))
 
         def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            pisa.pisa_attention(dq, dk, dv, B, K, order, out=out, workspace=ws)
-            ho.copy_(out, non_blocking=True)
+            for st_ in plan.streams:
+                st_.wait_stream(stream)
+            pisa.pisa_attention_host(hq, hk, hv, ho, plan)
+            for st_ in plan.streams:
+                stream.wait_stream(st_)
 
         for _ in range(max(1, args.warmup)):
             e2e_step()
@@ -431,8 +431,10 @@ def main():
         e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world)
         e2e = {"value": dense_flops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
-               "d2h_bytes_per_step": out.numel() * out.element_size()}
+               "d2h_bytes_per_step": out.numel() * out.element_size(),
+               "call": f"pisa_attention_host, {plan.chunk} heads per chunk, two streams"}
         pisa.pisa_poll_device_status()
+        del plan
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

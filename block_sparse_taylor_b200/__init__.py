@@ -85,6 +85,10 @@ def lib():
         L.pisa_fused_attention.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, ctypes.POINTER(_StatsT),
                                            vp, vp]
         L.pisa_attention_noalloc.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp]
+        L.pisa_attention_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, i, vp, sz, vp, vp]
+        L.pisa_attention_host.restype = ctypes.c_int
+        L.pisa_attention_host_bytes.argtypes = [i, i, i, i, i, i, i, i, i, i]
+        L.pisa_attention_host_bytes.restype = sz
         L.pisa_noalloc_scratch_bytes.restype = sz
         for fn in ("pisa_attention_noalloc", "pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
                    "pisa_poll_device_status", "pisa_resolve_path"):
@@ -275,6 +279,37 @@ def pisa_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B:
     _check(lib().pisa_attention_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d,
                                         _dtype_code(q.dtype), B, K, order, out.data_ptr(), _stream(stream)))
     return out
+
+
+class HostPlan:
+    """Device staging and streams for pisa_attention_host (allocated once)."""
+
+    def __init__(self, q: torch.Tensor, B: int, K: int, order: int = 1, path: str = "auto", chunk_heads: int = 4,
+                 device: Optional[torch.device] = None):
+        batch, heads, L, d = _shape(q)
+        self.args = (batch, heads, L, d, _dtype_code(q.dtype), B, K, order)
+        self.path, self.chunk = path, chunk_heads
+        nbytes = int(lib().pisa_attention_host_bytes(batch, heads, L, d, _dtype_code(q.dtype), B, K, order,
+                                                     PATHS[path], chunk_heads))
+        if nbytes == 0:
+            raise PisaError(PISA_ERR_INVALID_ARG, "no host plan for these arguments")
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+
+
+def pisa_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, plan: HostPlan,
+                        gate: bool = True, w_mode: str = "exact"):
+    """pisa_attention on pinned host tensors (q, k, v, out on the CPU); the work
+    is queued on the plan's two streams, which the caller synchronises."""
+    for t in (q, k, v, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("pisa_attention_host takes contiguous host tensors")
+    batch, heads, L, d, code, B, K, order = plan.args
+    flags = (FLAG_GATE_W if gate else 0) | (FLAG_POOLED_W if w_mode == "pooled" else 0)
+    _check(lib().pisa_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), batch, heads, L, d,
+                                     code, B, K, order, flags, PATHS[plan.path], plan.chunk, plan.buf.data_ptr(),
+                                     plan.buf.numel(), plan.streams[0].cuda_stream, plan.streams[1].cuda_stream))
 
 
 def pisa_poll_device_status(stream=None):

@@ -624,3 +624,80 @@ extern "C" pisa_status pisa_attention_noalloc(const void* q, const void* k, cons
 }
 
 extern "C" size_t pisa_noalloc_scratch_bytes(void) { return kNoallocScratchBytes; }
+
+// ---------------------------------------------------------------------------
+// Host-resident inputs: chunked, double-buffered pisa_attention_ex.
+// (batch, head) units are independent, so the heads are cut into chunks and
+// chunk c runs on stream c % 2: copy in, attention, copy out.  Copies of one
+// chunk overlap the attention of the other on the copy engines.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct HostSlot {
+    char *q, *k, *v, *o, *ws;
+};
+
+size_t host_slot_bytes(long chunk, int L, int d, int B, int K, int order, pisa_dtype dtype, pisa_path path) {
+    const size_t t = align_up((size_t)chunk * L * d * esize(dtype));
+    const size_t ws = pisa_workspace_bytes_ex(1, (int)chunk, L, d, B, K, order, dtype, path);
+    if (!ws) return 0;
+    return 4 * t + align_up(ws);
+}
+
+}  // namespace
+
+extern "C" size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K,
+                                            int order, pisa_path path, int chunk_heads) {
+    if (batch <= 0 || heads <= 0 || chunk_heads <= 0) return 0;
+    const long BH = (long)batch * heads;
+    const long chunk = chunk_heads < BH ? chunk_heads : BH;
+    const size_t slot = host_slot_bytes(chunk, L, d, B, K, order, dtype, path);
+    return slot ? 2 * slot : 0;
+}
+
+extern "C" pisa_status pisa_attention_host(const void* q_host, const void* k_host, const void* v_host,
+                                           void* out_host, int batch, int heads, int L, int d, pisa_dtype dtype,
+                                           int B, int K, int order, int gate_w, pisa_path path, int chunk_heads,
+                                           void* device_buf, size_t device_bytes, void* stream0, void* stream1) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!q_host || !k_host || !v_host || !out_host || !device_buf)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_host: null pointer");
+    if (chunk_heads <= 0) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_host: chunk_heads must be positive");
+    if ((uintptr_t)device_buf % kAlign)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_host: device_buf must be 256-byte aligned");
+    if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
+    const long chunk = chunk_heads < g.BH ? chunk_heads : g.BH;
+    const size_t slot = host_slot_bytes(chunk, L, d, B, K, order, dtype, path);
+    if (!slot) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_host: no path for these arguments");
+    if (device_bytes < 2 * slot)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_host: device_buf of %zu bytes, need %zu", device_bytes,
+                    2 * slot);
+    const size_t t = align_up((size_t)chunk * L * d * esize(dtype));
+    HostSlot sl[2];
+    for (int i = 0; i < 2; ++i) {
+        char* b = (char*)device_buf + i * slot;
+        sl[i] = HostSlot{b, b + t, b + 2 * t, b + 3 * t, b + 4 * t};
+    }
+    cudaStream_t st[2] = {(cudaStream_t)stream0, (cudaStream_t)stream1};
+    const size_t head_bytes = (size_t)L * d * esize(dtype);
+    int c = 0;
+    for (long h0 = 0; h0 < g.BH; h0 += chunk, ++c) {
+        const long nh = (g.BH - h0) < chunk ? (g.BH - h0) : chunk;
+        const HostSlot& s = sl[c & 1];
+        cudaStream_t sm = st[c & 1];
+        const size_t off = (size_t)h0 * head_bytes, nb = (size_t)nh * head_bytes;
+        cudaError_t e;
+        if ((e = cudaMemcpyAsync(s.q, (const char*)q_host + off, nb, cudaMemcpyHostToDevice, sm)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(s.k, (const char*)k_host + off, nb, cudaMemcpyHostToDevice, sm)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(s.v, (const char*)v_host + off, nb, cudaMemcpyHostToDevice, sm)) != cudaSuccess)
+            return cuda_fail(e, "pisa_attention_host: cudaMemcpyAsync (in)");
+        r = pisa_attention_ex(s.q, s.k, s.v, 1, (int)nh, L, d, dtype, B, K, order, gate_w, path, s.o, s.ws,
+                              slot - 4 * t, sm);
+        if (r != PISA_OK) return r;
+        if ((e = cudaMemcpyAsync((char*)out_host + off, s.o, nb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess)
+            return cuda_fail(e, "pisa_attention_host: cudaMemcpyAsync (out)");
+    }
+    return PISA_OK;
+}

@@ -207,6 +207,23 @@ pisa_status pisa_attention_noalloc(const void* q, const void* k, const void* v, 
 /* Size in bytes of the scratch array pisa_attention_noalloc uses. */
 size_t pisa_noalloc_scratch_bytes(void);
 
+/* Inputs and output in HOST memory (pinned, for the copies to overlap):
+ * pisa_attention_ex over chunks of chunk_heads (batch, head) units, alternating
+ * between stream0 and stream1; each chunk is copied in, computed and copied
+ * back on its stream, so the copies of one chunk overlap the attention of the
+ * other.  device_buf (256-byte aligned, pisa_attention_host_bytes(...) bytes,
+ * caller-owned) holds two chunks of q, k, v, out and their workspaces.
+ * Asynchronous: the result is in out_host once both streams have completed.
+ * The operation is the same as pisa_attention_ex's (heads are independent). */
+pisa_status pisa_attention_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                                int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
+                                int gate_w, pisa_path path, int chunk_heads, void* device_buf,
+                                size_t device_bytes, void* stream0, void* stream1);
+
+/* Bytes of device_buf pisa_attention_host needs (0 for invalid arguments). */
+size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
+                                 pisa_path path, int chunk_heads);
+
 /* The path AUTO resolves to for these arguments (or -1 if none can run). */
 int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order,
                       pisa_dtype dtype);

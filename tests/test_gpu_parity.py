@@ -333,3 +333,18 @@ def test_pooled_w_full_size_c2(path):
     tiles = sample_tiles(w.BH, w.nblk, 4, seed=17, heads=[0, 5, 11])
     ref = oracle.pisa_attention_ex(q, k, v, w.B, w.K, 2, hybrid=(path == "hybrid_tc"), w_pooled=True, tiles=tiles)
     assert rel_l2(rows_of(got, tiles, w.B), ref) <= TOL[w.dtype]
+
+
+def test_host_entry_point_matches_device_call():
+    # pisa_attention_host runs pisa_attention_ex per chunk of heads from pinned
+    # host memory; heads are independent, so the result equals the device call.
+    q, k, v = pisa_synth.random_qkv(990, 7, 2048, 128, scale=2.0, dtype="bf16")
+    qt, kt, vt = (torch.from_numpy(x).to(torch.bfloat16) for x in (q, k, v))
+    ref = pisa.pisa_attention(qt.cuda(), kt.cuda(), vt.cuda(), 64, 6, 1).cpu()
+    hq, hk, hv = (x.pin_memory() for x in (qt, kt, vt))
+    ho = torch.empty_like(hq).pin_memory()
+    plan = pisa.HostPlan(hq, 64, 6, 1, chunk_heads=3)  # 3 + 3 + 1: a ragged last chunk
+    pisa.pisa_attention_host(hq, hk, hv, ho, plan)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    assert torch.equal(ho, ref)
