@@ -26,6 +26,10 @@
 // first half of its S columns and the PV MMA reads it from TMEM as operand A.
 // MMA order per key tile jt: PV0(jt), S0(jt+1), PV1(jt), S1(jt+1), so each
 // softmax group works while the tensor core runs the other group's products.
+// P is handed over in two halves of 64 keys, each on its own barrier: the PV
+// of the first half runs while the softmax computes the second.  Every MMA has
+// N >= 128 (S: N = 128 keys; PV: N = d), the shapes at which tcgen05 with
+// M = 128 runs at its full rate; N = 64 takes as long as N = 128.
 // The running max is raised only when it grows by more than 2^8 (the output is
 // rescaled then), so most tiles need no correction of O.
 #pragma once
@@ -39,8 +43,6 @@
 
 namespace pisa {
 
-constexpr int kTcThreads = 320;
-constexpr long long kWaitLimitCycles = 2000000000ll;  // ~1 s at B200 clocks
 
 template <int D>
 struct TcCfg {
@@ -55,11 +57,107 @@ struct TcCfg {
     static constexpr uint32_t K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr uint32_t BAR_OFF = V_OFF + NS * TILE_BYTES;
-    static constexpr uint32_t NBAR = 1 + 4 * NS + 2 + 2 + 2 + 1;
+    // QFULL; KFULL, KEMPTY, VFULL, VEMPTY per stage; SFULL, PHALF, PFULL, OFULL
+    // per M tile; DONE
+    static constexpr uint32_t NBAR = 1 + 4 * NS + 2 + 2 + 2 + 2 + 1;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
     static constexpr uint32_t O_COL0 = 256;
     static constexpr uint32_t TMEM_COLS = 512;
 };
+
+// Pass 1 over the N logits of one key block (fp32 bits in x): returns the
+// block's candidate for the running max in log2 units.  Selected block: its
+// largest logit.  Unselected block: l = s-bar + w, with s-bar = mean of the
+// logits (= q.kbar_j) and w the second-order mass term (ORDER 2: from the
+// logits' spread, gated at ln B; ORDER 3: the pooled value w_pool); sbar and
+// l2 = l log2 e are returned too.  Reductions run on packed fp32 pairs in four
+// independent chains.
+template <int N, int ORDER>
+__device__ __forceinline__ float block_pass1(const uint32_t* x, bool sel, int gate, float ln_b, float w_pool,
+                                             float& sbar, float& l2) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    if (sel) {
+        float m4[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) m4[a] = fmaxf(__uint_as_float(x[2 * a]), __uint_as_float(x[2 * a + 1]));
+#pragma unroll
+        for (int e = 8; e < N; e += 8)
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                m4[a] = tc::max3(m4[a], __uint_as_float(x[e + 2 * a]), __uint_as_float(x[e + 2 * a + 1]));
+        sbar = 0.f;
+        l2 = 0.f;
+        return tc::max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * LOG2E;
+    }
+    uint64_t s2[4], q2[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        s2[a] = tc::f2_make(__uint_as_float(x[2 * a]), __uint_as_float(x[2 * a + 1]));
+        if (ORDER == 2) q2[a] = tc::f2_mul(s2[a], s2[a]);
+    }
+#pragma unroll
+    for (int e = 8; e < N; e += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const uint64_t p = tc::f2_make(__uint_as_float(x[e + 2 * a]), __uint_as_float(x[e + 2 * a + 1]));
+            s2[a] = tc::f2_add(s2[a], p);
+            if (ORDER == 2) q2[a] = tc::f2_fma(p, p, q2[a]);
+        }
+    constexpr float inv_n = 1.0f / (float)N;
+    const float2 st = tc::f2_split(tc::f2_add(tc::f2_add(s2[0], s2[1]), tc::f2_add(s2[2], s2[3])));
+    const float sb = (st.x + st.y) * inv_n;
+    float w = 0.f;
+    if (ORDER == 2) {
+        const float2 qq = tc::f2_split(tc::f2_add(tc::f2_add(q2[0], q2[1]), tc::f2_add(q2[2], q2[3])));
+        w = 0.5f * fmaf(-sb, sb, (qq.x + qq.y) * inv_n);
+        if (gate && w > ln_b) w = 0.f;
+    } else if (ORDER == 3) {
+        w = w_pool;
+    }
+    sbar = sb;
+    l2 = (sb + w) * LOG2E;
+    return l2;
+}
+
+// Pass 2 over 32 logits of one block: the bf16 weights as 16 packed pairs.
+// Selected: e^{x - m} (every fourth exponential on the FMA pipe); returns their
+// sum for the denominator.  Unselected: alpha x + c0 with alpha = e^{l - m} and
+// c0 = alpha (1 - s-bar) (ORDER >= 1), or alpha (ORDER 0); returns 0 (the
+// block's mass B alpha is added once per block by the caller).
+template <int ORDER>
+__device__ __forceinline__ float chunk_pass2(const uint32_t* x, bool sel, float m_run, float alpha, float c0,
+                                             uint32_t (&pk)[16]) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    if (sel) {
+        const uint64_t negm = tc::f2_make(-m_run, -m_run), log2e2 = tc::f2_make(LOG2E, LOG2E);
+        uint64_t d2[2] = {tc::f2_make(0.f, 0.f), tc::f2_make(0.f, 0.f)};
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 t = tc::f2_split(
+                tc::f2_fma(tc::f2_make(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), log2e2, negm));
+            const float a0 = tc::ex2(t.x);
+            const float a1 = (e & 1) ? tc::ex2_fma(t.y) : tc::ex2(t.y);
+            d2[e & 1] = tc::f2_add(d2[e & 1], tc::f2_make(a0, a1));
+            pk[e] = tc::pack_bf16x2(a0, a1);
+        }
+        const float2 dd = tc::f2_split(tc::f2_add(d2[0], d2[1]));
+        return dd.x + dd.y;
+    }
+    if (ORDER >= 1) {
+        const uint64_t al2 = tc::f2_make(alpha, alpha), c02 = tc::f2_make(c0, c0);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 wv = tc::f2_split(
+                tc::f2_fma(al2, tc::f2_make(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), c02));
+            pk[e] = tc::pack_bf16x2(wv.x, wv.y);
+        }
+    } else {
+        const uint32_t a2 = tc::pack_bf16x2(alpha, alpha);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = a2;
+    }
+    return 0.f;
+}
 
 template <int D, int BS, int ORDER>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -70,7 +168,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ORDER: 0 zeroth, 1 first, 2 first + exact w from the logits, 3 first + the
     // pooled diagonal w of wmat ([BH, nblk, nblk], row = query tile, already gated)
     using C = TcCfg<D>;
-    constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, N = 128 keys
     constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);     // O += P V, N = d, V MN-major
 
@@ -81,7 +178,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS;
-    const int B_SFULL = 1 + 4 * C::NS, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_DONE = B_OFULL + 2;
+    const int B_SFULL = 1 + 4 * C::NS, B_PHALF = B_SFULL + 2, B_PFULL = B_PHALF + 2, B_OFULL = B_PFULL + 2;
+    const int B_DONE = B_OFULL + 2;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int bh = blockIdx.y;
@@ -99,6 +197,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int h = 0; h < 2; ++h) {
             tc::mbar_init(bar(B_SFULL + h), 1);
+            tc::mbar_init(bar(B_PHALF + h), 128);
             tc::mbar_init(bar(B_PFULL + h), 128);
             tc::mbar_init(bar(B_OFULL + h), 1);
         }
@@ -175,9 +274,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                IDESC_S, kk > 0);
                 }
             };
-            auto issue_pv = [&](int h, int st, bool first) {
+            // PV over one half of the key tile (keys 64*half .. 64*half + 63)
+            auto issue_pv = [&](int h, int st, int half, bool first) {
 #pragma unroll
-                for (int kk = 0; kk < C::NK / 16; ++kk) {
+                for (int kk = half * 4; kk < half * 4 + 4; ++kk) {
                     tc::mma_ts(tmem + C::O_COL0 + h * D, tmem + (uint32_t)(h * 128) + kk * 8,
                                vdesc0 + st * kTileStep + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O, (first && kk == 0) ? 0u : 1u);
                 }
@@ -196,18 +296,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int st1 = (jt + 1) % C::NS, u1 = (jt + 1) / C::NS;
                 const bool more = jt + 1 < NT;
                 if (!tc::mbar_wait(bar(B_VFULL + st), u & 1, aborted, status, kWaitLimitCycles)) break;
+                if (!tc::mbar_wait(bar(B_PHALF + 0), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(0, st, 0, jt == 0);
                 if (!tc::mbar_wait(bar(B_PFULL + 0), jt & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_pv(0, st, jt == 0);
+                issue_pv(0, st, 1, false);
                 if (!more) tc::mma_commit(bar(B_OFULL + 0));
                 if (more) {
                     if (!tc::mbar_wait(bar(B_KFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
                     issue_s(0, st1);
                     tc::mma_commit(bar(B_SFULL + 0));
                 }
+                if (!tc::mbar_wait(bar(B_PHALF + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(1, st, 0, jt == 0);
                 if (!tc::mbar_wait(bar(B_PFULL + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_pv(1, st, jt == 0);
+                issue_pv(1, st, 1, false);
                 if (!more) tc::mma_commit(bar(B_OFULL + 1));
                 tc::mma_commit(bar(B_VEMPTY + st));
                 if (more) {
@@ -235,8 +341,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t s_addr = lane_base + (uint32_t)(h * 128);
         const uint32_t o_addr = lane_base + C::O_COL0 + h * D;
         constexpr int BPT = C::NK / BS;           // blocks per key tile
-        constexpr int CPB = BS / 32;              // 32-column chunks per block
-        const float inv_bs = 1.0f / (float)BS;
         float m_run = -INFINITY;                  // running max (log2 units)
         float dsum = 0.f;                         // denominator (scaled by 2^-m_run)
         int mword_idx = -1;                       // cached selection-mask word
@@ -246,7 +350,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!tc::mbar_wait_warp(bar(B_SFULL + h), jt & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
             bool sel[BPT];
-            float cand[BPT], sbar[BPT], l2[BPT];
+            float wp[BPT];
             if (((jt * BPT) >> 5) != mword_idx) {
                 mword_idx = (jt * BPT) >> 5;
                 mword = __ldg(mrow + mword_idx);
@@ -255,6 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int b = 0; b < BPT; ++b) {
                 const int j = jt * BPT + b;  // the BPT blocks of a tile share one mask word
                 sel[b] = (mword >> (j & 31)) & 1u;
+                wp[b] = (ORDER == 3 && !sel[b]) ? __ldg(wrow + j) : 0.f;
             }
             // the whole 128-column S tile in registers: one TMEM round trip per
             // tile, and pass 2 reuses the values
@@ -263,41 +368,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < C::NK / 32; ++c)
                 tc::tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c));
             tc::tmem_wait_ld();
-            // pass 1: per-block statistics of the logits (exact: max; Taylor:
-            // sum, and the sum of squares for order 2), four partial
-            // accumulators each so that the reductions are not one long chain
+            // pass 1: per-block statistic of the logits
+            float cand[BPT], sbar[BPT], l2[BPT];
 #pragma unroll
-            for (int b = 0; b < BPT; ++b) {
-                const uint32_t* x = sv + b * BS;
-                if (sel[b]) {
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                    for (int e = 0; e < BS; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(x[e]));
-                    cand[b] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * LOG2E;
-                    sbar[b] = 0.f;
-                    l2[b] = 0.f;
-                } else {
-                    float s4[4] = {0.f, 0.f, 0.f, 0.f}, q4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int e = 0; e < BS; ++e) {
-                        const float xe = __uint_as_float(x[e]);
-                        s4[e & 3] += xe;
-                        if (ORDER == 2) q4[e & 3] = fmaf(xe, xe, q4[e & 3]);
-                    }
-                    const float sb = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * inv_bs;
-                    float w = 0.f;
-                    if (ORDER == 2) {
-                        const float sq = (q4[0] + q4[1]) + (q4[2] + q4[3]);
-                        w = 0.5f * fmaf(-sb, sb, sq * inv_bs);
-                        if (gate && w > ln_b) w = 0.f;
-                    } else if (ORDER == 3) {
-                        w = __ldg(wrow + jt * BPT + b);
-                    }
-                    sbar[b] = sb;
-                    l2[b] = (sb + w) * LOG2E;
-                    cand[b] = l2[b];
-                }
-            }
+            for (int b = 0; b < BPT; ++b)
+                cand[b] = block_pass1<BS, ORDER>(sv + b * BS, sel[b], gate, ln_b, wp[b], sbar[b], l2[b]);
             float mc = cand[0];
 #pragma unroll
             for (int b = 1; b < BPT; ++b) mc = fmaxf(mc, cand[b]);
@@ -321,57 +396,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc::tmem_st16(o_addr + c * 16, raw);
                 }
             }
-            // pass 2: weights, written as bf16 over the S columns (32 columns
-            // -> 16 packed words per store)
+            // coefficients of the Taylor blocks and their mass B e^{l}
+            float alpha[BPT], c0[BPT];
 #pragma unroll
             for (int b = 0; b < BPT; ++b) {
-                const uint32_t* x = sv + b * BS;
-                if (sel[b]) {
-                    float d4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < CPB; ++c) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float xa = __uint_as_float(x[32 * c + 2 * e]);
-                            const float xb = __uint_as_float(x[32 * c + 2 * e + 1]);
-                            const float a0 = tc::ex2(fmaf(xa, LOG2E, -m_run));
-                            // every fourth exponential on the FMA pipe
-                            const float a1 = (e & 1) ? tc::ex2_fma(fmaf(xb, LOG2E, -m_run))
-                                                     : tc::ex2(fmaf(xb, LOG2E, -m_run));
-                            d4[e & 3] += a0 + a1;
-                            pk[e] = tc::pack_bf16x2(a0, a1);
-                        }
-                        tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
-                    }
-                    dsum += (d4[0] + d4[1]) + (d4[2] + d4[3]);
-                } else {
-                    const float alpha = tc::ex2(l2[b] - m_run);
-                    dsum = fmaf((float)BS, alpha, dsum);
-                    if (ORDER >= 1) {
-                        const float c0 = alpha * (1.0f - sbar[b]);
-#pragma unroll
-                        for (int c = 0; c < CPB; ++c) {
-                            uint32_t pk[16];
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                pk[e] = tc::pack_bf16x2(fmaf(alpha, __uint_as_float(x[32 * c + 2 * e]), c0),
-                                                        fmaf(alpha, __uint_as_float(x[32 * c + 2 * e + 1]), c0));
-                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
-                        }
-                    } else {
-                        uint32_t pk[16];
-                        const uint32_t a2 = tc::pack_bf16x2(alpha, alpha);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = a2;
-#pragma unroll
-                        for (int c = 0; c < CPB; ++c) tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
-                    }
+                alpha[b] = 0.f;
+                c0[b] = 0.f;
+                if (!sel[b]) {
+                    alpha[b] = tc::ex2(l2[b] - m_run);
+                    dsum = fmaf((float)BS, alpha[b], dsum);
+                    c0[b] = alpha[b] * (1.0f - sbar[b]);
                 }
             }
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            tc::mbar_arrive(bar(B_PFULL + h));
+            // pass 2 in two halves of 64 keys: P (bf16, 32 packed columns per
+            // half) goes over the S columns; each half is handed to the MMA
+            // warp on its own barrier, so the first half's PV runs while the
+            // second half is computed
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int col = half * 64 + c * 32;  // first key of this chunk
+                    const int b = col / BS;
+                    uint32_t pk[16];
+                    dsum += chunk_pass2<ORDER>(sv + col, sel[b], m_run, alpha[b], c0[b], pk);
+                    tc::tmem_st16(s_addr + col / 2, pk);
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar((half == 0 ? B_PHALF : B_PFULL) + h));
+            }
         }
         // epilogue: o = N / D
         if (tc::mbar_wait_warp(bar(B_OFULL + h), 0, aborted, status, kWaitLimitCycles)) {

@@ -10,6 +10,13 @@
 #include "common.cuh"
 
 namespace pisa {
+// Threads of the warp-specialised attention kernels: producer warp, MMA warp,
+// two softmax warpgroups.
+constexpr int kTcThreads = 320;
+// Upper bound of every mbarrier wait in the tensor-core kernels (~1 s at B200
+// clocks); a wait that runs out sets the status word and the CTA drains.
+constexpr long long kWaitLimitCycles = 2000000000ll;
+
 namespace tc {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -229,6 +236,39 @@ __device__ __forceinline__ float ex2_fma(float x) {
     const float f = x - (t - 12582912.0f);
     const float p = fmaf(fmaf(fmaf(0.05517139f, f, 0.24261111f), f, 0.69326103f), f, 0.99992806f);
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes of work per instruction).
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t r) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
