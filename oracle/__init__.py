@@ -31,19 +31,21 @@ def lib():
         li = ctypes.c_long
         L.oracle_block_stats.argtypes = [f32p, f32p, li, li, li, li, f64p, f64p, f64p, f64p, ctypes.c_int]
         L.oracle_select.argtypes = [f32p, f32p, li, li, li, li, li, ctypes.c_void_p, ctypes.c_void_p,
-                                    ctypes.c_void_p, ctypes.c_int]
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        L.oracle_route_bias.argtypes = [f32p, f32p, li, li, li, li, ctypes.c_float, ctypes.c_void_p, ctypes.c_int]
+        L.oracle_ln_f32.argtypes = [f32p, li, ctypes.c_void_p]
         L.oracle_pisa_attention.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_hybrid.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_attention_ex.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
-                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, li,
-                                               f64p, f64p, ctypes.c_int]
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                               ctypes.c_void_p, li, f64p, f64p, ctypes.c_int]
         L.oracle_pisa_bruteforce.argtypes = [f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
                                              ctypes.c_int, f64p, ctypes.c_int]
         L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
-        for fn in ("oracle_pisa_attention_ex", "oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
+        for fn in ("oracle_route_bias", "oracle_ln_f32", "oracle_pisa_attention_ex", "oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
                    "oracle_pisa_bruteforce", "oracle_dense_attention"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -95,17 +97,38 @@ def centroids_f32(k, B, nthreads=None):
     return out
 
 
-def select(q, k, B, K, nthreads=None, want_scores=False):
+def ln_f32(x):
+    """The reproducible fp32 natural logarithm the routing bias uses (element-wise)."""
+    x = _f32(x)
+    out = np.zeros_like(x)
+    _check(lib().oracle_ln_f32(x.ravel(), x.size, _ptr(out)), "ln_f32")
+    return out
+
+
+def route_bias(k, v, B, eps=1e-6, nthreads=None):
+    """Covariance-aware routing bias ln(||H_j||_F + eps), canonical fp32, [BH, nblk]."""
+    k, v = _f32(k), _f32(v)
+    BH, L, d = k.shape
+    out = np.zeros((BH, L // B), np.float32)
+    rc = lib().oracle_route_bias(k, v, BH, L, d, B, float(eps), _ptr(out), nthreads or default_threads())
+    _check(rc, "route_bias")
+    return out
+
+
+def select(q, k, B, K, nthreads=None, want_scores=False, bias=None):
     """Canonical fp32 selection: (idx [BH,nblk,K] int32 ascending, mask [BH,nblk,words] uint32,
-    scores [BH,nblk,nblk] float32 or None)."""
+    scores [BH,nblk,nblk] float32 or None).  With ``bias`` ([BH, nblk] fp32) every score
+    s_ij becomes s_ij + bias_j (one fp32 add) before the top-K."""
     q, k = _f32(q), _f32(k)
+    if bias is not None:
+        bias = _f32(bias)
     BH, L, d = q.shape
     nblk = L // B
     words = (nblk + 31) // 32
     idx = np.zeros((BH, nblk, K), np.int32)
     mask = np.zeros((BH, nblk, words), np.uint32)
     scores = np.zeros((BH, nblk, nblk), np.float32) if want_scores else None
-    rc = lib().oracle_select(q, k, BH, L, d, B, K, _ptr(idx), _ptr(mask), _ptr(scores),
+    rc = lib().oracle_select(q, k, BH, L, d, B, K, _ptr(idx), _ptr(mask), _ptr(scores), _ptr(bias),
                              nthreads or default_threads())
     _check(rc, "select")
     return idx, mask, scores
@@ -138,14 +161,17 @@ def pisa_hybrid(q, k, v, B, K, order=1, gate=True, tiles=None, nthreads=None, wa
     return _attention(lib().oracle_pisa_hybrid, q, k, v, B, K, order, gate, tiles, nthreads, want_lse)
 
 
-def pisa_attention_ex(q, k, v, B, K, order=1, gate=True, hybrid=False, w_pooled=False, tiles=None, nthreads=None,
-                      want_lse=False):
+def pisa_attention_ex(q, k, v, B, K, order=1, gate=True, hybrid=False, w_pooled=False, route_eps=None, tiles=None,
+                      nthreads=None, want_lse=False):
     """General form: ``hybrid`` uses the global H-bar (PISA hybrid), ``w_pooled``
-    PWT's diagonal + pooled second-order correction (order 2)."""
+    PWT's diagonal + pooled second-order correction (order 2), ``route_eps`` (a
+    positive float) the covariance-aware selection with bias ln(||H_j||_F + eps)."""
     fn = lib().oracle_pisa_attention_ex
+    reps = float(route_eps) if route_eps else 0.0
 
     def call(q_, k_, v_, BH, L, d, B_, K_, o_, g_, tl, n, out, lse, nt):
-        return fn(q_, k_, v_, BH, L, d, B_, K_, o_, g_, int(bool(hybrid)), int(bool(w_pooled)), tl, n, out, lse, nt)
+        return fn(q_, k_, v_, BH, L, d, B_, K_, o_, g_, int(bool(hybrid)), int(bool(w_pooled)), reps, tl, n, out,
+                  lse, nt)
 
     return _attention(call, q, k, v, B, K, order, gate, tiles, nthreads, want_lse)
 

@@ -64,6 +64,92 @@ float tree_sum_f32(float* a, long n) {
 
 bool is_pow2(long x) { return x > 0 && (x & (x - 1)) == 0; }
 
+// ---------------------------------------------------------------------------
+// Reproducible fp32 natural logarithm (for the routing bias, which decides the
+// block selection and so must be computed identically by every
+// implementation).  Method: x = 2^e m with m in [sqrt(1/2), sqrt(2)); then
+// ln m = 2 atanh(s) with s = (m - 1) / (m + 1), |s| <= 0.1716, from the series
+// atanh(s) = s + s^3/3 + s^5/5 + s^7/7 + s^9/9 (truncation below 2e-10
+// relative); ln x = e ln 2 + ln m.  Every step is one IEEE fp32 operation in a
+// fixed order (no FMA contraction).  Defined for finite x > 0 of normal range.
+// ---------------------------------------------------------------------------
+float ln_f32_canonical(float x) {
+    uint32_t bits;
+    std::memcpy(&bits, &x, 4);
+    int e = (int)((bits >> 23) & 0xffu) - 127;
+    uint32_t mb = (bits & 0x007fffffu) | 0x3f800000u;  // m in [1, 2)
+    float m;
+    std::memcpy(&m, &mb, 4);
+    if (m > 0x1.6a09e6p+0f) {  // fp32 sqrt(2)  // fold to [sqrt(1/2), sqrt(2)): halving is exact
+        volatile float h = m * 0.5f;
+        m = h;
+        e += 1;
+    }
+    volatile float num = m - 1.0f;  // exact (Sterbenz)
+    volatile float den = m + 1.0f;
+    volatile float sv = num / den;
+    const float s = sv;
+    volatile float s2 = s * s;
+    // Horner in s^2 on the coefficients 1/9, 1/7, 1/5, 1/3, 1 (each fp32 op rounded)
+    volatile float t = 0x1.c71c72p-4f * s2;  // fp32 1/9, 1/7, 1/5, 1/3 (round to nearest)
+    t = t + 0x1.24924ap-3f;
+    t = t * s2;
+    t = t + 0x1.99999ap-3f;
+    t = t * s2;
+    t = t + 0x1.555556p-2f;
+    t = t * s2;
+    t = t + 1.0f;
+    volatile float lnm = t * s;
+    lnm = lnm * 2.0f;
+    volatile float el = (float)e * 0x1.62e43p-1f;  // fp32 ln 2
+    volatile float r = el + lnm;
+    return r;
+}
+
+// Routing bias of one (bh) for the covariance-aware block selection ([pisa]
+// section 3.3 "Covariance-Aware Block Selection": log(M_j + eps) added to the
+// centroid score; [blog1] PWT section: log of the norm of H_j).  Canonical fp32:
+//   kbar_j[c]  = tree_sum_f32(k[jB..jB+B)[c]) * (1/B)           (the selection's means)
+//   dev[n][b]  = k_{j,n}[b] - kbar_j[b]
+//   h[a*d + b] = tree_sum_f32 over n of (v_{j,n}[a] * dev[n][b])   (H_j, value channel a)
+//   M_j        = sqrt(tree_sum_f32 over a*d+b of h^2)             (Frobenius norm)
+//   bias_j     = ln_f32_canonical(M_j + eps)
+void route_bias_one(const float* k, const float* v, long L, long d, long B, float eps, float* bias) {
+    const long nblk = L / B;
+    const float inv_b = 1.0f / (float)B;
+    std::vector<float> col(B), kb(d), dev(B * d), prod(B), h(d * d);
+    for (long j = 0; j < nblk; ++j) {
+        const float* kj = k + j * B * d;
+        const float* vj = v + j * B * d;
+        for (long c = 0; c < d; ++c) {
+            for (long n = 0; n < B; ++n) col[n] = kj[n * d + c];
+            volatile float m = tree_sum_f32(col.data(), B) * inv_b;
+            kb[c] = m;
+        }
+        for (long n = 0; n < B; ++n)
+            for (long c = 0; c < d; ++c) {
+                volatile float x = kj[n * d + c] - kb[c];
+                dev[n * d + c] = x;
+            }
+        for (long a = 0; a < d; ++a)
+            for (long b = 0; b < d; ++b) {
+                for (long n = 0; n < B; ++n) {
+                    volatile float p = vj[n * d + a] * dev[n * d + b];
+                    prod[n] = p;
+                }
+                h[a * d + b] = tree_sum_f32(prod.data(), B);
+            }
+        for (long e = 0; e < d * d; ++e) {
+            volatile float sq = h[e] * h[e];
+            h[e] = sq;
+        }
+        const float m2 = tree_sum_f32(h.data(), d * d);
+        volatile float mj = std::sqrt(m2);  // IEEE correctly rounded
+        volatile float arg = mj + eps;
+        bias[j] = ln_f32_canonical(arg);
+    }
+}
+
 // Per (bh): fp64 block statistics of the keys and values.
 //   kbar_j = (1/B) sum_n k_{j,n}                         ([blog1] notation)
 //   vsum_j = sum_n v_{j,n}                               ([pisa] Figure 3)
@@ -118,8 +204,9 @@ void block_stats_one(const float* k, const float* v, long L, long d, long B,
 //   kbar_j[c] = tree_sum_f32(k[jB..jB+B)[c]) * (1/B)      (fp32)
 //   s_ij      = tree_sum_f32(qbar_i[c] * kbar_j[c] over c) (products rounded)
 //   S_i = the K blocks first in the order (s descending, j ascending).
+//   with a routing bias (covariance-aware selection): s_ij = s_ij + bias_j (fp32).
 void select_one(const float* q, const float* k, long L, long d, long B, long K,
-                int32_t* idx, uint32_t* mask, float* scores) {
+                int32_t* idx, uint32_t* mask, float* scores, const float* bias = nullptr) {
     const long nblk = L / B;
     const long words = (nblk + 31) / 32;
     const float inv_b = 1.0f / (float)B;
@@ -144,6 +231,10 @@ void select_one(const float* q, const float* k, long L, long d, long B, long K,
                 prod[c] = p;
             }
             s[j] = tree_sum_f32(prod.data(), d);
+            if (bias) {
+                volatile float sb = s[j] + bias[j];
+                s[j] = sb;
+            }
             if (scores) scores[i * nblk + j] = s[j];
         }
         for (long j = 0; j < nblk; ++j) order[j] = j;
@@ -360,8 +451,26 @@ int oracle_centroids_f32(const float* k, long BH, long L, long d, long B, float*
     return 0;
 }
 
+// Canonical fp32 routing bias ln(||H_j||_F + eps): [BH, nblk].
+int oracle_route_bias(const float* k, const float* v, long BH, long L, long d, long B, float eps,
+                      float* bias, int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B || !(eps > 0.0f)) return -1;
+    const long nblk = L / B;
+    parallel_for(BH, nthreads, [&](long bh) {
+        route_bias_one(k + bh * L * d, v + bh * L * d, L, d, B, eps, bias + bh * nblk);
+    });
+    return 0;
+}
+
+// The reproducible fp32 logarithm, element-wise (for its pins).
+int oracle_ln_f32(const float* x, long n, float* out) {
+    for (long i = 0; i < n; ++i) out[i] = ln_f32_canonical(x[i]);
+    return 0;
+}
+
+// bias: null for the plain centroid score, else [BH, nblk] added to every score.
 int oracle_select(const float* q, const float* k, long BH, long L, long d, long B, long K,
-                  int32_t* idx, uint32_t* mask, float* scores, int nthreads) {
+                  int32_t* idx, uint32_t* mask, float* scores, const float* bias, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B) return -1;
     const long nblk = L / B;
     if (K < 0 || K > nblk) return -1;
@@ -369,7 +478,7 @@ int oracle_select(const float* q, const float* k, long BH, long L, long d, long 
     parallel_for(BH, nthreads, [&](long bh) {
         select_one(q + bh * L * d, k + bh * L * d, L, d, B, K,
                    idx ? idx + bh * nblk * K : nullptr, mask ? mask + bh * nblk * words : nullptr,
-                   scores ? scores + bh * nblk * nblk : nullptr);
+                   scores ? scores + bh * nblk * nblk : nullptr, bias ? bias + bh * nblk : nullptr);
     });
     return 0;
 }
@@ -380,8 +489,8 @@ int oracle_select(const float* q, const float* k, long BH, long L, long d, long 
 // The selection (canonical fp32) is recomputed here from q and k.
 static int pisa_attention_impl(const float* q, const float* k, const float* v, long BH, long L,
                                long d, long B, long K, int order, int gate, int global_h,
-                               int w_pooled, const int64_t* tiles, long ntiles, double* out,
-                               double* lse, int nthreads) {
+                               int w_pooled, float route_eps, const int64_t* tiles, long ntiles,
+                               double* out, double* lse, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     const long nblk = L / B;
     if (K < 0 || K > nblk) return -1;
@@ -407,7 +516,13 @@ static int pisa_attention_impl(const float* q, const float* k, const float* v, l
         block_stats_one(k + bh * L * d, v + bh * L * d, L, d, B, kbar[bh].data(), vsum[bh].data(),
                         order >= 1 ? H[bh].data() : nullptr, order == 2 ? C[bh].data() : nullptr);
         mask[bh].assign(nblk * words, 0u);
-        select_one(q + bh * L * d, k + bh * L * d, L, d, B, K, nullptr, mask[bh].data(), nullptr);
+        std::vector<float> rbias;
+        if (route_eps > 0.0f) {  // covariance-aware selection
+            rbias.assign(nblk, 0.0f);
+            route_bias_one(k + bh * L * d, v + bh * L * d, L, d, B, route_eps, rbias.data());
+        }
+        select_one(q + bh * L * d, k + bh * L * d, L, d, B, K, nullptr, mask[bh].data(), nullptr,
+                   rbias.empty() ? nullptr : rbias.data());
         if (global_h && order >= 1) {
             // H-bar = (B / L) sum over all blocks of H_j  ([blog1] "Sparse Linear Attention")
             Hbar[bh].assign(d * d, 0.0);
@@ -458,18 +573,19 @@ static int pisa_attention_impl(const float* q, const float* k, const float* v, l
 int oracle_pisa_attention(const float* q, const float* k, const float* v, long BH, long L,
                           long d, long B, long K, int order, int gate, const int64_t* tiles,
                           long ntiles, double* out, double* lse, int nthreads) {
-    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 0, 0, tiles, ntiles, out, lse,
-                               nthreads);
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 0, 0, 0.0f, tiles, ntiles, out,
+                               lse, nthreads);
 }
 
 // General form: global_h selects the PISA hybrid's H-bar, w_pooled PWT's
-// diagonal + pooled second-order correction (order 2).
+// diagonal + pooled second-order correction (order 2), route_eps > 0 the
+// covariance-aware selection with bias ln(||H_j||_F + route_eps).
 int oracle_pisa_attention_ex(const float* q, const float* k, const float* v, long BH, long L,
                              long d, long B, long K, int order, int gate, int global_h, int w_pooled,
-                             const int64_t* tiles, long ntiles, double* out, double* lse,
-                             int nthreads) {
-    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, global_h, w_pooled, tiles,
-                               ntiles, out, lse, nthreads);
+                             float route_eps, const int64_t* tiles, long ntiles, double* out,
+                             double* lse, int nthreads) {
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, global_h, w_pooled, route_eps,
+                               tiles, ntiles, out, lse, nthreads);
 }
 
 // The PISA hybrid: as oracle_pisa_attention with every H_j replaced by the
@@ -477,8 +593,8 @@ int oracle_pisa_attention_ex(const float* q, const float* k, const float* v, lon
 int oracle_pisa_hybrid(const float* q, const float* k, const float* v, long BH, long L, long d,
                        long B, long K, int order, int gate, const int64_t* tiles, long ntiles,
                        double* out, double* lse, int nthreads) {
-    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 1, 0, tiles, ntiles, out, lse,
-                               nthreads);
+    return pisa_attention_impl(q, k, v, BH, L, d, B, K, order, gate, 1, 0, 0.0f, tiles, ntiles, out,
+                               lse, nthreads);
 }
 
 // Token-wise form (no block statistics), same selection; full output [BH, L, d].

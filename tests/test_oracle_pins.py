@@ -444,3 +444,99 @@ def test_pooled_w_gate_and_other_orders():
     # the pooled flag changes nothing below order 2
     np.testing.assert_array_equal(oracle.pisa_attention_ex(q, k, v, B, 2, 1, w_pooled=True),
                                   oracle.pisa_attention(q, k, v, B, 2, 1))
+
+
+# --------------------------------------------------------------------------
+# Covariance-aware routing (PISA paper, section 3.3 "Covariance-Aware Block
+# Selection"; "Sparse Linear Attention" blog, PWT section: route by the block
+# score plus the log of the norm of H_j).  Reading: bias_j = ln(||H_j||_F + eps)
+# in a canonical fp32 procedure, added to the centroid score.
+# --------------------------------------------------------------------------
+
+
+def test_ln_f32_accuracy():
+    # error budget: the fp32 ln 2 constant and the rounding of e ln 2 (2 x 2^-24 |e ln 2|),
+    # the final add (2^-24 |ln x|), the series on [sqrt(1/2), sqrt(2)) (~1e-7 absolute)
+    rng = np.random.default_rng(31)
+    x = np.exp(rng.uniform(math.log(1e-6), math.log(1e30), 100000)).astype(np.float32)
+    x = np.concatenate([x, (1.0 + rng.uniform(-0.3, 0.3, 20000)).astype(np.float32)])
+    y = oracle.ln_f32(x).astype(np.float64)
+    ref = np.log(x.astype(np.float64))
+    assert np.all(np.abs(y - ref) <= 3 * 2.0 ** -24 * np.abs(ref) + 1.2e-7)
+
+
+def test_ln_f32_exact_points():
+    # ln 1 = 0 exactly; at x = 2^e the mantissa term vanishes and the result is fl(e * fl(ln 2))
+    assert oracle.ln_f32(np.array([1.0], np.float32))[0] == 0.0
+    es = np.arange(-19, 100, dtype=np.int64)
+    x = np.ldexp(np.ones(es.shape), es).astype(np.float32)
+    want = es.astype(np.float32) * np.float32(math.log(2.0))
+    np.testing.assert_array_equal(oracle.ln_f32(x), want)
+
+
+def test_route_bias_is_log_frobenius_norm_of_h():
+    q, k, v = small(41, L=256, d=16, scale=1.0)
+    B, eps = 16, 1e-6
+    _, _, H, _ = oracle.block_stats(k, v, B, order=1)
+    want = np.log(np.sqrt((H ** 2).sum(axis=(2, 3))) + eps)
+    got = oracle.route_bias(k, v, B, eps)
+    assert got.shape == want.shape and got.dtype == np.float32
+    np.testing.assert_allclose(got, want, rtol=0, atol=2e-5)
+
+
+def test_route_bias_of_a_constant_key_block_is_log_eps():
+    # identical keys inside a block: k - kbar = 0 exactly, H_j = 0, bias = ln(eps)
+    rng = np.random.default_rng(43)
+    B, d, nblk = 16, 8, 4
+    k = np.repeat(rng.integers(-8, 9, (1, nblk, 1, d)) / 8.0, B, axis=2).reshape(1, nblk * B, d).astype(np.float32)
+    v = rng.standard_normal((1, nblk * B, d)).astype(np.float32)
+    for eps in (1e-6, 0.5, 3.0):
+        got = oracle.route_bias(k, v, B, eps)
+        np.testing.assert_array_equal(got, np.full((1, nblk), oracle.ln_f32(np.array([eps], np.float32))[0]))
+        np.testing.assert_allclose(got, math.log(np.float32(eps)), rtol=0, atol=1e-6)
+
+
+def test_biased_selection_restated_in_numpy():
+    # the bias enters as one fp32 add after the canonical score, then the same
+    # total order (score descending, block index ascending)
+    q, k, v = small(47, L=512, d=16, scale=1.0)
+    B, K = 16, 7
+    _, _, s = oracle.select(q, k, B, K, want_scores=True)
+    bias = oracle.route_bias(k, v, B)
+    idx, mask, sb = oracle.select(q, k, B, K, want_scores=True, bias=bias)
+    s2 = (s + bias[:, None, :]).astype(np.float32)  # float32 + float32: one rounding
+    np.testing.assert_array_equal(sb, s2)
+    nblk = s.shape[-1]
+    for bh in range(s.shape[0]):
+        for i in range(nblk):
+            order = sorted(range(nblk), key=lambda j: (-float(s2[bh, i, j]), j))
+            np.testing.assert_array_equal(idx[bh, i], np.sort(order[:K]))
+
+
+def test_routing_sends_a_heterogeneous_block_to_the_exact_branch():
+    # two candidate blocks with (nearly) the same centroid score: block 1 has
+    # identical keys (Taylor is exact there, bias ln eps), block 2 spreads its keys
+    # (large H_j).  The plain score keeps block 1 (slightly higher); routing keeps block 2.
+    B, d = 16, 8
+    rng = np.random.default_rng(53)
+    base = np.zeros(d, np.float32)
+    base[0] = 1.0
+    k = np.zeros((1, 4 * B, d), np.float32)
+    k[0, 0:B] = -base                       # block 0: far away
+    k[0, B:2 * B] = base * 1.01             # block 1: identical keys, score slightly higher
+    spread = rng.choice([-2.0, 2.0], (B, d)).astype(np.float32)
+    spread -= spread.mean(axis=0)
+    k[0, 2 * B:3 * B] = base + spread       # block 2: same centroid direction, spread out
+    k[0, 3 * B:4 * B] = -2 * base           # block 3: far away
+    q = np.tile(base, (1, 4 * B, 1)).astype(np.float32)
+    v = rng.standard_normal((1, 4 * B, d)).astype(np.float32)
+    plain, _, _ = oracle.select(q, k, B, 1)
+    routed, _, _ = oracle.select(q, k, B, 1, bias=oracle.route_bias(k, v, B))
+    assert plain[0, 0, 0] == 1 and routed[0, 0, 0] == 2
+
+
+def test_routed_attention_matches_dense_when_every_block_is_selected():
+    q, k, v = small(59, L=256, d=16, scale=1.0)
+    B = 16
+    got = oracle.pisa_attention_ex(q, k, v, B, 256 // B, 1, route_eps=1e-6)
+    np.testing.assert_allclose(got, oracle.dense_attention(q, k, v), rtol=0, atol=1e-12)
