@@ -34,7 +34,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libpisa_b200.so")
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
 PISA_F32, PISA_BF16 = 0, 1
 PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2, "hybrid_tc": 3}
-FLAG_GATE_W, FLAG_POOLED_W = 1, 2
+FLAG_GATE_W, FLAG_POOLED_W, FLAG_COV_ROUTE = 1, 2, 4
+ROUTE_EPS = 1e-6
 PATH_NAMES = {v: k for k, v in PATHS.items()}
 
 
@@ -73,6 +74,9 @@ def lib():
         L.pisa_stats_bind.argtypes = [ctypes.POINTER(_StatsT), vp, sz, i, i, i, i, i, i, i]
         L.pisa_stats.argtypes = [vp, vp, ctypes.POINTER(_StatsT), vp]
         L.pisa_select.argtypes = [vp, ctypes.POINTER(_StatsT), i, vp, vp, vp]
+        L.pisa_select_biased.argtypes = [vp, ctypes.POINTER(_StatsT), i, vp, vp, vp, vp]
+        L.pisa_select_scores.argtypes = [vp, ctypes.POINTER(_StatsT), vp, vp, vp]
+        L.pisa_route_bias.argtypes = [vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, vp, vp]
         L.pisa_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
         L.pisa_workspace_bytes.restype = sz
         L.pisa_workspace_bytes_ex.argtypes = [i, i, i, i, i, i, i, i, i]
@@ -215,17 +219,55 @@ def pisa_fused_attention(q, k, v, B: int, mask: torch.Tensor, order: int = 1, ga
     return out
 
 
-def pisa_select(q: torch.Tensor, stats: Stats, K: int, stream=None):
-    """(idx [BH, nblk, K] int32 ascending, mask [BH, nblk, ceil(nblk/32)] int32 bit words)."""
+def pisa_route_bias(k: torch.Tensor, v: torch.Tensor, kbar: torch.Tensor, B: int, eps: float = ROUTE_EPS,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Covariance-aware routing bias ln(||H_j||_F + eps), [BH, nblk] fp32 (kbar: the
+    canonical centroids of pisa_centroids / pisa_stats)."""
+    _need_cuda(k, v, kbar)
+    batch, heads, L, d = _shape(k)
+    if out is None:
+        out = torch.empty((batch * heads, L // B), dtype=torch.float32, device=k.device)
+    _check(lib().pisa_route_bias(k.data_ptr(), v.data_ptr(), kbar.data_ptr(), batch, heads, L, d,
+                                 _dtype_code(k.dtype), B, float(eps), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def pisa_select(q: torch.Tensor, stats: Stats, K: int, stream=None, bias: Optional[torch.Tensor] = None):
+    """(idx [BH, nblk, K] int32 ascending, mask [BH, nblk, ceil(nblk/32)] int32 bit words).
+    With ``bias`` ([BH, nblk] fp32, e.g. pisa_route_bias) the covariance-aware selection."""
     _need_cuda(q)
     st = stats.raw
     BH = st.batch * st.heads
     words = (st.nblk + 31) // 32
     idx = torch.empty((BH, st.nblk, max(K, 0)), dtype=torch.int32, device=q.device)
     mask = torch.empty((BH, st.nblk, words), dtype=torch.int32, device=q.device)
-    _check(lib().pisa_select(q.data_ptr(), ctypes.byref(st), K, idx.data_ptr() if K > 0 else None,
-                             mask.data_ptr(), _stream(stream)))
+    if bias is None:
+        _check(lib().pisa_select(q.data_ptr(), ctypes.byref(st), K, idx.data_ptr() if K > 0 else None,
+                                 mask.data_ptr(), _stream(stream)))
+    else:
+        _need_cuda(bias)
+        _check(lib().pisa_select_biased(q.data_ptr(), ctypes.byref(st), K, bias.data_ptr(),
+                                        idx.data_ptr() if K > 0 else None, mask.data_ptr(), _stream(stream)))
     return idx, mask
+
+
+def _flags(gate: bool, w_mode: str, route: str) -> int:
+    if w_mode not in ("exact", "pooled"):
+        raise ValueError(f"w_mode must be 'exact' or 'pooled' (got {w_mode!r})")
+    if route not in ("centroid", "cov"):
+        raise ValueError(f"route must be 'centroid' or 'cov' (got {route!r})")
+    return ((FLAG_GATE_W if gate else 0) | (FLAG_POOLED_W if w_mode == "pooled" else 0)
+            | (FLAG_COV_ROUTE if route == "cov" else 0))
+
+
+def pisa_select_scores(q: torch.Tensor, stats: Stats, bias: Optional[torch.Tensor] = None, stream=None):
+    """The selection's fp32 score table [BH, nblk, nblk] (row = query tile), as the top-K sees it."""
+    _need_cuda(q)
+    st = stats.raw
+    scores = torch.empty((st.batch * st.heads, st.nblk, st.nblk), dtype=torch.float32, device=q.device)
+    _check(lib().pisa_select_scores(q.data_ptr(), ctypes.byref(st), None if bias is None else bias.data_ptr(),
+                                    scores.data_ptr(), _stream(stream)))
+    return scores
 
 
 def pisa_workspace_bytes(batch, heads, L, d, B, K, order, dtype: torch.dtype, path: str = "auto") -> int:
@@ -241,10 +283,13 @@ def pisa_resolve_path(batch, heads, L, d, B, K, order, dtype: torch.dtype) -> st
 
 def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
                    gate: bool = True, path: str = "auto", out: Optional[torch.Tensor] = None,
-                   workspace: Optional[torch.Tensor] = None, stream=None, w_mode: str = "exact") -> torch.Tensor:
+                   workspace: Optional[torch.Tensor] = None, stream=None, w_mode: str = "exact",
+                   route: str = "centroid") -> torch.Tensor:
     """Piecewise sparse attention forward; returns ``out`` (same shape and dtype as q).
     ``w_mode`` ("exact" or "pooled") picks the order-2 correction: the exact
-    1/2 q^T C_j q, or PWT's diagonal + pooled [query tile x block] estimate."""
+    1/2 q^T C_j q, or PWT's diagonal + pooled [query tile x block] estimate.
+    ``route`` ("centroid" or "cov") picks the selection score: the centroid score,
+    or the covariance-aware score plus ln(||H_j||_F + ROUTE_EPS)."""
     _need_cuda(q, k, v)
     if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k, v must share shape and dtype")
@@ -260,7 +305,7 @@ def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K:
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     _check(lib().pisa_attention_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d, code, B, K,
-                                   order, (FLAG_GATE_W if gate else 0) | (FLAG_POOLED_W if w_mode == "pooled" else 0),
+                                   order, _flags(gate, w_mode, route),
                                    PATHS[path], out.data_ptr(), workspace.data_ptr(),
                                    workspace.numel(), _stream(stream)))
     return out
@@ -299,14 +344,14 @@ class HostPlan:
 
 
 def pisa_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, plan: HostPlan,
-                        gate: bool = True, w_mode: str = "exact"):
+                        gate: bool = True, w_mode: str = "exact", route: str = "centroid"):
     """pisa_attention on pinned host tensors (q, k, v, out on the CPU); the work
     is queued on the plan's two streams, which the caller synchronises."""
     for t in (q, k, v, out):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError("pisa_attention_host takes contiguous host tensors")
     batch, heads, L, d, code, B, K, order = plan.args
-    flags = (FLAG_GATE_W if gate else 0) | (FLAG_POOLED_W if w_mode == "pooled" else 0)
+    flags = _flags(gate, w_mode, route)
     _check(lib().pisa_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), batch, heads, L, d,
                                      code, B, K, order, flags, PATHS[plan.path], plan.chunk, plan.buf.data_ptr(),
                                      plan.buf.numel(), plan.streams[0].cuda_stream, plan.streams[1].cuda_stream))

@@ -20,6 +20,7 @@
 #include "stats_tc.cuh"
 #include "hybrid_prep.cuh"
 #include "attn_hybrid.cuh"
+#include "route.cuh"
 
 using pisa::bf16;
 
@@ -187,7 +188,7 @@ pisa_status run_stats(const void* k, const void* v, const pisa_stats_t* st, cons
 }
 
 pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dtype dtype, int K, int32_t* idx,
-                       uint32_t* mask, cudaStream_t s) {
+                       uint32_t* mask, cudaStream_t s, const float* bias = nullptr, float* scores = nullptr) {
     return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
@@ -198,8 +199,25 @@ pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dty
         if (r != PISA_OK) return r;
         dim3 grid((unsigned)((g.nblk + QT - 1) / QT), (unsigned)g.BH);
         kern<<<grid, pisa::SelectCfg<D>::THREADS, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K,
-                                                              (int)g.words, QT, idx, mask);
+                                                              (int)g.words, QT, idx, mask, bias, scores);
         return launch_check("select_kernel");
+    });
+}
+
+// Covariance-aware routing bias ln(||H_j||_F + eps), [BH, nblk] fp32.
+pisa_status run_route_bias(const void* k, const void* v, const float* kbar, const Dims& g, pisa_dtype dtype,
+                           float eps, float* bias, cudaStream_t s) {
+    return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        const size_t smem = pisa::RouteCfg<D, BS>::SMEM;
+        auto kern = pisa::route_bias_kernel<T, D, BS>;
+        pisa_status r = set_smem(kern, smem);
+        if (r != PISA_OK) return r;
+        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        kern<<<grid, pisa::RouteCfg<D, BS>::THREADS, smem, s>>>((const T*)k, (const T*)v, kbar, (int)g.L,
+                                                                 (int)g.nblk, eps, bias);
+        return launch_check("route_bias_kernel");
     });
 }
 
@@ -247,7 +265,7 @@ pisa_status run_wpool(const void* q, const void* k, const Dims& g, pisa_dtype dt
 // workspace layout of pisa_attention
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t stats, mask, idx, total;
+    size_t stats, mask, idx, bias, total;
     StatsLayout sl;
     size_t kbar_bf, vsum_bf, hbar_acc, hbar_bf;  // hybrid path only
     size_t var, q2, wmat;                        // order 2: PWT's pooled w (used with the pooled flag)
@@ -269,6 +287,8 @@ WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path 
     o += align_up(sizeof(uint32_t) * g.BH * g.nblk * g.words);
     w.idx = o;
     o += align_up(sizeof(int32_t) * g.BH * g.nblk * (K > 0 ? K : 1));
+    w.bias = o;  // routing bias (used with PISA_FLAG_COV_ROUTE)
+    o += align_up(sizeof(float) * g.BH * g.nblk);
     if (path == PISA_PATH_HYBRID_TC) {
         w.kbar_bf = o;
         o += align_up(2 * g.BH * g.nblk * g.d);
@@ -381,6 +401,40 @@ pisa_status pisa_select(const void* q, const pisa_stats_t* st, int K, int32_t* i
     return run_select(q, st->kbar, g, st->dtype, K, K > 0 ? idx : nullptr, mask, (cudaStream_t)stream);
 }
 
+pisa_status pisa_select_biased(const void* q, const pisa_stats_t* st, int K, const float* bias, int32_t* idx,
+                               uint32_t* mask, void* stream) {
+    Dims g;
+    if (!st) return fail(PISA_ERR_INVALID_ARG, "null pisa_stats_t");
+    pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, 0, st->dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!st->kbar) return fail(PISA_ERR_INVALID_ARG, "pisa_select_biased: null kbar");
+    if (!q) return fail(PISA_ERR_INVALID_ARG, "pisa_select_biased: null q");
+    if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
+    if (!idx && !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_select_biased: idx and mask both null");
+    return run_select(q, st->kbar, g, st->dtype, K, K > 0 ? idx : nullptr, mask, (cudaStream_t)stream, bias);
+}
+
+pisa_status pisa_select_scores(const void* q, const pisa_stats_t* st, const float* bias, float* scores,
+                               void* stream) {
+    Dims g;
+    if (!st) return fail(PISA_ERR_INVALID_ARG, "null pisa_stats_t");
+    pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, 0, st->dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!st->kbar || !q || !scores) return fail(PISA_ERR_INVALID_ARG, "pisa_select_scores: null pointer");
+    return run_select(q, st->kbar, g, st->dtype, 0, nullptr, nullptr, (cudaStream_t)stream, bias, scores);
+}
+
+pisa_status pisa_route_bias(const void* k, const void* v, const float* kbar, int batch, int heads, int L, int d,
+                            pisa_dtype dtype, int B, float eps, float* bias, void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, 0, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (!k || !v || !kbar || !bias) return fail(PISA_ERR_INVALID_ARG, "pisa_route_bias: null pointer");
+    if (!(eps >= 1e-30f && eps <= 1e30f))
+        return fail(PISA_ERR_INVALID_ARG, "pisa_route_bias: eps must be in [1e-30, 1e30] (got %g)", (double)eps);
+    return run_route_bias(k, v, kbar, g, dtype, eps, bias, (cudaStream_t)stream);
+}
+
 int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order, pisa_dtype dtype) {
     Dims g;
     if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return -1;
@@ -422,6 +476,7 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         return fail(PISA_ERR_UNSUPPORTED, "hybrid path needs bf16, d and B in {64, 128}, L %% 128 == 0");
     const int gate = gate_w & PISA_FLAG_GATE_W;
     const bool pooled = (gate_w & PISA_FLAG_POOLED_W) != 0;
+    const bool route = (gate_w & PISA_FLAG_COV_ROUTE) != 0;
     if (path == PISA_PATH_HYBRID_TC && order == 2 && !pooled)
         return fail(PISA_ERR_UNSUPPORTED, "the hybrid's second order needs the pooled w (PISA_FLAG_POOLED_W)");
     if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC)
@@ -446,6 +501,7 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     st.cov = st.order == 2 ? (void*)(ws + w.stats + w.sl.cov) : nullptr;
     uint32_t* mask = (uint32_t*)(ws + w.mask);
     int32_t* idx = (int32_t*)(ws + w.idx);
+    float* rbias = route ? (float*)(ws + w.bias) : nullptr;
 
     float* wmat = nullptr;
     if (order == 2 && pooled) {
@@ -466,7 +522,11 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         r = pisa::run_hybrid_prep(k, v, st.kbar, kbar_bf, vsum_bf, hacc, hbf, g.BH, (int)g.L, (int)g.d, (int)g.B,
                                   (int)g.nblk, status, s, &g_last_error);
         if (r != PISA_OK) return r;
-        r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s);
+        if (route) {
+            r = run_route_bias(k, v, st.kbar, g, dtype, PISA_ROUTE_EPS, rbias, s);
+            if (r != PISA_OK) return r;
+        }
+        r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s, rbias);
         if (r != PISA_OK) return r;
         return pisa::run_attn_hybrid(q, k, v, kbar_bf, vsum_bf, hbf, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B,
                                      (int)g.nblk, (int)g.words, korder, wmat, status, s, &g_last_error);
@@ -478,7 +538,11 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         r = run_stats(k, v, &st, g, s);
         if (r != PISA_OK) return r;
     }
-    r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s);
+    if (route) {
+        r = run_route_bias(k, v, st.kbar, g, dtype, PISA_ROUTE_EPS, rbias, s);
+        if (r != PISA_OK) return r;
+    }
+    r = run_select(q, st.kbar, g, dtype, K, K > 0 ? idx : nullptr, mask, s, rbias);
     if (r != PISA_OK) return r;
     if (path == PISA_PATH_RECOMPUTE_TC) {
         unsigned int* status = device_status_ptr();

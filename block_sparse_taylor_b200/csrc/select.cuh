@@ -25,52 +25,25 @@ __device__ __forceinline__ uint32_t ordered_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ unsigned long long f2_pack(float2 v) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
-    return r;
-}
-__device__ __forceinline__ float2 f2_unpack(unsigned long long r) {
-    float2 v;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
-    return v;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
 // Canonical score: p_c = q_c * k_c rounded, then the pairwise tree
-// a[i] = a[i] + a[i + h], h = D/2 .. 1.  Lanes of packed pairs hold
-// (a[2m], a[2m+1]); every level with h >= 2 pairs up element-wise.
+// a[i] = a[i] + a[i + h], h = D/2 .. 1, every product and sum one IEEE fp32
+// round-to-nearest operation (__fmul_rn / __fadd_rn, which are never fused into
+// an FMA).  The first level is formed directly from the products of columns i
+// and i + D/2.  (Packed fp32x2 multiplies and adds do not reproduce separately
+// rounded scalar operations, so they are not used here.)
 template <int D>
-__device__ __forceinline__ float canonical_dot(const unsigned long long (&q2)[D / 2], const float* __restrict__ k) {
-    unsigned long long a[D / 4];
+__device__ __forceinline__ float canonical_dot(const float (&q)[D], const float* __restrict__ k) {
+    float a[D / 2];
     const float4* k4 = reinterpret_cast<const float4*>(k);
 #pragma unroll
-    for (int m = 0; m < D / 4; m += 2) {
-        // products of columns 2m .. 2m+3 and of D/2 + 2m .. D/2 + 2m + 3
-        const float4 lo = k4[m / 2], hi = k4[(D / 2 + 2 * m) / 4];
-        const unsigned long long plo0 = f2_mul(q2[m], f2_pack(make_float2(lo.x, lo.y)));
-        const unsigned long long plo1 = f2_mul(q2[m + 1], f2_pack(make_float2(lo.z, lo.w)));
-        const unsigned long long phi0 = f2_mul(q2[D / 4 + m], f2_pack(make_float2(hi.x, hi.y)));
-        const unsigned long long phi1 = f2_mul(q2[D / 4 + m + 1], f2_pack(make_float2(hi.z, hi.w)));
-        a[m] = f2_add(plo0, phi0);
-        a[m + 1] = f2_add(plo1, phi1);
+    for (int m = 0; m < D / 8; ++m) {
+        const float4 lo = k4[m], hi = k4[D / 8 + m];
+        a[4 * m + 0] = __fadd_rn(__fmul_rn(q[4 * m + 0], lo.x), __fmul_rn(q[D / 2 + 4 * m + 0], hi.x));
+        a[4 * m + 1] = __fadd_rn(__fmul_rn(q[4 * m + 1], lo.y), __fmul_rn(q[D / 2 + 4 * m + 1], hi.y));
+        a[4 * m + 2] = __fadd_rn(__fmul_rn(q[4 * m + 2], lo.z), __fmul_rn(q[D / 2 + 4 * m + 2], hi.z));
+        a[4 * m + 3] = __fadd_rn(__fmul_rn(q[4 * m + 3], lo.w), __fmul_rn(q[D / 2 + 4 * m + 3], hi.w));
     }
-#pragma unroll
-    for (int h = D / 8; h >= 1; h >>= 1) {
-#pragma unroll
-        for (int m = 0; m < h; ++m) a[m] = f2_add(a[m], a[m + h]);
-    }
-    const float2 last = f2_unpack(a[0]);
-    return __fadd_rn(last.x, last.y);
+    return tree_sum<D / 2>(a);
 }
 
 template <int D>
@@ -98,13 +71,16 @@ inline size_t select_smem_bytes(int QT, int nblk) {
 //   2. scores: lane t of every warp holds tile t's mean in registers, the
 //      centroids are staged JC at a time and read as broadcasts; warp w takes
 //      the blocks jj = w, w+8, ... of each chunk;
+//      with a routing bias ([BH, nblk], or null) each score gets bias_j added;
 //   3. top-K per tile (warp per tile): binary search for the K-th largest
 //      ordered score, then ties broken by ascending block index with ballots;
 //      the ballots are the mask words and give the ascending index list.
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                                                         int L, int nblk, int K, int words, int QT,
-                                                        int32_t* __restrict__ idx, uint32_t* __restrict__ mask) {
+                                                        int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
+                                                        const float* __restrict__ bias,
+                                                        float* __restrict__ scores_out) {
     using C = SelectCfg<D>;
     extern __shared__ __align__(16) float sm_sel[];
     float* qbar = sm_sel;                 // [QT][D]
@@ -143,11 +119,17 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
 
     // 2. scores
     const bool live = lane < nq;
-    unsigned long long q2[D / 2];
+    float qr[D];
     {
-        const float2* qs = reinterpret_cast<const float2*>(qbar + (live ? lane : 0) * D);
+        const float4* qs = reinterpret_cast<const float4*>(qbar + (live ? lane : 0) * D);
 #pragma unroll
-        for (int m = 0; m < D / 2; ++m) q2[m] = f2_pack(qs[m]);
+        for (int m = 0; m < D / 4; ++m) {
+            const float4 t = qs[m];
+            qr[4 * m] = t.x;
+            qr[4 * m + 1] = t.y;
+            qr[4 * m + 2] = t.z;
+            qr[4 * m + 3] = t.w;
+        }
     }
     const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nblk * D);
     for (int j0 = 0; j0 < nblk; j0 += C::JC) {
@@ -156,10 +138,20 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
         for (int e = tid; e < nj * D / 4; e += C::THREADS) kst4[e] = kb4[(size_t)j0 * D / 4 + e];
         __syncthreads();
         for (int jj = warp; jj < nj; jj += 8) {
-            const float s = canonical_dot<D>(q2, kst + jj * D);
+            float s = canonical_dot<D>(qr, kst + jj * D);
+            // covariance-aware routing: one fp32 add of the block's bias
+            if (bias) s = __fadd_rn(s, __ldg(bias + (size_t)bh * nblk + j0 + jj));
             if (live) sc[lane * SS + j0 + jj] = s;
         }
         __syncthreads();
+    }
+
+    // the score table itself, when asked for ([BH, nblk, nblk] fp32)
+    if (scores_out) {
+        for (int e = tid; e < nq * nblk; e += C::THREADS) {
+            const int t = e / nblk, jj = e % nblk;
+            scores_out[((size_t)bh * nblk + i0 + t) * nblk + jj] = sc[t * SS + jj];
+        }
     }
 
     // 3. top-K, one warp per tile.  For nblk <= 1024 every lane keeps its

@@ -133,6 +133,39 @@ pisa_status pisa_stats(const void* k, const void* v, const pisa_stats_t* st, voi
 pisa_status pisa_select(const void* q, const pisa_stats_t* st, int K, int32_t* idx,
                         uint32_t* mask, void* stream);
 
+/* Covariance-aware block selection (PISA paper, section 3.3 "Covariance-Aware
+ * Block Selection": the log of a block norm plus eps is added to the centroid
+ * score; "Sparse Linear Attention" blog, PWT section: route by the score plus
+ * the log of the norm of H_j).  As pisa_select with every score s_ij replaced
+ * by s_ij + bias[bh][j] (one fp32 add, round to nearest) before the top-K.
+ * bias: [BH, nblk] fp32 device array (pisa_route_bias output), or NULL for
+ * exactly pisa_select. */
+pisa_status pisa_select_biased(const void* q, const pisa_stats_t* st, int K, const float* bias,
+                               int32_t* idx, uint32_t* mask, void* stream);
+
+/* The score table of the selection: scores [BH, nblk, nblk] fp32 (row = query
+ * tile i, column = block j) holding s_ij exactly as pisa_select (bias NULL) or
+ * pisa_select_biased computes it before the top-K.  For inspection and tests. */
+pisa_status pisa_select_scores(const void* q, const pisa_stats_t* st, const float* bias, float* scores,
+                               void* stream);
+
+/* Routing bias bias[bh][j] = ln(||H_j||_F + eps) of every key block, from k and
+ * v ([BH, L, d], `dtype`) and the canonical centroids kbar ([BH, nblk, d] fp32,
+ * pisa_centroids or pisa_stats output).  It decides a selection, so it is
+ * computed in a fixed fp32 procedure that reproduces bit for bit:
+ *   dev[n][b]  = k_{j,n}[b] - kbar_j[b]
+ *   h[a*d + b] = tsum over the B rows n of (v_{j,n}[a] * dev[n][b])
+ *   M_j        = sqrt(tsum over the d*d entries a*d + b of h^2)   (IEEE sqrt)
+ *   bias_j     = ln_repro(M_j + eps)
+ * with tsum as in pisa_select and ln_repro the fixed-operation logarithm:
+ * x = 2^e m, m folded into [sqrt(1/2), sqrt(2)) (the fp32 constant 0x1.6a09e6p+0),
+ * s = (m - 1)/(m + 1), t = Horner in s^2 on the fp32 constants 1/9, 1/7, 1/5, 1/3
+ * and 1, ln x = e * fl(ln 2) + (t * s) * 2, every operation one IEEE fp32
+ * round-to-nearest step in that order.  eps in [1e-30, 1e30]
+ * (pisa_attention_ex uses PISA_ROUTE_EPS).  Output: bias [BH, nblk] fp32. */
+pisa_status pisa_route_bias(const void* k, const void* v, const float* kbar, int batch, int heads, int L,
+                            int d, pisa_dtype dtype, int B, float eps, float* bias, void* stream);
+
 /* Centroids only: kbar [BH, nblk, d] fp32 of k ([BH, L, d], `dtype`), in the
  * canonical fp32 order of pisa_select (pairwise tree over the B rows, times
  * 1/B).  This is the part of the prepare phase the token-form path needs. */
@@ -174,10 +207,14 @@ pisa_status pisa_attention(const void* q, const void* k, const void* v, int batc
                               * var_c(keys of block j), one value per (query tile, block),
                               * instead of the exact per-query 1/2 q^T C_j q.  Required
                               * for order 2 on the hybrid path; pisa_attention_ex only. */
+#define PISA_FLAG_COV_ROUTE 4 /* covariance-aware selection: pisa_route_bias with
+                               * PISA_ROUTE_EPS, then pisa_select_biased (pisa_attention_ex) */
+#define PISA_ROUTE_EPS 1e-6f
 
 /* As pisa_attention with the PWT options as flags (gate_w: PISA_FLAG_GATE_W,
- * PISA_FLAG_POOLED_W; 0 = exact w, never zeroed) and an explicit path.  The
- * workspace of an order-2 call also holds the pooled-w arrays. */
+ * PISA_FLAG_POOLED_W, PISA_FLAG_COV_ROUTE; 0 = exact w, never zeroed, centroid
+ * routing) and an explicit path.  The workspace of an order-2 call also holds
+ * the pooled-w arrays; every workspace holds the routing bias. */
 pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads,
                               int L, int d, pisa_dtype dtype, int B, int K, int order, int gate_w,
                               pisa_path path, void* out, void* workspace, size_t ws_bytes,

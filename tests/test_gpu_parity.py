@@ -122,6 +122,29 @@ def test_select_planted_ties():
         assert np.array_equal(idx, ridx) and np.array_equal(mask, rmask)
 
 
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d,B,L", [(64, 64, 2048), (128, 64, 4096), (128, 128, 4096), (64, 128, 1024)])
+def test_select_scores_bit_exact(dt, d, B, L):
+    # the canonical fp32 score table itself, not only the top-K it decides
+    q, k, v = pisa_synth.random_qkv(250 + d + B + L, 2, L, d, scale=1.0, dtype=dt)
+    st = pisa.pisa_centroids(dev(k, dt), B)
+    sc = pisa.pisa_select_scores(dev(q, dt), st)
+    torch.cuda.synchronize()
+    _, _, ref = oracle.select(q, k, B, 1, want_scores=True)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("name,heads", [("c3", 4), ("c4", 2), ("c2", 12), ("c5_L16896_s90", 4)])
+def test_select_scores_full_size_bit_exact(name, heads):
+    w = pisa_synth.workloads()[name].with_(heads=heads)
+    q, k, v = pisa_synth.generate(w)
+    st = pisa.pisa_centroids(dev(k, w.dtype), w.B)
+    sc = pisa.pisa_select_scores(dev(q, w.dtype), st)
+    torch.cuda.synchronize()
+    _, _, ref = oracle.select(q, k, w.B, 1, want_scores=True)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5_L4608_s75", "c5_L16896_s90"])
 def test_select_full_size(name):
     w, (q, k, v) = workload(name)
