@@ -435,7 +435,7 @@ def main():
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
         ho = torch.empty_like(hq).pin_memory()
-        plan = pisa.HostPlan(hq, B, K, order, chunk_heads=max(1, BH // 8))
+        plan = pisa.HostPlan(hq, B, K, order, chunk_heads=max(1, BH // 20))
 
         def e2e_step():
             for st_ in plan.streams:

@@ -225,7 +225,7 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for x in [-125, 64]: x = n + f with n = round(x)
+// 2^x on the FMA pipe, for x in [-125, 64] (0 below, -inf included): x = n + f with n = round(x)
 // (the 1.5 * 2^23 addition rounds to nearest and leaves n in the low mantissa
 // bits), 2^f for f in [-1/2, 1/2] by a cubic fitted to minimise the relative
 // error (max 7.5e-5, well below bf16's 2^-9), then n added to the exponent.
@@ -235,7 +235,8 @@ __device__ __forceinline__ float ex2_fma(float x) {
     const float t = x + 12582912.0f;
     const float f = x - (t - 12582912.0f);
     const float p = fmaf(fmaf(fmaf(0.05517139f, f, 0.24261111f), f, 0.69326103f), f, 0.99992806f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+    const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+    return x > -125.0f ? r : 0.0f;
 }
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes of work per instruction).
