@@ -168,6 +168,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ORDER: 0 zeroth, 1 first, 2 first + exact w from the logits, 3 first + the
     // pooled diagonal w of wmat ([BH, nblk, nblk], row = query tile, already gated)
     using C = TcCfg<D>;
+    // with two K/V stages the producer frees stages off group 1's S-full
+    // barrier, and the MMA thread issues no empty-barrier commits (each
+    // tcgen05.commit in the stream stalls the tensor pipe for tens of cycles)
+    constexpr bool kSfullRelease = (C::NS == 2);
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, N = 128 keys
     constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);     // O += P V, N = d, V MN-major
 
@@ -228,14 +232,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int lastK = -1, lastV = -1;
             for (int jt = 0; jt < NT; ++jt) {
                 const int st = jt % C::NS, u = jt / C::NS;
-                if (u > 0 && !tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                if (kSfullRelease) {
+                    // two stages: S1(jt-1) completing (group 1's S-full barrier) means
+                    // S0/S1(jt-2) and PV1(jt-2) are done, so the K and V stage of tile
+                    // jt-2 are free.  One wait per tile, phases in order; S1(jt) needs
+                    // K(jt), not loaded yet, so the barrier is never two phases ahead.
+                    if (jt >= 1 && !tc::mbar_wait(bar(B_SFULL + 1), (jt - 1) & 1, aborted, status, kWaitLimitCycles))
+                        break;
+                } else if (u > 0 &&
+                           !tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles)) {
                     break;
+                }
                 tc::mbar_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
                     tc::tma_load_2d(sbase + C::K_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_k,
                                     bar(B_KFULL + st), b * C::BOX, bh * L + jt * C::NK);
                 lastK = jt;
-                if (u > 0 && !tc::mbar_wait(bar(B_VEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                if (!kSfullRelease && u > 0 &&
+                    !tc::mbar_wait(bar(B_VEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
                     break;
                 tc::mbar_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
@@ -289,7 +303,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::mma_commit(bar(B_SFULL + 0));
                 issue_s(1, 0);
                 tc::mma_commit(bar(B_SFULL + 1));
-                tc::mma_commit(bar(B_KEMPTY + 0));
+                if (!kSfullRelease) tc::mma_commit(bar(B_KEMPTY + 0));
             }
             for (int jt = 0; ok && jt < NT; ++jt) {
                 const int st = jt % C::NS, u = jt / C::NS;
@@ -315,11 +329,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::fence_after_sync();
                 issue_pv(1, st, 1, false);
                 if (!more) tc::mma_commit(bar(B_OFULL + 1));
-                tc::mma_commit(bar(B_VEMPTY + st));
+                if (!kSfullRelease) tc::mma_commit(bar(B_VEMPTY + st));
                 if (more) {
                     issue_s(1, st1);
                     tc::mma_commit(bar(B_SFULL + 1));
-                    tc::mma_commit(bar(B_KEMPTY + st1));
+                    if (!kSfullRelease) tc::mma_commit(bar(B_KEMPTY + st1));
                 }
             }
             // every MMA issued by this thread has completed before TMEM is freed
