@@ -70,6 +70,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ORDER: 0 zeroth, 1 first (H-bar), 3 first + the pooled diagonal second-order
     // term of wmat ([BH, nblk, nblk], row = query tile, gated) on every virtual token
     using C = HybCfg<D, BS>;
+    // two K/V stages: stages are freed off group 1's S-full barrier (see the
+    // token-form kernel), with no empty-barrier commits in the MMA stream
+    constexpr bool kSfullRelease = (C::NS == 2);
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
     constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);
@@ -197,17 +200,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             for (int jt = 0; jt < NT; ++jt) {
                 const int st = jt % C::NS, u = jt / C::NS;
-                if (u > 0 && !tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                if (kSfullRelease) {
+                    // S1(jt-1) done: the stage of tile jt-2 is free (one wait per tile, in order)
+                    if (jt >= 1 && !tc::mbar_wait(bar(B_SFULL + 1), (jt - 1) & 1, aborted, status, kWaitLimitCycles))
+                        break;
+                } else if (u > 0 &&
+                           !tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles)) {
                     break;
+                }
                 load_tile(jt, sbase + C::K_OFF + st * C::TILE_BYTES, 0, true);
-                if (u > 0 && !tc::mbar_wait(bar(B_VEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                if (!kSfullRelease && u > 0 &&
+                    !tc::mbar_wait(bar(B_VEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
                     break;
                 load_tile(jt, 0, sbase + C::V_OFF + st * C::TILE_BYTES, false);
             }
             if (ORDER >= 1 && !aborted) {
                 // H-bar into the next K stage once it is free
                 const int st = NT % C::NS, u = NT / C::NS;
-                if (u == 0 || tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles)) {
+                const bool free_stage =
+                    kSfullRelease ? tc::mbar_wait(bar(B_SFULL + 1), (NT - 1) & 1, aborted, status, kWaitLimitCycles)
+                                  : (u == 0 ||
+                                     tc::mbar_wait(bar(B_KEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles));
+                if (free_stage) {
                     tc::mbar_expect_tx(bar(B_HFULL), (uint32_t)(D * D * 2));
                     for (int x = 0; x < C::NBOX; ++x)
                         tc::tma_load_2d(sbase + C::K_OFF + st * C::TILE_BYTES + x * C::BOX_BYTES, &tm_hb,
@@ -249,7 +263,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::mma_commit(bar(B_SFULL + 0));
                 issue_s(1, 0, IDESC_S);
                 tc::mma_commit(bar(B_SFULL + 1));
-                tc::mma_commit(bar(B_KEMPTY + 0));
+                if (!kSfullRelease) tc::mma_commit(bar(B_KEMPTY + 0));
             }
             for (int jt = 0; ok && jt < NT; ++jt) {
                 const int st = jt % C::NS, u = jt / C::NS;
@@ -267,11 +281,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!tc::mbar_wait(bar(B_PFULL + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
                 issue_pv(1, st, jt == 0);
-                tc::mma_commit(bar(B_VEMPTY + st));
+                if (!kSfullRelease) tc::mma_commit(bar(B_VEMPTY + st));
                 if (more) {
                     issue_s(1, st1, IDESC_S);
                     tc::mma_commit(bar(B_SFULL + 1));
-                    tc::mma_commit(bar(B_KEMPTY + st1));
+                    if (!kSfullRelease) tc::mma_commit(bar(B_KEMPTY + st1));
                 }
             }
             if (!aborted) {
