@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--heads", type=int, default=None, help="override head count (profiling small cases)")
     p.add_argument("--no-hybrid", action="store_true", help="skip the PISA-hybrid (global H-bar) record")
+    p.add_argument("--no-route", action="store_true", help="skip the covariance-aware routing record")
     return p.parse_args()
 
 
@@ -402,6 +403,34 @@ def main():
                      "frac_hbm": s_bytes / (s_ms * 1e-3) / 1e9 / hbm}
         del sbuf
 
+    # Covariance-aware routing (opt-in): the bias kernel ln(||H_j||_F + eps) and
+    # the biased selection, timed on their own on the same inputs.
+    route_rec = None
+    if path != "stats" and not args.no_route:
+        rb = torch.empty((BH, nblk), dtype=torch.float32, device="cuda")
+        st_c = pisa.pisa_centroids(k, B, kbar=kbar)
+        for _ in range(2):
+            pisa.pisa_route_bias(k, v, kbar, B, out=rb)
+        ra, rb_ev, rc_ev = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        reps = 5
+        ra.record(stream)
+        for _ in range(reps):
+            pisa.pisa_route_bias(k, v, kbar, B, out=rb)
+        rb_ev.record(stream)
+        for _ in range(reps):
+            pisa._check(pisa.lib().pisa_select_biased(q.data_ptr(), pisa.ctypes.byref(st_c.raw), K,
+                                                       rb.data_ptr(), idx.data_ptr() if K else None,
+                                                       mask.data_ptr(), stream.cuda_stream))
+        rc_ev.record(stream)
+        torch.cuda.synchronize()
+        pisa.pisa_poll_device_status()
+        r_ms = ra.elapsed_time(rb_ev) / reps
+        route_rec = {"bias_kernel": f"route_bias_kernel<{d},{B}>", "bias_ms": r_ms,
+                     "bias_gflops_fp32": 2.0 * BH * nblk * B * d * d / (r_ms * 1e-3) / 1e9,
+                     "select_biased_ms": rb_ev.elapsed_time(rc_ev) / reps,
+                     "note": "scalar IEEE fp32 in a canonical order (reproducible bit for bit), CUDA cores"}
+        del rb
+
     # The PISA hybrid (global H-bar, the paper's own speed path) on the same
     # inputs: a separate record, timed as whole calls of pisa_attention.
     hybrid_rec = None
@@ -482,6 +511,7 @@ def main():
             "per_kernel": per_kernel,
             "stats_kernel": stats_rec,
             "hybrid": hybrid_rec,
+            "routing": route_rec,
             "cpu_baseline": cpu,
             "clocks": clk,
             "e2e": e2e,

@@ -52,43 +52,52 @@ __device__ __forceinline__ float ln_repro(float x) {
 template <int D, int BS>
 struct RouteCfg {
     static constexpr int THREADS = 256;
-    static constexpr int NE = D * D / THREADS;  // H entries per thread (e = tid + 256 m)
-    static constexpr size_t SMEM = sizeof(float) * (2 * (size_t)BS * D + (size_t)D * D);
+    static constexpr int NE = D * D / THREADS;  // H entries per thread (e = tid + 256 m, one key channel)
+    static constexpr int VS = BS + 4;            // row stride of the transposed values (16-byte rows)
+    static constexpr size_t SMEM = sizeof(float) * ((size_t)D * VS + (size_t)D * D);
 };
 
 // One CTA per (key block j, bh).  Thread tid computes the entries
-// e = tid + 256 m of H_j (key channel b = e mod d) with scalar IEEE operations
-// (__fmul_rn / __fadd_rn, never fused; packed fp32x2 arithmetic does not
-// reproduce separately rounded scalar operations); the squares go to shared
-// memory and the canonical tree over all d^2 of them runs there.
+// e = tid + 256 m of H_j, which all share the key channel b = e mod d: its B
+// deviations dev[n][b] stay in registers, and the values are read transposed
+// (vT[a][n]) with 16-byte loads that the whole warp shares (a is the same for
+// all lanes of a warp).  Scalar IEEE operations only (__fmul_rn / __fadd_rn,
+// never fused; packed fp32x2 arithmetic does not reproduce separately rounded
+// scalar operations).  The squares go to shared memory and the canonical tree
+// over all d^2 of them runs there.
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(256) route_bias_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                                          const float* __restrict__ kbar, int L, int nblk,
                                                          float eps, float* __restrict__ bias) {
     using C = RouteCfg<D, BS>;
     extern __shared__ __align__(16) float sm_route[];
-    float* dev = sm_route;         // [BS][D]
-    float* vv = dev + BS * D;      // [BS][D]
-    float* sq = vv + BS * D;       // [D * D]
+    float* vT = sm_route;          // [D][VS]: vT[a][n] = v_{j,n}[a]
+    float* sq = vT + D * C::VS;    // [D * D]
     const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const size_t base = ((size_t)bh * L + (size_t)j * BS) * D;
-    const float* kb = kbar + ((size_t)bh * nblk + j) * D;
-    for (int e = tid; e < BS * D; e += C::THREADS) {
-        dev[e] = __fsub_rn(to_f(k[base + e]), kb[e % D]);
-        vv[e] = to_f(v[base + e]);
+    for (int e = tid; e < BS * D; e += C::THREADS) vT[(e % D) * C::VS + e / D] = to_f(v[base + e]);
+    const int b = tid % D;
+    float dv[BS];  // dev[n][b] = k_{j,n}[b] - kbar_j[b]
+    {
+        const float kb = kbar[((size_t)bh * nblk + j) * D + b];
+#pragma unroll
+        for (int n = 0; n < BS; ++n) dv[n] = __fsub_rn(to_f(k[base + (size_t)n * D + b]), kb);
     }
     __syncthreads();
-    const int b = tid % D;
 #pragma unroll 1
     for (int m = 0; m < C::NE; ++m) {
         const int e = tid + C::THREADS * m;
-        const int a = e / D;
+        const float4* va = reinterpret_cast<const float4*>(vT + (e / D) * C::VS);
         // first tree level pairs n with n + BS/2
         float p[BS / 2];
 #pragma unroll
-        for (int n = 0; n < BS / 2; ++n)
-            p[n] = __fadd_rn(__fmul_rn(vv[n * D + a], dev[n * D + b]),
-                             __fmul_rn(vv[(n + BS / 2) * D + a], dev[(n + BS / 2) * D + b]));
+        for (int i = 0; i < BS / 8; ++i) {
+            const float4 lo = va[i], hi = va[BS / 8 + i];
+            p[4 * i + 0] = __fadd_rn(__fmul_rn(lo.x, dv[4 * i + 0]), __fmul_rn(hi.x, dv[BS / 2 + 4 * i + 0]));
+            p[4 * i + 1] = __fadd_rn(__fmul_rn(lo.y, dv[4 * i + 1]), __fmul_rn(hi.y, dv[BS / 2 + 4 * i + 1]));
+            p[4 * i + 2] = __fadd_rn(__fmul_rn(lo.z, dv[4 * i + 2]), __fmul_rn(hi.z, dv[BS / 2 + 4 * i + 2]));
+            p[4 * i + 3] = __fadd_rn(__fmul_rn(lo.w, dv[4 * i + 3]), __fmul_rn(hi.w, dv[BS / 2 + 4 * i + 3]));
+        }
         const float h = tree_sum<BS / 2>(p);
         sq[e] = __fmul_rn(h, h);
     }
