@@ -13,8 +13,9 @@
 // Adding the Second-Order Term (PWT)" (w, the shared corrected logit, the
 // ln B gate).
 //
-// One CTA per (query tile, bh), 8 warps; warp w owns rows w, w+8, ...; the
-// running max, denominator and numerator of every row live in shared memory.
+// One CTA per (RQ query rows of a tile, bh), 8 warps; warp w owns rows w, w+8,
+// ...; the running max, denominator and numerator of every row live in shared
+// memory.  RQ = B, or B/2 when a whole tile's state does not fit (fp32, d = B = 128).
 // The block being processed (K_j and V_j, or H_j and C_j) is staged in shared
 // memory with padded rows so that lanes reading different rows hit different
 // banks.  This is the fp32 path and the reference path for the tensor-core
@@ -25,13 +26,22 @@
 
 namespace pisa {
 
-template <typename T, int D, int BS>
-struct AttnStatsSmem {
+template <typename T, int D, int BS, int RQ>
+struct AttnStatsSmemRQ {
     static constexpr int QS = D + 1;                           // fp32 row stride
     static constexpr int XS = D + (sizeof(T) == 2 ? 2 : 1);    // T row stride (odd word count)
     static constexpr int ROWS = (BS > D ? BS : D);
-    static constexpr size_t bytes = sizeof(float) * ((size_t)BS * QS + (size_t)BS * D + 2 * BS + 2 * D) +
+    static constexpr size_t bytes = sizeof(float) * ((size_t)RQ * QS + (size_t)RQ * D + 2 * RQ + 2 * D) +
                                     sizeof(T) * 2 * (size_t)ROWS * XS;
+};
+// query rows per CTA: the whole tile when it fits in 227 KB of shared memory, else half
+template <typename T, int D, int BS>
+struct AttnStatsSmem {
+    static constexpr int RQ = (AttnStatsSmemRQ<T, D, BS, BS>::bytes <= 227 * 1024) ? BS : BS / 2;
+    static constexpr int QS = AttnStatsSmemRQ<T, D, BS, RQ>::QS;
+    static constexpr int XS = AttnStatsSmemRQ<T, D, BS, RQ>::XS;
+    static constexpr int ROWS = AttnStatsSmemRQ<T, D, BS, RQ>::ROWS;
+    static constexpr size_t bytes = AttnStatsSmemRQ<T, D, BS, RQ>::bytes;
 };
 
 template <typename T, int D, int BS>
@@ -42,23 +52,23 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
     int words, int order, int gate, float ln_b, const float* __restrict__ wmat) {
     // wmat (order 2, optional): PWT's pooled diagonal w per (query tile, block), gated
     using SM = AttnStatsSmem<T, D, BS>;
-    constexpr int QS = SM::QS, XS = SM::XS, W = D / 32;
+    constexpr int QS = SM::QS, XS = SM::XS, W = D / 32, RQ = SM::RQ;
     extern __shared__ __align__(16) float sm_attn[];
-    float* qs = sm_attn;            // [BS][QS]
-    float* Ns = qs + BS * QS;       // [BS][D]
-    float* ms = Ns + BS * D;        // [BS]
-    float* ds = ms + BS;            // [BS]
-    float* aux = ds + BS;           // [2][D]: kbar_j, vsum_j
+    float* qs = sm_attn;            // [RQ][QS]
+    float* Ns = qs + RQ * QS;       // [RQ][D]
+    float* ms = Ns + RQ * D;        // [RQ]
+    float* ds = ms + RQ;            // [RQ]
+    float* aux = ds + RQ;           // [2][D]: kbar_j, vsum_j
     T* st0 = (T*)(aux + 2 * D);     // [ROWS][XS]: K_j or H_j
     T* st1 = st0 + SM::ROWS * XS;   // [ROWS][XS]: V_j or C_j
-    const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const int i = blockIdx.x / (BS / RQ), part = blockIdx.x % (BS / RQ), bh = blockIdx.y, tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
-    const size_t base = ((size_t)bh * L + (size_t)i * BS) * D;
-    for (int e = tid; e < BS * D; e += 256) {
+    const size_t base = ((size_t)bh * L + (size_t)i * BS + (size_t)part * RQ) * D;
+    for (int e = tid; e < RQ * D; e += 256) {
         qs[(e / D) * QS + e % D] = to_f(q[base + e]);
         Ns[e] = 0.f;
     }
-    for (int r = tid; r < BS; r += 256) {
+    for (int r = tid; r < RQ; r += 256) {
         ms[r] = -INFINITY;
         ds[r] = 0.f;
     }
@@ -89,7 +99,7 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
             }
         }
         __syncthreads();
-        for (int r = warp; r < BS; r += 8) {
+        for (int r = warp; r < RQ; r += 8) {
             const float* qr = qs + r * QS;
             const float m_old = ms[r], d_old = ds[r];
             float acc[W];
@@ -178,7 +188,7 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
         }
         __syncthreads();
     }
-    for (int e = tid; e < BS * D; e += 256) out[base + e] = from_f<T>(Ns[e] / ds[e / D]);
+    for (int e = tid; e < RQ * D; e += 256) out[base + e] = from_f<T>(Ns[e] / ds[e / D]);
 }
 
 }  // namespace pisa

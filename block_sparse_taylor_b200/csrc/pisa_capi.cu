@@ -231,7 +231,8 @@ pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pi
         auto kern = pisa::attn_stats_kernel<T, D, BS>;
         pisa_status r = set_smem(kern, smem);
         if (r != PISA_OK) return r;
-        dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        constexpr int parts = BS / pisa::AttnStatsSmem<T, D, BS>::RQ;  // CTAs per query tile
+        dim3 grid((unsigned)(g.nblk * parts), (unsigned)g.BH);
         kern<<<grid, 256, smem, s>>>((const T*)q, (const T*)k, (const T*)v, st->kbar, st->vsum,
                                      (const T*)st->hstat, (const T*)st->cov, mask, (T*)out, (int)g.L,
                                      (int)g.nblk, (int)g.words, order, gate, logf((float)g.B), wmat);

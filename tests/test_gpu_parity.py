@@ -178,7 +178,7 @@ def test_attention_small_bf16(path, d, B, order):
     assert err <= 5e-3, err  # the expected bf16 rounding level; a formulation slip is far above it
 
 
-@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128)])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
 @pytest.mark.parametrize("order", [0, 1, 2])
 def test_attention_small_f32(d, B, order):
     L = 1024
