@@ -200,7 +200,9 @@ inline pisa_status run_hybrid_prep(const void* k, const void* v, float* kbar, bf
             return PISA_ERR_CUDA;
         }
     }
-    const int G = 64;  // blocks per CTA
+    // blocks per CTA: 64, halved (down to 8) until the grid has about four CTAs per SM
+    int G = 64;
+    while (G > 8 && (long)((nblk + G - 1) / G) * BH < 4L * 148) G /= 2;
     dim3 grid((unsigned)((nblk + G - 1) / G), (unsigned)BH);
     const float scale = (float)B / (float)L;
     cudaError_t e = cudaSuccess;

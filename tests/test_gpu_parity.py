@@ -358,6 +358,20 @@ def test_pooled_w_full_size_c2(path):
     assert rel_l2(rows_of(got, tiles, w.B), ref) <= TOL[w.dtype]
 
 
+def test_host_entry_point_with_routing_matches_device_call():
+    q, k, v = pisa_synth.random_qkv(77, 6, 1024, 128, scale=2.0, dtype="bf16")
+    B, K = 64, 4
+    dq, dk, dv = (dev(x, "bf16") for x in (q, k, v))
+    want = pisa.pisa_attention(dq, dk, dv, B, K, 1, route="cov")
+    hq, hk, hv = (t.cpu().pin_memory() for t in (dq, dk, dv))
+    ho = torch.empty_like(hq).pin_memory()
+    plan = pisa.HostPlan(hq, B, K, 1, chunk_heads=4)
+    pisa.pisa_attention_host(hq, hk, hv, ho, plan, route="cov")
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    assert torch.equal(ho, want.cpu())
+
+
 def test_host_entry_point_matches_device_call():
     # pisa_attention_host runs pisa_attention_ex per chunk of heads from pinned
     # host memory; heads are independent, so the result equals the device call.
