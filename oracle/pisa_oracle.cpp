@@ -396,6 +396,118 @@ void row_brute(const float* qrow, const float* k, const float* v, long d, long B
     for (long c = 0; c < d; ++c) out[c] = num[c] / D;
 }
 
+// Gradients of the method's output for one (bh) (no equations on the pages;
+// derived here from the forward above, with the selection held fixed, as the
+// PWT blog describes training with the routing detached).  Per query row t,
+// with G_n = dO_t . v_n, delta = dO_t . o_t and, for an unselected block j,
+// E = e^{l}, u_n = x_n - s-bar, G-bar = (1/B) sum_n G_n:
+//   exact key n:       dL/dx_n = e^{x_n} (G_n - delta) / D
+//   unselected key m:  dL/dx_m = (E/D) [ (dl/dx_m) (sum_n G_n (1 + c1 u_n) - B delta)
+//                                        + c1 (G_m - G-bar) ],
+//   c1 = [order >= 1], dl/dx_m = 1/B, plus u_m / B for order 2 when the gate is
+//   open (w = (1/2B) sum u^2; the gate decision itself is held fixed);
+//   dq_t = sum_n dL/dx_tn k_n,  dk_n = sum_t dL/dx_tn q_t,
+//   dv_n = sum_t (weight_tn / D_t) dO_t  (weight = the numerator's e^{x} or E (1 + c1 u_n)).
+// Evaluated with the common max shift m (it cancels in weight / D).
+void backward_one(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B, long K,
+                  int order, int gate, double* dq, double* dk, double* dv) {
+    const long nblk = L / B;
+    const long words = (nblk + 31) / 32;
+    std::vector<uint32_t> mask(nblk * words, 0u);
+    select_one(q, k, L, d, B, K, nullptr, mask.data(), nullptr);
+    std::vector<double> kbar(nblk * d, 0.0);
+    for (long j = 0; j < nblk; ++j)
+        for (long c = 0; c < d; ++c) {
+            double sacc = 0.0;
+            for (long n = 0; n < B; ++n) sacc += (double)k[(j * B + n) * d + c];
+            kbar[j * d + c] = sacc / (double)B;
+        }
+    const double ln_b = std::log((double)B);
+    const int c1 = order >= 1 ? 1 : 0;
+    std::vector<double> x(L), wt(L), lj(nblk), wj(nblk), sbj(nblk), o(d), G(L), gx(L);
+    std::vector<char> open(nblk);
+    for (long t = 0; t < L; ++t) {
+        const long i = t / B;
+        const float* qt = q + t * d;
+        for (long n = 0; n < L; ++n) {
+            double sacc = 0.0;
+            for (long c = 0; c < d; ++c) sacc += (double)qt[c] * (double)k[n * d + c];
+            x[n] = sacc;
+        }
+        // forward: block logits and the common shift
+        double m = -INFINITY;
+        for (long j = 0; j < nblk; ++j) {
+            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+            if (sel) {
+                for (long n = j * B; n < (j + 1) * B; ++n) m = std::max(m, x[n]);
+                continue;
+            }
+            double sb = 0.0;
+            for (long c = 0; c < d; ++c) sb += (double)qt[c] * kbar[j * d + c];
+            double w = 0.0;
+            if (order == 2) {
+                for (long n = j * B; n < (j + 1) * B; ++n) w += (x[n] - sb) * (x[n] - sb);
+                w /= 2.0 * (double)B;
+            }
+            open[j] = !(gate && w > ln_b);
+            if (!open[j]) w = 0.0;
+            sbj[j] = sb;
+            wj[j] = w;
+            lj[j] = sb + w;
+            m = std::max(m, lj[j]);
+        }
+        double D = 0.0;
+        std::fill(o.begin(), o.end(), 0.0);
+        for (long j = 0; j < nblk; ++j) {
+            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+            for (long n = j * B; n < (j + 1) * B; ++n) {
+                wt[n] = sel ? std::exp(x[n] - m) : std::exp(lj[j] - m) * (1.0 + c1 * (x[n] - sbj[j]));
+                for (long c = 0; c < d; ++c) o[c] += wt[n] * (double)v[n * d + c];
+            }
+            D += sel ? 0.0 : (double)B * std::exp(lj[j] - m);
+            if (sel)
+                for (long n = j * B; n < (j + 1) * B; ++n) D += wt[n];
+        }
+        for (long c = 0; c < d; ++c) o[c] /= D;
+        const float* dOt = dO + t * d;
+        double delta = 0.0;
+        for (long c = 0; c < d; ++c) delta += (double)dOt[c] * o[c];
+        for (long n = 0; n < L; ++n) {
+            double g = 0.0;
+            for (long c = 0; c < d; ++c) g += (double)dOt[c] * (double)v[n * d + c];
+            G[n] = g;
+        }
+        // dL/dx
+        for (long j = 0; j < nblk; ++j) {
+            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+            if (sel) {
+                for (long n = j * B; n < (j + 1) * B; ++n) gx[n] = wt[n] * (G[n] - delta) / D;
+                continue;
+            }
+            const double E = std::exp(lj[j] - m);
+            double sg = 0.0, gbar = 0.0;
+            for (long n = j * B; n < (j + 1) * B; ++n) {
+                sg += G[n] * (1.0 + c1 * (x[n] - sbj[j]));
+                gbar += G[n];
+            }
+            gbar /= (double)B;
+            const double inner = sg - (double)B * delta;
+            for (long n = j * B; n < (j + 1) * B; ++n) {
+                double dl = 1.0 / (double)B;
+                if (order == 2 && open[j]) dl += (x[n] - sbj[j]) / (double)B;
+                gx[n] = (E / D) * (dl * inner + c1 * (G[n] - gbar));
+            }
+        }
+        for (long n = 0; n < L; ++n) {
+            for (long c = 0; c < d; ++c) {
+                dq[t * d + c] += gx[n] * (double)k[n * d + c];
+                dk[n * d + c] += gx[n] * (double)qt[c];
+                dv[n * d + c] += (wt[n] / D) * (double)dOt[c];
+            }
+        }
+    }
+}
+
 template <class F>
 void parallel_for(long n, int nthreads, F&& fn) {
     if (nthreads <= 1 || n <= 1) {
@@ -617,6 +729,22 @@ int oracle_pisa_bruteforce(const float* q, const float* k, const float* v, long 
                           sel.data(), order, gate, out + (bh * L + t) * d);
             }
         }
+    });
+    return 0;
+}
+
+// Gradients (dq, dk, dv) [BH, L, d] fp64 of sum_t dO_t . o_t for the method's
+// output o (pisa_attention's), selection held fixed.  Zero-initialised here.
+int oracle_pisa_backward(const float* q, const float* k, const float* v, const float* dO, long BH, long L, long d,
+                         long B, long K, int order, int gate, double* dq, double* dk, double* dv, int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
+    if (K < 0 || K > L / B) return -1;
+    std::fill(dq, dq + BH * L * d, 0.0);
+    std::fill(dk, dk + BH * L * d, 0.0);
+    std::fill(dv, dv + BH * L * d, 0.0);
+    parallel_for(BH, nthreads, [&](long bh) {
+        const long o = bh * L * d;
+        backward_one(q + o, k + o, v + o, dO + o, L, d, B, K, order, gate, dq + o, dk + o, dv + o);
     });
     return 0;
 }

@@ -540,3 +540,80 @@ def test_routed_attention_matches_dense_when_every_block_is_selected():
     B = 16
     got = oracle.pisa_attention_ex(q, k, v, B, 256 // B, 1, route_eps=1e-6)
     np.testing.assert_allclose(got, oracle.dense_attention(q, k, v), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Gradients (the backward pass; the pages print no equations, the oracle's
+# are derived from its forward with the selection held fixed)
+# --------------------------------------------------------------------------
+
+
+def _dyadic_qkv(seed, L, d):
+    rng = np.random.default_rng(seed)
+    return tuple((rng.integers(-64, 65, (1, L, d)) / 64.0).astype(np.float32) for _ in range(3))
+
+
+@pytest.mark.parametrize("order,gate", [(0, True), (1, True), (2, False), (2, True)])
+def test_backward_matches_central_differences(order, gate):
+    # dyadic inputs and step 2^-10 keep every perturbed input exact in fp32; the
+    # loss is sum(dO . o) in fp64; coordinates whose perturbation changes the
+    # (fixed) selection are skipped
+    L, d, B, K = 64, 4, 16, 2
+    q, k, v = _dyadic_qkv(61 + order, L, d)
+    q *= 2.0
+    dO = _dyadic_qkv(67, L, d)[0]
+    gq, gk, gv = oracle.pisa_backward(q, k, v, dO, B, K, order, gate)
+    _, mask0, _ = oracle.select(q, k, B, K)
+    h = 2.0 ** -10
+
+    def loss(q_, k_, v_):
+        return float((oracle.pisa_attention(q_, k_, v_, B, K, order, gate=gate) * dO).sum())
+
+    rng = np.random.default_rng(5)
+    checked = 0
+    for name, x, g in (("q", q, gq), ("k", k, gk), ("v", v, gv)):
+        for _ in range(20):
+            idx = (0, int(rng.integers(L)), int(rng.integers(d)))
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            if name != "v" and not (np.array_equal(oracle.select(args_p[0], args_p[1], B, K)[1], mask0) and
+                                    np.array_equal(oracle.select(args_m[0], args_m[1], B, K)[1], mask0)):
+                continue
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - g[idx]) <= 2e-5 * max(1.0, abs(g[idx])), (name, idx, fd, g[idx])
+            checked += 1
+    assert checked >= 40
+
+
+def test_backward_with_every_block_selected_is_the_dense_gradient():
+    # K = all blocks: the method is dense softmax attention; its gradient from
+    # torch autograd in fp64 (a library, independent of the derivation)
+    L, d, B = 64, 8, 16
+    q, k, v = small(71, BH=2, L=L, d=d, scale=1.5)
+    dO = small(72, BH=2, L=L, d=d)[0]
+    gq, gk, gv = oracle.pisa_backward(q, k, v, dO, B, L // B, 1)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.softmax(tq @ tk.transpose(1, 2), dim=-1) @ tv
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    for g, t in ((gq, tq), (gk, tk), (gv, tv)):
+        np.testing.assert_allclose(g, t.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_backward_order0_identical_keys_is_exact_attention_gradient_for_v():
+    # identical keys in every block: every unselected block's virtual token is
+    # exact, so the output equals dense attention and dv does too (dv is linear
+    # in the weights, which match exactly)
+    L, d, B, K = 64, 8, 16, 1
+    rng = np.random.default_rng(73)
+    k = np.repeat(rng.standard_normal((1, L // B, 1, d)), B, axis=2).reshape(1, L, d).astype(np.float32)
+    q = rng.standard_normal((1, L, d)).astype(np.float32)
+    v = rng.standard_normal((1, L, d)).astype(np.float32)
+    dO = rng.standard_normal((1, L, d)).astype(np.float32)
+    _, _, gv = oracle.pisa_backward(q, k, v, dO, B, K, 0)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.softmax(tq @ tk.transpose(1, 2), dim=-1) @ tv
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    np.testing.assert_allclose(gv, tv.grad.numpy(), rtol=0, atol=1e-11)
