@@ -23,8 +23,9 @@
 //      the CTA's union (already counted in step 1) or past nblk;
 //   3. epilogue: G = Q H-bar^T on the tensor cores into the freed S columns,
 //      o_t = (O_t + A_t G_t) / D_t with A_t = sum_{j in U_i} alpha_tj.
-// Pipeline, TMEM plan, warp roles, lazy running max and bounded waits are those
-// of the token-form kernel (attn_tc.cuh).
+// Pipeline, TMEM plan, warp roles, lazy running max, bounded waits and the
+// hand-over of P in two halves of 64 keys are those of the token-form kernel
+// (attn_tc.cuh).
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -49,7 +50,7 @@ struct HybCfg {
     static constexpr uint32_t K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr uint32_t BAR_OFF = V_OFF + NS * TILE_BYTES;
-    static constexpr uint32_t NBAR = 1 + 4 * NS + 2 + 2 + 2 + 1 + 1;
+    static constexpr uint32_t NBAR = 1 + 4 * NS + 2 + 2 + 2 + 2 + 1 + 1;
     static constexpr uint32_t SCHED_OFF = BAR_OFF + NBAR * 8 + 16;
     static constexpr int NQT = 256 / BS;  // query tiles per CTA
     static constexpr int MAXBLK = 4096;   // schedule capacity (nblk limit of the library)
@@ -87,8 +88,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint16_t* blist = (uint16_t*)(qwords + C::NQT * 128);         // [MAXBLK] union blocks ascending
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS;
-    const int B_SFULL = 1 + 4 * C::NS, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_DONE = B_OFULL + 2;
-    const int B_HFULL = B_DONE + 1;
+    const int B_SFULL = 1 + 4 * C::NS, B_PHALF = B_SFULL + 2, B_PFULL = B_PHALF + 2, B_OFULL = B_PFULL + 2;
+    const int B_DONE = B_OFULL + 2, B_HFULL = B_DONE + 1;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int bh = blockIdx.y;
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         for (int h = 0; h < 2; ++h) {
             tc::mbar_init(bar(B_SFULL + h), 1);
+            tc::mbar_init(bar(B_PHALF + h), 128);
             tc::mbar_init(bar(B_PFULL + h), 128);
             tc::mbar_init(bar(B_OFULL + h), 1);
         }
@@ -249,9 +251,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                idesc, kk > 0);
                 }
             };
-            auto issue_pv = [&](int h, int st, bool first) {
+            auto issue_pv = [&](int h, int st, int half, bool first) {
 #pragma unroll
-                for (int kk = 0; kk < C::NK / 16; ++kk)
+                for (int kk = half * 4; kk < half * 4 + 4; ++kk)
                     tc::mma_ts(tmem + C::O_COL0 + h * D, tmem + (uint32_t)(h * 128) + kk * 8,
                                vdesc0 + st * kTileStep + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O,
                                (first && kk == 0) ? 0u : 1u);
@@ -270,17 +272,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int st1 = (jt + 1) % C::NS, u1 = (jt + 1) / C::NS;
                 const bool more = jt + 1 < NT;
                 if (!tc::mbar_wait(bar(B_VFULL + st), u & 1, aborted, status, kWaitLimitCycles)) break;
+                if (!tc::mbar_wait(bar(B_PHALF + 0), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(0, st, 0, jt == 0);
                 if (!tc::mbar_wait(bar(B_PFULL + 0), jt & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_pv(0, st, jt == 0);
+                issue_pv(0, st, 1, false);
                 if (more) {
                     if (!tc::mbar_wait(bar(B_KFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
                     issue_s(0, st1, IDESC_S);
                     tc::mma_commit(bar(B_SFULL + 0));
                 }
+                if (!tc::mbar_wait(bar(B_PHALF + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_pv(1, st, 0, jt == 0);
                 if (!tc::mbar_wait(bar(B_PFULL + 1), jt & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_pv(1, st, jt == 0);
+                issue_pv(1, st, 1, false);
                 if (!kSfullRelease) tc::mma_commit(bar(B_VEMPTY + st));
                 if (more) {
                     issue_s(1, st1, IDESC_S);
@@ -426,6 +434,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 pk[e] = tc::pack_bf16x2(a0, a1);
                             }
                             tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                            if (b * CPB + c == 1) {  // keys 0..63 are in TMEM: hand over the first half
+                                tc::tmem_wait_st();
+                                tc::fence_before_sync();
+                                tc::mbar_arrive(bar(B_PHALF + h));
+                            }
                         }
                         dsum += (d4[0] + d4[1]) + (d4[2] + d4[3]);
                     } else {
@@ -438,7 +451,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = a2;
 #pragma unroll
-                        for (int c = 0; c < CPB; ++c) tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                        for (int c = 0; c < CPB; ++c) {
+                            tc::tmem_st16(s_addr + (b * CPB + c) * 16, pk);
+                            if (b * CPB + c == 1) {
+                                tc::tmem_wait_st();
+                                tc::fence_before_sync();
+                                tc::mbar_arrive(bar(B_PHALF + h));
+                            }
+                        }
                     }
                 }
             } else {
@@ -458,6 +478,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         pk[e] = tc::pack_bf16x2(a0, a1);
                     }
                     tc::tmem_st16(s_addr + c * 16, pk);
+                    if (c == 1) {
+                        tc::tmem_wait_st();
+                        tc::fence_before_sync();
+                        tc::mbar_arrive(bar(B_PHALF + h));
+                    }
                 }
                 const float asum = (a4[0] + a4[1]) + (a4[2] + a4[3]);
                 dsum = fmaf((float)BS, asum, dsum);
