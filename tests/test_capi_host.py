@@ -104,3 +104,36 @@ def test_stats_bind_layout():
                                pisa.PISA_BF16) == pisa.PISA_ERR_INVALID_ARG
     assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n, 2, 3, 1024, 64, 64, 1, pisa.PISA_BF16) == 0
     assert st.cov is None
+
+
+def test_routing_and_score_entry_points_reject_bad_arguments():
+    lib = pisa.lib()
+    bf = pisa.PISA_BF16
+    # eps outside [1e-30, 1e30], null pointers, a bad shape: rejected before any CUDA call
+    for eps in (0.0, -1.0, 1e31, float("nan")):
+        assert lib.pisa_route_bias(FAKE, FAKE, FAKE, 1, 1, 1024, 64, bf, 64, eps, FAKE, None) == \
+            pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_route_bias(None, FAKE, FAKE, 1, 1, 1024, 64, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_route_bias(FAKE, FAKE, FAKE, 1, 1, 1000, 64, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_route_bias(FAKE, FAKE, FAKE, 1, 1, 1024, 96, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_UNSUPPORTED
+    st = pisa._StatsT(1, 1, 1024, 64, 64, 16, 0, bf, FAKE.value, None, None, None)
+    assert lib.pisa_select_scores(FAKE, ctypes.byref(st), None, None, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_select_scores(None, ctypes.byref(st), None, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_select_biased(FAKE, ctypes.byref(st), 17, FAKE, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_select_biased(FAKE, ctypes.byref(st), 4, FAKE, None, None, None) == pisa.PISA_ERR_INVALID_ARG
+    assert lib.pisa_select_scores(FAKE, None, None, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+
+
+def test_binding_flags():
+    assert pisa._flags(True, "exact", "centroid") == pisa.FLAG_GATE_W
+    assert pisa._flags(False, "pooled", "cov") == pisa.FLAG_POOLED_W | pisa.FLAG_COV_ROUTE
+    for bad in (("exact", "nope"), ("nope", "centroid")):
+        with pytest.raises(ValueError):
+            pisa._flags(True, *bad)
+
+
+def test_workspace_holds_the_routing_bias():
+    # the routing bias is part of every workspace: enabling the flag never needs more
+    for path in ("recompute_tc", "hybrid_tc", "stats"):
+        n = pisa.pisa_workspace_bytes(1, 2, 2048, 128, 64, 8, 1, pisa.torch.bfloat16, path)
+        assert n > 2 * (2048 // 64) * 4
