@@ -409,100 +409,125 @@ void row_brute(const float* qrow, const float* k, const float* v, long d, long B
 //   dq_t = sum_n dL/dx_tn k_n,  dk_n = sum_t dL/dx_tn q_t,
 //   dv_n = sum_t (weight_tn / D_t) dO_t  (weight = the numerator's e^{x} or E (1 + c1 u_n)).
 // Evaluated with the common max shift m (it cancels in weight / D).
-void backward_one(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B, long K,
-                  int order, int gate, double* dq, double* dk, double* dv) {
+// Selection mask and fp64 centroids of one (batch, head), as the forward
+// forms them (route_eps > 0: the covariance-aware selection).
+void backward_prep(const float* q, const float* k, const float* v, long L, long d, long B, long K,
+                   float route_eps, std::vector<uint32_t>& mask, std::vector<double>& kbar) {
     const long nblk = L / B;
     const long words = (nblk + 31) / 32;
-    std::vector<uint32_t> mask(nblk * words, 0u);
-    select_one(q, k, L, d, B, K, nullptr, mask.data(), nullptr);
-    std::vector<double> kbar(nblk * d, 0.0);
+    mask.assign(nblk * words, 0u);
+    std::vector<float> rbias;
+    if (route_eps > 0.0f) {
+        rbias.resize(nblk);
+        route_bias_one(k, v, L, d, B, route_eps, rbias.data());
+    }
+    select_one(q, k, L, d, B, K, nullptr, mask.data(), nullptr, rbias.empty() ? nullptr : rbias.data());
+    kbar.assign(nblk * d, 0.0);
     for (long j = 0; j < nblk; ++j)
         for (long c = 0; c < d; ++c) {
             double sacc = 0.0;
             for (long n = 0; n < B; ++n) sacc += (double)k[(j * B + n) * d + c];
             kbar[j * d + c] = sacc / (double)B;
         }
+}
+
+// Query row t: gx[n] = dL/dx_n over all L keys (x_n = q_t.k_n) and pw[n] =
+// wt_n / D, the normalised weight of key n in o_t, with the selection (and
+// the gate decision) held fixed.
+void backward_row(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B,
+                  const uint32_t* mask, const double* kbar, int order, int gate, long t, double* gx, double* pw) {
+    const long nblk = L / B;
+    const long words = (nblk + 31) / 32;
+    const long i = t / B;
+    const float* qt = q + t * d;
     const double ln_b = std::log((double)B);
     const int c1 = order >= 1 ? 1 : 0;
-    std::vector<double> x(L), wt(L), lj(nblk), wj(nblk), sbj(nblk), o(d), G(L), gx(L);
+    std::vector<double> x(L), wt(L), lj(nblk), sbj(nblk), o(d, 0.0), G(L);
     std::vector<char> open(nblk);
+    for (long n = 0; n < L; ++n) {
+        double sacc = 0.0;
+        for (long c = 0; c < d; ++c) sacc += (double)qt[c] * (double)k[n * d + c];
+        x[n] = sacc;
+    }
+    // forward: block logits and the common shift
+    double m = -INFINITY;
+    for (long j = 0; j < nblk; ++j) {
+        const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+        if (sel) {
+            for (long n = j * B; n < (j + 1) * B; ++n) m = std::max(m, x[n]);
+            continue;
+        }
+        double sb = 0.0;
+        for (long c = 0; c < d; ++c) sb += (double)qt[c] * kbar[j * d + c];
+        double w = 0.0;
+        if (order == 2) {
+            for (long n = j * B; n < (j + 1) * B; ++n) w += (x[n] - sb) * (x[n] - sb);
+            w /= 2.0 * (double)B;
+        }
+        open[j] = !(gate && w > ln_b);
+        if (!open[j]) w = 0.0;
+        sbj[j] = sb;
+        lj[j] = sb + w;
+        m = std::max(m, lj[j]);
+    }
+    double D = 0.0;
+    for (long j = 0; j < nblk; ++j) {
+        const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+        for (long n = j * B; n < (j + 1) * B; ++n) {
+            wt[n] = sel ? std::exp(x[n] - m) : std::exp(lj[j] - m) * (1.0 + c1 * (x[n] - sbj[j]));
+            for (long c = 0; c < d; ++c) o[c] += wt[n] * (double)v[n * d + c];
+        }
+        D += sel ? 0.0 : (double)B * std::exp(lj[j] - m);
+        if (sel)
+            for (long n = j * B; n < (j + 1) * B; ++n) D += wt[n];
+    }
+    for (long c = 0; c < d; ++c) o[c] /= D;
+    const float* dOt = dO + t * d;
+    double delta = 0.0;
+    for (long c = 0; c < d; ++c) delta += (double)dOt[c] * o[c];
+    for (long n = 0; n < L; ++n) {
+        double g = 0.0;
+        for (long c = 0; c < d; ++c) g += (double)dOt[c] * (double)v[n * d + c];
+        G[n] = g;
+        pw[n] = wt[n] / D;
+    }
+    // dL/dx
+    for (long j = 0; j < nblk; ++j) {
+        const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
+        if (sel) {
+            for (long n = j * B; n < (j + 1) * B; ++n) gx[n] = wt[n] * (G[n] - delta) / D;
+            continue;
+        }
+        const double E = std::exp(lj[j] - m);
+        double sg = 0.0, gbar = 0.0;
+        for (long n = j * B; n < (j + 1) * B; ++n) {
+            sg += G[n] * (1.0 + c1 * (x[n] - sbj[j]));
+            gbar += G[n];
+        }
+        gbar /= (double)B;
+        const double inner = sg - (double)B * delta;
+        for (long n = j * B; n < (j + 1) * B; ++n) {
+            double dl = 1.0 / (double)B;
+            if (order == 2 && open[j]) dl += (x[n] - sbj[j]) / (double)B;
+            gx[n] = (E / D) * (dl * inner + c1 * (G[n] - gbar));
+        }
+    }
+}
+
+void backward_one(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B, long K,
+                  int order, int gate, float route_eps, double* dq, double* dk, double* dv) {
+    std::vector<uint32_t> mask;
+    std::vector<double> kbar, gx(L), pw(L);
+    backward_prep(q, k, v, L, d, B, K, route_eps, mask, kbar);
     for (long t = 0; t < L; ++t) {
-        const long i = t / B;
+        backward_row(q, k, v, dO, L, d, B, mask.data(), kbar.data(), order, gate, t, gx.data(), pw.data());
         const float* qt = q + t * d;
-        for (long n = 0; n < L; ++n) {
-            double sacc = 0.0;
-            for (long c = 0; c < d; ++c) sacc += (double)qt[c] * (double)k[n * d + c];
-            x[n] = sacc;
-        }
-        // forward: block logits and the common shift
-        double m = -INFINITY;
-        for (long j = 0; j < nblk; ++j) {
-            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
-            if (sel) {
-                for (long n = j * B; n < (j + 1) * B; ++n) m = std::max(m, x[n]);
-                continue;
-            }
-            double sb = 0.0;
-            for (long c = 0; c < d; ++c) sb += (double)qt[c] * kbar[j * d + c];
-            double w = 0.0;
-            if (order == 2) {
-                for (long n = j * B; n < (j + 1) * B; ++n) w += (x[n] - sb) * (x[n] - sb);
-                w /= 2.0 * (double)B;
-            }
-            open[j] = !(gate && w > ln_b);
-            if (!open[j]) w = 0.0;
-            sbj[j] = sb;
-            wj[j] = w;
-            lj[j] = sb + w;
-            m = std::max(m, lj[j]);
-        }
-        double D = 0.0;
-        std::fill(o.begin(), o.end(), 0.0);
-        for (long j = 0; j < nblk; ++j) {
-            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
-            for (long n = j * B; n < (j + 1) * B; ++n) {
-                wt[n] = sel ? std::exp(x[n] - m) : std::exp(lj[j] - m) * (1.0 + c1 * (x[n] - sbj[j]));
-                for (long c = 0; c < d; ++c) o[c] += wt[n] * (double)v[n * d + c];
-            }
-            D += sel ? 0.0 : (double)B * std::exp(lj[j] - m);
-            if (sel)
-                for (long n = j * B; n < (j + 1) * B; ++n) D += wt[n];
-        }
-        for (long c = 0; c < d; ++c) o[c] /= D;
         const float* dOt = dO + t * d;
-        double delta = 0.0;
-        for (long c = 0; c < d; ++c) delta += (double)dOt[c] * o[c];
-        for (long n = 0; n < L; ++n) {
-            double g = 0.0;
-            for (long c = 0; c < d; ++c) g += (double)dOt[c] * (double)v[n * d + c];
-            G[n] = g;
-        }
-        // dL/dx
-        for (long j = 0; j < nblk; ++j) {
-            const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
-            if (sel) {
-                for (long n = j * B; n < (j + 1) * B; ++n) gx[n] = wt[n] * (G[n] - delta) / D;
-                continue;
-            }
-            const double E = std::exp(lj[j] - m);
-            double sg = 0.0, gbar = 0.0;
-            for (long n = j * B; n < (j + 1) * B; ++n) {
-                sg += G[n] * (1.0 + c1 * (x[n] - sbj[j]));
-                gbar += G[n];
-            }
-            gbar /= (double)B;
-            const double inner = sg - (double)B * delta;
-            for (long n = j * B; n < (j + 1) * B; ++n) {
-                double dl = 1.0 / (double)B;
-                if (order == 2 && open[j]) dl += (x[n] - sbj[j]) / (double)B;
-                gx[n] = (E / D) * (dl * inner + c1 * (G[n] - gbar));
-            }
-        }
         for (long n = 0; n < L; ++n) {
             for (long c = 0; c < d; ++c) {
                 dq[t * d + c] += gx[n] * (double)k[n * d + c];
                 dk[n * d + c] += gx[n] * (double)qt[c];
-                dv[n * d + c] += (wt[n] / D) * (double)dOt[c];
+                dv[n * d + c] += pw[n] * (double)dOt[c];
             }
         }
     }
@@ -736,7 +761,8 @@ int oracle_pisa_bruteforce(const float* q, const float* k, const float* v, long 
 // Gradients (dq, dk, dv) [BH, L, d] fp64 of sum_t dO_t . o_t for the method's
 // output o (pisa_attention's), selection held fixed.  Zero-initialised here.
 int oracle_pisa_backward(const float* q, const float* k, const float* v, const float* dO, long BH, long L, long d,
-                         long B, long K, int order, int gate, double* dq, double* dk, double* dv, int nthreads) {
+                         long B, long K, int order, int gate, float route_eps, double* dq, double* dk, double* dv,
+                         int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     if (K < 0 || K > L / B) return -1;
     std::fill(dq, dq + BH * L * d, 0.0);
@@ -744,7 +770,39 @@ int oracle_pisa_backward(const float* q, const float* k, const float* v, const f
     std::fill(dv, dv + BH * L * d, 0.0);
     parallel_for(BH, nthreads, [&](long bh) {
         const long o = bh * L * d;
-        backward_one(q + o, k + o, v + o, dO + o, L, d, B, K, order, gate, dq + o, dk + o, dv + o);
+        backward_one(q + o, k + o, v + o, dO + o, L, d, B, K, order, gate, route_eps, dq + o, dk + o, dv + o);
+    });
+    return 0;
+}
+
+// dq of a list of query rows: rows[2*r] = bh, rows[2*r+1] = t; dq_rows
+// receives [nrows, d] fp64 (the rows of oracle_pisa_backward's dq).
+int oracle_pisa_backward_dq_rows(const float* q, const float* k, const float* v, const float* dO, long BH, long L,
+                                 long d, long B, long K, int order, int gate, float route_eps, const int64_t* rows,
+                                 long nrows, double* dq_rows, int nthreads) {
+    if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
+    if (K < 0 || K > L / B) return -1;
+    for (long r = 0; r < nrows; ++r)
+        if (rows[2 * r] < 0 || rows[2 * r] >= BH || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= L) return -1;
+    std::vector<std::vector<uint32_t>> mask(BH);
+    std::vector<std::vector<double>> kbar(BH);
+    std::vector<char> used(BH, 0);
+    for (long r = 0; r < nrows; ++r) used[rows[2 * r]] = 1;
+    parallel_for(BH, nthreads, [&](long bh) {
+        if (used[bh])
+            backward_prep(q + bh * L * d, k + bh * L * d, v + bh * L * d, L, d, B, K, route_eps, mask[bh], kbar[bh]);
+    });
+    parallel_for(nrows, nthreads, [&](long r) {
+        const long bh = rows[2 * r], t = rows[2 * r + 1];
+        const long o = bh * L * d;
+        std::vector<double> gx(L), pw(L);
+        backward_row(q + o, k + o, v + o, dO + o, L, d, B, mask[bh].data(), kbar[bh].data(), order, gate, t,
+                     gx.data(), pw.data());
+        for (long c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (long n = 0; n < L; ++n) acc += gx[n] * (double)k[o + n * d + c];
+            dq_rows[r * d + c] = acc;
+        }
     });
     return 0;
 }

@@ -617,3 +617,71 @@ def test_backward_order0_identical_keys_is_exact_attention_gradient_for_v():
     o = torch.softmax(tq @ tk.transpose(1, 2), dim=-1) @ tv
     (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
     np.testing.assert_allclose(gv, tv.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_backward_with_routing_matches_central_differences():
+    # covariance-aware selection (PISA paper section 3.3; PWT section of the
+    # "Sparse Linear Attention" blog): the routing only picks the blocks, so the
+    # gradient is the same formula on the routed selection; coordinates whose
+    # perturbation changes the routed selection are skipped
+    L, d, B, K = 64, 4, 16, 2
+    eps = 1e-6
+    q, k, v = _dyadic_qkv(81, L, d)
+    q *= 2.0
+    v[:, 16:32] *= 4.0  # a block with a large ||H_j||: routing changes the selection
+    dO = _dyadic_qkv(83, L, d)[0]
+    gq, gk, gv = oracle.pisa_backward(q, k, v, dO, B, K, 1, True, route_eps=eps)
+
+    def rmask(q_, k_, v_):
+        return oracle.select(q_, k_, B, K, bias=oracle.route_bias(k_, v_, B, eps))[1]
+
+    mask0 = rmask(q, k, v)
+    assert not np.array_equal(mask0, oracle.select(q, k, B, K)[1])
+    # the plain backward on other blocks differs: routing reaches the gradient
+    assert oracle.rel_l2(oracle.pisa_backward(q, k, v, dO, B, K, 1)[0], gq) > 1e-3
+    h = 2.0 ** -10
+
+    def loss(q_, k_, v_):
+        return float((oracle.pisa_attention_ex(q_, k_, v_, B, K, 1, route_eps=eps) * dO).sum())
+
+    rng = np.random.default_rng(7)
+    checked = 0
+    for name, x, g in (("q", q, gq), ("k", k, gk), ("v", v, gv)):
+        for _ in range(20):
+            idx = (0, int(rng.integers(L)), int(rng.integers(d)))
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            if not (np.array_equal(rmask(*args_p), mask0) and np.array_equal(rmask(*args_m), mask0)):
+                continue
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - g[idx]) <= 2e-5 * max(1.0, abs(g[idx])), (name, idx, fd, g[idx])
+            checked += 1
+    assert checked >= 40
+
+
+@pytest.mark.parametrize("order,gate", [(0, True), (1, True), (2, True), (2, False)])
+def test_backward_identities(order, gate):
+    # Two exact identities of the method (PISA paper section 3.2 with the
+    # blog's Taylor terms): adding one vector to every key shifts each row's
+    # logits x_n, the centroid score and l_tj by the same amount (u_n and w
+    # do not change), so o is unchanged and sum_n dk_n = 0; and each row's
+    # weights sum to D (sum_n u_n = 0 within a block), so sum_n dv_n = sum_t dO_t.
+    q, k, v = small(91 + order, BH=2, L=256, d=16, scale=3.0)
+    dO = small(97, BH=2, L=256, d=16)[0]
+    _, gk, gv = oracle.pisa_backward(q, k, v, dO, 32, 3, order, gate)
+    scale = np.abs(gk).sum(axis=1)
+    assert np.all(np.abs(gk.sum(axis=1)) <= 1e-12 * scale + 1e-13)
+    np.testing.assert_allclose(gv.sum(axis=1), dO.astype(np.float64).sum(axis=1), rtol=0, atol=1e-11)
+
+
+def test_backward_dq_rows_are_the_full_backward_rows():
+    q, k, v = small(101, BH=2, L=256, d=16, scale=2.0)
+    dO = small(103, BH=2, L=256, d=16)[0]
+    for order, reps in ((1, None), (2, None), (1, 1e-6)):
+        gq, _, _ = oracle.pisa_backward(q, k, v, dO, 32, 2, order, True, route_eps=reps)
+        rows = [(0, 0), (0, 31), (1, 32), (1, 200), (0, 255)]
+        got = oracle.pisa_backward_dq_rows(q, k, v, dO, 32, 2, rows, order, True, route_eps=reps)
+        np.testing.assert_array_equal(got, np.stack([gq[b, t] for b, t in rows]))
