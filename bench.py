@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--heads", type=int, default=None, help="override head count (profiling small cases)")
     p.add_argument("--no-hybrid", action="store_true", help="skip the PISA-hybrid (global H-bar) record")
     p.add_argument("--no-route", action="store_true", help="skip the covariance-aware routing record")
+    p.add_argument("--no-backward", action="store_true", help="skip the backward-pass record")
     return p.parse_args()
 
 
@@ -455,6 +456,44 @@ def main():
                       "speedup_vs_per_block_path": ms_step / h_ms, "launches_per_call": 5}
         del hws, hout
 
+    # The backward pass (training use) on the same inputs: dq, dk, dv of
+    # sum(dO * o) for the forward output o above, selection held fixed; timed
+    # as whole calls (centroids, selection, row statistics, dq, dk/dv).
+    bwd_rec = None
+    if not args.no_backward:
+        gen = torch.Generator(device="cuda").manual_seed(4321 + rank)
+        dO = torch.randn(q.shape, generator=gen, device="cuda", dtype=torch.float32).to(tdt)
+        grads = tuple(torch.empty(q.shape, dtype=torch.float32, device="cuda") for _ in range(3))
+        bws = torch.empty(pisa.pisa_backward_workspace_bytes(1, BH, L, d, B, K, order, tdt), dtype=torch.uint8,
+                          device="cuda")
+        pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws)
+        torch.cuda.synchronize()
+        pisa.pisa_poll_device_status()
+        ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 2
+        ba.record(stream)
+        for _ in range(reps):
+            pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws)
+        bb.record(stream)
+        torch.cuda.synchronize()
+        pisa.pisa_poll_device_status()
+        b_ms = ba.elapsed_time(bb) / reps
+        alg = 10.0 * L * L * d * BH       # S, dP, dq, dk, dv once each (five products of 2 L^2 d)
+        executed = 16.0 * L * L * d * BH  # S in all three kernels and dP in two are recomputed
+        bf16_peak = float(peaks["bf16_tflops"])
+        bwd_rec = {"kernels": [f"bwd_rowstat_kernel<{d},{B}>", f"bwd_dq_kernel<{d},{B}>",
+                               f"bwd_dkdv_kernel<{d},{B}>"],
+                   "ms_per_call": b_ms, "algorithmic_flops_per_call": alg,
+                   "algorithmic_tflops": alg / (b_ms * 1e-3) / 1e12,
+                   "executed_tflops": executed / (b_ms * 1e-3) / 1e12,
+                   "roofline": {"bound": "tensor", "peak": bf16_peak, "unit": "TFLOP/s",
+                                "frac": alg / (b_ms * 1e-3) / 1e12 / bf16_peak,
+                                "peak_source": f"{peak_kind} bf16 dense (burst)"},
+                   "tile_products": ("warp-level mma.sync m16n8k16, bf16 operands, fp32 accumulation"
+                                     if tdt == torch.bfloat16 else "fp32 FMA"),
+                   "launches_per_call": 5}
+        del dO, grads, bws
+
     # end to end through the public host-buffer call: pisa_attention_host on
     # pinned host q, k, v, out (per chunk of heads: H2D copies, the attention,
     # D2H copy; two streams so that the copies overlap the kernels)
@@ -512,6 +551,7 @@ def main():
             "stats_kernel": stats_rec,
             "hybrid": hybrid_rec,
             "routing": route_rec,
+            "backward": bwd_rec,
             "cpu_baseline": cpu,
             "clocks": clk,
             "e2e": e2e,

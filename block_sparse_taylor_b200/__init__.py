@@ -15,6 +15,8 @@ The functions carry the names of the C entry points:
 * ``pisa_attention(q, k, v, B, K, order)``: the full forward pass of piecewise
   sparse attention (PISA paper section 3.2; "Sparse Linear Attention" blog,
   PWT section for order 2).
+* ``pisa_attention_backward(q, k, v, o, dO, B, K, order)``: dq, dk, dv of that
+  forward with the block selection held fixed.
 
 Tensors are [batch*heads, L, d] (or [batch, heads, L, d]) contiguous CUDA
 tensors of dtype float32 or bfloat16; q must already be multiplied by
@@ -94,6 +96,10 @@ def lib():
         L.pisa_attention_host_bytes.argtypes = [i, i, i, i, i, i, i, i, i, i]
         L.pisa_attention_host_bytes.restype = sz
         L.pisa_noalloc_scratch_bytes.restype = sz
+        L.pisa_attention_backward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
+        L.pisa_attention_backward.restype = ctypes.c_int
+        L.pisa_backward_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+        L.pisa_backward_workspace_bytes.restype = sz
         for fn in ("pisa_attention_noalloc", "pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
                    "pisa_poll_device_status", "pisa_resolve_path"):
             getattr(L, fn).restype = ctypes.c_int
@@ -309,6 +315,41 @@ def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K:
                                    PATHS[path], out.data_ptr(), workspace.data_ptr(),
                                    workspace.numel(), _stream(stream)))
     return out
+
+
+def pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, dtype: torch.dtype) -> int:
+    return int(lib().pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, _dtype_code(dtype)))
+
+
+def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
+                            B: int, K: int, order: int = 1, gate: bool = True, route: str = "centroid",
+                            grads: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """(dq, dk, dv) fp32, the gradients of sum(dO * o) for o = pisa_attention(q, k, v, B, K, order,
+    gate=gate, route=route) on the per-block paths, the selection held fixed.  ``o`` is that
+    forward's output; ``grads`` optional preallocated fp32 (dq, dk, dv)."""
+    _need_cuda(q, k, v, o, dO)
+    if not (q.shape == k.shape == v.shape == o.shape == dO.shape
+            and q.dtype == k.dtype == v.dtype == o.dtype == dO.dtype):
+        raise ValueError("q, k, v, o, dO must share shape and dtype")
+    batch, heads, L, d = _shape(q)
+    code = _dtype_code(q.dtype)
+    if grads is None:
+        grads = tuple(torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
+    for g in grads:
+        _need_cuda(g)
+        if g.dtype != torch.float32 or g.shape != q.shape:
+            raise ValueError("grads must be fp32 tensors of q's shape")
+    nbytes = pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, q.dtype)
+    if nbytes == 0:
+        raise PisaError(PISA_ERR_INVALID_ARG, "no backward workspace size for these arguments")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = grads
+    _check(lib().pisa_attention_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(),
+                                         batch, heads, L, d, code, B, K, order, _flags(gate, "exact", route),
+                                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def pisa_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,

@@ -21,6 +21,7 @@
 #include "hybrid_prep.cuh"
 #include "attn_hybrid.cuh"
 #include "route.cuh"
+#include "backward.cuh"
 
 using pisa::bf16;
 
@@ -331,6 +332,63 @@ pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
     return tc_path_available(g, dtype) ? PISA_PATH_RECOMPUTE_TC : PISA_PATH_STATS;
 }
 
+// ---------------------------------------------------------------------------
+// backward pass: workspace layout and launches
+// ---------------------------------------------------------------------------
+struct BwdLayout {
+    size_t kbar, bias, mask, mstat, dstat, delta, total;
+};
+
+BwdLayout bwd_layout(const Dims& g) {
+    BwdLayout w{};
+    size_t o = 0;
+    w.kbar = o;
+    o += align_up(sizeof(float) * g.BH * g.nblk * g.d);
+    w.bias = o;
+    o += align_up(sizeof(float) * g.BH * g.nblk);
+    w.mask = o;
+    o += align_up(sizeof(uint32_t) * g.BH * g.nblk * g.words);
+    w.mstat = o;
+    o += align_up(sizeof(float) * g.BH * g.L);
+    w.dstat = o;
+    o += align_up(sizeof(float) * g.BH * g.L);
+    w.delta = o;
+    o += align_up(sizeof(float) * g.BH * g.L);
+    w.total = o;
+    return w;
+}
+
+pisa_status run_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const uint32_t* mask, const Dims& g, pisa_dtype dtype, int order, int gate, float* mst,
+                         float* dst, float* del, float* dq, float* dk, float* dv, cudaStream_t s) {
+    return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+        using T = decltype(t);
+        constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+        using C = pisa::bwd::Cfg<T, D, BS>;
+        auto k1 = pisa::bwd::bwd_rowstat_kernel<T, D, BS>;
+        auto k2 = pisa::bwd::bwd_dq_kernel<T, D, BS>;
+        auto k3 = pisa::bwd::bwd_dkdv_kernel<T, D, BS>;
+        pisa_status r = set_smem(k1, C::ROWSTAT_SMEM);
+        if (r == PISA_OK) r = set_smem(k2, C::DQ_SMEM);
+        if (r == PISA_OK) r = set_smem(k3, C::DKDV_SMEM);
+        if (r != PISA_OK) return r;
+        const int L = (int)g.L, nblk = (int)g.nblk, words = (int)g.words;
+        const dim3 gq((unsigned)(g.L / pisa::bwd::kQT), (unsigned)g.BH);
+        k1<<<gq, 128, C::ROWSTAT_SMEM, s>>>((const T*)q, (const T*)k, (const T*)o, (const T*)dO, mask, L, nblk, words,
+                                            order, gate, mst, dst, del);
+        r = launch_check("bwd_rowstat_kernel");
+        if (r != PISA_OK) return r;
+        k2<<<gq, 128, C::DQ_SMEM, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dO, mask, L, nblk, words,
+                                       order, gate, mst, dst, del, dq);
+        r = launch_check("bwd_dq_kernel");
+        if (r != PISA_OK) return r;
+        const dim3 gk((unsigned)g.nblk, (unsigned)g.BH);
+        k3<<<gk, 2 * BS, C::DKDV_SMEM, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dO, mask, L, nblk,
+                                            words, order, gate, mst, dst, del, dk, dv);
+        return launch_check("bwd_dkdv_kernel");
+    });
+}
+
 pisa_status check_stats(const pisa_stats_t* st, Dims* g) {
     if (!st) return fail(PISA_ERR_INVALID_ARG, "null pisa_stats_t");
     pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, st->order, st->dtype, g);
@@ -559,6 +617,56 @@ pisa_status pisa_attention(const void* q, const void* k, const void* v, int batc
                            void* stream) {
     return pisa_attention_ex(q, k, v, batch, heads, L, d, dtype, B, K, order, 1, PISA_PATH_AUTO, out, workspace,
                              ws_bytes, stream);
+}
+
+size_t pisa_backward_workspace_bytes(int batch, int heads, int L, int d, int B, int K, int order, pisa_dtype dtype) {
+    Dims g;
+    if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return 0;
+    if (K < 0 || K > g.nblk || g.BH > 65535) return 0;
+    return bwd_layout(g).total;
+}
+
+pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                    int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
+                                    int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+    Dims g;
+    pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
+    if (r != PISA_OK) return r;
+    if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
+    if (g.BH > 65535) return fail(PISA_ERR_UNSUPPORTED, "batch * heads must be <= 65535 (got %ld)", g.BH);
+    if (flags & ~(PISA_FLAG_GATE_W | PISA_FLAG_POOLED_W | PISA_FLAG_COV_ROUTE))
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: unknown flag bits 0x%x", flags);
+    if (flags & PISA_FLAG_POOLED_W)
+        return fail(PISA_ERR_UNSUPPORTED, "pisa_attention_backward: no backward for the pooled w");
+    if (!q || !k || !v || !o || !dO || !dq || !dk || !dv)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: null pointer");
+    const void* in16[5] = {q, k, v, o, dO};
+    for (const void* p : in16)
+        if ((uintptr_t)p % 16) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: inputs must be 16-byte aligned");
+    if ((uintptr_t)dq % 8 || (uintptr_t)dk % 8 || (uintptr_t)dv % 8)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: dq, dk, dv must be 8-byte aligned");
+    if (!workspace) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: null workspace");
+    if ((uintptr_t)workspace % kAlign)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: workspace must be 256-byte aligned");
+    const BwdLayout w = bwd_layout(g);
+    if (ws_bytes < w.total)
+        return fail(PISA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, w.total);
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    float* kbar = (float*)(ws + w.kbar);
+    uint32_t* mask = (uint32_t*)(ws + w.mask);
+    float* rbias = (flags & PISA_FLAG_COV_ROUTE) ? (float*)(ws + w.bias) : nullptr;
+    r = run_centroids(k, kbar, g, dtype, s);
+    if (r != PISA_OK) return r;
+    if (rbias) {
+        r = run_route_bias(k, v, kbar, g, dtype, PISA_ROUTE_EPS, rbias, s);
+        if (r != PISA_OK) return r;
+    }
+    r = run_select(q, kbar, g, dtype, K, nullptr, mask, s, rbias);
+    if (r != PISA_OK) return r;
+    return run_backward(q, k, v, o, dO, mask, g, dtype, order, flags & PISA_FLAG_GATE_W, (float*)(ws + w.mstat),
+                        (float*)(ws + w.dstat), (float*)(ws + w.delta), dq, dk, dv, s);
 }
 
 pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pisa_dtype dtype, int B, float* kbar,

@@ -261,6 +261,46 @@ pisa_status pisa_attention_host(const void* q_host, const void* k_host, const vo
 size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
                                  pisa_path path, int chunk_heads);
 
+/* Backward pass: gradients dq, dk, dv of sum_t dO_t . o_t, where o is the
+ * output of pisa_attention_ex on the same q, k, v with the same B, K, order
+ * and flags on the per-block (non-hybrid) paths.  The pages define only the forward
+ * (PISA paper section 3.2 "Formulation"; "Sparse Linear Attention" blog,
+ * sections "Sparse Linear Attention" and the PWT section); this differentiates
+ * that forward with the block selection held fixed (the routing is detached,
+ * as the PWT blog trains it) and, for order 2, the gate decision held fixed.
+ * Per query row t, with x_n = q_t.k_n, G_n = dO_t.v_n, delta = dO_t.o_t and
+ * m, D the forward's shared max and denominator:
+ *   selected key n:        dS_n = P_n (G_n - delta),  P_n = e^{x_n - m}/D
+ *   key n of unselected j: u_n = x_n - q_t.kbar_j,  a = e^{l_tj - m}/D,
+ *                          P_n = a (1 + [order>=1] u_n),
+ *                          dS_n = a (dl_n (sum_n G_n (1 + [order>=1] u_n) - B delta)
+ *                                    + [order>=1] (G_n - mean_n G_n)),
+ *                          dl_n = 1/B (+ u_n/B for order 2 with the gate open)
+ *   dq_t = sum_n dS_tn k_n,  dk_n = sum_t dS_tn q_t,  dv_n = sum_t P_tn dO_t.
+ * Arguments:
+ *   q, k, v, o, dO : [BH, L, d] of `dtype`, device, 16-byte aligned; o is the
+ *                    forward output (only delta = dO.o is taken from it).
+ *   flags          : PISA_FLAG_GATE_W and PISA_FLAG_COV_ROUTE as in
+ *                    pisa_attention_ex (the same selection is recomputed
+ *                    here); PISA_FLAG_POOLED_W returns PISA_ERR_UNSUPPORTED.
+ *   dq, dk, dv     : [BH, L, d] fp32 outputs, device, 8-byte aligned, fully
+ *                    overwritten (no accumulation into existing contents).
+ *   workspace      : ws_bytes >= pisa_backward_workspace_bytes(...) of device
+ *                    memory, 256-byte aligned; on return it holds the centroids,
+ *                    the selection mask and the per-row m, D and delta.
+ * Shapes as for pisa_attention plus batch * heads <= 65535.  bf16 inputs run
+ * their tile products on the tensor cores (fp32 accumulation; P and dS are
+ * rounded to bf16 as the operands of the dk, dv and dq products); fp32 inputs
+ * run in fp32 throughout. */
+pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                    int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
+                                    int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
+/* Workspace pisa_attention_backward needs (bytes); 0 for invalid arguments. */
+size_t pisa_backward_workspace_bytes(int batch, int heads, int L, int d, int B, int K, int order,
+                                     pisa_dtype dtype);
+
 /* The path AUTO resolves to for these arguments (or -1 if none can run). */
 int pisa_resolve_path(int batch, int heads, int L, int d, int B, int K, int order,
                       pisa_dtype dtype);

@@ -137,3 +137,43 @@ def test_workspace_holds_the_routing_bias():
     for path in ("recompute_tc", "hybrid_tc", "stats"):
         n = pisa.pisa_workspace_bytes(1, 2, 2048, 128, 64, 8, 1, pisa.torch.bfloat16, path)
         assert n > 2 * (2048 // 64) * 4
+
+
+def call_bwd(L=1024, d=64, B=64, K=4, order=1, dtype=pisa.PISA_BF16, flags=1, ws_bytes=1 << 30, batch=1, heads=1,
+             q=FAKE, o=FAKE, dq=FAKE, ws=FAKE):
+    return pisa.lib().pisa_attention_backward(q, FAKE, FAKE, o, FAKE, batch, heads, L, d, dtype, B, K, order, flags,
+                                              dq, FAKE, FAKE, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=1000), pisa.PISA_ERR_INVALID_ARG),                  # L % B
+    (dict(K=17), pisa.PISA_ERR_INVALID_ARG),                    # K > nblk
+    (dict(order=3), pisa.PISA_ERR_INVALID_ARG),
+    (dict(d=96), pisa.PISA_ERR_UNSUPPORTED),
+    (dict(flags=8), pisa.PISA_ERR_INVALID_ARG),                 # unknown flag bit
+    (dict(flags=pisa.FLAG_POOLED_W), pisa.PISA_ERR_UNSUPPORTED),  # no backward for the pooled w
+    (dict(batch=2, heads=40000), pisa.PISA_ERR_UNSUPPORTED),    # grid y limit
+    (dict(q=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(o=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(dq=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(q=ctypes.c_void_p(0x1008)), pisa.PISA_ERR_INVALID_ARG),   # inputs need 16-byte alignment
+    (dict(dq=ctypes.c_void_p(0x1004)), pisa.PISA_ERR_INVALID_ARG),  # gradients need 8-byte alignment
+    (dict(ws=None), pisa.PISA_ERR_INVALID_ARG),
+    (dict(ws=ctypes.c_void_p(0x1010)), pisa.PISA_ERR_INVALID_ARG),  # workspace needs 256-byte alignment
+    (dict(ws_bytes=64), pisa.PISA_ERR_INVALID_ARG),
+])
+def test_backward_rejects_bad_arguments_before_launch(kw, status):
+    assert call_bwd(**kw) == status
+    assert pisa.lib().pisa_last_error()
+
+
+def test_backward_workspace_size():
+    f = pisa.lib().pisa_backward_workspace_bytes
+    # centroids + bias + mask + three per-row arrays, each rounded up to 256 bytes
+    BH, L, d, B = 2, 1024, 64, 64
+    nblk = L // B
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = up(4 * BH * nblk * d) + up(4 * BH * nblk) + up(4 * BH * nblk * 1) + 3 * up(4 * BH * L)
+    assert f(1, BH, L, d, B, 4, 1, pisa.PISA_BF16) == want
+    assert f(1, 1, 1000, 64, 64, 4, 1, pisa.PISA_BF16) == 0
+    assert f(1, 1, 1024, 64, 64, 17, 1, pisa.PISA_BF16) == 0

@@ -1,0 +1,160 @@
+"""GPU parity of the backward pass (pisa_attention_backward) against the CPU
+oracle's gradients.
+
+The pages define only the forward (PISA paper section 3.2 "Formulation";
+"Sparse Linear Attention" blog, sparse-linear and PWT sections); both sides
+differentiate it with the block selection held fixed (and, for order 2, the
+gate decision).  The oracle's gradients are pinned in test_oracle_pins.py
+(central differences, autograd of dense attention at K = all, exact identities).
+
+Tolerances (rel-L2 per gradient tensor): fp32 inputs 1e-4 (fp32 arithmetic
+throughout, fp32 accumulation over L keys); bf16 inputs 2e-2 (P and dS are
+rounded to bf16 as operands of the dk, dv and dq products, and o arrives in
+bf16, which enters through delta = dO.o).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_taylor_b200 as pisa
+import oracle
+import pisa_synth
+
+pytestmark = pytest.mark.gpu
+
+TDT = {"f32": torch.float32, "bf16": torch.bfloat16}
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def dev(x, dt):
+    return torch.from_numpy(np.ascontiguousarray(x)).to("cuda").to(TDT[dt])
+
+
+def inputs(seed, BH, L, d, dt, scale=2.0):
+    q, k, v = pisa_synth.random_qkv(seed, BH, L, d, scale=scale, dtype=dt)
+    dO = pisa_synth.random_qkv(seed + 1, BH, L, d, scale=1.0, dtype=dt)[0]
+    return q, k, v, dO
+
+
+def gpu_backward(q, k, v, o, dO, B, K, order, gate, dt, route="centroid"):
+    grads = pisa.pisa_attention_backward(dev(q, dt), dev(k, dt), dev(v, dt), dev(o, dt), dev(dO, dt), B, K, order,
+                                         gate=gate, route=route)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    return [g.cpu().numpy().astype(np.float64) for g in grads]
+
+
+def check(got, want, dt):
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        err = oracle.rel_l2(g, w)
+        assert err <= TOL[dt], (name, err)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("order,gate", [(0, True), (1, True), (2, True), (2, False)])
+def test_backward_parity(dt, d, B, order, gate):
+    L = 1024
+    q, k, v, dO = inputs(1100 + d + B + 10 * order, 2, L, d, dt, scale=3.0 if order == 2 else 2.0)
+    K = (L // B) // 4
+    o = oracle.pisa_attention_ex(q, k, v, B, K, order, gate=gate)
+    got = gpu_backward(q, k, v, o, dO, B, K, order, gate, dt)
+    check(got, oracle.pisa_backward(q, k, v, dO, B, K, order, gate), dt)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("L,B", [(576, 64), (640, 128), (64, 64), (128, 128)])
+def test_backward_ragged_and_tiny_lengths(dt, L, B):
+    # lengths that are not a multiple of the 128-row forward tile, and a single block
+    d = 64
+    q, k, v, dO = inputs(1200 + L + B, 2, L, d, dt)
+    K = max(1, (L // B) // 3)
+    o = oracle.pisa_attention_ex(q, k, v, B, K, 1)
+    got = gpu_backward(q, k, v, o, dO, B, K, 1, True, dt)
+    check(got, oracle.pisa_backward(q, k, v, dO, B, K, 1), dt)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("K", ["none", "all"])
+@pytest.mark.parametrize("order", [1, 2])
+def test_backward_degenerate_selections(dt, K, order):
+    # K = 0: every block through its Taylor term; K = all: exact dense attention
+    L, d, B = 512, 64, 64
+    Kv = 0 if K == "none" else L // B
+    q, k, v, dO = inputs(1300 + order + Kv, 2, L, d, dt)
+    o = oracle.pisa_attention_ex(q, k, v, B, Kv, order)
+    got = gpu_backward(q, k, v, o, dO, B, Kv, order, True, dt)
+    check(got, oracle.pisa_backward(q, k, v, dO, B, Kv, order), dt)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 128)])
+def test_backward_with_routing(dt, d, B):
+    # covariance-aware selection recomputed inside the backward (bit-exact routing
+    # and selection), gradients on that selection
+    L = 1024
+    q, k, v, dO = inputs(1400 + d + B, 2, L, d, dt)
+    K = (L // B) // 4
+    o = oracle.pisa_attention_ex(q, k, v, B, K, 1, route_eps=pisa.ROUTE_EPS)
+    got = gpu_backward(q, k, v, o, dO, B, K, 1, True, dt, route="cov")
+    want = oracle.pisa_backward(q, k, v, dO, B, K, 1, True, route_eps=pisa.ROUTE_EPS)
+    check(got, want, dt)
+    plain = oracle.pisa_backward(q, k, v, dO, B, K, 1)
+    assert oracle.rel_l2(plain[0], want[0]) > 1e-3  # routing reaches the gradient on these inputs
+
+
+@pytest.mark.parametrize("path", ["recompute_tc", "stats"])
+def test_forward_then_backward_on_the_gpu(path):
+    # the training use: o from the library's own forward, then the backward
+    dt, L, d, B, order = "bf16", 1024, 128, 64, 1
+    q, k, v, dO = inputs(1500, 2, L, d, dt)
+    K = (L // B) // 4
+    o = pisa.pisa_attention(dev(q, dt), dev(k, dt), dev(v, dt), B, K, order, path=path)
+    grads = pisa.pisa_attention_backward(dev(q, dt), dev(k, dt), dev(v, dt), o, dev(dO, dt), B, K, order)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    check([g.cpu().numpy().astype(np.float64) for g in grads], oracle.pisa_backward(q, k, v, dO, B, K, order), dt)
+
+
+def test_backward_overwrites_its_outputs_and_repeats_bit_for_bit():
+    dt, L, d, B = "bf16", 512, 64, 64
+    q, k, v, dO = inputs(1600, 2, L, d, dt)
+    o = oracle.pisa_attention_ex(q, k, v, B, 2, 1)
+    args = [dev(x, dt) for x in (q, k, v, o, dO)]
+    first = [g.clone() for g in pisa.pisa_attention_backward(*args, B, 2)]
+    grads = tuple(torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda") for _ in range(3))
+    again = pisa.pisa_attention_backward(*args, B, 2, grads=grads)
+    torch.cuda.synchronize()
+    for a, b in zip(first, again):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name,heads", [("c3", 1), ("c2", 1)])
+def test_backward_full_size_sampled_rows_and_identities(name, heads):
+    # Full sequence length and block size of the workload, in the launch
+    # configuration bench.py times.  The oracle computes sampled dq rows one by
+    # one; dk and dv are checked through two exact identities of the method:
+    # sum_n dk_n = 0 (a common shift of all keys leaves o unchanged) and
+    # sum_n dv_n = sum_t dO_t (each row's weights sum to D).
+    w = pisa_synth.workloads()[name].with_(heads=heads)
+    q, k, v = pisa_synth.generate(w)
+    dt = w.dtype
+    BH, L, d = q.shape
+    dO = pisa_synth.random_qkv(1700, BH, L, d, scale=1.0, dtype=dt)[0]
+    qd, kd, vd, dOd = dev(q, dt), dev(k, dt), dev(v, dt), dev(dO, dt)
+    o = pisa.pisa_attention(qd, kd, vd, w.B, w.K, w.order)
+    dq, dk, dv = pisa.pisa_attention_backward(qd, kd, vd, o, dOd, w.B, w.K, w.order)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    rng = np.random.default_rng(17)
+    rows = [(int(rng.integers(BH)), int(t)) for t in rng.integers(0, L, 24)] + [(0, 0), (BH - 1, L - 1)]
+    want = oracle.pisa_backward_dq_rows(q, k, v, dO, w.B, w.K, rows, w.order)
+    got = np.stack([dq[b, t].cpu().numpy().astype(np.float64) for b, t in rows])
+    assert oracle.rel_l2(got, want) <= TOL[dt]
+    dk64, dv64 = dk.double(), dv.double()
+    for b in range(BH):
+        assert float(dk64[b].sum(0).norm()) <= 1e-2 * float(dk64[b].norm(dim=1).sum())
+        s_dv, s_do = dv64[b].sum(0), dOd[b].double().sum(0)
+        assert float((s_dv - s_do).norm()) <= 1e-2 * float(s_do.norm()) + 1e-3 * math.sqrt(L)
