@@ -336,7 +336,7 @@ pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
 // backward pass: workspace layout and launches
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-    size_t kbar, bias, mask, mstat, dstat, delta, total;
+    size_t kbar, bias, mask, mstat, dinv, delta, total;
 };
 
 BwdLayout bwd_layout(const Dims& g) {
@@ -350,7 +350,7 @@ BwdLayout bwd_layout(const Dims& g) {
     o += align_up(sizeof(uint32_t) * g.BH * g.nblk * g.words);
     w.mstat = o;
     o += align_up(sizeof(float) * g.BH * g.L);
-    w.dstat = o;
+    w.dinv = o;
     o += align_up(sizeof(float) * g.BH * g.L);
     w.delta = o;
     o += align_up(sizeof(float) * g.BH * g.L);
@@ -360,7 +360,7 @@ BwdLayout bwd_layout(const Dims& g) {
 
 pisa_status run_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const uint32_t* mask, const Dims& g, pisa_dtype dtype, int order, int gate, float* mst,
-                         float* dst, float* del, float* dq, float* dk, float* dv, cudaStream_t s) {
+                         float* dinv, float* del, float* dq, float* dk, float* dv, cudaStream_t s) {
     return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
@@ -375,16 +375,16 @@ pisa_status run_backward(const void* q, const void* k, const void* v, const void
         const int L = (int)g.L, nblk = (int)g.nblk, words = (int)g.words;
         const dim3 gq((unsigned)(g.L / pisa::bwd::kQT), (unsigned)g.BH);
         k1<<<gq, 128, C::ROWSTAT_SMEM, s>>>((const T*)q, (const T*)k, (const T*)o, (const T*)dO, mask, L, nblk, words,
-                                            order, gate, mst, dst, del);
+                                            order, gate, mst, dinv, del);
         r = launch_check("bwd_rowstat_kernel");
         if (r != PISA_OK) return r;
         k2<<<gq, 128, C::DQ_SMEM, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dO, mask, L, nblk, words,
-                                       order, gate, mst, dst, del, dq);
+                                       order, gate, mst, dinv, del, dq);
         r = launch_check("bwd_dq_kernel");
         if (r != PISA_OK) return r;
         const dim3 gk((unsigned)g.nblk, (unsigned)g.BH);
         k3<<<gk, 2 * BS, C::DKDV_SMEM, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dO, mask, L, nblk,
-                                            words, order, gate, mst, dst, del, dk, dv);
+                                            words, order, gate, mst, dinv, del, dk, dv);
         return launch_check("bwd_dkdv_kernel");
     });
 }
@@ -666,7 +666,7 @@ pisa_status pisa_attention_backward(const void* q, const void* k, const void* v,
     r = run_select(q, kbar, g, dtype, K, nullptr, mask, s, rbias);
     if (r != PISA_OK) return r;
     return run_backward(q, k, v, o, dO, mask, g, dtype, order, flags & PISA_FLAG_GATE_W, (float*)(ws + w.mstat),
-                        (float*)(ws + w.dstat), (float*)(ws + w.delta), dq, dk, dv, s);
+                        (float*)(ws + w.dinv), (float*)(ws + w.delta), dq, dk, dv, s);
 }
 
 pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pisa_dtype dtype, int B, float* kbar,

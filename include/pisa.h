@@ -287,7 +287,7 @@ size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype 
  *                    overwritten (no accumulation into existing contents).
  *   workspace      : ws_bytes >= pisa_backward_workspace_bytes(...) of device
  *                    memory, 256-byte aligned; on return it holds the centroids,
- *                    the selection mask and the per-row m, D and delta.
+ *                    the selection mask and the per-row m, 1/D and delta.
  * Shapes as for pisa_attention plus batch * heads <= 65535.  bf16 inputs run
  * their tile products on the tensor cores (fp32 accumulation; P and dS are
  * rounded to bf16 as the operands of the dk, dv and dq products); fp32 inputs
