@@ -150,6 +150,33 @@ __device__ __forceinline__ void warp_mma_kn(float (&acc)[NT][4], const bf16* A, 
     }
 }
 
+// Two nk products of the same shape in one k loop (acc1 += A1 B1, acc2 += A2 B2): twice the
+// independent accumulator chains; every accumulator sees the same operations in the same order
+// as in two separate calls.
+template <int NT, int KD>
+__device__ __forceinline__ void warp_mma_nk2(float (&acc1)[NT][4], const bf16* A1, const bf16* B1,
+                                             float (&acc2)[NT][4], const bf16* A2, const bf16* B2, int lda,
+                                             int ldb, int lane) {
+    const int m = lane >> 3, r = lane & 7;
+#pragma unroll
+    for (int k0 = 0; k0 < KD; k0 += 16) {
+        uint32_t a1[4], a2[4];
+        load_a(a1, A1, lda, k0, lane);
+        load_a(a2, A2, lda, k0, lane);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt += 2) {
+            uint32_t b1[4], b2[4];
+            const int off = ((nt + (m >> 1)) * 8 + r) * ldb + k0 + (m & 1) * 8;
+            ldsm4(b1, B1 + off);
+            ldsm4(b2, B2 + off);
+            mma16816(acc1[nt], a1, b1[0], b1[1]);
+            mma16816(acc2[nt], a2, b2[0], b2[1]);
+            mma16816(acc1[nt + 1], a1, b1[2], b1[3]);
+            mma16816(acc2[nt + 1], a2, b2[2], b2[3]);
+        }
+    }
+}
+
 // fp32 operands: the same accumulator fragment, fp32 FMAs in k order.
 template <int NT, int KD>
 __device__ __forceinline__ void warp_mma_nk(float (&acc)[NT][4], const float* A, int lda, const float* Bn, int ldb,
@@ -186,6 +213,22 @@ __device__ __forceinline__ void warp_mma_kn(float (&acc)[NT][4], const float* A,
             acc[nt][3] = fmaf(a1, b1, acc[nt][3]);
         }
     }
+}
+
+template <int NT, int KD>
+__device__ __forceinline__ void warp_mma_nk2(float (&acc1)[NT][4], const float* A1, const float* B1,
+                                             float (&acc2)[NT][4], const float* A2, const float* B2, int lda,
+                                             int ldb, int lane) {
+    warp_mma_nk<NT, KD>(acc1, A1, lda, B1, ldb, lane);
+    warp_mma_nk<NT, KD>(acc2, A2, lda, B2, ldb, lane);
+}
+
+// two adjacent elements (columns c, c+1) of a staged operand tile in one store
+__device__ __forceinline__ void st_pair(bf16* p, float x0, float x1) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x0, x1);
+}
+__device__ __forceinline__ void st_pair(float* p, float x0, float x1) {
+    *reinterpret_cast<float2*>(p) = make_float2(x0, x1);
 }
 
 template <int NT>
@@ -452,9 +495,7 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const T* __restrict__ q, co
         for (int nt = 0; nt < NS; ++nt)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    drow[(g + 8 * h) * C::LDS + nt * 8 + 2 * t + e] = from_f<T>(s[nt][2 * h + e]);
+                st_pair(drow + (g + 8 * h) * C::LDS + nt * 8 + 2 * t, s[nt][2 * h], s[nt][2 * h + 1]);
         __syncwarp();
         warp_mma_kn<ND, BS>(acc, drow, C::LDS, Ks, C::LD, lane);
     }
@@ -543,8 +584,7 @@ __global__ void __launch_bounds__(BS * 2) bwd_dkdv_kernel(const T* __restrict__ 
         float s[NC][4], gg[NC][4], p[NC][4];
         zero(s);
         zero(gg);
-        warp_mma_nk<NC, D>(s, Ks + warp * 16 * C::LD, C::LD, Qs, C::LD, lane);
-        warp_mma_nk<NC, D>(gg, Vs + warp * 16 * C::LD, C::LD, dOs, C::LD, lane);
+        warp_mma_nk2<NC, D>(s, Ks + warp * 16 * C::LD, Qs, gg, Vs + warp * 16 * C::LD, dOs, C::LD, C::LD, lane);
         const bool sel = selected(mask + ((size_t)bh * nblk + (c * kQC) / BS) * words, j);
         if (sel) {
 #pragma unroll
@@ -627,13 +667,11 @@ __global__ void __launch_bounds__(BS * 2) bwd_dkdv_kernel(const T* __restrict__ 
 #pragma unroll
         for (int nt = 0; nt < NC; ++nt)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int o2 = (g + 8 * h) * C::LDP + nt * 8 + 2 * t + e;
-                    prow[o2] = from_f<T>(p[nt][2 * h + e]);
-                    drow[o2] = from_f<T>(s[nt][2 * h + e]);
-                }
+            for (int h = 0; h < 2; ++h) {
+                const int o2 = (g + 8 * h) * C::LDP + nt * 8 + 2 * t;
+                st_pair(prow + o2, p[nt][2 * h], p[nt][2 * h + 1]);
+                st_pair(drow + o2, s[nt][2 * h], s[nt][2 * h + 1]);
+            }
         __syncwarp();
         warp_mma_kn<ND, kQC>(adv, prow, C::LDP, dOs, C::LD, lane);
         warp_mma_kn<ND, kQC>(adk, drow, C::LDP, Qs, C::LD, lane);
