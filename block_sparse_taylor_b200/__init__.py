@@ -16,7 +16,8 @@ The functions carry the names of the C entry points:
   sparse attention (PISA paper section 3.2; "Sparse Linear Attention" blog,
   PWT section for order 2).
 * ``pisa_attention_backward(q, k, v, o, dO, B, K, order)``: dq, dk, dv of that
-  forward with the block selection held fixed.
+  forward with the block selection held fixed; ``pisa_attention_autograd`` wraps
+  both as a torch.autograd.Function.
 
 Tensors are [batch*heads, L, d] (or [batch, heads, L, d]) contiguous CUDA
 tensors of dtype float32 or bfloat16; q must already be multiplied by
@@ -350,6 +351,34 @@ def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
                                          workspace.numel(), _stream(stream)))
     return dq, dk, dv
+
+
+class PisaAttentionFunction(torch.autograd.Function):
+    """pisa_attention as a torch.autograd.Function: the forward is pisa_attention, the backward
+    pisa_attention_backward (selection held fixed); gradients are returned in the inputs' dtype."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, B, K, order, gate, path, route):
+        out = pisa_attention(q, k, v, B, K, order, gate=gate, path=path, route=route)
+        ctx.save_for_backward(q, k, v, out)
+        ctx.cfg = (B, K, order, gate, route)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out = ctx.saved_tensors
+        B, K, order, gate, route = ctx.cfg
+        dq, dk, dv = pisa_attention_backward(q, k, v, out, dout.contiguous(), B, K, order, gate=gate, route=route)
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None, None, None, None
+
+
+def pisa_attention_autograd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
+                            gate: bool = True, path: str = "auto", route: str = "centroid") -> torch.Tensor:
+    """pisa_attention with gradients for training (the per-block paths: "auto", "recompute_tc",
+    "stats"; exact w).  The backward holds the block selection fixed."""
+    if path == "hybrid_tc":
+        raise PisaError(PISA_ERR_UNSUPPORTED, "no backward for the hybrid path")
+    return PisaAttentionFunction.apply(q, k, v, B, K, order, gate, path, route)
 
 
 def pisa_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,

@@ -158,3 +158,23 @@ def test_backward_full_size_sampled_rows_and_identities(name, heads):
         assert float(dk64[b].sum(0).norm()) <= 1e-2 * float(dk64[b].norm(dim=1).sum())
         s_dv, s_do = dv64[b].sum(0), dOd[b].double().sum(0)
         assert float((s_dv - s_do).norm()) <= 1e-2 * float(s_do.norm()) + 1e-3 * math.sqrt(L)
+
+
+def test_autograd_function():
+    # pisa_attention_autograd: gradients through torch.autograd equal the entry point's (cast to
+    # the input dtype) and match the oracle
+    dt, L, d, B, K = "bf16", 1024, 128, 64, 4
+    q, k, v, dO = inputs(1800, 2, L, d, dt)
+    qt, kt, vt = (dev(x, dt).requires_grad_() for x in (q, k, v))
+    out = pisa.pisa_attention_autograd(qt, kt, vt, B, K, 1)
+    out.backward(dev(dO, dt))
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    direct = pisa.pisa_attention_backward(dev(q, dt), dev(k, dt), dev(v, dt), out.detach(), dev(dO, dt), B, K, 1)
+    for t, g in zip((qt, kt, vt), direct):
+        assert t.grad.dtype == torch.bfloat16
+        assert torch.equal(t.grad, g.to(torch.bfloat16))
+    check([t.grad.float().cpu().numpy().astype(np.float64) for t in (qt, kt, vt)],
+          oracle.pisa_backward(q, k, v, dO, B, K, 1), dt)
+    with pytest.raises(pisa.PisaError):
+        pisa.pisa_attention_autograd(qt, kt, vt, B, K, 1, path="hybrid_tc")
