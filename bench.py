@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--no-hybrid", action="store_true", help="skip the PISA-hybrid (global H-bar) record")
     p.add_argument("--no-route", action="store_true", help="skip the covariance-aware routing record")
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass record")
+    p.add_argument("--no-dense", action="store_true", help="skip the dense-SDPA context record")
     return p.parse_args()
 
 
@@ -61,6 +62,41 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def pct(sorted_vals, p):
+    """p-th percentile of an ascending list (linear interpolation)."""
+    if not sorted_vals:
+        return None
+    x = (len(sorted_vals) - 1) * p / 100.0
+    lo = int(x)
+    hi = min(lo + 1, len(sorted_vals) - 1)
+    return sorted_vals[lo] + (sorted_vals[hi] - sorted_vals[lo]) * (x - lo)
+
+
+def dense_sdpa_record(q, k, v, stream, reps=3):
+    """Context only, not a target: torch's dense scaled_dot_product_attention (a library kernel:
+    flash, cuDNN or memory-efficient backend, never the L^2-memory math one) on the same inputs,
+    q already scaled.  Any failure is reported, not raised."""
+    try:
+        import torch
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        qd, kd, vd = (x.unsqueeze(0) for x in (q, k, v))
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]):
+            F.scaled_dot_product_attention(qd, kd, vd, scale=1.0)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                F.scaled_dot_product_attention(qd, kd, vd, scale=1.0)
+            b.record(stream)
+            torch.cuda.synchronize()
+        return {"ms_per_call": a.elapsed_time(b) / reps, "calls_timed": reps,
+                "note": "torch scaled_dot_product_attention, dense, library kernel; context only"}
+    except Exception as e:  # noqa: BLE001 - a context record never fails the benchmark
+        return {"unavailable": f"{type(e).__name__}: {e}"[:240]}
 
 
 def kernel_source_hash() -> str:
@@ -347,6 +383,8 @@ def main():
     k_sel = [e[1].elapsed_time(e[2]) for e in evs]
     k_attn = [e[2].elapsed_time(e[3]) for e in evs]
     attn_ms = statistics.mean(k_attn)
+    step_spans = sorted(e[0].elapsed_time(e[3]) for e in evs)  # this rank's per-step spans
+    step_pct = {"p10": pct(step_spans, 10), "median": pct(step_spans, 50), "p90": pct(step_spans, 90)}
 
     dense_flops = 4.0 * L * L * d * BH
     value = dense_flops * world / (ms_step * 1e-3) / 1e12
@@ -531,6 +569,12 @@ def main():
         pisa.pisa_poll_device_status()
         del plan
 
+    dense_rec = None
+    if not args.no_dense and rank == 0 and world == 1:
+        dense_rec = dense_sdpa_record(q, k, v, stream)
+        if "ms_per_call" in dense_rec:
+            dense_rec["speedup_of_pisa_step"] = dense_rec["ms_per_call"] / ms_step
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, q_h, k_h, v_h)
@@ -552,6 +596,8 @@ def main():
             "hybrid": hybrid_rec,
             "routing": route_rec,
             "backward": bwd_rec,
+            "step_ms_percentiles": step_pct,
+            "dense_sdpa_context": dense_rec,
             "cpu_baseline": cpu,
             "clocks": clk,
             "e2e": e2e,
