@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <string>
 
 #include "../../include/pisa.h"
@@ -84,6 +85,16 @@ pisa_status check_dims(int batch, int heads, int L, int d, int B, int order, pis
     out->B = B;
     out->nblk = nblk;
     out->words = (nblk + 31) / 32;
+    return PISA_OK;
+}
+
+// Device arrays that kernels move with 16-byte vector accesses or TMA must be
+// 16-byte aligned.  Contiguous tensors from an allocator always are; a view at an
+// odd element offset may not be, and would fault the kernel instead of failing here.
+pisa_status check_align16(const char* where, std::initializer_list<const void*> ptrs) {
+    for (const void* p : ptrs)
+        if (p && (uintptr_t)p % 16)
+            return fail(PISA_ERR_INVALID_ARG, "%s: device arrays must be 16-byte aligned", where);
     return PISA_OK;
 }
 
@@ -445,6 +456,8 @@ pisa_status pisa_stats(const void* k, const void* v, const pisa_stats_t* st, voi
     pisa_status r = check_stats(st, &g);
     if (r != PISA_OK) return r;
     if (!k || !v) return fail(PISA_ERR_INVALID_ARG, "pisa_stats: null k or v");
+    r = check_align16("pisa_stats", {k, v, st->kbar, st->vsum, st->hstat, st->cov});
+    if (r != PISA_OK) return r;
     return run_stats(k, v, st, g, (cudaStream_t)stream);
 }
 
@@ -457,6 +470,8 @@ pisa_status pisa_select(const void* q, const pisa_stats_t* st, int K, int32_t* i
     if (!q) return fail(PISA_ERR_INVALID_ARG, "pisa_select: null q");
     if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
     if (!idx && !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_select: idx and mask both null");
+    r = check_align16("pisa_select", {q, st->kbar});
+    if (r != PISA_OK) return r;
     return run_select(q, st->kbar, g, st->dtype, K, K > 0 ? idx : nullptr, mask, (cudaStream_t)stream);
 }
 
@@ -470,6 +485,8 @@ pisa_status pisa_select_biased(const void* q, const pisa_stats_t* st, int K, con
     if (!q) return fail(PISA_ERR_INVALID_ARG, "pisa_select_biased: null q");
     if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
     if (!idx && !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_select_biased: idx and mask both null");
+    r = check_align16("pisa_select_biased", {q, st->kbar});
+    if (r != PISA_OK) return r;
     return run_select(q, st->kbar, g, st->dtype, K, K > 0 ? idx : nullptr, mask, (cudaStream_t)stream, bias);
 }
 
@@ -480,6 +497,8 @@ pisa_status pisa_select_scores(const void* q, const pisa_stats_t* st, const floa
     pisa_status r = check_dims(st->batch, st->heads, st->L, st->d, st->B, 0, st->dtype, &g);
     if (r != PISA_OK) return r;
     if (!st->kbar || !q || !scores) return fail(PISA_ERR_INVALID_ARG, "pisa_select_scores: null pointer");
+    r = check_align16("pisa_select_scores", {q, st->kbar});
+    if (r != PISA_OK) return r;
     return run_select(q, st->kbar, g, st->dtype, 0, nullptr, nullptr, (cudaStream_t)stream, bias, scores);
 }
 
@@ -489,6 +508,8 @@ pisa_status pisa_route_bias(const void* k, const void* v, const float* kbar, int
     pisa_status r = check_dims(batch, heads, L, d, B, 0, dtype, &g);
     if (r != PISA_OK) return r;
     if (!k || !v || !kbar || !bias) return fail(PISA_ERR_INVALID_ARG, "pisa_route_bias: null pointer");
+    r = check_align16("pisa_route_bias", {k, v, kbar});
+    if (r != PISA_OK) return r;
     if (!(eps >= 1e-30f && eps <= 1e30f))
         return fail(PISA_ERR_INVALID_ARG, "pisa_route_bias: eps must be in [1e-30, 1e30] (got %g)", (double)eps);
     return run_route_bias(k, v, kbar, g, dtype, eps, bias, (cudaStream_t)stream);
@@ -525,6 +546,8 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     if (r != PISA_OK) return r;
     if (K < 0 || K > g.nblk) return fail(PISA_ERR_INVALID_ARG, "K must be in [0, %ld] (got %d)", g.nblk, K);
     if (!q || !k || !v || !out) return fail(PISA_ERR_INVALID_ARG, "pisa_attention: null q, k, v or out");
+    r = check_align16("pisa_attention", {q, k, v, out});
+    if (r != PISA_OK) return r;
     if (!workspace) return fail(PISA_ERR_INVALID_ARG, "pisa_attention: null workspace");
     if ((uintptr_t)workspace % kAlign)
         return fail(PISA_ERR_INVALID_ARG, "pisa_attention: workspace must be 256-byte aligned");
@@ -675,6 +698,8 @@ pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pi
     pisa_status r = check_dims(batch, heads, L, d, B, 0, dtype, &g);
     if (r != PISA_OK) return r;
     if (!k || !kbar) return fail(PISA_ERR_INVALID_ARG, "pisa_centroids: null k or kbar");
+    r = check_align16("pisa_centroids", {k, kbar});
+    if (r != PISA_OK) return r;
     return run_centroids(k, kbar, g, dtype, (cudaStream_t)stream);
 }
 
@@ -685,6 +710,12 @@ pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, in
     pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
     if (r != PISA_OK) return r;
     if (!q || !k || !v || !out || !mask) return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: null pointer");
+    r = check_align16("pisa_fused_attention", {q, k, v, out});
+    if (r != PISA_OK) return r;
+    if (st) {
+        r = check_align16("pisa_fused_attention", {st->kbar, st->vsum, st->hstat, st->cov});
+        if (r != PISA_OK) return r;
+    }
     if (path == PISA_PATH_AUTO) path = resolve(g, 0, order, dtype);
     if (path == PISA_PATH_RECOMPUTE_TC) {
         if (!tc_path_available(g, dtype))

@@ -37,6 +37,8 @@
  *     0 <= K <= L/B, order in {0, 1, 2}, L/B <= 4096.  Other shapes return
  *     PISA_ERR_UNSUPPORTED (valid but not implemented) or
  *     PISA_ERR_INVALID_ARG (meaningless).
+ *   - Device arrays (inputs, outputs, statistics) must be 16-byte aligned, as
+ *     contiguous allocations are; PISA_ERR_INVALID_ARG otherwise.
  *   - Non-finite inputs give undefined (but memory-safe) results.
  *   - On a non-OK status, pisa_last_error() returns a message for the calling
  *     thread.  Argument errors are detected before anything is enqueued.

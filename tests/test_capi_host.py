@@ -177,3 +177,26 @@ def test_backward_workspace_size():
     assert f(1, BH, L, d, B, 4, 1, pisa.PISA_BF16) == want
     assert f(1, 1, 1000, 64, 64, 4, 1, pisa.PISA_BF16) == 0
     assert f(1, 1, 1024, 64, 64, 17, 1, pisa.PISA_BF16) == 0
+
+
+MIS = ctypes.c_void_p(0x1008)  # 8-byte but not 16-byte aligned; never dereferenced
+
+
+def test_forward_entry_points_reject_misaligned_device_arrays():
+    L = pisa.lib()
+    args = (1, 1, 1024, 64, pisa.PISA_BF16, 64, 4, 1)
+    assert L.pisa_attention_ex(MIS, FAKE, FAKE, *args, 1, 0, FAKE, FAKE, 1 << 30, None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_attention_ex(FAKE, FAKE, FAKE, *args, 1, 0, MIS, FAKE, 1 << 30, None) == pisa.PISA_ERR_INVALID_ARG
+    assert "16-byte" in L.pisa_last_error().decode()
+    assert L.pisa_centroids(MIS, 1, 1, 1024, 64, pisa.PISA_BF16, 64, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_centroids(FAKE, 1, 1, 1024, 64, pisa.PISA_BF16, 64, MIS, None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_route_bias(FAKE, MIS, FAKE, 1, 1, 1024, 64, pisa.PISA_BF16, 64, ctypes.c_float(1e-6), FAKE,
+                             None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_fused_attention(FAKE, FAKE, MIS, 1, 1, 1024, 64, pisa.PISA_BF16, 64, 1, 1, 2, FAKE, None, FAKE,
+                                  None) == pisa.PISA_ERR_INVALID_ARG
+    st = pisa._StatsT(1, 1, 1024, 64, 64, 16, 0, pisa.PISA_BF16, MIS.value, None, None, None)
+    assert L.pisa_select(FAKE, ctypes.byref(st), 4, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_select_biased(FAKE, ctypes.byref(st), 4, FAKE, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_select_scores(FAKE, ctypes.byref(st), None, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+    st.kbar = FAKE.value
+    assert L.pisa_select(MIS, ctypes.byref(st), 4, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
