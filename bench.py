@@ -243,6 +243,37 @@ def cpu_baseline(w, q, k, v, budget_s=20.0):
     }
 
 
+def cpu_backward_baseline(w, q, k, v, dO):
+    """Time the oracle's backward, as it stands, on a bounded sample: dq of sampled query rows of
+    head 0, one row per thread, in calls of n and 8n rows so that the head's selection and
+    centroids (computed once per call) separate from the per-row cost.  Extrapolated the way the
+    oracle's whole backward runs (heads in parallel, each head's rows in series).  That backward
+    also accumulates dk and dv for every row, so the estimate is a lower bound on its time."""
+    import oracle
+
+    nt = oracle.default_threads()
+    qh, kh, vh, dh = q[:1], k[:1], v[:1], dO[:1]
+
+    def timed(n):
+        rows = [(0, int(t)) for t in np.linspace(0, w.L - 1, n).round()]
+        t0 = time.perf_counter()
+        oracle.pisa_backward_dq_rows(qh, kh, vh, dh, w.B, w.K, rows, w.order, nthreads=nt)
+        return time.perf_counter() - t0
+
+    t1, t8 = timed(nt), timed(8 * nt)
+    c_row = max((t8 - t1) / 7.0, 1e-9)
+    prep = max(t1 - c_row, 0.0)
+    t_full = math.ceil(w.BH / nt) * (prep + w.L * c_row)
+    flops = 10.0 * w.L * w.L * w.d * w.BH
+    return {"value": flops / t_full / 1e12, "unit": "TFLOP/s (algorithmic backward, 10*L^2*d*heads per call)",
+            "cores": nt, "kind": "oracle",
+            "sample": (f"head 0 of {w.BH}: dq of {nt} and {8 * nt} sampled rows ({t1:.2f} s, {t8:.2f} s): "
+                       f"{c_row * 1e3:.1f} ms per row, {prep:.2f} s per head for selection and centroids; "
+                       f"extrapolated to {w.BH} heads x {w.L} rows = {t_full:.0f} s per call (lower bound: "
+                       f"the full oracle backward also accumulates dk and dv per row)"),
+            "seconds_measured": t1 + t8}
+
+
 def describe(w) -> str:
     """One-line description of a named workload (its shape and generator)."""
     shape = {"c3": "Wan2.1-shaped DiT attention", "c4": "Hunyuan-Video-shaped DiT attention"}.get(w.name)
@@ -530,6 +561,11 @@ def main():
                    "tile_products": ("warp-level mma.sync m16n8k16, bf16 operands, fp32 accumulation"
                                      if tdt == torch.bfloat16 else "fp32 FMA"),
                    "launches_per_call": 5}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            try:
+                bwd_rec["cpu_baseline"] = cpu_backward_baseline(w, q_h, k_h, v_h, dO[:1].float().cpu().numpy())
+            except Exception as e:  # noqa: BLE001 - a baseline record never fails the benchmark
+                bwd_rec["cpu_baseline"] = {"unavailable": f"{type(e).__name__}: {e}"[:240]}
         del dO, grads, bws
 
     # end to end through the public host-buffer call: pisa_attention_host on
