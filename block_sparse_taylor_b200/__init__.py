@@ -101,6 +101,8 @@ def lib():
         L.pisa_attention_backward.restype = ctypes.c_int
         L.pisa_backward_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
         L.pisa_backward_workspace_bytes.restype = sz
+        L.pisa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+        L.pisa_selftest_wait_timeout.restype = ctypes.c_int
         for fn in ("pisa_attention_noalloc", "pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
                    "pisa_poll_device_status", "pisa_resolve_path"):
             getattr(L, fn).restype = ctypes.c_int
@@ -425,6 +427,13 @@ def pisa_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: 
     _check(lib().pisa_attention_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), batch, heads, L, d,
                                      code, B, K, order, flags, PATHS[plan.path], plan.chunk, plan.buf.data_ptr(),
                                      plan.buf.numel(), plan.streams[0].cuda_stream, plan.streams[1].cuda_stream))
+
+
+def pisa_selftest_wait_timeout(limit_cycles: int = 2_000_000, stream=None):
+    """Enqueue the failure-path self-test: a bounded device wait that runs out (see
+    include/pisa.h).  The next pisa_poll_device_status raises PisaError with status
+    PISA_ERR_DEVICE_TIMEOUT."""
+    _check(lib().pisa_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
 
 
 def pisa_poll_device_status(stream=None):

@@ -23,6 +23,7 @@
 #include "attn_hybrid.cuh"
 #include "route.cuh"
 #include "backward.cuh"
+#include "selftest.cuh"
 
 using pisa::bf16;
 
@@ -739,6 +740,16 @@ pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, in
     if (gate_w & PISA_FLAG_POOLED_W)
         return fail(PISA_ERR_UNSUPPORTED, "pisa_fused_attention: the pooled w needs pisa_attention_ex");
     return run_attn_stats(q, k, v, st, mask, out, g, order, gate_w & PISA_FLAG_GATE_W, (cudaStream_t)stream);
+}
+
+pisa_status pisa_selftest_wait_timeout(long long limit_cycles, void* stream) {
+    if (limit_cycles < 1 || limit_cycles > pisa::kWaitLimitCycles)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_selftest_wait_timeout: limit_cycles must be in [1, %lld] (got %lld)",
+                    (long long)pisa::kWaitLimitCycles, limit_cycles);
+    unsigned int* status = device_status_ptr();
+    if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+    pisa::wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status, limit_cycles);
+    return launch_check("wait_timeout_selftest_kernel");
 }
 
 pisa_status pisa_poll_device_status(void* stream) {

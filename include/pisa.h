@@ -316,7 +316,16 @@ const char* pisa_last_error(void);
  * PISA_ERR_CUDA on a CUDA error, PISA_OK otherwise. */
 pisa_status pisa_poll_device_status(void* stream);
 
-/* Library version string. */
+/* Failure-path self-test of the bounded device waits (no counterpart on the
+ * pages).  Enqueues one CTA whose single thread waits, bounded by limit_cycles
+ * SM clock cycles (1 .. 2e9), on a fresh mbarrier that nothing completes, with
+ * the same bounded wait the tensor-core kernels use.  The wait gives up, sets
+ * the timeout bit of the device status word and the kernel exits; the next
+ * pisa_poll_device_status returns PISA_ERR_DEVICE_TIMEOUT and clears the word.
+ * The context stays usable.  Errors: INVALID_ARG for a limit out of range. */
+pisa_status pisa_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/* Library version string. *//* Library version string. */
 const char* pisa_version(void);
 
 #ifdef __cplusplus

@@ -200,3 +200,10 @@ def test_forward_entry_points_reject_misaligned_device_arrays():
     assert L.pisa_select_scores(FAKE, ctypes.byref(st), None, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
     st.kbar = FAKE.value
     assert L.pisa_select(MIS, ctypes.byref(st), 4, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
+
+
+def test_selftest_wait_timeout_rejects_limits_out_of_range():
+    f = pisa.lib().pisa_selftest_wait_timeout
+    for bad in (0, -5, 2_000_000_001):
+        assert f(bad, None) == pisa.PISA_ERR_INVALID_ARG
+        assert b"limit_cycles" in pisa.lib().pisa_last_error()
