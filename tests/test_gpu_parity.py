@@ -385,3 +385,27 @@ def test_host_entry_point_matches_device_call():
     torch.cuda.synchronize()
     pisa.pisa_poll_device_status()
     assert torch.equal(ho, ref)
+
+
+# ---------------------------------------------------------------------------
+# the largest block count the C ABI accepts: L / B = 4096
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", ["recompute_tc", "hybrid_tc"])
+def test_maximum_block_count(path):
+    # L = 4096 blocks x 64 tokens, d = 64, one head, 10 % of the blocks kept: score rows of 4096,
+    # the top-K's scan branch and 128 mask words per row, bit-exact; sampled output tiles within
+    # the bf16 tolerance
+    B, d, K = 64, 64, 410
+    L = 4096 * B
+    q, k, v = pisa_synth.random_qkv(1900, 1, L, d, scale=2.0, dtype="bf16")
+    st = pisa.pisa_centroids(dev(k, "bf16"), B)
+    idx, mask = pisa.pisa_select(dev(q, "bf16"), st, K)
+    torch.cuda.synchronize()
+    ridx, rmask, _ = oracle.select(q, k, B, K)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_array_equal(mask.cpu().numpy().view(np.uint32), rmask)
+    got = run_attn(q, k, v, B, K, 1, "bf16", path)
+    tiles = sample_tiles(1, L // B, 8, seed=13)
+    ref = oracle.pisa_attention_ex(q, k, v, B, K, 1, hybrid=(path == "hybrid_tc"), tiles=tiles)
+    assert rel_l2(rows_of(got, tiles, B), ref) <= TOL["bf16"]
