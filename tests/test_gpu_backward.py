@@ -178,3 +178,21 @@ def test_autograd_function():
           oracle.pisa_backward(q, k, v, dO, B, K, 1), dt)
     with pytest.raises(pisa.PisaError):
         pisa.pisa_attention_autograd(qt, kt, vt, B, K, 1, path="hybrid_tc")
+
+
+def test_autograd_four_dimensional_inputs_with_routing_and_order2():
+    # [batch, heads, L, d] tensors through the autograd wrapper; covariance-aware routing and
+    # the gated second order; compared with the oracle on the folded [batch*heads, L, d] view
+    dt, L, d, B, K = "bf16", 512, 64, 64, 2
+    q, k, v, dO = inputs(1850, 6, L, d, dt, scale=3.0)
+    shape4 = (2, 3, L, d)
+    qt, kt, vt = (dev(x, dt).reshape(shape4).requires_grad_() for x in (q, k, v))
+    out = pisa.pisa_attention_autograd(qt, kt, vt, B, K, 2, route="cov")
+    assert out.shape == shape4
+    out.backward(dev(dO, dt).reshape(shape4))
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    want_o = oracle.pisa_attention_ex(q, k, v, B, K, 2, route_eps=pisa.ROUTE_EPS)
+    assert oracle.rel_l2(out.detach().float().reshape(6, L, d).cpu().numpy(), want_o) <= TOL[dt]
+    got = [t.grad.float().reshape(6, L, d).cpu().numpy().astype(np.float64) for t in (qt, kt, vt)]
+    check(got, oracle.pisa_backward(q, k, v, dO, B, K, 2, True, route_eps=pisa.ROUTE_EPS), dt)
