@@ -555,9 +555,10 @@ def main():
                    "ms_per_call": b_ms, "algorithmic_flops_per_call": alg,
                    "algorithmic_tflops": alg / (b_ms * 1e-3) / 1e12,
                    "executed_tflops": executed / (b_ms * 1e-3) / 1e12,
-                   "roofline": {"bound": "tensor", "peak": bf16_peak, "unit": "TFLOP/s",
-                                "frac": alg / (b_ms * 1e-3) / 1e12 / bf16_peak,
-                                "peak_source": f"{peak_kind} bf16 dense (burst)"},
+                   "roofline": ({"bound": "tensor", "peak": bf16_peak, "unit": "TFLOP/s",
+                                 "frac": alg / (b_ms * 1e-3) / 1e12 / bf16_peak,
+                                 "peak_source": f"{peak_kind} bf16 dense (burst)"}
+                                if tdt == torch.bfloat16 else None),
                    "tile_products": ("warp-level mma.sync m16n8k16, bf16 operands, fp32 accumulation"
                                      if tdt == torch.bfloat16 else "fp32 FMA"),
                    "launches_per_call": 5}
