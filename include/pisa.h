@@ -293,7 +293,11 @@ size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype 
  * Shapes as for pisa_attention plus batch * heads <= 65535.  bf16 inputs run
  * their tile products on the tensor cores (fp32 accumulation; P and dS are
  * rounded to bf16 as the operands of the dk, dv and dq products); fp32 inputs
- * run in fp32 throughout. */
+ * run in fp32 throughout.
+ * Errors (before anything is enqueued): INVALID_ARG for a null or misaligned
+ * pointer, unknown flag bits, K out of range or a small workspace;
+ * UNSUPPORTED for the pooled w, batch * heads > 65535 and the shapes
+ * pisa_attention does not support. */
 pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                     int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
                                     int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
