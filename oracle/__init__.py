@@ -262,4 +262,38 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
 
 
+def parity_metrics(got, ref) -> dict:
+    """Comparison figures of a result ``got`` against the oracle's ``ref`` (same shape; the
+    last axis is one output row):
+      rel_l2   ||got - ref||_F / ||ref||_F over everything compared;
+      row_max  max over rows t of ||got_t - ref_t|| / ||ref_t|| (rows whose reference norm is
+               below 1e-6 of the rms row norm are skipped: their relative error means nothing);
+      row_worst the index of that row in the flattened row list (-1 if none);
+      elem_max max over elements of |got - ref| / (rms(ref) + |ref|), rms over everything
+               compared, i.e. the smallest e with |got - ref| <= e rms(ref) + e |ref| everywhere;
+      rows     the number of rows compared."""
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    if g.shape != r.shape:
+        raise ValueError(f"shape mismatch {g.shape} vs {r.shape}")
+    d = g.shape[-1] if g.ndim else 1
+    g2, r2 = g.reshape(-1, d), r.reshape(-1, d)
+    diff = g2 - r2
+    rn = np.linalg.norm(r2, axis=1)
+    dn = np.linalg.norm(diff, axis=1)
+    rms_row = float(np.sqrt(np.mean(rn * rn))) if rn.size else 0.0
+    live = rn > 1e-6 * max(rms_row, 1e-300)
+    row_err = dn[live] / rn[live] if live.any() else np.zeros(0)
+    rms = float(np.sqrt(np.mean(r2 * r2))) if r2.size else 0.0
+    ratio = np.abs(diff) / (rms + np.abs(r2) + 1e-300)
+    worst = int(np.argmax(row_err)) if row_err.size else -1
+    return {
+        "rel_l2": float(np.linalg.norm(diff) / max(np.linalg.norm(r2), 1e-300)),
+        "row_max": float(row_err.max()) if row_err.size else 0.0,
+        "row_worst": int(np.flatnonzero(live)[worst]) if worst >= 0 else -1,
+        "elem_max": float(ratio.max()) if ratio.size else 0.0,
+        "rows": int(r2.shape[0]),
+    }
+
+
 LN = math.log

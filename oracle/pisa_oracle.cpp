@@ -20,8 +20,7 @@
 //           (o_t = N_t / D_t and D_t), Figure 3 caption (prepare phase),
 //           Appendix C "Notation" (k-bar_j, alpha_{t,j}, delta_{t,j,n}).
 //
-// Readings taken where the pages are silent (each is also listed in the
-// design notes):
+// Readings taken where the pages are silent:
 //   * N_t is not printed in any surviving equation; [blog1] "Sparse Linear
 //     Attention" names its three parts (exact, zeroth order, first-order
 //     correction with H_j), which gives

@@ -4,8 +4,10 @@ Callers that may not allocate device memory (a plugin whose host application
 owns the whole device memory pool, or a loop where cudaMalloc/cudaFree are not
 allowed) use this entry point; it takes its scratch from an array built into
 the library instead of a caller workspace.  These tests call it through the C
-ABI and check that it returns what pisa_attention returns, on two calls in a
-row (the second call finds the first call's data still in the shared scratch).
+ABI and check that it returns what pisa_attention returns, bit for bit (both
+run the same deterministic kernels on the same inputs), on two calls in a row
+(the second call finds the first call's data still in the shared scratch), and
+that a call leaves the device's free memory and torch's allocation unchanged.
 
 This file is collected last on purpose, so that a run stopping at its first
 failure has already run every other test.
@@ -46,11 +48,30 @@ def test_noalloc_matches_pisa_attention_on_two_calls(dt, d, B, order, L, BH):
                    pisa_synth.random_qkv(900 + seed, BH, L, d, scale=2.0,
                                          dtype="bf16" if dt == torch.bfloat16 else "f32"))
         ref = pisa.pisa_attention(q, k, v, B, K, order)
-        out = torch.empty_like(q)
+        out = torch.full_like(q, float("nan"))
         assert _c_noalloc(q, k, v, B, K, order, out) == pisa.PISA_OK, pisa.lib().pisa_last_error()
         pisa.pisa_poll_device_status()
+        assert torch.equal(out, ref)
         err = oracle.rel_l2(out.float().cpu().numpy(), ref.float().cpu().numpy())
         assert err <= TOL[dt], err
+
+
+@pytest.mark.gpu
+def test_noalloc_call_allocates_no_device_memory():
+    # After a first call on the device (which resolves the scratch array's address and loads the
+    # library's kernels), further calls change neither the device's free memory nor torch's
+    # allocation.
+    q, k, v = (torch.from_numpy(x).to("cuda").to(torch.bfloat16) for x in
+               pisa_synth.random_qkv(950, 4, 4096, 128, scale=2.0, dtype="bf16"))
+    out = torch.empty_like(q)
+    assert _c_noalloc(q, k, v, 64, 8, 1, out) == pisa.PISA_OK, pisa.lib().pisa_last_error()
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(3):
+        assert _c_noalloc(q, k, v, 64, 8, 1, out) == pisa.PISA_OK, pisa.lib().pisa_last_error()
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
 
 
 @pytest.mark.gpu
