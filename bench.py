@@ -10,11 +10,17 @@ that each kernel is bracketed by CUDA events on the launching stream.
 Default workload: Wan2.1-shaped attention, 1 x 40 heads, L = 32768, d = 128,
 bf16, B = 64, K = 77, order 1 (inputs 1 GiB > L2, so no flush is needed
 between steps).  Metric: full-attention-equivalent TFLOP/s, 4 L^2 d H / t,
-whole job (sum over ranks; weak scaling: every rank runs the full workload on
-its own inputs).
+whole job.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-Multi-GPU: launched by torch.distributed.run, one rank per GPU.
+                       [--shard heads|replicas]
+Multi-GPU: one rank per GPU.  Under torch.distributed.run WORLD_SIZE must equal
+--gpus; without it, --gpus N > 1 starts N ranks through torch.distributed.run
+itself.  --shard heads (default): the workload's (batch, head) units are split
+across the ranks, each rank times its own slice with the unchanged single-GPU
+call, and the value is the whole workload over the slowest rank's time (strong
+scaling; no collective on the data path).  --shard replicas: every rank runs
+the whole workload on its own inputs (weak scaling).
 """
 from __future__ import annotations
 
@@ -52,7 +58,37 @@ def parse():
     p.add_argument("--no-route", action="store_true", help="skip the covariance-aware routing record")
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass record")
     p.add_argument("--no-dense", action="store_true", help="skip the dense-SDPA context record")
+    p.add_argument("--shard", default="heads", choices=["heads", "replicas"],
+                   help="multi-GPU split: the workload's heads across ranks, or one replica per rank")
     return p.parse_args()
+
+
+def world_plan(gpus: int, env) -> str:
+    """"run" when the process layout matches --gpus, "launch" when N > 1 ranks must be
+    started (no torch.distributed.run around this process); raises SystemExit when
+    WORLD_SIZE contradicts --gpus."""
+    if gpus < 1:
+        raise SystemExit(f"--gpus must be >= 1 (got {gpus})")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}: launch one rank per GPU")
+        return "run"
+    return "launch" if gpus > 1 else "run"
+
+
+def launch_ranks(gpus: int) -> int:
+    """Start --gpus ranks of this same command through torch.distributed.run (one node,
+    rendezvous on 127.0.0.1) and return their exit status."""
+    import socket
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def load_peaks():
@@ -209,10 +245,12 @@ def rank_workload(w, rank: int):
     return w.with_(seed=w.seed + 1000 * rank) if rank else w
 
 
-def cpu_baseline(w, q, k, v, budget_s=20.0):
+def cpu_baseline(w, q, k, v, tiles_per_thread=4):
     """Time the CPU oracle, as it stands, on a bounded sample of the workload:
-    the block statistics of head 0 plus a few query tiles of head 0,
-    extrapolated to the whole call (all heads, all tiles)."""
+    the block statistics of head 0 plus a few query tiles of head 0 (spread
+    evenly, first and last included), extrapolated to the whole call (all
+    heads, all tiles).  The oracle's output rows of those tiles are returned
+    under "_ref" for the parity record."""
     import oracle
 
     nthreads = oracle.default_threads()
@@ -220,10 +258,10 @@ def cpu_baseline(w, q, k, v, budget_s=20.0):
     t0 = time.perf_counter()
     oracle.block_stats(kh, vh, w.B, order=w.order, nthreads=nthreads)
     t_stats = time.perf_counter() - t0
-    ntiles = max(1, min(w.nblk, nthreads))
-    tiles = [(0, int(i)) for i in np.linspace(0, w.nblk - 1, ntiles).round()]
+    ntiles = max(1, min(w.nblk, tiles_per_thread * nthreads))
+    tiles = sorted({(0, int(i)) for i in np.linspace(0, w.nblk - 1, ntiles).round()})
     t0 = time.perf_counter()
-    oracle.pisa_attention(qh, kh, vh, w.B, w.K, w.order, tiles=tiles, nthreads=nthreads)
+    ref = oracle.pisa_attention(qh, kh, vh, w.B, w.K, w.order, tiles=tiles, nthreads=nthreads)
     t_call = time.perf_counter() - t0
     # oracle.pisa_attention also recomputes the head's statistics and selection
     t_tiles = max(t_call - t_stats, 1e-9)
@@ -240,7 +278,30 @@ def cpu_baseline(w, q, k, v, budget_s=20.0):
                    f"({t_tiles:.2f} s, includes re-running that head's statistics and selection); extrapolated to "
                    f"{w.BH} heads x {w.nblk} tiles = {t_full:.0f} s per call"),
         "seconds_measured": t_stats + t_call,
+        "_ref": (tiles, ref),
     }
+
+
+def parity_record(w, out, mask, q_h, k_h, ref_tiles):
+    """The timed step's output against the oracle on the sampled tiles of head 0 (rel-L2, worst
+    row, worst element; tolerance 2e-2 bf16 / 1e-4 fp32), and the GPU selection of head 0
+    against the oracle's canonical selection (every query tile; must be 0 mismatches)."""
+    import oracle
+
+    tiles, ref = ref_tiles
+    B = w.B
+    got = np.stack([out[bh, i * B:(i + 1) * B].float().cpu().numpy() for bh, i in tiles])
+    m = oracle.parity_metrics(got, ref)
+    _, rmask, _ = oracle.select(q_h[:1], k_h[:1], B, w.K)
+    gmask = mask[0].cpu().numpy().view(np.uint32)
+    bad_tiles = int(np.sum(np.any(gmask != rmask[0], axis=1)))
+    bad_bits = int(sum(bin(int(x)).count("1") for x in np.bitwise_xor(gmask, rmask[0]).ravel()))
+    tol = 2e-2 if w.dtype == "bf16" else 1e-4
+    return {"rows_compared": m["rows"], "tiles": f"{len(tiles)} query tiles of head 0 (first, last, evenly spread)",
+            "rel_l2": m["rel_l2"], "row_max": m["row_max"], "elem_max": m["elem_max"], "tolerance": tol,
+            "within_tolerance": bool(m["rel_l2"] <= tol and m["row_max"] <= tol and m["elem_max"] <= tol),
+            "selection_mismatches": bad_tiles, "selection_bits_differing": bad_bits,
+            "selection_tiles_compared": int(gmask.shape[0])}
 
 
 def cpu_backward_baseline(w, q, k, v, dO):
@@ -274,6 +335,50 @@ def cpu_backward_baseline(w, q, k, v, dO):
             "seconds_measured": t1 + t8}
 
 
+def algorithmic_flops(w) -> float:
+    """The method's FLOPs per call (all heads): exact blocks 4 L K B d, centroid scores
+    2 L nblk d, zeroth order 2 L nU d, first order 2 L nU d^2 (order >= 1) and the exact
+    second-order mass 2 L nU d^2 (order 2), nU = nblk - K."""
+    nU = w.nblk - w.K
+    f = 4.0 * w.L * w.K * w.B * w.d + 2.0 * w.L * w.nblk * w.d + 2.0 * w.L * nU * w.d
+    if w.order >= 1:
+        f += 2.0 * w.L * nU * w.d * w.d
+    if w.order == 2:
+        f += 2.0 * w.L * nU * w.d * w.d
+    return f * w.BH
+
+
+def stc_executed_flops(w, mask) -> float:
+    """FLOPs the statistics-form tensor-core kernel executes for this selection: per CTA of
+    256 rows, its union U of the selected blocks of its query tiles runs in 128-key tiles
+    (S and PV: 4 d 128 per row and tile), every other block in items of g blocks (one MMA
+    with N = g d + 16 per row: 2 d (g d + 16)), g = 2 for d = 64 and 1 for d = 128."""
+    m = mask.cpu().numpy().view(np.uint32)  # [BH, nblk, words]
+    BH, nblk, words = m.shape
+    nqt, bpt, gb = 256 // w.B, 128 // w.B, (2 if w.d == 64 else 1)
+    ncta = (w.L + 255) // 256
+    pad = ncta * nqt - nblk
+    if pad > 0:
+        # rows past L repeat the last tile's selection (the kernel clamps the tile index)
+        m = np.concatenate([m, np.repeat(m[:, -1:], pad, axis=1)], axis=1)
+    u = np.bitwise_or.reduce(m.reshape(BH, ncta, nqt, words), axis=2)
+    nu = np.unpackbits(u.view(np.uint8), axis=-1).reshape(BH, ncta, -1).sum(axis=-1).astype(np.int64)
+    nut = (nu + bpt - 1) // bpt
+    ni = (nblk - nu + gb - 1) // gb
+    per_row = 4.0 * w.d * 128 * nut + 2.0 * w.d * (gb * w.d + 16) * ni
+    return float(256.0 * per_row.sum())
+
+
+def stats_bytes(w, order, es, kaug) -> float:
+    """Compulsory HBM bytes of the statistics kernel: read K and V, write kbar and vsum
+    (fp32), H_j (and C_j for order 2) in the input dtype, and the bf16 centroid split."""
+    b = 2.0 * w.BH * w.L * w.d * es + 2.0 * w.BH * w.nblk * w.d * 4
+    b += w.BH * w.nblk * w.d * w.d * es * (2 if order == 2 else 1)
+    if kaug:
+        b += w.BH * w.nblk * 8 * w.d * 2
+    return b
+
+
 def describe(w) -> str:
     """One-line description of a named workload (its shape and generator)."""
     shape = {"c3": "Wan2.1-shaped DiT attention", "c4": "Hunyuan-Video-shaped DiT attention"}.get(w.name)
@@ -303,6 +408,7 @@ def run_reference(args):
     base = None
     for _ in range(args.warmup + args.steps):
         r = cpu_baseline(w, q, k, v)
+        r.pop("_ref", None)
         times.append(r)
         base = r
     vals = [r["value"] for r in times[args.warmup:]] or [base["value"]]
@@ -322,6 +428,8 @@ def run_reference(args):
 
 def main():
     args = parse()
+    if world_plan(args.gpus, os.environ) == "launch":
+        sys.exit(launch_ranks(args.gpus))
     if args.impl == "reference":
         run_reference(args)
         return
@@ -332,16 +440,40 @@ def main():
 
     world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
-    w = pisa_synth.workloads()[args.workload]
+    w_all = pisa_synth.workloads()[args.workload]
     if args.heads:
-        w = w.with_(heads=args.heads)
-    # weak scaling: every rank draws its own inputs of the full workload
-    wr = rank_workload(w, rank)
-    q_h, k_h, v_h = pisa_synth.generate(wr)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    q = torch.from_numpy(q_h).to(tdt).cuda()
-    k = torch.from_numpy(k_h).to(tdt).cuda()
-    v = torch.from_numpy(v_h).to(tdt).cuda()
+        w_all = w_all.with_(heads=args.heads)
+    tdt = torch.bfloat16 if w_all.dtype == "bf16" else torch.float32
+    sharded = world > 1 and args.shard == "heads"
+    if sharded:
+        # one workload, its (batch, head) units split across the ranks: rank 0 draws the
+        # inputs once and broadcasts them (before anything is timed); each rank keeps its slice
+        from block_sparse_taylor_b200 import shard
+
+        u0, u1 = shard.unit_range(w_all.BH, world, rank)
+        full = []
+        if rank == 0:
+            q_h, k_h, v_h = pisa_synth.generate(w_all)
+            full = [torch.from_numpy(x).to(tdt).cuda() for x in (q_h, k_h, v_h)]
+        else:
+            q_h = k_h = v_h = None
+            full = [torch.empty((w_all.BH, w_all.L, w_all.d), dtype=tdt, device="cuda") for _ in range(3)]
+        import torch.distributed as dist
+
+        for t in full:
+            dist.broadcast(t, src=0)
+        q, k, v = (t[u0:u1].clone() for t in full)
+        del full
+        torch.cuda.synchronize()
+        w = w_all.with_(heads=u1 - u0, batch=1)
+    else:
+        # one rank, or weak scaling: every rank draws its own inputs of the whole workload
+        u0, u1 = 0, w_all.BH
+        w = rank_workload(w_all, rank)
+        q_h, k_h, v_h = pisa_synth.generate(w)
+        q = torch.from_numpy(q_h).to(tdt).cuda()
+        k = torch.from_numpy(k_h).to(tdt).cuda()
+        v = torch.from_numpy(v_h).to(tdt).cuda()
     BH, L, d, B, K, order = w.BH, w.L, w.d, w.B, w.K, w.order
     nblk = L // B
     path = pisa.pisa_resolve_path(1, BH, L, d, B, K, order, tdt)
@@ -352,14 +484,15 @@ def main():
     mask = torch.empty((BH, nblk, words), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
     stats_full = None
-    if path == "stats":
-        stats_full = pisa.pisa_stats(k, v, B, order)
+    stats_order = 1 if path == "stats_tc" else order  # the tensor-core statistics form reads H_j only
+    if path in ("stats", "stats_tc"):
+        stats_full = pisa.pisa_stats(k, v, B, stats_order)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        if path == "stats":
-            st = pisa.pisa_stats(k, v, B, order, buf=stats_full.buf)
+        if path in ("stats", "stats_tc"):
+            st = pisa.pisa_stats(k, v, B, stats_order, buf=stats_full.buf)
         else:
             st = pisa.pisa_centroids(k, B, kbar=kbar)
         if ev is not None:
@@ -369,7 +502,7 @@ def main():
                                     mask.data_ptr(), stream.cuda_stream))
         if ev is not None:
             ev[2].record(stream)
-        pisa.pisa_fused_attention(q, k, v, B, mask, order, path=path, stats=st if path == "stats" else None,
+        pisa.pisa_fused_attention(q, k, v, B, mask, order, path=path, stats=st if path != "recompute_tc" else None,
                                   out=out)
         if ev is not None:
             ev[3].record(stream)
@@ -417,17 +550,31 @@ def main():
     step_spans = sorted(e[0].elapsed_time(e[3]) for e in evs)  # this rank's per-step spans
     step_pct = {"p10": pct(step_spans, 10), "median": pct(step_spans, 50), "p90": pct(step_spans, 90)}
 
-    dense_flops = 4.0 * L * L * d * BH
-    value = dense_flops * world / (ms_step * 1e-3) / 1e12
+    dense_flops = 4.0 * L * L * d * BH  # this rank's share
+    # the whole job: every unit of the workload once (head-sharded), or one workload per rank
+    job_flops = 4.0 * L * L * d * w_all.BH if sharded else dense_flops * world
+    value = job_flops / (ms_step * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
-    if path == "recompute_tc":
-        exec_flops = 4.0 * L * L * d * BH  # QK^T and PV over every key block
-        achieved = exec_flops / (attn_ms * 1e-3) / 1e12
+    if path in ("recompute_tc", "stats_tc"):
+        # achieved = the method's algorithmic FLOPs (exact blocks, centroid scores,
+        # zeroth- and first-order terms) per launch over the kernel's event time;
+        # the FLOPs of the association actually executed are reported beside them
+        alg_flops = algorithmic_flops(w)
+        if path == "recompute_tc":
+            exec_flops = 4.0 * L * L * d * BH  # QK^T and PV over every key block
+            kname = f"attn_tc_kernel<{d},{B},{order}>"
+        else:
+            exec_flops = stc_executed_flops(w, mask)
+            kname = f"attn_stc_kernel<{d},{B},{order}>"
+        achieved = alg_flops / (attn_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": traffic_record(w.name) if not args.heads else None,
-                "kernel": f"attn_tc_kernel<{d},{B}>",
-                "algorithmic_flops_per_launch": exec_flops,
+                "traffic": traffic_record(w.name) if (not args.heads and path == "recompute_tc") else None,
+                "kernel": kname,
+                "algorithmic_flops_per_launch": alg_flops,
+                "executed_flops_per_launch": exec_flops,
+                "executed_tflops": exec_flops / (attn_ms * 1e-3) / 1e12,
+                "executed_frac": exec_flops / (attn_ms * 1e-3) / 1e12 / peak,
                 "peak_source": f"{peak_kind} bf16 dense (burst; the kernel is timed alone inside the step)"}
     else:
         # statistics path: CUDA-core kernel; report against the HBM roofline of its reads
@@ -436,11 +583,19 @@ def main():
         peak = float(peaks["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": None, "kernel": f"attn_stats_kernel<{d},{B}>", "peak_source": peak_kind}
-    # HBM figures of the small kernels (centroids read K once; select reads Q once + writes the mask)
-    prep_bytes = BH * L * d * q.element_size() + BH * nblk * d * 4
-    sel_bytes = BH * L * d * q.element_size() + BH * nblk * (words + K) * 4
+    # HBM figures of the small kernels (centroids read K once, or the statistics
+    # kernel reads K and V and writes the statistics; select reads Q once + writes the mask)
+    es = q.element_size()
+    if path in ("stats", "stats_tc"):
+        prep_bytes = stats_bytes(w, stats_order, es, kaug=(path == "stats_tc"))
+        prep_name = ("stats_tc_kernel" if tdt == torch.bfloat16 else "stats_simt_kernel") + f"<{d},{B},{stats_order}>"
+    else:
+        prep_bytes = BH * L * d * es + BH * nblk * d * 4
+        prep_name = f"centroid_kernel<{d},{B}>"
+    sel_bytes = BH * L * d * es + BH * nblk * (words + K) * 4
     hbm = float(peaks["hbm_gbs"])
     per_kernel = {
+        "prep_kernel": prep_name,
         "centroids_ms": statistics.mean(k_prep), "select_ms": statistics.mean(k_sel), "attn_ms": attn_ms,
         "centroids_gbs": prep_bytes / (statistics.mean(k_prep) * 1e-3) / 1e9,
         "select_gbs": sel_bytes / (statistics.mean(k_sel) * 1e-3) / 1e9,
@@ -452,7 +607,7 @@ def main():
     # C_j) is not on the token-form path; it is timed here on its own against
     # the HBM roofline of its compulsory traffic.
     stats_rec = None
-    if path != "stats":
+    if path not in ("stats", "stats_tc"):
         sorder = max(order, 1)
         sbuf = torch.empty(pisa.pisa_stats_bytes(1, BH, L, d, B, sorder, tdt), dtype=torch.uint8, device="cuda")
         for _ in range(2):
@@ -465,8 +620,7 @@ def main():
         sb.record(stream)
         torch.cuda.synchronize()
         s_ms = sa.elapsed_time(sb) / reps
-        es = q.element_size()
-        s_bytes = 2 * BH * L * d * es + 2 * BH * nblk * d * 4 + BH * nblk * d * d * es * (2 if sorder == 2 else 1)
+        s_bytes = stats_bytes(w, sorder, es, kaug=(tdt == torch.bfloat16))
         kname = "stats_tc_kernel" if tdt == torch.bfloat16 else "stats_simt_kernel"
         stats_rec = {"kernel": f"{kname}<{d},{B},{sorder}>", "order": sorder, "ms": s_ms,
                      "algorithmic_bytes": s_bytes, "gbs": s_bytes / (s_ms * 1e-3) / 1e9,
@@ -599,9 +753,11 @@ def main():
         torch.cuda.synchronize()
         barrier(world)
         e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world)
-        e2e = {"value": dense_flops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
-               "d2h_bytes_per_step": out.numel() * out.element_size(),
+        job_units = w_all.BH if sharded else BH * world
+        unit_bytes = L * d * q.element_size()
+        e2e = {"value": job_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * job_units * unit_bytes,
+               "d2h_bytes_per_step": job_units * unit_bytes,
                "call": f"pisa_attention_host, {plan.chunk} heads per chunk, two streams"}
         pisa.pisa_poll_device_status()
         del plan
@@ -613,17 +769,25 @@ def main():
             dense_rec["speedup_of_pisa_step"] = dense_rec["ms_per_call"] / ms_step
 
     cpu = None
+    par = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, q_h, k_h, v_h)
+        try:
+            par = parity_record(w, out, mask, q_h, k_h, cpu.pop("_ref"))
+        except Exception as e:  # noqa: BLE001 - reported, never raised
+            par = {"unavailable": f"{type(e).__name__}: {e}"[:240]}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": describe(w),
-                       "path": path, "global_batch": world, "seq_len": L,
-                       "parallelism": f"replicas x{world} (heads independent, no collective)",
+            "config": {"workload": describe(w_all),
+                       "path": path, "global_batch": 1 if sharded else world, "seq_len": L,
+                       "parallelism": (f"heads sharded over {world} ranks (rank 0: units {u0}..{u1 - 1} of "
+                                       f"{w_all.BH}; no data-path collective)" if sharded else
+                                       f"replicas x{world} (heads independent, no collective)"),
                        "l2": ("inputs exceed L2 (3 x {:.0f} MiB per rank), no flush" if big_inputs else
                               "inputs fit in L2 (3 x {:.0f} MiB per rank); L2 flushed before every step").format(
                            q.numel() * q.element_size() / 2 ** 20)},
@@ -636,6 +800,7 @@ def main():
             "step_ms_percentiles": step_pct,
             "dense_sdpa_context": dense_rec,
             "cpu_baseline": cpu,
+            "parity": par,
             "clocks": clk,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,

@@ -36,7 +36,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libpisa_b200.so")
 
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
 PISA_F32, PISA_BF16 = 0, 1
-PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2, "hybrid_tc": 3}
+PATHS = {"auto": 0, "stats": 1, "recompute_tc": 2, "hybrid_tc": 3, "stats_tc": 4}
 FLAG_GATE_W, FLAG_POOLED_W, FLAG_COV_ROUTE = 1, 2, 4
 ROUTE_EPS = 1e-6
 PATH_NAMES = {v: k for k, v in PATHS.items()}
@@ -56,7 +56,7 @@ class _StatsT(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("heads", ctypes.c_int), ("L", ctypes.c_int), ("d", ctypes.c_int),
                 ("B", ctypes.c_int), ("nblk", ctypes.c_int), ("order", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("kbar", ctypes.c_void_p), ("vsum", ctypes.c_void_p), ("hstat", ctypes.c_void_p),
-                ("cov", ctypes.c_void_p)]
+                ("cov", ctypes.c_void_p), ("kaug", ctypes.c_void_p)]
 
 
 _lib = None
@@ -103,6 +103,8 @@ def lib():
         L.pisa_backward_workspace_bytes.restype = sz
         L.pisa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
         L.pisa_selftest_wait_timeout.restype = ctypes.c_int
+        L.pisa_selftest_ex2.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
+        L.pisa_selftest_ex2.restype = ctypes.c_int
         for fn in ("pisa_attention_noalloc", "pisa_centroids", "pisa_fused_attention", "pisa_stats_bind", "pisa_stats", "pisa_select", "pisa_attention", "pisa_attention_ex",
                    "pisa_poll_device_status", "pisa_resolve_path"):
             getattr(L, fn).restype = ctypes.c_int
@@ -156,6 +158,7 @@ class Stats(NamedTuple):
     cov: Optional[torch.Tensor]    # [BH, nblk, d, d]
     raw: _StatsT
     buf: torch.Tensor
+    kaug: Optional[torch.Tensor] = None  # [BH, nblk, 8, d] bf16: high and low parts of kbar, zero rows
 
 
 def pisa_stats_bytes(batch, heads, L, d, B, order, dtype: torch.dtype) -> int:
@@ -197,7 +200,8 @@ def _stats_views(st: _StatsT, buf: torch.Tensor, dtype: torch.dtype) -> Stats:
     vsum = view(st.vsum, (BH, st.nblk, st.d), torch.float32)
     hstat = view(st.hstat, (BH, st.nblk, st.d, st.d), dtype)
     cov = view(st.cov, (BH, st.nblk, st.d, st.d), dtype)
-    return Stats(kbar, vsum, hstat, cov, st, buf)
+    kaug = view(st.kaug, (BH, st.nblk, 8, st.d), torch.bfloat16)
+    return Stats(kbar, vsum, hstat, cov, st, buf, kaug)
 
 
 def pisa_centroids(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, stream=None) -> Stats:
@@ -209,7 +213,7 @@ def pisa_centroids(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None,
         kbar = torch.empty((batch * heads, L // B, d), dtype=torch.float32, device=k.device)
     _check(lib().pisa_centroids(k.data_ptr(), batch, heads, L, d, _dtype_code(k.dtype), B, kbar.data_ptr(),
                                 _stream(stream)))
-    st = _StatsT(batch, heads, L, d, B, L // B, 0, _dtype_code(k.dtype), kbar.data_ptr(), None, None, None)
+    st = _StatsT(batch, heads, L, d, B, L // B, 0, _dtype_code(k.dtype), kbar.data_ptr(), None, None, None, None)
     return Stats(kbar, None, None, None, st, kbar)
 
 
@@ -434,6 +438,19 @@ def pisa_selftest_wait_timeout(limit_cycles: int = 2_000_000, stream=None):
     include/pisa.h).  The next pisa_poll_device_status raises PisaError with status
     PISA_ERR_DEVICE_TIMEOUT."""
     _check(lib().pisa_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
+
+
+def pisa_selftest_ex2(x: torch.Tensor, which: str = "fma", out: Optional[torch.Tensor] = None, stream=None):
+    """y = 2^x element-wise with one of the kernels' exponentials: "fma" (the FMA-pipe
+    polynomial) or "sfu" (ex2.approx); x a contiguous fp32 CUDA tensor."""
+    _need_cuda(x)
+    if x.dtype != torch.float32:
+        raise TypeError("pisa_selftest_ex2 takes float32")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().pisa_selftest_ex2(x.data_ptr(), out.data_ptr(), x.numel(), {"fma": 0, "sfu": 1}[which],
+                                   _stream(stream)))
+    return out
 
 
 def pisa_poll_device_status(stream=None):

@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
                         for (int b = 0; b < D; ++b) t = fmaf(to_f(ca[b]), qr[b], t);
                         part = fmaf(qr[a], t, part);
                     }
-                    wq = 0.5f * warp_sum(part);
+                    // C_j is PSD, so w >= 0 (Jensen); rounding of the stored C_j must not make it negative
+                    wq = fmaxf(0.5f * warp_sum(part), 0.f);
                     if (gate && wq > ln_b) wq = 0.f;
                 }
                 const float l = s + wq;

@@ -89,27 +89,38 @@ __device__ __forceinline__ float block_pass1(const uint32_t* x, bool sel, int ga
         l2 = 0.f;
         return tc::max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * LOG2E;
     }
-    uint64_t s2[4], q2[4];
+    uint64_t s2[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        s2[a] = tc::f2_make(__uint_as_float(x[2 * a]), __uint_as_float(x[2 * a + 1]));
-        if (ORDER == 2) q2[a] = tc::f2_mul(s2[a], s2[a]);
-    }
+    for (int a = 0; a < 4; ++a) s2[a] = tc::f2_make(__uint_as_float(x[2 * a]), __uint_as_float(x[2 * a + 1]));
 #pragma unroll
     for (int e = 8; e < N; e += 8)
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const uint64_t p = tc::f2_make(__uint_as_float(x[e + 2 * a]), __uint_as_float(x[e + 2 * a + 1]));
-            s2[a] = tc::f2_add(s2[a], p);
-            if (ORDER == 2) q2[a] = tc::f2_fma(p, p, q2[a]);
-        }
+        for (int a = 0; a < 4; ++a)
+            s2[a] = tc::f2_add(s2[a], tc::f2_make(__uint_as_float(x[e + 2 * a]), __uint_as_float(x[e + 2 * a + 1])));
     constexpr float inv_n = 1.0f / (float)N;
     const float2 st = tc::f2_split(tc::f2_add(tc::f2_add(s2[0], s2[1]), tc::f2_add(s2[2], s2[3])));
     const float sb = (st.x + st.y) * inv_n;
     float w = 0.f;
     if (ORDER == 2) {
+        // second pass over the deviations x_n - s-bar: a sum of squares, so w >= 0 as the
+        // pages have it (Jensen), and no cancellation when |s-bar| is large against the spread
+        const uint64_t negs = tc::f2_make(-sb, -sb);
+        uint64_t q2[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const uint64_t t = tc::f2_add(tc::f2_make(__uint_as_float(x[2 * a]), __uint_as_float(x[2 * a + 1])), negs);
+            q2[a] = tc::f2_mul(t, t);
+        }
+#pragma unroll
+        for (int e = 8; e < N; e += 8)
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const uint64_t t = tc::f2_add(
+                    tc::f2_make(__uint_as_float(x[e + 2 * a]), __uint_as_float(x[e + 2 * a + 1])), negs);
+                q2[a] = tc::f2_fma(t, t, q2[a]);
+            }
         const float2 qq = tc::f2_split(tc::f2_add(tc::f2_add(q2[0], q2[1]), tc::f2_add(q2[2], q2[3])));
-        w = 0.5f * fmaf(-sb, sb, (qq.x + qq.y) * inv_n);
+        w = 0.5f * (qq.x + qq.y) * inv_n;
         if (gate && w > ln_b) w = 0.f;
     } else if (ORDER == 3) {
         w = w_pool;

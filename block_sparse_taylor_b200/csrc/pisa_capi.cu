@@ -5,6 +5,7 @@
 // allocates device memory or synchronises, except pisa_poll_device_status.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -21,6 +22,7 @@
 #include "stats_tc.cuh"
 #include "hybrid_prep.cuh"
 #include "attn_hybrid.cuh"
+#include "attn_stc.cuh"
 #include "route.cuh"
 #include "backward.cuh"
 #include "selftest.cuh"
@@ -100,8 +102,11 @@ pisa_status check_align16(const char* where, std::initializer_list<const void*> 
 }
 
 struct StatsLayout {
-    size_t kbar, vsum, hstat, cov, total;
+    size_t kbar, vsum, hstat, cov, kaug, total;
 };
+
+// kaug (the bf16 high/low split of the centroids) exists for bf16, order >= 1
+bool has_kaug(int order, pisa_dtype dtype) { return dtype == PISA_BF16 && order >= 1; }
 
 StatsLayout stats_layout(const Dims& g, int order, pisa_dtype dtype) {
     StatsLayout s{};
@@ -114,6 +119,8 @@ StatsLayout stats_layout(const Dims& g, int order, pisa_dtype dtype) {
     if (order >= 1) o += align_up(esize(dtype) * g.BH * g.nblk * g.d * g.d);
     s.cov = o;
     if (order == 2) o += align_up(esize(dtype) * g.BH * g.nblk * g.d * g.d);
+    s.kaug = o;
+    if (has_kaug(order, dtype)) o += align_up(2 * g.BH * g.nblk * 8 * g.d);
     s.total = o;
     return s;
 }
@@ -183,8 +190,8 @@ pisa_status run_stats(const void* k, const void* v, const pisa_stats_t* st, cons
         // bf16: the Gram products H_j and C_j on the tensor cores
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
-        return pisa::run_stats_tc(k, v, st->kbar, st->vsum, st->hstat, st->cov, g.BH, (int)g.L, (int)g.d, (int)g.B,
-                                  (int)g.nblk, st->order, status, s, &g_last_error);
+        return pisa::run_stats_tc(k, v, st->kbar, st->vsum, st->hstat, st->cov, st->kaug, g.BH, (int)g.L, (int)g.d,
+                                  (int)g.B, (int)g.nblk, st->order, status, s, &g_last_error);
     }
     return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
@@ -291,6 +298,9 @@ WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path 
         // The token-form and hybrid paths need only the fp32 centroids (for the selection).
         w.sl = StatsLayout{};
         w.sl.total = align_up(sizeof(float) * g.BH * g.nblk * g.d);
+    } else if (path == PISA_PATH_STATS_TC) {
+        // kbar, vsum, H_j and the centroid split; the pooled second order needs no C_j
+        w.sl = stats_layout(g, 1, dtype);
     } else {
         w.sl = stats_layout(g, order, dtype);
     }
@@ -336,12 +346,30 @@ bool tc_path_available(const Dims& g, pisa_dtype dtype) {
            g.BH * g.L <= 0x7fffffffL;
 }
 
-// The tensor-core token-form path whenever it can run the shape, else the
+// The statistics form on the tensor cores: first order (or the pooled second order).
+bool stc_path_available(const Dims& g, pisa_dtype dtype, int order, bool pooled) {
+    return tc_path_available(g, dtype) && g.BH * g.nblk * g.d <= 0x7fffffffL &&
+           (order == 1 || (order == 2 && pooled));
+}
+
+// Executed FLOPs per query row of the statistics-form tensor-core kernel with the union of
+// the CTA's selections at its bound min(nblk, (256/B) K), and of the token form (4 L d).
+double stc_flops_per_row(const Dims& g, int K) {
+    const long nqt = 256 / g.B, bpt = 128 / g.B, gb = g.d == 64 ? 2 : 1;
+    const long u = std::min<long>(g.nblk, nqt * (long)K);
+    const long nut = (u + bpt - 1) / bpt, ni = (g.nblk - u + gb - 1) / gb;
+    return 4.0 * g.d * 128.0 * nut + 2.0 * g.d * (gb * g.d + 16) * ni;
+}
+double token_flops_per_row(const Dims& g) { return 4.0 * g.d * g.L; }
+
+// On the tensor cores, the association that executes fewer FLOPs (the statistics
+// form only for order 1: at order 2 its C_j contraction doubles it); else the
 // statistics path on CUDA cores.
 pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
-    (void)K;
-    (void)order;
-    return tc_path_available(g, dtype) ? PISA_PATH_RECOMPUTE_TC : PISA_PATH_STATS;
+    if (!tc_path_available(g, dtype)) return PISA_PATH_STATS;
+    if (stc_path_available(g, dtype, order, false) && stc_flops_per_row(g, K) < token_flops_per_row(g))
+        return PISA_PATH_STATS_TC;
+    return PISA_PATH_RECOMPUTE_TC;
 }
 
 // ---------------------------------------------------------------------------
@@ -409,6 +437,8 @@ pisa_status check_stats(const pisa_stats_t* st, Dims* g) {
     if (!st->kbar || !st->vsum) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null kbar or vsum");
     if (st->order >= 1 && !st->hstat) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null hstat for order >= 1");
     if (st->order == 2 && !st->cov) return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: null cov for order 2");
+    if (st->kaug && !has_kaug(st->order, st->dtype))
+        return fail(PISA_ERR_INVALID_ARG, "pisa_stats_t: kaug is for bf16 statistics of order >= 1 only");
     return PISA_OK;
 }
 
@@ -416,7 +446,7 @@ pisa_status check_stats(const pisa_stats_t* st, Dims* g) {
 
 extern "C" {
 
-const char* pisa_version(void) { return "pisa-b200 0.1"; }
+const char* pisa_version(void) { return "pisa-b200 0.2"; }
 
 const char* pisa_last_error(void) { return g_last_error.c_str(); }
 
@@ -449,6 +479,7 @@ pisa_status pisa_stats_bind(pisa_stats_t* st, void* buf, size_t bytes, int batch
     st->vsum = (float*)(b + s.vsum);
     st->hstat = order >= 1 ? (void*)(b + s.hstat) : nullptr;
     st->cov = order == 2 ? (void*)(b + s.cov) : nullptr;
+    st->kaug = has_kaug(order, dtype) ? (void*)(b + s.kaug) : nullptr;
     return PISA_OK;
 }
 
@@ -457,7 +488,7 @@ pisa_status pisa_stats(const void* k, const void* v, const pisa_stats_t* st, voi
     pisa_status r = check_stats(st, &g);
     if (r != PISA_OK) return r;
     if (!k || !v) return fail(PISA_ERR_INVALID_ARG, "pisa_stats: null k or v");
-    r = check_align16("pisa_stats", {k, v, st->kbar, st->vsum, st->hstat, st->cov});
+    r = check_align16("pisa_stats", {k, v, st->kbar, st->vsum, st->hstat, st->cov, st->kaug});
     if (r != PISA_OK) return r;
     return run_stats(k, v, st, g, (cudaStream_t)stream);
 }
@@ -531,7 +562,11 @@ size_t pisa_workspace_bytes_ex(int batch, int heads, int L, int d, int B, int K,
     if (path == PISA_PATH_AUTO) path = resolve(g, K, order, dtype);
     if (path == PISA_PATH_RECOMPUTE_TC && !tc_path_available(g, dtype)) return 0;
     if (path == PISA_PATH_HYBRID_TC && !hybrid_path_available(g, dtype, order)) return 0;
-    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC) return 0;
+    // order 2 runs on this path only with the pooled w, so size it for that
+    if (path == PISA_PATH_STATS_TC && !stc_path_available(g, dtype, order, order == 2)) return 0;
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC &&
+        path != PISA_PATH_STATS_TC)
+        return 0;
     return ws_layout(g, K, order, dtype, path).total;
 }
 
@@ -562,7 +597,12 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     const bool route = (gate_w & PISA_FLAG_COV_ROUTE) != 0;
     if (path == PISA_PATH_HYBRID_TC && order == 2 && !pooled)
         return fail(PISA_ERR_UNSUPPORTED, "the hybrid's second order needs the pooled w (PISA_FLAG_POOLED_W)");
-    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC)
+    if (path == PISA_PATH_STATS_TC && !stc_path_available(g, dtype, order, pooled))
+        return fail(PISA_ERR_UNSUPPORTED,
+                    "statistics-form tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0 and order 1 "
+                    "(order 2 only with PISA_FLAG_POOLED_W)");
+    if (path != PISA_PATH_STATS && path != PISA_PATH_RECOMPUTE_TC && path != PISA_PATH_HYBRID_TC &&
+        path != PISA_PATH_STATS_TC)
         return fail(PISA_ERR_INVALID_ARG, "unknown path %d", (int)path);
     const WsLayout w = ws_layout(g, K, order, dtype, path);
     if (ws_bytes < w.total)
@@ -577,11 +617,14 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     st.B = B;
     st.nblk = (int)g.nblk;
     st.dtype = dtype;
-    st.order = (path == PISA_PATH_RECOMPUTE_TC || path == PISA_PATH_HYBRID_TC) ? 0 : order;
+    st.order = (path == PISA_PATH_RECOMPUTE_TC || path == PISA_PATH_HYBRID_TC) ? 0
+               : (path == PISA_PATH_STATS_TC)                                ? 1
+                                                                             : order;
     st.kbar = (float*)(ws + w.stats + w.sl.kbar);
-    st.vsum = (path == PISA_PATH_STATS) ? (float*)(ws + w.stats + w.sl.vsum) : nullptr;
+    st.vsum = (path == PISA_PATH_STATS || path == PISA_PATH_STATS_TC) ? (float*)(ws + w.stats + w.sl.vsum) : nullptr;
     st.hstat = st.order >= 1 ? (void*)(ws + w.stats + w.sl.hstat) : nullptr;
     st.cov = st.order == 2 ? (void*)(ws + w.stats + w.sl.cov) : nullptr;
+    st.kaug = (path == PISA_PATH_STATS_TC) ? (void*)(ws + w.stats + w.sl.kaug) : nullptr;
     uint32_t* mask = (uint32_t*)(ws + w.mask);
     int32_t* idx = (int32_t*)(ws + w.idx);
     float* rbias = route ? (float*)(ws + w.bias) : nullptr;
@@ -632,6 +675,12 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
         return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
                                  (int)g.words, korder, gate, wmat, status, s, &g_last_error);
+    }
+    if (path == PISA_PATH_STATS_TC) {
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        return pisa::run_attn_stc(q, k, v, st.hstat, st.kaug, st.vsum, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B,
+                                  (int)g.nblk, (int)g.words, korder, gate, wmat, status, s, &g_last_error);
     }
     return run_attn_stats(q, k, v, &st, mask, out, g, order, gate, s, wmat);
 }
@@ -714,10 +763,31 @@ pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, in
     r = check_align16("pisa_fused_attention", {q, k, v, out});
     if (r != PISA_OK) return r;
     if (st) {
-        r = check_align16("pisa_fused_attention", {st->kbar, st->vsum, st->hstat, st->cov});
+        r = check_align16("pisa_fused_attention", {st->kbar, st->vsum, st->hstat, st->cov, st->kaug});
         if (r != PISA_OK) return r;
     }
-    if (path == PISA_PATH_AUTO) path = resolve(g, 0, order, dtype);
+    // without K, AUTO here takes the token form on the tensor cores, else the statistics path
+    if (path == PISA_PATH_AUTO) path = tc_path_available(g, dtype) ? PISA_PATH_RECOMPUTE_TC : PISA_PATH_STATS;
+    if (path == PISA_PATH_STATS_TC) {
+        if (!stc_path_available(g, dtype, order, false))
+            return fail(PISA_ERR_UNSUPPORTED, "statistics-form tensor-core path needs bf16, d and B in {64, 128}, "
+                                              "L %% 128 == 0 and order 1");
+        if (gate_w & PISA_FLAG_POOLED_W)
+            return fail(PISA_ERR_UNSUPPORTED, "pisa_fused_attention: the pooled w needs pisa_attention_ex");
+        Dims gs;
+        r = check_stats(st, &gs);
+        if (r != PISA_OK) return r;
+        if (gs.BH != g.BH || gs.L != g.L || gs.d != g.d || gs.B != g.B || st->dtype != dtype)
+            return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: statistics of another shape");
+        if (st->order < 1 || !st->kaug)
+            return fail(PISA_ERR_INVALID_ARG, "pisa_fused_attention: the statistics-form tensor-core path needs "
+                                              "statistics of order >= 1 with kaug");
+        unsigned int* status = device_status_ptr();
+        if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+        return pisa::run_attn_stc(q, k, v, st->hstat, st->kaug, st->vsum, mask, out, g.BH, (int)g.L, (int)g.d,
+                                  (int)g.B, (int)g.nblk, (int)g.words, order, gate_w & PISA_FLAG_GATE_W, nullptr,
+                                  status, (cudaStream_t)stream, &g_last_error);
+    }
     if (path == PISA_PATH_RECOMPUTE_TC) {
         if (!tc_path_available(g, dtype))
             return fail(PISA_ERR_UNSUPPORTED, "tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0");
@@ -750,6 +820,19 @@ pisa_status pisa_selftest_wait_timeout(long long limit_cycles, void* stream) {
     if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
     pisa::wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status, limit_cycles);
     return launch_check("wait_timeout_selftest_kernel");
+}
+
+pisa_status pisa_selftest_ex2(const float* x, float* y, long long n, int which, void* stream) {
+    if (n < 0) return fail(PISA_ERR_INVALID_ARG, "pisa_selftest_ex2: n must be >= 0 (got %lld)", n);
+    if (which != 0 && which != 1) return fail(PISA_ERR_INVALID_ARG, "pisa_selftest_ex2: which must be 0 or 1");
+    if (n == 0) return PISA_OK;
+    if (!x || !y) return fail(PISA_ERR_INVALID_ARG, "pisa_selftest_ex2: null pointer");
+    if ((uintptr_t)x % 4 || (uintptr_t)y % 4)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_selftest_ex2: arrays must be 4-byte aligned");
+    const long long blocks = (n + 255) / 256;
+    pisa::ex2_selftest_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, (cudaStream_t)stream>>>(x, y, n,
+                                                                                                       which);
+    return launch_check("ex2_selftest_kernel");
 }
 
 pisa_status pisa_poll_device_status(void* stream) {

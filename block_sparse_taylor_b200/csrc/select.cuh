@@ -9,8 +9,9 @@
 // Every fp32 operation follows the canonical order of the C ABI comment:
 // tile means by the pairwise tree over the B rows, scores by the pairwise
 // tree over the d products, each product and sum rounded on its own.  The
-// score tree runs on packed fp32x2 operations (two independent IEEE
-// round-to-nearest operations each), which leaves every rounding unchanged.
+// score tree runs on scalar __fmul_rn / __fadd_rn only: packed fp32x2
+// multiplies and adds were measured not to reproduce the separately rounded
+// scalar results.
 #pragma once
 
 #include "common.cuh"

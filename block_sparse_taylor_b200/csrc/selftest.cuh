@@ -26,4 +26,12 @@ __global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(unsigned* sta
     tc::mbar_wait(b, 0, aborted, status, limit);  // phase 0 never completes: times out
 }
 
+// Self-test of the two base-2 exponentials the attention kernels use: which = 0
+// evaluates the FMA-pipe polynomial tc::ex2_fma, which = 1 the special-function
+// unit's ex2.approx, element by element (y[i] = 2^x[i]).
+__global__ void ex2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int which) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        y[i] = which ? tc::ex2(x[i]) : tc::ex2_fma(x[i]);
+}
+
 }  // namespace pisa

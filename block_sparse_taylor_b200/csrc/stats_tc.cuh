@@ -14,6 +14,12 @@
 // d = 64 the A operand is [V_j^T ; K_j^T] stacked to M = 128, so one MMA gives
 // H_j (rows 0-63) and the uncentred C_j (rows 64-127).
 //
+// With kaug non-null it also writes, per block, the eight bf16 rows the
+// statistics-form tensor-core kernel appends to H_j as extra B-operand rows:
+// row 0 = bf16(kbar_j) (round to nearest), row 1 = bf16(kbar_j - row 0), rows
+// 2-7 = 0, so that one MMA gives q . kbar_j as two columns to within about
+// 2^-16 of the fp32 centroid.
+//
 // One CTA (128 threads) per (block, bh): warp 0 allocates TMEM, lane 0 of
 // warp 0 issues the TMA loads and the MMAs; all four warps then compute the
 // column sums from shared memory and run the epilogue (thread = TMEM lane).
@@ -56,8 +62,8 @@ template <int D, int BS, int ORDER>
 __global__ void __launch_bounds__(128) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                        const __grid_constant__ CUtensorMap tm_v,
                                                        float* __restrict__ kbar, float* __restrict__ vsum,
-                                                       bf16* __restrict__ hstat, bf16* __restrict__ cov, int L,
-                                                       int nblk, unsigned* status) {
+                                                       bf16* __restrict__ hstat, bf16* __restrict__ cov,
+                                                       bf16* __restrict__ kaug, int L, int nblk, unsigned* status) {
     using C = StatsTcCfg<D, BS>;
     // M = 128 always (d = 64 stacks V and K); N = d; both operands MN-major
     constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
@@ -125,6 +131,14 @@ __global__ void __launch_bounds__(128) stats_tc_kernel(const __grid_constant__ C
             const size_t so = ((size_t)bh * nblk + j) * D + c;
             kbar[so] = m;
             vsum[so] = s;
+            if (kaug) {
+                bf16* ka = kaug + ((size_t)bh * nblk + j) * 8 * D + c;
+                const bf16 hi = __float2bfloat16_rn(m);
+                ka[0] = hi;
+                ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
+#pragma unroll
+                for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
+            }
         }
     }
     __syncthreads();
@@ -179,9 +193,9 @@ __global__ void __launch_bounds__(128) stats_tc_kernel(const __grid_constant__ C
     }
 }
 
-inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float* vsum, void* hstat, void* cov, long BH,
-                                int L, int d, int B, int nblk, int order, unsigned* status, cudaStream_t s,
-                                std::string* err) {
+inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float* vsum, void* hstat, void* cov,
+                                void* kaug, long BH, int L, int d, int B, int nblk, int order, unsigned* status,
+                                cudaStream_t s, std::string* err) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
@@ -216,7 +230,7 @@ inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float
                                  (int)StatsTcCfg<DD, BB>::SMEM);                                              \
         if (e == cudaSuccess) {                                                                               \
             kern<<<grid, 128, StatsTcCfg<DD, BB>::SMEM, s>>>(maps[0], maps[1], kbar, vsum, (bf16*)hstat,      \
-                                                             (bf16*)cov, L, nblk, status);                    \
+                                                             (bf16*)cov, (bf16*)kaug, L, nblk, status);       \
             e = cudaGetLastError();                                                                           \
         }                                                                                                     \
     } else

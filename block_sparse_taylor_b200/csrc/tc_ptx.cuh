@@ -197,6 +197,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn) {
            ((uint32_t)(M >> 4) << 24);
 }
 
+// Per-warpgroup register budget (setmaxnreg): every thread of the warpgroup
+// executes it.  dec gives registers back to the CTA's pool; inc waits until the
+// pool (the registers the CTA was launched with) can supply them.
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
     float y;

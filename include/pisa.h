@@ -64,8 +64,11 @@ typedef enum {
 typedef enum { PISA_F32 = 0, PISA_BF16 = 1 } pisa_dtype;
 
 /* Which formulation pisa_attention_ex evaluates the unselected blocks with.
- *   PISA_PATH_AUTO          : PISA_PATH_RECOMPUTE_TC when it can run the
- *                             shape, else PISA_PATH_STATS.
+ *   PISA_PATH_AUTO          : on the tensor cores (bf16, d and B in {64, 128},
+ *                             L % 128 == 0) the one of PISA_PATH_RECOMPUTE_TC
+ *                             and PISA_PATH_STATS_TC that executes fewer FLOPs
+ *                             (STATS_TC only for order 1; see below), else
+ *                             PISA_PATH_STATS.
  *   PISA_PATH_STATS         : statistics form: uses kbar_j, vsum_j, H_j, C_j
  *                             from pisa_stats (CUDA cores, fp32 accumulation).
  *   PISA_PATH_RECOMPUTE_TC  : token form on tcgen05 tensor cores: the
@@ -73,12 +76,28 @@ typedef enum { PISA_F32 = 0, PISA_BF16 = 1 } pisa_dtype;
  *                             e^{l}(vsum_j + H_j q) is evaluated as
  *                             sum_n e^{l}(1 + q.(k_n - kbar_j)) v_n, which is
  *                             the same quantity; w is taken from the same
- *                             logits.  bf16 only, L % 128 == 0. */
+ *                             logits.  bf16 only, L % 128 == 0.  Executes
+ *                             4 L^2 d FLOPs per (batch, head).
+ *   PISA_PATH_STATS_TC      : statistics form on tcgen05 tensor cores: blocks
+ *                             selected by any query tile of a 256-row CTA run
+ *                             in the token form above; every other block's
+ *                             term is the contraction H_j q_t (one MMA per
+ *                             128 rows and block, with q_t . kbar_j from the
+ *                             same MMA).  bf16, L % 128 == 0, order 1 (order 2
+ *                             only with PISA_FLAG_POOLED_W).  With U the
+ *                             blocks selected by the CTA's tiles, it executes
+ *                             per 256 rows 256 (4 d 128 ceil(U / (128/B))
+ *                             + 2 d (g d + 16) ceil((L/B - U) / g)) FLOPs,
+ *                             g = 2 for d = 64 and 1 for d = 128: fewer than
+ *                             the token form when d <= B.  AUTO takes it when
+ *                             that count, with U at its bound
+ *                             min(L/B, (256/B) K), is below 4 L d per row. */
 typedef enum {
     PISA_PATH_AUTO = 0,
     PISA_PATH_STATS = 1,
     PISA_PATH_RECOMPUTE_TC = 2,
-    PISA_PATH_HYBRID_TC = 3
+    PISA_PATH_HYBRID_TC = 3,
+    PISA_PATH_STATS_TC = 4
 } pisa_path;
 /* PISA_PATH_HYBRID_TC is another method, requested explicitly (AUTO never
  * picks it): the PISA paper's hybrid, where every H_j of the first-order term
@@ -96,6 +115,11 @@ typedef enum {
  *                              (row = value channel), element type = dtype
  *   cov   [BH, nblk, d, d]   : C_j = (1/B) sum_n (k-kbar)(k-kbar)^T, element
  *                              type = dtype; NULL unless order == 2.
+ *   kaug  [BH, nblk, 8, d] bf16 : the centroid split for the tensor cores:
+ *                              row 0 = bf16(kbar_j) (round to nearest), row 1 =
+ *                              bf16(kbar_j - row 0), rows 2-7 zero; NULL unless
+ *                              dtype == PISA_BF16 and order >= 1 (read by
+ *                              PISA_PATH_STATS_TC).
  * hstat is NULL when order == 0.  Fill with pisa_stats_bind. */
 typedef struct {
     int batch, heads, L, d, B, nblk, order;
@@ -104,6 +128,7 @@ typedef struct {
     float* vsum;
     void* hstat;
     void* cov;
+    void* kaug;
 } pisa_stats_t;
 
 /* Bytes of device memory pisa_stats_bind needs for these dimensions
@@ -177,8 +202,11 @@ pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pi
 /* The fused attention kernel alone, given a selection mask from pisa_select
  * (phases 1-2 of the PISA paper's section 3.4 plus the normalisation).
  *   path PISA_PATH_STATS needs `st` (pisa_stats output with st->order >= order);
+ *   path PISA_PATH_STATS_TC needs `st` with kbar, vsum, hstat and kaug (bf16,
+ *   st->order >= 1) and order 1;
  *   path PISA_PATH_RECOMPUTE_TC ignores `st` (may be NULL); AUTO picks as
- *   pisa_attention does.
+ *   pisa_attention does (the K it needs is taken from the mask's shape: AUTO
+ *   here never picks PISA_PATH_STATS_TC, pass it explicitly).
  * mask: [BH, nblk, ceil(nblk/32)] uint32 as written by pisa_select. */
 pisa_status pisa_fused_attention(const void* q, const void* k, const void* v, int batch, int heads, int L,
                                  int d, pisa_dtype dtype, int B, int order, int gate_w, pisa_path path,
@@ -234,6 +262,16 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make that
  *     first call before any stream capture.
+ *   - When the 32 MiB is committed: with CUDA's lazy module loading (the
+ *     default since CUDA 12.2) the library's module, and the array with it,
+ *     is loaded on a device at the library's first kernel launch or symbol
+ *     lookup there, which can be this entry point's first call.  A host that
+ *     hands its whole memory pool out later should make one call (or any other
+ *     call of this library) on each device first, or set CUDA_MODULE_LOADING=EAGER.
+ *   - The cached address belongs to the device's primary context: a
+ *     cudaDeviceReset (or another teardown of that context) after the first
+ *     call is not supported; the same holds for the device status word that
+ *     every entry point caches.
  *   - A call whose workspace (pisa_workspace_bytes) exceeds the scratch size is
  *     rejected with PISA_ERR_INVALID_ARG before any work is enqueued.
  *   - All calls on a device share the one array and it keeps the last call's
@@ -329,7 +367,17 @@ pisa_status pisa_poll_device_status(void* stream);
  * The context stays usable.  Errors: INVALID_ARG for a limit out of range. */
 pisa_status pisa_selftest_wait_timeout(long long limit_cycles, void* stream);
 
-/* Library version string. *//* Library version string. */
+/* Self-test of the base-2 exponentials of the attention kernels' softmax (no
+ * counterpart on the pages): y[i] = 2^x[i] for i < n, evaluated with
+ * which = 0: the FMA-pipe polynomial (x = n + f, n = round(x), a cubic in
+ *            f in [-1/2, 1/2] fitted for relative error <= 7.5e-5, n added to
+ *            the exponent; exactly 0 for x <= -125; valid up to x = 64), or
+ * which = 1: the special-function unit's ex2.approx.ftz.
+ * x, y: fp32 device arrays of n elements, 4-byte aligned.  Errors:
+ * INVALID_ARG for n < 0, which not 0 or 1, a null or misaligned pointer. */
+pisa_status pisa_selftest_ex2(const float* x, float* y, long long n, int which, void* stream);
+
+/* Library version string. */
 const char* pisa_version(void);
 
 #ifdef __cplusplus

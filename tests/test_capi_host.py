@@ -91,6 +91,36 @@ def test_workspace_sizes_and_paths():
         1, 1, 1024, 64, 64, 4, 1, f32, 1)
 
 
+def test_auto_takes_the_association_with_fewer_flops():
+    # d = B = 128 (Hunyuan shape) and d = B = 64 (clustered shape), order 1: the statistics form on
+    # the tensor cores executes fewer FLOPs than the token form's 4 L d per row; d = 2B (Wan and
+    # FLUX shapes) and any order-2 call with the exact w keep the token form
+    bf = pisa.PISA_BF16
+    lib = pisa.lib()
+    st = pisa.PATHS["stats_tc"]
+    assert lib.pisa_resolve_path(1, 24, 118784, 128, 128, 93, 1, bf) == st
+    assert lib.pisa_resolve_path(1, 12, 8192, 64, 64, 16, 1, bf) == st
+    assert lib.pisa_resolve_path(1, 12, 8192, 64, 64, 16, 2, bf) == pisa.PATHS["recompute_tc"]
+    assert lib.pisa_resolve_path(1, 40, 32768, 128, 64, 77, 1, bf) == pisa.PATHS["recompute_tc"]
+    assert lib.pisa_resolve_path(1, 24, 4608, 128, 64, 36, 1, bf) == pisa.PATHS["recompute_tc"]
+    # with every block selected there is no statistics term, and the token form costs the same: token
+    assert lib.pisa_resolve_path(1, 12, 8192, 64, 64, 128, 1, bf) == pisa.PATHS["recompute_tc"]
+    # the statistics-form workspace holds H_j and the centroid split (no C_j), order 0 has no such path
+    ws = lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 1, bf, st)
+    ws_tok = lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 1, bf, 2)
+    assert ws - ws_tok >= 12 * 128 * (64 * 64 + 8 * 64) * 2 + 12 * 128 * 64 * 4
+    assert lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 0, bf, st) == 0
+    assert lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 1, pisa.PISA_F32, st) == 0
+    assert lib.pisa_workspace_bytes_ex(1, 12, 8192, 64, 64, 16, 2, bf, st) > ws  # pooled w arrays
+
+
+def test_statistics_form_path_rejects_what_it_cannot_run():
+    # order 2 needs the pooled w; order 0 has no statistics term; fp32 has no tensor-core path
+    assert call_ex(path=4, order=2) == pisa.PISA_ERR_UNSUPPORTED
+    assert call_ex(path=4, order=0) == pisa.PISA_ERR_UNSUPPORTED
+    assert call_ex(path=4, dtype=pisa.PISA_F32) == pisa.PISA_ERR_UNSUPPORTED
+
+
 def test_stats_bind_layout():
     st = pisa._StatsT()
     lib = pisa.lib()
@@ -102,8 +132,16 @@ def test_stats_bind_layout():
     assert (st.vsum - base) % 256 == 0 and (st.hstat - base) % 256 == 0 and (st.cov - base) % 256 == 0
     assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n - 1, 2, 3, 1024, 64, 64, 2,
                                pisa.PISA_BF16) == pisa.PISA_ERR_INVALID_ARG
+    assert (st.kaug - base) % 256 == 0 and st.kaug >= st.cov + 6 * 16 * 64 * 64 * 2
     assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n, 2, 3, 1024, 64, 64, 1, pisa.PISA_BF16) == 0
-    assert st.cov is None
+    assert st.cov is None and st.kaug is not None
+    # the centroid split exists only for bf16 statistics of order >= 1
+    n0 = lib.pisa_stats_bytes(2, 3, 1024, 64, 64, 0, pisa.PISA_BF16)
+    assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), n0, 2, 3, 1024, 64, 64, 0, pisa.PISA_BF16) == 0
+    assert st.kaug is None
+    nf = lib.pisa_stats_bytes(2, 3, 1024, 64, 64, 1, pisa.PISA_F32)
+    assert lib.pisa_stats_bind(ctypes.byref(st), ctypes.c_void_p(base), nf, 2, 3, 1024, 64, 64, 1, pisa.PISA_F32) == 0
+    assert st.kaug is None
 
 
 def test_routing_and_score_entry_points_reject_bad_arguments():
@@ -116,7 +154,7 @@ def test_routing_and_score_entry_points_reject_bad_arguments():
     assert lib.pisa_route_bias(None, FAKE, FAKE, 1, 1, 1024, 64, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
     assert lib.pisa_route_bias(FAKE, FAKE, FAKE, 1, 1, 1000, 64, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
     assert lib.pisa_route_bias(FAKE, FAKE, FAKE, 1, 1, 1024, 96, bf, 64, 1e-6, FAKE, None) == pisa.PISA_ERR_UNSUPPORTED
-    st = pisa._StatsT(1, 1, 1024, 64, 64, 16, 0, bf, FAKE.value, None, None, None)
+    st = pisa._StatsT(1, 1, 1024, 64, 64, 16, 0, bf, FAKE.value, None, None, None, None)
     assert lib.pisa_select_scores(FAKE, ctypes.byref(st), None, None, None) == pisa.PISA_ERR_INVALID_ARG
     assert lib.pisa_select_scores(None, ctypes.byref(st), None, FAKE, None) == pisa.PISA_ERR_INVALID_ARG
     assert lib.pisa_select_biased(FAKE, ctypes.byref(st), 17, FAKE, FAKE, FAKE, None) == pisa.PISA_ERR_INVALID_ARG

@@ -5,9 +5,10 @@
 * selection: index lists and masks bit-exact, on small shapes, planted ties and
   every full-size workload;
 * attention: relative L2 error (||gpu - oracle||_F / ||oracle||_F) at most 1e-4
-  on the fp32 path and 2e-2 on the bf16 path, on small shapes end to end and on
-  sampled query tiles (first, last and seeded random ones) of the full-size
-  workloads, through both formulations.
+  on the fp32 path and 2e-2 on the bf16 path, and the same bound on every row
+  and (relative to the output's rms) on every element (tests/parity.py), on
+  small shapes end to end and on sampled query tiles (first, last and seeded
+  random ones) of the full-size workloads, through every formulation.
 """
 import functools
 import math
@@ -18,6 +19,7 @@ import torch
 
 import block_sparse_taylor_b200 as pisa
 import oracle
+import parity
 import pisa_synth
 
 pytestmark = pytest.mark.gpu
@@ -70,11 +72,12 @@ def test_stats_parity(dt, d, B, order):
     kbar_ref = oracle.centroids_f32(k, B)
     assert np.array_equal(st.kbar.cpu().numpy().view(np.uint32), kbar_ref.view(np.uint32))
     _, vsum, H, C = oracle.block_stats(k, v, B, order=2)
-    assert rel_l2(st.vsum.cpu().numpy(), vsum) < 1e-6
+    parity.check(st.vsum.cpu().numpy(), vsum, dt, "vsum", tol=1e-6, row_tol=1e-6, elem_tol=1e-6)
+    # H_j and C_j are stored in the input dtype: bf16 rounding of every entry
     tol = 1e-5 if dt == "f32" else 8e-3
-    assert rel_l2(st.hstat.float().cpu().numpy(), H) < tol
+    parity.check(st.hstat.float().cpu().numpy(), H, dt, "H", tol=tol, row_tol=2 * tol, elem_tol=2 * tol)
     if order == 2:
-        assert rel_l2(st.cov.float().cpu().numpy(), C) < tol
+        parity.check(st.cov.float().cpu().numpy(), C, dt, "C", tol=tol, row_tol=2 * tol, elem_tol=2 * tol)
     else:
         assert st.cov is None
 
@@ -173,9 +176,8 @@ def test_attention_small_bf16(path, d, B, order):
     K = (L // B) // 4
     got = run_attn(q, k, v, B, K, order, "bf16", path)
     ref = oracle.pisa_attention(q, k, v, B, K, order)
-    err = rel_l2(got, ref)
-    assert err <= TOL["bf16"], err
-    assert err <= 5e-3, err  # the expected bf16 rounding level; a formulation slip is far above it
+    m = parity.check(got, ref, "bf16")
+    assert m["rel_l2"] <= 5e-3, m  # the expected bf16 rounding level; a formulation slip is far above it
 
 
 @pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
@@ -186,14 +188,14 @@ def test_attention_small_f32(d, B, order):
     K = (L // B) // 4
     got = run_attn(q, k, v, B, K, order, "f32")
     ref = oracle.pisa_attention(q, k, v, B, K, order)
-    assert rel_l2(got, ref) <= TOL["f32"]
+    parity.check(got, ref, "f32")
 
 
 def test_attention_c1_fp32():
     w, (q, k, v) = workload("c1")
     got = run_attn(q, k, v, w.B, w.K, w.order, w.dtype)
     ref = oracle.pisa_attention(q, k, v, w.B, w.K, w.order)
-    assert rel_l2(got, ref) <= TOL["f32"]
+    parity.check(got, ref, "f32")
 
 
 @pytest.mark.parametrize("path", ["stats", "recompute_tc"])
@@ -222,9 +224,9 @@ def test_attention_edge_cases(path, case):
     got = pisa.pisa_attention(qt, kt, vt, B, K, order, path=path).float().cpu().numpy().reshape(BH, L, d)
     pisa.pisa_poll_device_status()
     ref = oracle.pisa_attention(q, k, v, B, K, order)
-    assert rel_l2(got, ref) <= TOL["bf16"]
+    parity.check(got, ref, "bf16", case)
     if case == "Kall":
-        assert rel_l2(got, oracle.dense_attention(q, k, v)) <= TOL["bf16"]
+        parity.check(got, oracle.dense_attention(q, k, v), "bf16", "dense")
 
 
 def test_gate_changes_the_result_when_w_is_large():
@@ -235,8 +237,8 @@ def test_gate_changes_the_result_when_w_is_large():
     for path in ("stats", "recompute_tc"):
         on = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=True)
         off = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=False)
-        assert rel_l2(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True)) <= TOL["bf16"]
-        assert rel_l2(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False)) <= TOL["bf16"]
+        parity.check(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True), "bf16", "gate on")
+        parity.check(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False), "bf16", "gate off")
         assert rel_l2(on, off) > 1e-2
 
 
@@ -246,8 +248,12 @@ def test_gate_changes_the_result_when_w_is_large():
 
 FULL = [("c2", "recompute_tc", 1, 6), ("c2o2", "recompute_tc", 1, 6), ("c2", "stats", 1, 6),
         ("c2o2", "stats", 1, 6), ("c3", "recompute_tc", 2, None), ("c4", "recompute_tc", 1, 8),
-        ("c5_L4608_s50", "recompute_tc", 2, None), ("c5_L4608_s95", "recompute_tc", 2, None),
-        ("c5_L16896_s75", "recompute_tc", 2, 8), ("c5_L16896_s90", "recompute_tc", 2, 8)]
+        ("c5_L4608_s50", "recompute_tc", 2, None), ("c5_L4608_s75", "recompute_tc", 2, None),
+        ("c5_L4608_s90", "recompute_tc", 2, None), ("c5_L4608_s95", "recompute_tc", 2, None),
+        ("c5_L16896_s50", "recompute_tc", 2, 8), ("c5_L16896_s75", "recompute_tc", 2, 8),
+        ("c5_L16896_s90", "recompute_tc", 2, 8), ("c5_L16896_s95", "recompute_tc", 2, 8),
+        ("c2", "stats_tc", 1, 6), ("c4", "stats_tc", 1, 8), ("c3", "stats_tc", 1, 8),
+        ("c5_L16896_s90", "stats_tc", 2, 8), ("c5_L4608_s50", "stats_tc", 2, None)]
 
 
 @pytest.mark.parametrize("name,path,per_head,nheads", FULL)
@@ -257,8 +263,7 @@ def test_attention_full_size_sampled(name, path, per_head, nheads):
     heads = None if nheads is None else list(np.random.default_rng(7).choice(w.BH, nheads, replace=False))
     tiles = sample_tiles(w.BH, w.nblk, per_head, seed=11, heads=heads)
     ref = oracle.pisa_attention(q, k, v, w.B, w.K, w.order, tiles=tiles)
-    err = rel_l2(rows_of(got, tiles, w.B), ref)
-    assert err <= TOL[w.dtype], (name, err)
+    parity.check(rows_of(got, tiles, w.B), ref, w.dtype, name)
 
 
 def test_device_status_is_clean():
@@ -281,9 +286,8 @@ def test_hybrid_small(d, B, order, Kfrac):
     q, k, v = pisa_synth.random_qkv(800 + d + B + order, 2, L, d, scale=2.0, dtype="bf16")
     got = run_attn(q, k, v, B, K, order, "bf16", "hybrid_tc")
     ref = oracle.pisa_hybrid(q, k, v, B, K, order)
-    err = rel_l2(got, ref)
-    assert err <= TOL["bf16"], err
-    assert err <= 5e-3, err
+    m = parity.check(got, ref, "bf16")
+    assert m["rel_l2"] <= 5e-3, m
 
 
 @pytest.mark.parametrize("case", ["ragged", "clustered", "sharp"])
@@ -298,18 +302,18 @@ def test_hybrid_edge_cases(case):
         q, k, v = pisa_synth.random_qkv(850 + len(case), 2, L, d, scale=scale, dtype="bf16")
     got = run_attn(q, k, v, B, K, 1, "bf16", "hybrid_tc")
     ref = oracle.pisa_hybrid(q, k, v, B, K, 1)
-    assert rel_l2(got, ref) <= TOL["bf16"]
+    parity.check(got, ref, "bf16", case)
 
 
-@pytest.mark.parametrize("name,per_head,nheads", [("c3", 2, 8), ("c5_L16896_s90", 2, 8), ("c4", 1, 4)])
+@pytest.mark.parametrize("name,per_head,nheads", [("c3", 2, 8), ("c5_L16896_s90", 2, 8), ("c4", 1, 4),
+                                                   ("c5_L4608_s50", 2, 8), ("c5_L4608_s90", 2, 8)])
 def test_hybrid_full_size_sampled(name, per_head, nheads):
     w, (q, k, v) = workload(name)
     got = run_attn(q, k, v, w.B, w.K, 1, w.dtype, "hybrid_tc")
     heads = list(np.random.default_rng(9).choice(w.BH, nheads, replace=False))
     tiles = sample_tiles(w.BH, w.nblk, per_head, seed=13, heads=heads)
     ref = oracle.pisa_hybrid(q, k, v, w.B, w.K, 1, tiles=tiles)
-    err = rel_l2(rows_of(got, tiles, w.B), ref)
-    assert err <= TOL[w.dtype], (name, err)
+    parity.check(rows_of(got, tiles, w.B), ref, w.dtype, name)
 
 
 # ---------------------------------------------------------------------------
@@ -322,7 +326,7 @@ def run_attn_w(q, k, v, B, K, order, dt, path, w_mode, gate=True):
     return out.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("path", ["recompute_tc", "stats", "hybrid_tc"])
+@pytest.mark.parametrize("path", ["recompute_tc", "stats", "hybrid_tc", "stats_tc"])
 @pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (128, 128)])
 @pytest.mark.parametrize("gate", [True, False])
 def test_pooled_w_small(path, d, B, gate):
@@ -331,16 +335,15 @@ def test_pooled_w_small(path, d, B, gate):
     q, k, v = pisa_synth.random_qkv(900 + d + B, 2, L, d, scale=2.0, dtype="bf16")
     got = run_attn_w(q, k, v, B, K, 2, "bf16", path, "pooled", gate)
     ref = oracle.pisa_attention_ex(q, k, v, B, K, 2, gate=gate, hybrid=(path == "hybrid_tc"), w_pooled=True)
-    err = rel_l2(got, ref)
-    assert err <= TOL["bf16"], err
-    assert err <= 5e-3, err
+    m = parity.check(got, ref, "bf16")
+    assert m["rel_l2"] <= 5e-3, m
 
 
 def test_pooled_w_fp32_statistics_path():
     q, k, v = pisa_synth.random_qkv(950, 2, 1024, 64, scale=2.0, dtype="f32")
     got = run_attn_w(q, k, v, 64, 4, 2, "f32", "stats", "pooled")
     ref = oracle.pisa_attention_ex(q, k, v, 64, 4, 2, w_pooled=True)
-    assert rel_l2(got, ref) <= TOL["f32"]
+    parity.check(got, ref, "f32")
 
 
 def test_hybrid_order2_needs_pooled_w():
@@ -355,7 +358,7 @@ def test_pooled_w_full_size_c2(path):
     got = run_attn_w(q, k, v, w.B, w.K, 2, w.dtype, path, "pooled")
     tiles = sample_tiles(w.BH, w.nblk, 4, seed=17, heads=[0, 5, 11])
     ref = oracle.pisa_attention_ex(q, k, v, w.B, w.K, 2, hybrid=(path == "hybrid_tc"), w_pooled=True, tiles=tiles)
-    assert rel_l2(rows_of(got, tiles, w.B), ref) <= TOL[w.dtype]
+    parity.check(rows_of(got, tiles, w.B), ref, w.dtype, path)
 
 
 def test_host_entry_point_with_routing_matches_device_call():
@@ -408,4 +411,118 @@ def test_maximum_block_count(path):
     got = run_attn(q, k, v, B, K, 1, "bf16", path)
     tiles = sample_tiles(1, L // B, 8, seed=13)
     ref = oracle.pisa_attention_ex(q, k, v, B, K, 1, hybrid=(path == "hybrid_tc"), tiles=tiles)
-    assert rel_l2(rows_of(got, tiles, B), ref) <= TOL["bf16"]
+    parity.check(rows_of(got, tiles, B), ref, "bf16", path)
+
+
+# ---------------------------------------------------------------------------
+# numerics of the token form: the FMA-pipe exponential and w at a large offset
+# ---------------------------------------------------------------------------
+
+def test_ex2_fma_against_exact_powers_of_two():
+    # the FMA-pipe 2^x the softmax uses for part of its exponentials: relative error within
+    # the fitted 7.5e-5 (plus fp32 rounding) on [-125, 64], exactly 0 at and below -125
+    xs = np.concatenate([np.linspace(-124.999, 63.999, 1 << 20), np.arange(-124, 64, 0.5),
+                         [-125.0, -125.5, -200.0, -np.inf]]).astype(np.float32)
+    y = pisa.pisa_selftest_ex2(torch.from_numpy(xs).cuda(), "fma").cpu().numpy()
+    live = xs > -125.0
+    exact = np.exp2(xs[live].astype(np.float64))
+    rel = np.abs(y[live] - exact) / exact
+    assert rel.max() <= 7.5e-5 + 2.0 ** -23, float(rel.max())
+    assert np.all(y[~live] == 0.0)
+    # the special-function unit's ex2.approx, for comparison: a few ulp on the same range
+    z = pisa.pisa_selftest_ex2(torch.from_numpy(xs[live]).cuda(), "sfu").cpu().numpy()
+    assert (np.abs(z - exact) / exact).max() <= 2.0 ** -20
+
+
+@pytest.mark.parametrize("path", ["recompute_tc", "stats"])
+def test_order2_with_a_large_common_logit_offset(path):
+    # Every logit is about 300 (a shared channel) with a spread of about 1 inside each block, so
+    # that w = (1/2B) sum_n (x_n - s-bar)^2 is O(1) while E[x^2] is about 9e4: a one-pass
+    # variance in fp32 would lose w to cancellation.  The gate stays open (w < ln B).
+    rng = np.random.default_rng(2024)
+    BH, L, d, B, K = 2, 1024, 64, 64, 4
+    q = np.empty((BH, L, d), np.float32)
+    k = np.empty((BH, L, d), np.float32)
+    q[..., 0] = 17.0
+    k[..., 0] = 17.625  # 17 * 17.625 = 299.625, exact in bf16 products
+    q[..., 1:] = 0.35 * rng.standard_normal((BH, L, d - 1))
+    k[..., 1:] = 0.35 * rng.standard_normal((BH, L, d - 1))
+    v = rng.standard_normal((BH, L, d)).astype(np.float32)
+    q, k, v = (pisa_synth.round_bf16(x) for x in (q, k, v))
+    got = run_attn(q, k, v, B, K, 2, "bf16", path)
+    ref = oracle.pisa_attention(q, k, v, B, K, 2)
+    parity.check(got, ref, "bf16", path)
+    # w matters here: the result differs from order 1 by far more than the tolerance
+    assert rel_l2(ref, oracle.pisa_attention(q, k, v, B, K, 1)) > 5e-2
+
+
+# ---------------------------------------------------------------------------
+# the statistics form on the tensor cores (PISA_PATH_STATS_TC): blocks selected
+# by any tile of a 256-row CTA in the token form, every other block through the
+# H_j contraction
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("Kfrac", [0.0, 0.1, 0.25, 0.5, 1.0])
+def test_stats_tc_small(d, B, Kfrac):
+    # K = 0: only the H_j contraction; K = all: only the union tiles; in between, both phases
+    # with random selections (unions of different sizes, an odd number of contraction blocks
+    # for d = 64, which pairs them)
+    L = 2048
+    nblk = L // B
+    K = int(round(Kfrac * nblk))
+    q, k, v = pisa_synth.random_qkv(1000 + d + B, 2, L, d, scale=2.0, dtype="bf16")
+    got = run_attn(q, k, v, B, K, 1, "bf16", "stats_tc")
+    ref = oracle.pisa_attention(q, k, v, B, K, 1)
+    m = parity.check(got, ref, "bf16")
+    assert m["rel_l2"] <= 5e-3, m
+
+
+@pytest.mark.parametrize("case", ["ragged", "batched", "sharp", "clustered", "single_block", "max_raise"])
+def test_stats_tc_edge_cases(case):
+    d, B, L, BH, K, scale = 128, 128, 1024, 2, 2, 2.0
+    batch = 1
+    if case == "ragged":
+        L = 1152  # 4.5 CTAs of 256 rows
+        B = 64
+    elif case == "batched":
+        batch, BH = 2, 6
+    elif case == "sharp":
+        scale = 8.0  # large logits: the running max is raised in both phases
+    elif case == "single_block":
+        L, B, K = 128, 128, 0  # one block, one CTA with one live M tile
+    if case == "clustered":
+        w = pisa_synth.workloads()["c2"].with_(heads=2, L=4096)
+        q, k, v = pisa_synth.generate(w)
+        d, B, K = w.d, w.B, w.K
+    else:
+        q, k, v = pisa_synth.random_qkv(1100 + len(case), BH, L, d, scale=scale, dtype="bf16")
+    if case == "max_raise":
+        # the largest logits sit in the last blocks, which only the contraction phase reaches
+        q[..., 0] = 2.0
+        k[:, -2 * B:, 0] += 6.0
+        q, k = pisa_synth.round_bf16(q), pisa_synth.round_bf16(k)
+        K = 0
+    qt, kt, vt = (dev(x, "bf16") for x in (q, k, v))
+    if batch > 1:
+        qt, kt, vt = (x.view(batch, BH // batch, L, d) for x in (qt, kt, vt))
+    got = pisa.pisa_attention(qt, kt, vt, B, K, 1, path="stats_tc").float().cpu().numpy().reshape(q.shape)
+    pisa.pisa_poll_device_status()
+    parity.check(got, oracle.pisa_attention(q, k, v, B, K, 1), "bf16", case)
+
+
+def test_stats_tc_agrees_with_the_token_form():
+    # the two tensor-core associations of the same first-order term, on the same inputs
+    q, k, v = pisa_synth.random_qkv(1200, 3, 4096, 64, scale=2.0, dtype="bf16")
+    a = run_attn(q, k, v, 64, 12, 1, "bf16", "stats_tc")
+    b = run_attn(q, k, v, 64, 12, 1, "bf16", "recompute_tc")
+    parity.check(a, b, "bf16", "stats_tc vs recompute_tc")
+
+
+def test_auto_runs_the_statistics_form_at_the_hunyuan_and_clustered_shapes():
+    assert pisa.pisa_resolve_path(1, 24, 118784, 128, 128, 93, 1, torch.bfloat16) == "stats_tc"
+    assert pisa.pisa_resolve_path(1, 12, 8192, 64, 64, 16, 1, torch.bfloat16) == "stats_tc"
+    w = pisa_synth.workloads()["c2"].with_(heads=3)
+    q, k, v = pisa_synth.generate(w)
+    auto = run_attn(q, k, v, w.B, w.K, 1, w.dtype, "auto")
+    assert np.array_equal(auto, run_attn(q, k, v, w.B, w.K, 1, w.dtype, "stats_tc"))
