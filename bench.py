@@ -353,19 +353,36 @@ def stc_executed_flops(w, mask) -> float:
     256 rows, its union U of the selected blocks of its query tiles runs in 128-key tiles
     (S and PV: 4 d 128 per row and tile), every other block in items of g blocks (one MMA
     with N = g d + 16 per row: 2 d (g d + 16)), g = 2 for d = 64 and 1 for d = 128."""
+    nu = cta_unions(w, mask)
+    bpt, gb = 128 // w.B, (2 if w.d == 64 else 1)
+    nut = (nu + bpt - 1) // bpt
+    ni = (w.nblk - nu + gb - 1) // gb
+    per_row = 4.0 * w.d * 128 * nut + 2.0 * w.d * (gb * w.d + 16) * ni
+    return float(256.0 * per_row.sum())
+
+
+def cta_unions(w, mask):
+    """Per (bh, 256-row CTA): the number of blocks selected by any of its query tiles."""
     m = mask.cpu().numpy().view(np.uint32)  # [BH, nblk, words]
     BH, nblk, words = m.shape
-    nqt, bpt, gb = 256 // w.B, 128 // w.B, (2 if w.d == 64 else 1)
+    nqt = 256 // w.B
     ncta = (w.L + 255) // 256
     pad = ncta * nqt - nblk
     if pad > 0:
-        # rows past L repeat the last tile's selection (the kernel clamps the tile index)
+        # rows past L repeat the last tile's selection (the kernels clamp the tile index)
         m = np.concatenate([m, np.repeat(m[:, -1:], pad, axis=1)], axis=1)
     u = np.bitwise_or.reduce(m.reshape(BH, ncta, nqt, words), axis=2)
-    nu = np.unpackbits(u.view(np.uint8), axis=-1).reshape(BH, ncta, -1).sum(axis=-1).astype(np.int64)
-    nut = (nu + bpt - 1) // bpt
-    ni = (nblk - nu + gb - 1) // gb
-    per_row = 4.0 * w.d * 128 * nut + 2.0 * w.d * (gb * w.d + 16) * ni
+    return np.unpackbits(u.view(np.uint8), axis=-1).reshape(BH, ncta, -1).sum(axis=-1).astype(np.int64)
+
+
+def hybrid_executed_flops(w, mask) -> float:
+    """FLOPs the hybrid kernel executes for this selection: per 256-row CTA, its union tiles
+    and the ceil(nblk/128) virtual tiles (S and PV: 4 d 128 per row and tile), plus the
+    epilogue's G = Q H-bar^T (2 d^2 per row, order >= 1)."""
+    nu = cta_unions(w, mask)
+    bpt = 128 // w.B
+    tiles = (nu + bpt - 1) // bpt + (w.nblk + 127) // 128
+    per_row = 4.0 * w.d * 128 * tiles + (2.0 * w.d * w.d if w.order >= 1 else 0.0)
     return float(256.0 * per_row.sum())
 
 
@@ -673,10 +690,20 @@ def main():
         torch.cuda.synchronize()
         pisa.pisa_poll_device_status()
         h_ms = ha.elapsed_time(hb) / reps
+        h_exec = hybrid_executed_flops(w, mask)
+        bf16_peak = float(peaks["bf16_tflops"])
         hybrid_rec = {"method": "PISA hybrid: exact selected blocks, zeroth-order virtual tokens, global H-bar "
                                 "first-order term (not the per-block H_j formulation of the main line)",
                       "ms_per_call": h_ms, "full_attn_equiv_tflops": dense_flops / (h_ms * 1e-3) / 1e12,
-                      "speedup_vs_per_block_path": ms_step / h_ms, "launches_per_call": 5}
+                      "speedup_vs_per_block_path": ms_step / h_ms, "launches_per_call": 5,
+                      "roofline": {"bound": "tensor", "kernel": f"attn_hybrid_kernel<{d},{B},{order}>",
+                                   "executed_flops_per_call": h_exec,
+                                   "achieved": h_exec / (h_ms * 1e-3) / 1e12, "peak": bf16_peak,
+                                   "unit": "TFLOP/s", "frac": h_exec / (h_ms * 1e-3) / 1e12 / bf16_peak,
+                                   "note": "executed FLOPs of the attention kernel (union tiles, virtual tiles, "
+                                           "Q H-bar^T) over the whole call's time (prepare, select, attention): a "
+                                           "lower bound on the attention kernel's own fraction",
+                                   "peak_source": f"{peak_kind} bf16 dense (burst)"}}
         del hws, hout
 
     # The backward pass (training use) on the same inputs: dq, dk, dv of

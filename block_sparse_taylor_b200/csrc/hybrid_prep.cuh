@@ -15,8 +15,10 @@
 //     straight from the token tiles; d = 64 stacks [V ; K] to M = 128);
 //   - vsum_j kbar_j^T accumulated over the chunk in fp32 registers (thread a
 //     holds row a).
-// At the end each thread adds (B/L) (TMEM row - register row) into the fp32
-// H-bar accumulator of its (batch, head) with atomics (the caller zeroes it).
+// At the end each thread writes (B/L) (TMEM row - register row), the chunk's
+// share of H-bar, to the chunk's own fp32 slot; hbar_reduce_kernel then sums
+// the slots of each (batch, head) in chunk order and rounds to bf16, so H-bar
+// (and the hybrid's output) is the same on every run.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -43,7 +45,7 @@ struct HybPrepCfg {
 template <int D, int BS>
 __global__ void __launch_bounds__(128, 1) hybrid_prep_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, float* __restrict__ kbar,
-    bf16* __restrict__ kbar_bf, bf16* __restrict__ vsum_bf, float* __restrict__ hbar_acc, int L, int nblk, int G,
+    bf16* __restrict__ kbar_bf, bf16* __restrict__ vsum_bf, float* __restrict__ hbar_part, int L, int nblk, int G,
     float scale, unsigned* status) {
     using C = HybPrepCfg<D, BS>;
     constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
@@ -140,11 +142,11 @@ __global__ void __launch_bounds__(128, 1) hybrid_prep_kernel(
         __syncthreads();
     }
 
-    // every MMA has completed (thread 0 waited for each); add (B/L)(V^T K - R)
+    // every MMA has completed (thread 0 waited for each); this chunk's (B/L)(V^T K - R)
     tc::fence_after_sync();
     if (!aborted) {
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-        float* dst = hbar_acc + ((size_t)bh * D + (tid < D ? tid : 0)) * D;
+        float* dst = hbar_part + (((size_t)bh * gridDim.x + blockIdx.x) * D + (tid < D ? tid : 0)) * D;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t raw[32];
@@ -152,7 +154,12 @@ __global__ void __launch_bounds__(128, 1) hybrid_prep_kernel(
             tc::tmem_wait_ld();
             if (tid < D) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) atomicAdd(dst + c0 + e, scale * (__uint_as_float(raw[e]) - R[c0 + e]));
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + c0 + e) =
+                        make_float4(scale * (__uint_as_float(raw[e]) - R[c0 + e]),
+                                    scale * (__uint_as_float(raw[e + 1]) - R[c0 + e + 1]),
+                                    scale * (__uint_as_float(raw[e + 2]) - R[c0 + e + 2]),
+                                    scale * (__uint_as_float(raw[e + 3]) - R[c0 + e + 3]));
             }
         }
     }
@@ -165,16 +172,36 @@ __global__ void __launch_bounds__(128, 1) hybrid_prep_kernel(
     }
 }
 
-// H-bar fp32 accumulator -> bf16 (row = value channel, the K-major B operand of Q H-bar^T).
-__global__ void hbar_to_bf16_kernel(const float* __restrict__ acc, bf16* __restrict__ out, long n) {
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
-        out[i] = __float2bfloat16_rn(acc[i]);
+// H-bar = sum of the chunks' slots in chunk order (fixed, so reproducible), rounded to bf16
+// (row = value channel, the K-major B operand of Q H-bar^T).  part: [BH, nchunk, d*d].
+__global__ void hbar_reduce_kernel(const float* __restrict__ part, bf16* __restrict__ out, long BH, int nchunk,
+                                   int dd) {
+    const long n = BH * (long)dd;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+        const long bh = i / dd, e = i % dd;
+        const float* p = part + (size_t)bh * nchunk * dd + e;
+        float acc = 0.f;
+        for (int c = 0; c < nchunk; ++c) acc += p[(size_t)c * dd];
+        out[i] = __float2bfloat16_rn(acc);
+    }
 }
 
-// Host: tensor maps, the prepare kernel and the bf16 conversion of H-bar.
-// hacc must be zero on entry.
+// Blocks per CTA of the prepare kernel: 64, halved (down to 8) until the grid has
+// about four CTAs per SM.  The number of chunks (CTAs per head) sizes H-bar's slots.
+inline int hybrid_prep_chunk(long BH, int nblk) {
+    int G = 64;
+    while (G > 8 && (long)((nblk + G - 1) / G) * BH < 4L * 148) G /= 2;
+    return G;
+}
+inline int hybrid_prep_nchunk(long BH, int nblk) {
+    const int G = hybrid_prep_chunk(BH, nblk);
+    return (nblk + G - 1) / G;
+}
+
+// Host: tensor maps, the prepare kernel and the ordered reduction of H-bar.
+// hpart: [BH, hybrid_prep_nchunk(BH, nblk), d, d] fp32 (every slot is written).
 inline pisa_status run_hybrid_prep(const void* k, const void* v, float* kbar, bf16* kbar_bf, bf16* vsum_bf,
-                                   float* hacc, bf16* hbf, long BH, int L, int d, int B, int nblk, unsigned* status,
+                                   float* hpart, bf16* hbf, long BH, int L, int d, int B, int nblk, unsigned* status,
                                    cudaStream_t s, std::string* err) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -200,10 +227,9 @@ inline pisa_status run_hybrid_prep(const void* k, const void* v, float* kbar, bf
             return PISA_ERR_CUDA;
         }
     }
-    // blocks per CTA: 64, halved (down to 8) until the grid has about four CTAs per SM
-    int G = 64;
-    while (G > 8 && (long)((nblk + G - 1) / G) * BH < 4L * 148) G /= 2;
-    dim3 grid((unsigned)((nblk + G - 1) / G), (unsigned)BH);
+    const int G = hybrid_prep_chunk(BH, nblk);
+    const int nchunk = (nblk + G - 1) / G;
+    dim3 grid((unsigned)nchunk, (unsigned)BH);
     const float scale = (float)B / (float)L;
     cudaError_t e = cudaSuccess;
 #define PISA_HPREP(DD, BB)                                                                                     \
@@ -211,7 +237,7 @@ inline pisa_status run_hybrid_prep(const void* k, const void* v, float* kbar, bf
         auto kern = hybrid_prep_kernel<DD, BB>;                                                                \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HybPrepCfg<DD, BB>::SMEM); \
         if (e == cudaSuccess) {                                                                                \
-            kern<<<grid, 128, HybPrepCfg<DD, BB>::SMEM, s>>>(maps[0], maps[1], kbar, kbar_bf, vsum_bf, hacc, L, nblk, \
+            kern<<<grid, 128, HybPrepCfg<DD, BB>::SMEM, s>>>(maps[0], maps[1], kbar, kbar_bf, vsum_bf, hpart, L, nblk, \
                                                              G, scale, status);                                \
             e = cudaGetLastError();                                                                            \
         }                                                                                                      \
@@ -229,10 +255,11 @@ inline pisa_status run_hybrid_prep(const void* k, const void* v, float* kbar, bf
         return PISA_ERR_CUDA;
     }
     const long n = BH * (long)d * d;
-    hbar_to_bf16_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, s>>>(hacc, hbf, n);
+    hbar_reduce_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, s>>>(hpart, hbf, BH,
+                                                                                                 nchunk, d * d);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
-        *err = std::string("hbar_to_bf16_kernel launch: ") + cudaGetErrorString(e);
+        *err = std::string("hbar_reduce_kernel launch: ") + cudaGetErrorString(e);
         return PISA_ERR_CUDA;
     }
     return PISA_OK;

@@ -318,8 +318,8 @@ WsLayout ws_layout(const Dims& g, int K, int order, pisa_dtype dtype, pisa_path 
         o += align_up(2 * g.BH * g.nblk * g.d);
         w.vsum_bf = o;
         o += align_up(2 * g.BH * g.nblk * g.d);
-        w.hbar_acc = o;
-        o += align_up(4 * g.BH * g.d * g.d);
+        w.hbar_acc = o;  // H-bar's per-chunk slots, reduced in a fixed order
+        o += align_up(4 * g.BH * (size_t)pisa::hybrid_prep_nchunk(g.BH, (int)g.nblk) * g.d * g.d);
         w.hbar_bf = o;
         o += align_up(2 * g.BH * g.d * g.d);
     }
@@ -643,8 +643,6 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         bf16* vsum_bf = (bf16*)(ws + w.vsum_bf);
         float* hacc = (float*)(ws + w.hbar_acc);
         bf16* hbf = (bf16*)(ws + w.hbar_bf);
-        cudaError_t e = cudaMemsetAsync(hacc, 0, sizeof(float) * g.BH * g.d * g.d, s);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(H-bar)");
         r = pisa::run_hybrid_prep(k, v, st.kbar, kbar_bf, vsum_bf, hacc, hbf, g.BH, (int)g.L, (int)g.d, (int)g.B,
                                   (int)g.nblk, status, s, &g_last_error);
         if (r != PISA_OK) return r;

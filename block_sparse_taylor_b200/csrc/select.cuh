@@ -26,67 +26,78 @@ __device__ __forceinline__ uint32_t ordered_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Canonical score: p_c = q_c * k_c rounded, then the pairwise tree
-// a[i] = a[i] + a[i + h], h = D/2 .. 1, every product and sum one IEEE fp32
-// round-to-nearest operation (__fmul_rn / __fadd_rn, which are never fused into
-// an FMA).  The first level is formed directly from the products of columns i
-// and i + D/2.  (Packed fp32x2 multiplies and adds do not reproduce separately
-// rounded scalar operations, so they are not used here.)
+// Canonical score split over four lanes (one residue class mod 4 each).  The
+// canonical tree (a[i] = a[i] + a[i + h], first level i < D/2 pairing the
+// products of columns i and i + D/2, then h = D/4 .. 1) only ever adds two
+// entries of the same residue mod 4 while h >= 4, so lane r (the entries
+// i = r + 4m) runs those levels alone on its D/8 values; the last two levels
+// (h = 2: a[0] + a[2], a[1] + a[3]; h = 1: a[0] + a[1]) are two shuffles.  Every
+// product and sum is one IEEE fp32 round-to-nearest operation (__fmul_rn /
+// __fadd_rn, never fused), so the score is the same bit for bit as the serial
+// canonical order.  q holds q[r + 4m] (m < D/8) then q[D/2 + r + 4m]; k is the
+// block's segment for residue r in the same order.  The result is valid in
+// lane r = 0 of the group.  (Packed fp32x2 multiplies and adds do not
+// reproduce separately rounded scalar operations, so they are not used.)
 template <int D>
-__device__ __forceinline__ float canonical_dot(const float (&q)[D], const float* __restrict__ k) {
-    float a[D / 2];
+__device__ __forceinline__ float canonical_dot4(const float (&q)[D / 4], const float* __restrict__ k, int r) {
+    constexpr int H = D / 8;
+    float a[H];
     const float4* k4 = reinterpret_cast<const float4*>(k);
 #pragma unroll
-    for (int m = 0; m < D / 8; ++m) {
-        const float4 lo = k4[m], hi = k4[D / 8 + m];
-        a[4 * m + 0] = __fadd_rn(__fmul_rn(q[4 * m + 0], lo.x), __fmul_rn(q[D / 2 + 4 * m + 0], hi.x));
-        a[4 * m + 1] = __fadd_rn(__fmul_rn(q[4 * m + 1], lo.y), __fmul_rn(q[D / 2 + 4 * m + 1], hi.y));
-        a[4 * m + 2] = __fadd_rn(__fmul_rn(q[4 * m + 2], lo.z), __fmul_rn(q[D / 2 + 4 * m + 2], hi.z));
-        a[4 * m + 3] = __fadd_rn(__fmul_rn(q[4 * m + 3], lo.w), __fmul_rn(q[D / 2 + 4 * m + 3], hi.w));
+    for (int m = 0; m < H / 4; ++m) {
+        const float4 lo = k4[m], hi = k4[H / 4 + m];
+        a[4 * m + 0] = __fadd_rn(__fmul_rn(q[4 * m + 0], lo.x), __fmul_rn(q[H + 4 * m + 0], hi.x));
+        a[4 * m + 1] = __fadd_rn(__fmul_rn(q[4 * m + 1], lo.y), __fmul_rn(q[H + 4 * m + 1], hi.y));
+        a[4 * m + 2] = __fadd_rn(__fmul_rn(q[4 * m + 2], lo.z), __fmul_rn(q[H + 4 * m + 2], hi.z));
+        a[4 * m + 3] = __fadd_rn(__fmul_rn(q[4 * m + 3], lo.w), __fmul_rn(q[H + 4 * m + 3], hi.w));
     }
-    return tree_sum<D / 2>(a);
+    float v = tree_sum<H>(a);  // global levels h = D/4 .. 4: lane r now holds a[r]
+    v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, 2));  // h = 2 (lanes r = 0, 1)
+    v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, 1));  // h = 1 (lane r = 0)
+    (void)r;
+    return v;
 }
 
 template <int D>
 struct SelectCfg {
     static constexpr int THREADS = 256;
-    static constexpr int JC = 64;  // centroids staged per chunk
+    static constexpr int JC = 32;          // centroids staged per chunk
+    static constexpr int SEG = D / 4 + 4;  // floats per residue segment of a staged centroid (padded)
 };
 
-// Query tiles per CTA (one per lane of a warp, at most 32) so that the score
-// table fits next to the staged tile means and centroids.
-template <int D>
-inline int select_tiles_per_cta(int nblk) {
-    const long budget = 200 * 1024 - (long)sizeof(float) * (32 * D + SelectCfg<D>::JC * D);
-    long qt = budget / ((long)sizeof(float) * (nblk + 1));
-    return (int)(qt > 32 ? 32 : (qt < 1 ? 1 : qt));
-}
-
+// Query tiles per CTA: 16 (two groups of 8 tiles, four lanes a tile) when the score
+// table leaves room for three CTAs per SM, else 8.
 template <int D>
 inline size_t select_smem_bytes(int QT, int nblk) {
-    return sizeof(float) * ((size_t)QT * D + (size_t)SelectCfg<D>::JC * D + (size_t)QT * (nblk + 1));
+    return sizeof(float) * ((size_t)QT * D + (size_t)SelectCfg<D>::JC * 4 * SelectCfg<D>::SEG +
+                            (size_t)QT * (nblk + 1));
+}
+template <int D>
+inline int select_tiles_per_cta(int nblk) {
+    return select_smem_bytes<D>(16, nblk) <= 72 * 1024 ? 16 : 8;
 }
 
 // One CTA per (group of QT query tiles, bh), 8 warps.
 //   1. canonical tile means (thread per (tile, column));
-//   2. scores: lane t of every warp holds tile t's mean in registers, the
-//      centroids are staged JC at a time and read as broadcasts; warp w takes
-//      the blocks jj = w, w+8, ... of each chunk;
-//      with a routing bias ([BH, nblk], or null) each score gets bias_j added;
+//   2. scores: lane 4 tl + r of a warp works on tile tl of the warp's tile group
+//      and residue r of the canonical tree; the centroids are staged JC at a
+//      time, each split into its four residue segments; the warps of a tile
+//      group split the blocks of a chunk between them; with a routing bias
+//      ([BH, nblk], or null) each score gets bias_j added;
 //   3. top-K per tile (warp per tile): binary search for the K-th largest
 //      ordered score, then ties broken by ascending block index with ballots;
 //      the ballots are the mask words and give the ascending index list.
 template <typename T, int D, int BS>
-__global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+__global__ void __launch_bounds__(256, 2) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                                                         int L, int nblk, int K, int words, int QT,
                                                         int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
                                                         const float* __restrict__ bias,
                                                         float* __restrict__ scores_out) {
     using C = SelectCfg<D>;
     extern __shared__ __align__(16) float sm_sel[];
-    float* qbar = sm_sel;                 // [QT][D]
-    float* kst = qbar + QT * D;           // [JC][D]
-    float* sc = kst + C::JC * D;          // [QT][nblk + 1]
+    float* qbar = sm_sel;                    // [QT][D]
+    float* kst = qbar + QT * D;              // [JC][4][SEG]: residue segments of the staged centroids
+    float* sc = kst + C::JC * 4 * C::SEG;    // [QT][nblk + 1]
     const int SS = nblk + 1;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, bh = blockIdx.y;
     const int i0 = blockIdx.x * QT;
@@ -119,30 +130,43 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
     __syncthreads();
 
     // 2. scores
-    const bool live = lane < nq;
-    float qr[D];
+    const int ngroups = QT / 8;            // tile groups of 8 tiles
+    const int grp = warp % ngroups;        // this warp's tile group
+    const int wsplit = 8 / ngroups;        // warps sharing a tile group (they split the blocks)
+    const int wpart = warp / ngroups;
+    const int tl = lane >> 2, r = lane & 3;
+    const int t = grp * 8 + tl;            // tile of this lane inside the CTA
+    const bool live = t < nq;
+    float qr[D / 4];  // q[r + 4m], then q[D/2 + r + 4m]
     {
-        const float4* qs = reinterpret_cast<const float4*>(qbar + (live ? lane : 0) * D);
+        const float* qt_ = qbar + (live ? t : 0) * D;
 #pragma unroll
-        for (int m = 0; m < D / 4; ++m) {
-            const float4 t = qs[m];
-            qr[4 * m] = t.x;
-            qr[4 * m + 1] = t.y;
-            qr[4 * m + 2] = t.z;
-            qr[4 * m + 3] = t.w;
+        for (int m = 0; m < D / 8; ++m) {
+            qr[m] = qt_[r + 4 * m];
+            qr[D / 8 + m] = qt_[D / 2 + r + 4 * m];
         }
     }
     const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nblk * D);
     for (int j0 = 0; j0 < nblk; j0 += C::JC) {
         const int nj = min(C::JC, nblk - j0);
-        float4* kst4 = reinterpret_cast<float4*>(kst);
-        for (int e = tid; e < nj * D / 4; e += C::THREADS) kst4[e] = kb4[(size_t)j0 * D / 4 + e];
+        // stage the chunk split into residue segments: column i of block jj goes to
+        // segment i % 4 at position (i % (D/2)) / 4 + (i >= D/2 ? D/8 : 0)
+        for (int e = tid; e < nj * D / 4; e += C::THREADS) {
+            const int jj = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            const float4 v = kb4[(size_t)j0 * D / 4 + e];
+            const int pos = (c4 % (D / 2)) / 4 + (c4 >= D / 2 ? D / 8 : 0);
+            float* seg = kst + (jj * 4) * C::SEG + pos;
+            seg[0 * C::SEG] = v.x;
+            seg[1 * C::SEG] = v.y;
+            seg[2 * C::SEG] = v.z;
+            seg[3 * C::SEG] = v.w;
+        }
         __syncthreads();
-        for (int jj = warp; jj < nj; jj += 8) {
-            float s = canonical_dot<D>(qr, kst + jj * D);
+        for (int jj = wpart; jj < nj; jj += wsplit) {
+            float s = canonical_dot4<D>(qr, kst + (jj * 4 + r) * C::SEG, r);
             // covariance-aware routing: one fp32 add of the block's bias
             if (bias) s = __fadd_rn(s, __ldg(bias + (size_t)bh * nblk + j0 + jj));
-            if (live) sc[lane * SS + j0 + jj] = s;
+            if (live && r == 0) sc[t * SS + j0 + jj] = s;
         }
         __syncthreads();
     }
@@ -150,8 +174,8 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
     // the score table itself, when asked for ([BH, nblk, nblk] fp32)
     if (scores_out) {
         for (int e = tid; e < nq * nblk; e += C::THREADS) {
-            const int t = e / nblk, jj = e % nblk;
-            scores_out[((size_t)bh * nblk + i0 + t) * nblk + jj] = sc[t * SS + jj];
+            const int tt = e / nblk, jj = e % nblk;
+            scores_out[((size_t)bh * nblk + i0 + tt) * nblk + jj] = sc[tt * SS + jj];
         }
     }
 
@@ -159,9 +183,9 @@ __global__ void __launch_bounds__(256, 1) select_kernel(const T* __restrict__ q,
     // blocks' ordered keys (j = lane + 32 i) in registers during the search.
     const unsigned lt_mask = (1u << lane) - 1u;
     const int nk = (nblk + 31) / 32;
-    for (int t = warp; t < nq; t += 8) {
-        const float* st = sc + t * SS;
-        const size_t row = (size_t)bh * nblk + i0 + t;
+    for (int tt = warp; tt < nq; tt += 8) {
+        const float* st = sc + tt * SS;
+        const size_t row = (size_t)bh * nblk + i0 + tt;
         uint32_t thr = 0u;  // K-th largest ordered score (unused when K is 0 or nblk)
         int need = 0;       // how many of the ties at thr to take, lowest index first
         if (K > 0 && K < nblk) {

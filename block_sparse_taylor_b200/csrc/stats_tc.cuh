@@ -20,9 +20,7 @@
 // 2-7 = 0, so that one MMA gives q . kbar_j as two columns to within about
 // 2^-16 of the fp32 centroid.
 //
-// One CTA (128 threads) per (block, bh): warp 0 allocates TMEM, lane 0 of
-// warp 0 issues the TMA loads and the MMAs; all four warps then compute the
-// column sums from shared memory and run the epilogue (thread = TMEM lane).
+// Persistent CTAs (one per SM), each looping over blocks: see stats_tc_kernel.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -38,11 +36,14 @@ template <int D, int BS>
 struct StatsTcCfg {
     static constexpr uint32_t BOX_BYTES = BS * 128;             // BS rows x 64 bf16 columns
     static constexpr uint32_t TILE_BYTES = (D / 64) * BOX_BYTES;
-    static constexpr uint32_t V_OFF = 0;                        // V tile first: [V ; K] stacking for d = 64
-    static constexpr uint32_t K_OFF = TILE_BYTES;
-    static constexpr uint32_t BAR_OFF = 2 * TILE_BYTES;
-    static constexpr uint32_t KB_OFF = BAR_OFF + 64;            // fp32 kbar[D], vsum[D]
-    static constexpr uint32_t SMEM = KB_OFF + 2 * D * 4 + 1024;
+    static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;     // V tile, then K tile ([V ; K] for d = 64)
+    static constexpr int NSTG = (196608 / STAGE_BYTES) < 6 ? (int)(196608 / STAGE_BYTES) : 6;
+    static constexpr uint32_t BAR_OFF = NSTG * STAGE_BYTES;
+    // FULL, EMPTY per stage; MMADONE, EPIDONE, KBREADY per TMEM buffer; DONE
+    static constexpr uint32_t NBAR = 2 * NSTG + 6 + 1;
+    static constexpr uint32_t KB_OFF = BAR_OFF + NBAR * 8 + 8;  // fp32 kbar[2][D], vsum[2][D]
+    static constexpr uint32_t SMEM = KB_OFF + 4 * D * 4 + 1024;
+    static constexpr int THREADS = 192;                         // producer, MMA, four epilogue warps
 };
 
 template <int D, int ORDER>
@@ -58,34 +59,56 @@ __device__ __forceinline__ float swz_elem(const uint8_t* tile, int n, int c) {
     return __bfloat162float(*p);
 }
 
+// Persistent: CTA c takes the blocks c, c + grid, c + 2 grid, ... of the flattened
+// (bh, j) index.  Warp 0 streams K_j and V_j through NSTG TMA stages; warp 1 runs
+// the Gram MMAs into two TMEM buffers (block i into buffer i % 2); warps 2-5 take
+// the column sums from the stage, then the epilogue from TMEM.  A stage is free
+// again once its MMA has completed and the column sums have read it; a TMEM
+// buffer once the epilogue has read it.  So the loads of the next blocks and the
+// MMA of the next block overlap this block's epilogue.
 template <int D, int BS, int ORDER>
-__global__ void __launch_bounds__(128) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                                       const __grid_constant__ CUtensorMap tm_v,
-                                                       float* __restrict__ kbar, float* __restrict__ vsum,
-                                                       bf16* __restrict__ hstat, bf16* __restrict__ cov,
-                                                       bf16* __restrict__ kaug, int L, int nblk, unsigned* status) {
+__global__ void __launch_bounds__(192, 1) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                          const __grid_constant__ CUtensorMap tm_v,
+                                                          float* __restrict__ kbar, float* __restrict__ vsum,
+                                                          bf16* __restrict__ hstat, bf16* __restrict__ cov,
+                                                          bf16* __restrict__ kaug, int L, int nblk, long total,
+                                                          unsigned* status) {
     using C = StatsTcCfg<D, BS>;
     // M = 128 always (d = 64 stacks V and K); N = d; both operands MN-major
     constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    constexpr uint32_t TCOLS = stats_tmem_cols<D, ORDER>();  // one buffer
+    constexpr long long LIMIT = 2000000000ll;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_addr(smem);
-    const uint32_t bar_full = sbase + C::BAR_OFF, bar_mma = sbase + C::BAR_OFF + 8;
-    uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 16);
-    float* kb = (float*)(smem + C::KB_OFF);
-    float* vs = kb + D;
+    auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+    const int B_FULL = 0, B_EMPTY = C::NSTG, B_MMADONE = 2 * C::NSTG, B_EPIDONE = B_MMADONE + 2,
+              B_KBREADY = B_EPIDONE + 2, B_DONE = B_KBREADY + 2;
+    uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
+    float* kbs = (float*)(smem + C::KB_OFF);  // [2][D]
+    float* vss = kbs + 2 * D;                 // [2][D]
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int j = blockIdx.x, bh = blockIdx.y;
     bool aborted = false;
+    // number of blocks this CTA processes
+    const long first = blockIdx.x, stride = gridDim.x;
+    const int nmine = first < total ? (int)((total - 1 - first) / stride + 1) : 0;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(bar_full, 1);
-        tc::mbar_init(bar_mma, 1);
+        for (int s = 0; s < C::NSTG; ++s) {
+            tc::mbar_init(bar(B_FULL + s), 1);
+            tc::mbar_init(bar(B_EMPTY + s), 1 + 4);  // the MMA's commit + the four column-sum warps
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar(B_MMADONE + b), 1);
+            tc::mbar_init(bar(B_EPIDONE + b), 4);
+            tc::mbar_init(bar(B_KBREADY + b), 4);  // the four warps have written kbar/vsum of the block
+        }
+        tc::mbar_init(bar(B_DONE), 1);
         tc::fence_barrier_init();
     }
-    if (warp == 0) {
-        tc::tmem_alloc(tc::smem_addr(tmem_slot), stats_tmem_cols<D, ORDER>());
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), 2 * TCOLS);
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
@@ -93,103 +116,154 @@ __global__ void __launch_bounds__(128) stats_tc_kernel(const __grid_constant__ C
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (threadIdx.x == 0) {
-        const int row = bh * L + j * BS;
-        tc::mbar_expect_tx(bar_full, 2 * C::TILE_BYTES);
-        for (int b = 0; b < D / 64; ++b) {
-            tc::tma_load_2d(sbase + C::V_OFF + b * C::BOX_BYTES, &tm_v, bar_full, b * 64, row);
-            tc::tma_load_2d(sbase + C::K_OFF + b * C::BOX_BYTES, &tm_k, bar_full, b * 64, row);
-        }
-        if (tc::mbar_wait(bar_full, 0, aborted, status, 2000000000ll)) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < BS / 16; ++kk) {
-                const uint32_t off = kk * 16 * 128;  // 16 tokens further along K
-                // H_raw (d = 128), or [H_raw ; C_raw] (d = 64): A = V^T (stacked with K^T)
-                const uint64_t a_v = tc::sdesc_sw128(sbase + C::V_OFF + off, C::BOX_BYTES, 1024);
-                const uint64_t b_k = tc::sdesc_sw128(sbase + C::K_OFF + off, C::BOX_BYTES, 1024);
-                tc::mma_ss(tmem, a_v, b_k, IDESC, kk > 0);
-                if (D == 128 && ORDER == 2) {
-                    const uint64_t a_k = tc::sdesc_sw128(sbase + C::K_OFF + off, C::BOX_BYTES, 1024);
-                    tc::mma_ss(tmem + 128, a_k, b_k, IDESC, kk > 0);
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch(&tm_k);
+            tc::tma_prefetch(&tm_v);
+            int last = -1;
+            for (int i = 0; i < nmine; ++i) {
+                const int s = i % C::NSTG, u = i / C::NSTG;
+                if (u > 0 && !tc::mbar_wait(bar(B_EMPTY + s), (u - 1) & 1, aborted, status, LIMIT)) break;
+                const long blk = first + (long)i * stride;
+                const int bh = (int)(blk / nblk), j = (int)(blk % nblk);
+                const int row = bh * L + j * BS;
+                const uint32_t st = sbase + s * C::STAGE_BYTES;
+                tc::mbar_expect_tx(bar(B_FULL + s), C::STAGE_BYTES);
+                for (int b = 0; b < D / 64; ++b) {
+                    tc::tma_load_2d(st + b * C::BOX_BYTES, &tm_v, bar(B_FULL + s), b * 64, row);
+                    tc::tma_load_2d(st + C::TILE_BYTES + b * C::BOX_BYTES, &tm_k, bar(B_FULL + s), b * 64, row);
+                }
+                last = i;
+            }
+            if (aborted) {
+                // let the copies already issued land before the CTA exits
+                for (int i = (last - C::NSTG + 1 > 0 ? last - C::NSTG + 1 : 0); i <= last; ++i) {
+                    bool a2 = false;
+                    tc::mbar_wait(bar(B_FULL + i % C::NSTG), (i / C::NSTG) & 1, a2, status, LIMIT);
                 }
             }
-            tc::mma_commit(bar_mma);
         }
-    }
-    // column sums from shared memory (all threads), once the tiles have landed
-    if (tc::mbar_wait_warp(bar_full, 0, aborted, status, 2000000000ll)) {
-        for (int c = threadIdx.x; c < D; c += 128) {
-            float a[BS];
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            for (int i = 0; i < nmine; ++i) {
+                const int s = i % C::NSTG, u = i / C::NSTG, buf = i & 1, ub = i >> 1;
+                if (!tc::mbar_wait(bar(B_FULL + s), u & 1, aborted, status, LIMIT)) break;
+                if (ub > 0 && !tc::mbar_wait(bar(B_EPIDONE + buf), (ub - 1) & 1, aborted, status, LIMIT)) break;
+                tc::fence_after_sync();
+                const uint32_t sa = sbase + s * C::STAGE_BYTES;
+                const uint32_t dt = tmem + (uint32_t)(buf * TCOLS);
 #pragma unroll
-            for (int n = 0; n < BS; ++n) a[n] = swz_elem<BS>(smem + C::K_OFF, n, c);
-            const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-            float s = 0.f;
-            for (int n = 0; n < BS; ++n) s += swz_elem<BS>(smem + C::V_OFF, n, c);
-            kb[c] = m;
-            vs[c] = s;
-            const size_t so = ((size_t)bh * nblk + j) * D + c;
-            kbar[so] = m;
-            vsum[so] = s;
-            if (kaug) {
-                bf16* ka = kaug + ((size_t)bh * nblk + j) * 8 * D + c;
-                const bf16 hi = __float2bfloat16_rn(m);
-                ka[0] = hi;
-                ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
-#pragma unroll
-                for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
+                for (int kk = 0; kk < BS / 16; ++kk) {
+                    const uint32_t off = kk * 16 * 128;  // 16 tokens further along K
+                    // H_raw (d = 128), or [H_raw ; C_raw] (d = 64): A = V^T (stacked with K^T)
+                    const uint64_t a_v = tc::sdesc_sw128(sa + off, C::BOX_BYTES, 1024);
+                    const uint64_t b_k = tc::sdesc_sw128(sa + C::TILE_BYTES + off, C::BOX_BYTES, 1024);
+                    tc::mma_ss(dt, a_v, b_k, IDESC, kk > 0);
+                    if (D == 128 && ORDER == 2) tc::mma_ss(dt + 128, b_k, b_k, IDESC, kk > 0);
+                }
+                tc::mma_commit(bar(B_MMADONE + buf));
+                tc::mma_commit(bar(B_EMPTY + s));
             }
+            // every MMA issued by this thread has completed before TMEM is freed
+            tc::mma_commit(bar(B_DONE));
+            bool a2 = false;
+            tc::mbar_wait(bar(B_DONE), 0, a2, status, LIMIT);
         }
-    }
-    __syncthreads();
-    if (tc::mbar_wait_warp(bar_mma, 0, aborted, status, 2000000000ll)) {
-        tc::fence_after_sync();
-        const int r = warp * 32 + lane;  // TMEM lane = output row
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-        const size_t base = ((size_t)bh * nblk + j) * D * D;
+    } else {
+        // ------------------------------------------------ column sums, epilogue
+        const int ct = threadIdx.x - 64;         // 0 .. 127
+        const int quarter = warp % 4;            // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;       // TMEM lane = output row
         const float inv_b = 1.0f / (float)BS;
-        // which matrix and row this lane holds
-        const bool is_h = (D == 128) || (r < 64);
-        const int a = (D == 128) ? r : (r & 63);
-        const bool want = is_h || ORDER == 2;
-        const float rowv = is_h ? vs[a] : kb[a];
+        for (int i = 0; i < nmine; ++i) {
+            const int s = i % C::NSTG, u = i / C::NSTG, buf = i & 1, ub = i >> 1;
+            const long blk = first + (long)i * stride;
+            const int bh = (int)(blk / nblk), j = (int)(blk % nblk);
+            if (!tc::mbar_wait_warp(bar(B_FULL + s), u & 1, aborted, status, LIMIT)) break;
+            const uint8_t* st = smem + s * C::STAGE_BYTES;
+            for (int c = ct; c < D; c += 128) {
+                float a[BS];
 #pragma unroll
-        for (int part = 0; part < ((D == 128 && ORDER == 2) ? 2 : 1); ++part) {
-            const bool h_here = (D == 128) ? (part == 0) : is_h;
-            bf16* dst = (h_here ? hstat : cov) + base + (size_t)a * D;
-            const float rv = (D == 128) ? (part == 0 ? vs[a] : kb[a]) : rowv;
+                for (int n = 0; n < BS; ++n) a[n] = swz_elem<BS>(st + C::TILE_BYTES, n, c);
+                const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+                float sv = 0.f;
+                for (int n = 0; n < BS; ++n) sv += swz_elem<BS>(st, n, c);
+                kbs[buf * D + c] = m;
+                vss[buf * D + c] = sv;
+                const size_t so = ((size_t)bh * nblk + j) * D + c;
+                kbar[so] = m;
+                vsum[so] = sv;
+                if (kaug) {
+                    bf16* ka = kaug + ((size_t)bh * nblk + j) * 8 * D + c;
+                    const bf16 hi = __float2bfloat16_rn(m);
+                    ka[0] = hi;
+                    ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t raw[32];
-                tc::tmem_ld32(taddr + part * 128 + c0, raw);
-                tc::tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
-                    if (h_here) {
-                        x0 = fmaf(-rv, kb[c0 + 2 * e], x0);
-                        x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1);
-                    } else {
-                        x0 = fmaf(-rv, kb[c0 + 2 * e], x0 * inv_b);
-                        x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1 * inv_b);
-                    }
-                    pk[e] = tc::pack_bf16x2(x0, x1);
-                }
-                if (want) {
-                    uint4* o = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
                 }
             }
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(bar(B_EMPTY + s));    // this warp no longer reads the stage
+                tc::mbar_arrive(bar(B_KBREADY + buf));  // and its columns of kbar/vsum are in kbs/vss
+            }
+            // the block's kbar and vsum from all four warps (a bounded wait, unlike a named barrier,
+            // so a warp that gave up cannot hold the others forever)
+            if (!tc::mbar_wait_warp(bar(B_KBREADY + buf), ub & 1, aborted, status, LIMIT)) break;
+            if (!tc::mbar_wait_warp(bar(B_MMADONE + buf), ub & 1, aborted, status, LIMIT)) break;
+            tc::fence_after_sync();
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TCOLS);
+            const size_t base = ((size_t)bh * nblk + j) * D * D;
+            const float* kb = kbs + buf * D;
+            const float* vs = vss + buf * D;
+            // which matrix and row this lane holds
+            const bool is_h = (D == 128) || (r < 64);
+            const int ar = (D == 128) ? r : (r & 63);
+            const bool want = is_h || ORDER == 2;
+#pragma unroll
+            for (int part = 0; part < ((D == 128 && ORDER == 2) ? 2 : 1); ++part) {
+                const bool h_here = (D == 128) ? (part == 0) : is_h;
+                bf16* dst = (h_here ? hstat : cov) + base + (size_t)ar * D;
+                const float rv = h_here ? vs[ar] : kb[ar];
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t raw[32];
+                    tc::tmem_ld32(taddr + part * 128 + c0, raw);
+                    tc::tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
+                        if (h_here) {
+                            x0 = fmaf(-rv, kb[c0 + 2 * e], x0);
+                            x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1);
+                        } else {
+                            x0 = fmaf(-rv, kb[c0 + 2 * e], x0 * inv_b);
+                            x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1 * inv_b);
+                        }
+                        pk[e] = tc::pack_bf16x2(x0, x1);
+                    }
+                    if (want) {
+                        uint4* o = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(B_EPIDONE + buf));  // the TMEM buffer is read
         }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         __syncwarp();
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, stats_tmem_cols<D, ORDER>());
+        tc::tmem_dealloc(tmem, 2 * TCOLS);
     }
 }
 
@@ -221,7 +295,15 @@ inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float
             return PISA_ERR_CUDA;
         }
     }
-    dim3 grid((unsigned)nblk, (unsigned)BH);
+    // persistent: one CTA per SM (fewer when there are fewer blocks)
+    static int nsm = 0;
+    if (!nsm) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0) nsm = 148;
+    }
+    const long total = BH * (long)nblk;
+    dim3 grid((unsigned)(total < nsm ? total : nsm));
     cudaError_t e = cudaSuccess;
 #define PISA_STATS_TC(DD, BB, OO)                                                                             \
     if (d == DD && B == BB && order == OO) {                                                                  \
@@ -229,8 +311,8 @@ inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,                           \
                                  (int)StatsTcCfg<DD, BB>::SMEM);                                              \
         if (e == cudaSuccess) {                                                                               \
-            kern<<<grid, 128, StatsTcCfg<DD, BB>::SMEM, s>>>(maps[0], maps[1], kbar, vsum, (bf16*)hstat,      \
-                                                             (bf16*)cov, (bf16*)kaug, L, nblk, status);       \
+            kern<<<grid, StatsTcCfg<DD, BB>::THREADS, StatsTcCfg<DD, BB>::SMEM, s>>>(                         \
+                maps[0], maps[1], kbar, vsum, (bf16*)hstat, (bf16*)cov, (bf16*)kaug, L, nblk, total, status); \
             e = cudaGetLastError();                                                                           \
         }                                                                                                     \
     } else

@@ -82,6 +82,28 @@ def test_stats_parity(dt, d, B, order):
         assert st.cov is None
 
 
+@pytest.mark.parametrize("d,B,order", [(128, 64, 1), (128, 128, 2), (64, 64, 2), (64, 128, 1)])
+def test_stats_parity_many_blocks_per_cta(d, B, order):
+    # more blocks than SMs: every persistent CTA loops over several blocks, through the ring
+    # of stages and both TMEM buffers; also the bf16 high/low split of the centroids
+    q, k, v = pisa_synth.random_qkv(150 + d + B, 6, 8192, d, dtype="bf16")
+    st = pisa.pisa_stats(dev(k, "bf16"), dev(v, "bf16"), B, order)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    kbar_ref = oracle.centroids_f32(k, B)
+    assert np.array_equal(st.kbar.cpu().numpy().view(np.uint32), kbar_ref.view(np.uint32))
+    _, vsum, H, C = oracle.block_stats(k, v, B, order=2)
+    parity.check(st.vsum.cpu().numpy(), vsum, "bf16", "vsum", tol=1e-6, row_tol=1e-6, elem_tol=1e-6)
+    parity.check(st.hstat.float().cpu().numpy(), H, "bf16", "H", tol=8e-3, row_tol=1.6e-2, elem_tol=1.6e-2)
+    if order == 2:
+        parity.check(st.cov.float().cpu().numpy(), C, "bf16", "C", tol=8e-3, row_tol=1.6e-2, elem_tol=1.6e-2)
+    ka = st.kaug.float().cpu().numpy()
+    hi = pisa_synth.round_bf16(kbar_ref)
+    assert np.array_equal(ka[:, :, 0], hi)
+    assert np.array_equal(ka[:, :, 1], pisa_synth.round_bf16(kbar_ref - hi))
+    assert not np.any(ka[:, :, 2:])
+
+
 # ---------------------------------------------------------------------------
 # selection
 # ---------------------------------------------------------------------------
@@ -526,3 +548,12 @@ def test_auto_runs_the_statistics_form_at_the_hunyuan_and_clustered_shapes():
     q, k, v = pisa_synth.generate(w)
     auto = run_attn(q, k, v, w.B, w.K, 1, w.dtype, "auto")
     assert np.array_equal(auto, run_attn(q, k, v, w.B, w.K, 1, w.dtype, "stats_tc"))
+
+
+def test_hybrid_is_reproducible():
+    # H-bar is summed over the prepare kernel's chunks in a fixed order (no atomics), so two
+    # calls on the same inputs give the same output bit for bit
+    q, k, v = pisa_synth.random_qkv(870, 6, 8192, 128, scale=2.0, dtype="bf16")
+    a = run_attn(q, k, v, 64, 16, 1, "bf16", "hybrid_tc")
+    for _ in range(2):
+        assert np.array_equal(a, run_attn(q, k, v, 64, 16, 1, "bf16", "hybrid_tc"))
