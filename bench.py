@@ -648,6 +648,9 @@ def main():
     # the biased selection, timed on their own on the same inputs.
     route_rec = None
     if path != "stats" and not args.no_route:
+        # its own selection buffers: the timed step's mask stays for the parity record
+        idx_rt = torch.empty_like(idx)
+        mask_rt = torch.empty_like(mask)
         rb = torch.empty((BH, nblk), dtype=torch.float32, device="cuda")
         st_c = pisa.pisa_centroids(k, B, kbar=kbar)
         for _ in range(2):
@@ -660,8 +663,8 @@ def main():
         rb_ev.record(stream)
         for _ in range(reps):
             pisa._check(pisa.lib().pisa_select_biased(q.data_ptr(), pisa.ctypes.byref(st_c.raw), K,
-                                                       rb.data_ptr(), idx.data_ptr() if K else None,
-                                                       mask.data_ptr(), stream.cuda_stream))
+                                                       rb.data_ptr(), idx_rt.data_ptr() if K else None,
+                                                       mask_rt.data_ptr(), stream.cuda_stream))
         rc_ev.record(stream)
         torch.cuda.synchronize()
         pisa.pisa_poll_device_status()
@@ -670,7 +673,7 @@ def main():
                      "bias_gflops_fp32": 2.0 * BH * nblk * B * d * d / (r_ms * 1e-3) / 1e9,
                      "select_biased_ms": rb_ev.elapsed_time(rc_ev) / reps,
                      "note": "scalar IEEE fp32 in a canonical order (reproducible bit for bit), CUDA cores"}
-        del rb
+        del rb, idx_rt, mask_rt
 
     # The PISA hybrid (global H-bar, the paper's own speed path) on the same
     # inputs: a separate record, timed as whole calls of pisa_attention.
@@ -708,7 +711,8 @@ def main():
 
     # The backward pass (training use) on the same inputs: dq, dk, dv of
     # sum(dO * o) for the forward output o above, selection held fixed; timed
-    # as whole calls (centroids, selection, row statistics, dq, dk/dv).
+    # as whole calls (centroids, selection, delta, dq, dk/dv) given the
+    # forward's log-denominators, as the autograd function calls it.
     bwd_rec = None
     if not args.no_backward:
         gen = torch.Generator(device="cuda").manual_seed(4321 + rank)
@@ -716,39 +720,48 @@ def main():
         grads = tuple(torch.empty(q.shape, dtype=torch.float32, device="cuda") for _ in range(3))
         bws = torch.empty(pisa.pisa_backward_workspace_bytes(1, BH, L, d, B, K, order, tdt), dtype=torch.uint8,
                           device="cuda")
-        pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws)
+        _, lse = pisa.pisa_attention_lse(q, k, v, B, K, order)
+        for _ in range(2):
+            pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws, lse=lse)
         torch.cuda.synchronize()
         pisa.pisa_poll_device_status()
         ba, bb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 2
+        reps = 3
         ba.record(stream)
         for _ in range(reps):
-            pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws)
+            pisa.pisa_attention_backward(q, k, v, out, dO, B, K, order, grads=grads, workspace=bws, lse=lse)
         bb.record(stream)
         torch.cuda.synchronize()
         pisa.pisa_poll_device_status()
         b_ms = ba.elapsed_time(bb) / reps
+        tc_bwd = tdt == torch.bfloat16 and d in (64, 128) and B in (64, 128) and L % 128 == 0
         alg = 10.0 * L * L * d * BH       # S, dP, dq, dk, dv once each (five products of 2 L^2 d)
-        executed = 16.0 * L * L * d * BH  # S in all three kernels and dP in two are recomputed
+        # tcgen05 path: S, G, dQ in the dq kernel and S, G, dK, dV in the dk/dv kernel
+        executed = (14.0 if tc_bwd else 16.0) * L * L * d * BH
         bf16_peak = float(peaks["bf16_tflops"])
-        bwd_rec = {"kernels": [f"bwd_rowstat_kernel<{d},{B}>", f"bwd_dq_kernel<{d},{B}>",
-                               f"bwd_dkdv_kernel<{d},{B}>"],
+        kernels = ([f"bwd_delta_kernel<{d}>", f"bwd_dq_tc_kernel<{d},{B},{order}>",
+                    f"bwd_dkdv_tc_kernel<{d},{B},{order}>"] if tc_bwd else
+                   [f"bwd_rowstat_kernel<{d},{B}>", f"bwd_dq_kernel<{d},{B}>", f"bwd_dkdv_kernel<{d},{B}>"])
+        bwd_rec = {"kernels": kernels,
                    "ms_per_call": b_ms, "algorithmic_flops_per_call": alg,
                    "algorithmic_tflops": alg / (b_ms * 1e-3) / 1e12,
                    "executed_tflops": executed / (b_ms * 1e-3) / 1e12,
                    "roofline": ({"bound": "tensor", "peak": bf16_peak, "unit": "TFLOP/s",
                                  "frac": alg / (b_ms * 1e-3) / 1e12 / bf16_peak,
+                                 "frac_executed": executed / (b_ms * 1e-3) / 1e12 / bf16_peak,
                                  "peak_source": f"{peak_kind} bf16 dense (burst)"}
                                 if tdt == torch.bfloat16 else None),
-                   "tile_products": ("warp-level mma.sync m16n8k16, bf16 operands, fp32 accumulation"
+                   "tile_products": ("tcgen05 128xN tiles, bf16 operands, fp32 accumulation in TMEM" if tc_bwd else
+                                     "warp-level mma.sync m16n8k16, bf16 operands, fp32 accumulation"
                                      if tdt == torch.bfloat16 else "fp32 FMA"),
+                   "lse": "from the forward (pisa_attention_lse)",
                    "launches_per_call": 5}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             try:
                 bwd_rec["cpu_baseline"] = cpu_backward_baseline(w, q_h, k_h, v_h, dO[:1].float().cpu().numpy())
             except Exception as e:  # noqa: BLE001 - a baseline record never fails the benchmark
                 bwd_rec["cpu_baseline"] = {"unavailable": f"{type(e).__name__}: {e}"[:240]}
-        del dO, grads, bws
+        del dO, grads, bws, lse
 
     # end to end through the public host-buffer call: pisa_attention_host on
     # pinned host q, k, v, out (per chunk of heads: H2D copies, the attention,

@@ -99,6 +99,11 @@ def lib():
         L.pisa_noalloc_scratch_bytes.restype = sz
         L.pisa_attention_backward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
         L.pisa_attention_backward.restype = ctypes.c_int
+        L.pisa_attention_backward_lse.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, vp, vp, vp,
+                                                  sz, vp]
+        L.pisa_attention_backward_lse.restype = ctypes.c_int
+        L.pisa_attention_lse.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp, vp, sz, vp]
+        L.pisa_attention_lse.restype = ctypes.c_int
         L.pisa_backward_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
         L.pisa_backward_workspace_bytes.restype = sz
         L.pisa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
@@ -324,16 +329,47 @@ def pisa_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K:
     return out
 
 
+def pisa_attention_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
+                       gate: bool = True, path: str = "auto", out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                       w_mode: str = "exact", route: str = "centroid"):
+    """pisa_attention plus each row's log-denominator: returns (out, lse) with lse [batch*heads, L]
+    fp32, lse_t = ln D_t (what pisa_attention_backward takes to skip its own row statistics)."""
+    _need_cuda(q, k, v)
+    if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share shape and dtype")
+    batch, heads, L, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((batch * heads, L), dtype=torch.float32, device=q.device)
+    _need_cuda(out, lse)
+    nbytes = pisa_workspace_bytes(batch, heads, L, d, B, K, order, q.dtype, path)
+    if nbytes == 0:
+        raise PisaError(PISA_ERR_INVALID_ARG if path == "auto" else PISA_ERR_UNSUPPORTED,
+                        f"no workspace size for these arguments (path={path})")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().pisa_attention_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), batch, heads, L, d,
+                                    _dtype_code(q.dtype), B, K, order, _flags(gate, w_mode, route), PATHS[path],
+                                    out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                    _stream(stream)))
+    return out, lse
+
+
 def pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, dtype: torch.dtype) -> int:
     return int(lib().pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, _dtype_code(dtype)))
 
 
 def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
                             B: int, K: int, order: int = 1, gate: bool = True, route: str = "centroid",
-                            grads: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+                            grads: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                            lse: Optional[torch.Tensor] = None):
     """(dq, dk, dv) fp32, the gradients of sum(dO * o) for o = pisa_attention(q, k, v, B, K, order,
     gate=gate, route=route) on the per-block paths, the selection held fixed.  ``o`` is that
-    forward's output; ``grads`` optional preallocated fp32 (dq, dk, dv)."""
+    forward's output; ``lse`` optionally its log-denominators (pisa_attention_lse), which spares
+    the backward its own pass for the row statistics; ``grads`` optional preallocated fp32
+    (dq, dk, dv)."""
     _need_cuda(q, k, v, o, dO)
     if not (q.shape == k.shape == v.shape == o.shape == dO.shape
             and q.dtype == k.dtype == v.dtype == o.dtype == dO.dtype):
@@ -352,10 +388,20 @@ def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dq, dk, dv = grads
-    _check(lib().pisa_attention_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(),
-                                         batch, heads, L, d, code, B, K, order, _flags(gate, "exact", route),
-                                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                                         workspace.numel(), _stream(stream)))
+    if lse is None:
+        _check(lib().pisa_attention_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(),
+                                             batch, heads, L, d, code, B, K, order, _flags(gate, "exact", route),
+                                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                             workspace.numel(), _stream(stream)))
+    else:
+        _need_cuda(lse)
+        if lse.dtype != torch.float32 or lse.numel() != batch * heads * L:
+            raise ValueError("lse must be fp32 with batch*heads*L elements")
+        _check(lib().pisa_attention_backward_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                                 dO.data_ptr(), lse.data_ptr(), batch, heads, L, d, code, B, K, order,
+                                                 _flags(gate, "exact", route), dq.data_ptr(), dk.data_ptr(),
+                                                 dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                                 _stream(stream)))
     return dq, dk, dv
 
 
@@ -365,16 +411,17 @@ class PisaAttentionFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, B, K, order, gate, path, route):
-        out = pisa_attention(q, k, v, B, K, order, gate=gate, path=path, route=route)
-        ctx.save_for_backward(q, k, v, out)
+        out, lse = pisa_attention_lse(q, k, v, B, K, order, gate=gate, path=path, route=route)
+        ctx.save_for_backward(q, k, v, out, lse)
         ctx.cfg = (B, K, order, gate, route)
         return out
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, out = ctx.saved_tensors
+        q, k, v, out, lse = ctx.saved_tensors
         B, K, order, gate, route = ctx.cfg
-        dq, dk, dv = pisa_attention_backward(q, k, v, out, dout.contiguous(), B, K, order, gate=gate, route=route)
+        dq, dk, dv = pisa_attention_backward(q, k, v, out, dout.contiguous(), B, K, order, gate=gate, route=route,
+                                             lse=lse)
         return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None, None, None, None
 
 

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const float* __restrict__ kbar, const float* __restrict__ vsum, const T* __restrict__ hstat,
     const T* __restrict__ cov, const uint32_t* __restrict__ mask, T* __restrict__ out, int L, int nblk,
-    int words, int order, int gate, float ln_b, const float* __restrict__ wmat) {
+    int words, int order, int gate, float ln_b, const float* __restrict__ wmat, float* __restrict__ lse) {
     // wmat (order 2, optional): PWT's pooled diagonal w per (query tile, block), gated
     using SM = AttnStatsSmem<T, D, BS>;
     constexpr int QS = SM::QS, XS = SM::XS, W = D / 32, RQ = SM::RQ;
@@ -190,6 +190,9 @@ __global__ void __launch_bounds__(256) attn_stats_kernel(
         __syncthreads();
     }
     for (int e = tid; e < RQ * D; e += 256) out[base + e] = from_f<T>(Ns[e] / ds[e / D]);
+    // optional log-denominator ln D_t = m + ln(D scaled by e^-m), for the backward
+    if (lse)
+        for (int r = tid; r < RQ; r += 256) lse[(size_t)bh * L + (size_t)i * BS + (size_t)part * RQ + r] = ms[r] + logf(ds[r]);
 }
 
 }  // namespace pisa

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
                     const __grid_constant__ CUtensorMap tm_aug, const uint32_t* __restrict__ mask,
                     const float* __restrict__ vsum, bf16* __restrict__ out, int L, int nblk, int words, int gate,
-                    float ln_b, const float* __restrict__ wmat, unsigned* status) {
+                    float ln_b, const float* __restrict__ wmat, unsigned* status, float* __restrict__ lse) {
     // ORDER: 1 first order; 3 first order + the pooled diagonal w of wmat
     // ([BH, nblk, nblk], row = query tile, already gated) on every unselected block
     static_assert(ORDER == 1 || ORDER == 3, "statistics-form kernel: orders 1 and 3");
@@ -563,6 +563,8 @@ __global__ void __launch_bounds__(kStcThreads, 1)
         // ---- epilogue: o = N / D
         if (!aborted) {
             const float inv = 1.0f / dsum;
+            // optional log-denominator ln D_t = m ln 2 + ln(dsum) (m in log2 units), for the backward
+            if (lse && valid) lse[(size_t)bh * L + qrow] = fmaf(m_run, 0.6931471805599453f, logf(dsum));
             bf16* orow = out + ((size_t)bh * L + (valid ? qrow : 0)) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
 inline pisa_status run_attn_stc(const void* q, const void* k, const void* v, const void* hstat, const void* kaug,
                                 const float* vsum, const uint32_t* mask, void* out, long BH, int L, int d, int B,
                                 int nblk, int words, int order, int gate, const float* wmat, unsigned* status,
-                                cudaStream_t s, std::string* err) {
+                                cudaStream_t s, std::string* err, float* lse = nullptr) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
@@ -637,7 +639,8 @@ inline pisa_status run_attn_stc(const void* q, const void* k, const void* v, con
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StcCfg<DD, BB>::SMEM); \
         if (e == cudaSuccess && regs >= (int)kStcRegsLaunch) {                                                   \
             kern<<<grid, kStcThreads, StcCfg<DD, BB>::SMEM, s>>>(mq, mk, mv, mh, ma, mask, vsum, (bf16*)out, L,    \
-                                                                 nblk, words, gate, logf((float)B), wmat, status); \
+                                                                 nblk, words, gate, logf((float)B), wmat, status, \
+                                                                 lse);                                            \
             e = cudaGetLastError();                                                                              \
         }                                                                                                        \
     } else

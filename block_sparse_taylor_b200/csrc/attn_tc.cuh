@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const uint32_t* __restrict__ mask, bf16* __restrict__ out,
                    int L, int nblk, int words, int gate, float ln_b, const float* __restrict__ wmat,
-                   unsigned* status) {
+                   unsigned* status, float* __restrict__ lse) {
     // ORDER: 0 zeroth, 1 first, 2 first + exact w from the logits, 3 first + the
     // pooled diagonal w of wmat ([BH, nblk, nblk], row = query tile, already gated)
     using C = TcCfg<D>;
@@ -456,6 +456,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (tc::mbar_wait_warp(bar(B_OFULL + h), 0, aborted, status, kWaitLimitCycles)) {
             tc::fence_after_sync();
             const float inv = 1.0f / dsum;
+            // optional log-denominator ln D_t = m ln 2 + ln(dsum) (m in log2 units), for the backward
+            if (lse && valid) lse[(size_t)bh * L + qrow] = fmaf(m_run, 0.6931471805599453f, logf(dsum));
             bf16* orow = out + ((size_t)bh * L + (valid ? qrow : 0)) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -490,7 +492,7 @@ inline bool attn_tc_supported(int d, int B) { return (d == 64 || d == 128) && (B
 // order 3 = order 2 with the pooled w matrix `wmat` ([BH, nblk, nblk] fp32, gated).
 inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, const uint32_t* mask, void* out, long BH,
                                int L, int d, int B, int nblk, int words, int order, int gate, const float* wmat,
-                               unsigned* status, cudaStream_t s, std::string* err) {
+                               unsigned* status, cudaStream_t s, std::string* err, float* lse = nullptr) {
     if (L % 128) {
         *err = "tensor-core path needs L % 128 == 0";
         return PISA_ERR_UNSUPPORTED;
@@ -533,7 +535,7 @@ inline pisa_status run_attn_tc(const void* q, const void* k, const void* v, cons
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcCfg<DD>::SMEM);     \
         if (e == cudaSuccess) {                                                                                \
             kern<<<grid, kTcThreads, TcCfg<DD>::SMEM, s>>>(maps[0], maps[1], maps[2], mask, (bf16*)out, L, nblk, \
-                                                           words, gate, ln_b, wmat, status);                   \
+                                                           words, gate, ln_b, wmat, status, lse);              \
             e = cudaGetLastError();                                                                            \
         }                                                                                                      \
     } else

@@ -1,0 +1,748 @@
+// Backward pass of the piecewise sparse attention on tcgen05 tensor cores
+// (bf16 inputs): the gradients dq, dk, dv of sum_t dO_t . o_t, with the block
+// selection held fixed (the same derivative as backward.cuh; the pages define
+// only the forward: PISA paper section 3.2 "Formulation"; "Sparse Linear
+// Attention" blog, the sparse-linear and PWT sections).
+//
+// Per query row t (x_n = q_t.k_n, G_n = dO_t.v_n, delta = dO_t.o_t, lse_t = ln D_t
+// the forward's log-denominator):
+//   selected key n           P_n = e^{x_n - lse_t},       dS_n = P_n (G_n - delta)
+//   key n of unselected j    sb = mean_n x_n, u_n = x_n - sb, l = sb + w
+//                            (w = [order 2] sum u^2 / 2B, zeroed by the gate),
+//                            a = e^{l - lse_t},  P_n = a (1 + c1 u_n),
+//                            inner = sum_n G_n (1 + c1 u_n) - B delta,
+//                            dS_n = a (dl_n inner + c1 (G_n - mean G)),
+//                            dl_n = 1/B (+ u_n / B for order 2 with the gate open)
+//   dq_t = sum_n dS_tn k_n,   dk_n = sum_t dS_tn q_t,   dv_n = sum_t P_tn dO_t
+// (c1 = 1 for order >= 1, 0 for order 0).
+//
+// bwd_dq_tc_kernel (query-major): one 128-row M tile of one (batch, head) per
+// CTA, visiting every key tile of 128 keys.  Every reduction over a block
+// (sb, sum G, sum G u, the spread behind w) runs over the block's keys of one
+// query row, which are TMEM columns of one lane: each softmax thread does them
+// alone, from its row of S (held in registers) and G (streamed twice).
+//   warp 0      TMA producer: Q and dO once; K tiles through three stages, V
+//               tiles through two (V is free once G = dO V^T has completed)
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2-5   the four lane quarters of the M tile
+// TMEM: S_0 | S_1 | G | dQ.  S = Q K^T alternates between two buffers; the
+// softmax writes dS (bf16) over the first half of the buffer's columns, and
+// dQ += dS K runs from TMEM (K as the MN-major B operand).  MMA order after
+// the softmax of tile j has handed over dS_j and released G:
+//   G_{j+1}, dQ_j, S_{j+2}
+// so the softmax of tile j+1 starts after one product and the other two run
+// beside it.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace pisa {
+namespace bwdtc {
+
+constexpr int kThreads = 192;
+
+template <int D>
+struct DqCfg {
+    static constexpr int NK = 128;
+    static constexpr int NBOX = D / 64;
+    static constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 128 bytes
+    static constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;
+    static constexpr int NSK = 3, NSV = 2;             // K and V stages
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t DO_OFF = Q_OFF + TILE_BYTES;
+    static constexpr uint32_t K_OFF = DO_OFF + TILE_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + NSK * TILE_BYTES;
+    static constexpr uint32_t BAR_OFF = V_OFF + NSV * TILE_BYTES;
+    // QFULL; KFULL, KEMPTY per K stage; VFULL, VEMPTY per V stage; SFULL, DSREADY per
+    // S buffer; GFULL, GFREE; DQFULL; DONE
+    static constexpr uint32_t NBAR = 1 + 2 * NSK + 2 * NSV + 4 + 2 + 1 + 1;
+    static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+    static constexpr uint32_t G_COL = 256, DQ_COL = 384;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// delta_t = dO_t . o_t (one warp per row, fp32 accumulation)
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dO,
+                                                        long rows, float* __restrict__ delta) {
+    const long row = (long)blockIdx.x * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(o + row * D);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(dO + row * D);
+    float s = 0.f;
+#pragma unroll
+    for (int c = lane; c < D / 2; c += 32) {
+        const float2 x = __bfloat1622float2(a[c]), y = __bfloat1622float2(b[c]);
+        s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
+    }
+    s = warp_sum(s);
+    if (lane == 0) delta[row] = s;
+}
+
+// lse_t = m_t + ln D_t from the row statistics kernel's m_t and 1/D_t
+__global__ void bwd_lse_kernel(const float* __restrict__ m, const float* __restrict__ dinv, long n,
+                               float* __restrict__ lse) {
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+        lse[i] = m[i] - logf(dinv[i]);
+}
+
+// Block reductions of one query row over a key tile (TMEM columns of one lane), in one pass
+// over S and G shifted by the block's first logit x0 (the shift keeps the sums of
+// (x - x0) free of cancellation when the block's logits share a large offset):
+//   s1 = sum (x - x0), s2 = sum (x - x0)^2, sg = sum G, sgd = sum G (x - x0)
+// so that sb = x0 + s1/B, sum (x - sb)^2 = s2 - s1^2/B, sum G (x - sb) = sgd - (s1/B) sg.
+template <int BPT, int BS>
+struct RowBlockSums {
+    float x0[BPT], s1[BPT], s2[BPT], sg[BPT], sgd[BPT];
+};
+
+template <int BPT, int BS>
+__device__ __forceinline__ void row_block_sums(uint32_t s_addr, uint32_t g_addr, RowBlockSums<BPT, BS>& r) {
+#pragma unroll
+    for (int bb = 0; bb < BPT; ++bb) r.x0[bb] = r.s1[bb] = r.s2[bb] = r.sg[bb] = r.sgd[bb] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 128 / 16; ++c) {
+        uint32_t xs[16], gs[16];
+        tc::tmem_ld16(s_addr + c * 16, xs);
+        tc::tmem_ld16(g_addr + c * 16, gs);
+        tc::tmem_wait_ld();
+        const int bb = (c * 16) / BS;
+        if ((c * 16) % BS == 0) r.x0[bb] = __uint_as_float(xs[0]);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float dx = __uint_as_float(xs[e]) - r.x0[bb], gv = __uint_as_float(gs[e]);
+            r.s1[bb] += dx;
+            r.s2[bb] = fmaf(dx, dx, r.s2[bb]);
+            r.sg[bb] += gv;
+            r.sgd[bb] = fmaf(gv, dx, r.sgd[bb]);
+        }
+    }
+}
+
+// Per-block coefficients from the sums: sb (mean logit), a = e^{l - lse} (l = sb + w),
+// and dS_n = A G_n + X u_n + Cc, P_n = a + Pu u_n for an unselected block (u_n = x_n - sb).
+template <int BS, int ORDER>
+__device__ __forceinline__ void block_coefs(float x0, float s1, float s2, float sg, float sgd, float lse2, float del,
+                                            int gate, float ln_b, float& sb, float& a, float& A, float& X,
+                                            float& Cc, float& Pu) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr float INV_B = 1.0f / (float)BS;
+    constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
+    const float md = s1 * INV_B;
+    sb = x0 + md;
+    float w = 0.f, q2 = 0.f;
+    if (ORDER == 2) {
+        // w = (1/2B) sum (x - sb)^2 and the forward's gate decision held fixed: dl_n carries
+        // u_n / B only where w was kept
+        w = 0.5f * fmaxf(fmaf(-md, s1, s2), 0.f) * INV_B;
+        if (gate && w > ln_b) {
+            w = 0.f;
+        } else {
+            q2 = INV_B;
+        }
+    }
+    a = tc::ex2((sb + w) * LOG2E - lse2);
+    const float sgu = fmaf(-md, sg, sgd);  // sum G (x - sb)
+    const float inner = sg + C1 * sgu - (float)BS * del;
+    // dS_n = a (dl_n inner + c1 (G_n - mean G)),  dl_n = 1/B (+ q2 u_n)
+    A = a * C1;
+    X = a * q2 * inner;
+    Cc = a * (INV_B * inner - C1 * sg * INV_B);
+    Pu = a * C1;
+}
+
+template <int D, int BS, int ORDER>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const uint32_t* __restrict__ mask, const float* __restrict__ lse,
+                     const float* __restrict__ delta, float* __restrict__ dq, int L, int nblk, int words, int gate,
+                     unsigned* status) {
+    using C = DqCfg<D>;
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr float INV_B = 1.0f / (float)BS;
+    constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
+    constexpr int BPT = C::NK / BS;  // blocks per key tile
+    constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, G = dO V^T
+    constexpr uint32_t IDESC_Q = tc::idesc_bf16(128, D, true);     // dQ += dS K, K MN-major
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = tc::smem_addr(smem);
+    auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+    const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NSK, B_VFULL = 1 + 2 * C::NSK,
+              B_VEMPTY = B_VFULL + C::NSV, B_SFULL = B_VEMPTY + C::NSV, B_DSREADY = B_SFULL + 2,
+              B_GFULL = B_DSREADY + 2, B_GFREE = B_GFULL + 1, B_DQFULL = B_GFREE + 1, B_DONE = B_DQFULL + 1;
+    uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int bh = blockIdx.y;
+    const int q0 = blockIdx.x * 128;
+    const int NT = L / C::NK;
+    bool aborted = false;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar(B_QFULL), 1);
+        for (int s = 0; s < C::NSK; ++s) {
+            tc::mbar_init(bar(B_KFULL + s), 1);
+            tc::mbar_init(bar(B_KEMPTY + s), 1);
+        }
+        for (int s = 0; s < C::NSV; ++s) {
+            tc::mbar_init(bar(B_VFULL + s), 1);
+            tc::mbar_init(bar(B_VEMPTY + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar(B_SFULL + b), 1);
+            tc::mbar_init(bar(B_DSREADY + b), 128);
+        }
+        tc::mbar_init(bar(B_GFULL), 1);
+        tc::mbar_init(bar(B_GFREE), 128);
+        tc::mbar_init(bar(B_DQFULL), 1);
+        tc::mbar_init(bar(B_DONE), 1);
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch(&tm_q);
+            tc::tma_prefetch(&tm_k);
+            tc::tma_prefetch(&tm_v);
+            tc::tma_prefetch(&tm_do);
+            const int row0 = bh * L + q0;
+            tc::mbar_expect_tx(bar(B_QFULL), 2 * C::TILE_BYTES);
+            for (int b = 0; b < C::NBOX; ++b) {
+                tc::tma_load_2d(sbase + C::Q_OFF + b * C::BOX_BYTES, &tm_q, bar(B_QFULL), b * 64, row0);
+                tc::tma_load_2d(sbase + C::DO_OFF + b * C::BOX_BYTES, &tm_do, bar(B_QFULL), b * 64, row0);
+            }
+            int lastK = -1, lastV = -1;
+            for (int j = 0; j < NT; ++j) {
+                const int sk = j % C::NSK, uk = j / C::NSK, sv = j % C::NSV, uv = j / C::NSV;
+                if (uk > 0 && !tc::mbar_wait(bar(B_KEMPTY + sk), (uk - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_KFULL + sk), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::K_OFF + sk * C::TILE_BYTES + b * C::BOX_BYTES, &tm_k, bar(B_KFULL + sk),
+                                    b * 64, bh * L + j * C::NK);
+                lastK = j;
+                if (uv > 0 && !tc::mbar_wait(bar(B_VEMPTY + sv), (uv - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_VFULL + sv), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::V_OFF + sv * C::TILE_BYTES + b * C::BOX_BYTES, &tm_v, bar(B_VFULL + sv),
+                                    b * 64, bh * L + j * C::NK);
+                lastV = j;
+            }
+            if (aborted) {
+                // let every copy already issued land before the CTA exits
+                bool a2 = false;
+                tc::mbar_wait(bar(B_QFULL), 0, a2, status, kWaitLimitCycles);
+                for (int j = (lastK - C::NSK + 1 > 0 ? lastK - C::NSK + 1 : 0); j <= lastK; ++j) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_KFULL + j % C::NSK), (j / C::NSK) & 1, a2, status, kWaitLimitCycles);
+                }
+                for (int j = (lastV - C::NSV + 1 > 0 ? lastV - C::NSV + 1 : 0); j <= lastV; ++j) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_VFULL + j % C::NSV), (j / C::NSV) & 1, a2, status, kWaitLimitCycles);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint64_t qdesc = tc::sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+            const uint64_t dodesc = tc::sdesc_sw128(sbase + C::DO_OFF, 16, 1024);
+            const uint64_t kdesc0 = tc::sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+            const uint64_t kmn0 = tc::sdesc_sw128(sbase + C::K_OFF, C::BOX_BYTES, 1024);  // K as MN-major B
+            const uint64_t vdesc0 = tc::sdesc_sw128(sbase + C::V_OFF, 16, 1024);
+            constexpr uint64_t kTileStep = C::TILE_BYTES >> 4;
+            // D[dcol] = A (Q or dO) x B^T (K or V tile), K-dim = d
+            auto issue_kd = [&](uint32_t dcol, uint64_t adesc, uint64_t bdesc) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+                    tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_S, kk > 0);
+                }
+            };
+            // dQ += dS (TMEM, buffer b) x K_j (MN-major), K-dim = 128 keys
+            auto issue_dq = [&](int b, int sk, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < C::NK / 16; ++kk)
+                    tc::mma_ts(tmem + C::DQ_COL, tmem + (uint32_t)(b * 128) + kk * 8,
+                               kmn0 + sk * kTileStep + (uint64_t)((kk * 16 * 128) >> 4), IDESC_Q,
+                               (first && kk == 0) ? 0u : 1u);
+            };
+            bool ok = tc::mbar_wait(bar(B_QFULL), 0, aborted, status, kWaitLimitCycles);
+            // prologue: S_0, G_0, S_1
+            ok = ok && tc::mbar_wait(bar(B_KFULL + 0), 0, aborted, status, kWaitLimitCycles);
+            if (ok) {
+                issue_kd(0, qdesc, kdesc0);
+                tc::mma_commit(bar(B_SFULL + 0));
+            }
+            ok = ok && tc::mbar_wait(bar(B_VFULL + 0), 0, aborted, status, kWaitLimitCycles);
+            if (ok) {
+                issue_kd(C::G_COL, dodesc, vdesc0);
+                tc::mma_commit(bar(B_GFULL));
+                tc::mma_commit(bar(B_VEMPTY + 0));
+            }
+            if (ok && NT > 1) {
+                ok = tc::mbar_wait(bar(B_KFULL + 1), 0, aborted, status, kWaitLimitCycles);
+                if (ok) {
+                    issue_kd(128, qdesc, kdesc0 + 1 * kTileStep);
+                    tc::mma_commit(bar(B_SFULL + 1));
+                }
+            }
+            for (int j = 0; ok && j < NT; ++j) {
+                const int b = j & 1;
+                // the softmax of tile j has written dS_j and read G_j
+                if (!tc::mbar_wait(bar(B_DSREADY + b), (j >> 1) & 1, aborted, status, kWaitLimitCycles)) break;
+                if (!tc::mbar_wait(bar(B_GFREE), j & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                if (j + 1 < NT) {
+                    const int sv = (j + 1) % C::NSV, uv = (j + 1) / C::NSV;
+                    if (!tc::mbar_wait(bar(B_VFULL + sv), uv & 1, aborted, status, kWaitLimitCycles)) break;
+                    issue_kd(C::G_COL, dodesc, vdesc0 + sv * kTileStep);
+                    tc::mma_commit(bar(B_GFULL));
+                    tc::mma_commit(bar(B_VEMPTY + sv));
+                }
+                issue_dq(b, j % C::NSK, j == 0);
+                tc::mma_commit(bar(B_KEMPTY + j % C::NSK));
+                if (j + 2 < NT) {
+                    const int sk = (j + 2) % C::NSK, uk = (j + 2) / C::NSK;
+                    if (!tc::mbar_wait(bar(B_KFULL + sk), uk & 1, aborted, status, kWaitLimitCycles)) break;
+                    issue_kd((uint32_t)(b * 128), qdesc, kdesc0 + sk * kTileStep);
+                    tc::mma_commit(bar(B_SFULL + b));
+                }
+            }
+            if (!aborted) tc::mma_commit(bar(B_DQFULL));
+            // every MMA issued by this thread has completed before TMEM is freed
+            tc::mma_commit(bar(B_DONE));
+            bool a2 = false;
+            tc::mbar_wait(bar(B_DONE), 0, a2, status, kWaitLimitCycles);
+        }
+    } else {
+        // ------------------------------------------------------------- softmax
+        const int quarter = warp % 4;           // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;      // row inside the M tile = TMEM lane
+        const int qrow = q0 + r;
+        const bool valid = qrow < L;
+        const int qt = (valid ? qrow : L - 1) / BS;  // query tile (selection row)
+        const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
+        const float lse2 = (valid ? __ldg(lse + (size_t)bh * L + qrow) : 0.f) * LOG2E;  // log2 units
+        const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
+        const float ln_b = logf((float)BS);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t g_addr = lane_base + C::G_COL;
+        for (int j = 0; j < NT; ++j) {
+            const int b = j & 1;
+            if (!tc::mbar_wait_warp(bar(B_SFULL + b), (j >> 1) & 1, aborted, status, kWaitLimitCycles)) break;
+            if (!tc::mbar_wait_warp(bar(B_GFULL), j & 1, aborted, status, kWaitLimitCycles)) break;
+            tc::fence_after_sync();
+            const uint32_t s_addr = lane_base + (uint32_t)(b * 128);
+            bool sel[BPT];
+            const uint32_t mw = __ldg(mrow + ((j * BPT) >> 5));
+#pragma unroll
+            for (int bb = 0; bb < BPT; ++bb) sel[bb] = (mw >> ((j * BPT + bb) & 31)) & 1u;
+            RowBlockSums<BPT, BS> rs;
+            row_block_sums<BPT, BS>(s_addr, g_addr, rs);
+            float sb[BPT], A[BPT], X[BPT], Cc[BPT];
+#pragma unroll
+            for (int bb = 0; bb < BPT; ++bb) {
+                float a, Pu;
+                block_coefs<BS, ORDER>(rs.x0[bb], rs.s1[bb], rs.s2[bb], rs.sg[bb], rs.sgd[bb], lse2, del, gate, ln_b,
+                                       sb[bb], a, A[bb], X[bb], Cc[bb], Pu);
+            }
+            // dS (bf16) over the first half of the S buffer's columns, 32 keys per store; the
+            // columns written hold keys already read (key 2e and 2e+1 go to column e)
+#pragma unroll
+            for (int c = 0; c < C::NK / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t xs[16], gs[16];
+                    tc::tmem_ld16(s_addr + c * 32 + hh * 16, xs);
+                    tc::tmem_ld16(g_addr + c * 32 + hh * 16, gs);
+                    tc::tmem_wait_ld();
+                    const int bb = (c * 32 + hh * 16) / BS;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float ds[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const float xv = __uint_as_float(xs[2 * e + h]), gv = __uint_as_float(gs[2 * e + h]);
+                            if (sel[bb]) {
+                                ds[h] = tc::ex2(fmaf(xv, LOG2E, -lse2)) * (gv - del);
+                            } else {
+                                ds[h] = fmaf(A[bb], gv, fmaf(X[bb], xv - sb[bb], Cc[bb]));
+                            }
+                        }
+                        pk[hh * 8 + e] = tc::pack_bf16x2(ds[0], ds[1]);
+                    }
+                }
+                tc::tmem_st16(s_addr + c * 16, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_GFREE));
+            tc::mbar_arrive(bar(B_DSREADY + b));
+        }
+        // epilogue: dq row (fp32) to global
+        if (tc::mbar_wait_warp(bar(B_DQFULL), 0, aborted, status, kWaitLimitCycles)) {
+            tc::fence_after_sync();
+            float* drow = dq + ((size_t)bh * L + (valid ? qrow : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t raw[32];
+                tc::tmem_ld32(lane_base + C::DQ_COL + c * 32, raw);
+                tc::tmem_wait_ld();
+                if (valid) {
+                    float4* dst = reinterpret_cast<float4*>(drow + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(raw[4 * e]), __uint_as_float(raw[4 * e + 1]),
+                                             __uint_as_float(raw[4 * e + 2]), __uint_as_float(raw[4 * e + 3]));
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_dkdv_tc_kernel (key-major): one tile of 128 keys of one (batch, head) per
+// CTA, visiting every query tile of 128 rows.  S = Q K^T and G = dO V^T are
+// computed with the queries as TMEM lanes (the same orientation as the dq
+// kernel), so every reduction over a block's keys stays inside one thread.  The
+// softmax threads write P and dS (bf16) as rows of query t into shared memory
+// in the 128-byte-swizzled layout of a TMA tile; read with the keys as the
+// contiguous dimension, that is the MN-major A operand of
+//   dV += P^T dO,   dK += dS^T Q     (M = the 128 keys, N = d, K-dim = queries)
+// with dO and Q as MN-major B operands.  TMEM: S | G | dV | dK.
+//   warp 0      TMA producer: K and V once; Q and dO tiles through NSQ stages
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2-5   softmax: the four lane quarters (query rows), then the
+//               epilogue of dK and dV (key rows)
+// MMA order after the softmax of query tile i has handed over P_i and dS_i:
+//   NSQ = 2: S_{i+1}, G_{i+1}, dK_i, dV_i       NSQ = 1: dK_i, dV_i, S_{i+1}, G_{i+1}
+// (one stage of Q and dO at d = 128: its tiles are free only after dK_i, dV_i).
+// ---------------------------------------------------------------------------
+template <int D>
+struct DkvCfg {
+    static constexpr int NQ = 128;                     // query rows per tile
+    static constexpr int NBOX = D / 64;
+    static constexpr uint32_t BOX_BYTES = 128 * 128;
+    static constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;  // 128 rows x d bf16
+    static constexpr uint32_t PT_BYTES = 2 * BOX_BYTES;       // 128 queries x 128 keys bf16
+    static constexpr int NSQ = (D == 128) ? 1 : 2;      // stages of Q and dO
+    static constexpr uint32_t K_OFF = 0;
+    static constexpr uint32_t V_OFF = K_OFF + TILE_BYTES;
+    static constexpr uint32_t Q_OFF = V_OFF + TILE_BYTES;
+    static constexpr uint32_t DO_OFF = Q_OFF + NSQ * TILE_BYTES;
+    static constexpr uint32_t P_OFF = DO_OFF + NSQ * TILE_BYTES;
+    static constexpr uint32_t DS_OFF = P_OFF + PT_BYTES;
+    static constexpr uint32_t BAR_OFF = DS_OFF + PT_BYTES;
+    // KVFULL; QFULL, QEMPTY, DOFULL, DOEMPTY per stage; SFULL; PREADY; PFREE; DKVFULL; DONE
+    static constexpr uint32_t NBAR = 1 + 4 * NSQ + 5;
+    static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+    static constexpr uint32_t G_COL = 128, DV_COL = 256, DK_COL = 256 + D;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// 16 bytes (8 bf16) at chunk c of row t of a 128-byte-swizzled tile (64 columns per box)
+__device__ __forceinline__ void st_swz16(uint8_t* tile, int t, int col8, uint4 v) {
+    const int box = col8 >> 3, c = col8 & 7;
+    *reinterpret_cast<uint4*>(tile + box * (128 * 128) + t * 128 + ((c ^ (t & 7)) << 4)) = v;
+}
+
+template <int D, int BS, int ORDER>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const uint32_t* __restrict__ mask, const float* __restrict__ lse,
+                       const float* __restrict__ delta, float* __restrict__ dk, float* __restrict__ dv, int L,
+                       int nblk, int words, int gate, unsigned* status) {
+    using C = DkvCfg<D>;
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr float INV_B = 1.0f / (float)BS;
+    constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
+    constexpr int BPT = 128 / BS;  // blocks per key tile
+    constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
+    // M = 128 keys, N = d, A (P or dS) and B (dO or Q) both MN-major
+    constexpr uint32_t IDESC_KV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                  ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = tc::smem_addr(smem);
+    auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+    const int B_KVFULL = 0, B_QFULL = 1, B_QEMPTY = 1 + C::NSQ, B_DOFULL = 1 + 2 * C::NSQ,
+              B_DOEMPTY = 1 + 3 * C::NSQ, B_SFULL = 1 + 4 * C::NSQ, B_PREADY = B_SFULL + 1,
+              B_PFREE = B_PREADY + 1, B_DKVFULL = B_PFREE + 1, B_DONE = B_DKVFULL + 1;
+    uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int bh = blockIdx.y;
+    const int k0 = blockIdx.x * 128;  // first key of this tile
+    const int NQT = (L + C::NQ - 1) / C::NQ;
+    bool aborted = false;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar(B_KVFULL), 1);
+        for (int s = 0; s < C::NSQ; ++s) {
+            tc::mbar_init(bar(B_QFULL + s), 1);
+            tc::mbar_init(bar(B_QEMPTY + s), 1);
+            tc::mbar_init(bar(B_DOFULL + s), 1);
+            tc::mbar_init(bar(B_DOEMPTY + s), 1);
+        }
+        tc::mbar_init(bar(B_SFULL), 1);
+        tc::mbar_init(bar(B_PREADY), 128);
+        tc::mbar_init(bar(B_PFREE), 1);
+        tc::mbar_init(bar(B_DKVFULL), 1);
+        tc::mbar_init(bar(B_DONE), 1);
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch(&tm_q);
+            tc::tma_prefetch(&tm_k);
+            tc::tma_prefetch(&tm_v);
+            tc::tma_prefetch(&tm_do);
+            tc::mbar_expect_tx(bar(B_KVFULL), 2 * C::TILE_BYTES);
+            for (int b = 0; b < C::NBOX; ++b) {
+                tc::tma_load_2d(sbase + C::K_OFF + b * C::BOX_BYTES, &tm_k, bar(B_KVFULL), b * 64, bh * L + k0);
+                tc::tma_load_2d(sbase + C::V_OFF + b * C::BOX_BYTES, &tm_v, bar(B_KVFULL), b * 64, bh * L + k0);
+            }
+            int lastQ = -1, lastO = -1;
+            for (int i = 0; i < NQT; ++i) {
+                const int st = i % C::NSQ, u = i / C::NSQ;
+                const int row = bh * L + i * C::NQ;
+                if (u > 0 && !tc::mbar_wait(bar(B_QEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::mbar_expect_tx(bar(B_QFULL + st), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::Q_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q,
+                                    bar(B_QFULL + st), b * 64, row);
+                lastQ = i;
+                if (u > 0 && !tc::mbar_wait(bar(B_DOEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_DOFULL + st), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::DO_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_do,
+                                    bar(B_DOFULL + st), b * 64, row);
+                lastO = i;
+            }
+            if (aborted) {
+                bool a2 = false;
+                tc::mbar_wait(bar(B_KVFULL), 0, a2, status, kWaitLimitCycles);
+                for (int i = (lastQ - C::NSQ + 1 > 0 ? lastQ - C::NSQ + 1 : 0); i <= lastQ; ++i) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_QFULL + i % C::NSQ), (i / C::NSQ) & 1, a2, status, kWaitLimitCycles);
+                }
+                for (int i = (lastO - C::NSQ + 1 > 0 ? lastO - C::NSQ + 1 : 0); i <= lastO; ++i) {
+                    a2 = false;
+                    tc::mbar_wait(bar(B_DOFULL + i % C::NSQ), (i / C::NSQ) & 1, a2, status, kWaitLimitCycles);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint64_t kdesc = tc::sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+            const uint64_t vdesc = tc::sdesc_sw128(sbase + C::V_OFF, 16, 1024);
+            const uint64_t qdesc0 = tc::sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+            const uint64_t dodesc0 = tc::sdesc_sw128(sbase + C::DO_OFF, 16, 1024);
+            const uint64_t qmn0 = tc::sdesc_sw128(sbase + C::Q_OFF, C::BOX_BYTES, 1024);   // Q as MN-major B
+            const uint64_t domn0 = tc::sdesc_sw128(sbase + C::DO_OFF, C::BOX_BYTES, 1024); // dO as MN-major B
+            const uint64_t pmn = tc::sdesc_sw128(sbase + C::P_OFF, C::BOX_BYTES, 1024);    // P as MN-major A
+            const uint64_t dsmn = tc::sdesc_sw128(sbase + C::DS_OFF, C::BOX_BYTES, 1024);  // dS as MN-major A
+            constexpr uint64_t kTileStep = C::TILE_BYTES >> 4;
+            auto issue_sg = [&](int st) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+                    tc::mma_ss(tmem, qdesc0 + st * kTileStep + off, kdesc + off, IDESC_S, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+                    tc::mma_ss(tmem + C::G_COL, dodesc0 + st * kTileStep + off, vdesc + off, IDESC_S, kk > 0);
+                }
+            };
+            // D[dcol] (+)= A^T-tile (keys x queries, MN-major) x B-tile (queries x d, MN-major); K-dim = 128 queries
+            auto issue_kv = [&](uint32_t dcol, uint64_t adesc, uint64_t bdesc, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < C::NQ / 16; ++kk) {
+                    const uint64_t off = (uint64_t)((kk * 16 * 128) >> 4);  // 16 query rows further
+                    tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_KV, (first && kk == 0) ? 0u : 1u);
+                }
+            };
+            bool ok = tc::mbar_wait(bar(B_KVFULL), 0, aborted, status, kWaitLimitCycles);
+            ok = ok && tc::mbar_wait(bar(B_QFULL + 0), 0, aborted, status, kWaitLimitCycles);
+            ok = ok && tc::mbar_wait(bar(B_DOFULL + 0), 0, aborted, status, kWaitLimitCycles);
+            if (ok) {
+                issue_sg(0);
+                tc::mma_commit(bar(B_SFULL));
+            }
+            for (int i = 0; ok && i < NQT; ++i) {
+                const int st = i % C::NSQ;
+                const bool more = i + 1 < NQT;
+                const int st1 = (i + 1) % C::NSQ, u1 = (i + 1) / C::NSQ;
+                // the softmax has written P_i and dS_i (and read S_i and G_i)
+                if (!tc::mbar_wait(bar(B_PREADY), i & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                if (C::NSQ >= 2 && more) {
+                    if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
+                    if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
+                    issue_sg(st1);
+                    tc::mma_commit(bar(B_SFULL));
+                }
+                issue_kv(C::DK_COL, dsmn, qmn0 + st * kTileStep, i == 0);
+                tc::mma_commit(bar(B_QEMPTY + st));
+                issue_kv(C::DV_COL, pmn, domn0 + st * kTileStep, i == 0);
+                tc::mma_commit(bar(B_DOEMPTY + st));
+                tc::mma_commit(bar(B_PFREE));
+                if (C::NSQ == 1 && more) {
+                    if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
+                    if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
+                    issue_sg(st1);
+                    tc::mma_commit(bar(B_SFULL));
+                }
+            }
+            if (!aborted) tc::mma_commit(bar(B_DKVFULL));
+            tc::mma_commit(bar(B_DONE));
+            bool a2 = false;
+            tc::mbar_wait(bar(B_DONE), 0, a2, status, kWaitLimitCycles);
+        }
+    } else {
+        // ------------------------------------------------------------- softmax
+        const int quarter = warp % 4;
+        const int r = quarter * 32 + lane;  // TMEM lane: query row of the tile, then key row in the epilogue
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float ln_b = logf((float)BS);
+        const int jb0 = k0 / BS;  // first block of this key tile
+        uint8_t* ptile = smem + C::P_OFF;
+        uint8_t* dstile = smem + C::DS_OFF;
+        for (int i = 0; i < NQT; ++i) {
+            const int qrow = i * C::NQ + r;
+            const bool valid = qrow < L;
+            const int qt = (valid ? qrow : L - 1) / BS;
+            const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
+            const float lse2 = (valid ? __ldg(lse + (size_t)bh * L + qrow) : 0.f) * LOG2E;
+            const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
+            bool sel[BPT];
+#pragma unroll
+            for (int bb = 0; bb < BPT; ++bb) sel[bb] = (__ldg(mrow + ((jb0 + bb) >> 5)) >> ((jb0 + bb) & 31)) & 1u;
+            if (!tc::mbar_wait_warp(bar(B_SFULL), i & 1, aborted, status, kWaitLimitCycles)) break;
+            tc::fence_after_sync();
+            RowBlockSums<BPT, BS> rs;
+            row_block_sums<BPT, BS>(lane_base, lane_base + C::G_COL, rs);
+            float sb[BPT], aa[BPT], A[BPT], X[BPT], Cc[BPT], Pu[BPT];
+#pragma unroll
+            for (int bb = 0; bb < BPT; ++bb)
+                block_coefs<BS, ORDER>(rs.x0[bb], rs.s1[bb], rs.s2[bb], rs.sg[bb], rs.sgd[bb], lse2, del, gate, ln_b,
+                                       sb[bb], aa[bb], A[bb], X[bb], Cc[bb], Pu[bb]);
+            // the previous tile's dK and dV products have read P and dS
+            if (i > 0 && !tc::mbar_wait_warp(bar(B_PFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) break;
+            // P and dS rows (bf16) into shared memory, 16 keys at a time; rows past L are zero
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t xs[16], gs[16];
+                tc::tmem_ld16(lane_base + c * 16, xs);
+                tc::tmem_ld16(lane_base + C::G_COL + c * 16, gs);
+                tc::tmem_wait_ld();
+                const int bb = (c * 16) / BS;
+                uint32_t pp[8], dd[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float pv[2], dsv[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float xv = __uint_as_float(xs[2 * e + h]), gv = __uint_as_float(gs[2 * e + h]);
+                        if (sel[bb]) {
+                            pv[h] = tc::ex2(fmaf(xv, LOG2E, -lse2));
+                            dsv[h] = pv[h] * (gv - del);
+                        } else {
+                            const float u = xv - sb[bb];
+                            pv[h] = fmaf(Pu[bb], u, aa[bb]);
+                            dsv[h] = fmaf(A[bb], gv, fmaf(X[bb], u, Cc[bb]));
+                        }
+                        if (!valid) pv[h] = dsv[h] = 0.f;
+                    }
+                    pp[e] = tc::pack_bf16x2(pv[0], pv[1]);
+                    dd[e] = tc::pack_bf16x2(dsv[0], dsv[1]);
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 2; ++q4) {
+                    st_swz16(ptile, r, c * 2 + q4, make_uint4(pp[4 * q4], pp[4 * q4 + 1], pp[4 * q4 + 2], pp[4 * q4 + 3]));
+                    st_swz16(dstile, r, c * 2 + q4, make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]));
+                }
+            }
+            // generic-proxy stores -> the tensor core (async proxy) reads them
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_PREADY));
+        }
+        // epilogue: dK and dV rows (TMEM lane = key) to global
+        if (tc::mbar_wait_warp(bar(B_DKVFULL), 0, aborted, status, kWaitLimitCycles)) {
+            tc::fence_after_sync();
+            const int key = k0 + r;
+            float* krow = dk + ((size_t)bh * L + key) * D;
+            float* vrow = dv + ((size_t)bh * L + key) * D;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float* dst_row = part == 0 ? krow : vrow;
+                const uint32_t col = part == 0 ? C::DK_COL : C::DV_COL;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t raw[32];
+                    tc::tmem_ld32(lane_base + col + c * 32, raw);
+                    tc::tmem_wait_ld();
+                    float4* dst = reinterpret_cast<float4*>(dst_row + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(raw[4 * e]), __uint_as_float(raw[4 * e + 1]),
+                                             __uint_as_float(raw[4 * e + 2]), __uint_as_float(raw[4 * e + 3]));
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace bwdtc
+}  // namespace pisa

@@ -25,6 +25,7 @@
 #include "attn_stc.cuh"
 #include "route.cuh"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "selftest.cuh"
 
 using pisa::bf16;
@@ -243,7 +244,7 @@ pisa_status run_route_bias(const void* k, const void* v, const float* kbar, cons
 
 pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pisa_stats_t* st,
                            const uint32_t* mask, void* out, const Dims& g, int order, int gate,
-                           cudaStream_t s, const float* wmat = nullptr) {
+                           cudaStream_t s, const float* wmat = nullptr, float* lse = nullptr) {
     return dispatch(st->dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
@@ -255,7 +256,7 @@ pisa_status run_attn_stats(const void* q, const void* k, const void* v, const pi
         dim3 grid((unsigned)(g.nblk * parts), (unsigned)g.BH);
         kern<<<grid, 256, smem, s>>>((const T*)q, (const T*)k, (const T*)v, st->kbar, st->vsum,
                                      (const T*)st->hstat, (const T*)st->cov, mask, (T*)out, (int)g.L,
-                                     (int)g.nblk, (int)g.words, order, gate, logf((float)g.B), wmat);
+                                     (int)g.nblk, (int)g.words, order, gate, logf((float)g.B), wmat, lse);
         return launch_check("attn_stats_kernel");
     });
 }
@@ -376,7 +377,7 @@ pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
 // backward pass: workspace layout and launches
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-    size_t kbar, bias, mask, mstat, dinv, delta, total;
+    size_t kbar, bias, mask, mstat, dinv, delta, lse, total;
 };
 
 BwdLayout bwd_layout(const Dims& g) {
@@ -394,8 +395,112 @@ BwdLayout bwd_layout(const Dims& g) {
     o += align_up(sizeof(float) * g.BH * g.L);
     w.delta = o;
     o += align_up(sizeof(float) * g.BH * g.L);
+    w.lse = o;
+    o += align_up(sizeof(float) * g.BH * g.L);
     w.total = o;
     return w;
+}
+
+// The backward on tcgen05 (bf16, the tensor-core shapes): delta (and, without the forward's
+// lse, the row statistics turned into lse), then the dq and dk/dv kernels.
+pisa_status run_backward_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                            const uint32_t* mask, const Dims& g, int order, int gate, const float* lse_in,
+                            float* mst, float* dinv, float* del, float* lse_ws, float* dq, float* dk, float* dv,
+                            cudaStream_t s) {
+    unsigned int* status = device_status_ptr();
+    if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
+    const long rows = g.BH * g.L;
+    const float* lse = lse_in;
+    if (!lse_in) {
+        // m_t, 1/D_t and delta_t from the row-statistics kernel, then lse = m - ln(1/D)
+        pisa_status r = dispatch(PISA_BF16, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
+            using T = decltype(t);
+            constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
+            using C = pisa::bwd::Cfg<T, D, BS>;
+            auto k1 = pisa::bwd::bwd_rowstat_kernel<T, D, BS>;
+            pisa_status rr = set_smem(k1, C::ROWSTAT_SMEM);
+            if (rr != PISA_OK) return rr;
+            const dim3 gq((unsigned)(g.L / pisa::bwd::kQT), (unsigned)g.BH);
+            k1<<<gq, 128, C::ROWSTAT_SMEM, s>>>((const T*)q, (const T*)k, (const T*)o, (const T*)dO, mask, (int)g.L,
+                                                (int)g.nblk, (int)g.words, order, gate, mst, dinv, del);
+            return launch_check("bwd_rowstat_kernel");
+        });
+        if (r != PISA_OK) return r;
+        pisa::bwdtc::bwd_lse_kernel<<<(unsigned)((rows + 255) / 256 < 4096 ? (rows + 255) / 256 : 4096), 256, 0, s>>>(
+            mst, dinv, rows, lse_ws);
+        r = launch_check("bwd_lse_kernel");
+        if (r != PISA_OK) return r;
+        lse = lse_ws;
+    } else {
+        const unsigned nb = (unsigned)((rows + 7) / 8);
+        if (g.d == 64)
+            pisa::bwdtc::bwd_delta_kernel<64><<<nb, 256, 0, s>>>((const bf16*)o, (const bf16*)dO, rows, del);
+        else
+            pisa::bwdtc::bwd_delta_kernel<128><<<nb, 256, 0, s>>>((const bf16*)o, (const bf16*)dO, rows, del);
+        pisa_status r = launch_check("bwd_delta_kernel");
+        if (r != PISA_OK) return r;
+    }
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess || !fn)
+            return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+        encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    }
+    CUtensorMap maps[4];
+    const void* ptrs[4] = {q, k, v, dO};
+    for (int t = 0; t < 4; ++t) {
+        cuuint64_t gdim[2] = {(cuuint64_t)g.d, (cuuint64_t)rows};
+        cuuint64_t gstride[1] = {(cuuint64_t)g.d * 2};
+        cuuint32_t box[2] = {64, 128};
+        cuuint32_t estride[2] = {1, 1};
+        if (encode(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[t]), gdim, gstride, box,
+                   estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the backward kernels");
+    }
+    const dim3 grid((unsigned)(g.L / 128), (unsigned)g.BH);
+    cudaError_t e = cudaSuccess;
+    bool found = false;
+#define PISA_BWD_TC(DD, BB, OO)                                                                                   \
+    if (!found && g.d == DD && g.B == BB && order == OO) {                                                        \
+        found = true;                                                                                             \
+        auto kq = pisa::bwdtc::bwd_dq_tc_kernel<DD, BB, OO>;                                                      \
+        auto kk = pisa::bwdtc::bwd_dkdv_tc_kernel<DD, BB, OO>;                                                    \
+        e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pisa::bwdtc::DqCfg<DD>::SMEM); \
+        if (e == cudaSuccess)                                                                                     \
+            e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize,                             \
+                                     (int)pisa::bwdtc::DkvCfg<DD>::SMEM);                                         \
+        if (e == cudaSuccess) {                                                                                   \
+            kq<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DqCfg<DD>::SMEM, s>>>(                                 \
+                maps[0], maps[1], maps[2], maps[3], mask, lse, del, dq, (int)g.L, (int)g.nblk, (int)g.words, gate,  \
+                status);                                                                                          \
+            e = cudaGetLastError();                                                                               \
+        }                                                                                                         \
+        if (e == cudaSuccess) {                                                                                   \
+            kk<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DkvCfg<DD>::SMEM, s>>>(                                \
+                maps[0], maps[1], maps[2], maps[3], mask, lse, del, dk, dv, (int)g.L, (int)g.nblk, (int)g.words,    \
+                gate, status);                                                                                    \
+            e = cudaGetLastError();                                                                               \
+        }                                                                                                         \
+    }
+    PISA_BWD_TC(64, 64, 0)
+    PISA_BWD_TC(64, 64, 1)
+    PISA_BWD_TC(64, 64, 2)
+    PISA_BWD_TC(64, 128, 0)
+    PISA_BWD_TC(64, 128, 1)
+    PISA_BWD_TC(64, 128, 2)
+    PISA_BWD_TC(128, 64, 0)
+    PISA_BWD_TC(128, 64, 1)
+    PISA_BWD_TC(128, 64, 2)
+    PISA_BWD_TC(128, 128, 0)
+    PISA_BWD_TC(128, 128, 1)
+    PISA_BWD_TC(128, 128, 2)
+#undef PISA_BWD_TC
+    if (!found) return fail(PISA_ERR_UNSUPPORTED, "no tensor-core backward kernel for this d/B/order");
+    if (e != cudaSuccess) return cuda_fail(e, "backward tensor-core kernels");
+    return PISA_OK;
 }
 
 pisa_status run_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -574,9 +679,14 @@ size_t pisa_workspace_bytes(int batch, int heads, int L, int d, int B, int K, in
     return pisa_workspace_bytes_ex(batch, heads, L, d, B, K, order, dtype, PISA_PATH_AUTO);
 }
 
-pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
-                              pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
-                              void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// pisa_attention_ex with an optional per-row log-denominator output (lse may be null).
+pisa_status attention_impl(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                           pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
+                           float* lse, void* workspace, size_t ws_bytes, void* stream) {
     Dims g;
     pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
     if (r != PISA_OK) return r;
@@ -597,6 +707,9 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
     const bool route = (gate_w & PISA_FLAG_COV_ROUTE) != 0;
     if (path == PISA_PATH_HYBRID_TC && order == 2 && !pooled)
         return fail(PISA_ERR_UNSUPPORTED, "the hybrid's second order needs the pooled w (PISA_FLAG_POOLED_W)");
+    if (path == PISA_PATH_HYBRID_TC && lse)
+        return fail(PISA_ERR_UNSUPPORTED, "no log-denominator output on the hybrid path");
+    if (lse && (uintptr_t)lse % 4) return fail(PISA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
     if (path == PISA_PATH_STATS_TC && !stc_path_available(g, dtype, order, pooled))
         return fail(PISA_ERR_UNSUPPORTED,
                     "statistics-form tensor-core path needs bf16, d and B in {64, 128}, L %% 128 == 0 and order 1 "
@@ -672,15 +785,34 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
         return pisa::run_attn_tc(q, k, v, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B, (int)g.nblk,
-                                 (int)g.words, korder, gate, wmat, status, s, &g_last_error);
+                                 (int)g.words, korder, gate, wmat, status, s, &g_last_error, lse);
     }
     if (path == PISA_PATH_STATS_TC) {
         unsigned int* status = device_status_ptr();
         if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
         return pisa::run_attn_stc(q, k, v, st.hstat, st.kaug, st.vsum, mask, out, g.BH, (int)g.L, (int)g.d, (int)g.B,
-                                  (int)g.nblk, (int)g.words, korder, gate, wmat, status, s, &g_last_error);
+                                  (int)g.nblk, (int)g.words, korder, gate, wmat, status, s, &g_last_error, lse);
     }
-    return run_attn_stats(q, k, v, &st, mask, out, g, order, gate, s, wmat);
+    return run_attn_stats(q, k, v, &st, mask, out, g, order, gate, s, wmat, lse);
+}
+
+}  // namespace
+
+extern "C" {
+
+pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                              pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    return attention_impl(q, k, v, batch, heads, L, d, dtype, B, K, order, gate_w, path, out, nullptr, workspace,
+                          ws_bytes, stream);
+}
+
+pisa_status pisa_attention_lse(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                               pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
+                               float* lse, void* workspace, size_t ws_bytes, void* stream) {
+    if (!lse) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_lse: null lse");
+    return attention_impl(q, k, v, batch, heads, L, d, dtype, B, K, order, gate_w, path, out, lse, workspace,
+                          ws_bytes, stream);
 }
 
 pisa_status pisa_attention(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
@@ -697,10 +829,14 @@ size_t pisa_backward_workspace_bytes(int batch, int heads, int L, int d, int B, 
     return bwd_layout(g).total;
 }
 
-pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                                    int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
-                                    int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
-                                    void* stream) {
+}  // extern "C"
+
+namespace {
+
+pisa_status backward_impl(const void* q, const void* k, const void* v, const void* o, const void* dO, int batch,
+                          int heads, int L, int d, pisa_dtype dtype, int B, int K, int order, int flags,
+                          const float* lse, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                          void* stream) {
     Dims g;
     pisa_status r = check_dims(batch, heads, L, d, B, order, dtype, &g);
     if (r != PISA_OK) return r;
@@ -736,8 +872,33 @@ pisa_status pisa_attention_backward(const void* q, const void* k, const void* v,
     }
     r = run_select(q, kbar, g, dtype, K, nullptr, mask, s, rbias);
     if (r != PISA_OK) return r;
+    if (tc_path_available(g, dtype))
+        return run_backward_tc(q, k, v, o, dO, mask, g, order, flags & PISA_FLAG_GATE_W, lse, (float*)(ws + w.mstat),
+                               (float*)(ws + w.dinv), (float*)(ws + w.delta), (float*)(ws + w.lse), dq, dk, dv, s);
     return run_backward(q, k, v, o, dO, mask, g, dtype, order, flags & PISA_FLAG_GATE_W, (float*)(ws + w.mstat),
                         (float*)(ws + w.dinv), (float*)(ws + w.delta), dq, dk, dv, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                    int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
+                                    int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+    return backward_impl(q, k, v, o, dO, batch, heads, L, d, dtype, B, K, order, flags, nullptr, dq, dk, dv,
+                         workspace, ws_bytes, stream);
+}
+
+pisa_status pisa_attention_backward_lse(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                        const float* lse, int batch, int heads, int L, int d, pisa_dtype dtype, int B,
+                                        int K, int order, int flags, float* dq, float* dk, float* dv,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+    if (!lse) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward_lse: null lse");
+    if ((uintptr_t)lse % 4) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward_lse: lse must be 4-byte aligned");
+    return backward_impl(q, k, v, o, dO, batch, heads, L, d, dtype, B, K, order, flags, lse, dq, dk, dv, workspace,
+                         ws_bytes, stream);
 }
 
 pisa_status pisa_centroids(const void* k, int batch, int heads, int L, int d, pisa_dtype dtype, int B, float* kbar,

@@ -250,6 +250,18 @@ pisa_status pisa_attention_ex(const void* q, const void* k, const void* v, int b
                               pisa_path path, void* out, void* workspace, size_t ws_bytes,
                               void* stream);
 
+/* As pisa_attention_ex, plus the log of each row's denominator:
+ *   lse [BH, L] fp32 (device, 4-byte aligned): lse_t = ln D_t with D_t the
+ *   shared denominator of the PISA paper's section 3.2 "Formulation" (exact
+ *   keys e^{q.k} plus B e^{l_tj} per unselected block), i.e. m_t + ln sum e^{. - m_t}
+ *   for the kernel's running max m_t.  pisa_attention_backward_lse takes it, so
+ *   that the backward needs no pass of its own over the keys for m_t and D_t.
+ * Errors as pisa_attention_ex; INVALID_ARG for a null or misaligned lse;
+ * UNSUPPORTED on the hybrid path. */
+pisa_status pisa_attention_lse(const void* q, const void* k, const void* v, int batch, int heads, int L, int d,
+                               pisa_dtype dtype, int B, int K, int order, int gate_w, pisa_path path, void* out,
+                               float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* Allocation-free pisa_attention (the paper has no counterpart: this is an
  * interface for callers that may not allocate device memory, such as a plugin
  * whose host application owns the whole device memory pool, or a loop where
@@ -328,10 +340,12 @@ size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype 
  *   workspace      : ws_bytes >= pisa_backward_workspace_bytes(...) of device
  *                    memory, 256-byte aligned; on return it holds the centroids,
  *                    the selection mask and the per-row m, 1/D and delta.
- * Shapes as for pisa_attention plus batch * heads <= 65535.  bf16 inputs run
- * their tile products on the tensor cores (fp32 accumulation; P and dS are
- * rounded to bf16 as the operands of the dk, dv and dq products); fp32 inputs
- * run in fp32 throughout.
+ * Shapes as for pisa_attention plus batch * heads <= 65535.  bf16 inputs with
+ * d and B in {64, 128} and L % 128 == 0 run on tcgen05 tensor cores: a dq
+ * kernel (query-major) and a dk/dv kernel (key-major), fp32 accumulation in
+ * TMEM, P and dS rounded to bf16 as the operands of the dq, dk and dv
+ * products; other bf16 shapes use warp-level MMAs with the same roundings;
+ * fp32 inputs run in fp32 throughout.
  * Errors (before anything is enqueued): INVALID_ARG for a null or misaligned
  * pointer, unknown flag bits, K out of range or a small workspace;
  * UNSUPPORTED for the pooled w, batch * heads > 65535 and the shapes
@@ -340,6 +354,16 @@ pisa_status pisa_attention_backward(const void* q, const void* k, const void* v,
                                     int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,
                                     int flags, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
                                     void* stream);
+
+/* As pisa_attention_backward, given the forward's log-denominators lse [BH, L] fp32
+ * (pisa_attention_lse on the same inputs and options; device, 4-byte aligned):
+ * the backward then takes m and D from lse (P_n = e^{x_n - lse_t},
+ * a = e^{l_tj - lse_t}) instead of recomputing them.  Errors as
+ * pisa_attention_backward; INVALID_ARG for a null or misaligned lse. */
+pisa_status pisa_attention_backward_lse(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                        const float* lse, int batch, int heads, int L, int d, pisa_dtype dtype, int B,
+                                        int K, int order, int flags, float* dq, float* dk, float* dv,
+                                        void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace pisa_attention_backward needs (bytes); 0 for invalid arguments. */
 size_t pisa_backward_workspace_bytes(int batch, int heads, int L, int d, int B, int K, int order,

@@ -262,12 +262,15 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
 
 
-def parity_metrics(got, ref) -> dict:
+def parity_metrics(got, ref, row_floor=0.0) -> dict:
     """Comparison figures of a result ``got`` against the oracle's ``ref`` (same shape; the
     last axis is one output row):
       rel_l2   ||got - ref||_F / ||ref||_F over everything compared;
-      row_max  max over rows t of ||got_t - ref_t|| / ||ref_t|| (rows whose reference norm is
-               below 1e-6 of the rms row norm are skipped: their relative error means nothing);
+      row_max  max over rows t of ||got_t - ref_t|| / max(||ref_t||, row_floor rms_row), rms_row
+               the rms of the rows' reference norms (row_floor 0: the plain relative error; a
+               gradient row can cancel to nearly nothing, and its relative error then means
+               little, so gradients are compared with row_floor 1).  Rows whose reference norm
+               is below 1e-6 of rms_row are skipped when row_floor is 0;
       row_worst the index of that row in the flattened row list (-1 if none);
       elem_max max over elements of |got - ref| / (rms(ref) + |ref|), rms over everything
                compared, i.e. the smallest e with |got - ref| <= e rms(ref) + e |ref| everywhere;
@@ -282,8 +285,9 @@ def parity_metrics(got, ref) -> dict:
     rn = np.linalg.norm(r2, axis=1)
     dn = np.linalg.norm(diff, axis=1)
     rms_row = float(np.sqrt(np.mean(rn * rn))) if rn.size else 0.0
-    live = rn > 1e-6 * max(rms_row, 1e-300)
-    row_err = dn[live] / rn[live] if live.any() else np.zeros(0)
+    live = rn > 1e-6 * max(rms_row, 1e-300) if row_floor <= 0 else np.ones(rn.shape, bool)
+    den = np.maximum(rn, row_floor * rms_row)
+    row_err = dn[live] / den[live] if live.any() else np.zeros(0)
     rms = float(np.sqrt(np.mean(r2 * r2))) if r2.size else 0.0
     ratio = np.abs(diff) / (rms + np.abs(r2) + 1e-300)
     worst = int(np.argmax(row_err)) if row_err.size else -1

@@ -207,11 +207,11 @@ def test_backward_rejects_bad_arguments_before_launch(kw, status):
 
 def test_backward_workspace_size():
     f = pisa.lib().pisa_backward_workspace_bytes
-    # centroids + bias + mask + three per-row arrays, each rounded up to 256 bytes
+    # centroids + bias + mask + four per-row arrays (m, 1/D, delta, lse), each rounded up to 256 bytes
     BH, L, d, B = 2, 1024, 64, 64
     nblk = L // B
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    want = up(4 * BH * nblk * d) + up(4 * BH * nblk) + up(4 * BH * nblk * 1) + 3 * up(4 * BH * L)
+    want = up(4 * BH * nblk * d) + up(4 * BH * nblk) + up(4 * BH * nblk * 1) + 4 * up(4 * BH * L)
     assert f(1, BH, L, d, B, 4, 1, pisa.PISA_BF16) == want
     assert f(1, 1, 1000, 64, 64, 4, 1, pisa.PISA_BF16) == 0
     assert f(1, 1, 1024, 64, 64, 17, 1, pisa.PISA_BF16) == 0

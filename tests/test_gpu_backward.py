@@ -50,7 +50,7 @@ def gpu_backward(q, k, v, o, dO, B, K, order, gate, dt, route="centroid"):
 
 def check(got, want, dt):
     for name, g, w in zip(("dq", "dk", "dv"), got, want):
-        parity.check(g, w, dt, name)
+        parity.check(g, w, dt, name, grad=True)
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -153,7 +153,7 @@ def test_backward_full_size_sampled_rows_and_identities(name, heads):
     rows = [(int(rng.integers(BH)), int(t)) for t in rng.integers(0, L, 24)] + [(0, 0), (BH - 1, L - 1)]
     want = oracle.pisa_backward_dq_rows(q, k, v, dO, w.B, w.K, rows, w.order)
     got = np.stack([dq[b, t].cpu().numpy().astype(np.float64) for b, t in rows])
-    parity.check(got, want, dt, "dq rows")
+    parity.check(got, want, dt, "dq rows", grad=True)
     dk64, dv64 = dk.double(), dv.double()
     for b in range(BH):
         assert float(dk64[b].sum(0).norm()) <= 1e-2 * float(dk64[b].norm(dim=1).sum())
@@ -197,3 +197,33 @@ def test_autograd_four_dimensional_inputs_with_routing_and_order2():
     parity.check(out.detach().float().reshape(6, L, d).cpu().numpy(), want_o, dt, "o")
     got = [t.grad.float().reshape(6, L, d).cpu().numpy().astype(np.float64) for t in (qt, kt, vt)]
     check(got, oracle.pisa_backward(q, k, v, dO, B, K, 2, True, route_eps=pisa.ROUTE_EPS), dt)
+
+
+@pytest.mark.parametrize("path,dt", [("recompute_tc", "bf16"), ("stats_tc", "bf16"), ("stats", "bf16"),
+                                     ("stats", "f32")])
+def test_forward_lse_is_the_log_denominator(path, dt):
+    # pisa_attention_lse: ln D_t of the shared denominator, against the oracle's log D_t
+    L, d, B, K = 1024, 64, 64, 4
+    q, k, v = pisa_synth.random_qkv(1910, 2, L, d, scale=2.0, dtype=dt)
+    out, lse = pisa.pisa_attention_lse(dev(q, dt), dev(k, dt), dev(v, dt), B, K, 1, path=path)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    ref_o, ref_lse = oracle.pisa_attention(q, k, v, B, K, 1, want_lse=True)
+    parity.check(out.float().cpu().numpy(), ref_o, dt, "o")
+    tol = 1e-5 if dt == "f32" else 2e-3  # absolute, in natural-log units (a relative 2e-3 of D)
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= tol
+
+
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_backward_with_the_forwards_lse(d, B, order):
+    # the tensor-core backward given the forward's log-denominators: no row-statistics pass
+    dt, L = "bf16", 1024
+    q, k, v, dO = inputs(1950 + d + B + order, 2, L, d, dt, scale=3.0 if order == 2 else 2.0)
+    K = (L // B) // 4
+    qd, kd, vd, dOd = dev(q, dt), dev(k, dt), dev(v, dt), dev(dO, dt)
+    o, lse = pisa.pisa_attention_lse(qd, kd, vd, B, K, order)
+    grads = pisa.pisa_attention_backward(qd, kd, vd, o, dOd, B, K, order, lse=lse)
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    check([g.cpu().numpy().astype(np.float64) for g in grads], oracle.pisa_backward(q, k, v, dO, B, K, order), dt)

@@ -58,6 +58,39 @@ def rel_l2(a, b):
     return oracle.rel_l2(a, b)
 
 
+def rows_clear_of_the_gate(q, k, B, K):
+    """[BH, L] bool: rows none of whose unselected blocks has w_tj = 1/2 q_t^T C_j q_t (fp64,
+    from the oracle's statistics) within 2^-8 of 1/2 |q_t|^T |C_j| |q_t| of ln B, twice the
+    worst-case error of C_j's entries rounded to bf16 (2^-9 each).  The gate is a step at
+    w = ln B, and the CUDA-core statistics path reads C_j in bf16: a row with a block that close
+    to the threshold can take the other branch of the gate on the GPU and change by a factor of
+    up to e^{ln B} on that block.  Such rows are ill-conditioned, not wrong; they are left to
+    the pooled bound."""
+    _, _, _, C = oracle.block_stats(k, k, B, order=2)
+    _, mask, _ = oracle.select(q, k, B, K)
+    BH, L, d = q.shape
+    nblk = L // B
+    lnb = math.log(B)
+    keep = np.ones((BH, L), bool)
+    bits = np.unpackbits(mask.view(np.uint8), axis=-1, bitorder="little")[:, :, :nblk].astype(bool)
+    for bh in range(BH):
+        q64 = q[bh].astype(np.float64)
+        w = 0.5 * np.einsum("ld,jde,le->lj", q64, C[bh], q64)
+        wabs = 0.5 * np.einsum("ld,jde,le->lj", np.abs(q64), np.abs(C[bh]), np.abs(q64))
+        near = (np.abs(w - lnb) <= 2.0 ** -8 * wabs) & ~bits[bh][np.arange(L) // B]
+        keep[bh] = ~near.any(axis=1)
+    return keep
+
+
+def check_gated(got, ref, q, k, B, K, what):
+    """The pooled bound on every row; the row and element bounds on the rows clear of the gate
+    threshold (rows_clear_of_the_gate), which must be most of them."""
+    keep = rows_clear_of_the_gate(q, k, B, K)
+    assert keep.mean() > 0.8, keep.mean()
+    assert rel_l2(got, ref) <= TOL["bf16"]
+    parity.check(got[keep], ref[keep], "bf16", what)
+
+
 # ---------------------------------------------------------------------------
 # statistics
 # ---------------------------------------------------------------------------
@@ -246,7 +279,10 @@ def test_attention_edge_cases(path, case):
     got = pisa.pisa_attention(qt, kt, vt, B, K, order, path=path).float().cpu().numpy().reshape(BH, L, d)
     pisa.pisa_poll_device_status()
     ref = oracle.pisa_attention(q, k, v, B, K, order)
-    parity.check(got, ref, "bf16", case)
+    if case == "gate":
+        check_gated(got, ref, q, k, B, K, case)
+    else:
+        parity.check(got, ref, "bf16", case)
     if case == "Kall":
         parity.check(got, oracle.dense_attention(q, k, v), "bf16", "dense")
 
@@ -259,7 +295,7 @@ def test_gate_changes_the_result_when_w_is_large():
     for path in ("stats", "recompute_tc"):
         on = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=True)
         off = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=False)
-        parity.check(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True), "bf16", "gate on")
+        check_gated(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True), q, k, B, 4, "gate on")
         parity.check(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False), "bf16", "gate off")
         assert rel_l2(on, off) > 1e-2
 
