@@ -32,18 +32,25 @@
 
 namespace pisa {
 
-template <int D, int BS>
+template <int D, int BS, int ORDER>
 struct StatsTcCfg {
     static constexpr uint32_t BOX_BYTES = BS * 128;             // BS rows x 64 bf16 columns
     static constexpr uint32_t TILE_BYTES = (D / 64) * BOX_BYTES;
     static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;     // V tile, then K tile ([V ; K] for d = 64)
-    static constexpr int NSTG = (196608 / STAGE_BYTES) < 6 ? (int)(196608 / STAGE_BYTES) : 6;
-    static constexpr uint32_t BAR_OFF = NSTG * STAGE_BYTES;
+    // output staging: per epilogue warp one 32-row x 64-column box (4 KB) per matrix it writes
+    static constexpr int OUT_BOXES = (D == 128 && ORDER == 2) ? 2 : 1;
+    static constexpr uint32_t OUT_BYTES = 8 * OUT_BOXES * 4096;
+    static constexpr int NSTG_FIT = (int)((204800 - OUT_BYTES) / STAGE_BYTES);
+    static constexpr int NSTG = NSTG_FIT < 6 ? NSTG_FIT : 6;
+    static constexpr uint32_t OUT_OFF = NSTG * STAGE_BYTES;
+    static constexpr uint32_t BAR_OFF = OUT_OFF + OUT_BYTES;
     // FULL, EMPTY per stage; MMADONE, EPIDONE, KBREADY per TMEM buffer; DONE
     static constexpr uint32_t NBAR = 2 * NSTG + 6 + 1;
     static constexpr uint32_t KB_OFF = BAR_OFF + NBAR * 8 + 8;  // fp32 kbar[2][D], vsum[2][D]
     static constexpr uint32_t SMEM = KB_OFF + 4 * D * 4 + 1024;
-    static constexpr int THREADS = 192;                         // producer, MMA, four epilogue warps
+    static constexpr int THREADS = 320;                         // producer, MMA, eight epilogue warps
+    static_assert(NSTG >= 2, "the statistics kernel needs two stages");
+    static_assert(SMEM <= 232448, "shared memory over the per-CTA limit");
 };
 
 template <int D, int ORDER>
@@ -61,24 +68,32 @@ __device__ __forceinline__ float swz_elem(const uint8_t* tile, int n, int c) {
 
 // Persistent: CTA c takes the blocks c, c + grid, c + 2 grid, ... of the flattened
 // (bh, j) index.  Warp 0 streams K_j and V_j through NSTG TMA stages; warp 1 runs
-// the Gram MMAs into two TMEM buffers (block i into buffer i % 2); warps 2-5 take
-// the column sums from the stage, then the epilogue from TMEM.  A stage is free
-// again once its MMA has completed and the column sums have read it; a TMEM
-// buffer once the epilogue has read it.  So the loads of the next blocks and the
-// MMA of the next block overlap this block's epilogue.
+// the Gram MMAs into two TMEM buffers (block i into buffer i % 2); warps 2-9 take
+// the column sums from the stage (one column of K or of V a thread), then the
+// epilogue from TMEM: warp w reads TMEM lane quarter w % 4, and for d = 128 the
+// column half (w - 2) / 4 of it, so each warp owns one 32-row x 64-column box of
+// H_j (and of C_j) and writes it with one TMA store from its own staging box in
+// shared memory (128-byte swizzle, so the row-per-thread writes are free of
+// bank conflicts).  A stage is free again once its MMA has completed and the
+// column sums have read it; a TMEM buffer once the epilogue has read it; a
+// staging box once the warp's previous store has read it.  So the loads of the
+// next blocks, the MMA of the next block and the stores of the previous one all
+// overlap this block's epilogue.
 template <int D, int BS, int ORDER>
-__global__ void __launch_bounds__(192, 1) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                           const __grid_constant__ CUtensorMap tm_v,
+                                                          const __grid_constant__ CUtensorMap tm_h,
+                                                          const __grid_constant__ CUtensorMap tm_c,
                                                           float* __restrict__ kbar, float* __restrict__ vsum,
-                                                          bf16* __restrict__ hstat, bf16* __restrict__ cov,
-                                                          bf16* __restrict__ kaug, int L, int nblk, long total,
+                                                          bf16* __restrict__ kaug, int nblk, int L, long total,
                                                           unsigned* status) {
-    using C = StatsTcCfg<D, BS>;
+    using C = StatsTcCfg<D, BS, ORDER>;
     // M = 128 always (d = 64 stacks V and K); N = d; both operands MN-major
     constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
     constexpr uint32_t TCOLS = stats_tmem_cols<D, ORDER>();  // one buffer
     constexpr long long LIMIT = 2000000000ll;
+    constexpr int NEPI = 8;  // epilogue warps
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_addr(smem);
@@ -97,12 +112,12 @@ __global__ void __launch_bounds__(192, 1) stats_tc_kernel(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NSTG; ++s) {
             tc::mbar_init(bar(B_FULL + s), 1);
-            tc::mbar_init(bar(B_EMPTY + s), 1 + 4);  // the MMA's commit + the four column-sum warps
+            tc::mbar_init(bar(B_EMPTY + s), 1 + NEPI);  // the MMA's commit + the column-sum warps
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(bar(B_MMADONE + b), 1);
-            tc::mbar_init(bar(B_EPIDONE + b), 4);
-            tc::mbar_init(bar(B_KBREADY + b), 4);  // the four warps have written kbar/vsum of the block
+            tc::mbar_init(bar(B_EPIDONE + b), NEPI);
+            tc::mbar_init(bar(B_KBREADY + b), NEPI);  // every warp has written its kbar/vsum columns
         }
         tc::mbar_init(bar(B_DONE), 1);
         tc::fence_barrier_init();
@@ -173,90 +188,122 @@ __global__ void __launch_bounds__(192, 1) stats_tc_kernel(const __grid_constant_
         }
     } else {
         // ------------------------------------------------ column sums, epilogue
-        const int ct = threadIdx.x - 64;         // 0 .. 127
-        const int quarter = warp % 4;            // TMEM lane quarter of this warp
-        const int r = quarter * 32 + lane;       // TMEM lane = output row
+        const int ct = threadIdx.x - 64;          // 0 .. 255
+        const int quarter = warp % 4;             // TMEM lane quarter of this warp
+        const int half = (warp - 2) / 4;          // column half (d = 128)
+        const int r = quarter * 32 + lane;        // TMEM lane = output row
         const float inv_b = 1.0f / (float)BS;
+        // this warp's share of the TMEM epilogue: for d = 64 the warps of half 0 take
+        // all 64 columns of their rows (rows 0-63 H_j, 64-127 the uncentred C_j)
+        const bool is_h = (D == 128) || (quarter < 2);
+        const bool writes = ((D == 128) || half == 0) && (is_h || ORDER == 2);
+        const int ar = (D == 128) ? r : (r & 63);        // row of the output matrix
+        const int col0 = (D == 128) ? half * 64 : 0;     // first column of this warp's box
+        const uint32_t stg = sbase + C::OUT_OFF + (uint32_t)(warp - 2) * (C::OUT_BOXES * 4096u);
         for (int i = 0; i < nmine; ++i) {
             const int s = i % C::NSTG, u = i / C::NSTG, buf = i & 1, ub = i >> 1;
             const long blk = first + (long)i * stride;
-            const int bh = (int)(blk / nblk), j = (int)(blk % nblk);
             if (!tc::mbar_wait_warp(bar(B_FULL + s), u & 1, aborted, status, LIMIT)) break;
             const uint8_t* st = smem + s * C::STAGE_BYTES;
-            for (int c = ct; c < D; c += 128) {
+            // column sums: thread ct < D takes column ct of K (kbar, the centroid split),
+            // D <= ct < 2 D column ct - D of V (vsum)
+            if (ct < 2 * D) {
+                const bool is_k = ct < D;
+                const int c = is_k ? ct : ct - D;
                 float a[BS];
 #pragma unroll
-                for (int n = 0; n < BS; ++n) a[n] = swz_elem<BS>(st + C::TILE_BYTES, n, c);
-                const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-                float sv = 0.f;
-                for (int n = 0; n < BS; ++n) sv += swz_elem<BS>(st, n, c);
-                kbs[buf * D + c] = m;
-                vss[buf * D + c] = sv;
-                const size_t so = ((size_t)bh * nblk + j) * D + c;
-                kbar[so] = m;
-                vsum[so] = sv;
-                if (kaug) {
-                    bf16* ka = kaug + ((size_t)bh * nblk + j) * 8 * D + c;
-                    const bf16 hi = __float2bfloat16_rn(m);
-                    ka[0] = hi;
-                    ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
+                for (int n = 0; n < BS; ++n) a[n] = swz_elem<BS>(st + (is_k ? C::TILE_BYTES : 0u), n, c);
+                const size_t so = (size_t)blk * D + c;
+                if (is_k) {
+                    const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
+                    kbs[buf * D + c] = m;
+                    kbar[so] = m;
+                    if (kaug) {
+                        bf16* ka = kaug + (size_t)blk * 8 * D + c;
+                        const bf16 hi = __float2bfloat16_rn(m);
+                        ka[0] = hi;
+                        ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
 #pragma unroll
-                    for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
+                        for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
+                    }
+                } else {
+                    float sv = 0.f;
+#pragma unroll
+                    for (int n = 0; n < BS; ++n) sv += a[n];
+                    vss[buf * D + c] = sv;
+                    vsum[so] = sv;
                 }
             }
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_arrive(bar(B_EMPTY + s));    // this warp no longer reads the stage
-                tc::mbar_arrive(bar(B_KBREADY + buf));  // and its columns of kbar/vsum are in kbs/vss
+                tc::mbar_arrive(bar(B_EMPTY + s));      // this warp no longer reads the stage
+                tc::mbar_arrive(bar(B_KBREADY + buf));  // and its kbar/vsum columns are in kbs/vss
             }
-            // the block's kbar and vsum from all four warps (a bounded wait, unlike a named barrier,
+            // the block's kbar and vsum from all warps (a bounded wait, unlike a named barrier,
             // so a warp that gave up cannot hold the others forever)
             if (!tc::mbar_wait_warp(bar(B_KBREADY + buf), ub & 1, aborted, status, LIMIT)) break;
             if (!tc::mbar_wait_warp(bar(B_MMADONE + buf), ub & 1, aborted, status, LIMIT)) break;
             tc::fence_after_sync();
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TCOLS);
-            const size_t base = ((size_t)bh * nblk + j) * D * D;
-            const float* kb = kbs + buf * D;
-            const float* vs = vss + buf * D;
-            // which matrix and row this lane holds
-            const bool is_h = (D == 128) || (r < 64);
-            const int ar = (D == 128) ? r : (r & 63);
-            const bool want = is_h || ORDER == 2;
+            if (writes) {
+                // the staging box is free once this warp's previous store has read it
+                if (lane == 0) tc::bulk_wait_read<0>();
+                __syncwarp();
+                const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TCOLS);
+                const float* kb = kbs + buf * D;
+                const float* vs = vss + buf * D;
 #pragma unroll
-            for (int part = 0; part < ((D == 128 && ORDER == 2) ? 2 : 1); ++part) {
-                const bool h_here = (D == 128) ? (part == 0) : is_h;
-                bf16* dst = (h_here ? hstat : cov) + base + (size_t)ar * D;
-                const float rv = h_here ? vs[ar] : kb[ar];
+                for (int part = 0; part < C::OUT_BOXES; ++part) {
+                    const bool h_here = (D == 128) ? (part == 0) : is_h;
+                    const float rv = h_here ? vs[ar] : kb[ar];
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t raw[32];
-                    tc::tmem_ld32(taddr + part * 128 + c0, raw);
-                    tc::tmem_wait_ld();
-                    uint32_t pk[16];
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        uint32_t raw[32];
+                        tc::tmem_ld32(taddr + (uint32_t)(part * 128 + col0 + c0), raw);
+                        tc::tmem_wait_ld();
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
-                        if (h_here) {
-                            x0 = fmaf(-rv, kb[c0 + 2 * e], x0);
-                            x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1);
-                        } else {
-                            x0 = fmaf(-rv, kb[c0 + 2 * e], x0 * inv_b);
-                            x1 = fmaf(-rv, kb[c0 + 2 * e + 1], x1 * inv_b);
+                        for (int e = 0; e < 16; ++e) {
+                            const int cc = col0 + c0 + 2 * e;
+                            float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
+                            if (h_here) {
+                                x0 = fmaf(-rv, kb[cc], x0);
+                                x1 = fmaf(-rv, kb[cc + 1], x1);
+                            } else {
+                                x0 = fmaf(-rv, kb[cc], x0 * inv_b);
+                                x1 = fmaf(-rv, kb[cc + 1], x1 * inv_b);
+                            }
+                            pk[e] = tc::pack_bf16x2(x0, x1);
                         }
-                        pk[e] = tc::pack_bf16x2(x0, x1);
-                    }
-                    if (want) {
-                        uint4* o = reinterpret_cast<uint4*>(dst + c0);
+                        // row `lane` of the box, 16-byte chunks c0/8 .. c0/8 + 3, swizzled
+                        const uint32_t rowa = stg + (uint32_t)part * 4096u + (uint32_t)lane * 128u;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t chunk = (uint32_t)((c0 / 8 + e) ^ (lane & 7));
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + chunk * 16u),
+                                         "r"(pk[4 * e]), "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
+                                         : "memory");
+                        }
                     }
                 }
+                tc::fence_before_sync();
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int y = (int)((long)blk * D + (ar - lane));  // first row of the box
+#pragma unroll
+                    for (int part = 0; part < C::OUT_BOXES; ++part) {
+                        const bool h_here = (D == 128) ? (part == 0) : is_h;
+                        tc::tma_store_2d(h_here ? &tm_h : &tm_c, stg + (uint32_t)part * 4096u, col0, y);
+                    }
+                    tc::bulk_commit();
+                }
             }
-            tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(B_EPIDONE + buf));  // the TMEM buffer is read
         }
+        // the stores have landed before the CTA exits
+        if (lane == 0) tc::bulk_wait<0>();
+        __syncwarp();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -280,15 +327,27 @@ inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float
         }
         encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
     }
-    CUtensorMap maps[2];
-    const void* ptrs[2] = {k, v};
-    for (int t = 0; t < 2; ++t) {
-        cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)(BH * L)};
+    if (order == 2 && !cov) {
+        *err = "the second-order statistics need a C_j buffer";
+        return PISA_ERR_INVALID_ARG;
+    }
+    // K and V as loaded (box 64 columns x B rows); H_j and C_j as stored (box 64 columns x
+    // 32 rows of the [BH nblk d, d] matrices)
+    CUtensorMap maps[4];
+    const long mrows = BH * (long)nblk * d;
+    struct MapSpec {
+        const void* p;
+        long rows;
+        uint32_t box_rows;
+    } specs[4] = {{k, BH * (long)L, (uint32_t)B}, {v, BH * (long)L, (uint32_t)B}, {hstat, mrows, 32u},
+                  {cov ? cov : hstat, mrows, 32u}};
+    for (int t = 0; t < 4; ++t) {
+        cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)specs[t].rows};
         cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
-        cuuint32_t box[2] = {64, (cuuint32_t)B};
+        cuuint32_t box[2] = {64, specs[t].box_rows};
         cuuint32_t estride[2] = {1, 1};
-        CUresult cr = encode(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[t]), gdim, gstride,
-                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        CUresult cr = encode(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(specs[t].p), gdim,
+                             gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (cr != CUDA_SUCCESS) {
             *err = "cuTensorMapEncodeTiled failed (" + std::to_string((int)cr) + ")";
@@ -307,12 +366,12 @@ inline pisa_status run_stats_tc(const void* k, const void* v, float* kbar, float
     cudaError_t e = cudaSuccess;
 #define PISA_STATS_TC(DD, BB, OO)                                                                             \
     if (d == DD && B == BB && order == OO) {                                                                  \
+        using SC = StatsTcCfg<DD, BB, OO>;                                                                    \
         auto kern = stats_tc_kernel<DD, BB, OO>;                                                              \
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,                           \
-                                 (int)StatsTcCfg<DD, BB>::SMEM);                                              \
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC::SMEM);           \
         if (e == cudaSuccess) {                                                                               \
-            kern<<<grid, StatsTcCfg<DD, BB>::THREADS, StatsTcCfg<DD, BB>::SMEM, s>>>(                         \
-                maps[0], maps[1], kbar, vsum, (bf16*)hstat, (bf16*)cov, (bf16*)kaug, L, nblk, total, status); \
+            kern<<<grid, SC::THREADS, SC::SMEM, s>>>(maps[0], maps[1], maps[2], maps[3], kbar, vsum,           \
+                                                     (bf16*)kaug, nblk, L, total, status);                    \
             e = cudaGetLastError();                                                                           \
         }                                                                                                     \
     } else

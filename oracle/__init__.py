@@ -45,11 +45,12 @@ def lib():
                                              ctypes.c_int, f64p, ctypes.c_int]
         L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
-        L.oracle_pisa_backward.argtypes = [f32p, f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int, ctypes.c_int,
-                                           ctypes.c_float, f64p, f64p, f64p, ctypes.c_int]
-        L.oracle_pisa_backward_dq_rows.argtypes = [f32p, f32p, f32p, f32p, li, li, li, li, li, ctypes.c_int,
-                                                   ctypes.c_int, ctypes.c_float, ctypes.c_void_p, li, f64p,
-                                                   ctypes.c_int]
+        L.oracle_pisa_backward.argtypes = [f32p, f32p, f32p, f32p, ctypes.c_void_p, li, li, li, li, li,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_float, f64p, f64p, f64p,
+                                           ctypes.c_int]
+        L.oracle_pisa_backward_dq_rows.argtypes = [f32p, f32p, f32p, f32p, ctypes.c_void_p, li, li, li, li, li,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, li,
+                                                   f64p, ctypes.c_int]
         for fn in ("oracle_pisa_backward", "oracle_pisa_backward_dq_rows", "oracle_route_bias", "oracle_ln_f32", "oracle_pisa_attention_ex", "oracle_pisa_hybrid", "oracle_centroids_f32", "oracle_block_stats", "oracle_select", "oracle_pisa_attention",
                    "oracle_pisa_bruteforce", "oracle_dense_attention"):
             getattr(L, fn).restype = ctypes.c_int
@@ -216,30 +217,38 @@ def pisa_bruteforce(q, k, v, B, K, order=1, gate=True, nthreads=None):
     return out
 
 
-def pisa_backward(q, k, v, dO, B, K, order=1, gate=True, route_eps=None, nthreads=None):
+def pisa_backward(q, k, v, dO, B, K, order=1, gate=True, route_eps=None, nthreads=None, o=None):
     """(dq, dk, dv) [BH, L, d] fp64: gradients of sum_t dO_t . o_t for pisa_attention's
     output o, with the block selection held fixed (``route_eps``: the covariance-aware
-    selection, as in pisa_attention_ex)."""
+    selection, as in pisa_attention_ex).  ``o``: None (delta_t = dO_t . o_t from the
+    recomputed fp64 output) or the forward output the caller holds ([BH, L, d], taken as
+    fp32), as a backward operator of (q, k, v, o, dO) receives it."""
     q, k, v, dO = _f32(q), _f32(k), _f32(v), _f32(dO)
     BH, L, d = q.shape
+    og = None if o is None else _f32(o)
+    if og is not None and og.shape != q.shape:
+        raise ValueError("o must have q's shape")
     dq, dk, dv = (np.zeros((BH, L, d)) for _ in range(3))
     reps = float(route_eps) if route_eps else 0.0
-    rc = lib().oracle_pisa_backward(q, k, v, dO, BH, L, d, B, K, int(order), int(bool(gate)), reps, _ptr(dq),
-                                    _ptr(dk), _ptr(dv), nthreads or default_threads())
+    rc = lib().oracle_pisa_backward(q, k, v, dO, _ptr(og), BH, L, d, B, K, int(order), int(bool(gate)), reps,
+                                    _ptr(dq), _ptr(dk), _ptr(dv), nthreads or default_threads())
     _check(rc, "pisa_backward")
     return dq, dk, dv
 
 
-def pisa_backward_dq_rows(q, k, v, dO, B, K, rows, order=1, gate=True, route_eps=None, nthreads=None):
+def pisa_backward_dq_rows(q, k, v, dO, B, K, rows, order=1, gate=True, route_eps=None, nthreads=None, o=None):
     """dq of the query rows ``rows`` (a sequence of (bh, t)), [nrows, d] fp64: the same
     rows of pisa_backward's dq, computed one row at a time (for sampled checks at sizes
-    where the whole backward is too slow on the CPU)."""
+    where the whole backward is too slow on the CPU); ``o`` as in pisa_backward."""
     q, k, v, dO = _f32(q), _f32(k), _f32(v), _f32(dO)
     BH, L, d = q.shape
+    og = None if o is None else _f32(o)
+    if og is not None and og.shape != q.shape:
+        raise ValueError("o must have q's shape")
     rl = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2))
     out = np.zeros((rl.shape[0], d))
     reps = float(route_eps) if route_eps else 0.0
-    rc = lib().oracle_pisa_backward_dq_rows(q, k, v, dO, BH, L, d, B, K, int(order), int(bool(gate)), reps,
+    rc = lib().oracle_pisa_backward_dq_rows(q, k, v, dO, _ptr(og), BH, L, d, B, K, int(order), int(bool(gate)), reps,
                                             _ptr(rl), rl.shape[0], _ptr(out), nthreads or default_threads())
     _check(rc, "pisa_backward_dq_rows")
     return out

@@ -432,9 +432,13 @@ void backward_prep(const float* q, const float* k, const float* v, long L, long 
 
 // Query row t: gx[n] = dL/dx_n over all L keys (x_n = q_t.k_n) and pw[n] =
 // wt_n / D, the normalised weight of key n in o_t, with the selection (and
-// the gate decision) held fixed.
-void backward_row(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B,
-                  const uint32_t* mask, const double* kbar, int order, int gate, long t, double* gx, double* pw) {
+// the gate decision) held fixed.  o_given (null, or [L, d]): the forward output
+// the caller holds, as a backward operator of (q, k, v, o, dO) receives it;
+// delta = dO_t . o_t then uses its row t instead of the recomputed o_t (the
+// only place o enters the gradient).
+void backward_row(const float* q, const float* k, const float* v, const float* dO, const float* o_given, long L,
+                  long d, long B, const uint32_t* mask, const double* kbar, int order, int gate, long t, double* gx,
+                  double* pw) {
     const long nblk = L / B;
     const long words = (nblk + 31) / 32;
     const long i = t / B;
@@ -483,7 +487,10 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
     for (long c = 0; c < d; ++c) o[c] /= D;
     const float* dOt = dO + t * d;
     double delta = 0.0;
-    for (long c = 0; c < d; ++c) delta += (double)dOt[c] * o[c];
+    if (o_given)
+        for (long c = 0; c < d; ++c) delta += (double)dOt[c] * (double)o_given[t * d + c];
+    else
+        for (long c = 0; c < d; ++c) delta += (double)dOt[c] * o[c];
     for (long n = 0; n < L; ++n) {
         double g = 0.0;
         for (long c = 0; c < d; ++c) g += (double)dOt[c] * (double)v[n * d + c];
@@ -513,13 +520,14 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
     }
 }
 
-void backward_one(const float* q, const float* k, const float* v, const float* dO, long L, long d, long B, long K,
-                  int order, int gate, float route_eps, double* dq, double* dk, double* dv) {
+void backward_one(const float* q, const float* k, const float* v, const float* dO, const float* o_given, long L,
+                  long d, long B, long K, int order, int gate, float route_eps, double* dq, double* dk, double* dv) {
     std::vector<uint32_t> mask;
     std::vector<double> kbar, gx(L), pw(L);
     backward_prep(q, k, v, L, d, B, K, route_eps, mask, kbar);
     for (long t = 0; t < L; ++t) {
-        backward_row(q, k, v, dO, L, d, B, mask.data(), kbar.data(), order, gate, t, gx.data(), pw.data());
+        backward_row(q, k, v, dO, o_given, L, d, B, mask.data(), kbar.data(), order, gate, t, gx.data(),
+                     pw.data());
         const float* qt = q + t * d;
         const float* dOt = dO + t * d;
         for (long n = 0; n < L; ++n) {
@@ -759,9 +767,11 @@ int oracle_pisa_bruteforce(const float* q, const float* k, const float* v, long 
 
 // Gradients (dq, dk, dv) [BH, L, d] fp64 of sum_t dO_t . o_t for the method's
 // output o (pisa_attention's), selection held fixed.  Zero-initialised here.
-int oracle_pisa_backward(const float* q, const float* k, const float* v, const float* dO, long BH, long L, long d,
-                         long B, long K, int order, int gate, float route_eps, double* dq, double* dk, double* dv,
-                         int nthreads) {
+// o_given: null (delta from the recomputed fp64 o) or [BH, L, d], the forward
+// output the caller holds (delta = dO_t . o_given_t).
+int oracle_pisa_backward(const float* q, const float* k, const float* v, const float* dO, const float* o_given,
+                         long BH, long L, long d, long B, long K, int order, int gate, float route_eps, double* dq,
+                         double* dk, double* dv, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     if (K < 0 || K > L / B) return -1;
     std::fill(dq, dq + BH * L * d, 0.0);
@@ -769,16 +779,17 @@ int oracle_pisa_backward(const float* q, const float* k, const float* v, const f
     std::fill(dv, dv + BH * L * d, 0.0);
     parallel_for(BH, nthreads, [&](long bh) {
         const long o = bh * L * d;
-        backward_one(q + o, k + o, v + o, dO + o, L, d, B, K, order, gate, route_eps, dq + o, dk + o, dv + o);
+        backward_one(q + o, k + o, v + o, dO + o, o_given ? o_given + o : nullptr, L, d, B, K, order, gate, route_eps,
+                     dq + o, dk + o, dv + o);
     });
     return 0;
 }
 
 // dq of a list of query rows: rows[2*r] = bh, rows[2*r+1] = t; dq_rows
 // receives [nrows, d] fp64 (the rows of oracle_pisa_backward's dq).
-int oracle_pisa_backward_dq_rows(const float* q, const float* k, const float* v, const float* dO, long BH, long L,
-                                 long d, long B, long K, int order, int gate, float route_eps, const int64_t* rows,
-                                 long nrows, double* dq_rows, int nthreads) {
+int oracle_pisa_backward_dq_rows(const float* q, const float* k, const float* v, const float* dO,
+                                 const float* o_given, long BH, long L, long d, long B, long K, int order, int gate,
+                                 float route_eps, const int64_t* rows, long nrows, double* dq_rows, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     if (K < 0 || K > L / B) return -1;
     for (long r = 0; r < nrows; ++r)
@@ -795,8 +806,8 @@ int oracle_pisa_backward_dq_rows(const float* q, const float* k, const float* v,
         const long bh = rows[2 * r], t = rows[2 * r + 1];
         const long o = bh * L * d;
         std::vector<double> gx(L), pw(L);
-        backward_row(q + o, k + o, v + o, dO + o, L, d, B, mask[bh].data(), kbar[bh].data(), order, gate, t,
-                     gx.data(), pw.data());
+        backward_row(q + o, k + o, v + o, dO + o, o_given ? o_given + o : nullptr, L, d, B, mask[bh].data(),
+                     kbar[bh].data(), order, gate, t, gx.data(), pw.data());
         for (long c = 0; c < d; ++c) {
             double acc = 0.0;
             for (long n = 0; n < L; ++n) acc += gx[n] * (double)k[o + n * d + c];

@@ -296,7 +296,12 @@ def test_gate_changes_the_result_when_w_is_large():
         on = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=True)
         off = run_attn(q, k, v, B, 4, 2, "bf16", path, gate=False)
         check_gated(on, oracle.pisa_attention(q, k, v, B, 4, 2, gate=True), q, k, B, 4, "gate on")
-        parity.check(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False), "bf16", "gate off")
+        # With the gate off, w reaches several hundred on these inputs (that is what the
+        # scaled key column is for), and a row's output follows e^w of its largest block:
+        # the statistics path's bf16 C_j moves w by up to 2^-9 (1/2 |q|^T |C_j| |q|), over
+        # 2^-5 on every row here.  Such rows are ill-conditioned, so the gate-off arm keeps
+        # the pooled bound only; the gate-on arm (w <= ln B) has all three.
+        assert rel_l2(off, oracle.pisa_attention(q, k, v, B, 4, 2, gate=False)) <= TOL["bf16"]
         assert rel_l2(on, off) > 1e-2
 
 

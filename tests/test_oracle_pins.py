@@ -685,3 +685,33 @@ def test_backward_dq_rows_are_the_full_backward_rows():
         rows = [(0, 0), (0, 31), (1, 32), (1, 200), (0, 255)]
         got = oracle.pisa_backward_dq_rows(q, k, v, dO, 32, 2, rows, order, True, route_eps=reps)
         np.testing.assert_array_equal(got, np.stack([gq[b, t] for b, t in rows]))
+
+
+def test_backward_with_a_given_forward_output():
+    # delta_t = dO_t . o_t is the only place the forward output enters the gradient.
+    # (1) given the method's own output, the gradients are those of the recomputed one
+    # (up to o's rounding to fp32); (2) dv does not depend on o; (3) at K = all (dense
+    # softmax attention) a change e_t of delta_t moves dq_t by -e_t sum_n P_tn k_n and dk_n
+    # by -sum_t e_t P_tn q_t, P the dense softmax weights (written out here in numpy).
+    L, d, B = 64, 8, 16
+    q, k, v = small(111, BH=2, L=L, d=d, scale=1.5)
+    dO = small(112, BH=2, L=L, d=d)[0]
+    for order, gate, K in ((1, True, 1), (2, False, 2), (0, True, 1), (1, True, L // B)):
+        o = oracle.pisa_attention_ex(q, k, v, B, K, order, gate=gate)
+        g0 = oracle.pisa_backward(q, k, v, dO, B, K, order, gate)
+        g1 = oracle.pisa_backward(q, k, v, dO, B, K, order, gate, o=o)
+        for a, b in zip(g0, g1):
+            assert oracle.rel_l2(b, a) <= 1e-6
+    K = L // B
+    o = oracle.pisa_attention_ex(q, k, v, B, K, 1).astype(np.float32)
+    o2 = (o + 0.25 * np.random.default_rng(113).standard_normal(o.shape)).astype(np.float32)
+    ga = oracle.pisa_backward(q, k, v, dO, B, K, 1, o=o)
+    gb = oracle.pisa_backward(q, k, v, dO, B, K, 1, o=o2)
+    q64, k64, dO64 = (x.astype(np.float64) for x in (q, k, dO))
+    e = np.einsum("btc,btc->bt", dO64, o2.astype(np.float64) - o.astype(np.float64))
+    x = q64 @ k64.transpose(0, 2, 1)
+    P = np.exp(x - x.max(axis=-1, keepdims=True))
+    P /= P.sum(axis=-1, keepdims=True)
+    np.testing.assert_allclose(gb[0] - ga[0], -e[..., None] * (P @ k64), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(gb[1] - ga[1], -np.einsum("bt,btn,btc->bnc", e, P, q64), rtol=0, atol=1e-11)
+    np.testing.assert_array_equal(gb[2], ga[2])
