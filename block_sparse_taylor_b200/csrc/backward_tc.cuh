@@ -19,19 +19,20 @@
 // bwd_dq_tc_kernel (query-major): one 128-row M tile of one (batch, head) per
 // CTA, visiting every key tile of 128 keys.  Every reduction over a block
 // (sb, sum G, sum G u, the spread behind w) runs over the block's keys of one
-// query row, which are TMEM columns of one lane: each softmax thread does them
-// alone, from its row of S (held in registers) and G (streamed twice).
+// query row, which are TMEM columns of one lane.
 //   warp 0      TMA producer: Q and dO once; K tiles through three stages, V
 //               tiles through two (V is free once G = dO V^T has completed)
 //   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2-5   the four lane quarters of the M tile
-// TMEM: S_0 | S_1 | G | dQ.  S = Q K^T alternates between two buffers; the
-// softmax writes dS (bf16) over the first half of the buffer's columns, and
-// dQ += dS K runs from TMEM (K as the MN-major B operand).  MMA order after
-// the softmax of tile j has handed over dS_j and released G:
-//   G_{j+1}, dQ_j, S_{j+2}
-// so the softmax of tile j+1 starts after one product and the other two run
-// beside it.
+//   warps 2-9   softmax: warp w takes lane quarter w % 4 and key half (w - 2) / 4
+//               of each tile, 64 keys: it loads its S and G columns into
+//               registers with one wait, releases G, forms the block sums in
+//               one shifted pass (at B = 128 the two halves of a block add their
+//               sums through four spare TMEM columns), and writes dS in bf16 over
+//               the first 32 of its S columns
+// TMEM: S_0 | S_1 | G | dQ.  S = Q K^T alternates between two buffers; dQ +=
+// dS K runs from TMEM (K as the MN-major B operand).  MMA order per tile j:
+// G_{j+1} as soon as the softmax holds G_j in registers, then dQ_j and S_{j+2}
+// once dS_j is written, so the next G product runs beside the softmax.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -44,7 +45,7 @@
 namespace pisa {
 namespace bwdtc {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, eight softmax warps (two per lane quarter)
 
 template <int D>
 struct DqCfg {
@@ -59,8 +60,8 @@ struct DqCfg {
     static constexpr uint32_t V_OFF = K_OFF + NSK * TILE_BYTES;
     static constexpr uint32_t BAR_OFF = V_OFF + NSV * TILE_BYTES;
     // QFULL; KFULL, KEMPTY per K stage; VFULL, VEMPTY per V stage; SFULL, DSREADY per
-    // S buffer; GFULL, GFREE; DQFULL; DONE
-    static constexpr uint32_t NBAR = 1 + 2 * NSK + 2 * NSV + 4 + 2 + 1 + 1;
+    // S buffer; GFULL, GFREE; DQFULL; DONE; PAIR per lane quarter (B = 128 block sums)
+    static constexpr uint32_t NBAR = 1 + 2 * NSK + 2 * NSV + 4 + 2 + 1 + 1 + 4;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t G_COL = 256, DQ_COL = 384;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -92,35 +93,67 @@ __global__ void bwd_lse_kernel(const float* __restrict__ m, const float* __restr
         lse[i] = m[i] - logf(dinv[i]);
 }
 
-// Block reductions of one query row over a key tile (TMEM columns of one lane), in one pass
-// over S and G shifted by the block's first logit x0 (the shift keeps the sums of
-// (x - x0) free of cancellation when the block's logits share a large offset):
+// Block sums of one query row over the 64 keys of a half tile that this thread holds
+// (S and G as raw fp32 bits, two 32-key chunks each), in one pass shifted by x0, the
+// block's first logit (the shift keeps the sums of (x - x0) free of cancellation when the
+// block's logits share a large offset):
 //   s1 = sum (x - x0), s2 = sum (x - x0)^2, sg = sum G, sgd = sum G (x - x0)
 // so that sb = x0 + s1/B, sum (x - sb)^2 = s2 - s1^2/B, sum G (x - sb) = sgd - (s1/B) sg.
-template <int BPT, int BS>
-struct RowBlockSums {
-    float x0[BPT], s1[BPT], s2[BPT], sg[BPT], sgd[BPT];
+// Packed fp32 pairs: the even and the odd keys accumulate separately.
+struct HalfSums {
+    float s1, s2, sg, sgd;
 };
 
-template <int BPT, int BS>
-__device__ __forceinline__ void row_block_sums(uint32_t s_addr, uint32_t g_addr, RowBlockSums<BPT, BS>& r) {
+__device__ __forceinline__ HalfSums half_sums(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
+                                              const uint32_t (&ga)[32], const uint32_t (&gb)[32], float x0) {
+    const uint64_t nx0 = tc::f2_make(-x0, -x0);
+    uint64_t a1 = 0ull, a2 = 0ull, ag = 0ull, agd = 0ull;
 #pragma unroll
-    for (int bb = 0; bb < BPT; ++bb) r.x0[bb] = r.s1[bb] = r.s2[bb] = r.sg[bb] = r.sgd[bb] = 0.f;
+    for (int e = 0; e < 32; ++e) {
+        const uint32_t* xs = e < 16 ? xa : xb;
+        const uint32_t* gs = e < 16 ? ga : gb;
+        const int o = 2 * (e & 15);
+        const uint64_t x2 = tc::f2_make(__uint_as_float(xs[o]), __uint_as_float(xs[o + 1]));
+        const uint64_t g2 = tc::f2_make(__uint_as_float(gs[o]), __uint_as_float(gs[o + 1]));
+        const uint64_t dx = tc::f2_add(x2, nx0);
+        a1 = tc::f2_add(a1, dx);
+        a2 = tc::f2_fma(dx, dx, a2);
+        ag = tc::f2_add(ag, g2);
+        agd = tc::f2_fma(g2, dx, agd);
+    }
+    const float2 s1 = tc::f2_split(a1), s2 = tc::f2_split(a2), sg = tc::f2_split(ag), sgd = tc::f2_split(agd);
+    return HalfSums{s1.x + s1.y, s2.x + s2.y, sg.x + sg.y, sgd.x + sgd.y};
+}
+
+// dS (or P and dS) of 32 keys (one chunk of a half tile), packed as bf16 pairs (keys 2e,
+// 2e + 1 in word e).  Selected block: P = 2^{x log2 e - lse2}, dS = P (G - delta);
+// unselected block: u = x - sb, P = a + Pu u, dS = A G + X u + Cc.
+template <bool WANT_P>
+__device__ __forceinline__ void chunk_ds(const uint32_t (&xs)[32], const uint32_t (&gs)[32], bool sel, bool valid,
+                                         float lse2, float del, float sb, float a, float A, float X, float Cc,
+                                         float Pu, uint32_t (&pp)[16], uint32_t (&dd)[16]) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    const uint64_t ndel = tc::f2_make(-del, -del), nsb = tc::f2_make(-sb, -sb);
+    const uint64_t A2 = tc::f2_make(A, A), X2 = tc::f2_make(X, X), C2 = tc::f2_make(Cc, Cc);
+    const uint64_t a2 = tc::f2_make(a, a), P2 = tc::f2_make(Pu, Pu);
 #pragma unroll
-    for (int c = 0; c < 128 / 16; ++c) {
-        uint32_t xs[16], gs[16];
-        tc::tmem_ld16(s_addr + c * 16, xs);
-        tc::tmem_ld16(g_addr + c * 16, gs);
-        tc::tmem_wait_ld();
-        const int bb = (c * 16) / BS;
-        if ((c * 16) % BS == 0) r.x0[bb] = __uint_as_float(xs[0]);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const float dx = __uint_as_float(xs[e]) - r.x0[bb], gv = __uint_as_float(gs[e]);
-            r.s1[bb] += dx;
-            r.s2[bb] = fmaf(dx, dx, r.s2[bb]);
-            r.sg[bb] += gv;
-            r.sgd[bb] = fmaf(gv, dx, r.sgd[bb]);
+    for (int e = 0; e < 16; ++e) {
+        const float x0 = __uint_as_float(xs[2 * e]), x1 = __uint_as_float(xs[2 * e + 1]);
+        const uint64_t g2 = tc::f2_make(__uint_as_float(gs[2 * e]), __uint_as_float(gs[2 * e + 1]));
+        uint64_t p2, d2;
+        if (sel) {
+            p2 = tc::f2_make(tc::ex2(fmaf(x0, LOG2E, -lse2)), tc::ex2(fmaf(x1, LOG2E, -lse2)));
+            d2 = tc::f2_mul(p2, tc::f2_add(g2, ndel));
+        } else {
+            const uint64_t u2 = tc::f2_add(tc::f2_make(x0, x1), nsb);
+            p2 = tc::f2_fma(P2, u2, a2);
+            d2 = tc::f2_fma(A2, g2, tc::f2_fma(X2, u2, C2));
+        }
+        const float2 d = tc::f2_split(d2);
+        dd[e] = valid ? tc::pack_bf16x2(d.x, d.y) : 0u;
+        if (WANT_P) {
+            const float2 pv = tc::f2_split(p2);
+            pp[e] = valid ? tc::pack_bf16x2(pv.x, pv.y) : 0u;
         }
     }
 }
@@ -166,9 +199,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      unsigned* status) {
     using C = DqCfg<D>;
     constexpr float LOG2E = 1.4426950408889634f;
-    constexpr float INV_B = 1.0f / (float)BS;
-    constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
-    constexpr int BPT = C::NK / BS;  // blocks per key tile
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, G = dO V^T
     constexpr uint32_t IDESC_Q = tc::idesc_bf16(128, D, true);     // dQ += dS K, K MN-major
 
@@ -178,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NSK, B_VFULL = 1 + 2 * C::NSK,
               B_VEMPTY = B_VFULL + C::NSV, B_SFULL = B_VEMPTY + C::NSV, B_DSREADY = B_SFULL + 2,
-              B_GFULL = B_DSREADY + 2, B_GFREE = B_GFULL + 1, B_DQFULL = B_GFREE + 1, B_DONE = B_DQFULL + 1;
+              B_GFULL = B_DSREADY + 2, B_GFREE = B_GFULL + 1, B_DQFULL = B_GFREE + 1, B_DONE = B_DQFULL + 1,
+              B_PAIR = B_DONE + 1;
     uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -199,12 +230,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(bar(B_SFULL + b), 1);
-            tc::mbar_init(bar(B_DSREADY + b), 128);
+            tc::mbar_init(bar(B_DSREADY + b), 256);
         }
         tc::mbar_init(bar(B_GFULL), 1);
-        tc::mbar_init(bar(B_GFREE), 128);
+        tc::mbar_init(bar(B_GFREE), 256);
         tc::mbar_init(bar(B_DQFULL), 1);
         tc::mbar_init(bar(B_DONE), 1);
+        for (int qq = 0; qq < 4; ++qq) tc::mbar_init(bar(B_PAIR + qq), 64);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -278,11 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_S, kk > 0);
                 }
             };
-            // dQ += dS (TMEM, buffer b) x K_j (MN-major), K-dim = 128 keys
+            // dQ += dS (TMEM, buffer b) x K_j (MN-major), K-dim = 128 keys.  dS of keys
+            // 64h .. 64h + 63 sits packed in columns 64h .. 64h + 31 of the buffer.
             auto issue_dq = [&](int b, int sk, bool first) {
 #pragma unroll
                 for (int kk = 0; kk < C::NK / 16; ++kk)
-                    tc::mma_ts(tmem + C::DQ_COL, tmem + (uint32_t)(b * 128) + kk * 8,
+                    tc::mma_ts(tmem + C::DQ_COL, tmem + (uint32_t)(b * 128 + kk * 8 + (kk >= 4 ? 32 : 0)),
                                kmn0 + sk * kTileStep + (uint64_t)((kk * 16 * 128) >> 4), IDESC_Q,
                                (first && kk == 0) ? 0u : 1u);
             };
@@ -308,8 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0; ok && j < NT; ++j) {
                 const int b = j & 1;
-                // the softmax of tile j has written dS_j and read G_j
-                if (!tc::mbar_wait(bar(B_DSREADY + b), (j >> 1) & 1, aborted, status, kWaitLimitCycles)) break;
+                // the softmax has read G_j (and S_j) into registers: G_{j+1} may overwrite it
                 if (!tc::mbar_wait(bar(B_GFREE), j & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
                 if (j + 1 < NT) {
@@ -319,6 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_commit(bar(B_GFULL));
                     tc::mma_commit(bar(B_VEMPTY + sv));
                 }
+                // the softmax of tile j has written dS_j
+                if (!tc::mbar_wait(bar(B_DSREADY + b), (j >> 1) & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
                 issue_dq(b, j % C::NSK, j == 0);
                 tc::mma_commit(bar(B_KEMPTY + j % C::NSK));
                 if (j + 2 < NT) {
@@ -336,7 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- softmax
-        const int quarter = warp % 4;           // TMEM lane quarter of this warp
+        // Warp w takes lane quarter w % 4 (32 query rows) and key half (w - 2) / 4 of every
+        // tile: 64 keys, one block at B = 64, half of one at B = 128 (whose sums the two warps
+        // of a quarter exchange).
+        const int quarter = warp % 4;
+        const int half = (warp - 2) / 4;
         const int r = quarter * 32 + lane;      // row inside the M tile = TMEM lane
         const int qrow = q0 + r;
         const bool valid = qrow < L;
@@ -346,68 +385,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
         const float ln_b = logf((float)BS);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t g_addr = lane_base + C::G_COL;
+        const uint32_t g_addr = lane_base + C::G_COL + 64 * half;
         for (int j = 0; j < NT; ++j) {
             const int b = j & 1;
             if (!tc::mbar_wait_warp(bar(B_SFULL + b), (j >> 1) & 1, aborted, status, kWaitLimitCycles)) break;
             if (!tc::mbar_wait_warp(bar(B_GFULL), j & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
-            const uint32_t s_addr = lane_base + (uint32_t)(b * 128);
-            bool sel[BPT];
-            const uint32_t mw = __ldg(mrow + ((j * BPT) >> 5));
-#pragma unroll
-            for (int bb = 0; bb < BPT; ++bb) sel[bb] = (mw >> ((j * BPT + bb) & 31)) & 1u;
-            RowBlockSums<BPT, BS> rs;
-            row_block_sums<BPT, BS>(s_addr, g_addr, rs);
-            float sb[BPT], A[BPT], X[BPT], Cc[BPT];
-#pragma unroll
-            for (int bb = 0; bb < BPT; ++bb) {
-                float a, Pu;
-                block_coefs<BS, ORDER>(rs.x0[bb], rs.s1[bb], rs.s2[bb], rs.sg[bb], rs.sgd[bb], lse2, del, gate, ln_b,
-                                       sb[bb], a, A[bb], X[bb], Cc[bb], Pu);
+            const uint32_t s_tile = lane_base + (uint32_t)(b * 128);
+            const uint32_t s_addr = s_tile + 64 * half;
+            uint32_t xa[32], xb[32], ga[32], gb[32];
+            tc::tmem_ld32(s_addr, xa);
+            tc::tmem_ld32(s_addr + 32, xb);
+            tc::tmem_ld32(g_addr, ga);
+            tc::tmem_ld32(g_addr + 32, gb);
+            uint32_t x0raw = 0u;
+            if (BS == 128 && half == 1) x0raw = tc::tmem_ld1(s_tile);  // the block's first logit
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_GFREE));
+            const int jb = (j * C::NK + 64 * half) / BS;  // this half's block
+            const bool sel = (__ldg(mrow + (jb >> 5)) >> (jb & 31)) & 1u;
+            const float x0 = (BS == 128 && half == 1) ? __uint_as_float(x0raw) : __uint_as_float(xa[0]);
+            HalfSums hs = half_sums(xa, xb, ga, gb, x0);
+            if (BS == 128) {
+                // the other half's sums, through four TMEM columns of this buffer that hold
+                // S of keys this warp has already read (the dS columns are the first 32)
+                uint32_t mine[4] = {__float_as_uint(hs.s1), __float_as_uint(hs.s2), __float_as_uint(hs.sg),
+                                    __float_as_uint(hs.sgd)};
+                tc::tmem_st4(s_addr + 32, mine);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar(B_PAIR + quarter));
+                if (!tc::mbar_wait_warp(bar(B_PAIR + quarter), j & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                uint32_t other[4];
+                tc::tmem_ld4(s_tile + 64 * (1 - half) + 32, other);
+                tc::tmem_wait_ld();
+                hs.s1 += __uint_as_float(other[0]);
+                hs.s2 += __uint_as_float(other[1]);
+                hs.sg += __uint_as_float(other[2]);
+                hs.sgd += __uint_as_float(other[3]);
             }
-            // dS (bf16) over the first half of the S buffer's columns, 32 keys per store; the
-            // columns written hold keys already read (key 2e and 2e+1 go to column e)
-#pragma unroll
-            for (int c = 0; c < C::NK / 32; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t xs[16], gs[16];
-                    tc::tmem_ld16(s_addr + c * 32 + hh * 16, xs);
-                    tc::tmem_ld16(g_addr + c * 32 + hh * 16, gs);
-                    tc::tmem_wait_ld();
-                    const int bb = (c * 32 + hh * 16) / BS;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float ds[2];
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const float xv = __uint_as_float(xs[2 * e + h]), gv = __uint_as_float(gs[2 * e + h]);
-                            if (sel[bb]) {
-                                ds[h] = tc::ex2(fmaf(xv, LOG2E, -lse2)) * (gv - del);
-                            } else {
-                                ds[h] = fmaf(A[bb], gv, fmaf(X[bb], xv - sb[bb], Cc[bb]));
-                            }
-                        }
-                        pk[hh * 8 + e] = tc::pack_bf16x2(ds[0], ds[1]);
-                    }
-                }
-                tc::tmem_st16(s_addr + c * 16, pk);
+            float sb, a, A, X, Cc, Pu;
+            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, sb, a, A, X, Cc, Pu);
+            // dS (bf16) over the first 32 columns of this half: keys 2e and 2e + 1 in column e
+            {
+                uint32_t pp[16], dd[16];
+                chunk_ds<false>(xa, ga, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp, dd);
+                tc::tmem_st16(s_addr, dd);
+                chunk_ds<false>(xb, gb, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp, dd);
+                tc::tmem_st16(s_addr + 16, dd);
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(bar(B_GFREE));
             tc::mbar_arrive(bar(B_DSREADY + b));
         }
-        // epilogue: dq row (fp32) to global
+        // epilogue: this warp's column half of the dq row (fp32) to global
         if (tc::mbar_wait_warp(bar(B_DQFULL), 0, aborted, status, kWaitLimitCycles)) {
             tc::fence_after_sync();
-            float* drow = dq + ((size_t)bh * L + (valid ? qrow : 0)) * D;
+            float* drow = dq + ((size_t)bh * L + (valid ? qrow : 0)) * D + half * (D / 2);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t raw[32];
-                tc::tmem_ld32(lane_base + C::DQ_COL + c * 32, raw);
+                tc::tmem_ld32(lane_base + C::DQ_COL + half * (D / 2) + c * 32, raw);
                 tc::tmem_wait_ld();
                 if (valid) {
                     float4* dst = reinterpret_cast<float4*>(drow + c * 32);
@@ -440,11 +480,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // with dO and Q as MN-major B operands.  TMEM: S | G | dV | dK.
 //   warp 0      TMA producer: K and V once; Q and dO tiles through NSQ stages
 //   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2-5   softmax: the four lane quarters (query rows), then the
-//               epilogue of dK and dV (key rows)
-// MMA order after the softmax of query tile i has handed over P_i and dS_i:
-//   NSQ = 2: S_{i+1}, G_{i+1}, dK_i, dV_i       NSQ = 1: dK_i, dV_i, S_{i+1}, G_{i+1}
-// (one stage of Q and dO at d = 128: its tiles are free only after dK_i, dV_i).
+//   warps 2-9   softmax: warp w takes lane quarter w % 4 (query rows, then key
+//               rows in the epilogue of dK and dV) and key half (w - 2) / 4; it
+//               loads its S and G columns into registers with one wait and
+//               releases them (SGFREE) before it forms the block sums (at B = 128
+//               the two halves of a block add their sums through shared memory)
+// MMA order per query tile i:
+//   NSQ = 2: S_{i+1}, G_{i+1} once S_i, G_i are in registers; dK_i, dV_i once
+//            P_i, dS_i are written
+//   NSQ = 1: dK_i, dV_i, then S_{i+1} (Q_{i+1} lands once dK_i has read Q_i) and
+//            G_{i+1} (dO_{i+1} once dV_i has read dO_i): at d = 128 one stage of Q
+//            and dO is what shared memory holds beside K, V, P and dS.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvCfg {
@@ -460,9 +506,13 @@ struct DkvCfg {
     static constexpr uint32_t DO_OFF = Q_OFF + NSQ * TILE_BYTES;
     static constexpr uint32_t P_OFF = DO_OFF + NSQ * TILE_BYTES;
     static constexpr uint32_t DS_OFF = P_OFF + PT_BYTES;
-    static constexpr uint32_t BAR_OFF = DS_OFF + PT_BYTES;
-    // KVFULL; QFULL, QEMPTY, DOFULL, DOEMPTY per stage; SFULL; PREADY; PFREE; DKVFULL; DONE
-    static constexpr uint32_t NBAR = 1 + 4 * NSQ + 5;
+    // B = 128 block sums exchanged between the two warps of a lane quarter:
+    // fp32 [tile parity][key half][128 rows][4]
+    static constexpr uint32_t XCH_OFF = DS_OFF + PT_BYTES;
+    static constexpr uint32_t BAR_OFF = XCH_OFF + 2 * 2 * 128 * 4 * 4;
+    // KVFULL; QFULL, QEMPTY, DOFULL, DOEMPTY per stage; SFULL; PREADY; PFREE; DKVFULL; DONE;
+    // SGFREE; PAIR per lane quarter
+    static constexpr uint32_t NBAR = 1 + 4 * NSQ + 5 + 1 + 4;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t G_COL = 128, DV_COL = 256, DK_COL = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -483,9 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int nblk, int words, int gate, unsigned* status) {
     using C = DkvCfg<D>;
     constexpr float LOG2E = 1.4426950408889634f;
-    constexpr float INV_B = 1.0f / (float)BS;
-    constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
-    constexpr int BPT = 128 / BS;  // blocks per key tile
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
     // M = 128 keys, N = d, A (P or dS) and B (dO or Q) both MN-major
     constexpr uint32_t IDESC_KV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
@@ -497,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_KVFULL = 0, B_QFULL = 1, B_QEMPTY = 1 + C::NSQ, B_DOFULL = 1 + 2 * C::NSQ,
               B_DOEMPTY = 1 + 3 * C::NSQ, B_SFULL = 1 + 4 * C::NSQ, B_PREADY = B_SFULL + 1,
-              B_PFREE = B_PREADY + 1, B_DKVFULL = B_PFREE + 1, B_DONE = B_DKVFULL + 1;
+              B_PFREE = B_PREADY + 1, B_DKVFULL = B_PFREE + 1, B_DONE = B_DKVFULL + 1, B_SGFREE = B_DONE + 1,
+              B_PAIR = B_SGFREE + 1;
     uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -515,10 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(bar(B_DOEMPTY + s), 1);
         }
         tc::mbar_init(bar(B_SFULL), 1);
-        tc::mbar_init(bar(B_PREADY), 128);
+        tc::mbar_init(bar(B_PREADY), 256);
         tc::mbar_init(bar(B_PFREE), 1);
         tc::mbar_init(bar(B_DKVFULL), 1);
         tc::mbar_init(bar(B_DONE), 1);
+        tc::mbar_init(bar(B_SGFREE), 256);
+        for (int qq = 0; qq < 4; ++qq) tc::mbar_init(bar(B_PAIR + qq), 64);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -585,12 +635,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pmn = tc::sdesc_sw128(sbase + C::P_OFF, C::BOX_BYTES, 1024);    // P as MN-major A
             const uint64_t dsmn = tc::sdesc_sw128(sbase + C::DS_OFF, C::BOX_BYTES, 1024);  // dS as MN-major A
             constexpr uint64_t kTileStep = C::TILE_BYTES >> 4;
-            auto issue_sg = [&](int st) {
+            auto issue_s = [&](int st) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
                     tc::mma_ss(tmem, qdesc0 + st * kTileStep + off, kdesc + off, IDESC_S, kk > 0);
                 }
+            };
+            auto issue_g = [&](int st) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
@@ -605,37 +657,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_KV, (first && kk == 0) ? 0u : 1u);
                 }
             };
-            bool ok = tc::mbar_wait(bar(B_KVFULL), 0, aborted, status, kWaitLimitCycles);
-            ok = ok && tc::mbar_wait(bar(B_QFULL + 0), 0, aborted, status, kWaitLimitCycles);
-            ok = ok && tc::mbar_wait(bar(B_DOFULL + 0), 0, aborted, status, kWaitLimitCycles);
-            if (ok) {
-                issue_sg(0);
+            // S_{i+1} and G_{i+1} into the single S | G buffer (stage st1, use u1)
+            auto next_sg = [&](int st1, int u1) -> bool {
+                if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) return false;
+                tc::fence_after_sync();
+                issue_s(st1);
+                if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) return false;
+                tc::fence_after_sync();
+                issue_g(st1);
                 tc::mma_commit(bar(B_SFULL));
-            }
+                return true;
+            };
+            bool ok = tc::mbar_wait(bar(B_KVFULL), 0, aborted, status, kWaitLimitCycles);
+            ok = ok && next_sg(0, 0);
             for (int i = 0; ok && i < NQT; ++i) {
                 const int st = i % C::NSQ;
                 const bool more = i + 1 < NQT;
                 const int st1 = (i + 1) % C::NSQ, u1 = (i + 1) / C::NSQ;
-                // the softmax has written P_i and dS_i (and read S_i and G_i)
+                // two stages: S_{i+1}, G_{i+1} as soon as the softmax holds S_i and G_i in registers
+                if (C::NSQ >= 2 && more) {
+                    if (!tc::mbar_wait(bar(B_SGFREE), i & 1, aborted, status, kWaitLimitCycles)) break;
+                    if (!next_sg(st1, u1)) break;
+                }
+                // the softmax has written P_i and dS_i
                 if (!tc::mbar_wait(bar(B_PREADY), i & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                if (C::NSQ >= 2 && more) {
-                    if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
-                    if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
-                    issue_sg(st1);
-                    tc::mma_commit(bar(B_SFULL));
-                }
                 issue_kv(C::DK_COL, dsmn, qmn0 + st * kTileStep, i == 0);
                 tc::mma_commit(bar(B_QEMPTY + st));
                 issue_kv(C::DV_COL, pmn, domn0 + st * kTileStep, i == 0);
                 tc::mma_commit(bar(B_DOEMPTY + st));
                 tc::mma_commit(bar(B_PFREE));
-                if (C::NSQ == 1 && more) {
-                    if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
-                    if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) break;
-                    issue_sg(st1);
-                    tc::mma_commit(bar(B_SFULL));
-                }
+                // one stage (d = 128): Q_{i+1} lands once dK_i has read Q_i, dO_{i+1} once dV_i has
+                // read dO_i; S_{i+1} goes first so that it runs while dO_{i+1} arrives
+                if (C::NSQ == 1 && more && !next_sg(st1, u1)) break;
             }
             if (!aborted) tc::mma_commit(bar(B_DKVFULL));
             tc::mma_commit(bar(B_DONE));
@@ -644,13 +698,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- softmax
+        // Warp w takes lane quarter w % 4 (32 query rows of each tile, then 32 key rows in
+        // the epilogue) and key half (w - 2) / 4: 64 of the tile's keys, one block at B = 64,
+        // half of one at B = 128 (whose sums the two warps of a quarter exchange).
         const int quarter = warp % 4;
-        const int r = quarter * 32 + lane;  // TMEM lane: query row of the tile, then key row in the epilogue
+        const int half = (warp - 2) / 4;
+        const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float ln_b = logf((float)BS);
-        const int jb0 = k0 / BS;  // first block of this key tile
+        const int jb = (k0 + 64 * half) / BS;  // this half's block
         uint8_t* ptile = smem + C::P_OFF;
         uint8_t* dstile = smem + C::DS_OFF;
+        float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);
         for (int i = 0; i < NQT; ++i) {
             const int qrow = i * C::NQ + r;
             const bool valid = qrow < L;
@@ -658,71 +717,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
             const float lse2 = (valid ? __ldg(lse + (size_t)bh * L + qrow) : 0.f) * LOG2E;
             const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
-            bool sel[BPT];
-#pragma unroll
-            for (int bb = 0; bb < BPT; ++bb) sel[bb] = (__ldg(mrow + ((jb0 + bb) >> 5)) >> ((jb0 + bb) & 31)) & 1u;
+            const bool sel = (__ldg(mrow + (jb >> 5)) >> (jb & 31)) & 1u;
             if (!tc::mbar_wait_warp(bar(B_SFULL), i & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
-            RowBlockSums<BPT, BS> rs;
-            row_block_sums<BPT, BS>(lane_base, lane_base + C::G_COL, rs);
-            float sb[BPT], aa[BPT], A[BPT], X[BPT], Cc[BPT], Pu[BPT];
-#pragma unroll
-            for (int bb = 0; bb < BPT; ++bb)
-                block_coefs<BS, ORDER>(rs.x0[bb], rs.s1[bb], rs.s2[bb], rs.sg[bb], rs.sgd[bb], lse2, del, gate, ln_b,
-                                       sb[bb], aa[bb], A[bb], X[bb], Cc[bb], Pu[bb]);
+            uint32_t xa[32], xb[32], ga[32], gb[32];
+            tc::tmem_ld32(lane_base + 64 * half, xa);
+            tc::tmem_ld32(lane_base + 64 * half + 32, xb);
+            tc::tmem_ld32(lane_base + C::G_COL + 64 * half, ga);
+            tc::tmem_ld32(lane_base + C::G_COL + 64 * half + 32, gb);
+            uint32_t x0raw = 0u;
+            if (BS == 128 && half == 1) x0raw = tc::tmem_ld1(lane_base);  // the block's first logit
+            tc::tmem_wait_ld();
+            // S_i and G_i are in registers: the next tile's products may overwrite them
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_SGFREE));
+            const float x0 = (BS == 128 && half == 1) ? __uint_as_float(x0raw) : __uint_as_float(xa[0]);
+            HalfSums hs = half_sums(xa, xb, ga, gb, x0);
+            if (BS == 128) {
+                float4* mine = reinterpret_cast<float4*>(xch + ((((i & 1) * 2 + half) * 128) + r) * 4);
+                *mine = make_float4(hs.s1, hs.s2, hs.sg, hs.sgd);
+                tc::mbar_arrive(bar(B_PAIR + quarter));
+                if (!tc::mbar_wait_warp(bar(B_PAIR + quarter), i & 1, aborted, status, kWaitLimitCycles)) break;
+                // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
+                (void)tc::mbar_try_wait(bar(B_PAIR + quarter), i & 1);
+                const float4 o = *reinterpret_cast<const float4*>(xch + ((((i & 1) * 2 + (1 - half)) * 128) + r) * 4);
+                hs.s1 += o.x;
+                hs.s2 += o.y;
+                hs.sg += o.z;
+                hs.sgd += o.w;
+            }
+            float sb, a, A, X, Cc, Pu;
+            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, sb, a, A, X, Cc, Pu);
             // the previous tile's dK and dV products have read P and dS
             if (i > 0 && !tc::mbar_wait_warp(bar(B_PFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) break;
-            // P and dS rows (bf16) into shared memory, 16 keys at a time; rows past L are zero
+            // row r of P and dS (bf16), this half's 64 keys = box `half` of each tile, 32 keys a chunk
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t xs[16], gs[16];
-                tc::tmem_ld16(lane_base + c * 16, xs);
-                tc::tmem_ld16(lane_base + C::G_COL + c * 16, gs);
-                tc::tmem_wait_ld();
-                const int bb = (c * 16) / BS;
-                uint32_t pp[8], dd[8];
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t pp[16], dd[16];
+                chunk_ds<true>(ch == 0 ? xa : xb, ch == 0 ? ga : gb, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp,
+                               dd);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float pv[2], dsv[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float xv = __uint_as_float(xs[2 * e + h]), gv = __uint_as_float(gs[2 * e + h]);
-                        if (sel[bb]) {
-                            pv[h] = tc::ex2(fmaf(xv, LOG2E, -lse2));
-                            dsv[h] = pv[h] * (gv - del);
-                        } else {
-                            const float u = xv - sb[bb];
-                            pv[h] = fmaf(Pu[bb], u, aa[bb]);
-                            dsv[h] = fmaf(A[bb], gv, fmaf(X[bb], u, Cc[bb]));
-                        }
-                        if (!valid) pv[h] = dsv[h] = 0.f;
-                    }
-                    pp[e] = tc::pack_bf16x2(pv[0], pv[1]);
-                    dd[e] = tc::pack_bf16x2(dsv[0], dsv[1]);
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 2; ++q4) {
-                    st_swz16(ptile, r, c * 2 + q4, make_uint4(pp[4 * q4], pp[4 * q4 + 1], pp[4 * q4 + 2], pp[4 * q4 + 3]));
-                    st_swz16(dstile, r, c * 2 + q4, make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]));
+                for (int c = 0; c < 4; ++c) {
+                    st_swz16(ptile, r, 8 * half + 4 * ch + c,
+                             make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]));
+                    st_swz16(dstile, r, 8 * half + 4 * ch + c,
+                             make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]));
                 }
             }
             // generic-proxy stores -> the tensor core (async proxy) reads them
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::fence_proxy_async_smem();
             tc::fence_before_sync();
             tc::mbar_arrive(bar(B_PREADY));
         }
-        // epilogue: dK and dV rows (TMEM lane = key) to global
+        // epilogue: this warp's column half of the dK and dV rows (TMEM lane = key) to global
         if (tc::mbar_wait_warp(bar(B_DKVFULL), 0, aborted, status, kWaitLimitCycles)) {
             tc::fence_after_sync();
             const int key = k0 + r;
-            float* krow = dk + ((size_t)bh * L + key) * D;
-            float* vrow = dv + ((size_t)bh * L + key) * D;
+            float* krow = dk + ((size_t)bh * L + key) * D + half * (D / 2);
+            float* vrow = dv + ((size_t)bh * L + key) * D + half * (D / 2);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 float* dst_row = part == 0 ? krow : vrow;
-                const uint32_t col = part == 0 ? C::DK_COL : C::DV_COL;
+                const uint32_t col = (part == 0 ? C::DK_COL : C::DV_COL) + half * (D / 2);
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t raw[32];
                     tc::tmem_ld32(lane_base + col + c * 32, raw);
                     tc::tmem_wait_ld();

@@ -189,7 +189,11 @@ def test_autograd_function():
     out.backward(dev(dO, dt))
     torch.cuda.synchronize()
     pisa.pisa_poll_device_status()
-    direct = pisa.pisa_attention_backward(dev(q, dt), dev(k, dt), dev(v, dt), out.detach(), dev(dO, dt), B, K, 1)
+    # the autograd function hands the backward its forward's lse; the same deterministic
+    # forward gives the same lse here
+    _, lse = pisa.pisa_attention_lse(dev(q, dt), dev(k, dt), dev(v, dt), B, K, 1)
+    direct = pisa.pisa_attention_backward(dev(q, dt), dev(k, dt), dev(v, dt), out.detach(), dev(dO, dt), B, K, 1,
+                                          lse=lse)
     for t, g in zip((qt, kt, vt), direct):
         assert t.grad.dtype == torch.bfloat16
         assert torch.equal(t.grad, g.to(torch.bfloat16))
