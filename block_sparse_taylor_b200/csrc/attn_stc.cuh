@@ -24,7 +24,9 @@
 //     q_t . kbar_j as the sum of a bf16 high part and a bf16 low part of the fp32
 //     centroid (the "aug" rows of the statistics).  The softmax warps read G back
 //     from TMEM and accumulate e^{l - m}(G + vsum_j) in registers, so the row
-//     weight is applied on the way out and the tensor core never waits for it.
+//     weight is applied on the way out and the tensor core never waits for it;
+//     vsum_j comes through a ring of shared-memory slots that the producer fills
+//     with bulk copies, so the softmax reads it at shared-memory latency.
 // The phase-1 accumulator O is read into the same registers between the phases.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer, warps
@@ -85,10 +87,16 @@ struct StcCfg {
     static constexpr uint32_t SLOT_STRIDE = 160;         // TMEM columns between G slots
     static constexpr int NQT = 256 / BS;                 // query tiles per CTA
     static constexpr int MAXBLK = 4096;                  // nblk limit of the library
+    // phase 2: the items' value sums (fp32, GB blocks each) through their own ring of
+    // NV slots, filled by bulk copies and released by the softmax threads
+    static constexpr int NV = 4;
+    static constexpr uint32_t VS_BYTES = GB * D * 4;
+    static constexpr uint32_t VS_OFF = KV_OFF + KV_BYTES;
     // QFULL; KFULL, KEMPTY, VFULL, VEMPTY per stage; SFULL, PHALF, PFULL, OFULL per
-    // M tile; ODRAIN; F2FULL, F2EMPTY per phase-2 stage; GFULL, GEMPTY per slot; DONE
-    static constexpr uint32_t NBAR = 1 + 4 * NS + 8 + 1 + 2 * NS2 + 2 * NSLOT + 1;
-    static constexpr uint32_t BAR_OFF = KV_OFF + KV_BYTES;
+    // M tile; ODRAIN; F2FULL, F2EMPTY per phase-2 stage; GFULL, GEMPTY per slot; DONE;
+    // VSFULL, VSEMPTY per value-sum slot
+    static constexpr uint32_t NBAR = 1 + 4 * NS + 8 + 1 + 2 * NS2 + 2 * NSLOT + 1 + 2 * NV;
+    static constexpr uint32_t BAR_OFF = VS_OFF + NV * VS_BYTES;
     static constexpr uint32_t SCHED_OFF = BAR_OFF + NBAR * 8 + 16;
     // schedule: union words [128], per-tile words [NQT][128], union list [MAXBLK],
     // list of the other blocks [MAXBLK]
@@ -132,6 +140,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
     const int B_SFULL = 1 + 4 * C::NS, B_PHALF = B_SFULL + 2, B_PFULL = B_PHALF + 2, B_OFULL = B_PFULL + 2;
     const int B_ODRAIN = B_OFULL + 2, B_F2FULL = B_ODRAIN + 1, B_F2EMPTY = B_F2FULL + C::NS2;
     const int B_GFULL = B_F2EMPTY + C::NS2, B_GEMPTY = B_GFULL + C::NSLOT, B_DONE = B_GEMPTY + C::NSLOT;
+    const int B_VSFULL = B_DONE + 1, B_VSEMPTY = B_VSFULL + C::NV;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int bh = blockIdx.y;
@@ -213,6 +222,10 @@ __global__ void __launch_bounds__(kStcThreads, 1)
             tc::mbar_init(bar(B_GEMPTY + s), 128);
         }
         tc::mbar_init(bar(B_DONE), 1);
+        for (int s = 0; s < C::NV; ++s) {
+            tc::mbar_init(bar(B_VSFULL + s), 1);
+            tc::mbar_init(bar(B_VSEMPTY + s), 256);
+        }
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -286,6 +299,17 @@ __global__ void __launch_bounds__(kStcThreads, 1)
                         tc::tma_load_2d(dst + x * C::BOX2_BYTES + C::AUG_ROW0 * 128 + b * 1024, &tm_aug,
                                         bar(B_F2FULL + st), x * 64, arow);
                     }
+                }
+                // the item's value sums into their slot, once the softmax is done with the slot's last item
+                const int vs = g % C::NV, vu = g / C::NV;
+                if (vu > 0 && !tc::mbar_wait(bar(B_VSEMPTY + vs), (vu - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_VSFULL + vs), C::VS_BYTES);
+                for (int b = 0; b < C::GB; ++b) {
+                    const int li = g * C::GB + b;
+                    const int blk = nlist[li < nn ? li : nn - 1];
+                    tc::bulk_load(sbase + C::VS_OFF + vs * C::VS_BYTES + b * D * 4,
+                                  vsum + ((size_t)bh * nblk + blk) * D, D * 4, bar(B_VSFULL + vs));
                 }
             }
             if (aborted) {
@@ -510,12 +534,17 @@ __global__ void __launch_bounds__(kStcThreads, 1)
         // ---- phase 2: blocks unselected by every tile of the CTA
         for (int g = 0; !aborted && g < NI; ++g) {
             const int it = 2 * g + h, slot = it % C::NSLOT, use = it / C::NSLOT;
+            const int vs = g % C::NV;
             if (!tc::mbar_wait_warp(bar(B_GFULL + slot), use & 1, aborted, status, kWaitLimitCycles)) break;
+            if (!tc::mbar_wait_warp(bar(B_VSFULL + vs), (g / C::NV) & 1, aborted, status, kWaitLimitCycles)) break;
+            // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
+            (void)tc::mbar_try_wait(bar(B_VSFULL + vs), (g / C::NV) & 1);
             tc::fence_after_sync();
             const uint32_t gaddr = lane_base + (uint32_t)(slot * C::SLOT_STRIDE);
             uint32_t sc[16];  // the 16 centroid columns: high and low part of q . kbar_j, 8 apart
             tc::tmem_ld16(gaddr + C::AUG_ROW0, sc);
             tc::tmem_wait_ld();
+            const float* vsm = reinterpret_cast<const float*>(smem + C::VS_OFF + vs * C::VS_BYTES);
 #pragma unroll
             for (int b = 0; b < C::GB; ++b) {
                 const int li = g * C::GB + b;
@@ -536,7 +565,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
                 const float alpha = live ? tc::ex2(l2 - m_run) : 0.f;
                 dsum = fmaf((float)BS, alpha, dsum);
                 const uint64_t al2 = tc::f2_make(alpha, alpha);
-                const float4* vrow = reinterpret_cast<const float4*>(vsum + ((size_t)bh * nblk + blk) * D);
+                const float4* vrow = reinterpret_cast<const float4*>(vsm + b * D);
 #pragma unroll
                 for (int c = 0; c < D / 16; ++c) {
                     uint32_t gr[16];
@@ -544,7 +573,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 vv = __ldg(vrow + c * 4 + e4);
+                        const float4 vv = vrow[c * 4 + e4];
                         const uint64_t g0 = tc::f2_add(
                             tc::f2_make(__uint_as_float(gr[4 * e4]), __uint_as_float(gr[4 * e4 + 1])),
                             tc::f2_make(vv.x, vv.y));
@@ -558,6 +587,7 @@ __global__ void __launch_bounds__(kStcThreads, 1)
             }
             tc::fence_before_sync();
             tc::mbar_arrive(bar(B_GEMPTY + slot));
+            tc::mbar_arrive(bar(B_VSEMPTY + vs));
         }
 
         // ---- epilogue: o = N / D

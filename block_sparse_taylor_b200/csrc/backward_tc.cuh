@@ -492,30 +492,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 //            G_{i+1} (dO_{i+1} once dV_i has read dO_i): at d = 128 one stage of Q
 //            and dO is what shared memory holds beside K, V, P and dS.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int BS>
 struct DkvCfg {
     static constexpr int NQ = 128;                     // query rows per tile
     static constexpr int NBOX = D / 64;
     static constexpr uint32_t BOX_BYTES = 128 * 128;
     static constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;  // 128 rows x d bf16
     static constexpr uint32_t PT_BYTES = 2 * BOX_BYTES;       // 128 queries x 128 keys bf16
-    static constexpr int NSQ = (D == 128) ? 1 : 2;      // stages of Q and dO
+    // stages of Q and of dO.  At d = 128 shared memory holds K, V, P, dS and three
+    // tiles of Q and dO: the second dO stage at B = 64, the exchange buffer of the
+    // B = 128 block sums otherwise.
+    static constexpr int NSQ = (D == 128) ? 1 : 2;
+    static constexpr int NSO = (D == 128 && BS == 128) ? 1 : 2;
     static constexpr uint32_t K_OFF = 0;
     static constexpr uint32_t V_OFF = K_OFF + TILE_BYTES;
     static constexpr uint32_t Q_OFF = V_OFF + TILE_BYTES;
     static constexpr uint32_t DO_OFF = Q_OFF + NSQ * TILE_BYTES;
-    static constexpr uint32_t P_OFF = DO_OFF + NSQ * TILE_BYTES;
+    static constexpr uint32_t P_OFF = DO_OFF + NSO * TILE_BYTES;
     static constexpr uint32_t DS_OFF = P_OFF + PT_BYTES;
     // B = 128 block sums exchanged between the two warps of a lane quarter:
     // fp32 [tile parity][key half][128 rows][4]
     static constexpr uint32_t XCH_OFF = DS_OFF + PT_BYTES;
-    static constexpr uint32_t BAR_OFF = XCH_OFF + 2 * 2 * 128 * 4 * 4;
-    // KVFULL; QFULL, QEMPTY, DOFULL, DOEMPTY per stage; SFULL; PREADY; PFREE; DKVFULL; DONE;
-    // SGFREE; PAIR per lane quarter
-    static constexpr uint32_t NBAR = 1 + 4 * NSQ + 5 + 1 + 4;
+    static constexpr uint32_t XCH_BYTES = (BS == 128) ? 2 * 2 * 128 * 4 * 4 : 0;
+    static constexpr uint32_t BAR_OFF = XCH_OFF + XCH_BYTES;
+    // KVFULL; QFULL, QEMPTY per Q stage; DOFULL, DOEMPTY per dO stage; SFULL; PREADY;
+    // PFREE; DKVFULL; DONE; SGFREE; PAIR per lane quarter
+    static constexpr uint32_t NBAR = 1 + 2 * NSQ + 2 * NSO + 5 + 1 + 4;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t G_COL = 128, DV_COL = 256, DK_COL = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(SMEM <= 232448, "shared memory over the per-CTA limit");
 };
 
 // 16 bytes (8 bf16) at chunk c of row t of a 128-byte-swizzled tile (64 columns per box)
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const uint32_t* __restrict__ mask, const float* __restrict__ lse,
                        const float* __restrict__ delta, float* __restrict__ dk, float* __restrict__ dv, int L,
                        int nblk, int words, int gate, unsigned* status) {
-    using C = DkvCfg<D>;
+    using C = DkvCfg<D, BS>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
     // M = 128 keys, N = d, A (P or dS) and B (dO or Q) both MN-major
@@ -543,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = tc::smem_addr(smem);
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_KVFULL = 0, B_QFULL = 1, B_QEMPTY = 1 + C::NSQ, B_DOFULL = 1 + 2 * C::NSQ,
-              B_DOEMPTY = 1 + 3 * C::NSQ, B_SFULL = 1 + 4 * C::NSQ, B_PREADY = B_SFULL + 1,
+              B_DOEMPTY = B_DOFULL + C::NSO, B_SFULL = B_DOEMPTY + C::NSO, B_PREADY = B_SFULL + 1,
               B_PFREE = B_PREADY + 1, B_DKVFULL = B_PFREE + 1, B_DONE = B_DKVFULL + 1, B_SGFREE = B_DONE + 1,
               B_PAIR = B_SGFREE + 1;
     uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
@@ -559,6 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < C::NSQ; ++s) {
             tc::mbar_init(bar(B_QFULL + s), 1);
             tc::mbar_init(bar(B_QEMPTY + s), 1);
+        }
+        for (int s = 0; s < C::NSO; ++s) {
             tc::mbar_init(bar(B_DOFULL + s), 1);
             tc::mbar_init(bar(B_DOEMPTY + s), 1);
         }
@@ -594,21 +602,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int lastQ = -1, lastO = -1;
             for (int i = 0; i < NQT; ++i) {
-                const int st = i % C::NSQ, u = i / C::NSQ;
                 const int row = bh * L + i * C::NQ;
-                if (u > 0 && !tc::mbar_wait(bar(B_QEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles)) break;
-                tc::mbar_expect_tx(bar(B_QFULL + st), C::TILE_BYTES);
-                for (int b = 0; b < C::NBOX; ++b)
-                    tc::tma_load_2d(sbase + C::Q_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q,
-                                    bar(B_QFULL + st), b * 64, row);
-                lastQ = i;
-                if (u > 0 && !tc::mbar_wait(bar(B_DOEMPTY + st), (u - 1) & 1, aborted, status, kWaitLimitCycles))
+                // dO first: its stage frees up with dV_{i - NSO}, which the MMA issues
+                // before the dK that frees Q's stage
+                const int so = i % C::NSO, uo = i / C::NSO;
+                if (uo > 0 && !tc::mbar_wait(bar(B_DOEMPTY + so), (uo - 1) & 1, aborted, status, kWaitLimitCycles))
                     break;
-                tc::mbar_expect_tx(bar(B_DOFULL + st), C::TILE_BYTES);
+                tc::mbar_expect_tx(bar(B_DOFULL + so), C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
-                    tc::tma_load_2d(sbase + C::DO_OFF + st * C::TILE_BYTES + b * C::BOX_BYTES, &tm_do,
-                                    bar(B_DOFULL + st), b * 64, row);
+                    tc::tma_load_2d(sbase + C::DO_OFF + so * C::TILE_BYTES + b * C::BOX_BYTES, &tm_do,
+                                    bar(B_DOFULL + so), b * 64, row);
                 lastO = i;
+                const int sq = i % C::NSQ, uq = i / C::NSQ;
+                if (uq > 0 && !tc::mbar_wait(bar(B_QEMPTY + sq), (uq - 1) & 1, aborted, status, kWaitLimitCycles))
+                    break;
+                tc::mbar_expect_tx(bar(B_QFULL + sq), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::Q_OFF + sq * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q,
+                                    bar(B_QFULL + sq), b * 64, row);
+                lastQ = i;
             }
             if (aborted) {
                 bool a2 = false;
@@ -617,9 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a2 = false;
                     tc::mbar_wait(bar(B_QFULL + i % C::NSQ), (i / C::NSQ) & 1, a2, status, kWaitLimitCycles);
                 }
-                for (int i = (lastO - C::NSQ + 1 > 0 ? lastO - C::NSQ + 1 : 0); i <= lastO; ++i) {
+                for (int i = (lastO - C::NSO + 1 > 0 ? lastO - C::NSO + 1 : 0); i <= lastO; ++i) {
                     a2 = false;
-                    tc::mbar_wait(bar(B_DOFULL + i % C::NSQ), (i / C::NSQ) & 1, a2, status, kWaitLimitCycles);
+                    tc::mbar_wait(bar(B_DOFULL + i % C::NSO), (i / C::NSO) & 1, a2, status, kWaitLimitCycles);
                 }
             }
         }
@@ -657,39 +669,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_KV, (first && kk == 0) ? 0u : 1u);
                 }
             };
-            // S_{i+1} and G_{i+1} into the single S | G buffer (stage st1, use u1)
-            auto next_sg = [&](int st1, int u1) -> bool {
-                if (!tc::mbar_wait(bar(B_QFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) return false;
+            // S_i into the S columns (Q stage i % NSQ), G_i into the G columns (dO stage i % NSO)
+            auto put_s = [&](int i) -> bool {
+                const int sq = i % C::NSQ, uq = i / C::NSQ;
+                if (!tc::mbar_wait(bar(B_QFULL + sq), uq & 1, aborted, status, kWaitLimitCycles)) return false;
                 tc::fence_after_sync();
-                issue_s(st1);
-                if (!tc::mbar_wait(bar(B_DOFULL + st1), u1 & 1, aborted, status, kWaitLimitCycles)) return false;
-                tc::fence_after_sync();
-                issue_g(st1);
-                tc::mma_commit(bar(B_SFULL));
+                issue_s(sq);
                 return true;
             };
+            auto put_g = [&](int i) -> bool {
+                const int so = i % C::NSO, uo = i / C::NSO;
+                if (!tc::mbar_wait(bar(B_DOFULL + so), uo & 1, aborted, status, kWaitLimitCycles)) return false;
+                tc::fence_after_sync();
+                issue_g(so);
+                return true;
+            };
+            constexpr bool kEarlyS = C::NSQ >= 2, kEarlyG = C::NSO >= 2;
             bool ok = tc::mbar_wait(bar(B_KVFULL), 0, aborted, status, kWaitLimitCycles);
-            ok = ok && next_sg(0, 0);
+            ok = ok && put_s(0) && put_g(0);
+            if (ok) tc::mma_commit(bar(B_SFULL));
             for (int i = 0; ok && i < NQT; ++i) {
-                const int st = i % C::NSQ;
+                const int sq = i % C::NSQ, so = i % C::NSO;
                 const bool more = i + 1 < NQT;
-                const int st1 = (i + 1) % C::NSQ, u1 = (i + 1) / C::NSQ;
-                // two stages: S_{i+1}, G_{i+1} as soon as the softmax holds S_i and G_i in registers
-                if (C::NSQ >= 2 && more) {
+                // the products of tile i + 1 whose operand has a stage of its own go in as soon
+                // as the softmax holds S_i and G_i in registers (SGFREE)
+                if (more && (kEarlyS || kEarlyG)) {
                     if (!tc::mbar_wait(bar(B_SGFREE), i & 1, aborted, status, kWaitLimitCycles)) break;
-                    if (!next_sg(st1, u1)) break;
+                    if (kEarlyS && !put_s(i + 1)) break;
+                    if (kEarlyG && !put_g(i + 1)) break;
+                    if (kEarlyS && kEarlyG) tc::mma_commit(bar(B_SFULL));
                 }
                 // the softmax has written P_i and dS_i
                 if (!tc::mbar_wait(bar(B_PREADY), i & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_kv(C::DK_COL, dsmn, qmn0 + st * kTileStep, i == 0);
-                tc::mma_commit(bar(B_QEMPTY + st));
-                issue_kv(C::DV_COL, pmn, domn0 + st * kTileStep, i == 0);
-                tc::mma_commit(bar(B_DOEMPTY + st));
+                issue_kv(C::DK_COL, dsmn, qmn0 + sq * kTileStep, i == 0);
+                tc::mma_commit(bar(B_QEMPTY + sq));
+                issue_kv(C::DV_COL, pmn, domn0 + so * kTileStep, i == 0);
+                tc::mma_commit(bar(B_DOEMPTY + so));
                 tc::mma_commit(bar(B_PFREE));
-                // one stage (d = 128): Q_{i+1} lands once dK_i has read Q_i, dO_{i+1} once dV_i has
-                // read dO_i; S_{i+1} goes first so that it runs while dO_{i+1} arrives
-                if (C::NSQ == 1 && more && !next_sg(st1, u1)) break;
+                // a single stage: Q_{i+1} lands once dK_i has read Q_i (dO_{i+1} once dV_i has
+                // read dO_i)
+                if (more && !(kEarlyS && kEarlyG)) {
+                    if (!kEarlyS && !put_s(i + 1)) break;
+                    if (!kEarlyG && !put_g(i + 1)) break;
+                    tc::mma_commit(bar(B_SFULL));
+                }
             }
             if (!aborted) tc::mma_commit(bar(B_DKVFULL));
             tc::mma_commit(bar(B_DONE));

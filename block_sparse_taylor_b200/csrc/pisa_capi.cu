@@ -471,7 +471,7 @@ pisa_status run_backward_tc(const void* q, const void* k, const void* v, const v
         e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pisa::bwdtc::DqCfg<DD>::SMEM); \
         if (e == cudaSuccess)                                                                                     \
             e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize,                             \
-                                     (int)pisa::bwdtc::DkvCfg<DD>::SMEM);                                         \
+                                     (int)pisa::bwdtc::DkvCfg<DD, BB>::SMEM);                                         \
         if (e == cudaSuccess) {                                                                                   \
             kq<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DqCfg<DD>::SMEM, s>>>(                                 \
                 maps[0], maps[1], maps[2], maps[3], mask, lse, del, dq, (int)g.L, (int)g.nblk, (int)g.words, gate,  \
@@ -479,7 +479,7 @@ pisa_status run_backward_tc(const void* q, const void* k, const void* v, const v
             e = cudaGetLastError();                                                                               \
         }                                                                                                         \
         if (e == cudaSuccess) {                                                                                   \
-            kk<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DkvCfg<DD>::SMEM, s>>>(                                \
+            kk<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DkvCfg<DD, BB>::SMEM, s>>>(                                \
                 maps[0], maps[1], maps[2], maps[3], mask, lse, del, dk, dv, (int)g.L, (int)g.nblk, (int)g.words,    \
                 gate, status);                                                                                    \
             e = cudaGetLastError();                                                                               \

@@ -58,6 +58,47 @@ __device__ __forceinline__ float canonical_dot4(const float (&q)[D / 4], const f
     return v;
 }
 
+// The K-th largest of the warp's ordered keys, NKT per lane (key j = lane + 32 i of the
+// score row st, j < nblk; 0 < K < nblk): a binary search on the key's bits, from the
+// highest bit in which the warp's smallest and largest keys differ (the bits above it
+// are common to every key, so to the answer).  Sets `need` to how many of the keys equal
+// to the result are taken (the lowest block indices first).
+template <int NKT>
+__device__ __forceinline__ uint32_t kth_ordered_key(const float* st, int nblk, int K, int& need) {
+    const int lane = threadIdx.x & 31;
+    uint32_t kv[NKT];
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int i = 0; i < NKT; ++i) {
+        const int j = lane + 32 * i;
+        kv[i] = j < nblk ? ordered_key(st[j]) : 0u;  // 0 sorts below every score
+        if (j < nblk) {
+            lo = min(lo, kv[i]);
+            hi = max(hi, kv[i]);
+        }
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    uint32_t thr = hi;
+    if (lo != hi) {
+        const int top = 31 - __clz(lo ^ hi);  // highest differing bit
+        thr = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+        for (int bit = top; bit >= 0; --bit) {
+            const uint32_t cand = thr | (1u << bit);
+            int cnt = 0;
+#pragma unroll
+            for (int i = 0; i < NKT; ++i) cnt += kv[i] >= cand;
+            cnt = __reduce_add_sync(0xffffffffu, cnt);
+            if (cnt >= K) thr = cand;
+        }
+    }
+    int gt = 0;
+#pragma unroll
+    for (int i = 0; i < NKT; ++i) gt += kv[i] > thr;
+    need = K - __reduce_add_sync(0xffffffffu, gt);
+    return thr;
+}
+
 template <int D>
 struct SelectCfg {
     static constexpr int THREADS = 256;
@@ -88,7 +129,7 @@ inline int select_tiles_per_cta(int nblk) {
 //      ordered score, then ties broken by ascending block index with ballots;
 //      the ballots are the mask words and give the ascending index list.
 template <typename T, int D, int BS>
-__global__ void __launch_bounds__(256, 2) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+__global__ void __launch_bounds__(256, 3) select_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                                                         int L, int nblk, int K, int words, int QT,
                                                         int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
                                                         const float* __restrict__ bias,
@@ -180,7 +221,8 @@ __global__ void __launch_bounds__(256, 2) select_kernel(const T* __restrict__ q,
     }
 
     // 3. top-K, one warp per tile.  For nblk <= 1024 every lane keeps its
-    // blocks' ordered keys (j = lane + 32 i) in registers during the search.
+    // blocks' ordered keys (j = lane + 32 i) in registers during the search
+    // (kth_ordered_key); longer rows are searched from shared memory.
     const unsigned lt_mask = (1u << lane) - 1u;
     const int nk = (nblk + 31) / 32;
     for (int tt = warp; tt < nq; tt += 8) {
@@ -190,24 +232,15 @@ __global__ void __launch_bounds__(256, 2) select_kernel(const T* __restrict__ q,
         int need = 0;       // how many of the ties at thr to take, lowest index first
         if (K > 0 && K < nblk) {
             if (nk <= 32) {
-                uint32_t kv[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int j = lane + 32 * i;
-                    kv[i] = (i < nk && j < nblk) ? ordered_key(st[j]) : 0u;  // 0 sorts below every score
-                }
-                for (int bit = 31; bit >= 0; --bit) {
-                    const uint32_t cand = thr | (1u << bit);
-                    int cnt = 0;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) cnt += (i < nk) & (kv[i] >= cand);
-                    cnt = __reduce_add_sync(0xffffffffu, cnt);
-                    if (cnt >= K) thr = cand;
-                }
-                int gt = 0;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) gt += (i < nk) & (kv[i] > thr);
-                need = K - __reduce_add_sync(0xffffffffu, gt);
+                // every lane keeps its blocks' ordered keys in registers during the search
+                if (nk <= 4)
+                    thr = kth_ordered_key<4>(st, nblk, K, need);
+                else if (nk <= 8)
+                    thr = kth_ordered_key<8>(st, nblk, K, need);
+                else if (nk <= 16)
+                    thr = kth_ordered_key<16>(st, nblk, K, need);
+                else
+                    thr = kth_ordered_key<32>(st, nblk, K, need);
             } else {
                 for (int bit = 31; bit >= 0; --bit) {
                     const uint32_t cand = thr | (1u << bit);

@@ -204,6 +204,9 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
             const int s = i % C::NSTG, u = i / C::NSTG, buf = i & 1, ub = i >> 1;
             const long blk = first + (long)i * stride;
             if (!tc::mbar_wait_warp(bar(B_FULL + s), u & 1, aborted, status, LIMIT)) break;
+            // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
+            // of the stage's bytes
+            (void)tc::mbar_try_wait(bar(B_FULL + s), u & 1);
             const uint8_t* st = smem + s * C::STAGE_BYTES;
             // column sums: thread ct < D takes column ct of K (kbar, the centroid split),
             // D <= ct < 2 D column ct - D of V (vsum)
