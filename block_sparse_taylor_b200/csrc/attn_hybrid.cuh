@@ -471,9 +471,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const int e0 = 32 * c + 2 * e;
                         const float a0 = ((okw[c] >> (2 * e)) & 1u) ? tc::ex2(fmaf(__uint_as_float(sv[e0]), LOG2E, -m_run))
                                                                     : 0.f;
-                        const float a1 = ((okw[c] >> (2 * e + 1)) & 1u)
-                                             ? tc::ex2(fmaf(__uint_as_float(sv[e0 + 1]), LOG2E, -m_run))
-                                             : 0.f;
+                        // a quarter of the exponentials on the FMA pipe, as in the union tiles
+                        const float x1 = fmaf(__uint_as_float(sv[e0 + 1]), LOG2E, -m_run);
+                        const float a1 = ((okw[c] >> (2 * e + 1)) & 1u) ? ((e & 1) ? tc::ex2_fma(x1) : tc::ex2(x1))
+                                                                        : 0.f;
                         a4[e & 3] += a0 + a1;
                         pk[e] = tc::pack_bf16x2(a0, a1);
                     }

@@ -99,6 +99,46 @@ __device__ __forceinline__ uint32_t kth_ordered_key(const float* st, int nblk, i
     return thr;
 }
 
+// Two canonical scores of the same tile at once (blocks ka and kb, each given as the
+// lane's residue segment): the same operations as canonical_dot4, interleaved so that
+// each lane has two independent chains in flight.
+template <int D>
+__device__ __forceinline__ void canonical_dot4x2(const float (&q)[D / 4], const float* __restrict__ ka,
+                                                 const float* __restrict__ kb, float& sa, float& sb) {
+    constexpr int H = D / 8;
+    float a[H], b[H];
+    const float4* ka4 = reinterpret_cast<const float4*>(ka);
+    const float4* kb4 = reinterpret_cast<const float4*>(kb);
+#pragma unroll
+    for (int m = 0; m < H / 4; ++m) {
+        const float4 alo = ka4[m], ahi = ka4[H / 4 + m];
+        const float4 blo = kb4[m], bhi = kb4[H / 4 + m];
+        a[4 * m + 0] = __fadd_rn(__fmul_rn(q[4 * m + 0], alo.x), __fmul_rn(q[H + 4 * m + 0], ahi.x));
+        b[4 * m + 0] = __fadd_rn(__fmul_rn(q[4 * m + 0], blo.x), __fmul_rn(q[H + 4 * m + 0], bhi.x));
+        a[4 * m + 1] = __fadd_rn(__fmul_rn(q[4 * m + 1], alo.y), __fmul_rn(q[H + 4 * m + 1], ahi.y));
+        b[4 * m + 1] = __fadd_rn(__fmul_rn(q[4 * m + 1], blo.y), __fmul_rn(q[H + 4 * m + 1], bhi.y));
+        a[4 * m + 2] = __fadd_rn(__fmul_rn(q[4 * m + 2], alo.z), __fmul_rn(q[H + 4 * m + 2], ahi.z));
+        b[4 * m + 2] = __fadd_rn(__fmul_rn(q[4 * m + 2], blo.z), __fmul_rn(q[H + 4 * m + 2], bhi.z));
+        a[4 * m + 3] = __fadd_rn(__fmul_rn(q[4 * m + 3], alo.w), __fmul_rn(q[H + 4 * m + 3], ahi.w));
+        b[4 * m + 3] = __fadd_rn(__fmul_rn(q[4 * m + 3], blo.w), __fmul_rn(q[H + 4 * m + 3], bhi.w));
+    }
+#pragma unroll
+    for (int h = H / 2; h >= 1; h >>= 1) {
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            a[i] = __fadd_rn(a[i], a[i + h]);
+            b[i] = __fadd_rn(b[i], b[i + h]);
+        }
+    }
+    float va = a[0], vb = b[0];
+    const float pa = __shfl_down_sync(0xffffffffu, va, 2), pb = __shfl_down_sync(0xffffffffu, vb, 2);
+    va = __fadd_rn(va, pa);  // h = 2
+    vb = __fadd_rn(vb, pb);
+    const float ra = __shfl_down_sync(0xffffffffu, va, 1), rb = __shfl_down_sync(0xffffffffu, vb, 1);
+    sa = __fadd_rn(va, ra);  // h = 1
+    sb = __fadd_rn(vb, rb);
+}
+
 template <int D>
 struct SelectCfg {
     static constexpr int THREADS = 256;
@@ -203,11 +243,21 @@ __global__ void __launch_bounds__(256, 3) select_kernel(const T* __restrict__ q,
             seg[3 * C::SEG] = v.w;
         }
         __syncthreads();
-        for (int jj = wpart; jj < nj; jj += wsplit) {
-            float s = canonical_dot4<D>(qr, kst + (jj * 4 + r) * C::SEG, r);
+        // two blocks per iteration (jj and jj + wsplit) for two independent chains a lane
+        for (int jj = wpart; jj < nj; jj += 2 * wsplit) {
+            const int jj2 = jj + wsplit;
+            const bool two = jj2 < nj;
+            float s, s2;
+            canonical_dot4x2<D>(qr, kst + (jj * 4 + r) * C::SEG, kst + ((two ? jj2 : jj) * 4 + r) * C::SEG, s, s2);
             // covariance-aware routing: one fp32 add of the block's bias
-            if (bias) s = __fadd_rn(s, __ldg(bias + (size_t)bh * nblk + j0 + jj));
-            if (live && r == 0) sc[t * SS + j0 + jj] = s;
+            if (bias) {
+                s = __fadd_rn(s, __ldg(bias + (size_t)bh * nblk + j0 + jj));
+                if (two) s2 = __fadd_rn(s2, __ldg(bias + (size_t)bh * nblk + j0 + jj2));
+            }
+            if (live && r == 0) {
+                sc[t * SS + j0 + jj] = s;
+                if (two) sc[t * SS + j0 + jj2] = s2;
+            }
         }
         __syncthreads();
     }

@@ -50,6 +50,7 @@ struct StatsTcCfg {
     static constexpr uint32_t SMEM = KB_OFF + 4 * D * 4 + 1024;
     static constexpr int THREADS = 320;                         // producer, MMA, eight epilogue warps
     static_assert(NSTG >= 2, "the statistics kernel needs two stages");
+    static_assert(KB_OFF % 16 == 0, "kbar and vsum are read as 16-byte vectors");
     static_assert(SMEM <= 232448, "shared memory over the per-CTA limit");
 };
 
@@ -213,9 +214,16 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
             if (ct < 2 * D) {
                 const bool is_k = ct < D;
                 const int c = is_k ? ct : ct - D;
+                // element (n, c) of the swizzled tile: box c / 64, row n, 16-byte chunk
+                // ((c % 64) / 8) ^ (n % 8), so eight per-thread offsets cover every row
+                const uint8_t* col = st + (is_k ? C::TILE_BYTES : 0u) + (c >> 6) * C::BOX_BYTES + (c & 7) * 2;
+                uint32_t off[8];
+#pragma unroll
+                for (int k8 = 0; k8 < 8; ++k8) off[k8] = (uint32_t)((((c & 63) >> 3) ^ k8) << 4);
                 float a[BS];
 #pragma unroll
-                for (int n = 0; n < BS; ++n) a[n] = swz_elem<BS>(st + (is_k ? C::TILE_BYTES : 0u), n, c);
+                for (int n = 0; n < BS; ++n)
+                    a[n] = __bfloat162float(*reinterpret_cast<const bf16*>(col + n * 128 + off[n & 7]));
                 const size_t so = (size_t)blk * D + c;
                 if (is_k) {
                     const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
@@ -264,18 +272,24 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
                         tc::tmem_ld32(taddr + (uint32_t)(part * 128 + col0 + c0), raw);
                         tc::tmem_wait_ld();
                         uint32_t pk[16];
+                        const float4* kb4 = reinterpret_cast<const float4*>(kb + col0 + c0);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int cc = col0 + c0 + 2 * e;
-                            float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
-                            if (h_here) {
-                                x0 = fmaf(-rv, kb[cc], x0);
-                                x1 = fmaf(-rv, kb[cc + 1], x1);
-                            } else {
-                                x0 = fmaf(-rv, kb[cc], x0 * inv_b);
-                                x1 = fmaf(-rv, kb[cc + 1], x1 * inv_b);
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 kv = kb4[e4];  // kbar of the four columns (a broadcast read)
+                            const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                            for (int e2 = 0; e2 < 2; ++e2) {
+                                const int e = 2 * e4 + e2;
+                                float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
+                                if (h_here) {
+                                    x0 = fmaf(-rv, kk[2 * e2], x0);
+                                    x1 = fmaf(-rv, kk[2 * e2 + 1], x1);
+                                } else {
+                                    x0 = fmaf(-rv, kk[2 * e2], x0 * inv_b);
+                                    x1 = fmaf(-rv, kk[2 * e2 + 1], x1 * inv_b);
+                                }
+                                pk[e] = tc::pack_bf16x2(x0, x1);
                             }
-                            pk[e] = tc::pack_bf16x2(x0, x1);
                         }
                         // row `lane` of the box, 16-byte chunks c0/8 .. c0/8 + 3, swizzled
                         const uint32_t rowa = stg + (uint32_t)part * 4096u + (uint32_t)lane * 128u;
