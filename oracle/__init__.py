@@ -46,8 +46,8 @@ def lib():
         L.oracle_centroids_f32.argtypes = [f32p, li, li, li, li, ctypes.c_void_p, ctypes.c_int]
         L.oracle_dense_attention.argtypes = [f32p, f32p, f32p, li, li, li, f64p, ctypes.c_int]
         L.oracle_pisa_backward.argtypes = [f32p, f32p, f32p, f32p, ctypes.c_void_p, li, li, li, li, li,
-                                           ctypes.c_int, ctypes.c_int, ctypes.c_float, f64p, f64p, f64p,
-                                           ctypes.c_int]
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, f64p, f64p,
+                                           f64p, ctypes.c_int]
         L.oracle_pisa_backward_dq_rows.argtypes = [f32p, f32p, f32p, f32p, ctypes.c_void_p, li, li, li, li, li,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, li,
                                                    f64p, ctypes.c_int]
@@ -217,12 +217,14 @@ def pisa_bruteforce(q, k, v, B, K, order=1, gate=True, nthreads=None):
     return out
 
 
-def pisa_backward(q, k, v, dO, B, K, order=1, gate=True, route_eps=None, nthreads=None, o=None):
+def pisa_backward(q, k, v, dO, B, K, order=1, gate=True, route_eps=None, nthreads=None, o=None, w_pooled=False):
     """(dq, dk, dv) [BH, L, d] fp64: gradients of sum_t dO_t . o_t for pisa_attention's
     output o, with the block selection held fixed (``route_eps``: the covariance-aware
     selection, as in pisa_attention_ex).  ``o``: None (delta_t = dO_t . o_t from the
     recomputed fp64 output) or the forward output the caller holds ([BH, L, d], taken as
-    fp32), as a backward operator of (q, k, v, o, dO) receives it."""
+    fp32), as a backward operator of (q, k, v, o, dO) receives it.  ``w_pooled`` (order 2):
+    the output of pisa_attention_ex(..., w_pooled=True), PWT's diagonal + pooled w, with its
+    gate decisions held fixed."""
     q, k, v, dO = _f32(q), _f32(k), _f32(v), _f32(dO)
     BH, L, d = q.shape
     og = None if o is None else _f32(o)
@@ -230,8 +232,9 @@ def pisa_backward(q, k, v, dO, B, K, order=1, gate=True, route_eps=None, nthread
         raise ValueError("o must have q's shape")
     dq, dk, dv = (np.zeros((BH, L, d)) for _ in range(3))
     reps = float(route_eps) if route_eps else 0.0
-    rc = lib().oracle_pisa_backward(q, k, v, dO, _ptr(og), BH, L, d, B, K, int(order), int(bool(gate)), reps,
-                                    _ptr(dq), _ptr(dk), _ptr(dv), nthreads or default_threads())
+    rc = lib().oracle_pisa_backward(q, k, v, dO, _ptr(og), BH, L, d, B, K, int(order), int(bool(gate)),
+                                    int(bool(w_pooled)), reps, _ptr(dq), _ptr(dk), _ptr(dv),
+                                    nthreads or default_threads())
     _check(rc, "pisa_backward")
     return dq, dk, dv
 

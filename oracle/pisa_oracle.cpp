@@ -436,9 +436,13 @@ void backward_prep(const float* q, const float* k, const float* v, long L, long 
 // the caller holds, as a backward operator of (q, k, v, o, dO) receives it;
 // delta = dO_t . o_t then uses its row t instead of the recomputed o_t (the
 // only place o enters the gradient).
+// wpool (null, or [nblk]): the pooled second-order w of this row's tile per block (PWT's
+// diagonal + pooled variant, already gated), which replaces the row's own w; it does not
+// depend on the row's logits, so dl/dx_n is 1/B.  dlj (with wpool, [nblk]) receives
+// dL/dl_tj = (E/D) inner for the unselected blocks (0 for the selected ones).
 void backward_row(const float* q, const float* k, const float* v, const float* dO, const float* o_given, long L,
                   long d, long B, const uint32_t* mask, const double* kbar, int order, int gate, long t, double* gx,
-                  double* pw) {
+                  double* pw, const double* wpool = nullptr, double* dlj = nullptr) {
     const long nblk = L / B;
     const long words = (nblk + 31) / 32;
     const long i = t / B;
@@ -463,12 +467,17 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
         double sb = 0.0;
         for (long c = 0; c < d; ++c) sb += (double)qt[c] * kbar[j * d + c];
         double w = 0.0;
-        if (order == 2) {
-            for (long n = j * B; n < (j + 1) * B; ++n) w += (x[n] - sb) * (x[n] - sb);
-            w /= 2.0 * (double)B;
+        if (order == 2 && wpool) {
+            w = wpool[j];
+            open[j] = 0;  // no per-row dependence of w on the logits
+        } else {
+            if (order == 2) {
+                for (long n = j * B; n < (j + 1) * B; ++n) w += (x[n] - sb) * (x[n] - sb);
+                w /= 2.0 * (double)B;
+            }
+            open[j] = !(gate && w > ln_b);
+            if (!open[j]) w = 0.0;
         }
-        open[j] = !(gate && w > ln_b);
-        if (!open[j]) w = 0.0;
         sbj[j] = sb;
         lj[j] = sb + w;
         m = std::max(m, lj[j]);
@@ -502,6 +511,7 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
         const bool sel = (mask[i * words + j / 32] >> (j % 32)) & 1u;
         if (sel) {
             for (long n = j * B; n < (j + 1) * B; ++n) gx[n] = wt[n] * (G[n] - delta) / D;
+            if (dlj) dlj[j] = 0.0;
             continue;
         }
         const double E = std::exp(lj[j] - m);
@@ -512,6 +522,7 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
         }
         gbar /= (double)B;
         const double inner = sg - (double)B * delta;
+        if (dlj) dlj[j] = (E / D) * inner;
         for (long n = j * B; n < (j + 1) * B; ++n) {
             double dl = 1.0 / (double)B;
             if (order == 2 && open[j]) dl += (x[n] - sbj[j]) / (double)B;
@@ -521,20 +532,72 @@ void backward_row(const float* q, const float* k, const float* v, const float* d
 }
 
 void backward_one(const float* q, const float* k, const float* v, const float* dO, const float* o_given, long L,
-                  long d, long B, long K, int order, int gate, float route_eps, double* dq, double* dk, double* dv) {
+                  long d, long B, long K, int order, int gate, int w_pooled, float route_eps, double* dq, double* dk,
+                  double* dv) {
     std::vector<uint32_t> mask;
     std::vector<double> kbar, gx(L), pw(L);
     backward_prep(q, k, v, L, d, B, K, route_eps, mask, kbar);
-    for (long t = 0; t < L; ++t) {
-        backward_row(q, k, v, dO, o_given, L, d, B, mask.data(), kbar.data(), order, gate, t, gx.data(),
-                     pw.data());
-        const float* qt = q + t * d;
-        const float* dOt = dO + t * d;
-        for (long n = 0; n < L; ++n) {
+    const long nblk = L / B;
+    const bool pooled = order == 2 && w_pooled;
+    // PWT's pooled w (the forward's definition): w_ij = 1/2 sum_c q2_ic sigma2_jc, with
+    // q2_ic the tile mean of q_c^2 and sigma2_jc = C_j[c][c] the block's channel variance,
+    // gated at ln B.  It is shared by the tile's rows, so its gradient gathers
+    // W_ij = sum_{t in tile i} dL/dl_tj over them, then reaches q through q2 and k through
+    // sigma2:  dq_mc += W_ij sigma2_jc q_mc / B,  dk_nc += W_ij q2_ic (k_nc - kbar_jc) / B.
+    std::vector<double> sig2, q2(d), wp(nblk), dlj(nblk), W(nblk);
+    std::vector<char> keep(nblk);
+    if (pooled) {
+        sig2.assign(nblk * d, 0.0);
+        for (long j = 0; j < nblk; ++j)
             for (long c = 0; c < d; ++c) {
-                dq[t * d + c] += gx[n] * (double)k[n * d + c];
-                dk[n * d + c] += gx[n] * (double)qt[c];
-                dv[n * d + c] += pw[n] * (double)dOt[c];
+                double s2 = 0.0;
+                for (long n = j * B; n < (j + 1) * B; ++n) {
+                    const double u = (double)k[n * d + c] - kbar[j * d + c];
+                    s2 += u * u;
+                }
+                sig2[j * d + c] = s2 / (double)B;
+            }
+    }
+    const double ln_b = std::log((double)B);
+    for (long i = 0; i < nblk; ++i) {
+        if (pooled) {
+            std::fill(q2.begin(), q2.end(), 0.0);
+            for (long m = i * B; m < (i + 1) * B; ++m)
+                for (long c = 0; c < d; ++c) q2[c] += (double)q[m * d + c] * (double)q[m * d + c];
+            for (long c = 0; c < d; ++c) q2[c] /= (double)B;
+            for (long j = 0; j < nblk; ++j) {
+                double w = 0.0;
+                for (long c = 0; c < d; ++c) w += q2[c] * sig2[j * d + c];
+                w *= 0.5;
+                keep[j] = !(gate && w > ln_b);
+                wp[j] = keep[j] ? w : 0.0;
+                W[j] = 0.0;
+            }
+        }
+        for (long t = i * B; t < (i + 1) * B; ++t) {
+            backward_row(q, k, v, dO, o_given, L, d, B, mask.data(), kbar.data(), order, gate, t, gx.data(),
+                         pw.data(), pooled ? wp.data() : nullptr, pooled ? dlj.data() : nullptr);
+            const float* qt = q + t * d;
+            const float* dOt = dO + t * d;
+            for (long n = 0; n < L; ++n) {
+                for (long c = 0; c < d; ++c) {
+                    dq[t * d + c] += gx[n] * (double)k[n * d + c];
+                    dk[n * d + c] += gx[n] * (double)qt[c];
+                    dv[n * d + c] += pw[n] * (double)dOt[c];
+                }
+            }
+            if (pooled)
+                for (long j = 0; j < nblk; ++j)
+                    if (keep[j]) W[j] += dlj[j];
+        }
+        if (pooled) {
+            for (long j = 0; j < nblk; ++j) {
+                if (!keep[j] || W[j] == 0.0) continue;
+                for (long m = i * B; m < (i + 1) * B; ++m)
+                    for (long c = 0; c < d; ++c) dq[m * d + c] += W[j] * sig2[j * d + c] * (double)q[m * d + c] / (double)B;
+                for (long n = j * B; n < (j + 1) * B; ++n)
+                    for (long c = 0; c < d; ++c)
+                        dk[n * d + c] += W[j] * q2[c] * ((double)k[n * d + c] - kbar[j * d + c]) / (double)B;
             }
         }
     }
@@ -768,10 +831,11 @@ int oracle_pisa_bruteforce(const float* q, const float* k, const float* v, long 
 // Gradients (dq, dk, dv) [BH, L, d] fp64 of sum_t dO_t . o_t for the method's
 // output o (pisa_attention's), selection held fixed.  Zero-initialised here.
 // o_given: null (delta from the recomputed fp64 o) or [BH, L, d], the forward
-// output the caller holds (delta = dO_t . o_given_t).
+// output the caller holds (delta = dO_t . o_given_t).  w_pooled (order 2): the
+// gradient of PWT's diagonal + pooled w, the gate decisions held fixed.
 int oracle_pisa_backward(const float* q, const float* k, const float* v, const float* dO, const float* o_given,
-                         long BH, long L, long d, long B, long K, int order, int gate, float route_eps, double* dq,
-                         double* dk, double* dv, int nthreads) {
+                         long BH, long L, long d, long B, long K, int order, int gate, int w_pooled, float route_eps,
+                         double* dq, double* dk, double* dv, int nthreads) {
     if (!is_pow2(B) || !is_pow2(d) || L % B || order < 0 || order > 2) return -1;
     if (K < 0 || K > L / B) return -1;
     std::fill(dq, dq + BH * L * d, 0.0);
@@ -779,8 +843,8 @@ int oracle_pisa_backward(const float* q, const float* k, const float* v, const f
     std::fill(dv, dv + BH * L * d, 0.0);
     parallel_for(BH, nthreads, [&](long bh) {
         const long o = bh * L * d;
-        backward_one(q + o, k + o, v + o, dO + o, o_given ? o_given + o : nullptr, L, d, B, K, order, gate, route_eps,
-                     dq + o, dk + o, dv + o);
+        backward_one(q + o, k + o, v + o, dO + o, o_given ? o_given + o : nullptr, L, d, B, K, order, gate, w_pooled,
+                     route_eps, dq + o, dk + o, dv + o);
     });
     return 0;
 }

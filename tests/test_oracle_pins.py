@@ -715,3 +715,58 @@ def test_backward_with_a_given_forward_output():
     np.testing.assert_allclose(gb[0] - ga[0], -e[..., None] * (P @ k64), rtol=0, atol=1e-11)
     np.testing.assert_allclose(gb[1] - ga[1], -np.einsum("bt,btn,btc->bnc", e, P, q64), rtol=0, atol=1e-11)
     np.testing.assert_array_equal(gb[2], ga[2])
+
+
+@pytest.mark.parametrize("gate", [True, False])
+def test_pooled_w_backward_matches_central_differences(gate):
+    # PWT's diagonal + pooled w (one w per query tile and block, from the tile mean of q^2
+    # and the block's channel variances): its gradient reaches q and k through w as well;
+    # coordinates whose perturbation changes the selection or a gate decision are skipped
+    L, d, B, K = 64, 4, 16, 2
+    q, k, v = _dyadic_qkv(131, L, d)
+    q *= 2.0
+    k *= 2.0
+    dO = _dyadic_qkv(137, L, d)[0]
+    gq, gk, gv = oracle.pisa_backward(q, k, v, dO, B, K, 2, gate, w_pooled=True)
+    _, mask0, _ = oracle.select(q, k, B, K)
+    h = 2.0 ** -10
+
+    def kept(q_, k_):
+        # which (tile, block) pooled w pass the ln B gate (numpy, from the definition)
+        q64, k64 = q_[0].astype(np.float64), k_[0].astype(np.float64)
+        q2 = (q64.reshape(-1, B, d) ** 2).mean(axis=1)
+        kb = k64.reshape(-1, B, d)
+        sig2 = ((kb - kb.mean(axis=1, keepdims=True)) ** 2).mean(axis=1)
+        return 0.5 * q2 @ sig2.T <= math.log(B)
+
+    keep0 = kept(q, k)
+    if gate:
+        assert 0 < keep0.sum() < keep0.size  # both branches of the gate are exercised
+
+    def loss(q_, k_, v_):
+        return float((oracle.pisa_attention_ex(q_, k_, v_, B, K, 2, gate=gate, w_pooled=True) * dO).sum())
+
+    # the pooled term moves the gradient: without it dq and dk differ
+    gq_exact = oracle.pisa_backward(q, k, v, dO, B, K, 2, gate)[0]
+    assert oracle.rel_l2(gq_exact, gq) > 1e-3
+    rng = np.random.default_rng(9)
+    checked = 0
+    for name, x, g in (("q", q, gq), ("k", k, gk), ("v", v, gv)):
+        for _ in range(24):
+            idx = (0, int(rng.integers(L)), int(rng.integers(d)))
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            if name != "v":
+                if not (np.array_equal(oracle.select(args_p[0], args_p[1], B, K)[1], mask0) and
+                        np.array_equal(oracle.select(args_m[0], args_m[1], B, K)[1], mask0)):
+                    continue
+                if gate and not (np.array_equal(kept(args_p[0], args_p[1]), keep0) and
+                                 np.array_equal(kept(args_m[0], args_m[1]), keep0)):
+                    continue
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - g[idx]) <= 2e-5 * max(1.0, abs(g[idx])), (name, idx, fd, g[idx])
+            checked += 1
+    assert checked >= 45
