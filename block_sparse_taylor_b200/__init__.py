@@ -364,12 +364,12 @@ def pisa_backward_workspace_bytes(batch, heads, L, d, B, K, order, dtype: torch.
 def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
                             B: int, K: int, order: int = 1, gate: bool = True, route: str = "centroid",
                             grads: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None, stream=None,
-                            lse: Optional[torch.Tensor] = None):
+                            lse: Optional[torch.Tensor] = None, w_mode: str = "exact"):
     """(dq, dk, dv) fp32, the gradients of sum(dO * o) for o = pisa_attention(q, k, v, B, K, order,
-    gate=gate, route=route) on the per-block paths, the selection held fixed.  ``o`` is that
-    forward's output; ``lse`` optionally its log-denominators (pisa_attention_lse), which spares
-    the backward its own pass for the row statistics; ``grads`` optional preallocated fp32
-    (dq, dk, dv)."""
+    gate=gate, route=route, w_mode=w_mode) on the per-block paths, the selection held fixed.
+    ``o`` is that forward's output; ``lse`` optionally its log-denominators (pisa_attention_lse),
+    which spares the backward its own pass for the row statistics (the pooled w, order 2,
+    requires it); ``grads`` optional preallocated fp32 (dq, dk, dv)."""
     _need_cuda(q, k, v, o, dO)
     if not (q.shape == k.shape == v.shape == o.shape == dO.shape
             and q.dtype == k.dtype == v.dtype == o.dtype == dO.dtype):
@@ -390,7 +390,7 @@ def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     dq, dk, dv = grads
     if lse is None:
         _check(lib().pisa_attention_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(),
-                                             batch, heads, L, d, code, B, K, order, _flags(gate, "exact", route),
+                                             batch, heads, L, d, code, B, K, order, _flags(gate, w_mode, route),
                                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
                                              workspace.numel(), _stream(stream)))
     else:
@@ -399,7 +399,7 @@ def pisa_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
             raise ValueError("lse must be fp32 with batch*heads*L elements")
         _check(lib().pisa_attention_backward_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                                  dO.data_ptr(), lse.data_ptr(), batch, heads, L, d, code, B, K, order,
-                                                 _flags(gate, "exact", route), dq.data_ptr(), dk.data_ptr(),
+                                                 _flags(gate, w_mode, route), dq.data_ptr(), dk.data_ptr(),
                                                  dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                                  _stream(stream)))
     return dq, dk, dv
@@ -410,28 +410,30 @@ class PisaAttentionFunction(torch.autograd.Function):
     pisa_attention_backward (selection held fixed); gradients are returned in the inputs' dtype."""
 
     @staticmethod
-    def forward(ctx, q, k, v, B, K, order, gate, path, route):
-        out, lse = pisa_attention_lse(q, k, v, B, K, order, gate=gate, path=path, route=route)
+    def forward(ctx, q, k, v, B, K, order, gate, path, route, w_mode):
+        out, lse = pisa_attention_lse(q, k, v, B, K, order, gate=gate, path=path, route=route, w_mode=w_mode)
         ctx.save_for_backward(q, k, v, out, lse)
-        ctx.cfg = (B, K, order, gate, route)
+        ctx.cfg = (B, K, order, gate, route, w_mode)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
-        B, K, order, gate, route = ctx.cfg
+        B, K, order, gate, route, w_mode = ctx.cfg
         dq, dk, dv = pisa_attention_backward(q, k, v, out, dout.contiguous(), B, K, order, gate=gate, route=route,
-                                             lse=lse)
-        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None, None, None, None
+                                             lse=lse, w_mode=w_mode)
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None, None, None, None, None
 
 
 def pisa_attention_autograd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,
-                            gate: bool = True, path: str = "auto", route: str = "centroid") -> torch.Tensor:
+                            gate: bool = True, path: str = "auto", route: str = "centroid",
+                            w_mode: str = "exact") -> torch.Tensor:
     """pisa_attention with gradients for training (the per-block paths: "auto", "recompute_tc",
-    "stats"; exact w).  The backward holds the block selection fixed."""
+    "stats", "stats_tc"; exact w, or PWT's pooled w at order 2 on the tensor-core shapes).  The
+    backward holds the block selection (and the gate decisions) fixed."""
     if path == "hybrid_tc":
         raise PisaError(PISA_ERR_UNSUPPORTED, "no backward for the hybrid path")
-    return PisaAttentionFunction.apply(q, k, v, B, K, order, gate, path, route)
+    return PisaAttentionFunction.apply(q, k, v, B, K, order, gate, path, route, w_mode)
 
 
 def pisa_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B: int, K: int, order: int = 1,

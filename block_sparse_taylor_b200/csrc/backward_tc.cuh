@@ -159,11 +159,14 @@ __device__ __forceinline__ void chunk_ds(const uint32_t (&xs)[32], const uint32_
 }
 
 // Per-block coefficients from the sums: sb (mean logit), a = e^{l - lse} (l = sb + w),
-// and dS_n = A G_n + X u_n + Cc, P_n = a + Pu u_n for an unselected block (u_n = x_n - sb).
+// and dS_n = A G_n + X u_n + Cc, P_n = a + Pu u_n for an unselected block (u_n = x_n - sb);
+// `inner` = sum_n G_n (1 + c1 u_n) - B delta, so that dL/dl = a inner.  ORDER 3 is the first
+// order with PWT's pooled w (wp, the tile's gated value for this block): it does not depend
+// on the row's logits, so dl_n = 1/B.
 template <int BS, int ORDER>
 __device__ __forceinline__ void block_coefs(float x0, float s1, float s2, float sg, float sgd, float lse2, float del,
-                                            int gate, float ln_b, float& sb, float& a, float& A, float& X,
-                                            float& Cc, float& Pu) {
+                                            int gate, float ln_b, float wp, float& sb, float& a, float& A, float& X,
+                                            float& Cc, float& Pu, float& inner) {
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr float INV_B = 1.0f / (float)BS;
     constexpr float C1 = ORDER >= 1 ? 1.f : 0.f;
@@ -179,10 +182,12 @@ __device__ __forceinline__ void block_coefs(float x0, float s1, float s2, float 
         } else {
             q2 = INV_B;
         }
+    } else if (ORDER == 3) {
+        w = wp;
     }
     a = tc::ex2((sb + w) * LOG2E - lse2);
     const float sgu = fmaf(-md, sg, sgd);  // sum G (x - sb)
-    const float inner = sg + C1 * sgu - (float)BS * del;
+    inner = sg + C1 * sgu - (float)BS * del;
     // dS_n = a (dl_n inner + c1 (G_n - mean G)),  dl_n = 1/B (+ q2 u_n)
     A = a * C1;
     X = a * q2 * inner;
@@ -196,7 +201,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const uint32_t* __restrict__ mask, const float* __restrict__ lse,
                      const float* __restrict__ delta, float* __restrict__ dq, int L, int nblk, int words, int gate,
-                     unsigned* status) {
+                     unsigned* status, const float* __restrict__ wmat, float* __restrict__ wpart) {
+    // ORDER 3 (first order + PWT's pooled w): wmat [BH, nblk, nblk] the gated w of each (query
+    // tile, block); wpart [BH, L / 32, nblk] receives, per 32 query rows and block, the sum of
+    // dL/dl over those rows (0 for selected blocks and blocks whose w is 0), the pooled w's
+    // gradient before it reaches q and k
     using C = DqCfg<D>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);  // S = Q K^T, G = dO V^T
@@ -426,8 +435,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 hs.sg += __uint_as_float(other[2]);
                 hs.sgd += __uint_as_float(other[3]);
             }
-            float sb, a, A, X, Cc, Pu;
-            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, sb, a, A, X, Cc, Pu);
+            float sb, a, A, X, Cc, Pu, inner;
+            const float wp = (ORDER == 3) ? __ldg(wmat + ((size_t)bh * nblk + qt) * nblk + jb) : 0.f;
+            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, wp, sb, a, A, X, Cc, Pu,
+                                   inner);
+            if (ORDER == 3) {
+                float gw = (!sel && valid && wp > 0.f) ? a * inner : 0.f;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) gw += __shfl_xor_sync(0xffffffffu, gw, o);
+                if (lane == 0 && (BS == 64 || half == 0))
+                    wpart[((size_t)bh * (L / 32) + (q0 / 32 + quarter)) * nblk + jb] = gw;
+            }
             // dS (bf16) over the first 32 columns of this half: keys 2e and 2e + 1 in column e
             {
                 uint32_t pp[16], dd[16];
@@ -536,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const uint32_t* __restrict__ mask, const float* __restrict__ lse,
                        const float* __restrict__ delta, float* __restrict__ dk, float* __restrict__ dv, int L,
-                       int nblk, int words, int gate, unsigned* status) {
+                       int nblk, int words, int gate, unsigned* status, const float* __restrict__ wmat) {
     using C = DkvCfg<D, BS>;
     constexpr float LOG2E = 1.4426950408889634f;
     constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false);
@@ -770,8 +788,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 hs.sg += o.z;
                 hs.sgd += o.w;
             }
-            float sb, a, A, X, Cc, Pu;
-            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, sb, a, A, X, Cc, Pu);
+            float sb, a, A, X, Cc, Pu, inner;
+            const float wp = (ORDER == 3) ? __ldg(wmat + ((size_t)bh * nblk + qt) * nblk + jb) : 0.f;
+            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, wp, sb, a, A, X, Cc, Pu,
+                                   inner);
             // the previous tile's dK and dV products have read P and dS
             if (i > 0 && !tc::mbar_wait_warp(bar(B_PFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) break;
             // row r of P and dS (bf16), this half's 64 keys = box `half` of each tile, 32 keys a chunk
@@ -823,6 +843,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// The pooled w's gradient into dq and dk (after the dq and dk/dv kernels).  With W_ij the
+// sum over query tile i's rows of dL/dl_tj (wpart, per 32 rows) on the blocks whose w was
+// kept (wmat > 0), w_ij = 1/2 sum_c q2_ic var_jc gives
+//   dq_mc += q_mc u_ic / B,   u_ic = sum_j W_ij var_jc          (rows m of tile i)
+//   dk_nc += (k_nc - kbar_jc) z_jc / B,  z_jc = sum_i W_ij q2_ic  (keys n of block j)
+// Every sum runs in a fixed order, so the result is the same on every run.
+// bwd_pooled_dq_kernel: one CTA per (tile i, bh), 128 threads; also writes W (wsum).
+template <int D, int BS>
+__global__ void __launch_bounds__(128) bwd_pooled_dq_kernel(const bf16* __restrict__ q, const float* __restrict__ wmat,
+                                                            const float* __restrict__ wpart,
+                                                            const float* __restrict__ var, float* __restrict__ wsum,
+                                                            float* __restrict__ dq, int L, int nblk) {
+    extern __shared__ float ws_row[];  // [nblk]
+    const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    constexpr int CPT = BS / 32;  // 32-row chunks per query tile
+    const float* wr = wmat + ((size_t)bh * nblk + i) * nblk;
+    for (int j = tid; j < nblk; j += 128) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) s += wpart[((size_t)bh * (L / 32) + i * CPT + c) * nblk + j];
+        s = wr[j] > 0.f ? s : 0.f;
+        ws_row[j] = s;
+        wsum[((size_t)bh * nblk + i) * nblk + j] = s;
+    }
+    __syncthreads();
+    if (tid >= D) return;
+    float u = 0.f;
+    const float* vb = var + (size_t)bh * nblk * D + tid;
+    for (int j = 0; j < nblk; ++j) u = fmaf(ws_row[j], vb[(size_t)j * D], u);
+    u *= 1.0f / (float)BS;
+    for (int m = 0; m < BS; ++m) {
+        const size_t e = ((size_t)bh * L + (size_t)i * BS + m) * D + tid;
+        dq[e] = fmaf(__bfloat162float(q[e]), u, dq[e]);
+    }
+}
+
+// bwd_pooled_dk_kernel: one CTA per (block j, bh), 128 threads.
+template <int D, int BS>
+__global__ void __launch_bounds__(128) bwd_pooled_dk_kernel(const bf16* __restrict__ k, const float* __restrict__ kbar,
+                                                            const float* __restrict__ wsum,
+                                                            const float* __restrict__ q2, float* __restrict__ dk,
+                                                            int L, int nblk) {
+    const int j = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    if (tid >= D) return;
+    float z = 0.f;
+    const float* wc = wsum + (size_t)bh * nblk * nblk + j;
+    const float* qb = q2 + (size_t)bh * nblk * D + tid;
+    for (int i = 0; i < nblk; ++i) z = fmaf(wc[(size_t)i * nblk], qb[(size_t)i * D], z);
+    z *= 1.0f / (float)BS;
+    const float kb = kbar[((size_t)bh * nblk + j) * D + tid];
+    for (int n = 0; n < BS; ++n) {
+        const size_t e = ((size_t)bh * L + (size_t)j * BS + n) * D + tid;
+        dk[e] = fmaf(__bfloat162float(k[e]) - kb, z, dk[e]);
     }
 }
 

@@ -377,10 +377,13 @@ pisa_path resolve(const Dims& g, int K, int order, pisa_dtype dtype) {
 // backward pass: workspace layout and launches
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-    size_t kbar, bias, mask, mstat, dinv, delta, lse, total;
+    size_t kbar, bias, mask, mstat, dinv, delta, lse;
+    // order 2 only: PWT's pooled w and its gradient (var, q2 [BH, nblk, d]; wmat, wsum
+    // [BH, nblk, nblk]; wpart [BH, L / 32, nblk])
+    size_t var, q2, wmat, wsum, wpart, total;
 };
 
-BwdLayout bwd_layout(const Dims& g) {
+BwdLayout bwd_layout(const Dims& g, int order) {
     BwdLayout w{};
     size_t o = 0;
     w.kbar = o;
@@ -397,6 +400,19 @@ BwdLayout bwd_layout(const Dims& g) {
     o += align_up(sizeof(float) * g.BH * g.L);
     w.lse = o;
     o += align_up(sizeof(float) * g.BH * g.L);
+    w.var = w.q2 = w.wmat = w.wsum = w.wpart = 0;
+    if (order == 2) {
+        w.var = o;
+        o += align_up(sizeof(float) * g.BH * g.nblk * g.d);
+        w.q2 = o;
+        o += align_up(sizeof(float) * g.BH * g.nblk * g.d);
+        w.wmat = o;
+        o += align_up(sizeof(float) * g.BH * g.nblk * g.nblk);
+        w.wsum = o;
+        o += align_up(sizeof(float) * g.BH * g.nblk * g.nblk);
+        w.wpart = o;
+        o += align_up(sizeof(float) * g.BH * (g.L / 32) * g.nblk);
+    }
     w.total = o;
     return w;
 }
@@ -406,7 +422,8 @@ BwdLayout bwd_layout(const Dims& g) {
 pisa_status run_backward_tc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                             const uint32_t* mask, const Dims& g, int order, int gate, const float* lse_in,
                             float* mst, float* dinv, float* del, float* lse_ws, float* dq, float* dk, float* dv,
-                            cudaStream_t s) {
+                            cudaStream_t s, const float* wmat = nullptr, float* wpart = nullptr) {
+    // order 3: the first order with PWT's pooled w (wmat), its gradient gathered in wpart
     unsigned int* status = device_status_ptr();
     if (!status) return fail(PISA_ERR_CUDA, "cannot resolve the device status word");
     const long rows = g.BH * g.L;
@@ -475,13 +492,13 @@ pisa_status run_backward_tc(const void* q, const void* k, const void* v, const v
         if (e == cudaSuccess) {                                                                                   \
             kq<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DqCfg<DD>::SMEM, s>>>(                                 \
                 maps[0], maps[1], maps[2], maps[3], mask, lse, del, dq, (int)g.L, (int)g.nblk, (int)g.words, gate,  \
-                status);                                                                                          \
+                status, wmat, wpart);                                                                             \
             e = cudaGetLastError();                                                                               \
         }                                                                                                         \
         if (e == cudaSuccess) {                                                                                   \
             kk<<<grid, pisa::bwdtc::kThreads, pisa::bwdtc::DkvCfg<DD, BB>::SMEM, s>>>(                                \
                 maps[0], maps[1], maps[2], maps[3], mask, lse, del, dk, dv, (int)g.L, (int)g.nblk, (int)g.words,    \
-                gate, status);                                                                                    \
+                gate, status, wmat);                                                                              \
             e = cudaGetLastError();                                                                               \
         }                                                                                                         \
     }
@@ -497,6 +514,10 @@ pisa_status run_backward_tc(const void* q, const void* k, const void* v, const v
     PISA_BWD_TC(128, 128, 0)
     PISA_BWD_TC(128, 128, 1)
     PISA_BWD_TC(128, 128, 2)
+    PISA_BWD_TC(64, 64, 3)
+    PISA_BWD_TC(64, 128, 3)
+    PISA_BWD_TC(128, 64, 3)
+    PISA_BWD_TC(128, 128, 3)
 #undef PISA_BWD_TC
     if (!found) return fail(PISA_ERR_UNSUPPORTED, "no tensor-core backward kernel for this d/B/order");
     if (e != cudaSuccess) return cuda_fail(e, "backward tensor-core kernels");
@@ -826,7 +847,7 @@ size_t pisa_backward_workspace_bytes(int batch, int heads, int L, int d, int B, 
     Dims g;
     if (check_dims(batch, heads, L, d, B, order, dtype, &g) != PISA_OK) return 0;
     if (K < 0 || K > g.nblk || g.BH > 65535) return 0;
-    return bwd_layout(g).total;
+    return bwd_layout(g, order).total;
 }
 
 }  // extern "C"
@@ -844,8 +865,17 @@ pisa_status backward_impl(const void* q, const void* k, const void* v, const voi
     if (g.BH > 65535) return fail(PISA_ERR_UNSUPPORTED, "batch * heads must be <= 65535 (got %ld)", g.BH);
     if (flags & ~(PISA_FLAG_GATE_W | PISA_FLAG_POOLED_W | PISA_FLAG_COV_ROUTE))
         return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: unknown flag bits 0x%x", flags);
-    if (flags & PISA_FLAG_POOLED_W)
-        return fail(PISA_ERR_UNSUPPORTED, "pisa_attention_backward: no backward for the pooled w");
+    const bool pooled = (flags & PISA_FLAG_POOLED_W) != 0;
+    if (pooled && order != 2)
+        return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: the pooled w is an order-2 option");
+    if (pooled && !tc_path_available(g, dtype))
+        return fail(PISA_ERR_UNSUPPORTED,
+                    "pisa_attention_backward: the pooled-w backward runs on the tensor-core path (bf16, d and B in "
+                    "{64, 128}, L a multiple of 128)");
+    if (pooled && !lse)
+        return fail(PISA_ERR_UNSUPPORTED,
+                    "pisa_attention_backward: the pooled-w backward takes the forward's lse "
+                    "(pisa_attention_backward_lse)");
     if (!q || !k || !v || !o || !dO || !dq || !dk || !dv)
         return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: null pointer");
     const void* in16[5] = {q, k, v, o, dO};
@@ -856,7 +886,7 @@ pisa_status backward_impl(const void* q, const void* k, const void* v, const voi
     if (!workspace) return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: null workspace");
     if ((uintptr_t)workspace % kAlign)
         return fail(PISA_ERR_INVALID_ARG, "pisa_attention_backward: workspace must be 256-byte aligned");
-    const BwdLayout w = bwd_layout(g);
+    const BwdLayout w = bwd_layout(g, order);
     if (ws_bytes < w.total)
         return fail(PISA_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, w.total);
     cudaStream_t s = (cudaStream_t)stream;
@@ -872,6 +902,42 @@ pisa_status backward_impl(const void* q, const void* k, const void* v, const voi
     }
     r = run_select(q, kbar, g, dtype, K, nullptr, mask, s, rbias);
     if (r != PISA_OK) return r;
+    if (pooled) {
+        // PWT's pooled w as the forward forms it, then the order-3 kernels and the pooled w's
+        // gradient into dq and dk
+        float* var = (float*)(ws + w.var);
+        float* q2 = (float*)(ws + w.q2);
+        float* wmat = (float*)(ws + w.wmat);
+        float* wsum = (float*)(ws + w.wsum);
+        float* wpart = (float*)(ws + w.wpart);
+        r = run_wpool(q, k, g, dtype, flags & PISA_FLAG_GATE_W, var, q2, wmat, s);
+        if (r != PISA_OK) return r;
+        r = run_backward_tc(q, k, v, o, dO, mask, g, 3, flags & PISA_FLAG_GATE_W, lse, (float*)(ws + w.mstat),
+                            (float*)(ws + w.dinv), (float*)(ws + w.delta), (float*)(ws + w.lse), dq, dk, dv, s, wmat,
+                            wpart);
+        if (r != PISA_OK) return r;
+        const dim3 grid((unsigned)g.nblk, (unsigned)g.BH);
+        const size_t smem = sizeof(float) * g.nblk;
+        cudaError_t e = cudaSuccess;
+#define PISA_POOLED_BWD(DD, BB)                                                                                   \
+    if (g.d == DD && g.B == BB) {                                                                                 \
+        pisa::bwdtc::bwd_pooled_dq_kernel<DD, BB><<<grid, 128, smem, s>>>((const bf16*)q, wmat, wpart, var, wsum, \
+                                                                         dq, (int)g.L, (int)g.nblk);            \
+        e = cudaGetLastError();                                                                                   \
+        if (e == cudaSuccess) {                                                                                   \
+            pisa::bwdtc::bwd_pooled_dk_kernel<DD, BB><<<grid, 128, 0, s>>>((const bf16*)k, kbar, wsum, q2, dk,    \
+                                                                          (int)g.L, (int)g.nblk);               \
+            e = cudaGetLastError();                                                                               \
+        }                                                                                                         \
+    }
+        PISA_POOLED_BWD(64, 64)
+        PISA_POOLED_BWD(64, 128)
+        PISA_POOLED_BWD(128, 64)
+        PISA_POOLED_BWD(128, 128)
+#undef PISA_POOLED_BWD
+        if (e != cudaSuccess) return cuda_fail(e, "pooled-w backward kernels");
+        return PISA_OK;
+    }
     if (tc_path_available(g, dtype))
         return run_backward_tc(q, k, v, o, dO, mask, g, order, flags & PISA_FLAG_GATE_W, lse, (float*)(ws + w.mstat),
                                (float*)(ws + w.dinv), (float*)(ws + w.delta), (float*)(ws + w.lse), dq, dk, dv, s);

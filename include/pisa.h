@@ -346,9 +346,16 @@ size_t pisa_attention_host_bytes(int batch, int heads, int L, int d, pisa_dtype 
  * TMEM, P and dS rounded to bf16 as the operands of the dq, dk and dv
  * products; other bf16 shapes use warp-level MMAs with the same roundings;
  * fp32 inputs run in fp32 throughout.
+ * PISA_FLAG_POOLED_W (order 2; the "Sparse Linear Attention" blog, PWT section,
+ * the diagonal + pooled variant): w_ij = 1/2 sum_c q2_ic var_jc of the forward,
+ * recomputed here, with its gate decisions held fixed; its gradient reaches q
+ * through the tile means of q^2 and k through the blocks' channel variances.
+ * It runs on the tensor-core shapes and takes the forward's lse
+ * (pisa_attention_backward_lse); the order-2 workspace holds its arrays.
  * Errors (before anything is enqueued): INVALID_ARG for a null or misaligned
- * pointer, unknown flag bits, K out of range or a small workspace;
- * UNSUPPORTED for the pooled w, batch * heads > 65535 and the shapes
+ * pointer, unknown flag bits, K out of range, the pooled w at an order other
+ * than 2, or a small workspace; UNSUPPORTED for batch * heads > 65535, the
+ * pooled w off the tensor-core shapes or without lse, and the shapes
  * pisa_attention does not support. */
 pisa_status pisa_attention_backward(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                     int batch, int heads, int L, int d, pisa_dtype dtype, int B, int K, int order,

@@ -189,7 +189,7 @@ def call_bwd(L=1024, d=64, B=64, K=4, order=1, dtype=pisa.PISA_BF16, flags=1, ws
     (dict(order=3), pisa.PISA_ERR_INVALID_ARG),
     (dict(d=96), pisa.PISA_ERR_UNSUPPORTED),
     (dict(flags=8), pisa.PISA_ERR_INVALID_ARG),                 # unknown flag bit
-    (dict(flags=pisa.FLAG_POOLED_W), pisa.PISA_ERR_UNSUPPORTED),  # no backward for the pooled w
+    (dict(flags=pisa.FLAG_POOLED_W), pisa.PISA_ERR_INVALID_ARG),  # the pooled w is an order-2 option
     (dict(batch=2, heads=40000), pisa.PISA_ERR_UNSUPPORTED),    # grid y limit
     (dict(q=None), pisa.PISA_ERR_INVALID_ARG),
     (dict(o=None), pisa.PISA_ERR_INVALID_ARG),
@@ -215,6 +215,24 @@ def test_backward_workspace_size():
     assert f(1, BH, L, d, B, 4, 1, pisa.PISA_BF16) == want
     assert f(1, 1, 1000, 64, 64, 4, 1, pisa.PISA_BF16) == 0
     assert f(1, 1, 1024, 64, 64, 17, 1, pisa.PISA_BF16) == 0
+    # order 2 adds the pooled w's arrays: var, q2 [BH, nblk, d]; w, W [BH, nblk, nblk];
+    # the per-32-row partial sums [BH, L / 32, nblk]
+    pooled = 2 * up(4 * BH * nblk * d) + 2 * up(4 * BH * nblk * nblk) + up(4 * BH * (L // 32) * nblk)
+    assert f(1, BH, L, d, B, 4, 2, pisa.PISA_BF16) == want + pooled
+
+
+def test_pooled_w_backward_rejects_what_it_cannot_run():
+    # host checks before anything touches the device: the pooled w is an order-2 option, runs
+    # on the tensor-core shapes and takes the forward's lse
+    L = pisa.lib()
+    ws = ctypes.c_void_p(0x100000)
+    args = lambda order, dt, flags: (None, None, None, None, None, 1, 1, 1024, 64, dt, 64, 4, order,  # noqa: E731
+                                     flags, None, None, None, ws, 1 << 30, None)
+    pooled = pisa.FLAG_POOLED_W | pisa.FLAG_GATE_W
+    assert L.pisa_attention_backward(*args(1, pisa.PISA_BF16, pooled)) == pisa.PISA_ERR_INVALID_ARG
+    assert L.pisa_attention_backward(*args(2, pisa.PISA_F32, pooled)) == pisa.PISA_ERR_UNSUPPORTED
+    assert L.pisa_attention_backward(*args(2, pisa.PISA_BF16, pooled)) == pisa.PISA_ERR_UNSUPPORTED
+    assert "lse" in L.pisa_last_error().decode()
 
 
 MIS = ctypes.c_void_p(0x1008)  # 8-byte but not 16-byte aligned; never dereferenced

@@ -251,3 +251,62 @@ def test_backward_with_the_forwards_lse(d, B, order):
     pisa.pisa_poll_device_status()
     check([g.cpu().numpy().astype(np.float64) for g in grads],
           oracle.pisa_backward(q, k, v, dO, B, K, order, o=host(o)), dt)
+
+
+def _pooled_inputs(seed, d, B, L=1024):
+    # half of the key blocks 1.4 times wider: their pooled w lands above ln B, the others'
+    # below, so both branches of the gate run, every (tile, block) pair well clear of it
+    q, k, v, dO = inputs(seed, 2, L, d, "bf16", scale=2.4)
+    kk = k.reshape(2, L // B, B, d).copy()
+    kk[:, 1::2] *= 1.4
+    k = pisa_synth.round_bf16(kk.reshape(2, L, d))
+    q64, k64 = q.astype(np.float64), k.astype(np.float64)
+    q2 = (q64.reshape(2, -1, B, d) ** 2).mean(axis=2)
+    kb = k64.reshape(2, -1, B, d)
+    var = ((kb - kb.mean(axis=2, keepdims=True)) ** 2).mean(axis=2)
+    w = 0.5 * np.einsum("bic,bjc->bij", q2, var)
+    assert np.abs(w - math.log(B)).min() > 0.05 * math.log(B)
+    assert 0.2 < (w > math.log(B)).mean() < 0.8
+    return q, k, v, dO
+
+
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("gate", [True, False])
+def test_pooled_w_backward(d, B, gate):
+    # PWT's diagonal + pooled w at order 2 (the forward's pooled path, then the backward with
+    # its lse): the pooled w's gradient reaches q and k through the tile means of q^2 and the
+    # blocks' channel variances
+    dt, L = "bf16", 1024
+    q, k, v, dO = _pooled_inputs(2300 + d + B, d, B, L)
+    K = (L // B) // 4
+    qd, kd, vd, dOd = dev(q, dt), dev(k, dt), dev(v, dt), dev(dO, dt)
+    o, lse = pisa.pisa_attention_lse(qd, kd, vd, B, K, 2, gate=gate, w_mode="pooled")
+    grads = pisa.pisa_attention_backward(qd, kd, vd, o, dOd, B, K, 2, gate=gate, lse=lse, w_mode="pooled")
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    parity.check(o.float().cpu().numpy(), oracle.pisa_attention_ex(q, k, v, B, K, 2, gate=gate, w_pooled=True),
+                 dt, "o")
+    want = oracle.pisa_backward(q, k, v, dO, B, K, 2, gate, o=host(o), w_pooled=True)
+    check([g.cpu().numpy().astype(np.float64) for g in grads], want, dt)
+    # the pooled w's gradient is a visible part of dq and dk on these inputs
+    plain = oracle.pisa_backward(q, k, v, dO, B, K, 1, gate, o=host(o))
+    assert oracle.rel_l2(plain[0], want[0]) > 1e-2 and oracle.rel_l2(plain[1], want[1]) > 1e-2
+
+
+def test_pooled_w_backward_repeats_bit_for_bit_and_through_autograd():
+    dt, L, d, B, K = "bf16", 1024, 128, 64, 4
+    q, k, v, dO = _pooled_inputs(2400, d, B, L)
+    qt, kt, vt = (dev(x, dt).requires_grad_() for x in (q, k, v))
+    out = pisa.pisa_attention_autograd(qt, kt, vt, B, K, 2, w_mode="pooled")
+    out.backward(dev(dO, dt))
+    _, lse = pisa.pisa_attention_lse(dev(q, dt), dev(k, dt), dev(v, dt), B, K, 2, w_mode="pooled")
+    args = (dev(q, dt), dev(k, dt), dev(v, dt), out.detach(), dev(dO, dt), B, K, 2)
+    first = pisa.pisa_attention_backward(*args, lse=lse, w_mode="pooled")
+    again = pisa.pisa_attention_backward(*args, lse=lse, w_mode="pooled")
+    torch.cuda.synchronize()
+    pisa.pisa_poll_device_status()
+    for t, a, b in zip((qt, kt, vt), first, again):
+        assert torch.equal(a, b)  # fixed-order sums: the same result on every run
+        assert torch.equal(t.grad, a.to(torch.bfloat16))
+    with pytest.raises(pisa.PisaError):  # the pooled-w backward takes the forward's lse
+        pisa.pisa_attention_backward(*args, w_mode="pooled")
