@@ -213,17 +213,6 @@ pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dty
     return dispatch(dtype, (int)g.d, (int)g.B, [&](auto t, auto dd, auto bb) {
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
-        if (g.nblk <= pisa::SelLaneCfg<D>::MAXBLK) {
-            // lane-pair form: 32 query tiles per CTA
-            const size_t smem = pisa::select_lane_smem_bytes<D>((int)g.nblk);
-            auto kern = pisa::select_lane_kernel<T, D, BS>;
-            pisa_status r = set_smem(kern, smem);
-            if (r != PISA_OK) return r;
-            dim3 grid((unsigned)((g.nblk + pisa::SelLaneCfg<D>::QT - 1) / pisa::SelLaneCfg<D>::QT), (unsigned)g.BH);
-            kern<<<grid, pisa::SelLaneCfg<D>::THREADS, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K,
-                                                                  (int)g.words, idx, mask, bias, scores);
-            return launch_check("select_lane_kernel");
-        }
         const int QT = pisa::select_tiles_per_cta<D>((int)g.nblk);
         const size_t smem = pisa::select_smem_bytes<D>(QT, (int)g.nblk);
         auto kern = pisa::select_kernel<T, D, BS>;

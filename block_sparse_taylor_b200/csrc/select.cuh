@@ -322,172 +322,4 @@ __global__ void __launch_bounds__(256, 3) select_kernel(const T* __restrict__ q,
     }
 }
 
-// ---------------------------------------------------------------------------
-// Lane-pair form of the same selection (for nblk <= 1024, where a CTA's score
-// table for 32 query tiles fits in shared memory).
-//
-// The canonical tree over the d products, read depth-first, visits the leaves in
-// bit-reversed index order: the last level adds the sums over the even and over the
-// odd indices, and within each half the leaves h + 2 bitrev(p), p = 0 .. d/2 - 1, are
-// combined as adjacent pairs, then adjacent pairs of those, and so on.  So lane 2u + h
-// of a warp holds half h of tile u's mean in that order, a block's centroid is staged in
-// the same two orders, each lane reduces its d/2 products as adjacent pairs, and one
-// shuffle and one add join the halves: the same separately rounded operations as the
-// level-by-level tree, bit for bit, with no per-score shuffles inside the tree and
-// 16-byte shared-memory reads that the lanes of a half share.
-template <int D>
-struct SelLaneCfg {
-    static constexpr int THREADS = 256;
-    static constexpr int QT = 32;  // query tiles per CTA: two groups of 16, a lane pair each
-    static constexpr int JC = 32;  // centroids staged per chunk
-    static constexpr int MAXBLK = 1024;
-};
-
-template <int D>
-inline size_t select_lane_smem_bytes(int nblk) {
-    return sizeof(float) * ((size_t)SelLaneCfg<D>::QT * D + (size_t)SelLaneCfg<D>::JC * D +
-                            (size_t)SelLaneCfg<D>::QT * (nblk + 1));
-}
-
-// d/2 products of one lane's half, reduced as adjacent pairs (see above)
-template <int H>
-__device__ __forceinline__ float half_tree(const float (&q)[H], const float* __restrict__ k) {
-    float a[H];
-    const float4* k4 = reinterpret_cast<const float4*>(k);
-#pragma unroll
-    for (int m = 0; m < H / 4; ++m) {
-        const float4 kv = k4[m];
-        a[4 * m + 0] = __fmul_rn(q[4 * m + 0], kv.x);
-        a[4 * m + 1] = __fmul_rn(q[4 * m + 1], kv.y);
-        a[4 * m + 2] = __fmul_rn(q[4 * m + 2], kv.z);
-        a[4 * m + 3] = __fmul_rn(q[4 * m + 3], kv.w);
-    }
-#pragma unroll
-    for (int n = H / 2; n >= 1; n >>= 1) {
-#pragma unroll
-        for (int i = 0; i < n; ++i) a[i] = __fadd_rn(a[2 * i], a[2 * i + 1]);
-    }
-    return a[0];
-}
-
-// One CTA per (group of 32 query tiles, bh), 8 warps: warp w scores the 16 tiles of group
-// w % 2 against the blocks j = w / 2 (mod 4) of each staged chunk.  Phases 1 and 3 (tile
-// means, top-K) are those of select_kernel.
-template <typename T, int D, int BS>
-__global__ void __launch_bounds__(256, 2) select_lane_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
-                                                             int L, int nblk, int K, int words,
-                                                             int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
-                                                             const float* __restrict__ bias,
-                                                             float* __restrict__ scores_out) {
-    using C = SelLaneCfg<D>;
-    constexpr int H = D / 2;
-    constexpr int HB = (H == 64) ? 6 : 5;  // log2(d/2)
-    extern __shared__ __align__(16) float sm_lane[];
-    float* qbar = sm_lane;                  // [QT][D]
-    float* kst = qbar + C::QT * D;          // [JC][D]: per block, half 0 then half 1, tree order
-    float* sc = kst + C::JC * D;            // [QT][nblk + 1]
-    const int SS = nblk + 1;
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, bh = blockIdx.y;
-    const int i0 = blockIdx.x * C::QT;
-    const int nq = min(C::QT, nblk - i0);
-
-    // 1. canonical tile means (as select_kernel)
-    constexpr int VEC = (sizeof(T) == 2 && BS <= 64) ? 2 : 1;
-    constexpr int CPT = D / VEC;
-    for (int e = tid; e < nq * CPT; e += C::THREADS) {
-        const int t = e / CPT, c = (e % CPT) * VEC;
-        const T* src = q + ((size_t)bh * L + (size_t)(i0 + t) * BS) * D + c;
-        if constexpr (VEC == 2) {
-            float a0[BS], a1[BS];
-#pragma unroll
-            for (int n = 0; n < BS; ++n) {
-                const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(src + (size_t)n * D);
-                a0[n] = __low2float(p);
-                a1[n] = __high2float(p);
-            }
-            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a0), 1.0f / (float)BS);
-            qbar[t * D + c + 1] = __fmul_rn(tree_sum<BS>(a1), 1.0f / (float)BS);
-        } else {
-            float a[BS];
-#pragma unroll
-            for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
-            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-        }
-    }
-    __syncthreads();
-
-    // 2. scores
-    const int grp = warp & 1, bpart = warp >> 1;   // tile group, block subset (of 4)
-    const int u = lane >> 1, hh = lane & 1;        // tile in the group, index half
-    const int t = grp * 16 + u;
-    const bool live = t < nq;
-    float qh[H];  // tile mean at indices hh + 2 bitrev(p), p = 0 .. H - 1
-    {
-        const float* qt_ = qbar + (live ? t : 0) * D;
-#pragma unroll
-        for (int p = 0; p < H; ++p) qh[p] = qt_[hh + 2 * (int)(__brev((unsigned)p) >> (32 - HB))];
-    }
-    for (int j0 = 0; j0 < nblk; j0 += C::JC) {
-        const int nj = min(C::JC, nblk - j0);
-        // stage the chunk: block jj, position h * H + p holds index h + 2 bitrev(p)
-        for (int e = tid; e < nj * D; e += C::THREADS) {
-            const int jj = e / D, pos = e % D;
-            const int h = pos / H, pp = pos % H;
-            const int src = h + 2 * (int)(__brev((unsigned)pp) >> (32 - HB));
-            kst[e] = __ldg(kbar + ((size_t)bh * nblk + j0 + jj) * D + src);
-        }
-        __syncthreads();
-        for (int jj = bpart; jj < nj; jj += 4) {
-            const float v = half_tree<H>(qh, kst + jj * D + hh * H);
-            const float w = __shfl_xor_sync(0xffffffffu, v, 1);
-            float s = __fadd_rn(hh == 0 ? v : w, hh == 0 ? w : v);  // even half + odd half
-            // covariance-aware routing: one fp32 add of the block's bias
-            if (bias) s = __fadd_rn(s, __ldg(bias + (size_t)bh * nblk + j0 + jj));
-            if (live && hh == 0) sc[t * SS + j0 + jj] = s;
-        }
-        __syncthreads();
-    }
-
-    if (scores_out) {
-        for (int e = tid; e < nq * nblk; e += C::THREADS) {
-            const int tt = e / nblk, jj = e % nblk;
-            scores_out[((size_t)bh * nblk + i0 + tt) * nblk + jj] = sc[tt * SS + jj];
-        }
-    }
-
-    // 3. top-K, one warp per tile (nblk <= 1024: keys in registers)
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const int nk = (nblk + 31) / 32;
-    for (int tt = warp; tt < nq; tt += C::THREADS / 32) {
-        const float* st = sc + tt * SS;
-        const size_t row = (size_t)bh * nblk + i0 + tt;
-        uint32_t thr = 0u;
-        int need = 0;
-        if (K > 0 && K < nblk) {
-            if (nk <= 4)
-                thr = kth_ordered_key<4>(st, nblk, K, need);
-            else if (nk <= 8)
-                thr = kth_ordered_key<8>(st, nblk, K, need);
-            else if (nk <= 16)
-                thr = kth_ordered_key<16>(st, nblk, K, need);
-            else
-                thr = kth_ordered_key<32>(st, nblk, K, need);
-        }
-        int off = 0, eq_seen = 0;
-        for (int w = 0; w < words; ++w) {
-            const int j = w * 32 + lane;
-            const bool in = j < nblk;
-            const uint32_t o = in ? ordered_key(st[j]) : 0u;
-            const unsigned eq = __ballot_sync(0xffffffffu, in && o == thr);
-            const int rank = eq_seen + __popc(eq & lt_mask);
-            eq_seen += __popc(eq);
-            const bool sel = in && (K == nblk || (K > 0 && (o > thr || (o == thr && rank < need))));
-            const unsigned bits = __ballot_sync(0xffffffffu, sel);
-            if (mask && lane == 0) mask[row * words + w] = bits;
-            if (idx && sel) idx[row * K + off + __popc(bits & lt_mask)] = j;
-            off += __popc(bits);
-        }
-    }
-}
-
 }  // namespace pisa
