@@ -37,18 +37,20 @@ struct StatsTcCfg {
     static constexpr uint32_t BOX_BYTES = BS * 128;             // BS rows x 64 bf16 columns
     static constexpr uint32_t TILE_BYTES = (D / 64) * BOX_BYTES;
     static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;     // V tile, then K tile ([V ; K] for d = 64)
-    // output staging: per epilogue warp one 32-row x 64-column box (4 KB) per matrix it writes
-    static constexpr int OUT_BOXES = (D == 128 && ORDER == 2) ? 2 : 1;
-    static constexpr uint32_t OUT_BYTES = 8 * OUT_BOXES * 4096;
+    // output staging: per epilogue warp one 32-row x 64-column box (4 KB) per matrix and column half
+    static constexpr int HALVES = D / 64;                       // 64-column boxes per output row
+    static constexpr int OUT_BOXES = ((D == 128 && ORDER == 2) ? 2 : 1) * HALVES;
+    static constexpr uint32_t OUT_BYTES = 4 * OUT_BOXES * 4096;
     static constexpr int NSTG_FIT = (int)((204800 - OUT_BYTES) / STAGE_BYTES);
     static constexpr int NSTG = NSTG_FIT < 6 ? NSTG_FIT : 6;
     static constexpr uint32_t OUT_OFF = NSTG * STAGE_BYTES;
     static constexpr uint32_t BAR_OFF = OUT_OFF + OUT_BYTES;
-    // FULL, EMPTY per stage; MMADONE, EPIDONE, KBREADY per TMEM buffer; DONE
-    static constexpr uint32_t NBAR = 2 * NSTG + 6 + 1;
+    // FULL, EMPTY per stage; MMADONE, EPIDONE per TMEM buffer; KBREADY, KBFREE per
+    // kbar/vsum buffer; DONE
+    static constexpr uint32_t NBAR = 2 * NSTG + 8 + 1;
     static constexpr uint32_t KB_OFF = BAR_OFF + NBAR * 8 + 8;  // fp32 kbar[2][D], vsum[2][D]
     static constexpr uint32_t SMEM = KB_OFF + 4 * D * 4 + 1024;
-    static constexpr int THREADS = 320;                         // producer, MMA, eight epilogue warps
+    static constexpr int THREADS = 320;  // producer, MMA, four column-sum warps, four epilogue warps
     static_assert(NSTG >= 2, "the statistics kernel needs two stages");
     static_assert(KB_OFF % 16 == 0, "kbar and vsum are read as 16-byte vectors");
     static_assert(SMEM <= 232448, "shared memory over the per-CTA limit");
@@ -67,19 +69,61 @@ __device__ __forceinline__ float swz_elem(const uint8_t* tile, int n, int c) {
     return __bfloat162float(*p);
 }
 
+template <int BITS>
+__host__ __device__ constexpr int bit_reverse(int x) {
+    int r = 0;
+    for (int b = 0; b < BITS; ++b) r |= ((x >> b) & 1) << (BITS - 1 - b);
+    return r;
+}
+
+// Column c of a swizzled B-row tile (see swz_elem), summed two ways: `tree` the canonical
+// pairwise tree (rows n and n + B/2 first, then n and n + B/4, ...), evaluated depth-first
+// over the rows in bit-reversed order, where each level combines adjacent partial sums, so
+// at most log2(B) + 1 of them are live; `serial` in row order.  The tree is the same
+// sequence of separately rounded adds as tree_sum<B>.
+template <int BS, bool TREE>
+__device__ __forceinline__ float column_sum(const uint8_t* tile, int c) {
+    constexpr int LB = (BS == 128) ? 7 : 6;
+    const uint8_t* col = tile + (c >> 6) * (BS * 128) + (c & 7) * 2;
+    const int c8 = (c & 63) >> 3;
+    if constexpr (TREE) {
+        float st[LB + 1];
+#pragma unroll
+        for (int p = 0; p < BS; ++p) {
+            const int n = bit_reverse<LB>(p);
+            float v = __bfloat162float(*reinterpret_cast<const bf16*>(col + n * 128 + ((c8 ^ (n & 7)) << 4)));
+            int lvl = 0;
+#pragma unroll
+            for (int t = 0; t < LB; ++t) {
+                if (((p >> t) & 1) && lvl == t) {
+                    v = __fadd_rn(st[t], v);
+                    lvl = t + 1;
+                }
+            }
+            st[lvl] = v;
+        }
+        return st[LB];
+    } else {
+        float sv = 0.f;
+#pragma unroll
+        for (int n = 0; n < BS; ++n)
+            sv += __bfloat162float(*reinterpret_cast<const bf16*>(col + n * 128 + ((c8 ^ (n & 7)) << 4)));
+        return sv;
+    }
+}
+
 // Persistent: CTA c takes the blocks c, c + grid, c + 2 grid, ... of the flattened
-// (bh, j) index.  Warp 0 streams K_j and V_j through NSTG TMA stages; warp 1 runs
-// the Gram MMAs into two TMEM buffers (block i into buffer i % 2); warps 2-9 take
-// the column sums from the stage (one column of K or of V a thread), then the
-// epilogue from TMEM: warp w reads TMEM lane quarter w % 4, and for d = 128 the
-// column half (w - 2) / 4 of it, so each warp owns one 32-row x 64-column box of
-// H_j (and of C_j) and writes it with one TMA store from its own staging box in
-// shared memory (128-byte swizzle, so the row-per-thread writes are free of
-// bank conflicts).  A stage is free again once its MMA has completed and the
-// column sums have read it; a TMEM buffer once the epilogue has read it; a
-// staging box once the warp's previous store has read it.  So the loads of the
-// next blocks, the MMA of the next block and the stores of the previous one all
-// overlap this block's epilogue.
+// (bh, j) index.  Warp 0 streams K_j and V_j through NSTG TMA stages; warp 1 runs the
+// Gram MMAs into two TMEM buffers (block i into buffer i % 2); warps 2-5 take the
+// column sums of block i from its stage (k-bar by the canonical tree, the value sums in
+// row order) into a double-buffered kbar/vsum pair; warps 6-9 run the epilogue of block
+// i from TMEM: warp w reads lane quarter w % 4, applies the rank-1 corrections, rounds
+// to bf16 into its own 128-byte-swizzled staging boxes (32 rows x 64 columns each; the
+// row-per-thread 16-byte stores hit distinct banks) and writes each box with one TMA
+// store.  The two roles overlap: the column sums of block i + 1 run beside the epilogue
+// of block i.  A stage is free again once its MMA has completed and the column-sum warps
+// have read it; a TMEM buffer once the epilogue has read it; a kbar/vsum buffer once the
+// epilogue of its block is done; a staging box once the warp's previous store has read it.
 template <int D, int BS, int ORDER>
 __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                           const __grid_constant__ CUtensorMap tm_v,
@@ -94,13 +138,13 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
                                ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
     constexpr uint32_t TCOLS = stats_tmem_cols<D, ORDER>();  // one buffer
     constexpr long long LIMIT = 2000000000ll;
-    constexpr int NEPI = 8;  // epilogue warps
+    constexpr int NSUM = 4, NEPI = 4;  // column-sum warps, epilogue warps
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_addr(smem);
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
     const int B_FULL = 0, B_EMPTY = C::NSTG, B_MMADONE = 2 * C::NSTG, B_EPIDONE = B_MMADONE + 2,
-              B_KBREADY = B_EPIDONE + 2, B_DONE = B_KBREADY + 2;
+              B_KBREADY = B_EPIDONE + 2, B_KBFREE = B_KBREADY + 2, B_DONE = B_KBFREE + 2;
     uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
     float* kbs = (float*)(smem + C::KB_OFF);  // [2][D]
     float* vss = kbs + 2 * D;                 // [2][D]
@@ -113,12 +157,13 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NSTG; ++s) {
             tc::mbar_init(bar(B_FULL + s), 1);
-            tc::mbar_init(bar(B_EMPTY + s), 1 + NEPI);  // the MMA's commit + the column-sum warps
+            tc::mbar_init(bar(B_EMPTY + s), 1 + NSUM);  // the MMA's commit + the column-sum warps
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(bar(B_MMADONE + b), 1);
             tc::mbar_init(bar(B_EPIDONE + b), NEPI);
-            tc::mbar_init(bar(B_KBREADY + b), NEPI);  // every warp has written its kbar/vsum columns
+            tc::mbar_init(bar(B_KBREADY + b), NSUM);  // the block's kbar/vsum are in kbs/vss
+            tc::mbar_init(bar(B_KBFREE + b), NEPI);   // the epilogue has read them
         }
         tc::mbar_init(bar(B_DONE), 1);
         tc::fence_barrier_init();
@@ -187,136 +232,142 @@ __global__ void __launch_bounds__(320, 1) stats_tc_kernel(const __grid_constant_
             bool a2 = false;
             tc::mbar_wait(bar(B_DONE), 0, a2, status, LIMIT);
         }
-    } else {
-        // ------------------------------------------------ column sums, epilogue
-        const int ct = threadIdx.x - 64;          // 0 .. 255
-        const int quarter = warp % 4;             // TMEM lane quarter of this warp
-        const int half = (warp - 2) / 4;          // column half (d = 128)
-        const int r = quarter * 32 + lane;        // TMEM lane = output row
-        const float inv_b = 1.0f / (float)BS;
-        // this warp's share of the TMEM epilogue: for d = 64 the warps of half 0 take
-        // all 64 columns of their rows (rows 0-63 H_j, 64-127 the uncentred C_j)
-        const bool is_h = (D == 128) || (quarter < 2);
-        const bool writes = ((D == 128) || half == 0) && (is_h || ORDER == 2);
-        const int ar = (D == 128) ? r : (r & 63);        // row of the output matrix
-        const int col0 = (D == 128) ? half * 64 : 0;     // first column of this warp's box
-        const uint32_t stg = sbase + C::OUT_OFF + (uint32_t)(warp - 2) * (C::OUT_BOXES * 4096u);
+    } else if (warp < 2 + NSUM) {
+        // ---------------------------------------------------------------- column sums
+        // d = 128: thread ct takes k column ct and v column ct; d = 64: threads 0-63 the k
+        // columns, 64-127 the v columns
+        const int ct = threadIdx.x - 64;  // 0 .. 127
         for (int i = 0; i < nmine; ++i) {
-            const int s = i % C::NSTG, u = i / C::NSTG, buf = i & 1, ub = i >> 1;
+            const int s = i % C::NSTG, u = i / C::NSTG, kb = i & 1, ukb = i >> 1;
             const long blk = first + (long)i * stride;
             if (!tc::mbar_wait_warp(bar(B_FULL + s), u & 1, aborted, status, LIMIT)) break;
             // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
             // of the stage's bytes
             (void)tc::mbar_try_wait(bar(B_FULL + s), u & 1);
+            // the kbar/vsum buffer is free once the epilogue of block i - 2 has read it
+            if (ukb > 0 && !tc::mbar_wait_warp(bar(B_KBFREE + kb), (ukb - 1) & 1, aborted, status, LIMIT)) break;
             const uint8_t* st = smem + s * C::STAGE_BYTES;
-            // column sums: thread ct < D takes column ct of K (kbar, the centroid split),
-            // D <= ct < 2 D column ct - D of V (vsum)
-            if (ct < 2 * D) {
-                const bool is_k = ct < D;
-                const int c = is_k ? ct : ct - D;
-                // element (n, c) of the swizzled tile: box c / 64, row n, 16-byte chunk
-                // ((c % 64) / 8) ^ (n % 8), so eight per-thread offsets cover every row
-                const uint8_t* col = st + (is_k ? C::TILE_BYTES : 0u) + (c >> 6) * C::BOX_BYTES + (c & 7) * 2;
-                uint32_t off[8];
+            const size_t so = (size_t)blk * D;
+            const bool do_k = (D == 128) || ct < D;
+            const bool do_v = (D == 128) || ct >= D;
+            const int c = (D == 128) ? ct : (ct & (D - 1));
+            if (do_k) {
+                const float m = __fmul_rn(column_sum<BS, true>(st + C::TILE_BYTES, c), 1.0f / (float)BS);
+                kbs[kb * D + c] = m;
+                kbar[so + c] = m;
+                if (kaug) {
+                    bf16* ka = kaug + (size_t)blk * 8 * D + c;
+                    const bf16 hi = __float2bfloat16_rn(m);
+                    ka[0] = hi;
+                    ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) off[k8] = (uint32_t)((((c & 63) >> 3) ^ k8) << 4);
-                float a[BS];
-#pragma unroll
-                for (int n = 0; n < BS; ++n)
-                    a[n] = __bfloat162float(*reinterpret_cast<const bf16*>(col + n * 128 + off[n & 7]));
-                const size_t so = (size_t)blk * D + c;
-                if (is_k) {
-                    const float m = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-                    kbs[buf * D + c] = m;
-                    kbar[so] = m;
-                    if (kaug) {
-                        bf16* ka = kaug + (size_t)blk * 8 * D + c;
-                        const bf16 hi = __float2bfloat16_rn(m);
-                        ka[0] = hi;
-                        ka[D] = __float2bfloat16_rn(m - __bfloat162float(hi));
-#pragma unroll
-                        for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
-                    }
-                } else {
-                    float sv = 0.f;
-#pragma unroll
-                    for (int n = 0; n < BS; ++n) sv += a[n];
-                    vss[buf * D + c] = sv;
-                    vsum[so] = sv;
+                    for (int rr = 2; rr < 8; ++rr) ka[rr * D] = __float2bfloat16_rn(0.f);
                 }
+            }
+            if (do_v) {
+                const float sv = column_sum<BS, false>(st, c);
+                vss[kb * D + c] = sv;
+                vsum[so + c] = sv;
             }
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_arrive(bar(B_EMPTY + s));      // this warp no longer reads the stage
-                tc::mbar_arrive(bar(B_KBREADY + buf));  // and its kbar/vsum columns are in kbs/vss
+                tc::mbar_arrive(bar(B_EMPTY + s));     // this warp no longer reads the stage
+                tc::mbar_arrive(bar(B_KBREADY + kb));  // and its kbar/vsum columns are in kbs/vss
             }
-            // the block's kbar and vsum from all warps (a bounded wait, unlike a named barrier,
-            // so a warp that gave up cannot hold the others forever)
-            if (!tc::mbar_wait_warp(bar(B_KBREADY + buf), ub & 1, aborted, status, LIMIT)) break;
+        }
+    } else {
+        // ----------------------------------------------------------------- epilogue
+        const int quarter = warp % 4;  // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;  // TMEM lane = output row
+        const float inv_b = 1.0f / (float)BS;
+        // for d = 64, rows 0-63 are H_j and rows 64-127 the uncentred C_j
+        const bool is_h = (D == 128) || (quarter < 2);
+        const bool writes = is_h || ORDER == 2;
+        const int ar = (D == 128) ? r : (r & 63);  // row of the output matrix
+        const uint32_t stg = sbase + C::OUT_OFF + (uint32_t)(warp - 2 - NSUM) * (C::OUT_BOXES * 4096u);
+        for (int i = 0; i < nmine; ++i) {
+            const int buf = i & 1, ub = i >> 1, kb = i & 1;
+            const long blk = first + (long)i * stride;
+            if (!tc::mbar_wait_warp(bar(B_KBREADY + kb), ub & 1, aborted, status, LIMIT)) break;
+            // kbs/vss were written by the column-sum threads: each thread's own test is its acquire
+            (void)tc::mbar_try_wait(bar(B_KBREADY + kb), ub & 1);
             if (!tc::mbar_wait_warp(bar(B_MMADONE + buf), ub & 1, aborted, status, LIMIT)) break;
             tc::fence_after_sync();
             if (writes) {
-                // the staging box is free once this warp's previous store has read it
+                // the staging boxes are free once this warp's previous stores have read them
                 if (lane == 0) tc::bulk_wait_read<0>();
                 __syncwarp();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TCOLS);
-                const float* kb = kbs + buf * D;
-                const float* vs = vss + buf * D;
+                const float* kbp = kbs + kb * D;
+                const float* vsp = vss + kb * D;
 #pragma unroll
-                for (int part = 0; part < C::OUT_BOXES; ++part) {
+                for (int part = 0; part < C::OUT_BOXES / C::HALVES; ++part) {
                     const bool h_here = (D == 128) ? (part == 0) : is_h;
-                    const float rv = h_here ? vs[ar] : kb[ar];
+                    const float rv = h_here ? vsp[ar] : kbp[ar];
 #pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        uint32_t raw[32];
-                        tc::tmem_ld32(taddr + (uint32_t)(part * 128 + col0 + c0), raw);
-                        tc::tmem_wait_ld();
-                        uint32_t pk[16];
-                        const float4* kb4 = reinterpret_cast<const float4*>(kb + col0 + c0);
+                    for (int hf = 0; hf < C::HALVES; ++hf) {
+                        const uint32_t box = stg + (uint32_t)(part * C::HALVES + hf) * 4096u;
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            const float4 kv = kb4[e4];  // kbar of the four columns (a broadcast read)
-                            const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+                        for (int c0 = 0; c0 < 64; c0 += 32) {
+                            uint32_t raw[32];
+                            tc::tmem_ld32(taddr + (uint32_t)(part * 128 + hf * 64 + c0), raw);
+                            tc::tmem_wait_ld();
+                            uint32_t pk[16];
+                            const float4* kb4 = reinterpret_cast<const float4*>(kbp + hf * 64 + c0);
 #pragma unroll
-                            for (int e2 = 0; e2 < 2; ++e2) {
-                                const int e = 2 * e4 + e2;
-                                float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
-                                if (h_here) {
-                                    x0 = fmaf(-rv, kk[2 * e2], x0);
-                                    x1 = fmaf(-rv, kk[2 * e2 + 1], x1);
-                                } else {
-                                    x0 = fmaf(-rv, kk[2 * e2], x0 * inv_b);
-                                    x1 = fmaf(-rv, kk[2 * e2 + 1], x1 * inv_b);
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 kv = kb4[e4];  // kbar of the four columns (a broadcast read)
+                                const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                                for (int e2 = 0; e2 < 2; ++e2) {
+                                    const int e = 2 * e4 + e2;
+                                    float x0 = __uint_as_float(raw[2 * e]), x1 = __uint_as_float(raw[2 * e + 1]);
+                                    if (h_here) {
+                                        x0 = fmaf(-rv, kk[2 * e2], x0);
+                                        x1 = fmaf(-rv, kk[2 * e2 + 1], x1);
+                                    } else {
+                                        x0 = fmaf(-rv, kk[2 * e2], x0 * inv_b);
+                                        x1 = fmaf(-rv, kk[2 * e2 + 1], x1 * inv_b);
+                                    }
+                                    pk[e] = tc::pack_bf16x2(x0, x1);
                                 }
-                                pk[e] = tc::pack_bf16x2(x0, x1);
                             }
-                        }
-                        // row `lane` of the box, 16-byte chunks c0/8 .. c0/8 + 3, swizzled
-                        const uint32_t rowa = stg + (uint32_t)part * 4096u + (uint32_t)lane * 128u;
+                            // row `lane` of the box, 16-byte chunks c0/8 .. c0/8 + 3, swizzled
+                            const uint32_t rowa = box + (uint32_t)lane * 128u;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const uint32_t chunk = (uint32_t)((c0 / 8 + e) ^ (lane & 7));
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + chunk * 16u),
-                                         "r"(pk[4 * e]), "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
-                                         : "memory");
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t chunk = (uint32_t)((c0 / 8 + e) ^ (lane & 7));
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + chunk * 16u),
+                                             "r"(pk[4 * e]), "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
+                                             : "memory");
+                            }
                         }
                     }
                 }
-                tc::fence_before_sync();
+            }
+            // TMEM and kbs/vss are read: the MMA may reuse the buffer, the column sums the pair
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(bar(B_EPIDONE + buf));
+                tc::mbar_arrive(bar(B_KBFREE + kb));
+            }
+            if (writes) {
                 tc::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int y = (int)((long)blk * D + (ar - lane));  // first row of the box
+                    const int y = (int)((long)blk * D + (ar - lane));  // first row of the boxes
 #pragma unroll
-                    for (int part = 0; part < C::OUT_BOXES; ++part) {
+                    for (int part = 0; part < C::OUT_BOXES / C::HALVES; ++part) {
                         const bool h_here = (D == 128) ? (part == 0) : is_h;
-                        tc::tma_store_2d(h_here ? &tm_h : &tm_c, stg + (uint32_t)part * 4096u, col0, y);
+#pragma unroll
+                        for (int hf = 0; hf < C::HALVES; ++hf)
+                            tc::tma_store_2d(h_here ? &tm_h : &tm_c, stg + (uint32_t)(part * C::HALVES + hf) * 4096u,
+                                             hf * 64, y);
                     }
                     tc::bulk_commit();
                 }
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(B_EPIDONE + buf));  // the TMEM buffer is read
         }
         // the stores have landed before the CTA exits
         if (lane == 0) tc::bulk_wait<0>();
