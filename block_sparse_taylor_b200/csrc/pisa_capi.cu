@@ -214,17 +214,6 @@ pisa_status run_select(const void* q, const float* kbar, const Dims& g, pisa_dty
         using T = decltype(t);
         constexpr int D = decltype(dd)::value, BS = decltype(bb)::value;
         const int QT = pisa::select_tiles_per_cta<D>((int)g.nblk);
-        if (!scores && g.nblk <= 1024) {
-            // the mask and list through bounded approximate scores (the same selection)
-            const size_t smem = pisa::select_fast_smem_bytes<D>(QT, (int)g.nblk);
-            auto kern = pisa::select_fast_kernel<T, D, BS>;
-            pisa_status r = set_smem(kern, smem);
-            if (r != PISA_OK) return r;
-            dim3 grid((unsigned)((g.nblk + QT - 1) / QT), (unsigned)g.BH);
-            kern<<<grid, pisa::SelectCfg<D>::THREADS, smem, s>>>((const T*)q, kbar, (int)g.L, (int)g.nblk, K,
-                                                                  (int)g.words, QT, idx, mask, bias);
-            return launch_check("select_fast_kernel");
-        }
         const size_t smem = pisa::select_smem_bytes<D>(QT, (int)g.nblk);
         auto kern = pisa::select_kernel<T, D, BS>;
         pisa_status r = set_smem(kern, smem);

@@ -15,7 +15,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "tc_ptx.cuh"
 
 namespace pisa {
 
@@ -320,326 +319,6 @@ __global__ void __launch_bounds__(256, 3) select_kernel(const T* __restrict__ q,
             if (idx && sel) idx[row * K + off + __popc(bits & lt_mask)] = j;
             off += __popc(bits);
         }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Selection through bounded approximate scores (mask and index list; the score table
-// itself comes from select_kernel).
-//
-// The canonical score s_ij (products rounded, pairwise tree over d) and an fp32 dot in
-// another order both lie within a few units in the last place of sum_c |q_c k_c| of the
-// exact dot, so |s~_ij - s_ij| <= e_ij = 2^-16 |q-bar_i| |k-bar_j| + 2^-20 (|s~_ij| + |bias_j|)
-// + 10^-30: 2^-16 is about ten times the sum of the two worst-case bounds at d = 128
-// ((1 + log2 d) u for the tree, about 12 u for the chains of approx_dot4, u = 2^-24;
-// |q| |k| bounds sum |q_c k_c| by Cauchy-Schwarz), the relative term covers the roundings
-// of the bias add and of the comparisons, the absolute one underflowed products.  With T~
-// the K-th largest approximate score of a row and E its largest e, a block with
-// s~ - e > T~ + E is in the top K whatever the exact scores are (the exact K-th largest is
-// at most the K-th largest of s~ + e, at most T~ + E), and one with s~ + e < T~ - E is not.
-// The canonical score is computed only for the blocks in between (typically none or a
-// few), and the top K is the sure blocks plus the best of the undecided ones by (exact
-// score, lower index): the canonical selection, bit for bit.
-constexpr float kSelGamma = 1.52587890625e-05f;  // 2^-16
-constexpr float kSelRel = 9.5367431640625e-07f;  // 2^-20
-constexpr float kSelAbs = 1e-30f;
-
-// Approximate score over the lane's residue segment (packed fp32 FMAs in two chains), the
-// four lanes of a tile joined by two xor shuffles, so that every lane holds the sum.
-template <int D>
-__device__ __forceinline__ float approx_dot4(const float (&q)[D / 4], const float* __restrict__ k) {
-    const float4* k4 = reinterpret_cast<const float4*>(k);
-    uint64_t a = 0ull, b = 0ull;
-#pragma unroll
-    for (int m = 0; m < D / 16; ++m) {
-        const float4 kv = k4[m];
-        a = tc::f2_fma(tc::f2_make(q[4 * m + 0], q[4 * m + 1]), tc::f2_make(kv.x, kv.y), a);
-        b = tc::f2_fma(tc::f2_make(q[4 * m + 2], q[4 * m + 3]), tc::f2_make(kv.z, kv.w), b);
-    }
-    const float2 s2 = tc::f2_split(tc::f2_add(a, b));
-    float v = s2.x + s2.y;
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    return v;
-}
-
-// The canonical score from a centroid row in global memory: lane r of a four-lane group
-// gathers its residue segment in canonical_dot4's order; valid in lane r = 0.
-template <int D>
-__device__ __forceinline__ float canonical_dot4_global(const float (&q)[D / 4], const float* __restrict__ kj, int r) {
-    constexpr int H = D / 8;
-    float a[H];
-#pragma unroll
-    for (int m = 0; m < H; ++m)
-        a[m] = __fadd_rn(__fmul_rn(q[m], __ldg(kj + r + 4 * m)), __fmul_rn(q[H + m], __ldg(kj + D / 2 + r + 4 * m)));
-    float v = tree_sum<H>(a);
-    v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, 2));
-    v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, 1));
-    return v;
-}
-
-__device__ __forceinline__ float ordered_to_float(uint32_t o) {
-    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
-}
-
-// K-th largest of the keys NKT a lane (0 = absent, below every score), with `need` the
-// number of keys equal to it that are taken (lowest index first).
-template <int NKT>
-__device__ __forceinline__ uint32_t kth_key_regs(const uint32_t (&kv)[NKT], int K, int& need) {
-    uint32_t lo = 0xffffffffu, hi = 0u;
-#pragma unroll
-    for (int i = 0; i < NKT; ++i)
-        if (kv[i]) {
-            lo = min(lo, kv[i]);
-            hi = max(hi, kv[i]);
-        }
-    lo = __reduce_min_sync(0xffffffffu, lo);
-    hi = __reduce_max_sync(0xffffffffu, hi);
-    uint32_t thr = hi;
-    if (lo < hi) {
-        const int top = 31 - __clz(lo ^ hi);
-        thr = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
-        for (int bit = top; bit >= 0; --bit) {
-            const uint32_t cand = thr | (1u << bit);
-            int cnt = 0;
-#pragma unroll
-            for (int i = 0; i < NKT; ++i) cnt += kv[i] >= cand;
-            cnt = __reduce_add_sync(0xffffffffu, cnt);
-            if (cnt >= K) thr = cand;
-        }
-    }
-    int gt = 0;
-#pragma unroll
-    for (int i = 0; i < NKT; ++i) gt += kv[i] > thr;
-    need = K - __reduce_add_sync(0xffffffffu, gt);
-    return thr;
-}
-
-template <int D>
-inline size_t select_fast_smem_bytes(int QT, int nblk) {
-    return select_smem_bytes<D>(QT, nblk) + sizeof(float) * ((size_t)nblk + QT);
-}
-
-// Top K of one tile's row (one warp; nblk <= 32 NKT): st holds the approximate scores
-// and receives the canonical ones of the undecided blocks.
-template <int D, int NKT>
-__device__ __forceinline__ void topk_bounded(float* __restrict__ st, const float* __restrict__ kn, float qnorm,
-                                             const float* __restrict__ qbar_t, const float* __restrict__ kbar_bh,
-                                             const float* __restrict__ bias_bh, int nblk, int K, int words,
-                                             size_t row, int32_t* __restrict__ idx, uint32_t* __restrict__ mask) {
-    const int lane = threadIdx.x & 31;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const float gq = kSelGamma * qnorm;
-    auto bound = [&](int j, float sj) {
-        const float bj = bias_bh ? fabsf(__ldg(bias_bh + j)) : 0.f;
-        return fmaf(gq, kn[j], fmaf(kSelRel, fabsf(sj) + bj, kSelAbs));
-    };
-    uint32_t in_bits = 0u, un_bits = 0u;  // bit i: block lane + 32 i
-    int need = 0;
-    uint32_t thr = 0u;
-    if (K > 0 && K < nblk) {
-        uint32_t kv[NKT];
-        float emax = 0.f;
-#pragma unroll
-        for (int i = 0; i < NKT; ++i) {
-            const int j = lane + 32 * i;
-            kv[i] = 0u;
-            if (j < nblk) {
-                const float sj = st[j];
-                kv[i] = ordered_key(sj);
-                emax = fmaxf(emax, bound(j, sj));
-            }
-        }
-        emax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(emax)));  // e >= 0
-        int need0;
-        const float tf = ordered_to_float(kth_key_regs<NKT>(kv, K, need0));
-        const float in_cut = tf + emax, out_cut = tf - emax;
-        int n_in = 0;
-#pragma unroll
-        for (int i = 0; i < NKT; ++i) {
-            const int j = lane + 32 * i;
-            bool in = false, un = false;
-            if (j < nblk) {
-                const float sj = st[j];
-                const float e = bound(j, sj);
-                in = sj - e > in_cut;
-                un = !in && !(sj + e < out_cut);
-            }
-            in_bits |= (uint32_t)in << i;
-            un_bits |= (uint32_t)un << i;
-            n_in += __popc(__ballot_sync(0xffffffffu, in));
-        }
-        need = K - n_in;
-        if (need > 0) {
-            // canonical scores of the undecided blocks, eight at a time (four lanes each)
-            const int g = lane >> 2, r = lane & 3;
-            float qr[D / 4];
-#pragma unroll
-            for (int m = 0; m < D / 8; ++m) {
-                qr[m] = qbar_t[r + 4 * m];
-                qr[D / 8 + m] = qbar_t[D / 2 + r + 4 * m];
-            }
-#pragma unroll
-            for (int i = 0; i < NKT; ++i) {
-                unsigned u = __ballot_sync(0xffffffffu, (un_bits >> i) & 1u);
-                while (u) {
-                    const int cnt = __popc(u);
-                    const int bit = g < cnt ? (int)__fns(u, 0, g + 1) : -1;
-                    const int jj = (bit >= 0 ? bit : 0) + 32 * i;
-                    float sx = canonical_dot4_global<D>(qr, kbar_bh + (size_t)jj * D, r);
-                    if (bias_bh) sx = __fadd_rn(sx, __ldg(bias_bh + jj));
-                    if (bit >= 0 && r == 0) st[jj] = sx;
-                    for (int c = 0; c < 8 && u; ++c) u &= u - 1u;
-                }
-            }
-            __syncwarp();
-            uint32_t kx[NKT];
-#pragma unroll
-            for (int i = 0; i < NKT; ++i) kx[i] = ((un_bits >> i) & 1u) ? ordered_key(st[lane + 32 * i]) : 0u;
-            thr = kth_key_regs<NKT>(kx, need, need);
-        }
-    }
-    // emit: sure blocks, then the undecided ones above the exact threshold and the first
-    // `need` ties at it by ascending index; the ballots give the mask words and the list
-    int off = 0, eq_seen = 0;
-    for (int w = 0; w < words; ++w) {
-        const int j = w * 32 + lane;
-        const bool in_w = j < nblk;
-        bool sel;
-        if (K >= nblk) {
-            sel = in_w;
-        } else if (K <= 0) {
-            sel = false;
-        } else {
-            const bool in = w < NKT ? ((in_bits >> w) & 1u) : false;
-            const bool un = w < NKT ? ((un_bits >> w) & 1u) : false;
-            const uint32_t o = un ? ordered_key(st[j]) : 0u;
-            const unsigned eq = __ballot_sync(0xffffffffu, un && need > 0 && o == thr);
-            const int rank = eq_seen + __popc(eq & lt_mask);
-            eq_seen += __popc(eq);
-            sel = in || (un && need > 0 && (o > thr || (o == thr && rank < need)));
-        }
-        const unsigned bits = __ballot_sync(0xffffffffu, sel);
-        if (mask && lane == 0) mask[row * words + w] = bits;
-        if (idx && sel) idx[row * K + off + __popc(bits & lt_mask)] = j;
-        off += __popc(bits);
-    }
-}
-
-// select_kernel's CTA shape and phases 1 and 2, with approximate scores and block and
-// tile-mean norms; phase 3 is topk_bounded.  For nblk <= 1024.
-template <typename T, int D, int BS>
-__global__ void __launch_bounds__(256, 3) select_fast_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
-                                                             int L, int nblk, int K, int words, int QT,
-                                                             int32_t* __restrict__ idx, uint32_t* __restrict__ mask,
-                                                             const float* __restrict__ bias) {
-    using C = SelectCfg<D>;
-    extern __shared__ __align__(16) float sm_fast[];
-    float* qbar = sm_fast;                   // [QT][D]
-    float* kst = qbar + QT * D;              // [JC][4][SEG]
-    float* sc = kst + C::JC * 4 * C::SEG;    // [QT][nblk + 1]
-    const int SS = nblk + 1;
-    float* kn = sc + QT * SS;                // [nblk] centroid norms
-    float* qn = kn + nblk;                   // [QT] tile-mean norms
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, bh = blockIdx.y;
-    const int i0 = blockIdx.x * QT;
-    const int nq = min(QT, nblk - i0);
-
-    // 1. canonical tile means (as select_kernel), then their norms
-    constexpr int VEC = (sizeof(T) == 2 && BS <= 64) ? 2 : 1;
-    constexpr int CPT = D / VEC;
-    for (int e = tid; e < nq * CPT; e += C::THREADS) {
-        const int t = e / CPT, c = (e % CPT) * VEC;
-        const T* src = q + ((size_t)bh * L + (size_t)(i0 + t) * BS) * D + c;
-        if constexpr (VEC == 2) {
-            float a0[BS], a1[BS];
-#pragma unroll
-            for (int n = 0; n < BS; ++n) {
-                const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(src + (size_t)n * D);
-                a0[n] = __low2float(p);
-                a1[n] = __high2float(p);
-            }
-            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a0), 1.0f / (float)BS);
-            qbar[t * D + c + 1] = __fmul_rn(tree_sum<BS>(a1), 1.0f / (float)BS);
-        } else {
-            float a[BS];
-#pragma unroll
-            for (int n = 0; n < BS; ++n) a[n] = to_f(src[(size_t)n * D]);
-            qbar[t * D + c] = __fmul_rn(tree_sum<BS>(a), 1.0f / (float)BS);
-        }
-    }
-    __syncthreads();
-    for (int t = warp; t < nq; t += 8) {
-        float s2 = 0.f;
-        for (int c = lane; c < D; c += 32) s2 = fmaf(qbar[t * D + c], qbar[t * D + c], s2);
-        s2 = warp_sum(s2);
-        if (lane == 0) qn[t] = sqrtf(s2);
-    }
-
-    // 2. approximate scores (lanes as in select_kernel) and the centroid norms
-    const int ngroups = QT / 8;
-    const int grp = warp % ngroups;
-    const int wsplit = 8 / ngroups;
-    const int wpart = warp / ngroups;
-    const int tl = lane >> 2, r = lane & 3;
-    const int t = grp * 8 + tl;
-    const bool live = t < nq;
-    float qr[D / 4];
-    {
-        const float* qt_ = qbar + (live ? t : 0) * D;
-#pragma unroll
-        for (int m = 0; m < D / 8; ++m) {
-            qr[m] = qt_[r + 4 * m];
-            qr[D / 8 + m] = qt_[D / 2 + r + 4 * m];
-        }
-    }
-    const float* kb_bh = kbar + (size_t)bh * nblk * D;
-    const float4* kb4 = reinterpret_cast<const float4*>(kb_bh);
-    const float* bias_bh = bias ? bias + (size_t)bh * nblk : nullptr;
-    for (int j0 = 0; j0 < nblk; j0 += C::JC) {
-        const int nj = min(C::JC, nblk - j0);
-        for (int e = tid; e < nj * D / 4; e += C::THREADS) {
-            const int jj = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            const float4 v = kb4[(size_t)j0 * D / 4 + e];
-            const int pos = (c4 % (D / 2)) / 4 + (c4 >= D / 2 ? D / 8 : 0);
-            float* seg = kst + (jj * 4) * C::SEG + pos;
-            seg[0 * C::SEG] = v.x;
-            seg[1 * C::SEG] = v.y;
-            seg[2 * C::SEG] = v.z;
-            seg[3 * C::SEG] = v.w;
-        }
-        for (int jj = warp; jj < nj; jj += 8) {
-            float s2 = 0.f;
-            for (int c = lane; c < D; c += 32) {
-                const float x = __ldg(kb_bh + (size_t)(j0 + jj) * D + c);
-                s2 = fmaf(x, x, s2);
-            }
-            s2 = warp_sum(s2);
-            if (lane == 0) kn[j0 + jj] = sqrtf(s2);
-        }
-        __syncthreads();
-        for (int jj = wpart; jj < nj; jj += wsplit) {
-            float sx = approx_dot4<D>(qr, kst + (jj * 4 + r) * C::SEG);
-            if (bias_bh) sx += __ldg(bias_bh + j0 + jj);
-            if (live && r == 0) sc[t * SS + j0 + jj] = sx;
-        }
-        __syncthreads();
-    }
-
-    // 3. top K per tile, one warp per tile
-    const int nk = (nblk + 31) / 32;
-    for (int tt = warp; tt < nq; tt += 8) {
-        float* st = sc + tt * SS;
-        const size_t row = (size_t)bh * nblk + i0 + tt;
-        const float* qb_t = qbar + tt * D;
-        if (nk <= 4)
-            topk_bounded<D, 4>(st, kn, qn[tt], qb_t, kb_bh, bias_bh, nblk, K, words, row, idx, mask);
-        else if (nk <= 8)
-            topk_bounded<D, 8>(st, kn, qn[tt], qb_t, kb_bh, bias_bh, nblk, K, words, row, idx, mask);
-        else if (nk <= 16)
-            topk_bounded<D, 16>(st, kn, qn[tt], qb_t, kb_bh, bias_bh, nblk, K, words, row, idx, mask);
-        else
-            topk_bounded<D, 32>(st, kn, qn[tt], qb_t, kb_bh, bias_bh, nblk, K, words, row, idx, mask);
     }
 }
 

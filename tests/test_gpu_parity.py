@@ -180,6 +180,27 @@ def test_select_planted_ties():
         assert np.array_equal(idx, ridx) and np.array_equal(mask, rmask)
 
 
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 64), (128, 128)])
+def test_select_near_ties_decided_by_the_canonical_scores(d, B):
+    # every key block is one base block plus a perturbation of a few ulp of a single entry,
+    # so the scores of a row differ by less than the approximate scores' error bound: the
+    # selection must fall back to the canonical scores for most blocks and still match
+    L = 2048
+    nblk = L // B
+    rng = np.random.default_rng(31 + d + B)
+    base = rng.standard_normal((B, d)).astype(np.float32)
+    k = np.tile(base, (nblk, 1))[None].copy()
+    for j in range(nblk):
+        c = int(rng.integers(d))
+        toward = np.float32(np.inf) if j % 2 else np.float32(-np.inf)
+        k[0, j * B:(j + 1) * B, c] = np.nextafter(k[0, j * B:(j + 1) * B, c], toward)
+    q = rng.standard_normal((1, L, d)).astype(np.float32)
+    for K in (1, nblk // 4, nblk // 2, nblk - 1):
+        idx, mask = gpu_select(q, k, B, K, "f32")
+        ridx, rmask, _ = oracle.select(q, k, B, K)
+        assert np.array_equal(idx, ridx) and np.array_equal(mask, rmask)
+
+
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("d,B,L", [(64, 64, 2048), (128, 64, 4096), (128, 128, 4096), (64, 128, 1024)])
 def test_select_scores_bit_exact(dt, d, B, L):
