@@ -389,8 +389,8 @@ def test_hybrid_edge_cases(case):
     parity.check(got, ref, "bf16", case)
 
 
-@pytest.mark.parametrize("name,per_head,nheads", [("c3", 2, 8), ("c5_L16896_s90", 2, 8), ("c4", 1, 4),
-                                                   ("c5_L4608_s50", 2, 8), ("c5_L4608_s90", 2, 8)])
+@pytest.mark.parametrize("name,per_head,nheads", [("c3", 2, 8), ("c4", 1, 4)] + [
+    (f"c5_L{L}_s{sp}", 2, 8) for L in (4608, 16896) for sp in (50, 75, 90, 95)])
 def test_hybrid_full_size_sampled(name, per_head, nheads):
     w, (q, k, v) = workload(name)
     got = run_attn(q, k, v, w.B, w.K, 1, w.dtype, "hybrid_tc")
