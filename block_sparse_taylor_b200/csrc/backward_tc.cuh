@@ -125,35 +125,33 @@ __device__ __forceinline__ HalfSums half_sums(const uint32_t (&xa)[32], const ui
     return HalfSums{s1.x + s1.y, s2.x + s2.y, sg.x + sg.y, sgd.x + sgd.y};
 }
 
-// dS (or P and dS) of 32 keys (one chunk of a half tile), packed as bf16 pairs (keys 2e,
-// 2e + 1 in word e).  Selected block: P = 2^{x log2 e - lse2}, dS = P (G - delta);
-// unselected block: u = x - sb, P = a + Pu u, dS = A G + X u + Cc.
-template <bool WANT_P>
-__device__ __forceinline__ void chunk_ds(const uint32_t (&xs)[32], const uint32_t (&gs)[32], bool sel, bool valid,
-                                         float lse2, float del, float sb, float a, float A, float X, float Cc,
-                                         float Pu, uint32_t (&pp)[16], uint32_t (&dd)[16]) {
+// dS of 32 keys (one chunk of a half tile), packed as bf16 pairs (keys 2e, 2e + 1 in word
+// e).  Selected block: P = 2^{x log2 e - lse2}, dS = P (G - delta); unselected block:
+// u = x - sb, dS = A G + X u + Cc.  The test of `sel` stays outside the loops (it is the
+// same for the 32 rows of a warp), so that only selected rows pay for the exponentials.
+// A row past the sequence end comes in with lse2 = +inf and delta = 0: every term is 0.
+__device__ __forceinline__ void chunk_ds(const uint32_t (&xs)[32], const uint32_t (&gs)[32], bool sel, float lse2,
+                                         float del, float sb, float A, float X, float Cc, uint32_t (&dd)[16]) {
     constexpr float LOG2E = 1.4426950408889634f;
-    const uint64_t ndel = tc::f2_make(-del, -del), nsb = tc::f2_make(-sb, -sb);
-    const uint64_t A2 = tc::f2_make(A, A), X2 = tc::f2_make(X, X), C2 = tc::f2_make(Cc, Cc);
-    const uint64_t a2 = tc::f2_make(a, a), P2 = tc::f2_make(Pu, Pu);
+    if (sel) {
+        const uint64_t ndel = tc::f2_make(-del, -del);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const float x0 = __uint_as_float(xs[2 * e]), x1 = __uint_as_float(xs[2 * e + 1]);
-        const uint64_t g2 = tc::f2_make(__uint_as_float(gs[2 * e]), __uint_as_float(gs[2 * e + 1]));
-        uint64_t p2, d2;
-        if (sel) {
-            p2 = tc::f2_make(tc::ex2(fmaf(x0, LOG2E, -lse2)), tc::ex2(fmaf(x1, LOG2E, -lse2)));
-            d2 = tc::f2_mul(p2, tc::f2_add(g2, ndel));
-        } else {
-            const uint64_t u2 = tc::f2_add(tc::f2_make(x0, x1), nsb);
-            p2 = tc::f2_fma(P2, u2, a2);
-            d2 = tc::f2_fma(A2, g2, tc::f2_fma(X2, u2, C2));
+        for (int e = 0; e < 16; ++e) {
+            const uint64_t g2 = tc::f2_make(__uint_as_float(gs[2 * e]), __uint_as_float(gs[2 * e + 1]));
+            const uint64_t p2 = tc::f2_make(tc::ex2(fmaf(__uint_as_float(xs[2 * e]), LOG2E, -lse2)),
+                                            tc::ex2(fmaf(__uint_as_float(xs[2 * e + 1]), LOG2E, -lse2)));
+            const float2 d = tc::f2_split(tc::f2_mul(p2, tc::f2_add(g2, ndel)));
+            dd[e] = tc::pack_bf16x2(d.x, d.y);
         }
-        const float2 d = tc::f2_split(d2);
-        dd[e] = valid ? tc::pack_bf16x2(d.x, d.y) : 0u;
-        if (WANT_P) {
-            const float2 pv = tc::f2_split(p2);
-            pp[e] = valid ? tc::pack_bf16x2(pv.x, pv.y) : 0u;
+    } else {
+        const uint64_t nsb = tc::f2_make(-sb, -sb);
+        const uint64_t A2 = tc::f2_make(A, A), X2 = tc::f2_make(X, X), C2 = tc::f2_make(Cc, Cc);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const uint64_t g2 = tc::f2_make(__uint_as_float(gs[2 * e]), __uint_as_float(gs[2 * e + 1]));
+            const uint64_t u2 = tc::f2_add(tc::f2_make(__uint_as_float(xs[2 * e]), __uint_as_float(xs[2 * e + 1])), nsb);
+            const float2 d = tc::f2_split(tc::f2_fma(A2, g2, tc::f2_fma(X2, u2, C2)));
+            dd[e] = tc::pack_bf16x2(d.x, d.y);
         }
     }
 }
@@ -390,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = qrow < L;
         const int qt = (valid ? qrow : L - 1) / BS;  // query tile (selection row)
         const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
-        const float lse2 = (valid ? __ldg(lse + (size_t)bh * L + qrow) : 0.f) * LOG2E;  // log2 units
+        // log2 units; +inf past the sequence end, where it makes every coefficient 0
+        const float lse2 = valid ? __ldg(lse + (size_t)bh * L + qrow) * LOG2E : __int_as_float(0x7f800000);
         const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
         const float ln_b = logf((float)BS);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -448,10 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // dS (bf16) over the first 32 columns of this half: keys 2e and 2e + 1 in column e
             {
-                uint32_t pp[16], dd[16];
-                chunk_ds<false>(xa, ga, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp, dd);
+                uint32_t dd[16];
+                chunk_ds(xa, ga, sel, lse2, del, sb, A, X, Cc, dd);
                 tc::tmem_st16(s_addr, dd);
-                chunk_ds<false>(xb, gb, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp, dd);
+                chunk_ds(xb, gb, sel, lse2, del, sb, A, X, Cc, dd);
                 tc::tmem_st16(s_addr + 16, dd);
             }
             tc::tmem_wait_st();
@@ -496,19 +495,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // contiguous dimension, that is the MN-major A operand of
 //   dV += P^T dO,   dK += dS^T Q     (M = the 128 keys, N = d, K-dim = queries)
 // with dO and Q as MN-major B operands.  TMEM: S | G | dV | dK.
-//   warp 0      TMA producer: K and V once; Q and dO tiles through NSQ stages
+//   warp 0      TMA producer: K and V once; Q and dO tiles through their stages
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //   warps 2-9   softmax: warp w takes lane quarter w % 4 (query rows, then key
-//               rows in the epilogue of dK and dV) and key half (w - 2) / 4; it
-//               loads its S and G columns into registers with one wait and
-//               releases them (SGFREE) before it forms the block sums (at B = 128
-//               the two halves of a block add their sums through shared memory)
-// MMA order per query tile i:
-//   NSQ = 2: S_{i+1}, G_{i+1} once S_i, G_i are in registers; dK_i, dV_i once
-//            P_i, dS_i are written
-//   NSQ = 1: dK_i, dV_i, then S_{i+1} (Q_{i+1} lands once dK_i has read Q_i) and
-//            G_{i+1} (dO_{i+1} once dV_i has read dO_i): at d = 128 one stage of Q
-//            and dO is what shared memory holds beside K, V, P and dS.
+//               rows in the epilogue of dK and dV) and key half (w - 2) / 4.
+// Per query tile the softmax works in two passes: from S alone it forms the
+// block sums of the logits, the coefficients that P needs and P itself, writes P
+// (the dV product can start) and only then reads G for the sums of G, the rest
+// of the coefficients and dS.  S and G are released as soon as they are in
+// registers, so S of the next tile, and G where dO has a second stage, run beside
+// the softmax.  MMA issue order per tile i:
+//   S_{i+1} (two Q stages), dV_i, G_{i+1} (two dO stages), dK_i,
+//   S_{i+1} (one Q stage: Q_{i+1} lands once dK_i has read Q_i),
+//   G_{i+1} (one dO stage: dO_{i+1} lands once dV_i has read dO_i).
+// Shared memory at d = 128 holds K, V, P, dS and three tiles of Q and dO: two Q
+// stages at B = 64, one (and the B = 128 exchange buffer) at B = 128.
 // ---------------------------------------------------------------------------
 template <int D, int BS>
 struct DkvCfg {
@@ -517,25 +518,22 @@ struct DkvCfg {
     static constexpr uint32_t BOX_BYTES = 128 * 128;
     static constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;  // 128 rows x d bf16
     static constexpr uint32_t PT_BYTES = 2 * BOX_BYTES;       // 128 queries x 128 keys bf16
-    // stages of Q and of dO.  At d = 128 shared memory holds K, V, P, dS and three
-    // tiles of Q and dO: the second dO stage at B = 64, the exchange buffer of the
-    // B = 128 block sums otherwise.
-    static constexpr int NSQ = (D == 128) ? 1 : 2;
-    static constexpr int NSO = (D == 128 && BS == 128) ? 1 : 2;
+    static constexpr int NSQ = (D == 128 && BS == 128) ? 1 : 2;
+    static constexpr int NSO = (D == 128) ? 1 : 2;
     static constexpr uint32_t K_OFF = 0;
     static constexpr uint32_t V_OFF = K_OFF + TILE_BYTES;
     static constexpr uint32_t Q_OFF = V_OFF + TILE_BYTES;
     static constexpr uint32_t DO_OFF = Q_OFF + NSQ * TILE_BYTES;
     static constexpr uint32_t P_OFF = DO_OFF + NSO * TILE_BYTES;
     static constexpr uint32_t DS_OFF = P_OFF + PT_BYTES;
-    // B = 128 block sums exchanged between the two warps of a lane quarter:
-    // fp32 [tile parity][key half][128 rows][4]
+    // B = 128: the two halves of a block add their sums through shared memory, twice a
+    // tile (logit sums, then G sums): fp32 [exchange][key half][128 rows][2]
     static constexpr uint32_t XCH_OFF = DS_OFF + PT_BYTES;
-    static constexpr uint32_t XCH_BYTES = (BS == 128) ? 2 * 2 * 128 * 4 * 4 : 0;
+    static constexpr uint32_t XCH_BYTES = (BS == 128) ? 2 * 2 * 128 * 2 * 4 : 0;
     static constexpr uint32_t BAR_OFF = XCH_OFF + XCH_BYTES;
-    // KVFULL; QFULL, QEMPTY per Q stage; DOFULL, DOEMPTY per dO stage; SFULL; PREADY;
-    // PFREE; DKVFULL; DONE; SGFREE; PAIR per lane quarter
-    static constexpr uint32_t NBAR = 1 + 2 * NSQ + 2 * NSO + 5 + 1 + 4;
+    // KVFULL; QFULL, QEMPTY per Q stage; DOFULL, DOEMPTY per dO stage; SFULL, GFULL, SFREE,
+    // GFREE, PREADY, DSREADY, PFREE, DSFREE, DKVFULL, DONE; PAIR per lane quarter
+    static constexpr uint32_t NBAR = 1 + 2 * NSQ + 2 * NSO + 10 + 4;
     static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t G_COL = 128, DV_COL = 256, DK_COL = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -546,6 +544,62 @@ struct DkvCfg {
 __device__ __forceinline__ void st_swz16(uint8_t* tile, int t, int col8, uint4 v) {
     const int box = col8 >> 3, c = col8 & 7;
     *reinterpret_cast<uint4*>(tile + box * (128 * 128) + t * 128 + ((c ^ (t & 7)) << 4)) = v;
+}
+
+// Sums of (x - x0) and (x - x0)^2 over the 64 logits of a half tile (packed pairs).
+__device__ __forceinline__ float2 half_logit_sums(const uint32_t (&xa)[32], const uint32_t (&xb)[32], float x0) {
+    const uint64_t nx0 = tc::f2_make(-x0, -x0);
+    uint64_t a1 = 0ull, a2 = 0ull;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const uint32_t* xs = e < 16 ? xa : xb;
+        const int o = 2 * (e & 15);
+        const uint64_t dx = tc::f2_add(tc::f2_make(__uint_as_float(xs[o]), __uint_as_float(xs[o + 1])), nx0);
+        a1 = tc::f2_add(a1, dx);
+        a2 = tc::f2_fma(dx, dx, a2);
+    }
+    const float2 s1 = tc::f2_split(a1), s2 = tc::f2_split(a2);
+    return make_float2(s1.x + s1.y, s2.x + s2.y);
+}
+
+// Sums of G and G (x - x0) over the half tile.
+__device__ __forceinline__ float2 half_g_sums(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
+                                              const uint32_t (&ga)[32], const uint32_t (&gb)[32], float x0) {
+    const uint64_t nx0 = tc::f2_make(-x0, -x0);
+    uint64_t ag = 0ull, agd = 0ull;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const uint32_t* xs = e < 16 ? xa : xb;
+        const uint32_t* gs = e < 16 ? ga : gb;
+        const int o = 2 * (e & 15);
+        const uint64_t dx = tc::f2_add(tc::f2_make(__uint_as_float(xs[o]), __uint_as_float(xs[o + 1])), nx0);
+        const uint64_t g2 = tc::f2_make(__uint_as_float(gs[o]), __uint_as_float(gs[o + 1]));
+        ag = tc::f2_add(ag, g2);
+        agd = tc::f2_fma(g2, dx, agd);
+    }
+    const float2 sg = tc::f2_split(ag), sgd = tc::f2_split(agd);
+    return make_float2(sg.x + sg.y, sgd.x + sgd.y);
+}
+
+// P of 32 keys from the logits alone (selected: 2^{x log2 e - lse2}; unselected: a + Pu u),
+// with the same warp-uniform branch and the same zero rows past the sequence end as chunk_ds.
+__device__ __forceinline__ void chunk_p(const uint32_t (&xs)[32], bool sel, float lse2, float sb, float a, float Pu,
+                                        uint32_t (&pp)[16]) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    if (sel) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            pp[e] = tc::pack_bf16x2(tc::ex2(fmaf(__uint_as_float(xs[2 * e]), LOG2E, -lse2)),
+                                    tc::ex2(fmaf(__uint_as_float(xs[2 * e + 1]), LOG2E, -lse2)));
+    } else {
+        const uint64_t nsb = tc::f2_make(-sb, -sb), a2 = tc::f2_make(a, a), P2 = tc::f2_make(Pu, Pu);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const uint64_t u2 = tc::f2_add(tc::f2_make(__uint_as_float(xs[2 * e]), __uint_as_float(xs[2 * e + 1])), nsb);
+            const float2 p = tc::f2_split(tc::f2_fma(P2, u2, a2));
+            pp[e] = tc::pack_bf16x2(p.x, p.y);
+        }
+    }
 }
 
 template <int D, int BS, int ORDER>
@@ -561,15 +615,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // M = 128 keys, N = d, A (P or dS) and B (dO or Q) both MN-major
     constexpr uint32_t IDESC_KV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                   ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    constexpr bool kEarlyS = C::NSQ >= 2, kEarlyG = C::NSO >= 2;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_addr(smem);
     auto bar = [&](int i) { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
-    const int B_KVFULL = 0, B_QFULL = 1, B_QEMPTY = 1 + C::NSQ, B_DOFULL = 1 + 2 * C::NSQ,
-              B_DOEMPTY = B_DOFULL + C::NSO, B_SFULL = B_DOEMPTY + C::NSO, B_PREADY = B_SFULL + 1,
-              B_PFREE = B_PREADY + 1, B_DKVFULL = B_PFREE + 1, B_DONE = B_DKVFULL + 1, B_SGFREE = B_DONE + 1,
-              B_PAIR = B_SGFREE + 1;
+    const int B_KVFULL = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + C::NSQ, B_DOFULL = B_QEMPTY + C::NSQ,
+              B_DOEMPTY = B_DOFULL + C::NSO, B_SFULL = B_DOEMPTY + C::NSO, B_GFULL = B_SFULL + 1,
+              B_SFREE = B_GFULL + 1, B_GFREE = B_SFREE + 1, B_PREADY = B_GFREE + 1, B_DSREADY = B_PREADY + 1,
+              B_PFREE = B_DSREADY + 1, B_DSFREE = B_PFREE + 1, B_DKVFULL = B_DSFREE + 1, B_DONE = B_DKVFULL + 1,
+              B_PAIR = B_DONE + 1;
     uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + C::NBAR * 8);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -589,11 +645,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(bar(B_DOEMPTY + s), 1);
         }
         tc::mbar_init(bar(B_SFULL), 1);
+        tc::mbar_init(bar(B_GFULL), 1);
+        tc::mbar_init(bar(B_SFREE), 256);
+        tc::mbar_init(bar(B_GFREE), 256);
         tc::mbar_init(bar(B_PREADY), 256);
+        tc::mbar_init(bar(B_DSREADY), 256);
         tc::mbar_init(bar(B_PFREE), 1);
+        tc::mbar_init(bar(B_DSFREE), 1);
         tc::mbar_init(bar(B_DKVFULL), 1);
         tc::mbar_init(bar(B_DONE), 1);
-        tc::mbar_init(bar(B_SGFREE), 256);
         for (int qq = 0; qq < 4; ++qq) tc::mbar_init(bar(B_PAIR + qq), 64);
         tc::fence_barrier_init();
     }
@@ -619,26 +679,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::tma_load_2d(sbase + C::V_OFF + b * C::BOX_BYTES, &tm_v, bar(B_KVFULL), b * 64, bh * L + k0);
             }
             int lastQ = -1, lastO = -1;
-            for (int i = 0; i < NQT; ++i) {
-                const int row = bh * L + i * C::NQ;
-                // dO first: its stage frees up with dV_{i - NSO}, which the MMA issues
-                // before the dK that frees Q's stage
-                const int so = i % C::NSO, uo = i / C::NSO;
-                if (uo > 0 && !tc::mbar_wait(bar(B_DOEMPTY + so), (uo - 1) & 1, aborted, status, kWaitLimitCycles))
-                    break;
-                tc::mbar_expect_tx(bar(B_DOFULL + so), C::TILE_BYTES);
-                for (int b = 0; b < C::NBOX; ++b)
-                    tc::tma_load_2d(sbase + C::DO_OFF + so * C::TILE_BYTES + b * C::BOX_BYTES, &tm_do,
-                                    bar(B_DOFULL + so), b * 64, row);
-                lastO = i;
+            // the loads in the order the MMA issuer consumes them: with two Q stages S_{i+1}
+            // comes first (Q_{i+1}'s stage was freed by dK_{i-1}) and dO_{i+1} waits for dV_i;
+            // with one, dV_i frees dO's stage before dK_i frees Q's
+            auto load_q = [&](int i, int row) -> bool {
                 const int sq = i % C::NSQ, uq = i / C::NSQ;
                 if (uq > 0 && !tc::mbar_wait(bar(B_QEMPTY + sq), (uq - 1) & 1, aborted, status, kWaitLimitCycles))
-                    break;
+                    return false;
                 tc::mbar_expect_tx(bar(B_QFULL + sq), C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
                     tc::tma_load_2d(sbase + C::Q_OFF + sq * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q,
                                     bar(B_QFULL + sq), b * 64, row);
                 lastQ = i;
+                return true;
+            };
+            auto load_do = [&](int i, int row) -> bool {
+                const int so = i % C::NSO, uo = i / C::NSO;
+                if (uo > 0 && !tc::mbar_wait(bar(B_DOEMPTY + so), (uo - 1) & 1, aborted, status, kWaitLimitCycles))
+                    return false;
+                tc::mbar_expect_tx(bar(B_DOFULL + so), C::TILE_BYTES);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tc::tma_load_2d(sbase + C::DO_OFF + so * C::TILE_BYTES + b * C::BOX_BYTES, &tm_do,
+                                    bar(B_DOFULL + so), b * 64, row);
+                lastO = i;
+                return true;
+            };
+            for (int i = 0; i < NQT; ++i) {
+                const int row = bh * L + i * C::NQ;
+                if (kEarlyS) {
+                    if (!load_q(i, row) || !load_do(i, row)) break;
+                } else {
+                    if (!load_do(i, row) || !load_q(i, row)) break;
+                }
             }
             if (aborted) {
                 bool a2 = false;
@@ -687,51 +759,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ss(tmem + dcol, adesc + off, bdesc + off, IDESC_KV, (first && kk == 0) ? 0u : 1u);
                 }
             };
-            // S_i into the S columns (Q stage i % NSQ), G_i into the G columns (dO stage i % NSO)
+            // S_i into the S columns (Q stage i % NSQ) once the softmax holds S_{i-1}; G_i likewise
             auto put_s = [&](int i) -> bool {
+                if (i > 0 && !tc::mbar_wait(bar(B_SFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) return false;
                 const int sq = i % C::NSQ, uq = i / C::NSQ;
                 if (!tc::mbar_wait(bar(B_QFULL + sq), uq & 1, aborted, status, kWaitLimitCycles)) return false;
                 tc::fence_after_sync();
                 issue_s(sq);
+                tc::mma_commit(bar(B_SFULL));
                 return true;
             };
             auto put_g = [&](int i) -> bool {
+                if (i > 0 && !tc::mbar_wait(bar(B_GFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) return false;
                 const int so = i % C::NSO, uo = i / C::NSO;
                 if (!tc::mbar_wait(bar(B_DOFULL + so), uo & 1, aborted, status, kWaitLimitCycles)) return false;
                 tc::fence_after_sync();
                 issue_g(so);
+                tc::mma_commit(bar(B_GFULL));
                 return true;
             };
-            constexpr bool kEarlyS = C::NSQ >= 2, kEarlyG = C::NSO >= 2;
             bool ok = tc::mbar_wait(bar(B_KVFULL), 0, aborted, status, kWaitLimitCycles);
             ok = ok && put_s(0) && put_g(0);
-            if (ok) tc::mma_commit(bar(B_SFULL));
             for (int i = 0; ok && i < NQT; ++i) {
                 const int sq = i % C::NSQ, so = i % C::NSO;
                 const bool more = i + 1 < NQT;
-                // the products of tile i + 1 whose operand has a stage of its own go in as soon
-                // as the softmax holds S_i and G_i in registers (SGFREE)
-                if (more && (kEarlyS || kEarlyG)) {
-                    if (!tc::mbar_wait(bar(B_SGFREE), i & 1, aborted, status, kWaitLimitCycles)) break;
-                    if (kEarlyS && !put_s(i + 1)) break;
-                    if (kEarlyG && !put_g(i + 1)) break;
-                    if (kEarlyS && kEarlyG) tc::mma_commit(bar(B_SFULL));
-                }
-                // the softmax has written P_i and dS_i
+                if (kEarlyS && more && !put_s(i + 1)) break;
+                // dV_i once P_i is written
                 if (!tc::mbar_wait(bar(B_PREADY), i & 1, aborted, status, kWaitLimitCycles)) break;
                 tc::fence_after_sync();
-                issue_kv(C::DK_COL, dsmn, qmn0 + sq * kTileStep, i == 0);
-                tc::mma_commit(bar(B_QEMPTY + sq));
                 issue_kv(C::DV_COL, pmn, domn0 + so * kTileStep, i == 0);
                 tc::mma_commit(bar(B_DOEMPTY + so));
                 tc::mma_commit(bar(B_PFREE));
-                // a single stage: Q_{i+1} lands once dK_i has read Q_i (dO_{i+1} once dV_i has
-                // read dO_i)
-                if (more && !(kEarlyS && kEarlyG)) {
-                    if (!kEarlyS && !put_s(i + 1)) break;
-                    if (!kEarlyG && !put_g(i + 1)) break;
-                    tc::mma_commit(bar(B_SFULL));
-                }
+                if (kEarlyG && more && !put_g(i + 1)) break;
+                // dK_i once dS_i is written
+                if (!tc::mbar_wait(bar(B_DSREADY), i & 1, aborted, status, kWaitLimitCycles)) break;
+                tc::fence_after_sync();
+                issue_kv(C::DK_COL, dsmn, qmn0 + sq * kTileStep, i == 0);
+                tc::mma_commit(bar(B_QEMPTY + sq));
+                tc::mma_commit(bar(B_DSFREE));
+                if (!kEarlyS && more && !put_s(i + 1)) break;
+                if (!kEarlyG && more && !put_g(i + 1)) break;
             }
             if (!aborted) tc::mma_commit(bar(B_DKVFULL));
             tc::mma_commit(bar(B_DONE));
@@ -740,9 +807,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- softmax
-        // Warp w takes lane quarter w % 4 (32 query rows of each tile, then 32 key rows in
-        // the epilogue) and key half (w - 2) / 4: 64 of the tile's keys, one block at B = 64,
-        // half of one at B = 128 (whose sums the two warps of a quarter exchange).
         const int quarter = warp % 4;
         const int half = (warp - 2) / 4;
         const int r = quarter * 32 + lane;
@@ -752,66 +816,84 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* ptile = smem + C::P_OFF;
         uint8_t* dstile = smem + C::DS_OFF;
         float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);
+        // B = 128: add the other half's two sums (exchange ex of this tile, 0 or 1)
+        auto exchange = [&](float2 mine, int ex) -> float2 {
+            float2* slot = reinterpret_cast<float2*>(xch + (((ex * 2 + half) * 128) + r) * 2);
+            *slot = mine;
+            tc::mbar_arrive(bar(B_PAIR + quarter));
+            if (!tc::mbar_wait_warp(bar(B_PAIR + quarter), ex, aborted, status, kWaitLimitCycles)) return mine;
+            // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
+            (void)tc::mbar_try_wait(bar(B_PAIR + quarter), ex);
+            const float2 o = *reinterpret_cast<const float2*>(xch + (((ex * 2 + (1 - half)) * 128) + r) * 2);
+            return make_float2(mine.x + o.x, mine.y + o.y);
+        };
         for (int i = 0; i < NQT; ++i) {
             const int qrow = i * C::NQ + r;
             const bool valid = qrow < L;
             const int qt = (valid ? qrow : L - 1) / BS;
             const uint32_t* mrow = mask + ((size_t)bh * nblk + qt) * words;
-            const float lse2 = (valid ? __ldg(lse + (size_t)bh * L + qrow) : 0.f) * LOG2E;
+            const float lse2 = valid ? __ldg(lse + (size_t)bh * L + qrow) * LOG2E : __int_as_float(0x7f800000);
             const float del = valid ? __ldg(delta + (size_t)bh * L + qrow) : 0.f;
             const bool sel = (__ldg(mrow + (jb >> 5)) >> (jb & 31)) & 1u;
+            const float wp = (ORDER == 3) ? __ldg(wmat + ((size_t)bh * nblk + qt) * nblk + jb) : 0.f;
+            // ---- pass 1: S alone -> P
             if (!tc::mbar_wait_warp(bar(B_SFULL), i & 1, aborted, status, kWaitLimitCycles)) break;
             tc::fence_after_sync();
-            uint32_t xa[32], xb[32], ga[32], gb[32];
+            uint32_t xa[32], xb[32];
             tc::tmem_ld32(lane_base + 64 * half, xa);
             tc::tmem_ld32(lane_base + 64 * half + 32, xb);
-            tc::tmem_ld32(lane_base + C::G_COL + 64 * half, ga);
-            tc::tmem_ld32(lane_base + C::G_COL + 64 * half + 32, gb);
             uint32_t x0raw = 0u;
             if (BS == 128 && half == 1) x0raw = tc::tmem_ld1(lane_base);  // the block's first logit
             tc::tmem_wait_ld();
-            // S_i and G_i are in registers: the next tile's products may overwrite them
             tc::fence_before_sync();
-            tc::mbar_arrive(bar(B_SGFREE));
+            tc::mbar_arrive(bar(B_SFREE));
             const float x0 = (BS == 128 && half == 1) ? __uint_as_float(x0raw) : __uint_as_float(xa[0]);
-            HalfSums hs = half_sums(xa, xb, ga, gb, x0);
-            if (BS == 128) {
-                float4* mine = reinterpret_cast<float4*>(xch + ((((i & 1) * 2 + half) * 128) + r) * 4);
-                *mine = make_float4(hs.s1, hs.s2, hs.sg, hs.sgd);
-                tc::mbar_arrive(bar(B_PAIR + quarter));
-                if (!tc::mbar_wait_warp(bar(B_PAIR + quarter), i & 1, aborted, status, kWaitLimitCycles)) break;
-                // the phase is complete (lane 0 saw it); each thread's own test of it is its acquire
-                (void)tc::mbar_try_wait(bar(B_PAIR + quarter), i & 1);
-                const float4 o = *reinterpret_cast<const float4*>(xch + ((((i & 1) * 2 + (1 - half)) * 128) + r) * 4);
-                hs.s1 += o.x;
-                hs.s2 += o.y;
-                hs.sg += o.z;
-                hs.sgd += o.w;
-            }
+            float2 ls = half_logit_sums(xa, xb, x0);
+            if (BS == 128) ls = exchange(ls, 0);
+            if (aborted) break;
+            // the coefficients P needs: sb, w (gate held fixed), a = e^{l - lse}, Pu = c1 a
             float sb, a, A, X, Cc, Pu, inner;
-            const float wp = (ORDER == 3) ? __ldg(wmat + ((size_t)bh * nblk + qt) * nblk + jb) : 0.f;
-            block_coefs<BS, ORDER>(x0, hs.s1, hs.s2, hs.sg, hs.sgd, lse2, del, gate, ln_b, wp, sb, a, A, X, Cc, Pu,
-                                   inner);
-            // the previous tile's dK and dV products have read P and dS
+            block_coefs<BS, ORDER>(x0, ls.x, ls.y, 0.f, 0.f, lse2, del, gate, ln_b, wp, sb, a, A, X, Cc, Pu, inner);
             if (i > 0 && !tc::mbar_wait_warp(bar(B_PFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) break;
-            // row r of P and dS (bf16), this half's 64 keys = box `half` of each tile, 32 keys a chunk
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
-                uint32_t pp[16], dd[16];
-                chunk_ds<true>(ch == 0 ? xa : xb, ch == 0 ? ga : gb, sel, valid, lse2, del, sb, a, A, X, Cc, Pu, pp,
-                               dd);
+                uint32_t pp[16];
+                chunk_p(ch == 0 ? xa : xb, sel, lse2, sb, a, Pu, pp);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 4; ++c)
                     st_swz16(ptile, r, 8 * half + 4 * ch + c,
                              make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]));
-                    st_swz16(dstile, r, 8 * half + 4 * ch + c,
-                             make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]));
-                }
             }
-            // generic-proxy stores -> the tensor core (async proxy) reads them
             tc::fence_proxy_async_smem();
             tc::fence_before_sync();
             tc::mbar_arrive(bar(B_PREADY));
+            // ---- pass 2: G -> dS
+            if (!tc::mbar_wait_warp(bar(B_GFULL), i & 1, aborted, status, kWaitLimitCycles)) break;
+            tc::fence_after_sync();
+            uint32_t ga[32], gb[32];
+            tc::tmem_ld32(lane_base + C::G_COL + 64 * half, ga);
+            tc::tmem_ld32(lane_base + C::G_COL + 64 * half + 32, gb);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_GFREE));
+            float2 gsum = half_g_sums(xa, xb, ga, gb, x0);
+            if (BS == 128) gsum = exchange(gsum, 1);
+            if (aborted) break;
+            block_coefs<BS, ORDER>(x0, ls.x, ls.y, gsum.x, gsum.y, lse2, del, gate, ln_b, wp, sb, a, A, X, Cc, Pu,
+                                   inner);
+            if (i > 0 && !tc::mbar_wait_warp(bar(B_DSFREE), (i - 1) & 1, aborted, status, kWaitLimitCycles)) break;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t dd[16];
+                chunk_ds(ch == 0 ? xa : xb, ch == 0 ? ga : gb, sel, lse2, del, sb, A, X, Cc, dd);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    st_swz16(dstile, r, 8 * half + 4 * ch + c,
+                             make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]));
+            }
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(B_DSREADY));
         }
         // epilogue: this warp's column half of the dK and dV rows (TMEM lane = key) to global
         if (tc::mbar_wait_warp(bar(B_DKVFULL), 0, aborted, status, kWaitLimitCycles)) {
